@@ -1,0 +1,103 @@
+"""Hidden-MLP up-projection variant of the Dust estimator, in fp64.
+
+The perturbed layer is the up-projection u = W_up x (d_ff outputs per token).
+Per the pages ("Dust：无需反向传播的Transformer零阶预训练", §1: noise on every
+linear layer's output per token, layer types perturbed in separate passes
+with unperturbed intermediates cached; "不用反向传播训练Transformer：Dust零阶
+优化获突破": cache unperturbed intermediates, recompute only what the
+perturbation changes), a draw adds sigma*eps to u and recomputes GELU, the
+down-projection and the head from the cached x, u and clean logits:
+
+  clean:     u = x W_up^T, a = GELU(u), h = x + a W_down^T, z = h W_head^T
+  perturbed: da = GELU(u + sigma eps) - GELU(u), dh = da W_down^T,
+             dz = dh W_head^T,
+             r  = dz_y - log1p(sum_j p_j expm1(dz_j))       (= L - L')
+  estimate:  g_t = -(1/(K sigma)) sum_i r_i eps_i   (d_ff entries)
+             G_up = sum_t g_t x_t^T                  (d_ff x d)
+
+Readings: GELU is the exact erf form (the only GELU the pages show is
+PyTorch's default ``nn.GELU()`` in the listing of "Dust：无需反向传播的
+Transformer 预训练方法"); there is no LayerNorm and no bias. The GEMM operands
+that the bf16 workload rounds to bf16 (a, h, da, dh) are rounded here at the
+same points (``mirror_bf16``) so that comparisons measure implementation
+error, not the configured quantisation.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf
+
+from .params import Params
+from .philox import TAG_MLP_UP, gaussians
+
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    """Exact GELU: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2))."""
+    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+
+
+def bf16_rne(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (8 significant bits, ties to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m 2^e, 0.5 <= |m| < 1
+    m = np.round(m * 256.0) / 256.0         # np.round: half to even
+    return np.ldexp(m, e)
+
+
+def clean_mlp(X, W_up, W_down, W_head, targets, mirror_bf16: bool = True) -> dict:
+    X = np.asarray(X, dtype=np.float64)
+    rnd = bf16_rne if mirror_bf16 else (lambda v: v)
+    u = X @ np.asarray(W_up, dtype=np.float64).T
+    a = rnd(gelu(u))
+    h = X + a @ np.asarray(W_down, dtype=np.float64).T
+    hb = rnd(h)
+    z = hb @ np.asarray(W_head, dtype=np.float64).T
+    zmax = z.max(axis=1)
+    lse = zmax + np.log(np.exp(z - zmax[:, None]).sum(axis=1))
+    y = np.asarray(targets, dtype=np.int64)
+    loss = lse - z[np.arange(z.shape[0]), y]
+    p = np.exp(z - lse[:, None])
+    return {"u": u, "a": a, "h": hb, "z": z, "lse": lse, "loss": loss, "p": p}
+
+
+def mlp_draws(u_t, p_t, y_t, eps, W_down, W_head, sig, mirror_bf16=True):
+    """Rewards and sum_i r_i eps_i for n draws of noise ``eps`` (n, d_ff) on u_t."""
+    rnd = bf16_rne if mirror_bf16 else (lambda v: v)
+    da = rnd(gelu(u_t[None, :] + sig * eps) - gelu(u_t)[None, :])
+    dh = rnd(da @ W_down.T)
+    dz = dh @ W_head.T
+    r = dz[:, y_t] - np.log1p((p_t[None, :] * np.expm1(dz)).sum(axis=1))
+    acc = (r[:, None] * eps).sum(axis=0)
+    return r, acc
+
+
+def mlp_grad(X, W_up, W_down, W_head, targets, prm: Params, mirror_bf16: bool = True,
+             draw_chunk: int = 64) -> dict:
+    X = np.asarray(X, dtype=np.float64)
+    Wd = np.asarray(W_down, dtype=np.float64)
+    Wh = np.asarray(W_head, dtype=np.float64)
+    y = np.asarray(targets, dtype=np.int64)
+    clean = clean_mlp(X, W_up, W_down, W_head, y, mirror_bf16)
+    u, p = clean["u"], clean["p"]
+    T, d_ff = u.shape
+    sig = prm.sigma32
+    rewards = np.zeros((T, prm.K))
+    g = np.zeros((T, d_ff))
+    for t in range(T):
+        t_abs = t + prm.token_offset
+        for i0 in range(0, prm.K, draw_chunk):
+            i1 = min(prm.K, i0 + draw_chunk)
+            draws = np.arange(i0, i1, dtype=np.int64) + prm.draw_offset
+            eps = gaussians(prm.seed, t_abs, draws, np.arange(d_ff), TAG_MLP_UP, prm.stream_id)
+            r, acc = mlp_draws(u[t], p[t], y[t], eps, Wd, Wh, sig, mirror_bf16)
+            rewards[t, i0:i1] = r
+            g[t] += acc
+    if sig == 0.0:
+        g[:] = 0.0
+    else:
+        g *= -1.0 / (prm.K * sig)
+    G = np.einsum("tc,td->cd", g, X)
+    return {"loss": clean["loss"], "lse": clean["lse"], "rewards": rewards, "g": g, "G": G,
+            "u": u, "p": p, "z": clean["z"]}

@@ -1,0 +1,121 @@
+"""Pins for the oracle's MLP up-projection estimator.
+
+Checked against torch's GELU, bf16 conversion and autograd, brute-force
+finite differences and the exact expectation over enumerated noise.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+
+def _mlp_problem(T=4, d=5, d_ff=7, V=9, seed=0):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((T, d))
+    W_up = rng.standard_normal((d_ff, d)) / math.sqrt(d)
+    W_down = rng.standard_normal((d, d_ff)) / math.sqrt(d_ff)
+    W_head = rng.standard_normal((V, d)) / math.sqrt(d)
+    y = rng.integers(0, V, size=T)
+    return X, W_up, W_down, W_head, y
+
+
+def _torch_loss(X, W_up, W_down, W_head, y, wrt=None):
+    tens = {k: torch.tensor(v, dtype=torch.float64) for k, v in
+            dict(X=X, W_up=W_up, W_down=W_down, W_head=W_head).items()}
+    if wrt and wrt != "u":
+        tens[wrt].requires_grad_(True)
+    u = tens["X"] @ tens["W_up"].T
+    if wrt == "u":
+        u = u.detach().requires_grad_(True)
+        tens["u"] = u
+    a = torch.nn.functional.gelu(u, approximate="none")
+    h = tens["X"] + a @ tens["W_down"].T
+    z = h @ tens["W_head"].T
+    loss = torch.nn.functional.cross_entropy(z, torch.tensor(y), reduction="sum")
+    if wrt:
+        loss.backward()
+        return loss.item(), tens[wrt].grad.numpy()
+    return loss.item(), None
+
+
+def test_gelu_matches_torch():
+    x = np.linspace(-8, 8, 4001)
+    ref = torch.nn.functional.gelu(torch.tensor(x), approximate="none").numpy()
+    np.testing.assert_allclose(oracle.gelu(x), ref, rtol=0, atol=1e-15)
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    x = np.concatenate([x, np.float32([0.0, 1.0, -2.5, 1 + 2 ** -8, 1 + 3 * 2 ** -8])])
+    ref = torch.tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.bf16_rne(x.astype(np.float64)), ref)
+
+
+def test_clean_forward_matches_torch():
+    X, Wu, Wd, Wh, y = _mlp_problem(T=6)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y, mirror_bf16=False)
+    ref, _ = _torch_loss(X, Wu, Wd, Wh, y)
+    assert c["loss"].sum() == pytest.approx(ref, abs=1e-12)
+
+
+def test_sigma_zero_gives_zero_reward():
+    X, Wu, Wd, Wh, y = _mlp_problem()
+    prm = oracle.Params(T=4, d=5, V=9, d_ff=7, K=6, sigma=0.0, seed=2)
+    out = oracle.mlp_grad(X, Wu, Wd, Wh, y, prm)
+    assert np.all(out["rewards"] == 0.0) and np.all(out["G"] == 0.0)
+
+
+def test_estimate_is_unbiased_exact_expectation():
+    """Over +-sqrt(d_ff) e_m noise, g equals dL/du from torch autograd (to O(sigma^2))."""
+    X, Wu, Wd, Wh, y = _mlp_problem(T=3)
+    _, gu = _torch_loss(X, Wu, Wd, Wh, y, wrt="u")
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y, mirror_bf16=False)
+    d_ff = Wu.shape[0]
+    eps = np.concatenate([np.eye(d_ff), -np.eye(d_ff)]) * math.sqrt(d_ff)
+    sig = 1e-6
+    for t in range(3):
+        r, acc = oracle.mlp_draws(c["u"][t], c["p"][t], y[t], eps, Wd, Wh, sig, mirror_bf16=False)
+        g = -acc / (eps.shape[0] * sig)
+        np.testing.assert_allclose(g, gu[t], rtol=0, atol=1e-8)
+
+
+def test_closed_form_up_gradient_matches_finite_differences():
+    """sum_t [GELU'(u) * W_down^T W_head^T (p - e_y)] x^T against brute force."""
+    X, Wu, Wd, Wh, y = _mlp_problem(T=3, d=3, d_ff=4, V=5)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y, mirror_bf16=False)
+    u, p = c["u"], c["p"]
+    dgelu = 0.5 * (1 + np.vectorize(math.erf)(u / math.sqrt(2))) + u * np.exp(-u * u / 2) / math.sqrt(2 * math.pi)
+    closed = np.zeros_like(Wu)
+    for t in range(3):
+        gz = p[t].copy()
+        gz[y[t]] -= 1.0
+        closed += np.outer(dgelu[t] * (Wd.T @ (Wh.T @ gz)), X[t])
+    fd = np.zeros_like(Wu)
+    h = 1e-5
+    for i in range(Wu.shape[0]):
+        for j in range(Wu.shape[1]):
+            P, M = Wu.copy(), Wu.copy()
+            P[i, j] += h
+            M[i, j] -= h
+            fd[i, j] = (oracle.clean_mlp(X, P, Wd, Wh, y, False)["loss"].sum()
+                        - oracle.clean_mlp(X, M, Wd, Wh, y, False)["loss"].sum()) / (2 * h)
+    np.testing.assert_allclose(fd, closed, rtol=0, atol=1e-8)
+    _, gW = _torch_loss(X, Wu, Wd, Wh, y, wrt="W_up")
+    np.testing.assert_allclose(gW, closed, rtol=0, atol=1e-12)
+
+
+def test_estimate_converges_with_population():
+    X, Wu, Wd, Wh, y = _mlp_problem(T=4, d=4, d_ff=6, V=7, seed=3)
+    _, gW = _torch_loss(X, Wu, Wd, Wh, y, wrt="W_up")
+    errs = []
+    for K in (256, 4096):
+        prm = oracle.Params(T=4, d=4, V=7, d_ff=6, K=K, sigma=1e-4, seed=8)
+        G = oracle.mlp_grad(X, Wu, Wd, Wh, y, prm, mirror_bf16=False, draw_chunk=4096)["G"]
+        assert G.shape == Wu.shape
+        errs.append(np.linalg.norm(G - gW) / np.linalg.norm(gW))
+    assert errs[1] < errs[0] / 2.5
+    assert errs[1] < 0.25
