@@ -1,0 +1,393 @@
+"""Benchmark of the Dust per-token activation-space gradient estimator.
+
+One step = one full estimator call over one batch of synthetic input: clean
+logits GEMM, log-sum-exp, the K perturbed draws with rewards and the
+reward-weighted noise average g, and the G_W GEMM. The default workload is
+the LM head at d=1024, V=50304 with T=16384 tokens, K=16384 draws and
+vocabulary-subset draws of S=512 (the large-subset workload); ``--config``
+selects another one.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl dust|reference]
+
+Rank 0 prints one JSON line. Under torchrun (N > 1) each rank runs its own
+token shard (token_offset = rank * T, so the noise is that of one N*T-token
+run) with no collective on the data path: weak scaling, value = all ranks'
+token-draws / the slowest rank's time. ``--impl reference`` times the CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "token-draws/sec of Dust gradient estimate (LM head d=1024,V=50304); % roofline"
+UNIT = "token-draws/s"
+SM_COUNT = 148
+LANES_PER_SM = 128           # 4 schedulers x 32 lanes issue per clock
+# Algorithmic instruction slots per perturbed element:
+# Philox4x32-10 10, Gaussian transform 4, expm1 2, reward multiply-add and
+# its operand load 2, g accumulation multiply and add 2.
+ALU_OPS_PER_ELEM = 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, out_path=None):
+        self.proc = None
+        self.path = out_path or os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return None
+        idx = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0]
+        mine = [r for r in rows if r[0] == idx] or [r for r in rows if r[0] == rows[0][0]]
+        sm = [float(r[1]) for r in mine if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in mine for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(mine)}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+def _oracle_tokens(args):
+    """Worker: the oracle on a few tokens of a workload (spawned process).
+
+    Returns (tokens done, seconds spent in the oracle); input generation is
+    not timed."""
+    import oracle
+    import synth
+    name, toks = args
+    wl = synth.CONFIGS[name]
+    if wl.variant == "head":
+        inp = synth.make_head_inputs(wl)
+        t0 = time.perf_counter()
+        for t in toks:
+            prm = oracle.Params(T=1, d=wl.d, V=wl.V, K=wl.K, S=wl.S, sigma=wl.sigma,
+                                seed=wl.seed, token_offset=t)
+            oracle.head_grad(inp["H"][t:t + 1], inp["W"], inp["targets"][t:t + 1], prm)
+    else:
+        inp = synth.make_mlp_inputs(wl)
+        t0 = time.perf_counter()
+        for t in toks:
+            prm = oracle.Params(T=1, d=wl.d, V=wl.V, d_ff=wl.d_ff, K=wl.K, sigma=wl.sigma,
+                                seed=wl.seed, token_offset=t)
+            oracle.mlp_grad(inp["X"][t:t + 1], inp["W_up"], inp["W_down"], inp["W_head"],
+                            inp["targets"][t:t + 1], prm)
+    return len(toks), time.perf_counter() - t0
+
+
+def cpu_baseline(name: str, budget_tokens: int = 0) -> dict:
+    """Time the oracle as it stands on a bounded token sample.
+
+    The sample is spread over spawned single-threaded worker processes (one
+    per host core, at most 16); each worker times only its oracle calls and
+    the sample's throughput is tokens x K / the slowest worker's time."""
+    import multiprocessing as mp
+    import synth
+    wl = synth.CONFIGS[name]
+    cores = max(1, min(os.cpu_count() or 1, 16))
+    ntok = min(budget_tokens or cores, wl.T)
+    toks = [int(t) for t in np.linspace(0, wl.T - 1, ntok).round()] if ntok > 1 else [0]
+    chunks = [(name, toks[i::cores]) for i in range(cores) if toks[i::cores]]
+    saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS",
+                                            "MKL_NUM_THREADS")}
+    for k in saved:
+        os.environ[k] = "1"
+    try:
+        with mp.get_context("spawn").Pool(len(chunks)) as pool:
+            res = pool.map(_oracle_tokens, chunks, chunksize=1)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    done = sum(r[0] for r in res)
+    dt = max(r[1] for r in res)
+    value = done * wl.K / dt
+    return {"value": value, "unit": UNIT, "cores": len(chunks), "kind": "oracle",
+            "sample": f"{done} tokens x all {wl.K} draws of {name}, fp64 NumPy oracle, "
+                      f"{len(chunks)} spawned single-threaded workers, slowest {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- helpers
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
+    """ALU-issue roofline of the draw kernel (algorithmic elements x ops / time)."""
+    if wl.S > 0:
+        elems = wl.T * wl.K * (wl.S + 1)
+    else:
+        elems = wl.T * wl.K * wl.V
+    achieved = elems * ALU_OPS_PER_ELEM / (draw_ms * 1e-3) / 1e12      # Tops/s
+    f = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    peak = SM_COUNT * LANES_PER_SM * f / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s",
+            "frac": achieved / peak, "traffic": None, "kernel": "subset_draws" if wl.S > 0 else "reward+g",
+            "elements": elems, "ops_per_element": ALU_OPS_PER_ELEM, "kernel_ms": draw_ms,
+            "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)"}
+
+
+# ----------------------------------------------------------------------------- main arms
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return 0
+    import synth
+    wl = synth.CONFIGS[args.config]
+    per_step = []
+    cb = None
+    for _ in range(args.warmup):
+        cpu_baseline(args.config, budget_tokens=args.ref_tokens)
+    for _ in range(args.steps):
+        cb = cpu_baseline(args.config, budget_tokens=args.ref_tokens)
+        per_step.append(cb["value"])
+    value = statistics.median(per_step)
+    cb["value"] = value
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wl.token_draws / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.config, "T": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
+                       "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_dust(args):
+    import numpy as np
+    import torch
+    import synth
+    import zeroth_order_transformer_dust_b200 as dust
+
+    world, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_kind = _peaks()
+    wl = synth.CONFIGS[args.config]
+    ctx = dust.Context(local)
+    t_off = rank * wl.T
+
+    if wl.variant == "head":
+        inp = synth.make_head_inputs(wl)
+        tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        H = torch.from_numpy(inp["H"]).to(tdt)
+        W = torch.from_numpy(inp["W"]).to(tdt)
+        y = torch.from_numpy(inp["targets"]).to(torch.int32)
+        Hd, Wd, yd = H.to(dev), W.to(dev), y.to(dev)
+        outs = {"G": torch.empty(wl.V, wl.d, dtype=torch.float32, device=dev),
+                "loss": torch.empty(wl.T, dtype=torch.float32, device=dev)}
+
+        def step():
+            ctx.head_grad(Hd, Wd, yd, K=wl.K, sigma=wl.sigma, S=wl.S, seed=wl.seed,
+                          token_offset=t_off, out=outs, asynchronous=True)
+    else:
+        inp = synth.make_mlp_inputs(wl)
+        X, Wu, Wdn, Wh = (torch.from_numpy(inp[k]).to(torch.bfloat16).to(dev)
+                          for k in ("X", "W_up", "W_down", "W_head"))
+        yd = torch.from_numpy(inp["targets"]).to(torch.int32).to(dev)
+        outs = {"G": torch.empty(wl.d_ff, wl.d, dtype=torch.float32, device=dev),
+                "loss": torch.empty(wl.T, dtype=torch.float32, device=dev)}
+
+        def step():
+            ctx.mlp_grad(X, Wu, Wdn, Wh, yd, K=wl.K, sigma=wl.sigma, seed=wl.seed,
+                         token_offset=t_off, out=outs)
+
+    # L2 flush buffer (larger than the 126 MB L2), written between timed steps
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        step()
+    ctx.check()
+    _barrier(world)
+
+    ctx.set_stage_timing(True)
+    clocks = ClockSampler()
+    clocks.start()
+    launches0 = ctx.kernel_launches
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    stage_ms = []
+    _barrier(world)
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+        stage_ms.append(ctx.stage_times())
+    _barrier(world)
+    clk = clocks.stop()
+    launches = ctx.kernel_launches - launches0
+    ctx.check()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = _max_over_ranks(sum(step_ms) / len(step_ms), world)
+    ctx.set_stage_timing(False)
+
+    stages = {}
+    for s in stage_ms:
+        for k_, v in s.items():
+            stages.setdefault(k_, []).append(v)
+    stages = {k_: sum(v) / len(v) for k_, v in stages.items()}
+
+    value = world * wl.token_draws / (ms * 1e-3)
+
+    # end to end through the host-buffer C-ABI call (head workloads)
+    e2e = None
+    if wl.variant == "head" and not args.no_e2e:
+        Hp, Wp, yp = H.pin_memory(), W.pin_memory(), y.pin_memory()
+        hout = {"G": torch.empty(wl.V, wl.d, dtype=torch.float32).pin_memory(),
+                "loss": torch.empty(wl.T, dtype=torch.float32).pin_memory()}
+        ctx.head_grad_host(Hp, Wp, yp, K=wl.K, sigma=wl.sigma, S=wl.S, seed=wl.seed,
+                           token_offset=t_off, out=hout)
+        _barrier(world)
+        times = []
+        for k in range(max(1, min(args.steps, 3))):
+            flush.fill_(k & 0xFF)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            ctx.head_grad_host(Hp, Wp, yp, K=wl.K, sigma=wl.sigma, S=wl.S, seed=wl.seed,
+                               token_offset=t_off, out=hout)
+            times.append(time.perf_counter() - t0)
+        e_ms = _max_over_ranks(1e3 * sum(times) / len(times), world)
+        h2d = Hp.numel() * Hp.element_size() + Wp.numel() * Wp.element_size() + yp.numel() * 4
+        d2h = hout["G"].numel() * 4 + hout["loss"].numel() * 4
+        e2e = {"value": world * wl.token_draws / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    roof = None
+    draw_key = "subset_draws" if wl.S > 0 else None
+    if wl.variant == "head":
+        draw_ms = stages.get("subset_draws") if wl.S > 0 else stages.get("reward", 0) + stages.get("g", 0)
+        if draw_ms:
+            roof = _alu_roofline(wl, draw_ms, peaks)
+            roof["peak_kind"] = peak_kind
+    gemm_flops = 2.0 * wl.T * wl.d * wl.V
+    extra = {}
+    if wl.variant == "head":
+        for key in ("clean_gemm", "gw_gemm"):
+            if stages.get(key):
+                extra[key + "_tflops"] = gemm_flops / (stages[key] * 1e-3) / 1e12
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(args.config, budget_tokens=args.ref_tokens)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic",
+                "config": {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V,
+                           "K": wl.K, "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype,
+                           "d_ff": wl.d_ff, "l2": "flushed between timed steps (256 MiB write)",
+                           "parallelism": f"token-sharded x{world}, no collective"},
+                "stage_ms": stages, "gpu_launches": launches, "e2e": e2e, "roofline": roof,
+                "cpu_baseline": cb, "clocks": clk, **extra}
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="large_subset_bf16")
+    ap.add_argument("--impl", default="dust", choices=["dust", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="oracle sample size in tokens (default: one or two per host core)")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_dust(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

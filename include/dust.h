@@ -1,0 +1,184 @@
+/*
+ * dust.h — C ABI of the Dust per-token activation-space gradient estimator
+ * (B200, sm_100a).
+ *
+ * What is computed. For a linear layer y_t = W x_t with cached inputs x_t and
+ * cached clean outputs, K draws add independent per-token Gaussian noise
+ * sigma*eps_t^(i) to y_t; the downstream per-token loss is recomputed from
+ * cached intermediates; the reward is the loss reduction
+ * r_t^(i) = L_t(clean) - L_t(perturbed); the output-error estimate is
+ * g_t = -(1/(K sigma)) sum_i r_t^(i) eps_t^(i) and the weight gradient is
+ * G_W = sum_t g_t x_t^T. Sources: "Dust：无需反向传播的Transformer零阶预训练"
+ * §1 (激活空间扰动, 无需反向传播的信用分配, 减少干扰) and "Dust: предобучение
+ * трансформеров без обратного распространения ошибки" ("Механика такая").
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor arguments are DEVICE pointers owned by the caller, row-major,
+ *    contiguous, 16-byte aligned, unless an entry point says HOST.
+ *  - Floating inputs are fp32 (dtype DUST_F32) or bf16 bit patterns stored as
+ *    uint16 (DUST_BF16). Outputs are always fp32.
+ *  - Every call is enqueued on the context's stream. By default the call ends
+ *    by reading back a device status word (one 4-byte copy and a stream
+ *    synchronisation), so device-detected errors (a target outside [0, V))
+ *    are returned by the call itself; DUST_FLAG_ASYNC skips that read and
+ *    leaves the status for dust_check().
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns DUST_ERR_ARG and launches nothing.
+ *  - The context owns its scratch memory (grown on demand, freed by
+ *    dust_destroy). A context is not thread-safe; use one per thread.
+ *  - Noise is Philox4x32-10 keyed by (seed, token, draw, slot) and is never
+ *    stored: slot k of (token t, draw i) is output word ((k>>5)&3) of counter
+ *    (((k>>7)<<5)|(k&31), t+token_offset, i+draw_offset, tag|(stream_id<<8)),
+ *    key (seed lo, seed hi), turned into N(0,1) by Box-Muller on 24-bit
+ *    uniforms (words 0,1 -> cos, sin; words 2,3 -> cos, sin). Tags: 0 = head
+ *    logits, 1 = subset offset, 2 = MLP up-projection.
+ */
+#ifndef DUST_H
+#define DUST_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dust_ctx dust_ctx;
+
+typedef enum {
+  DUST_OK = 0,
+  DUST_ERR_ARG = 1,          /* invalid argument: nothing was launched */
+  DUST_ERR_CUDA = 2,         /* a CUDA runtime or driver call failed */
+  DUST_ERR_OOM = 3,          /* scratch allocation failed */
+  DUST_ERR_BOUNDS = 4,       /* device-detected out-of-range index (a target) */
+  DUST_ERR_TIMEOUT = 5,      /* a bounded device wait expired */
+  DUST_ERR_UNSUPPORTED = 6   /* valid but not supported (shape, device) */
+} dust_status;
+
+typedef enum { DUST_F32 = 0, DUST_BF16 = 1 } dust_dtype;
+
+enum {
+  /* Scale the target coordinate of subset draws by V/S like the others (the
+     literal reading; biased). Default: 1 for the target, V/S otherwise. */
+  DUST_FLAG_LITERAL_TARGET_SCALE = 1u << 0,
+  /* Do not read back the device status word at the end of the call. */
+  DUST_FLAG_ASYNC = 1u << 1
+};
+
+/* Variants accepted by dust_validate. */
+enum { DUST_VARIANT_HEAD = 0, DUST_VARIANT_MLP = 1 };
+
+typedef struct dust_params {
+  int64_t T;            /* tokens in this call (>= 1) */
+  int64_t d;            /* layer input width (head: hidden; MLP: model width) */
+  int64_t V;            /* vocabulary size (>= 1) */
+  int64_t d_ff;         /* MLP hidden width (MLP variant only) */
+  int32_t K;            /* draws per token (>= 1) */
+  int32_t S;            /* head: <= 0 full vocabulary, else subset size (<= V) */
+  float sigma;          /* noise scale (>= 0, finite); 0 gives zero estimates */
+  int32_t dtype;        /* dust_dtype of the floating inputs */
+  uint64_t seed;        /* Philox key */
+  int64_t token_offset; /* absolute index of token 0 (noise counter word 1) */
+  int64_t draw_offset;  /* absolute index of draw 0 (noise counter word 2) */
+  int64_t subset_a;     /* subset stride a (coprime to V); 0: smallest integer
+                           >= V (sqrt5-1)/2 coprime to V */
+  uint32_t stream_id;   /* layer id, < 2^24 (noise counter word 3 bits 8..31) */
+  uint32_t flags;       /* DUST_FLAG_* */
+} dust_params;
+
+/* Create a context on CUDA device `device`, enqueuing on `cuda_stream`
+   (a cudaStream_t; NULL = the legacy default stream). */
+dust_status dust_create(dust_ctx** out, int device, void* cuda_stream);
+dust_status dust_set_stream(dust_ctx* ctx, void* cuda_stream);
+/* Frees the context's scratch memory; waits for its stream first. */
+void dust_destroy(dust_ctx* ctx);
+/* Last error message of the context (never NULL). */
+const char* dust_last_error(const dust_ctx* ctx);
+const char* dust_status_string(dust_status s);
+/* Host-only check of a parameter block for `variant` (no GPU needed).
+   `msg` (may be NULL) receives a reason of at most `msg_len` bytes. */
+dust_status dust_validate(const dust_params* p, int variant, char* msg, int msg_len);
+/* Subset stride the library uses for these parameters (the default when
+   p->subset_a == 0); 0 if the parameters are invalid. Host-only. */
+int64_t dust_subset_stride(const dust_params* p);
+/* Reads and clears the device status word after DUST_FLAG_ASYNC calls. */
+dust_status dust_check(dust_ctx* ctx);
+
+/*
+ * LM-head estimator on cached logits ("Dust：无需反向传播的Transformer零阶预训练"
+ * §1 减少干扰: the head is perturbed on cached logits and each draw evaluates a
+ * small subset of the vocabulary; "不用反向传播训练Transformer：Dust零阶优化获突破":
+ * only the affected loss is recomputed).
+ *   H        T x d   layer input (hidden states), dtype
+ *   W        V x d   head weight, dtype
+ *   targets  T       int32 token ids in [0, V)
+ *   G_out    V x d   fp32 estimated weight gradient sum_t g_t h_t^T   (or NULL)
+ *   loss_out T       fp32 clean per-token cross-entropy (natural log) (or NULL)
+ *   rewards_out T x K fp32 r[t*K + i] = L_t - L'_t,i                  (or NULL)
+ *   g_out    T x V   fp32 output-error estimate g_t, vocabulary order  (or NULL)
+ * Full vocabulary (S <= 0): eps covers all V logits. Subset (S > 0): slot
+ * k < S perturbs logit (a k + b) mod V with b = floor(w0 V / 2^32), w0 the
+ * first word of counter (0, t, i, 1|(stream_id<<8)); the target is always
+ * included (as slot S when not drawn); g is scaled per coordinate by its
+ * inverse inclusion probability (V/S; 1 for the target).
+ * Errors: DUST_ERR_ARG (validation), DUST_ERR_BOUNDS (a target outside
+ * [0, V): outputs are then unspecified), DUST_ERR_OOM, DUST_ERR_CUDA.
+ */
+dust_status dust_head_grad(dust_ctx* ctx, const dust_params* p,
+                           const void* H, const void* W, const int32_t* targets,
+                           float* G_out, float* loss_out, float* rewards_out,
+                           float* g_out);
+
+/* Same as dust_head_grad with every tensor argument in HOST memory (pinned
+   memory gives the fastest copies). The inputs are copied to the device, the
+   estimator runs, and the requested outputs are copied back before return. */
+dust_status dust_head_grad_host(dust_ctx* ctx, const dust_params* p,
+                                const void* H, const void* W, const int32_t* targets,
+                                float* G_out, float* loss_out, float* rewards_out,
+                                float* g_out);
+
+/*
+ * Hidden-MLP up-projection estimator ("Dust：无需反向传播的Transformer零阶预训练"
+ * §1: noise on each linear layer's output; 减少干扰: layer types perturbed in
+ * separate passes with unperturbed intermediates cached). Noise goes on
+ * u = x W_up^T (d_ff entries per token); each draw recomputes
+ * GELU(u + sigma eps) - GELU(u), the down-projection and the head from the
+ * cached x, u and clean logits (exact-erf GELU, residual h = x + a W_down^T,
+ * no norm, no bias; bf16 workloads round a, h and the per-draw deltas to bf16
+ * as GEMM operands).
+ *   X        T x d     input, dtype        W_up   d_ff x d   dtype
+ *   W_down   d x d_ff  dtype               W_head V x d      dtype
+ *   targets  T int32
+ *   G_up_out d_ff x d  fp32 sum_t g_t x_t^T   (or NULL)
+ *   loss_out T         fp32 clean CE           (or NULL)
+ *   rewards_out T x K  fp32                    (or NULL)
+ *   g_out    T x d_ff  fp32                    (or NULL)
+ * p->S must be <= 0 (all d_ff channels are perturbed).
+ */
+dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* p,
+                          const void* X, const void* W_up, const void* W_down,
+                          const void* W_head, const int32_t* targets,
+                          float* G_up_out, float* loss_out, float* rewards_out,
+                          float* g_out);
+
+/* Per-stage device timing: when enabled, each call records CUDA events on
+   the context's stream between its stages (clean GEMM, log-sum-exp, draws,
+   g, G_W GEMM...). dust_stage_times waits for the last call's final event
+   and fills names[i] / ms[i] for i < cap; it returns the number of stages. */
+dust_status dust_set_stage_timing(dust_ctx* ctx, int enable);
+int dust_stage_times(dust_ctx* ctx, const char** names, float* ms, int cap);
+/* Number of kernels the context has launched since it was created. */
+int64_t dust_kernel_launches(const dust_ctx* ctx);
+
+/* Debug: raw Philox4x32-10 words. ctr4 (n x 4 uint32, device) -> out (n x 4). */
+dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4,
+                              int64_t n, uint32_t* out);
+/* Debug: eps for tokens [0, nt), draws [0, ni), slots [0, nslots) of tag `tag`
+   under p's seed, offsets and stream_id -> out[(t*ni + i)*nslots + k] fp32. */
+dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag,
+                             int64_t nt, int64_t ni, int64_t nslots, float* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUST_H */

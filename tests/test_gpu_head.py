@@ -1,0 +1,186 @@
+"""LM-head estimator on the GPU vs the fp64 oracle, element by element.
+
+Small cases span several tiles and ragged tails; the large workloads are
+checked on token slices (token_offset reproduces the exact noise of the
+full run) and, at full size in the launch configuration the benchmark uses,
+on sampled token rows plus the outer-product identity for G_W.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import zeroth_order_transformer_dust_b200 as dust
+from _util import TOL_G, TOL_GW_BF16, TOL_GW_F32, TOL_LOSS, np64, rel_fro, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ctx(cuda_ok):
+    return dust.Context(0)
+
+
+def _inputs(wl, T=None, t0=0):
+    inp = synth.make_head_inputs(wl)
+    sl = slice(t0, t0 + (T or wl.T))
+    return inp["H"][sl], inp["W"], inp["targets"][sl]
+
+
+def _gpu(ctx, H, W, y, wl, **kw):
+    out = ctx.head_grad(to_dev(H, wl.dtype), to_dev(W, wl.dtype), to_dev(y, "i32"), K=wl.K,
+                        sigma=wl.sigma, S=wl.S, seed=wl.seed, want_rewards=True, want_g=True, **kw)
+    torch.cuda.synchronize()
+    return {k: np64(v) for k, v in out.items()}
+
+
+def _oracle(H, W, y, wl, **kw):
+    prm = oracle.Params(T=H.shape[0], d=H.shape[1], V=W.shape[0], K=wl.K, S=wl.S, sigma=wl.sigma,
+                        seed=wl.seed, **kw)
+    return oracle.head_grad(H, W, y, prm)
+
+
+def _compare(got, ref, gw_tol):
+    assert np.abs(got["loss"] - ref["loss"]).max() < TOL_LOSS
+    assert np.abs(got["rewards"] - ref["rewards"]).max() < TOL_LOSS
+    assert rel_fro(got["g"], ref["g"]) < TOL_G
+    assert rel_fro(got["G"], ref["G"]) < gw_tol
+
+
+def test_tiny_fp32_full_vocab(ctx):
+    wl = synth.CONFIGS["tiny_fp32"]
+    H, W, y = _inputs(wl)
+    _compare(_gpu(ctx, H, W, y, wl), _oracle(H, W, y, wl), TOL_GW_F32)
+
+
+def test_full_vocab_bf16_slice(ctx):
+    wl = synth.CONFIGS["full_bf16"]
+    t0, n = 1000, 6
+    H, W, y = _inputs(wl, n, t0)
+    got = _gpu(ctx, H, W, y, wl, token_offset=t0)
+    _compare(got, _oracle(H, W, y, wl, token_offset=t0), TOL_GW_BF16)
+
+
+def test_subset_bf16_slice(ctx):
+    wl = synth.CONFIGS["subset_bf16"]
+    t0, n = 4321, 8
+    H, W, y = _inputs(wl, n, t0)
+    got = _gpu(ctx, H, W, y, wl, token_offset=t0)
+    _compare(got, _oracle(H, W, y, wl, token_offset=t0), TOL_GW_BF16)
+
+
+def test_large_subset_slice(ctx):
+    wl = synth.CONFIGS["large_subset_bf16"]
+    t0, n = 16381, 3
+    H, W, y = _inputs(wl, n, t0)
+    got = _gpu(ctx, H, W, y, wl, token_offset=t0)
+    _compare(got, _oracle(H, W, y, wl, token_offset=t0), TOL_GW_BF16)
+
+
+def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
+    wl = synth.Workload("small", "head", T=T, d=d, V=V, K=K, S=S, sigma=sigma, seed=seed,
+                        dtype=dtype, targets="zipf")
+    return wl
+
+
+@pytest.mark.parametrize("kw", [
+    dict(), dict(S=100), dict(S=1000), dict(S=1), dict(S=129, K=33), dict(T=1), dict(K=1),
+    dict(K=1, S=3), dict(V=257, S=256), dict(V=5, S=2, d=3), dict(d=1), dict(sigma=0.2),
+    dict(sigma=0.2, S=300), dict(dtype="f32"), dict(dtype="f32", S=77), dict(V=4099, S=640, K=40),
+])
+def test_edge_shapes(ctx, kw):
+    wl = _small(**kw)
+    H, W, y = _inputs(wl)
+    got = _gpu(ctx, H, W, y, wl)
+    ref = _oracle(H, W, y, wl)
+    _compare(got, ref, TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
+
+
+def test_single_entry_vocabulary(ctx):
+    # V = 1: the loss is exactly 0 and every reward vanishes (up to rounding)
+    for S in (0, 1):
+        wl = _small(V=1, S=S, K=3)
+        H, W, y = _inputs(wl)
+        got = _gpu(ctx, H, W, y, wl)
+        assert np.abs(got["loss"]).max() < TOL_LOSS
+        assert np.abs(got["rewards"]).max() < TOL_LOSS
+
+
+def test_sigma_zero_is_exactly_zero(ctx):
+    for S in (0, 50):
+        wl = _small(sigma=0.0, S=S)
+        H, W, y = _inputs(wl)
+        got = _gpu(ctx, H, W, y, wl)
+        assert np.all(got["rewards"] == 0) and np.all(got["g"] == 0) and np.all(got["G"] == 0)
+
+
+def test_options_stream_id_stride_literal(ctx):
+    wl = _small(S=64, K=12)
+    H, W, y = _inputs(wl)
+    for kw, okw in ((dict(stream_id=9), dict(stream_id=9)), (dict(subset_a=7), dict(subset_a=7)),
+                    (dict(literal_target_scale=True), dict(literal_target_scale=True))):
+        got = _gpu(ctx, H, W, y, wl, **kw)
+        ref = _oracle(H, W, y, wl, **okw)
+        _compare(got, ref, TOL_GW_BF16)
+
+
+def test_token_slices_and_draw_splits_compose(ctx):
+    wl = _small(T=50, S=200, K=24)
+    H, W, y = _inputs(wl)
+    full = _gpu(ctx, H, W, y, wl)
+    part = _gpu(ctx, H[17:29], W, y[17:29], wl, token_offset=17)
+    np.testing.assert_array_equal(part["rewards"], full["rewards"][17:29])
+    np.testing.assert_allclose(part["g"], full["g"][17:29], rtol=0, atol=1e-6)
+    # draws [0, 10) + [10, 24): rewards concatenate, K*g sums
+    a = _gpu(ctx, H, W, y, wl.with_(K=10))
+    b = _gpu(ctx, H, W, y, wl.with_(K=14), draw_offset=10)
+    np.testing.assert_array_equal(np.concatenate([a["rewards"], b["rewards"]], axis=1), full["rewards"])
+    np.testing.assert_allclose(10 * a["g"] + 14 * b["g"], 24 * full["g"], rtol=0, atol=1e-4)
+
+
+def test_bad_target_is_reported(ctx):
+    wl = _small()
+    H, W, y = _inputs(wl)
+    y = y.copy()
+    y[3] = wl.V
+    with pytest.raises(dust.DustError) as ei:
+        _gpu(ctx, H, W, y, wl)
+    assert ei.value.status == 4
+    # the context stays usable
+    y[3] = 0
+    _gpu(ctx, H, W, y, wl)
+
+
+def test_deterministic_rewards(ctx):
+    wl = _small(S=100, K=64)
+    H, W, y = _inputs(wl)
+    a = _gpu(ctx, H, W, y, wl)
+    b = _gpu(ctx, H, W, y, wl)
+    np.testing.assert_array_equal(a["rewards"], b["rewards"])
+    np.testing.assert_array_equal(a["loss"], b["loss"])
+    assert rel_fro(a["g"], b["g"]) < 1e-6
+
+
+@pytest.mark.parametrize("name,rows", [("full_bf16", (0, 2049, 4095)),
+                                       ("subset_bf16", (1, 8191)),
+                                       ("large_subset_bf16", (0, 9999))])
+def test_full_size_sampled_rows(ctx, name, rows):
+    """Full-size call (the benchmark's launch configuration); sampled token rows vs the oracle,
+    and G_W against sum_t g_t h_t^T rebuilt in fp64 from the returned g on sampled rows."""
+    wl = synth.CONFIGS[name]
+    inp = synth.make_head_inputs(wl)
+    H, W, y = inp["H"], inp["W"], inp["targets"]
+    Hd, Wd, yd = to_dev(H, wl.dtype), to_dev(W, wl.dtype), to_dev(y, "i32")
+    out = ctx.head_grad(Hd, Wd, yd, K=wl.K, sigma=wl.sigma, S=wl.S, seed=wl.seed,
+                        want_rewards=True, want_g=True)
+    torch.cuda.synchronize()
+    for t in rows:
+        ref = _oracle(H[t:t + 1], W, y[t:t + 1], wl, token_offset=t)
+        assert abs(out["loss"][t].item() - ref["loss"][0]) < TOL_LOSS
+        assert np.abs(np64(out["rewards"][t]) - ref["rewards"][0]).max() < TOL_LOSS
+        assert rel_fro(np64(out["g"][t]), ref["g"][0]) < TOL_G
+    vs = torch.randint(0, wl.V, (64,), generator=torch.Generator().manual_seed(0))
+    g_cols = out["g"][:, vs.cuda()].double()
+    ref_rows = (g_cols.T @ Hd.double()).cpu().numpy()
+    assert rel_fro(np64(out["G"][vs.cuda()]), ref_rows) < TOL_GW_BF16

@@ -1,0 +1,320 @@
+"""Dust per-token activation-space gradient estimator on B200 (sm_100a).
+
+Thin ctypes binding over the C ABI declared in ``include/dust.h``
+(``libdust.so``, built in-tree by ``python -m zeroth_order_transformer_dust_b200.build``).
+This module only marshals arguments: torch provides device memory and the
+CUDA stream, and every step of the estimator runs in the library's kernels.
+There is no CPU fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdust.so")
+
+DUST_OK = 0
+STATUS_NAMES = {0: "DUST_OK", 1: "DUST_ERR_ARG", 2: "DUST_ERR_CUDA", 3: "DUST_ERR_OOM",
+                4: "DUST_ERR_BOUNDS", 5: "DUST_ERR_TIMEOUT", 6: "DUST_ERR_UNSUPPORTED"}
+DUST_F32, DUST_BF16 = 0, 1
+FLAG_LITERAL_TARGET_SCALE = 1 << 0
+FLAG_ASYNC = 1 << 1
+VARIANT_HEAD, VARIANT_MLP = 0, 1
+TAG_HEAD, TAG_SUBSET_OFFSET, TAG_MLP_UP = 0, 1, 2
+
+# Every extern "C" symbol include/dust.h declares.
+EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
+           "dust_status_string", "dust_validate", "dust_subset_stride", "dust_check",
+           "dust_head_grad", "dust_head_grad_host", "dust_mlp_grad", "dust_debug_philox",
+           "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
+           "dust_kernel_launches")
+
+
+class DustParams(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("V", ctypes.c_int64),
+                ("d_ff", ctypes.c_int64), ("K", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("sigma", ctypes.c_float), ("dtype", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("token_offset", ctypes.c_int64), ("draw_offset", ctypes.c_int64),
+                ("subset_a", ctypes.c_int64), ("stream_id", ctypes.c_uint32),
+                ("flags", ctypes.c_uint32)]
+
+
+class DustError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libdust.so (raises FileNotFoundError when it has not been built)."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise FileNotFoundError(
+                f"{path} is missing: build it with `python -m zeroth_order_transformer_dust_b200.build`")
+        L = ctypes.CDLL(path)
+        P, I64, I32, U32, U64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                 ctypes.c_uint32, ctypes.c_uint64)
+        PP = ctypes.POINTER(DustParams)
+        sig = {
+            "dust_create": (I32, [ctypes.POINTER(P), ctypes.c_int, P]),
+            "dust_set_stream": (I32, [P, P]),
+            "dust_destroy": (None, [P]),
+            "dust_last_error": (ctypes.c_char_p, [P]),
+            "dust_status_string": (ctypes.c_char_p, [I32]),
+            "dust_validate": (I32, [PP, ctypes.c_int, ctypes.c_char_p, ctypes.c_int]),
+            "dust_subset_stride": (I64, [PP]),
+            "dust_check": (I32, [P]),
+            "dust_head_grad": (I32, [P, PP, P, P, P, P, P, P, P]),
+            "dust_head_grad_host": (I32, [P, PP, P, P, P, P, P, P, P]),
+            "dust_mlp_grad": (I32, [P, PP, P, P, P, P, P, P, P, P, P]),
+            "dust_debug_philox": (I32, [P, U64, P, I64, P]),
+            "dust_debug_gauss": (I32, [P, PP, I32, I64, I64, I64, P]),
+            "dust_set_stage_timing": (I32, [P, ctypes.c_int]),
+            "dust_stage_times": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_char_p),
+                                                ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
+            "dust_kernel_launches": (I64, [P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+        return L
+
+
+def make_params(T, d, V, K, sigma, *, S=0, d_ff=0, dtype=DUST_BF16, seed=0, token_offset=0,
+                draw_offset=0, subset_a=0, stream_id=0, flags=0) -> DustParams:
+    return DustParams(T=T, d=d, V=V, d_ff=d_ff, K=K, S=S, sigma=float(sigma), dtype=dtype,
+                      seed=seed & 0xFFFFFFFFFFFFFFFF, token_offset=token_offset,
+                      draw_offset=draw_offset, subset_a=subset_a, stream_id=stream_id,
+                      flags=flags)
+
+
+def validate(params: DustParams, variant: int = VARIANT_HEAD):
+    """Host-only parameter check; returns (status, message)."""
+    L = load_library()
+    buf = ctypes.create_string_buffer(256)
+    st = L.dust_validate(ctypes.byref(params), variant, buf, 256)
+    return st, buf.value.decode()
+
+
+def subset_stride(params: DustParams) -> int:
+    return int(load_library().dust_subset_stride(ctypes.byref(params)))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DUST_BF16
+    if t.dtype == torch.float32:
+        return DUST_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: use float32 or bfloat16")
+
+
+class Context:
+    """A library context bound to one CUDA device and (by default) torch's current stream."""
+
+    def __init__(self, device: Optional[int] = None, stream: Optional[torch.cuda.Stream] = None):
+        self._L = load_library()
+        if device is None:
+            device = torch.cuda.current_device()
+        self.device = int(device)
+        h = ctypes.c_void_p()
+        st = self._L.dust_create(ctypes.byref(h), self.device, None)
+        if st != DUST_OK:
+            raise DustError(st, f"dust_create(device={self.device}) failed")
+        self._h = h
+        self._stream = stream
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._L.dust_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- helpers ---------------------------------------------------------------
+    def _bind_stream(self):
+        s = self._stream if self._stream is not None else torch.cuda.current_stream(self.device)
+        self._L.dust_set_stream(self._h, ctypes.c_void_p(s.cuda_stream))
+
+    def _check(self, st: int):
+        if st != DUST_OK:
+            msg = self._L.dust_last_error(self._h).decode()
+            raise DustError(st, msg)
+
+    def check(self):
+        self._check(self._L.dust_check(self._h))
+
+    def _dev(self, t: torch.Tensor, name: str):
+        if not t.is_cuda or t.device.index != self.device:
+            raise ValueError(f"{name} must be on cuda:{self.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        return t
+
+    # -- estimator ---------------------------------------------------------------
+    def head_grad(self, H, W, targets, *, K, sigma, S=0, seed=0, token_offset=0, draw_offset=0,
+                  subset_a=0, stream_id=0, literal_target_scale=False, want_G=True,
+                  want_loss=True, want_rewards=False, want_g=False, asynchronous=False,
+                  out=None) -> dict:
+        """LM-head estimator. H (T x d), W (V x d) on this device, fp32 or bf16;
+        targets (T,) int32. Returns a dict of the requested fp32 outputs."""
+        self._dev(H, "H"), self._dev(W, "W"), self._dev(targets, "targets")
+        if H.dtype != W.dtype:
+            raise TypeError("H and W must share a dtype")
+        if targets.dtype != torch.int32:
+            raise TypeError("targets must be int32")
+        T, d = H.shape
+        V = W.shape[0]
+        flags = (FLAG_LITERAL_TARGET_SCALE if literal_target_scale else 0) | (
+            FLAG_ASYNC if asynchronous else 0)
+        prm = make_params(T, d, V, K, sigma, S=S, dtype=_dtype_code(H), seed=seed,
+                          token_offset=token_offset, draw_offset=draw_offset, subset_a=subset_a,
+                          stream_id=stream_id, flags=flags)
+        out = dict(out or {})
+        dev = H.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        if want_G and "G" not in out:
+            out["G"] = torch.empty(V, d, **f32)
+        if want_loss and "loss" not in out:
+            out["loss"] = torch.empty(T, **f32)
+        if want_rewards and "rewards" not in out:
+            out["rewards"] = torch.empty(T, K, **f32)
+        if want_g and "g" not in out:
+            out["g"] = torch.empty(T, V, **f32)
+        self._bind_stream()
+        st = self._L.dust_head_grad(self._h, ctypes.byref(prm), _ptr(H), _ptr(W), _ptr(targets),
+                                    _ptr(out.get("G")), _ptr(out.get("loss")),
+                                    _ptr(out.get("rewards")), _ptr(out.get("g")))
+        self._check(st)
+        return out
+
+    def head_grad_host(self, H, W, targets, *, K, sigma, S=0, seed=0, token_offset=0,
+                       draw_offset=0, subset_a=0, stream_id=0, out=None, want_G=True,
+                       want_loss=True) -> dict:
+        """Same estimator with every tensor in host memory (pin it for fast copies)."""
+        for t, n in ((H, "H"), (W, "W"), (targets, "targets")):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous host tensor")
+        T, d = H.shape
+        V = W.shape[0]
+        prm = make_params(T, d, V, K, sigma, S=S, dtype=_dtype_code(H), seed=seed,
+                          token_offset=token_offset, draw_offset=draw_offset, subset_a=subset_a,
+                          stream_id=stream_id)
+        out = dict(out or {})
+        if want_G and "G" not in out:
+            out["G"] = torch.empty(V, d, dtype=torch.float32, pin_memory=True)
+        if want_loss and "loss" not in out:
+            out["loss"] = torch.empty(T, dtype=torch.float32, pin_memory=True)
+        self._bind_stream()
+        st = self._L.dust_head_grad_host(self._h, ctypes.byref(prm), _ptr(H), _ptr(W),
+                                         _ptr(targets), _ptr(out.get("G")), _ptr(out.get("loss")),
+                                         None, None)
+        self._check(st)
+        return out
+
+    def mlp_grad(self, X, W_up, W_down, W_head, targets, *, K, sigma, seed=0, token_offset=0,
+                 draw_offset=0, stream_id=0, want_G=True, want_loss=True, want_rewards=False,
+                 want_g=False, out=None) -> dict:
+        """MLP up-projection estimator (bf16 inputs). Returns the requested fp32 outputs."""
+        for t, n in ((X, "X"), (W_up, "W_up"), (W_down, "W_down"), (W_head, "W_head"),
+                     (targets, "targets")):
+            self._dev(t, n)
+        T, d = X.shape
+        d_ff = W_up.shape[0]
+        V = W_head.shape[0]
+        prm = make_params(T, d, V, K, sigma, d_ff=d_ff, dtype=_dtype_code(X), seed=seed,
+                          token_offset=token_offset, draw_offset=draw_offset, stream_id=stream_id)
+        out = dict(out or {})
+        f32 = dict(dtype=torch.float32, device=X.device)
+        if want_G and "G" not in out:
+            out["G"] = torch.empty(d_ff, d, **f32)
+        if want_loss and "loss" not in out:
+            out["loss"] = torch.empty(T, **f32)
+        if want_rewards and "rewards" not in out:
+            out["rewards"] = torch.empty(T, K, **f32)
+        if want_g and "g" not in out:
+            out["g"] = torch.empty(T, d_ff, **f32)
+        self._bind_stream()
+        st = self._L.dust_mlp_grad(self._h, ctypes.byref(prm), _ptr(X), _ptr(W_up), _ptr(W_down),
+                                   _ptr(W_head), _ptr(targets), _ptr(out.get("G")),
+                                   _ptr(out.get("loss")), _ptr(out.get("rewards")),
+                                   _ptr(out.get("g")))
+        self._check(st)
+        return out
+
+    # -- instrumentation -------------------------------------------------------------
+    def set_stage_timing(self, enable: bool = True):
+        self._check(self._L.dust_set_stage_timing(self._h, 1 if enable else 0))
+
+    def stage_times(self) -> dict:
+        """Per-stage device milliseconds of the last call (stage timing must be on)."""
+        names = (ctypes.c_char_p * 16)()
+        ms = (ctypes.c_float * 16)()
+        n = self._L.dust_stage_times(self._h, names, ms, 16)
+        return {names[i].decode(): float(ms[i]) for i in range(min(n, 16))}
+
+    @property
+    def kernel_launches(self) -> int:
+        return int(self._L.dust_kernel_launches(self._h))
+
+    # -- debug exports -------------------------------------------------------------
+    def debug_philox(self, seed: int, ctr: torch.Tensor) -> torch.Tensor:
+        """Raw Philox4x32-10 words for counters ctr (n x 4, int32 storage of uint32)."""
+        self._dev(ctr, "ctr")
+        out = torch.empty_like(ctr)
+        self._bind_stream()
+        self._check(self._L.dust_debug_philox(self._h, seed & 0xFFFFFFFFFFFFFFFF, _ptr(ctr),
+                                              ctr.shape[0], _ptr(out)))
+        return out
+
+    def debug_gauss(self, nt, ni, nslots, *, tag=TAG_HEAD, seed=0, token_offset=0, draw_offset=0,
+                    stream_id=0) -> torch.Tensor:
+        prm = make_params(1, 1, 1, 1, 0.0, seed=seed, token_offset=token_offset,
+                          draw_offset=draw_offset, stream_id=stream_id)
+        out = torch.empty(nt, ni, nslots, dtype=torch.float32, device=f"cuda:{self.device}")
+        self._bind_stream()
+        self._check(self._L.dust_debug_gauss(self._h, ctypes.byref(prm), tag, nt, ni, nslots,
+                                             _ptr(out)))
+        return out
+
+
+_contexts: dict = {}
+
+
+def context(device: Optional[int] = None) -> Context:
+    """Per-device default context."""
+    if device is None:
+        device = torch.cuda.current_device()
+    ctx = _contexts.get(device)
+    if ctx is None:
+        ctx = _contexts[device] = Context(device)
+    return ctx
+
+
+def head_grad(H, W, targets, **kw) -> dict:
+    return context(H.device.index).head_grad(H, W, targets, **kw)
+
+
+def mlp_grad(X, W_up, W_down, W_head, targets, **kw) -> dict:
+    return context(X.device.index).mlp_grad(X, W_up, W_down, W_head, targets, **kw)

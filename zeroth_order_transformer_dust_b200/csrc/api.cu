@@ -1,0 +1,556 @@
+// C ABI of the estimator: validation, scratch management and the order of
+// the kernel stages. Every numerical step runs in the kernels this file
+// launches; nothing here computes on the host beyond index bookkeeping.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.cuh"
+
+using namespace dust;
+
+namespace {
+
+dust_status fail(dust_ctx* ctx, dust_status s, const char* fmt, ...) {
+  if (ctx) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    ctx->last_error = buf;
+  }
+  return s;
+}
+
+#define DUST_CU(call)                                                                   \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(ctx, DUST_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define DUST_TRY(expr)            \
+  do {                            \
+    dust_status s_ = (expr);      \
+    if (s_ != DUST_OK) return s_; \
+  } while (0)
+
+int64_t gcd64(int64_t a, int64_t b) {
+  while (b) {
+    const int64_t t = a % b;
+    a = b;
+    b = t;
+  }
+  return a < 0 ? -a : a;
+}
+
+// Inverse of a modulo m (gcd(a, m) = 1), extended Euclid.
+int64_t modinv(int64_t a, int64_t m) {
+  if (m == 1) return 0;
+  int64_t t = 0, nt = 1, r = m, nr = a % m;
+  while (nr != 0) {
+    const int64_t q = r / nr;
+    int64_t tmp = t - q * nt;
+    t = nt;
+    nt = tmp;
+    tmp = r - q * nr;
+    r = nr;
+    nr = tmp;
+  }
+  return t < 0 ? t + m : t;
+}
+
+int64_t default_stride(int64_t V) {
+  int64_t a = (int64_t)std::ceil((double)V * ((std::sqrt(5.0) - 1.0) / 2.0));
+  if (a < 1) a = 1;
+  while (gcd64(a, V) != 1) ++a;
+  return a;
+}
+
+dust_status check_params(const dust_params* p, int variant, char* msg, int msg_len) {
+  auto bad = [&](const char* why) {
+    if (msg && msg_len > 0) snprintf(msg, (size_t)msg_len, "%s", why);
+    return DUST_ERR_ARG;
+  };
+  if (!p) return bad("params is NULL");
+  if (variant != DUST_VARIANT_HEAD && variant != DUST_VARIANT_MLP) return bad("unknown variant");
+  if (p->T < 1) return bad("T must be >= 1");
+  if (p->d < 1) return bad("d must be >= 1");
+  if (p->V < 1) return bad("V must be >= 1");
+  if (p->V > 0x7fffffffLL) return bad("V must fit int32 targets");
+  if (p->K < 1) return bad("K must be >= 1");
+  if (!std::isfinite(p->sigma) || p->sigma < 0.0f) return bad("sigma must be finite and >= 0");
+  if (p->dtype != DUST_F32 && p->dtype != DUST_BF16) return bad("dtype must be DUST_F32 or DUST_BF16");
+  if (p->token_offset < 0 || p->token_offset + p->T > (1LL << 32))
+    return bad("token_offset + T must lie in [0, 2^32]");
+  if (p->draw_offset < 0 || p->draw_offset + (int64_t)p->K > (1LL << 32))
+    return bad("draw_offset + K must lie in [0, 2^32]");
+  if (p->stream_id >= (1u << 24)) return bad("stream_id must be < 2^24");
+  if (p->T > (1LL << 40) / p->V) return bad("T * V too large");
+  if (p->T > (1LL << 40) / p->K) return bad("T * K too large");
+  if (variant == DUST_VARIANT_HEAD) {
+    if (p->S > p->V) return bad("S must be <= V");
+    if (p->S > 0 && p->subset_a != 0) {
+      if (p->subset_a < 1) return bad("subset_a must be >= 1");
+      if (gcd64(p->subset_a, p->V) != 1) return bad("subset_a must be coprime to V");
+    }
+  } else {
+    if (p->d_ff < 1) return bad("d_ff must be >= 1");
+    if (p->S > 0) return bad("the MLP variant perturbs all d_ff channels: S must be <= 0");
+    if (p->dtype != DUST_BF16) return bad("the MLP variant takes bf16 inputs");
+    if (p->T > (1LL << 40) / p->d_ff) return bad("T * d_ff too large");
+  }
+  if (msg && msg_len > 0) msg[0] = 0;
+  return DUST_OK;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+dust_status ensure(dust_ctx* ctx, Buf& b, size_t bytes) {
+  if (bytes == 0 || b.bytes >= bytes) return DUST_OK;
+  if (b.p) {
+    cudaStreamSynchronize(ctx->stream);
+    cudaFree(b.p);
+    b.p = nullptr;
+    b.bytes = 0;
+  }
+  const size_t gran = 2u << 20;
+  const size_t nb = (bytes + gran - 1) / gran * gran;
+  if (cudaMalloc(&b.p, nb) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ctx, DUST_ERR_OOM, "cudaMalloc of %zu bytes failed", nb);
+  }
+  b.bytes = nb;
+  return DUST_OK;
+}
+
+dust_status finish(dust_ctx* ctx, uint32_t flags) {
+  DUST_CU(cudaGetLastError());
+  if (flags & DUST_FLAG_ASYNC) return DUST_OK;
+  return dust_check(ctx);
+}
+
+dust_status run_gemm(dust_ctx* ctx, const GemmDesc& g, const EpiDesc& e) {
+  ctx->launches += 1;
+  if (tc_gemm_supported(g, e)) {
+    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count));
+  } else {
+    DUST_CU(launch_gemm_simt(ctx->stream, g, e));
+  }
+  return DUST_OK;
+}
+
+size_t elem_size(int dtype) { return dtype == DUST_BF16 ? 2 : 4; }
+
+// Stage marks: mark(ctx, nullptr) opens a call, mark(ctx, "name") closes the
+// stage that ran since the previous mark.
+void mark(dust_ctx* ctx, const char* name) {
+  if (!ctx->timing) return;
+  if (!name) ctx->nmarks = 0;
+  if (ctx->nmarks >= dust_ctx::kMaxMarks) return;
+  cudaEventRecord(ctx->ev[ctx->nmarks], ctx->stream);
+  ctx->mark_name[ctx->nmarks] = name;
+  ctx->nmarks++;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dust_status_string(dust_status s) {
+  switch (s) {
+    case DUST_OK: return "DUST_OK";
+    case DUST_ERR_ARG: return "DUST_ERR_ARG";
+    case DUST_ERR_CUDA: return "DUST_ERR_CUDA";
+    case DUST_ERR_OOM: return "DUST_ERR_OOM";
+    case DUST_ERR_BOUNDS: return "DUST_ERR_BOUNDS";
+    case DUST_ERR_TIMEOUT: return "DUST_ERR_TIMEOUT";
+    case DUST_ERR_UNSUPPORTED: return "DUST_ERR_UNSUPPORTED";
+  }
+  return "DUST_ERR_UNKNOWN";
+}
+
+dust_status dust_validate(const dust_params* p, int variant, char* msg, int msg_len) {
+  return check_params(p, variant, msg, msg_len);
+}
+
+int64_t dust_subset_stride(const dust_params* p) {
+  if (check_params(p, DUST_VARIANT_HEAD, nullptr, 0) != DUST_OK || p->S <= 0) return 0;
+  return p->subset_a ? p->subset_a % p->V : default_stride(p->V);
+}
+
+dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
+  if (!out) return DUST_ERR_ARG;
+  *out = nullptr;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return DUST_ERR_CUDA;
+  }
+  dust_ctx* ctx = new dust_ctx();
+  ctx->device = device;
+  ctx->stream = (cudaStream_t)cuda_stream;
+  if (cudaSetDevice(device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess ||
+      cudaMalloc(&ctx->d_status, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMallocHost(&ctx->h_status, sizeof(uint32_t)) != cudaSuccess ||
+      cudaMemset(ctx->d_status, 0, sizeof(uint32_t)) != cudaSuccess) {
+    cudaGetLastError();
+    dust_destroy(ctx);
+    return DUST_ERR_CUDA;
+  }
+  *out = ctx;
+  return DUST_OK;
+}
+
+dust_status dust_set_stream(dust_ctx* ctx, void* cuda_stream) {
+  if (!ctx) return DUST_ERR_ARG;
+  ctx->stream = (cudaStream_t)cuda_stream;
+  return DUST_OK;
+}
+
+void dust_destroy(dust_ctx* ctx) {
+  if (!ctx) return;
+  cudaSetDevice(ctx->device);
+  if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+  Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
+                 &ctx->gT, &ctx->hT, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
+                 &ctx->mlp_da, &ctx->mlp_dh, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
+                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv};
+  for (Buf* b : bufs)
+    if (b->p) cudaFree(b->p);
+  for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
+    if (ctx->ev[i]) cudaEventDestroy(ctx->ev[i]);
+  if (ctx->d_status) cudaFree(ctx->d_status);
+  if (ctx->h_status) cudaFreeHost(ctx->h_status);
+  cudaGetLastError();
+  delete ctx;
+}
+
+const char* dust_last_error(const dust_ctx* ctx) {
+  return ctx ? ctx->last_error.c_str() : "no context";
+}
+
+dust_status dust_check(dust_ctx* ctx) {
+  if (!ctx) return DUST_ERR_ARG;
+  DUST_CU(cudaMemcpyAsync(ctx->h_status, ctx->d_status, sizeof(uint32_t), cudaMemcpyDeviceToHost,
+                          ctx->stream));
+  DUST_CU(cudaStreamSynchronize(ctx->stream));
+  const uint32_t st = *ctx->h_status;
+  if (st) DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), ctx->stream));
+  if (st & kStatusBadTarget) return fail(ctx, DUST_ERR_BOUNDS, "a target lies outside [0, V)");
+  if (st & kStatusTimeout) return fail(ctx, DUST_ERR_TIMEOUT, "a bounded device wait expired");
+  return DUST_OK;
+}
+
+dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, const void* W,
+                           const int32_t* targets, float* G_out, float* loss_out,
+                           float* rewards_out, float* g_out) {
+  if (!ctx) return DUST_ERR_ARG;
+  char why[256];
+  if (check_params(pp, DUST_VARIANT_HEAD, why, sizeof(why)) != DUST_OK)
+    return fail(ctx, DUST_ERR_ARG, "%s", why);
+  const dust_params p = *pp;
+  if (!H || !W || !targets) return fail(ctx, DUST_ERR_ARG, "H, W and targets must be non-NULL");
+  if (!aligned(H, 16) || !aligned(W, 16) || !aligned(targets, 4) || !aligned(G_out, 4) ||
+      !aligned(loss_out, 4) || !aligned(rewards_out, 4) || !aligned(g_out, 4))
+    return fail(ctx, DUST_ERR_ARG, "H and W must be 16-byte aligned, the other pointers 4-byte");
+  DUST_CU(cudaSetDevice(ctx->device));
+  const bool subset = p.S > 0;
+  const int64_t a = subset ? (p.subset_a ? p.subset_a % p.V : default_stride(p.V)) : 0;
+  const int64_t a_inv = subset ? modinv(a, p.V) : 0;
+  const size_t TV = (size_t)p.T * (size_t)p.V;
+  DUST_TRY(ensure(ctx, ctx->z, TV * 4));
+  DUST_TRY(ensure(ctx, ctx->lse, (size_t)p.T * 4));
+  DUST_TRY(ensure(ctx, ctx->gop, TV * elem_size(p.dtype)));
+  float* loss = loss_out;
+  if (!loss) {
+    DUST_TRY(ensure(ctx, ctx->loss, (size_t)p.T * 4));
+    loss = (float*)ctx->loss.p;
+  }
+  float* Z = (float*)ctx->z.p;
+  const cudaStream_t st = ctx->stream;
+  DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), st));
+  mark(ctx, nullptr);
+
+  // 1. clean logits z = H W^T (permuted columns for subset draws)
+  GemmDesc g{};
+  g.M = p.T; g.N = p.V; g.K = p.d;
+  g.A = H; g.lda = p.d; g.a_kmajor = true;
+  g.B = W; g.ldb = p.d; g.b_kmajor = true;
+  g.b_row_mul = subset ? a : 0;
+  g.dtype = p.dtype;
+  EpiDesc e{};
+  e.kind = kEpiF32; e.C = Z; e.ldc = p.V;
+  DUST_TRY(run_gemm(ctx, g, e));
+  mark(ctx, "clean_gemm");
+  // 2. log-sum-exp, clean loss, softmax in place
+  DUST_CU(launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, (float*)ctx->lse.p, loss,
+                          true, ctx->d_status));
+  ctx->launches += 1;
+  mark(ctx, "lse");
+  // 3. perturbed losses, rewards, g
+  if (!subset) {
+    float* r = rewards_out;
+    if (!r) {
+      DUST_TRY(ensure(ctx, ctx->rew, (size_t)p.T * p.K * 4));
+      r = (float*)ctx->rew.p;
+    }
+    DUST_TRY(ensure(ctx, ctx->part, (size_t)p.T * full_vocab_nslab(p.V) * p.K * 4));
+    DUST_CU(launch_full_reward_partial(st, p, Z, (float*)ctx->part.p));
+    DUST_CU(launch_full_reward_combine(st, p, (float*)ctx->part.p, targets, r));
+    ctx->launches += 2;
+    mark(ctx, "reward");
+    DUST_CU(launch_full_g(st, p, r, g_out, ctx->gop.p));
+    ctx->launches += 1;
+    mark(ctx, "g");
+  } else {
+    float* gacc = nullptr;
+    const size_t gb = subset_gacc_bytes(p.T, p.V, ctx->max_smem_optin);
+    if (gb) {
+      DUST_TRY(ensure(ctx, ctx->part, gb));
+      gacc = (float*)ctx->part.p;
+    }
+    DUST_CU(launch_subset_impl(st, p, a, a_inv, Z, targets, rewards_out, g_out, ctx->gop.p, gacc,
+                               ctx->max_smem_optin));
+    ctx->launches += 1;
+    mark(ctx, "subset_draws");
+  }
+  // 4. G_W = sum_t g_t h_t^T (rows un-permuted on the store)
+  if (G_out) {
+    GemmDesc w{};
+    w.M = p.V; w.N = p.d; w.K = p.T;
+    w.A = ctx->gop.p; w.lda = p.V; w.a_kmajor = false;
+    w.B = H; w.ldb = p.d; w.b_kmajor = false;
+    w.dtype = p.dtype;
+    EpiDesc we{};
+    we.kind = kEpiF32; we.C = G_out; we.ldc = p.d; we.c_row_mul = subset ? a : 0;
+    DUST_TRY(run_gemm(ctx, w, we));
+    mark(ctx, "gw_gemm");
+  }
+  return finish(ctx, p.flags);
+}
+
+dust_status dust_head_grad_host(dust_ctx* ctx, const dust_params* pp, const void* H, const void* W,
+                                const int32_t* targets, float* G_out, float* loss_out,
+                                float* rewards_out, float* g_out) {
+  if (!ctx) return DUST_ERR_ARG;
+  char why[256];
+  if (check_params(pp, DUST_VARIANT_HEAD, why, sizeof(why)) != DUST_OK)
+    return fail(ctx, DUST_ERR_ARG, "%s", why);
+  if (!H || !W || !targets) return fail(ctx, DUST_ERR_ARG, "H, W and targets must be non-NULL");
+  const dust_params p = *pp;
+  DUST_CU(cudaSetDevice(ctx->device));
+  const size_t es = elem_size(p.dtype);
+  const size_t hb = (size_t)p.T * p.d * es, wb = (size_t)p.V * p.d * es, yb = (size_t)p.T * 4;
+  DUST_TRY(ensure(ctx, ctx->in_h, hb));
+  DUST_TRY(ensure(ctx, ctx->in_w, wb));
+  DUST_TRY(ensure(ctx, ctx->in_y, yb));
+  if (G_out) DUST_TRY(ensure(ctx, ctx->out_g, (size_t)p.V * p.d * 4));
+  if (loss_out) DUST_TRY(ensure(ctx, ctx->out_loss, (size_t)p.T * 4));
+  if (rewards_out) DUST_TRY(ensure(ctx, ctx->out_r, (size_t)p.T * p.K * 4));
+  if (g_out) DUST_TRY(ensure(ctx, ctx->out_gv, (size_t)p.T * p.V * 4));
+  const cudaStream_t st = ctx->stream;
+  DUST_CU(cudaMemcpyAsync(ctx->in_h.p, H, hb, cudaMemcpyHostToDevice, st));
+  DUST_CU(cudaMemcpyAsync(ctx->in_w.p, W, wb, cudaMemcpyHostToDevice, st));
+  DUST_CU(cudaMemcpyAsync(ctx->in_y.p, targets, yb, cudaMemcpyHostToDevice, st));
+  dust_params q = p;
+  q.flags |= DUST_FLAG_ASYNC;
+  DUST_TRY(dust_head_grad(ctx, &q, ctx->in_h.p, ctx->in_w.p, (const int32_t*)ctx->in_y.p,
+                          G_out ? (float*)ctx->out_g.p : nullptr,
+                          loss_out ? (float*)ctx->out_loss.p : nullptr,
+                          rewards_out ? (float*)ctx->out_r.p : nullptr,
+                          g_out ? (float*)ctx->out_gv.p : nullptr));
+  if (G_out) DUST_CU(cudaMemcpyAsync(G_out, ctx->out_g.p, (size_t)p.V * p.d * 4, cudaMemcpyDeviceToHost, st));
+  if (loss_out) DUST_CU(cudaMemcpyAsync(loss_out, ctx->out_loss.p, (size_t)p.T * 4, cudaMemcpyDeviceToHost, st));
+  if (rewards_out) DUST_CU(cudaMemcpyAsync(rewards_out, ctx->out_r.p, (size_t)p.T * p.K * 4, cudaMemcpyDeviceToHost, st));
+  if (g_out) DUST_CU(cudaMemcpyAsync(g_out, ctx->out_gv.p, (size_t)p.T * p.V * 4, cudaMemcpyDeviceToHost, st));
+  if (p.flags & DUST_FLAG_ASYNC) {
+    DUST_CU(cudaStreamSynchronize(st));
+    return DUST_OK;
+  }
+  return dust_check(ctx);
+}
+
+dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, const void* W_up,
+                          const void* W_down, const void* W_head, const int32_t* targets,
+                          float* G_up_out, float* loss_out, float* rewards_out, float* g_out) {
+  if (!ctx) return DUST_ERR_ARG;
+  char why[256];
+  if (check_params(pp, DUST_VARIANT_MLP, why, sizeof(why)) != DUST_OK)
+    return fail(ctx, DUST_ERR_ARG, "%s", why);
+  const dust_params p = *pp;
+  if (!X || !W_up || !W_down || !W_head || !targets)
+    return fail(ctx, DUST_ERR_ARG, "X, W_up, W_down, W_head and targets must be non-NULL");
+  if (!aligned(X, 16) || !aligned(W_up, 16) || !aligned(W_down, 16) || !aligned(W_head, 16) ||
+      !aligned(targets, 4) || !aligned(G_up_out, 4) || !aligned(loss_out, 4) ||
+      !aligned(rewards_out, 4) || !aligned(g_out, 4))
+    return fail(ctx, DUST_ERR_ARG, "weights and X must be 16-byte aligned, the rest 4-byte");
+  DUST_CU(cudaSetDevice(ctx->device));
+  const cudaStream_t st = ctx->stream;
+  const int64_t T = p.T, d = p.d, dff = p.d_ff, V = p.V, K = p.K;
+  DUST_TRY(ensure(ctx, ctx->mlp_u, (size_t)T * dff * 4));
+  DUST_TRY(ensure(ctx, ctx->mlp_a, (size_t)T * dff * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_h, (size_t)T * d * 2));
+  DUST_TRY(ensure(ctx, ctx->z, (size_t)T * V * 4));
+  DUST_TRY(ensure(ctx, ctx->lse, (size_t)T * 4));
+  DUST_TRY(ensure(ctx, ctx->gop, (size_t)T * dff * 2));
+  float* loss = loss_out;
+  if (!loss) {
+    DUST_TRY(ensure(ctx, ctx->loss, (size_t)T * 4));
+    loss = (float*)ctx->loss.p;
+  }
+  float* r = rewards_out;
+  if (!r) {
+    DUST_TRY(ensure(ctx, ctx->rew, (size_t)T * K * 4));
+    r = (float*)ctx->rew.p;
+  }
+  float* u = (float*)ctx->mlp_u.p;
+  __nv_bfloat16* abf = (__nv_bfloat16*)ctx->mlp_a.p;
+  __nv_bfloat16* hbf = (__nv_bfloat16*)ctx->mlp_h.p;
+  float* Z = (float*)ctx->z.p;
+  DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), st));
+  mark(ctx, nullptr);
+
+  // clean pass: u = x W_up^T (fp32), a = bf16(GELU(u)), h = bf16(x + a W_down^T), z = h W_head^T
+  {
+    GemmDesc g{};
+    g.M = T; g.N = dff; g.K = d; g.A = X; g.lda = d; g.a_kmajor = true;
+    g.B = W_up; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
+    EpiDesc e{};
+    e.kind = kEpiGelu; e.C = u; e.Cb = abf; e.ldc = dff;
+    DUST_TRY(run_gemm(ctx, g, e));
+  }
+  {
+    GemmDesc g{};
+    g.M = T; g.N = d; g.K = dff; g.A = abf; g.lda = dff; g.a_kmajor = true;
+    g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+    EpiDesc e{};
+    e.kind = kEpiResidBF16; e.Cb = hbf; e.ldc = d; e.resid = X; e.ldr = d;
+    DUST_TRY(run_gemm(ctx, g, e));
+  }
+  {
+    GemmDesc g{};
+    g.M = T; g.N = V; g.K = d; g.A = hbf; g.lda = d; g.a_kmajor = true;
+    g.B = W_head; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
+    EpiDesc e{};
+    e.kind = kEpiF32; e.C = Z; e.ldc = V;
+    DUST_TRY(run_gemm(ctx, g, e));
+  }
+  mark(ctx, "clean_gemms");
+  DUST_CU(launch_lse_rows(st, Z, T, V, targets, 0, (float*)ctx->lse.p, loss, true, ctx->d_status));
+  ctx->launches += 1;
+  mark(ctx, "lse");
+
+  // perturbed passes, a chunk of tokens (all K draws each) at a time
+  const int64_t max_rows = 131072;
+  int64_t tchunk = max_rows / K;
+  if (tchunk < 1) tchunk = 1;
+  if (tchunk > T) tchunk = T;
+  const int64_t rows_cap = tchunk * K;
+  const int nparts = (int)((V + 127) / 128);
+  DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * dff * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_dh, (size_t)rows_cap * d * 2));
+  DUST_TRY(ensure(ctx, ctx->part, (size_t)rows_cap * nparts * 4));
+  DUST_TRY(ensure(ctx, ctx->dzy, (size_t)rows_cap * 4));
+  __nv_bfloat16* da = (__nv_bfloat16*)ctx->mlp_da.p;
+  __nv_bfloat16* dh = (__nv_bfloat16*)ctx->mlp_dh.p;
+  for (int64_t t0 = 0; t0 < T; t0 += tchunk) {
+    const int64_t nt = (t0 + tchunk <= T) ? tchunk : T - t0;
+    const int64_t rows = nt * K;
+    DUST_CU(launch_mlp_delta_a(st, p, u, t0, nt, da, true, nullptr));
+    ctx->launches += 1;
+    {
+      GemmDesc g{};
+      g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = dff; g.a_kmajor = true;
+      g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      EpiDesc e{};
+      e.kind = kEpiBF16; e.Cb = dh; e.ldc = d;
+      DUST_TRY(run_gemm(ctx, g, e));
+    }
+    {
+      GemmDesc g{};
+      g.M = rows; g.N = V; g.K = d; g.A = dh; g.lda = d; g.a_kmajor = true;
+      g.B = W_head; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
+      DUST_CU(launch_reward_gemm_simt(st, g, Z, targets, t0, p.K, (float*)ctx->part.p,
+                                      (float*)ctx->dzy.p));
+    }
+    DUST_CU(launch_reward_combine_rows(st, (float*)ctx->part.p, nparts, (float*)ctx->dzy.p, rows,
+                                       t0 * K, p.K, r));
+    ctx->launches += 2;
+  }
+  mark(ctx, "perturbed");
+  DUST_CU(launch_mlp_g(st, p, r, g_out, ctx->gop.p));
+  ctx->launches += 1;
+  mark(ctx, "g");
+  if (G_up_out) {
+    GemmDesc w{};
+    w.M = dff; w.N = d; w.K = T; w.A = ctx->gop.p; w.lda = dff; w.a_kmajor = false;
+    w.B = X; w.ldb = d; w.b_kmajor = false; w.dtype = DUST_BF16;
+    EpiDesc we{};
+    we.kind = kEpiF32; we.C = G_up_out; we.ldc = d;
+    DUST_TRY(run_gemm(ctx, w, we));
+    mark(ctx, "gw_gemm");
+  }
+  return finish(ctx, p.flags);
+}
+
+dust_status dust_set_stage_timing(dust_ctx* ctx, int enable) {
+  if (!ctx) return DUST_ERR_ARG;
+  DUST_CU(cudaSetDevice(ctx->device));
+  if (enable && !ctx->ev[0]) {
+    for (int i = 0; i < dust_ctx::kMaxMarks; ++i) DUST_CU(cudaEventCreate(&ctx->ev[i]));
+  }
+  ctx->timing = enable != 0;
+  ctx->nmarks = 0;
+  return DUST_OK;
+}
+
+int dust_stage_times(dust_ctx* ctx, const char** names, float* ms, int cap) {
+  if (!ctx || !ctx->timing || ctx->nmarks < 2) return 0;
+  cudaSetDevice(ctx->device);
+  if (cudaEventSynchronize(ctx->ev[ctx->nmarks - 1]) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const int n = ctx->nmarks - 1;
+  for (int i = 0; i < n && i < cap; ++i) {
+    float t = 0.0f;
+    cudaEventElapsedTime(&t, ctx->ev[i], ctx->ev[i + 1]);
+    if (names) names[i] = ctx->mark_name[i + 1];
+    if (ms) ms[i] = t;
+  }
+  return n;
+}
+
+int64_t dust_kernel_launches(const dust_ctx* ctx) { return ctx ? ctx->launches : 0; }
+
+dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4, int64_t n,
+                              uint32_t* out) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (n < 0 || (n > 0 && (!ctr4 || !out))) return fail(ctx, DUST_ERR_ARG, "bad philox arguments");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(launch_debug_philox(ctx->stream, seed, ctr4, n, out));
+  ctx->launches += 1;
+  DUST_CU(cudaStreamSynchronize(ctx->stream));
+  return DUST_OK;
+}
+
+dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag, int64_t nt,
+                             int64_t ni, int64_t nslots, float* out) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (!p || nt < 0 || ni < 0 || nslots < 0 || tag < 0 || tag > 255 || !out ||
+      p->stream_id >= (1u << 24) || p->token_offset < 0 || p->draw_offset < 0 ||
+      p->token_offset + nt > (1LL << 32) || p->draw_offset + ni > (1LL << 32))
+    return fail(ctx, DUST_ERR_ARG, "bad gauss arguments");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(launch_debug_gauss(ctx->stream, *p, tag, nt, ni, nslots, out));
+  ctx->launches += 1;
+  DUST_CU(cudaStreamSynchronize(ctx->stream));
+  return DUST_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,132 @@
+// Internal declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+#include <string>
+
+#include "../../include/dust.h"
+
+namespace dust {
+
+// Bits of the device status word.
+enum : uint32_t {
+  kStatusBadTarget = 1u << 0,
+  kStatusTimeout = 1u << 1,
+};
+
+struct Buf {
+  void* p = nullptr;
+  size_t bytes = 0;
+};
+
+// Launch geometry of the GEMMs: A(m, k) and B(n, k) addressing.
+struct GemmDesc {
+  int64_t M, N, K;
+  const void* A;
+  int64_t lda;        // A(m,k) = A[m*lda + k] if a_kmajor, else A[k*lda + m]
+  bool a_kmajor;
+  const void* B;
+  int64_t ldb;        // B(n,k) = B[n*ldb + k] if b_kmajor, else B[k*ldb + n]
+  bool b_kmajor;
+  int64_t b_row_mul;  // nonzero: B row n is source row (n * b_row_mul) mod N
+  int dtype;          // DUST_F32 or DUST_BF16 for both operands
+};
+
+enum EpiKind {
+  kEpiF32 = 0,        // C[m*ldc + n] = acc   (row m written at (m*c_row_mul) mod M if set)
+  kEpiBF16 = 1,       // Cb[m*ldc + n] = bf16(acc)
+  kEpiGelu = 2,       // C = acc (u, fp32) and Cb = bf16(GELU(acc))
+  kEpiResidBF16 = 3,  // Cb = bf16(resid[m*ldr + n] + acc), resid in dtype
+};
+
+struct EpiDesc {
+  int kind = kEpiF32;
+  float* C = nullptr;
+  __nv_bfloat16* Cb = nullptr;
+  int64_t ldc = 0;
+  int64_t c_row_mul = 0;
+  const void* resid = nullptr;
+  int64_t ldr = 0;
+};
+
+}  // namespace dust
+
+struct dust_ctx {
+  int device = 0;
+  cudaStream_t stream = nullptr;
+  int sm_count = 0;
+  int max_smem_optin = 0;
+  std::string last_error;
+  uint32_t* d_status = nullptr;
+  uint32_t* h_status = nullptr;  // pinned
+  // stage timing (events recorded between the stages of a call)
+  static constexpr int kMaxMarks = 16;
+  bool timing = false;
+  cudaEvent_t ev[kMaxMarks] = {};
+  const char* mark_name[kMaxMarks] = {};
+  int nmarks = 0;
+  int64_t launches = 0;
+  // scratch, grown on demand
+  dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, dzy, mlp_u, mlp_a, mlp_h, mlp_da, mlp_dh,
+      in_h, in_w, in_y, out_g, out_loss, out_r, out_gv;
+};
+
+namespace dust {
+
+// Kernel launchers (all enqueue on `st`, return cudaGetLastError()).
+cudaError_t launch_debug_philox(cudaStream_t st, uint64_t seed, const uint32_t* ctr, int64_t n,
+                                uint32_t* out);
+cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, int64_t nt,
+                               int64_t ni, int64_t nslots, float* out);
+
+cudaError_t launch_gemm_simt(cudaStream_t st, const GemmDesc& g, const EpiDesc& e);
+
+// Row-wise log-sum-exp of Z (T x V). Writes lse[t], loss[t] = lse - Z[t, col(y_t)]
+// with col(y) = y (col_mul == 0) or (y * col_mul) mod V; if to_prob, overwrites Z
+// with exp(Z - lse). Sets kStatusBadTarget for targets outside [0, V).
+cudaError_t launch_lse_rows(cudaStream_t st, float* Z, int64_t T, int64_t V, const int32_t* y,
+                            int64_t col_mul, float* lse, float* loss, bool to_prob,
+                            uint32_t* status);
+
+// Full-vocabulary reward, stage 1: partial sums sum_j p_j expm1(sigma eps_j) per
+// (token, slab, draw) -> part[(t * nslab + slab) * K + i]. Returns nslab.
+int full_vocab_nslab(int64_t V);
+cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* P,
+                                       float* part);
+// Stage 2: r[t*K + i] = sigma eps_y - log1p(sum_slab part).
+cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, const float* part,
+                                       const int32_t* y, float* r);
+// Stage 3: g_t = -(1/(K sigma)) sum_i r_i eps_i; writes g (fp32, optional) and the
+// GEMM operand gop (bf16 or fp32 by p.dtype).
+cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
+                          void* gop);
+
+// Subset draws, fused reward + accumulation. P is the probability matrix in
+// permuted column order (column q holds vocabulary index (a q) mod V).
+// gacc: T x V fp32 accumulator, needed only when a row does not fit in
+// shared memory (subset_gacc_bytes() > 0).
+size_t subset_gacc_bytes(int64_t T, int64_t V, int max_smem_optin);
+cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
+                               const float* P, const int32_t* y, float* rewards, float* g_out,
+                               void* gop, float* gacc, int max_smem_optin);
+
+// Tensor-core GEMM (tcgen05): shapes it takes, and its launcher.
+bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e);
+cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count);
+
+// MLP helpers.
+cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const float* u,
+                               int64_t t0, int64_t nt, __nv_bfloat16* da, bool round_bf16,
+                               float* da_f32);
+cudaError_t launch_reward_gemm_simt(cudaStream_t st, const GemmDesc& g, const float* P,
+                                    const int32_t* y, int64_t t0, int32_t K, float* part,
+                                    float* dzy);
+cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int nparts,
+                                       const float* dzy, int64_t rows, int64_t row0, int32_t K,
+                                       float* r);
+cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
+                         void* gop);
+
+}  // namespace dust

@@ -1,0 +1,231 @@
+// Hidden-MLP up-projection draws ("Dust：无需反向传播的Transformer零阶预训练",
+// §1: noise on the linear layer's output u = W_up x; 减少干扰: only what the
+// perturbation changes is recomputed from cached x, u and the clean logits):
+//   da = GELU(u + sigma eps) - GELU(u)        (rows (t, i), d_ff columns)
+//   dh = da W_down^T,  dz = dh W_head^T,
+//   r  = dz_y - log1p(sum_j p_j expm1(dz_j)),
+//   g_t = -(1/(K sigma)) sum_i r_i eps_i.
+#include "internal.cuh"
+#include "noise.cuh"
+
+namespace dust {
+namespace {
+
+__device__ __forceinline__ float gelu_erf(float x) {
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+// One thread per (row, 128-channel block, lane).
+__global__ void k_mlp_delta_a(Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3, float sigma,
+                              int64_t d_ff, int32_t K, const float* __restrict__ u, int64_t t0,
+                              int64_t rows, __nv_bfloat16* __restrict__ da_bf,
+                              float* __restrict__ da_f32) {
+  const int64_t nblk = (d_ff + 127) / 128;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= rows * nblk * 32) return;
+  const uint32_t lane = (uint32_t)(gid & 31);
+  const int64_t rest = gid >> 5;
+  const int64_t blk = rest % nblk;
+  const int64_t row = rest / nblk;
+  const int64_t t = t0 + row / K;
+  const int32_t i = (int32_t)(row % K);
+  U4 c{slot_ctr0((uint32_t)blk, lane), t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3};
+  const G4 g = gauss4(philox10(c, key.k0, key.k1));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t ch = blk * 128 + lane + 32 * j;
+    if (ch < d_ff) {
+      const float uv = u[t * d_ff + ch];
+      const float d = gelu_erf(uv + sigma * g.v[j]) - gelu_erf(uv);
+      if (da_bf) da_bf[row * d_ff + ch] = __float2bfloat16_rn(d);
+      if (da_f32) da_f32[row * d_ff + ch] = d;
+    }
+  }
+}
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+constexpr int BM = 128, BN = 128, BKT = 16, PAD = 4;
+
+// dz tile = dh (rows x d) . W_head^T, fused reward epilogue: per row and
+// 128-column tile, sum_n p[t(row), n] expm1(dz) -> part[row * nparts + tile];
+// dz at the target column -> dzy[row].
+template <typename TI>
+__global__ __launch_bounds__(256) void k_reward_gemm_simt(GemmDesc g, const float* __restrict__ P,
+                                                          const int32_t* __restrict__ y,
+                                                          int64_t t0, int32_t K,
+                                                          float* __restrict__ part,
+                                                          float* __restrict__ dzy) {
+  __shared__ __align__(16) float As[BKT][BM + PAD];
+  __shared__ __align__(16) float Bs[BKT][BN + PAD];
+  const TI* A = (const TI*)g.A;
+  const TI* B = (const TI*)g.B;
+  const int64_t m0 = (int64_t)blockIdx.y * BM;
+  const int64_t n0 = (int64_t)blockIdx.x * BN;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int tid = threadIdx.x;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  for (int64_t k0 = 0; k0 < g.K; k0 += BKT) {
+    {
+      const int r = tid >> 1, kk0 = (tid & 1) * 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int64_t k = k0 + kk0 + q;
+        const int64_t ma = m0 + r, nb = n0 + r;
+        As[kk0 + q][r] = (ma < g.M && k < g.K) ? to_f(A[ma * g.lda + k]) : 0.0f;
+        Bs[kk0 + q][r] = (nb < g.N && k < g.K) ? to_f(B[nb * g.ldb + k]) : 0.0f;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BKT; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const int64_t nparts = (g.N + BN - 1) / BN;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    const bool mrow = m < g.M;
+    const int64_t t = t0 + (mrow ? m / K : 0);
+    int32_t yt = mrow ? y[t] : -1;
+    if (yt < 0 || (int64_t)yt >= g.N) yt = 0;  // reported by the loss kernel
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
+      if (mrow && n < g.N) {
+        s = fmaf(P[t * g.N + n], expm1f(acc[i][j]), s);
+        if (n == yt) dzy[m] = acc[i][j];
+      }
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (mrow && tx == 0) part[m * nparts + blockIdx.x] = s;
+  }
+}
+
+__global__ void k_reward_combine_rows(const float* __restrict__ part, int nparts,
+                                      const float* __restrict__ dzy, int64_t rows, int64_t row0,
+                                      float* __restrict__ r) {
+  const int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= rows) return;
+  float s = 0.0f;
+  for (int q = 0; q < nparts; ++q) s += part[m * nparts + q];
+  r[row0 + m] = dzy[m] - log1pf(s);
+}
+
+template <typename TO>
+__device__ __forceinline__ void store_op(TO* p, int64_t o, float v);
+template <>
+__device__ __forceinline__ void store_op<float>(float* p, int64_t o, float v) { p[o] = v; }
+template <>
+__device__ __forceinline__ void store_op<__nv_bfloat16>(__nv_bfloat16* p, int64_t o, float v) {
+  p[o] = __float2bfloat16_rn(v);
+}
+
+// g_t[c] = scale * sum_i r[t*K + i] eps(t, i, c): one warp per 128 channels.
+template <typename TO>
+__global__ __launch_bounds__(256) void k_noise_g(Key key, uint32_t t_off, uint32_t i_off,
+                                                 uint32_t ctr3, float scale, int64_t width,
+                                                 int32_t K, const float* __restrict__ r,
+                                                 float* __restrict__ g_out, TO* __restrict__ gop) {
+  __shared__ float rs[1024];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t t = blockIdx.x;
+  const int64_t blk = (int64_t)blockIdx.y * 8 + warp;
+  const uint32_t t_abs = t_off + (uint32_t)t;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i0 = 0; i0 < K; i0 += 1024) {
+    const int n = min(1024, K - i0);
+    __syncthreads();
+    for (int q = threadIdx.x; q < n; q += blockDim.x) rs[q] = r[t * K + i0 + q];
+    __syncthreads();
+    if (blk * 128 < width) {
+      for (int ii = 0; ii < n; ++ii) {
+        U4 c{slot_ctr0((uint32_t)blk, (uint32_t)lane), t_abs, i_off + (uint32_t)(i0 + ii), ctr3};
+        const G4 g = gauss4(philox10(c, key.k0, key.k1));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = fmaf(rs[ii], g.v[j], acc[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t ch = blk * 128 + lane + 32 * j;
+    if (ch < width) {
+      const float v = acc[j] * scale;
+      if (g_out) g_out[t * width + ch] = v;
+      store_op<TO>(gop, t * width + ch, v);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const float* u, int64_t t0,
+                               int64_t nt, __nv_bfloat16* da, bool round_bf16, float* da_f32) {
+  const int64_t rows = nt * p.K;
+  const int64_t nblk = (p.d_ff + 127) / 128;
+  const int64_t total = rows * nblk * 32;
+  if (total <= 0) return cudaSuccess;
+  const int threads = 256;
+  k_mlp_delta_a<<<(unsigned)((total + threads - 1) / threads), threads, 0, st>>>(
+      key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
+      ctr3_of(kTagMlpUp, p.stream_id), p.sigma, p.d_ff, p.K, u, t0, rows,
+      round_bf16 ? da : nullptr, da_f32);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reward_gemm_simt(cudaStream_t st, const GemmDesc& g, const float* P,
+                                    const int32_t* y, int64_t t0, int32_t K, float* part,
+                                    float* dzy) {
+  dim3 grid((unsigned)((g.N + BN - 1) / BN), (unsigned)((g.M + BM - 1) / BM));
+  if (g.dtype == DUST_BF16)
+    k_reward_gemm_simt<__nv_bfloat16><<<grid, 256, 0, st>>>(g, P, y, t0, K, part, dzy);
+  else
+    k_reward_gemm_simt<float><<<grid, 256, 0, st>>>(g, P, y, t0, K, part, dzy);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int nparts,
+                                       const float* dzy, int64_t rows, int64_t row0, int32_t K,
+                                       float* r) {
+  (void)K;
+  const int threads = 256;
+  k_reward_combine_rows<<<(unsigned)((rows + threads - 1) / threads), threads, 0, st>>>(
+      part, nparts, dzy, rows, row0, r);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
+                         void* gop) {
+  dim3 grid((unsigned)p.T, (unsigned)((p.d_ff + 1023) / 1024));
+  const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
+  const Key key = key_of(p.seed);
+  const uint32_t c3 = ctr3_of(kTagMlpUp, p.stream_id);
+  if (p.dtype == DUST_BF16)
+    k_noise_g<__nv_bfloat16><<<grid, 256, 0, st>>>(key, (uint32_t)p.token_offset,
+        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (__nv_bfloat16*)gop);
+  else
+    k_noise_g<float><<<grid, 256, 0, st>>>(key, (uint32_t)p.token_offset,
+        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (float*)gop);
+  return cudaGetLastError();
+}
+
+}  // namespace dust

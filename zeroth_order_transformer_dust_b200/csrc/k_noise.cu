@@ -1,0 +1,66 @@
+// Debug kernels exposing the raw Philox stream and the Gaussian slots.
+#include "internal.cuh"
+#include "noise.cuh"
+
+namespace dust {
+
+__global__ void k_debug_philox(uint64_t seed, const uint32_t* __restrict__ ctr, int64_t n,
+                               uint32_t* __restrict__ out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const Key key = key_of(seed);
+  U4 c{ctr[4 * i], ctr[4 * i + 1], ctr[4 * i + 2], ctr[4 * i + 3]};
+  const U4 w = philox10(c, key.k0, key.k1);
+  out[4 * i] = w.x;
+  out[4 * i + 1] = w.y;
+  out[4 * i + 2] = w.z;
+  out[4 * i + 3] = w.w;
+}
+
+cudaError_t launch_debug_philox(cudaStream_t st, uint64_t seed, const uint32_t* ctr, int64_t n,
+                                uint32_t* out) {
+  if (n <= 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  k_debug_philox<<<(unsigned)blocks, threads, 0, st>>>(seed, ctr, n, out);
+  return cudaGetLastError();
+}
+
+// One thread per (token, draw, counter block of 128 slots, lane): one Philox
+// call gives slots lane, lane+32, lane+64, lane+96 of the block.
+__global__ void k_debug_gauss(Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3, int64_t nt,
+                              int64_t ni, int64_t nslots, float* __restrict__ out) {
+  const int64_t nblk = (nslots + 127) / 128;
+  const int64_t total = nt * ni * nblk * 32;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= total) return;
+  const uint32_t lane = (uint32_t)(gid & 31);
+  int64_t rest = gid >> 5;
+  const int64_t blk = rest % nblk;
+  rest /= nblk;
+  const int64_t i = rest % ni;
+  const int64_t t = rest / ni;
+  U4 c{slot_ctr0((uint32_t)blk, lane), t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3};
+  const G4 g = gauss4(philox10(c, key.k0, key.k1));
+  float* row = out + (t * ni + i) * nslots;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t k = blk * 128 + lane + 32 * j;
+    if (k < nslots) row[k] = g.v[j];
+  }
+}
+
+cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, int64_t nt,
+                               int64_t ni, int64_t nslots, float* out) {
+  const int64_t nblk = (nslots + 127) / 128;
+  const int64_t total = nt * ni * nblk * 32;
+  if (total <= 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (total + threads - 1) / threads;
+  k_debug_gauss<<<(unsigned)blocks, threads, 0, st>>>(
+      key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
+      ctr3_of(tag, p.stream_id), nt, ni, nslots, out);
+  return cudaGetLastError();
+}
+
+}  // namespace dust

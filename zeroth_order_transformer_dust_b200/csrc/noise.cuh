@@ -1,0 +1,190 @@
+// Counter-based Gaussian noise for the estimator, generated in registers.
+//
+// The Dust pages fix only that the noise is Gaussian and independent per
+// token and per draw ("Dust：无需反向传播的Transformer零阶预训练", §1,
+// 激活空间扰动). This build draws it from Philox4x32-10 (Salmon et al.,
+// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) and Box-Muller on
+// 24-bit uniforms; the slot -> (counter, word) layout puts the four words of
+// one counter on slots l, l+32, l+64, l+96 of a 128-slot block so that a warp
+// lane owns four coalesced columns per call.
+#pragma once
+#include <cstdint>
+
+namespace dust {
+
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
+constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
+constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
+
+constexpr int kTagHead = 0;
+constexpr int kTagSubsetOffset = 1;
+constexpr int kTagMlpUp = 2;
+
+struct U4 {
+  uint32_t x, y, z, w;
+};
+
+__host__ __device__ __forceinline__ uint32_t ctr3_of(int tag, uint32_t stream_id) {
+  return (uint32_t)(tag & 0xff) | (stream_id << 8);
+}
+
+// One Philox round: two 32x32->64 products, hi/lo halves recombined with XOR.
+__device__ __forceinline__ U4 philox_round(U4 c, uint32_t k0, uint32_t k1) {
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * c.x;
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * c.z;
+  U4 o;
+  o.x = (uint32_t)(p1 >> 32) ^ c.y ^ k0;
+  o.y = (uint32_t)p1;
+  o.z = (uint32_t)(p0 >> 32) ^ c.w ^ k1;
+  o.w = (uint32_t)p0;
+  return o;
+}
+
+// Philox4x32-10: ten rounds, key bumped between rounds.
+__device__ __forceinline__ U4 philox10(U4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    c = philox_round(c, k0, k1);
+    k0 += kPhiloxW0;
+    k1 += kPhiloxW1;
+  }
+  return c;
+}
+
+// -ln(u) for u in (0, 1], accurate to a few ulp relative to the result,
+// including u -> 1. u = 2^e m with m in [sqrt(1/2), sqrt(2)); ln m is
+// 2 atanh(s), s = (m-1)/(m+1), |s| <= 0.172, from its Taylor series
+// (2 s (1 + s^2/3 + s^4/5 + s^6/7 + s^8/9), truncation < 1e-9 relative);
+// e ln 2 uses ln 2 split in a high part with 8 trailing zero bits (exact
+// products for |e| <= 2^8) and a low correction (Cody and Waite's argument
+// reduction).
+__device__ __forceinline__ float neg_log_unit(float u) {
+  int bits = __float_as_int(u);
+  int e = ((bits >> 23) & 0xff) - 127;
+  float m = __int_as_float((bits & 0x007fffff) | 0x3f800000);
+  if (m > 1.41421356f) {
+    m *= 0.5f;
+    e += 1;
+  }
+  const float f = m - 1.0f;  // exact (Sterbenz)
+  const float s = __fdividef(f, m + 1.0f);
+  const float w = s * s;
+  float poly = fmaf(w, 2.0f / 9.0f, 2.0f / 7.0f);
+  poly = fmaf(w, poly, 2.0f / 5.0f);
+  poly = fmaf(w, poly, 2.0f / 3.0f);
+  poly = fmaf(w, poly, 2.0f);
+  const float ln_m = s * poly;
+  const float fe = (float)e;
+  const float kLn2Hi = 0.693145751953125f;        // 0x3f317200
+  const float kLn2Lo = 1.428606765330187e-06f;    // ln 2 - kLn2Hi
+  const float ln_u = fmaf(fe, kLn2Hi, fmaf(fe, kLn2Lo, ln_m));
+  return -ln_u;
+}
+
+// cos and sin of 2 pi m 2^-24 for an integer m in [0, 2^24). The nearest
+// quarter turn is removed exactly in integer arithmetic, leaving
+// |x| <= pi/4, where the Taylor series of sin (to x^9) and cos (to x^8) are
+// truncated below 3e-8.
+__device__ __forceinline__ void sincos_turn24(uint32_t m, float* s_out, float* c_out) {
+  const uint32_t q = (m + (1u << 21)) >> 22;          // 0..4
+  const int r = (int)m - (int)(q << 22);               // [-2^21, 2^21)
+  const float x = (float)r * 3.7450702e-07f;           // 2 pi / 2^24
+  const float x2 = x * x;
+  float sp = fmaf(x2, 2.7557319e-06f, -1.9841270e-04f);  // 1/9!, -1/7!
+  sp = fmaf(x2, sp, 8.3333333e-03f);                      // 1/5!
+  sp = fmaf(x2, sp, -1.6666667e-01f);                     // -1/3!
+  const float sn = fmaf(x * x2, sp, x);
+  float cp = fmaf(x2, 2.4801587e-05f, -1.3888889e-03f);  // 1/8!, -1/6!
+  cp = fmaf(x2, cp, 4.1666668e-02f);                      // 1/4!
+  cp = fmaf(x2, cp, -0.5f);
+  const float cs = fmaf(x2, cp, 1.0f);
+  const uint32_t qq = q & 3u;
+  float c = (qq & 1u) ? sn : cs;
+  float s = (qq & 1u) ? cs : sn;
+  c = (qq == 1u || qq == 2u) ? -c : c;
+  s = (qq >= 2u) ? -s : s;
+  *s_out = s;
+  *c_out = c;
+}
+
+// Box-Muller on 24-bit uniforms: u1 = ((wa>>8)+1) 2^-24, u2 = (wb>>8) 2^-24;
+// returns (R cos 2 pi u2, R sin 2 pi u2), R = sqrt(-2 ln u1).
+__device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb) {
+  const float u1 = (float)((wa >> 8) + 1u) * 5.9604645e-08f;  // exact
+  const float radius = sqrtf(2.0f * neg_log_unit(u1));
+  float s, c;
+  sincos_turn24(wb >> 8, &s, &c);
+  return make_float2(radius * c, radius * s);
+}
+
+// Four Gaussians of one counter: element j is output word j.
+struct G4 {
+  float v[4];
+};
+
+__device__ __forceinline__ G4 gauss4(U4 w) {
+  const float2 a = box_muller(w.x, w.y);
+  const float2 b = box_muller(w.z, w.w);
+  G4 g;
+  g.v[0] = a.x;
+  g.v[1] = a.y;
+  g.v[2] = b.x;
+  g.v[3] = b.y;
+  return g;
+}
+
+// Counter word 0 for slot block `blk` (128 slots) and lane `lane`.
+__host__ __device__ __forceinline__ uint32_t slot_ctr0(uint32_t blk, uint32_t lane) {
+  return (blk << 5) | lane;
+}
+
+// Key of a 64-bit seed.
+struct Key {
+  uint32_t k0, k1;
+};
+__host__ __device__ __forceinline__ Key key_of(uint64_t seed) {
+  return Key{(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
+}
+
+// eps of one slot (generic path; the hot kernels generate a whole counter).
+__device__ __forceinline__ float gauss_slot(Key key, uint32_t t_abs, uint32_t i_abs,
+                                            uint32_t ctr3, uint32_t k) {
+  U4 c{slot_ctr0(k >> 7, k & 31u), t_abs, i_abs, ctr3};
+  const U4 w = philox10(c, key.k0, key.k1);
+  const uint32_t word = (k >> 5) & 3u;
+  const uint32_t wa = (word < 2) ? w.x : w.z;
+  const uint32_t wb = (word < 2) ? w.y : w.w;
+  const float2 n = box_muller(wa, wb);
+  return (word & 1u) ? n.y : n.x;
+}
+
+// Subset offset b = floor(w0 V / 2^32) of (token, draw).
+__device__ __forceinline__ uint32_t subset_offset(Key key, uint32_t t_abs, uint32_t i_abs,
+                                                  uint32_t stream_id, uint32_t V) {
+  U4 c{0u, t_abs, i_abs, ctr3_of(kTagSubsetOffset, stream_id)};
+  const U4 w = philox10(c, key.k0, key.k1);
+  return (uint32_t)(((uint64_t)w.x * V) >> 32);
+}
+
+// expm1 for |x| <= 0.03 (degree 4) or 0.06 (degree 5) from its Taylor series,
+// relative truncation error below 7e-9 and 2e-9; larger arguments use expm1f.
+template <int DEG>
+__device__ __forceinline__ float expm1_small(float x) {
+  if constexpr (DEG == 4) {
+    float q = fmaf(x, 1.0f / 24.0f, 1.0f / 6.0f);
+    q = fmaf(x, q, 0.5f);
+    q = fmaf(x, q, 1.0f);
+    return x * q;
+  } else if constexpr (DEG == 5) {
+    float q = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
+    q = fmaf(x, q, 1.0f / 6.0f);
+    q = fmaf(x, q, 0.5f);
+    q = fmaf(x, q, 1.0f);
+    return x * q;
+  } else {
+    return expm1f(x);
+  }
+}
+
+}  // namespace dust
