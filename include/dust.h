@@ -169,6 +169,13 @@ int dust_stage_times(dust_ctx* ctx, const char** names, float* ms, int cap);
 /* Number of kernels the context has launched since it was created. */
 int64_t dust_kernel_launches(const dust_ctx* ctx);
 
+/* Debug: C (M x N, fp32, row-major) = A B^T for bf16 row-major A (M x K) and
+   B (N x K), through the library's GEMMs: path 0 = automatic, 1 = CUDA cores,
+   2 = tcgen05 tensor cores (DUST_ERR_UNSUPPORTED when the shape does not fit:
+   K a multiple of 8 and N >= 16 are needed). Synchronous. */
+dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
+                                 const void* B, float* C, int path);
+
 /* Debug: raw Philox4x32-10 words. ctr4 (n x 4 uint32, device) -> out (n x 4). */
 dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4,
                               int64_t n, uint32_t* out);

@@ -32,7 +32,7 @@ EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
            "dust_status_string", "dust_validate", "dust_subset_stride", "dust_check",
            "dust_head_grad", "dust_head_grad_host", "dust_mlp_grad", "dust_debug_philox",
            "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
-           "dust_kernel_launches")
+           "dust_kernel_launches", "dust_debug_gemm_bf16")
 
 
 class DustParams(ctypes.Structure):
@@ -85,6 +85,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "dust_stage_times": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_char_p),
                                                 ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
             "dust_kernel_launches": (I64, [P]),
+            "dust_debug_gemm_bf16": (I32, [P, I64, I64, I64, P, P, P, ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -279,6 +280,18 @@ class Context:
         return int(self._L.dust_kernel_launches(self._h))
 
     # -- debug exports -------------------------------------------------------------
+    def debug_gemm(self, A: torch.Tensor, B: torch.Tensor, path: int = 0) -> torch.Tensor:
+        """C = A B^T (bf16 operands, fp32 out); path 0 auto, 1 CUDA cores, 2 tensor cores."""
+        self._dev(A, "A"), self._dev(B, "B")
+        if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
+            raise TypeError("A and B must be bfloat16")
+        M, K = A.shape
+        N = B.shape[0]
+        C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+        self._bind_stream()
+        self._check(self._L.dust_debug_gemm_bf16(self._h, M, N, K, _ptr(A), _ptr(B), _ptr(C), path))
+        return C
+
     def debug_philox(self, seed: int, ctr: torch.Tensor) -> torch.Tensor:
         """Raw Philox4x32-10 words for counters ctr (n x 4, int32 storage of uint32)."""
         self._dev(ctr, "ctr")

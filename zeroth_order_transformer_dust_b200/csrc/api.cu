@@ -132,10 +132,13 @@ dust_status finish(dust_ctx* ctx, uint32_t flags) {
   return dust_check(ctx);
 }
 
-dust_status run_gemm(dust_ctx* ctx, const GemmDesc& g, const EpiDesc& e) {
+// path: 0 automatic, 1 CUDA cores, 2 tensor cores.
+dust_status run_gemm(dust_ctx* ctx, const GemmDesc& g, const EpiDesc& e, int path = 0) {
+  const bool tc = path != 1 && (path == 2 || ctx->tc_enabled) && tc_gemm_supported(g, e);
+  if (path == 2 && !tc) return fail(ctx, DUST_ERR_UNSUPPORTED, "shape not taken by the tensor-core GEMM");
   ctx->launches += 1;
-  if (tc_gemm_supported(g, e)) {
-    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count));
+  if (tc) {
+    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count, ctx->d_status));
   } else {
     DUST_CU(launch_gemm_simt(ctx->stream, g, e));
   }
@@ -143,6 +146,51 @@ dust_status run_gemm(dust_ctx* ctx, const GemmDesc& g, const EpiDesc& e) {
 }
 
 size_t elem_size(int dtype) { return dtype == DUST_BF16 ? 2 : 4; }
+
+// Bytes of the g GEMM operand: fp32, or bf16 hi and lo planes.
+size_t gop_bytes(int dtype, int64_t T, int64_t width) {
+  return dtype == DUST_BF16 ? (size_t)2 * T * width * 2 : (size_t)T * width * 4;
+}
+
+// out (width x N, fp32) = sum_t g_t x_t^T, row w written at (w * row_mul) mod width
+// when row_mul != 0. gop holds g (T x width) as fp32 or as bf16 hi/lo planes;
+// X is T x N in p.dtype. The bf16 path contracts over 2T (both planes against
+// a duplicated X), on tensor cores after transposing both operands to K-major.
+dust_status weight_grad(dust_ctx* ctx, const dust_params& p, const void* gop, int64_t width,
+                        const void* X, int64_t N, float* out, int64_t row_mul) {
+  const int64_t T = p.T;
+  EpiDesc e{};
+  e.kind = kEpiF32; e.C = out; e.ldc = N; e.c_row_mul = row_mul;
+  if (p.dtype != DUST_BF16) {
+    GemmDesc g{};
+    g.M = width; g.N = N; g.K = T; g.A = gop; g.lda = width; g.a_kmajor = false;
+    g.B = X; g.ldb = N; g.b_kmajor = false; g.dtype = DUST_F32;
+    return run_gemm(ctx, g, e);
+  }
+  const int64_t K2 = 2 * T;
+  const size_t xb = (size_t)T * N * 2;
+  DUST_TRY(ensure(ctx, ctx->xdup, 2 * xb));
+  DUST_CU(cudaMemcpyAsync(ctx->xdup.p, X, xb, cudaMemcpyDeviceToDevice, ctx->stream));
+  DUST_CU(cudaMemcpyAsync((char*)ctx->xdup.p + xb, X, xb, cudaMemcpyDeviceToDevice, ctx->stream));
+  const int64_t ld = (K2 + 7) / 8 * 8;
+  DUST_TRY(ensure(ctx, ctx->gT, (size_t)width * ld * 2));
+  DUST_TRY(ensure(ctx, ctx->hT, (size_t)N * ld * 2));
+  GemmDesc g{};
+  g.M = width; g.N = N; g.K = K2; g.A = ctx->gT.p; g.lda = ld; g.a_kmajor = true;
+  g.B = ctx->hT.p; g.ldb = ld; g.b_kmajor = true; g.dtype = DUST_BF16;
+  if (ctx->tc_enabled && tc_gemm_supported(g, e)) {
+    DUST_CU(launch_transpose_bf16(ctx->stream, (const __nv_bfloat16*)gop, K2, width,
+                                  (__nv_bfloat16*)ctx->gT.p, ld));
+    DUST_CU(launch_transpose_bf16(ctx->stream, (const __nv_bfloat16*)ctx->xdup.p, K2, N,
+                                  (__nv_bfloat16*)ctx->hT.p, ld));
+    ctx->launches += 2;
+    return run_gemm(ctx, g, e);
+  }
+  GemmDesc s{};
+  s.M = width; s.N = N; s.K = K2; s.A = gop; s.lda = width; s.a_kmajor = false;
+  s.B = ctx->xdup.p; s.ldb = N; s.b_kmajor = false; s.dtype = DUST_BF16;
+  return run_gemm(ctx, s, e);
+}
 
 // Stage marks: mark(ctx, nullptr) opens a call, mark(ctx, "name") closes the
 // stage that ran since the previous mark.
@@ -192,6 +240,8 @@ dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
   dust_ctx* ctx = new dust_ctx();
   ctx->device = device;
   ctx->stream = (cudaStream_t)cuda_stream;
+  const char* no_tc = getenv("DUST_DISABLE_TC");
+  ctx->tc_enabled = !(no_tc && no_tc[0] && no_tc[0] != '0');
   if (cudaSetDevice(device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess ||
@@ -217,7 +267,7 @@ void dust_destroy(dust_ctx* ctx) {
   cudaSetDevice(ctx->device);
   if (ctx->stream) cudaStreamSynchronize(ctx->stream);
   Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
-                 &ctx->gT, &ctx->hT, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
+                 &ctx->gT, &ctx->hT, &ctx->xdup, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv};
   for (Buf* b : bufs)
@@ -265,7 +315,7 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   const size_t TV = (size_t)p.T * (size_t)p.V;
   DUST_TRY(ensure(ctx, ctx->z, TV * 4));
   DUST_TRY(ensure(ctx, ctx->lse, (size_t)p.T * 4));
-  DUST_TRY(ensure(ctx, ctx->gop, TV * elem_size(p.dtype)));
+  DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(p.dtype, p.T, p.V)));
   float* loss = loss_out;
   if (!loss) {
     DUST_TRY(ensure(ctx, ctx->loss, (size_t)p.T * 4));
@@ -276,12 +326,24 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), st));
   mark(ctx, nullptr);
 
-  // 1. clean logits z = H W^T (permuted columns for subset draws)
+  // 1. clean logits z = H W^T (permuted columns for subset draws: the bf16
+  //    path gathers the rows of W once so the tensor-core GEMM reads them
+  //    contiguously; the CUDA-core path gathers on the fly)
+  const void* Wuse = W;
+  int64_t bmul = subset ? a : 0;
+  if (subset && p.dtype == DUST_BF16) {
+    DUST_TRY(ensure(ctx, ctx->wperm, (size_t)p.V * p.d * 2));
+    DUST_CU(launch_permute_rows_bf16(st, (const __nv_bfloat16*)W, p.V, p.d, a,
+                                     (__nv_bfloat16*)ctx->wperm.p));
+    ctx->launches += 1;
+    Wuse = ctx->wperm.p;
+    bmul = 0;
+  }
   GemmDesc g{};
   g.M = p.T; g.N = p.V; g.K = p.d;
   g.A = H; g.lda = p.d; g.a_kmajor = true;
-  g.B = W; g.ldb = p.d; g.b_kmajor = true;
-  g.b_row_mul = subset ? a : 0;
+  g.B = Wuse; g.ldb = p.d; g.b_kmajor = true;
+  g.b_row_mul = bmul;
   g.dtype = p.dtype;
   EpiDesc e{};
   e.kind = kEpiF32; e.C = Z; e.ldc = p.V;
@@ -321,14 +383,7 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   }
   // 4. G_W = sum_t g_t h_t^T (rows un-permuted on the store)
   if (G_out) {
-    GemmDesc w{};
-    w.M = p.V; w.N = p.d; w.K = p.T;
-    w.A = ctx->gop.p; w.lda = p.V; w.a_kmajor = false;
-    w.B = H; w.ldb = p.d; w.b_kmajor = false;
-    w.dtype = p.dtype;
-    EpiDesc we{};
-    we.kind = kEpiF32; we.C = G_out; we.ldc = p.d; we.c_row_mul = subset ? a : 0;
-    DUST_TRY(run_gemm(ctx, w, we));
+    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, p.V, H, p.d, G_out, subset ? a : 0));
     mark(ctx, "gw_gemm");
   }
   return finish(ctx, p.flags);
@@ -397,7 +452,7 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   DUST_TRY(ensure(ctx, ctx->mlp_h, (size_t)T * d * 2));
   DUST_TRY(ensure(ctx, ctx->z, (size_t)T * V * 4));
   DUST_TRY(ensure(ctx, ctx->lse, (size_t)T * 4));
-  DUST_TRY(ensure(ctx, ctx->gop, (size_t)T * dff * 2));
+  DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(DUST_BF16, T, dff)));
   float* loss = loss_out;
   if (!loss) {
     DUST_TRY(ensure(ctx, ctx->loss, (size_t)T * 4));
@@ -487,12 +542,7 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   ctx->launches += 1;
   mark(ctx, "g");
   if (G_up_out) {
-    GemmDesc w{};
-    w.M = dff; w.N = d; w.K = T; w.A = ctx->gop.p; w.lda = dff; w.a_kmajor = false;
-    w.B = X; w.ldb = d; w.b_kmajor = false; w.dtype = DUST_BF16;
-    EpiDesc we{};
-    we.kind = kEpiF32; we.C = G_up_out; we.ldc = d;
-    DUST_TRY(run_gemm(ctx, w, we));
+    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, dff, X, d, G_up_out, 0));
     mark(ctx, "gw_gemm");
   }
   return finish(ctx, p.flags);
@@ -527,6 +577,22 @@ int dust_stage_times(dust_ctx* ctx, const char** names, float* ms, int cap) {
 }
 
 int64_t dust_kernel_launches(const dust_ctx* ctx) { return ctx ? ctx->launches : 0; }
+
+dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
+                                 const void* B, float* C, int path) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || path < 0 || path > 2)
+    return fail(ctx, DUST_ERR_ARG, "bad gemm arguments");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), ctx->stream));
+  GemmDesc g{};
+  g.M = M; g.N = N; g.K = K; g.A = A; g.lda = K; g.a_kmajor = true;
+  g.B = B; g.ldb = K; g.b_kmajor = true; g.dtype = DUST_BF16;
+  EpiDesc e{};
+  e.kind = kEpiF32; e.C = C; e.ldc = N;
+  DUST_TRY(run_gemm(ctx, g, e, path));
+  return dust_check(ctx);
+}
 
 dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4, int64_t n,
                               uint32_t* out) {

@@ -51,6 +51,20 @@ struct EpiDesc {
   int64_t ldr = 0;
 };
 
+// The bf16 GEMM operand of g is stored as two planes, hi = bf16(v) and
+// lo = bf16(v - hi), `plane` elements apart, so sum_t g_t h_t^T computed over
+// both planes carries about 2^-17 relative error from the operand instead of
+// the 2^-9 of a single bf16 rounding.
+__device__ __forceinline__ void store_g_operand(__nv_bfloat16* gop, int64_t plane, int64_t o,
+                                                float v) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  gop[o] = hi;
+  gop[plane + o] = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+__device__ __forceinline__ void store_g_operand(float* gop, int64_t, int64_t o, float v) {
+  gop[o] = v;
+}
+
 }  // namespace dust
 
 struct dust_ctx {
@@ -68,9 +82,11 @@ struct dust_ctx {
   const char* mark_name[kMaxMarks] = {};
   int nmarks = 0;
   int64_t launches = 0;
+  // tensor-core GEMMs on (DUST_DISABLE_TC=1 at creation routes all GEMMs to CUDA cores)
+  bool tc_enabled = true;
   // scratch, grown on demand
-  dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, dzy, mlp_u, mlp_a, mlp_h, mlp_da, mlp_dh,
-      in_h, in_w, in_y, out_g, out_loss, out_r, out_gv;
+  dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
+      mlp_dh, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv;
 };
 
 namespace dust {
@@ -112,9 +128,19 @@ cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a,
                                const float* P, const int32_t* y, float* rewards, float* g_out,
                                void* gop, float* gacc, int max_smem_optin);
 
-// Tensor-core GEMM (tcgen05): shapes it takes, and its launcher.
+// Tensor-core GEMM (tcgen05): shapes it takes, and its launcher. A bounded
+// wait that expires sets kStatusTimeout in *status.
 bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e);
-cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count);
+cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
+                           uint32_t* status);
+
+// Transpose of a row-major bf16 matrix (rows x cols) into dst (cols x rows,
+// row stride ld_dst >= rows; columns [rows, ld_dst) of dst are zeroed).
+cudaError_t launch_transpose_bf16(cudaStream_t st, const __nv_bfloat16* src, int64_t rows,
+                                  int64_t cols, __nv_bfloat16* dst, int64_t ld_dst);
+// dst row q = src row (q * mul) mod rows (rows x cols bf16).
+cudaError_t launch_permute_rows_bf16(cudaStream_t st, const __nv_bfloat16* src, int64_t rows,
+                                     int64_t cols, int64_t mul, __nv_bfloat16* dst);
 
 // MLP helpers.
 cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const float* u,

@@ -85,20 +85,11 @@ __global__ void k_full_reward_combine(Key key, uint32_t t_off, uint32_t i_off, u
 }
 
 template <typename TO>
-__device__ __forceinline__ void store_op(TO* p, int64_t o, float v);
-template <>
-__device__ __forceinline__ void store_op<float>(float* p, int64_t o, float v) { p[o] = v; }
-template <>
-__device__ __forceinline__ void store_op<__nv_bfloat16>(__nv_bfloat16* p, int64_t o, float v) {
-  p[o] = __float2bfloat16_rn(v);
-}
-
-template <typename TO>
 __global__ __launch_bounds__(kWarps * 32) void k_full_g(Key key, uint32_t t_off, uint32_t i_off,
                                                         uint32_t ctr3, float scale, int64_t V,
                                                         int32_t K, const float* __restrict__ r,
                                                         float* __restrict__ g_out,
-                                                        TO* __restrict__ gop) {
+                                                        TO* __restrict__ gop, int64_t plane) {
   __shared__ float rs[1024];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = blockIdx.x;
@@ -136,7 +127,7 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(Key key, uint32_t t_off,
       if (pos < V) {
         const float v = acc[b][j] * scale;
         if (g_out) g_out[t * V + pos] = v;
-        store_op<TO>(gop, t * V + pos, v);
+        store_g_operand(gop, plane, t * V + pos, v);
       }
     }
 }
@@ -190,12 +181,13 @@ cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r,
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
   const Key key = key_of(p.seed);
   const uint32_t c3 = ctr3_of(kTagHead, p.stream_id);
+  const int64_t plane = p.T * p.V;
   if (p.dtype == DUST_BF16)
     k_full_g<__nv_bfloat16><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.V, p.K, r, g_out, (__nv_bfloat16*)gop);
+        (uint32_t)p.draw_offset, c3, scale, p.V, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
   else
     k_full_g<float><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.V, p.K, r, g_out, (float*)gop);
+        (uint32_t)p.draw_offset, c3, scale, p.V, p.K, r, g_out, (float*)gop, plane);
   return cudaGetLastError();
 }
 

@@ -1,13 +1,341 @@
-// Tensor-core (tcgen05) GEMM: placeholder until the sm_100a kernel lands;
-// every GEMM currently takes the CUDA-core path.
+// Tensor-core GEMM for sm_100a: C = A B^T with bf16 operands and fp32
+// accumulation, A (M x K) and B (N x K) both K-major.
+//
+// Persistent, warp-specialised CTA (one per SM): warp 0 issues TMA tile loads
+// into a 4-stage shared-memory ring, warp 1 issues tcgen05.mma (128 x 256 x 16)
+// into one of two TMEM accumulators, warps 2-5 drain the other accumulator
+// with tcgen05.ld and run the epilogue, so the epilogue of tile i overlaps
+// the MMAs of tile i+1. Every mbarrier wait is bounded in time: on expiry the
+// CTA raises the timeout bit of the device status word, drains its own
+// copies and MMAs (bounded again), frees its TMEM and returns.
+#include <cudaTypedefs.h>
+
 #include "internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace dust {
+namespace {
 
-bool tc_gemm_supported(const GemmDesc&, const EpiDesc&) { return false; }
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int THREADS = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
 
-cudaError_t launch_gemm_tc(cudaStream_t, const GemmDesc&, const EpiDesc&, int) {
-  return cudaErrorNotSupported;
+struct TcParams {
+  int64_t M, N, K;
+  int m_tiles, n_tiles, num_kb;
+  EpiDesc e;
+  uint32_t* status;
+};
+
+struct Shared {
+  uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float gelu_erf(float x) {
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+// Epilogue of 32 consecutive columns [n, n+32) of row m (output row mo).
+template <int KIND>
+__device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t mo, int64_t n,
+                                           const float* v) {
+  const EpiDesc& e = p.e;
+  const bool full = n + 32 <= p.N;
+  if (KIND == kEpiF32 || KIND == kEpiGelu) {
+    float* dst = e.C + mo * e.ldc + n;
+    if (full && ((e.ldc & 3) == 0) && (((uintptr_t)e.C & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+      for (int q = 0; q < 32; ++q)
+        if (n + q < p.N) dst[q] = v[q];
+    }
+  }
+  if (KIND == kEpiBF16 || KIND == kEpiGelu || KIND == kEpiResidBF16) {
+    float w[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) w[q] = v[q];
+    if (KIND == kEpiGelu) {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) w[q] = gelu_erf(w[q]);
+    }
+    if (KIND == kEpiResidBF16) {
+      const __nv_bfloat16* r = (const __nv_bfloat16*)e.resid + m * e.ldr + n;
+      for (int q = 0; q < 32; ++q)
+        if (n + q < p.N) w[q] += __bfloat162float(r[q]);
+    }
+    __nv_bfloat16* dst = e.Cb + mo * e.ldc + n;
+    if (full && ((e.ldc & 7) == 0) && (((uintptr_t)e.Cb & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(w[8 * q + 0], w[8 * q + 1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(w[8 * q + 2], w[8 * q + 3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(w[8 * q + 4], w[8 * q + 5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(w[8 * q + 6], w[8 * q + 7]);
+        uint4 u;
+        u.x = *reinterpret_cast<uint32_t*>(&h0);
+        u.y = *reinterpret_cast<uint32_t*>(&h1);
+        u.z = *reinterpret_cast<uint32_t*>(&h2);
+        u.w = *reinterpret_cast<uint32_t*>(&h3);
+        reinterpret_cast<uint4*>(dst)[q] = u;
+      }
+    } else {
+      for (int q = 0; q < 32; ++q)
+        if (n + q < p.N) dst[q] = __float2bfloat16_rn(w[q]);
+    }
+  }
+}
+
+template <int KIND>
+__global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ CUtensorMap tmA,
+                                                        const __grid_constant__ CUtensorMap tmB,
+                                                        TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* basep = smem_raw + (base - raw);
+  const uint32_t sA = base;                           // STAGES x A tile
+  const uint32_t sB = base + STAGES * A_BYTES;        // STAGES x B tile
+  Shared* sh = reinterpret_cast<Shared*>(basep + STAGES * STAGE_BYTES);
+  volatile int* abort = &sh->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = p.m_tiles * p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&sh->full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&sh->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(ptx::smem_u32(&sh->tfull[a]), 1);
+      ptx::mbar_init(ptx::smem_u32(&sh->tempty[a]), 4);
+    }
+    ptx::mbar_init(ptx::smem_u32(&sh->drain), 1);
+    sh->abort = 0;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async();
+    ptx::prefetch_map(&tmA);
+    ptx::prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool armed[STAGES] = {};
+      uint32_t armed_parity[STAGES] = {};
+      for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+        const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bounded(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort, p.status)) break;
+          const uint32_t fb = ptx::smem_u32(&sh->full[stage]);
+          ptx::mbar_expect_tx(fb, STAGE_BYTES);
+          ptx::tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, m_blk * BM, fb);
+          ptx::tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, n_blk * BN, fb);
+          armed[stage] = true;
+          armed_parity[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // every copy this thread issued has landed before the CTA can exit
+      int dummy = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (armed[s])
+          wait_bounded(ptx::smem_u32(&sh->full[s]), armed_parity[s], &dummy, p.status);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+        if (!wait_bounded(ptx::smem_u32(&sh->tempty[acc]), acc_phase ^ 1u, abort, p.status)) break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bounded(ptx::smem_u32(&sh->full[stage]), phase, abort, p.status)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = sA + stage * A_BYTES, b0 = sB + stage * B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            ptx::mma_f16(d_tmem, ptx::sdesc_kmajor_sw128(a0 + k * 32),
+                         ptx::sdesc_kmajor_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+          }
+          issued = true;
+          ptx::mma_commit(ptx::smem_u32(&sh->empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_u32(&sh->tfull[acc]));
+      }
+      if (issued) {
+        // all MMAs of this CTA complete before TMEM is released
+        ptx::mma_commit(ptx::smem_u32(&sh->drain));
+        int dummy = 0;
+        wait_bounded(ptx::smem_u32(&sh->drain), 0, &dummy, p.status);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 ----------------
+    const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
+    const int row = quad * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      if (!wait_bounded(ptx::smem_u32(&sh->tfull[acc]), acc_phase, abort, p.status)) break;
+      ptx::tc_fence_after();
+      const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+      const int64_t m = (int64_t)m_blk * BM + row;
+      int64_t mo = m;
+      if (p.e.c_row_mul != 0 && m < p.M)
+        mo = (int64_t)(((unsigned long long)m * (unsigned long long)p.e.c_row_mul) %
+                       (unsigned long long)p.M);
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int64_t n = (int64_t)n_blk * BN + c * 32;
+        float v[32];
+        ptx::tmem_ld32(taddr + (uint32_t)(c * 32), v);
+        if (m < p.M && n < p.N) epilogue32<KIND>(p, m, mo, n, v);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sh->tempty[acc]));
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, TMEM_COLS);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix (rows x cols, row stride ld elements) as a TMA map with
+// a box of 64 columns x box_rows rows and 128-byte swizzling.
+bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
+              int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND>
+cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
+                        const TcParams& p, int sm_count) {
+  auto fn = k_gemm_tc<KIND>;
+  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < sm_count ? tiles : sm_count;
+  fn<<<grid, THREADS, SMEM_BYTES, st>>>(a, b, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
+  if (g.dtype != DUST_BF16 || !g.a_kmajor || !g.b_kmajor || g.b_row_mul != 0) return false;
+  if (g.M < 1 || g.N < 16 || g.K < 16) return false;
+  if ((g.lda & 7) || (g.ldb & 7)) return false;
+  if (((uintptr_t)g.A & 15) || ((uintptr_t)g.B & 15)) return false;
+  if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX) return false;
+  if (e.kind == kEpiResidBF16 && !e.resid) return false;
+  if (!encode_fn()) return false;
+  return e.kind == kEpiF32 || e.kind == kEpiBF16 || e.kind == kEpiGelu || e.kind == kEpiResidBF16;
+}
+
+cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
+                           uint32_t* status) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, g.A, g.M, g.K, g.lda, BM) || !make_map(&mb, g.B, g.N, g.K, g.ldb, BN))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.m_tiles = (int)((g.M + BM - 1) / BM);
+  p.n_tiles = (int)((g.N + BN - 1) / BN);
+  p.num_kb = (int)((g.K + BK - 1) / BK);
+  p.e = e;
+  p.status = status;
+  if (!p.status) return cudaErrorInvalidValue;
+  switch (e.kind) {
+    case kEpiF32: return launch_kind<kEpiF32>(st, ma, mb, p, sm_count);
+    case kEpiBF16: return launch_kind<kEpiBF16>(st, ma, mb, p, sm_count);
+    case kEpiGelu: return launch_kind<kEpiGelu>(st, ma, mb, p, sm_count);
+    case kEpiResidBF16: return launch_kind<kEpiResidBF16>(st, ma, mb, p, sm_count);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace dust

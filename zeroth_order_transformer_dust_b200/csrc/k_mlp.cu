@@ -130,21 +130,13 @@ __global__ void k_reward_combine_rows(const float* __restrict__ part, int nparts
   r[row0 + m] = dzy[m] - log1pf(s);
 }
 
-template <typename TO>
-__device__ __forceinline__ void store_op(TO* p, int64_t o, float v);
-template <>
-__device__ __forceinline__ void store_op<float>(float* p, int64_t o, float v) { p[o] = v; }
-template <>
-__device__ __forceinline__ void store_op<__nv_bfloat16>(__nv_bfloat16* p, int64_t o, float v) {
-  p[o] = __float2bfloat16_rn(v);
-}
-
 // g_t[c] = scale * sum_i r[t*K + i] eps(t, i, c): one warp per 128 channels.
 template <typename TO>
 __global__ __launch_bounds__(256) void k_noise_g(Key key, uint32_t t_off, uint32_t i_off,
                                                  uint32_t ctr3, float scale, int64_t width,
                                                  int32_t K, const float* __restrict__ r,
-                                                 float* __restrict__ g_out, TO* __restrict__ gop) {
+                                                 float* __restrict__ g_out, TO* __restrict__ gop,
+                                                 int64_t plane) {
   __shared__ float rs[1024];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = blockIdx.x;
@@ -171,7 +163,7 @@ __global__ __launch_bounds__(256) void k_noise_g(Key key, uint32_t t_off, uint32
     if (ch < width) {
       const float v = acc[j] * scale;
       if (g_out) g_out[t * width + ch] = v;
-      store_op<TO>(gop, t * width + ch, v);
+      store_g_operand(gop, plane, t * width + ch, v);
     }
   }
 }
@@ -219,12 +211,13 @@ cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, 
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
   const Key key = key_of(p.seed);
   const uint32_t c3 = ctr3_of(kTagMlpUp, p.stream_id);
+  const int64_t plane = p.T * p.d_ff;
   if (p.dtype == DUST_BF16)
     k_noise_g<__nv_bfloat16><<<grid, 256, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (__nv_bfloat16*)gop);
+        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
   else
     k_noise_g<float><<<grid, 256, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (float*)gop);
+        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (float*)gop, plane);
   return cudaGetLastError();
 }
 

@@ -36,6 +36,7 @@ struct SubsetArgs {
   void* gop;
   float* gacc;  // global accumulator rows (only when the row does not fit in smem)
   int gop_bf16;
+  int64_t plane;  // distance between the hi and lo planes of the bf16 operand
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -166,7 +167,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset(SubsetArgs A) {
   for (int64_t q = threadIdx.x; q < V; q += kThreads) {
     const float v = G[q] * ((uint32_t)q == qy ? A.scale_target : A.scale_other) * A.fac;
     if (A.gop_bf16)
-      ((__nv_bfloat16*)A.gop)[t * V + q] = __float2bfloat16_rn(v);
+      store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * V + q, v);
     else
       ((float*)A.gop)[t * V + q] = v;
     if (A.g_out) A.g_out[t * V + mulmod((uint32_t)q, (uint64_t)A.a, V)] = v;
@@ -235,6 +236,7 @@ cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a,
   A.gop = gop;
   A.gacc = gacc;
   A.gop_bf16 = p.dtype == DUST_BF16;
+  A.plane = p.T * p.V;
   const int deg = expm1_degree(p.sigma);
   const size_t smem = (size_t)p.V * 4;
   if (smem <= (size_t)max_smem_optin) return launch_g<true>(st, A, p.T, smem, deg);
