@@ -17,10 +17,11 @@ down-projection and the head from the cached x, u and clean logits:
 
 Readings: GELU is the exact erf form (the only GELU the pages show is
 PyTorch's default ``nn.GELU()`` in the listing of "Dust：无需反向传播的
-Transformer 预训练方法"); there is no LayerNorm and no bias. The GEMM operands
-that the bf16 workload rounds to bf16 (a, h, da, dh) are rounded here at the
-same points (``mirror_bf16``) so that comparisons measure implementation
-error, not the configured quantisation.
+Transformer 预训练方法"); there is no LayerNorm and no bias. Precision (the
+pages state none): the clean activations a = GELU(u) and h are carried at full
+precision; the per-draw deltas da and dh are GEMM operands in bf16, rounded
+once each (round to nearest even). ``mirror_bf16`` applies those two roundings
+here so that comparisons measure implementation error, not the quantisation.
 """
 from __future__ import annotations
 
@@ -47,12 +48,12 @@ def bf16_rne(x: np.ndarray) -> np.ndarray:
 
 
 def clean_mlp(X, W_up, W_down, W_head, targets, mirror_bf16: bool = True) -> dict:
+    """Clean pass (no rounding: ``mirror_bf16`` concerns the per-draw deltas only)."""
     X = np.asarray(X, dtype=np.float64)
-    rnd = bf16_rne if mirror_bf16 else (lambda v: v)
     u = X @ np.asarray(W_up, dtype=np.float64).T
-    a = rnd(gelu(u))
+    a = gelu(u)
     h = X + a @ np.asarray(W_down, dtype=np.float64).T
-    hb = rnd(h)
+    hb = h
     z = hb @ np.asarray(W_head, dtype=np.float64).T
     zmax = z.max(axis=1)
     lse = zmax + np.log(np.exp(z - zmax[:, None]).sum(axis=1))

@@ -242,6 +242,8 @@ dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
   ctx->stream = (cudaStream_t)cuda_stream;
   const char* no_tc = getenv("DUST_DISABLE_TC");
   ctx->tc_enabled = !(no_tc && no_tc[0] && no_tc[0] != '0');
+  const char* sk = getenv("DUST_SUBSET_KERNEL");
+  ctx->subset2_enabled = !(sk && sk[0] == '1');
   if (cudaSetDevice(device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess ||
@@ -268,7 +270,7 @@ void dust_destroy(dust_ctx* ctx) {
   if (ctx->stream) cudaStreamSynchronize(ctx->stream);
   Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
                  &ctx->gT, &ctx->hT, &ctx->xdup, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
-                 &ctx->mlp_da, &ctx->mlp_dh, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
+                 &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
@@ -349,9 +351,12 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   e.kind = kEpiF32; e.C = Z; e.ldc = p.V;
   DUST_TRY(run_gemm(ctx, g, e));
   mark(ctx, "clean_gemm");
-  // 2. log-sum-exp, clean loss, softmax in place
+  // 2. log-sum-exp, clean loss, softmax in place (the shared-memory subset
+  //    kernel forms p itself while it loads a row)
+  const bool smem_subset =
+      subset && ctx->subset2_enabled && subset2_cluster_size(p.V, p.S, ctx->max_smem_optin) > 0;
   DUST_CU(launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, (float*)ctx->lse.p, loss,
-                          true, ctx->d_status));
+                          !smem_subset, ctx->d_status));
   ctx->launches += 1;
   mark(ctx, "lse");
   // 3. perturbed losses, rewards, g
@@ -369,6 +374,11 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
     DUST_CU(launch_full_g(st, p, r, g_out, ctx->gop.p));
     ctx->launches += 1;
     mark(ctx, "g");
+  } else if (smem_subset) {
+    DUST_CU(launch_subset2(st, p, a, a_inv, Z, (const float*)ctx->lse.p, targets, rewards_out,
+                           g_out, ctx->gop.p, ctx->max_smem_optin, ctx->sm_count));
+    ctx->launches += 1;
+    mark(ctx, "subset_draws");
   } else {
     float* gacc = nullptr;
     const size_t gb = subset_gacc_bytes(p.T, p.V, ctx->max_smem_optin);
@@ -448,8 +458,8 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   const cudaStream_t st = ctx->stream;
   const int64_t T = p.T, d = p.d, dff = p.d_ff, V = p.V, K = p.K;
   DUST_TRY(ensure(ctx, ctx->mlp_u, (size_t)T * dff * 4));
-  DUST_TRY(ensure(ctx, ctx->mlp_a, (size_t)T * dff * 2));
-  DUST_TRY(ensure(ctx, ctx->mlp_h, (size_t)T * d * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_a, (size_t)T * 2 * dff * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_h, (size_t)T * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->z, (size_t)T * V * 4));
   DUST_TRY(ensure(ctx, ctx->lse, (size_t)T * 4));
   DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(DUST_BF16, T, dff)));
@@ -470,27 +480,39 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), st));
   mark(ctx, nullptr);
 
-  // clean pass: u = x W_up^T (fp32), a = bf16(GELU(u)), h = bf16(x + a W_down^T), z = h W_head^T
+  // clean pass, activations at full precision as bf16 hi/lo planes:
+  //   u = x W_up^T (fp32); a = GELU(u) (fp64) -> [a_hi | a_lo] (T x 2 d_ff);
+  //   h = x + a W_down^T -> [h_hi | h_lo] (T x 2d); z = h W_head^T.
+  // The planes are contracted against weights duplicated along K.
+  DUST_TRY(ensure(ctx, ctx->wd2, (size_t)d * 2 * dff * 2));
+  DUST_TRY(ensure(ctx, ctx->wh2, (size_t)V * 2 * d * 2));
+  for (int half = 0; half < 2; ++half) {
+    DUST_CU(cudaMemcpy2DAsync((char*)ctx->wd2.p + (size_t)half * dff * 2, (size_t)2 * dff * 2,
+                              W_down, (size_t)dff * 2, (size_t)dff * 2, (size_t)d,
+                              cudaMemcpyDeviceToDevice, st));
+    DUST_CU(cudaMemcpy2DAsync((char*)ctx->wh2.p + (size_t)half * d * 2, (size_t)2 * d * 2, W_head,
+                              (size_t)d * 2, (size_t)d * 2, (size_t)V, cudaMemcpyDeviceToDevice, st));
+  }
   {
     GemmDesc g{};
     g.M = T; g.N = dff; g.K = d; g.A = X; g.lda = d; g.a_kmajor = true;
     g.B = W_up; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
     EpiDesc e{};
-    e.kind = kEpiGelu; e.C = u; e.Cb = abf; e.ldc = dff;
+    e.kind = kEpiGeluSplit; e.C = u; e.ldc = dff; e.Cb = abf; e.ldcb = 2 * dff; e.split = dff;
     DUST_TRY(run_gemm(ctx, g, e));
   }
   {
     GemmDesc g{};
-    g.M = T; g.N = d; g.K = dff; g.A = abf; g.lda = dff; g.a_kmajor = true;
-    g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+    g.M = T; g.N = d; g.K = 2 * dff; g.A = abf; g.lda = 2 * dff; g.a_kmajor = true;
+    g.B = ctx->wd2.p; g.ldb = 2 * dff; g.b_kmajor = true; g.dtype = DUST_BF16;
     EpiDesc e{};
-    e.kind = kEpiResidBF16; e.Cb = hbf; e.ldc = d; e.resid = X; e.ldr = d;
+    e.kind = kEpiResidSplit; e.Cb = hbf; e.ldcb = 2 * d; e.split = d; e.resid = X; e.ldr = d;
     DUST_TRY(run_gemm(ctx, g, e));
   }
   {
     GemmDesc g{};
-    g.M = T; g.N = V; g.K = d; g.A = hbf; g.lda = d; g.a_kmajor = true;
-    g.B = W_head; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
+    g.M = T; g.N = V; g.K = 2 * d; g.A = hbf; g.lda = 2 * d; g.a_kmajor = true;
+    g.B = ctx->wh2.p; g.ldb = 2 * d; g.b_kmajor = true; g.dtype = DUST_BF16;
     EpiDesc e{};
     e.kind = kEpiF32; e.C = Z; e.ldc = V;
     DUST_TRY(run_gemm(ctx, g, e));
@@ -523,7 +545,7 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
       g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = dff; g.a_kmajor = true;
       g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
-      e.kind = kEpiBF16; e.Cb = dh; e.ldc = d;
+      e.kind = kEpiBF16; e.Cb = dh; e.ldcb = d;
       DUST_TRY(run_gemm(ctx, g, e));
     }
     {

@@ -35,21 +35,46 @@ struct GemmDesc {
 };
 
 enum EpiKind {
-  kEpiF32 = 0,        // C[m*ldc + n] = acc   (row m written at (m*c_row_mul) mod M if set)
-  kEpiBF16 = 1,       // Cb[m*ldc + n] = bf16(acc)
-  kEpiGelu = 2,       // C = acc (u, fp32) and Cb = bf16(GELU(acc))
-  kEpiResidBF16 = 3,  // Cb = bf16(resid[m*ldr + n] + acc), resid in dtype
+  kEpiF32 = 0,         // C[mo*ldc + n] = acc, mo = (m*c_row_mul) mod M when c_row_mul != 0
+  kEpiBF16 = 1,        // Cb[m*ldcb + n] = bf16(acc)
+  kEpiGeluSplit = 2,   // C[m*ldc + n] = acc (u); a = GELU(acc) in fp64, stored as bf16
+                       // hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
+  kEpiResidSplit = 3,  // h = resid[m*ldr + n] (bf16) + acc, stored as bf16 hi/lo planes
 };
 
 struct EpiDesc {
   int kind = kEpiF32;
   float* C = nullptr;
-  __nv_bfloat16* Cb = nullptr;
   int64_t ldc = 0;
+  __nv_bfloat16* Cb = nullptr;
+  int64_t ldcb = 0;
+  int64_t split = 0;
   int64_t c_row_mul = 0;
   const void* resid = nullptr;
   int64_t ldr = 0;
 };
+
+// Exact-erf GELU in fp64 (the clean activation of the MLP variant).
+__device__ __forceinline__ double gelu64(double x) {
+  return 0.5 * x * (1.0 + erf(x * 0.70710678118654752440));
+}
+
+// v as a bf16 pair with v ~= hi + lo (relative error about 2^-17).
+__device__ __forceinline__ void split_bf16(double v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn((float)v);
+  *hi = h;
+  *lo = __float2bfloat16_rn((float)(v - (double)__bfloat162float(h)));
+}
+
+// Round an fp64 value to the nearest bf16 (8 significant bits, ties to even)
+// in one step: the mantissa is rounded on the fp64 bit pattern, after which the
+// value is exactly representable in fp32 and bf16.
+__device__ __forceinline__ __nv_bfloat16 bf16_from_f64(double v) {
+  unsigned long long b = (unsigned long long)__double_as_longlong(v);
+  const unsigned long long keep = (b >> 45) & 1ull;  // lowest kept mantissa bit
+  b = (b + 0x00000FFFFFFFFFFFull + keep) & ~0x00001FFFFFFFFFFFull;
+  return __float2bfloat16_rn((float)__longlong_as_double((long long)b));
+}
 
 // The bf16 GEMM operand of g is stored as two planes, hi = bf16(v) and
 // lo = bf16(v - hi), `plane` elements apart, so sum_t g_t h_t^T computed over
@@ -84,9 +109,11 @@ struct dust_ctx {
   int64_t launches = 0;
   // tensor-core GEMMs on (DUST_DISABLE_TC=1 at creation routes all GEMMs to CUDA cores)
   bool tc_enabled = true;
+  // shared-memory subset kernel on (DUST_SUBSET_KERNEL=1 selects the first, L2-fed one)
+  bool subset2_enabled = true;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
-      mlp_dh, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv;
+      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv;
 };
 
 namespace dust {
@@ -127,6 +154,15 @@ size_t subset_gacc_bytes(int64_t T, int64_t V, int max_smem_optin);
 cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                                const float* P, const int32_t* y, float* rewards, float* g_out,
                                void* gop, float* gacc, int max_smem_optin);
+
+// Subset draws with the probability row and the g accumulator resident in
+// shared memory, one cluster of 1 or 2 CTAs per token (0: not applicable to
+// this V, S). Z holds clean logits in permuted column order, lse the row
+// log-sum-exp; p = exp(z - lse) is formed while the row is loaded.
+int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin);
+cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
+                           const float* Z, const float* lse, const int32_t* y, float* rewards,
+                           float* g_out, void* gop, int max_smem_optin, int sm_count);
 
 // Tensor-core GEMM (tcgen05): shapes it takes, and its launcher. A bounded
 // wait that expires sets kStatusTimeout in *status.

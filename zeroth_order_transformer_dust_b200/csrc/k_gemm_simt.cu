@@ -11,10 +11,6 @@ constexpr int BM = 128, BN = 128, BKT = 16, PAD = 4;
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-__device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
-}
-
 // Loads the A (or B) tile of rows [r0, r0+128) and k in [k0, k0+16) into
 // S[k][row] as fp32, zero-filling outside the matrix.
 template <typename TI, bool KMAJOR>
@@ -96,21 +92,20 @@ __global__ __launch_bounds__(256) void k_gemm_simt(GemmDesc g, EpiDesc e) {
       const int64_t n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
       if (n >= g.N) continue;
       const float v = acc[i][j];
-      const int64_t o = mo * e.ldc + n;
       switch (e.kind) {
         case kEpiF32:
-          e.C[o] = v;
+          e.C[mo * e.ldc + n] = v;
           break;
         case kEpiBF16:
-          e.Cb[o] = __float2bfloat16_rn(v);
+          e.Cb[m * e.ldcb + n] = __float2bfloat16_rn(v);
           break;
-        case kEpiGelu:
-          e.C[o] = v;
-          e.Cb[o] = __float2bfloat16_rn(gelu_erf(v));
+        case kEpiGeluSplit:
+          e.C[m * e.ldc + n] = v;
+          split_bf16(gelu64((double)v), &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
           break;
-        case kEpiResidBF16: {
-          const float r = to_f(((const TI*)e.resid)[m * e.ldr + n]);
-          e.Cb[o] = __float2bfloat16_rn(r + v);
+        case kEpiResidSplit: {
+          const double r = (double)to_f(((const TI*)e.resid)[m * e.ldr + n]);
+          split_bf16(r + (double)v, &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
           break;
         }
       }

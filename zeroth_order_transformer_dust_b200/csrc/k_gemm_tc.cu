@@ -54,18 +54,14 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
   }
 }
 
-__device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
-}
-
 // Epilogue of 32 consecutive columns [n, n+32) of row m (output row mo).
 template <int KIND>
 __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t mo, int64_t n,
                                            const float* v) {
   const EpiDesc& e = p.e;
   const bool full = n + 32 <= p.N;
-  if (KIND == kEpiF32 || KIND == kEpiGelu) {
-    float* dst = e.C + mo * e.ldc + n;
+  if (KIND == kEpiF32 || KIND == kEpiGeluSplit) {
+    float* dst = e.C + (KIND == kEpiF32 ? mo : m) * e.ldc + n;
     if (full && ((e.ldc & 3) == 0) && (((uintptr_t)e.C & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -75,27 +71,15 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
         if (n + q < p.N) dst[q] = v[q];
     }
   }
-  if (KIND == kEpiBF16 || KIND == kEpiGelu || KIND == kEpiResidBF16) {
-    float w[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) w[q] = v[q];
-    if (KIND == kEpiGelu) {
-#pragma unroll
-      for (int q = 0; q < 32; ++q) w[q] = gelu_erf(w[q]);
-    }
-    if (KIND == kEpiResidBF16) {
-      const __nv_bfloat16* r = (const __nv_bfloat16*)e.resid + m * e.ldr + n;
-      for (int q = 0; q < 32; ++q)
-        if (n + q < p.N) w[q] += __bfloat162float(r[q]);
-    }
-    __nv_bfloat16* dst = e.Cb + mo * e.ldc + n;
-    if (full && ((e.ldc & 7) == 0) && (((uintptr_t)e.Cb & 15) == 0)) {
+  if (KIND == kEpiBF16) {
+    __nv_bfloat16* dst = e.Cb + m * e.ldcb + n;
+    if (full && ((e.ldcb & 7) == 0) && (((uintptr_t)e.Cb & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(w[8 * q + 0], w[8 * q + 1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(w[8 * q + 2], w[8 * q + 3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(w[8 * q + 4], w[8 * q + 5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(w[8 * q + 6], w[8 * q + 7]);
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * q + 0], v[8 * q + 1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * q + 2], v[8 * q + 3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 4], v[8 * q + 5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * q + 6], v[8 * q + 7]);
         uint4 u;
         u.x = *reinterpret_cast<uint32_t*>(&h0);
         u.y = *reinterpret_cast<uint32_t*>(&h1);
@@ -105,7 +89,20 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
       }
     } else {
       for (int q = 0; q < 32; ++q)
-        if (n + q < p.N) dst[q] = __float2bfloat16_rn(w[q]);
+        if (n + q < p.N) dst[q] = __float2bfloat16_rn(v[q]);
+    }
+  }
+  if (KIND == kEpiGeluSplit || KIND == kEpiResidSplit) {
+    __nv_bfloat16* hi = e.Cb + m * e.ldcb + n;
+    __nv_bfloat16* lo = hi + e.split;
+    const __nv_bfloat16* r = KIND == kEpiResidSplit ? (const __nv_bfloat16*)e.resid + m * e.ldr + n : nullptr;
+#pragma unroll 4
+    for (int q = 0; q < 32; ++q) {
+      if (n + q < p.N) {
+        const double x = KIND == kEpiGeluSplit ? gelu64((double)v[q])
+                                               : (double)__bfloat162float(r[q]) + (double)v[q];
+        split_bf16(x, hi + q, lo + q);
+      }
     }
   }
 }
@@ -305,13 +302,14 @@ cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap
 
 bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
   if (g.dtype != DUST_BF16 || !g.a_kmajor || !g.b_kmajor || g.b_row_mul != 0) return false;
-  if (g.M < 1 || g.N < 16 || g.K < 16) return false;
+  if (g.M < 1 || g.N < 16 || g.K < 8) return false;
   if ((g.lda & 7) || (g.ldb & 7)) return false;
   if (((uintptr_t)g.A & 15) || ((uintptr_t)g.B & 15)) return false;
   if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX) return false;
-  if (e.kind == kEpiResidBF16 && !e.resid) return false;
+  if (e.kind == kEpiResidSplit && !e.resid) return false;
   if (!encode_fn()) return false;
-  return e.kind == kEpiF32 || e.kind == kEpiBF16 || e.kind == kEpiGelu || e.kind == kEpiResidBF16;
+  return e.kind == kEpiF32 || e.kind == kEpiBF16 || e.kind == kEpiGeluSplit ||
+         e.kind == kEpiResidSplit;
 }
 
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
@@ -332,8 +330,8 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e,
   switch (e.kind) {
     case kEpiF32: return launch_kind<kEpiF32>(st, ma, mb, p, sm_count);
     case kEpiBF16: return launch_kind<kEpiBF16>(st, ma, mb, p, sm_count);
-    case kEpiGelu: return launch_kind<kEpiGelu>(st, ma, mb, p, sm_count);
-    case kEpiResidBF16: return launch_kind<kEpiResidBF16>(st, ma, mb, p, sm_count);
+    case kEpiGeluSplit: return launch_kind<kEpiGeluSplit>(st, ma, mb, p, sm_count);
+    case kEpiResidSplit: return launch_kind<kEpiResidSplit>(st, ma, mb, p, sm_count);
   }
   return cudaErrorInvalidValue;
 }

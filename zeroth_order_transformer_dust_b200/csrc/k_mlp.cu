@@ -11,11 +11,10 @@
 namespace dust {
 namespace {
 
-__device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
-}
-
-// One thread per (row, 128-channel block, lane).
+// One thread per (row, 128-channel block, lane). The difference of the two
+// GELU values is formed in fp64 (in fp32 it would cancel to ~1e-7 absolute,
+// enough to move values across bf16 rounding boundaries) and rounded to bf16
+// once.
 __global__ void k_mlp_delta_a(Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3, float sigma,
                               int64_t d_ff, int32_t K, const float* __restrict__ u, int64_t t0,
                               int64_t rows, __nv_bfloat16* __restrict__ da_bf,
@@ -35,10 +34,10 @@ __global__ void k_mlp_delta_a(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
   for (int j = 0; j < 4; ++j) {
     const int64_t ch = blk * 128 + lane + 32 * j;
     if (ch < d_ff) {
-      const float uv = u[t * d_ff + ch];
-      const float d = gelu_erf(uv + sigma * g.v[j]) - gelu_erf(uv);
-      if (da_bf) da_bf[row * d_ff + ch] = __float2bfloat16_rn(d);
-      if (da_f32) da_f32[row * d_ff + ch] = d;
+      const double uv = (double)u[t * d_ff + ch];
+      const double d = gelu64(uv + (double)sigma * (double)g.v[j]) - gelu64(uv);
+      if (da_bf) da_bf[row * d_ff + ch] = bf16_from_f64(d);
+      if (da_f32) da_f32[row * d_ff + ch] = (float)d;
     }
   }
 }

@@ -1,0 +1,400 @@
+// Vocabulary-subset LM-head draws, shared-memory resident (the kernel the
+// large-subset workload spends its time in).
+//
+// Method ("Dust：无需反向传播的Transformer零阶预训练", §1 减少干扰: the head is
+// perturbed on cached logits and each draw evaluates a small subset of the
+// vocabulary): draw i of token t perturbs logits j_k = (a k + b) mod V, k < S,
+// plus the target; in the permuted column order q (logit a q mod V) the drawn
+// set is the window [c, c+S) mod V, c = a^-1 b. LSE' = LSE +
+// log1p(sum_drawn p_j expm1(sigma eps_j)), r = sigma eps_y - log1p(.), and
+// r eps (scaled by the inverse inclusion probability) accumulates into g_t.
+//
+// B200 mapping: one cluster of CS CTAs (one per SM) per token at a time,
+// persistent over tokens. CTA r of the cluster holds the probability row and
+// the g accumulator for its slice of q in shared memory (CS = 2 at V = 50304:
+// 2 x 100.6 KB per CTA), so the hot loop touches no global memory. A draw is
+// processed by one warp of the CTA that owns its window start; the few
+// windows that run into the next slice (or wrap past V) reach the partner's
+// shared memory through DSMEM. The noise of a draw is generated once, kept in
+// registers from the reward to the accumulation, and the first two Philox
+// rounds are evaluated once per draw and once per slot block (they depend on
+// the draw index or on the slot block only).
+#include <cooperative_groups.h>
+
+#include "internal.cuh"
+#include "noise.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace dust {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+
+struct Sub2Args {
+  Key key;
+  uint32_t t_off, i_off, ctr3, stream_id;
+  float sigma;
+  int64_t T, V;
+  int32_t K, S;
+  uint32_t a, a_inv;
+  uint32_t seg;  // q-slice length owned by one CTA (multiple of 4)
+  float scale_other, scale_target, fac;
+  const float* Z;    // clean logits, permuted columns (T x V)
+  const float* lse;  // T
+  const int32_t* y;
+  float* rewards;
+  float* g_out;
+  void* gop;
+  int gop_bf16;
+  int64_t plane;
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ uint32_t mulmod32(uint32_t x, uint32_t y, uint32_t m) {
+  return (uint32_t)(((uint64_t)x * y) % m);
+}
+
+// Philox4x32-10 with rounds 0 and 1 precomputed. Round 0 maps the counter
+// (c0, t, i, c3) to (A, B, C, D) with A, B functions of the draw and C, D of
+// the slot block; round 1 maps it to (E ^ B, F, G ^ D', H) with E, F, D' per
+// slot block and G, H per draw. Rounds 2..9 follow.
+struct DrawConst {
+  uint32_t B, G, H;
+};
+struct BlockConst {
+  uint32_t E, F, Dp;
+};
+
+__device__ __forceinline__ BlockConst block_const(Key key, uint32_t c0, uint32_t c3) {
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * c0;
+  const uint32_t C = (uint32_t)(p0 >> 32) ^ c3 ^ key.k1;
+  const uint32_t D = (uint32_t)p0;
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * C;
+  BlockConst b;
+  b.E = (uint32_t)(p1 >> 32) ^ (key.k0 + kPhiloxW0);
+  b.F = (uint32_t)p1;
+  b.Dp = D ^ (key.k1 + kPhiloxW1);
+  return b;
+}
+
+__device__ __forceinline__ DrawConst draw_const(Key key, uint32_t t_abs, uint32_t i_abs) {
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * i_abs;
+  const uint32_t A = (uint32_t)(p1 >> 32) ^ t_abs ^ key.k0;
+  DrawConst d;
+  d.B = (uint32_t)p1;
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * A;
+  d.G = (uint32_t)(p0 >> 32);
+  d.H = (uint32_t)p0;
+  return d;
+}
+
+__device__ __forceinline__ U4 philox_from2(const BlockConst& bc, const DrawConst& dc, Key key) {
+  U4 c{bc.E ^ dc.B, bc.F, dc.G ^ bc.Dp, dc.H};
+  uint32_t k0 = key.k0 + 2u * kPhiloxW0, k1 = key.k1 + 2u * kPhiloxW1;
+#pragma unroll
+  for (int r = 2; r < 10; ++r) {
+    c = philox_round(c, k0, k1);
+    k0 += kPhiloxW0;
+    k1 += kPhiloxW1;
+  }
+  return c;
+}
+
+// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
+template <int CS, int NB, bool FULL, int DEG>
+__global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
+  extern __shared__ __align__(16) float smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const uint32_t rank = CS > 1 ? cluster.block_rank() : 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t V = (uint32_t)A.V;
+  const uint32_t seg = A.seg;
+  const uint32_t lo = rank * seg;
+  const uint32_t hi = min(V, lo + seg);
+  const uint32_t n_own = hi - lo;
+  float* sp = smem;        // p of q in [lo, hi)
+  float* sg = smem + seg;  // g accumulator of q in [lo, hi)
+  // partner slices (CS = 2): generic pointers into the other CTA's shared memory
+  float* sp_peer = sp;
+  float* sg_peer = sg;
+  if (CS > 1) {
+    sp_peer = cluster.map_shared_rank(sp, rank ^ 1u);
+    sg_peer = cluster.map_shared_rank(sg, rank ^ 1u);
+  }
+  const int S = A.S;
+  const uint32_t nclusters = gridDim.x / CS;
+  const uint32_t cid = blockIdx.x / CS;
+
+  // per-lane constants of each slot block (rounds 0 and 1 of Philox)
+  BlockConst bc[NB];
+#pragma unroll
+  for (int m = 0; m < NB; ++m) bc[m] = block_const(A.key, slot_ctr0((uint32_t)m, (uint32_t)lane), A.ctr3);
+  const bool vec = (V & 3u) == 0;  // rows start 16-byte aligned
+
+  for (int64_t t = cid; t < A.T; t += nclusters) {
+    // ---- load p = exp(z - LSE) for the owned slice, clear g
+    const float* zrow = A.Z + t * A.V;
+    const float lse_t = A.lse[t];
+    for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
+      if (vec && q + 3 < n_own) {
+        const float4 z = *reinterpret_cast<const float4*>(zrow + lo + q);
+        *reinterpret_cast<float4*>(sp + q) =
+            make_float4(expf(z.x - lse_t), expf(z.y - lse_t), expf(z.z - lse_t), expf(z.w - lse_t));
+        *reinterpret_cast<float4*>(sg + q) = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        for (uint32_t u = q; u < n_own; ++u) {
+          sp[u] = expf(zrow[lo + u] - lse_t);
+          sg[u] = 0.0f;
+        }
+      }
+    }
+    int32_t yt = A.y[t];
+    if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
+    const uint32_t qy = mulmod32((uint32_t)yt, A.a_inv, V);
+    const float py = expf(zrow[qy] - lse_t);
+    float* gy = (qy >= lo && qy < hi) ? sg + (qy - lo) : sg_peer + (qy - (lo ^ seg * (CS > 1)));
+    if (CS > 1) cluster.sync(); else __syncthreads();
+
+    const uint32_t t_abs = A.t_off + (uint32_t)t;
+    // ---- draws: warp w scans draws w*32 + lane, keeps those whose window starts here
+    for (int i0 = warp * 32; i0 < A.K; i0 += kWarps * 32) {
+      const int iq = i0 + lane;
+      uint32_t c = 0;
+      bool mine = false;
+      if (iq < A.K) {
+        const uint32_t b = subset_offset(A.key, t_abs, A.i_off + (uint32_t)iq, A.stream_id, V);
+        c = mulmod32(b, A.a_inv, V);
+        mine = (c >= lo) && (c < hi);
+      }
+      uint32_t mask = __ballot_sync(0xffffffffu, mine);
+      while (mask) {
+        const int src = __ffs(mask) - 1;
+        mask &= mask - 1;
+        const int i = i0 + src;
+        const uint32_t cw = __shfl_sync(0xffffffffu, c, src);
+        const uint32_t i_abs = A.i_off + (uint32_t)i;
+        const DrawConst dc = draw_const(A.key, t_abs, i_abs);
+        const uint32_t ky = (qy >= cw) ? qy - cw : qy + V - cw;
+        const bool in_win = ky < (uint32_t)S;
+        const bool local = (cw + (uint32_t)S) <= hi;  // whole window in this slice
+        float n[NB][4];
+        float s = 0.0f;
+        if (local) {
+          const float* pw = sp + (cw - lo) + lane;
+          float pv[NB][4];
+#pragma unroll
+          for (int m = 0; m < NB; ++m)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int k = m * 128 + lane + 32 * j;
+              pv[m][j] = (FULL || k < S) ? pw[m * 128 + 32 * j] : 0.0f;
+            }
+#pragma unroll
+          for (int m = 0; m < NB; ++m) {
+            const G4 g = gauss4(philox_from2(bc[m], dc, A.key));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int k = m * 128 + lane + 32 * j;
+              const float e = (FULL || k < S) ? g.v[j] : 0.0f;
+              n[m][j] = e;
+              s = fmaf(pv[m][j], expm1_small<DEG>(A.sigma * e), s);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int m = 0; m < NB; ++m) {
+            const G4 g = gauss4(philox_from2(bc[m], dc, A.key));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int k = m * 128 + lane + 32 * j;
+              float e = 0.0f;
+              if (FULL || k < S) {
+                uint32_t q = cw + (uint32_t)k;
+                if (q >= V) q -= V;
+                const float pq = (q >= lo && q < hi) ? sp[q - lo] : sp_peer[q - (lo ^ seg)];
+                e = g.v[j];
+                s = fmaf(pq, expm1_small<DEG>(A.sigma * e), s);
+              }
+              n[m][j] = e;
+            }
+          }
+        }
+        float ey;
+        if (in_win) {
+          const int my = (int)(ky >> 7), jy = (int)((ky >> 5) & 3u);
+          float cand = 0.0f;
+#pragma unroll
+          for (int m = 0; m < NB; ++m)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (m == my && j == jy) cand = n[m][j];
+          ey = __shfl_sync(0xffffffffu, cand, (int)(ky & 31u));
+        } else {
+          // the appended target takes slot S: counter block S >> 7, lane S & 31,
+          // word (S >> 5) & 3 (computed by every lane; the warp needs one value)
+          const BlockConst bs =
+              block_const(A.key, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u), A.ctr3);
+          const U4 w = philox_from2(bs, dc, A.key);
+          const uint32_t word = ((uint32_t)S >> 5) & 3u;
+          const float2 nn = box_muller(word < 2 ? w.x : w.z, word < 2 ? w.y : w.w);
+          ey = (word & 1u) ? nn.y : nn.x;
+          if (lane == 0) s = fmaf(py, expm1_small<DEG>(A.sigma * ey), s);
+        }
+        s = warp_sum(s);
+        const float r = A.sigma * ey - log1pf(s);
+        if (A.rewards && lane == 0) A.rewards[t * A.K + i] = r;
+        if (local) {
+          float* gw = sg + (cw - lo) + lane;
+#pragma unroll
+          for (int m = 0; m < NB; ++m)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int k = m * 128 + lane + 32 * j;
+              if (FULL || k < S) atomicAdd(gw + m * 128 + 32 * j, r * n[m][j]);
+            }
+        } else {
+#pragma unroll
+          for (int m = 0; m < NB; ++m)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int k = m * 128 + lane + 32 * j;
+              if (FULL || k < S) {
+                uint32_t q = cw + (uint32_t)k;
+                if (q >= V) q -= V;
+                float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - (lo ^ seg));
+                atomicAdd(dst, r * n[m][j]);
+              }
+            }
+        }
+        if (!in_win && lane == 0) atomicAdd(gy, r * ey);
+      }
+    }
+    if (CS > 1) cluster.sync(); else __syncthreads();
+
+    // ---- scale and write the owned slice of g
+    for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
+      const uint32_t qg = lo + q;
+      const float v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
+      if (A.gop_bf16)
+        store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + qg, v);
+      else
+        ((float*)A.gop)[t * A.V + qg] = v;
+      if (A.g_out) A.g_out[t * A.V + mulmod32(qg, A.a, V)] = v;
+    }
+    __syncthreads();
+  }
+  if (CS > 1) cluster.sync();
+}
+
+int expm1_degree2(float sigma) {
+  const float xmax = sigma * 5.7686f;
+  if (xmax <= 0.03f) return 4;
+  if (xmax <= 0.06f) return 5;
+  return 0;
+}
+
+template <int CS, int NB, bool FULL, int DEG>
+cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_count) {
+  auto fn = k_subset2<CS, NB, FULL, DEG>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_clusters = sm_count / CS;
+  cfg.gridDim = dim3((unsigned)(max_clusters * CS));
+  int active = 0;
+  if (cudaOccupancyMaxActiveClusters(&active, (void*)fn, &cfg) == cudaSuccess && active > 0)
+    max_clusters = active;
+  cudaGetLastError();
+  int64_t nc = A.T < max_clusters ? A.T : max_clusters;
+  cfg.gridDim = dim3((unsigned)(nc * CS));
+  e = cudaLaunchKernelEx(&cfg, fn, A);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int CS, int NB, bool FULL>
+cudaError_t launch_deg(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
+  if (deg == 4) return launch_one<CS, NB, FULL, 4>(st, A, smem, sm);
+  if (deg == 5) return launch_one<CS, NB, FULL, 5>(st, A, smem, sm);
+  return launch_one<CS, NB, FULL, 0>(st, A, smem, sm);
+}
+
+template <int CS>
+cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
+  const int nb = (A.S + 127) / 128;
+  const bool full = (A.S % 128) == 0;
+  switch (nb) {
+    case 1: return full ? launch_deg<CS, 1, true>(st, A, smem, sm, deg) : launch_deg<CS, 1, false>(st, A, smem, sm, deg);
+    case 2: return full ? launch_deg<CS, 2, true>(st, A, smem, sm, deg) : launch_deg<CS, 2, false>(st, A, smem, sm, deg);
+    case 3: return launch_deg<CS, 3, false>(st, A, smem, sm, deg);
+    case 4: return full ? launch_deg<CS, 4, true>(st, A, smem, sm, deg) : launch_deg<CS, 4, false>(st, A, smem, sm, deg);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace
+
+// Cluster size the shared-memory kernel would use (0: not applicable).
+int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
+  if (S < 1 || S > 512) return 0;
+  const int64_t slack = 1024;
+  if (2 * V * 4 + slack <= max_smem_optin && V <= 65536) return 1;
+  const int64_t seg = ((V + 1) / 2 + 3) / 4 * 4;
+  if (2 * seg * 4 + slack <= max_smem_optin && S <= V - seg && S <= seg) return 2;
+  return 0;
+}
+
+cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
+                           const float* Z, const float* lse, const int32_t* y, float* rewards,
+                           float* g_out, void* gop, int max_smem_optin, int sm_count) {
+  const int cs = subset2_cluster_size(p.V, p.S, max_smem_optin);
+  if (!cs) return cudaErrorNotSupported;
+  Sub2Args A;
+  A.key = key_of(p.seed);
+  A.t_off = (uint32_t)p.token_offset;
+  A.i_off = (uint32_t)p.draw_offset;
+  A.ctr3 = ctr3_of(kTagHead, p.stream_id);
+  A.stream_id = p.stream_id;
+  A.sigma = p.sigma;
+  A.T = p.T;
+  A.V = p.V;
+  A.K = p.K;
+  A.S = p.S;
+  A.a = (uint32_t)a;
+  A.a_inv = (uint32_t)a_inv;
+  A.seg = cs == 1 ? (uint32_t)((p.V + 3) / 4 * 4) : (uint32_t)(((p.V + 1) / 2 + 3) / 4 * 4);
+  A.scale_other = (float)((double)p.V / (double)p.S);
+  A.scale_target = (p.flags & DUST_FLAG_LITERAL_TARGET_SCALE) ? A.scale_other : 1.0f;
+  A.fac = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
+  A.Z = Z;
+  A.lse = lse;
+  A.y = y;
+  A.rewards = rewards;
+  A.g_out = g_out;
+  A.gop = gop;
+  A.gop_bf16 = p.dtype == DUST_BF16;
+  A.plane = p.T * p.V;
+  const size_t smem = (size_t)2 * A.seg * 4;
+  const int deg = expm1_degree2(p.sigma);
+  if (cs == 1) return launch_cs<1>(st, A, smem, sm_count, deg);
+  return launch_cs<2>(st, A, smem, sm_count, deg);
+}
+
+}  // namespace dust
