@@ -42,4 +42,4 @@ from .params import Params  # noqa: F401
 from .head import (  # noqa: F401
     clean_head, head_grad, head_linear_estimate, full_vocab_draws, subset_draws,
 )
-from .mlp import clean_mlp, mlp_grad, mlp_draws, gelu, bf16_rne  # noqa: F401
+from .mlp import clean_mlp, mlp_grad, mlp_draws, gelu  # noqa: F401

@@ -47,17 +47,9 @@ def test_gelu_matches_torch():
     np.testing.assert_allclose(oracle.gelu(x), ref, rtol=0, atol=1e-15)
 
 
-def test_bf16_rounding_matches_torch():
-    rng = np.random.default_rng(1)
-    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
-    x = np.concatenate([x, np.float32([0.0, 1.0, -2.5, 1 + 2 ** -8, 1 + 3 * 2 ** -8])])
-    ref = torch.tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
-    np.testing.assert_array_equal(oracle.bf16_rne(x.astype(np.float64)), ref)
-
-
 def test_clean_forward_matches_torch():
     X, Wu, Wd, Wh, y = _mlp_problem(T=6)
-    c = oracle.clean_mlp(X, Wu, Wd, Wh, y, mirror_bf16=False)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y)
     ref, _ = _torch_loss(X, Wu, Wd, Wh, y)
     assert c["loss"].sum() == pytest.approx(ref, abs=1e-12)
 
@@ -73,12 +65,12 @@ def test_estimate_is_unbiased_exact_expectation():
     """Over +-sqrt(d_ff) e_m noise, g equals dL/du from torch autograd (to O(sigma^2))."""
     X, Wu, Wd, Wh, y = _mlp_problem(T=3)
     _, gu = _torch_loss(X, Wu, Wd, Wh, y, wrt="u")
-    c = oracle.clean_mlp(X, Wu, Wd, Wh, y, mirror_bf16=False)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y)
     d_ff = Wu.shape[0]
     eps = np.concatenate([np.eye(d_ff), -np.eye(d_ff)]) * math.sqrt(d_ff)
     sig = 1e-6
     for t in range(3):
-        r, acc = oracle.mlp_draws(c["u"][t], c["p"][t], y[t], eps, Wd, Wh, sig, mirror_bf16=False)
+        r, acc = oracle.mlp_draws(c["u"][t], c["p"][t], y[t], eps, Wd, Wh, sig)
         g = -acc / (eps.shape[0] * sig)
         np.testing.assert_allclose(g, gu[t], rtol=0, atol=1e-8)
 
@@ -86,7 +78,7 @@ def test_estimate_is_unbiased_exact_expectation():
 def test_closed_form_up_gradient_matches_finite_differences():
     """sum_t [GELU'(u) * W_down^T W_head^T (p - e_y)] x^T against brute force."""
     X, Wu, Wd, Wh, y = _mlp_problem(T=3, d=3, d_ff=4, V=5)
-    c = oracle.clean_mlp(X, Wu, Wd, Wh, y, mirror_bf16=False)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y)
     u, p = c["u"], c["p"]
     dgelu = 0.5 * (1 + np.vectorize(math.erf)(u / math.sqrt(2))) + u * np.exp(-u * u / 2) / math.sqrt(2 * math.pi)
     closed = np.zeros_like(Wu)
@@ -101,8 +93,8 @@ def test_closed_form_up_gradient_matches_finite_differences():
             P, M = Wu.copy(), Wu.copy()
             P[i, j] += h
             M[i, j] -= h
-            fd[i, j] = (oracle.clean_mlp(X, P, Wd, Wh, y, False)["loss"].sum()
-                        - oracle.clean_mlp(X, M, Wd, Wh, y, False)["loss"].sum()) / (2 * h)
+            fd[i, j] = (oracle.clean_mlp(X, P, Wd, Wh, y)["loss"].sum()
+                        - oracle.clean_mlp(X, M, Wd, Wh, y)["loss"].sum()) / (2 * h)
     np.testing.assert_allclose(fd, closed, rtol=0, atol=1e-8)
     _, gW = _torch_loss(X, Wu, Wd, Wh, y, wrt="W_up")
     np.testing.assert_allclose(gW, closed, rtol=0, atol=1e-12)
@@ -114,7 +106,7 @@ def test_estimate_converges_with_population():
     errs = []
     for K in (256, 4096):
         prm = oracle.Params(T=4, d=4, V=7, d_ff=6, K=K, sigma=1e-4, seed=8)
-        G = oracle.mlp_grad(X, Wu, Wd, Wh, y, prm, mirror_bf16=False, draw_chunk=4096)["G"]
+        G = oracle.mlp_grad(X, Wu, Wd, Wh, y, prm, draw_chunk=4096)["G"]
         assert G.shape == Wu.shape
         errs.append(np.linalg.norm(G - gW) / np.linalg.norm(gW))
     assert errs[1] < errs[0] / 2.5

@@ -529,8 +529,8 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   if (tchunk > T) tchunk = T;
   const int64_t rows_cap = tchunk * K;
   const int nparts = (int)((V + 127) / 128);
-  DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * dff * 2));
-  DUST_TRY(ensure(ctx, ctx->mlp_dh, (size_t)rows_cap * d * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * 2 * dff * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_dh, (size_t)rows_cap * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->part, (size_t)rows_cap * nparts * 4));
   DUST_TRY(ensure(ctx, ctx->dzy, (size_t)rows_cap * 4));
   __nv_bfloat16* da = (__nv_bfloat16*)ctx->mlp_da.p;
@@ -542,16 +542,16 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
     ctx->launches += 1;
     {
       GemmDesc g{};
-      g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = dff; g.a_kmajor = true;
-      g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = d; g.K = 2 * dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
+      g.B = ctx->wd2.p; g.ldb = 2 * dff; g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
-      e.kind = kEpiBF16; e.Cb = dh; e.ldcb = d;
+      e.kind = kEpiSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       DUST_TRY(run_gemm(ctx, g, e));
     }
     {
       GemmDesc g{};
-      g.M = rows; g.N = V; g.K = d; g.A = dh; g.lda = d; g.a_kmajor = true;
-      g.B = W_head; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = V; g.K = 2 * d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
+      g.B = ctx->wh2.p; g.ldb = 2 * d; g.b_kmajor = true; g.dtype = DUST_BF16;
       DUST_CU(launch_reward_gemm_simt(st, g, Z, targets, t0, p.K, (float*)ctx->part.p,
                                       (float*)ctx->dzy.p));
     }

@@ -40,6 +40,7 @@ enum EpiKind {
   kEpiGeluSplit = 2,   // C[m*ldc + n] = acc (u); a = GELU(acc) in fp64, stored as bf16
                        // hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
   kEpiResidSplit = 3,  // h = resid[m*ldr + n] (bf16) + acc, stored as bf16 hi/lo planes
+  kEpiSplit = 4,       // acc stored as bf16 hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
 };
 
 struct EpiDesc {
@@ -54,9 +55,11 @@ struct EpiDesc {
   int64_t ldr = 0;
 };
 
-// Exact-erf GELU in fp64 (the clean activation of the MLP variant).
+// Exact-erf GELU in fp64. The last product is rounded on its own
+// (__dmul_rn) so that a difference GELU(x) - GELU(x') is not contracted
+// into a fused multiply-add: equal arguments then give an exact zero.
 __device__ __forceinline__ double gelu64(double x) {
-  return 0.5 * x * (1.0 + erf(x * 0.70710678118654752440));
+  return __dmul_rn(0.5 * x, 1.0 + erf(x * 0.70710678118654752440));
 }
 
 // v as a bf16 pair with v ~= hi + lo (relative error about 2^-17).

@@ -108,6 +108,9 @@ __global__ __launch_bounds__(256) void k_gemm_simt(GemmDesc g, EpiDesc e) {
           split_bf16(r + (double)v, &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
           break;
         }
+        case kEpiSplit:
+          split_bf16((double)v, &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
+          break;
       }
     }
   }

@@ -105,6 +105,29 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
       }
     }
   }
+  if (KIND == kEpiSplit) {
+    __nv_bfloat16* hi = e.Cb + m * e.ldcb + n;
+    __nv_bfloat16* lo = hi + e.split;
+    if (full && ((e.ldcb & 7) == 0) && ((e.split & 7) == 0) && (((uintptr_t)e.Cb & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float a = v[8 * q + 2 * h], b = v[8 * q + 2 * h + 1];
+          const __nv_bfloat162 hh = __floats2bfloat162_rn(a, b);
+          const __nv_bfloat162 ll = __floats2bfloat162_rn(a - __low2float(hh), b - __high2float(hh));
+          hw[h] = *reinterpret_cast<const uint32_t*>(&hh);
+          lw[h] = *reinterpret_cast<const uint32_t*>(&ll);
+        }
+        reinterpret_cast<uint4*>(hi)[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        reinterpret_cast<uint4*>(lo)[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    } else {
+      for (int q = 0; q < 32; ++q)
+        if (n + q < p.N) split_bf16((double)v[q], hi + q, lo + q);
+    }
+  }
 }
 
 template <int KIND>
@@ -309,7 +332,7 @@ bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
   if (e.kind == kEpiResidSplit && !e.resid) return false;
   if (!encode_fn()) return false;
   return e.kind == kEpiF32 || e.kind == kEpiBF16 || e.kind == kEpiGeluSplit ||
-         e.kind == kEpiResidSplit;
+         e.kind == kEpiResidSplit || e.kind == kEpiSplit;
 }
 
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
@@ -332,6 +355,7 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e,
     case kEpiBF16: return launch_kind<kEpiBF16>(st, ma, mb, p, sm_count);
     case kEpiGeluSplit: return launch_kind<kEpiGeluSplit>(st, ma, mb, p, sm_count);
     case kEpiResidSplit: return launch_kind<kEpiResidSplit>(st, ma, mb, p, sm_count);
+    case kEpiSplit: return launch_kind<kEpiSplit>(st, ma, mb, p, sm_count);
   }
   return cudaErrorInvalidValue;
 }

@@ -12,9 +12,8 @@ namespace dust {
 namespace {
 
 // One thread per (row, 128-channel block, lane). The difference of the two
-// GELU values is formed in fp64 (in fp32 it would cancel to ~1e-7 absolute,
-// enough to move values across bf16 rounding boundaries) and rounded to bf16
-// once.
+// GELU values is formed in fp64 (in fp32 it would cancel to ~1e-7 absolute)
+// and stored as bf16 hi/lo planes, da[row*2d_ff + c] and da[row*2d_ff + d_ff + c].
 __global__ void k_mlp_delta_a(Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3, float sigma,
                               int64_t d_ff, int32_t K, const float* __restrict__ u, int64_t t0,
                               int64_t rows, __nv_bfloat16* __restrict__ da_bf,
@@ -36,7 +35,7 @@ __global__ void k_mlp_delta_a(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
     if (ch < d_ff) {
       const double uv = (double)u[t * d_ff + ch];
       const double d = gelu64(uv + (double)sigma * (double)g.v[j]) - gelu64(uv);
-      if (da_bf) da_bf[row * d_ff + ch] = bf16_from_f64(d);
+      if (da_bf) split_bf16(d, &da_bf[row * 2 * d_ff + ch], &da_bf[row * 2 * d_ff + d_ff + ch]);
       if (da_f32) da_f32[row * d_ff + ch] = (float)d;
     }
   }

@@ -12,13 +12,16 @@
 // B200 mapping: one cluster of CS CTAs (one per SM) per token at a time,
 // persistent over tokens. CTA r of the cluster holds the probability row and
 // the g accumulator for its slice of q in shared memory (CS = 2 at V = 50304:
-// 2 x 100.6 KB per CTA), so the hot loop touches no global memory. A draw is
-// processed by one warp of the CTA that owns its window start; the few
-// windows that run into the next slice (or wrap past V) reach the partner's
-// shared memory through DSMEM. The noise of a draw is generated once, kept in
-// registers from the reward to the accumulation, and the first two Philox
-// rounds are evaluated once per draw and once per slot block (they depend on
-// the draw index or on the slot block only).
+// 2 x 100.6 KB per CTA), so the hot loop touches no global memory. Warps take
+// batches of 32 draws from a shared counter; in a batch each lane works out
+// one draw's window start, whether its window holds the target and the noise
+// of the appended target slot, and the warp then processes, one after the
+// other, the draws whose window starts in its CTA's slice. Windows that run
+// into the next slice (or wrap past V) reach the partner's shared memory
+// through DSMEM. The noise of a draw is generated once, already multiplied by
+// sigma, kept in registers from the reward to the accumulation, and the
+// first two Philox rounds are evaluated once per draw and once per slot
+// block (they depend on the draw index or on the slot block only).
 #include <cooperative_groups.h>
 
 #include "internal.cuh"
@@ -30,10 +33,10 @@ namespace dust {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
 
 struct Sub2Args {
   Key key;
+  uint32_t rk0[10], rk1[10];  // round keys k + r (0x9E3779B9, 0xBB67AE85)
   uint32_t t_off, i_off, ctr3, stream_id;
   float sigma;
   int64_t T, V;
@@ -72,56 +75,53 @@ struct BlockConst {
   uint32_t E, F, Dp;
 };
 
-__device__ __forceinline__ BlockConst block_const(Key key, uint32_t c0, uint32_t c3) {
+__device__ __forceinline__ BlockConst block_const(const Sub2Args& A, uint32_t c0) {
   const uint64_t p0 = (uint64_t)kPhiloxM0 * c0;
-  const uint32_t C = (uint32_t)(p0 >> 32) ^ c3 ^ key.k1;
+  const uint32_t C = (uint32_t)(p0 >> 32) ^ A.ctr3 ^ A.rk1[0];
   const uint32_t D = (uint32_t)p0;
   const uint64_t p1 = (uint64_t)kPhiloxM1 * C;
   BlockConst b;
-  b.E = (uint32_t)(p1 >> 32) ^ (key.k0 + kPhiloxW0);
+  b.E = (uint32_t)(p1 >> 32) ^ A.rk0[1];
   b.F = (uint32_t)p1;
-  b.Dp = D ^ (key.k1 + kPhiloxW1);
+  b.Dp = D ^ A.rk1[1];
   return b;
 }
 
-__device__ __forceinline__ DrawConst draw_const(Key key, uint32_t t_abs, uint32_t i_abs) {
+__device__ __forceinline__ DrawConst draw_const(const Sub2Args& A, uint32_t t_abs, uint32_t i_abs) {
   const uint64_t p1 = (uint64_t)kPhiloxM1 * i_abs;
-  const uint32_t A = (uint32_t)(p1 >> 32) ^ t_abs ^ key.k0;
+  const uint32_t Aw = (uint32_t)(p1 >> 32) ^ t_abs ^ A.rk0[0];
   DrawConst d;
   d.B = (uint32_t)p1;
-  const uint64_t p0 = (uint64_t)kPhiloxM0 * A;
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * Aw;
   d.G = (uint32_t)(p0 >> 32);
   d.H = (uint32_t)p0;
   return d;
 }
 
-__device__ __forceinline__ U4 philox_from2(const BlockConst& bc, const DrawConst& dc, Key key) {
+__device__ __forceinline__ U4 philox_from2(const BlockConst& bc, const DrawConst& dc,
+                                           const Sub2Args& A) {
   U4 c{bc.E ^ dc.B, bc.F, dc.G ^ bc.Dp, dc.H};
-  uint32_t k0 = key.k0 + 2u * kPhiloxW0, k1 = key.k1 + 2u * kPhiloxW1;
 #pragma unroll
-  for (int r = 2; r < 10; ++r) {
-    c = philox_round(c, k0, k1);
-    k0 += kPhiloxW0;
-    k1 += kPhiloxW1;
-  }
+  for (int r = 2; r < 10; ++r) c = philox_round(c, A.rk0[r], A.rk1[r]);
   return c;
 }
 
 // NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
 template <int CS, int NB, bool FULL, int DEG>
-__global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
+__global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__ Sub2Args A) {
   extern __shared__ __align__(16) float smem[];
+  __shared__ int s_next;  // next draw batch of the current token
   cg::cluster_group cluster = cg::this_cluster();
   const uint32_t rank = CS > 1 ? cluster.block_rank() : 0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const uint32_t V = (uint32_t)A.V;
   const uint32_t seg = A.seg;
   const uint32_t lo = rank * seg;
   const uint32_t hi = min(V, lo + seg);
   const uint32_t n_own = hi - lo;
+  const uint32_t lo_peer = lo ^ seg;  // CS = 2: the partner's slice start
   float* sp = smem;        // p of q in [lo, hi)
   float* sg = smem + seg;  // g accumulator of q in [lo, hi)
-  // partner slices (CS = 2): generic pointers into the other CTA's shared memory
   float* sp_peer = sp;
   float* sg_peer = sg;
   if (CS > 1) {
@@ -131,11 +131,14 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
   const int S = A.S;
   const uint32_t nclusters = gridDim.x / CS;
   const uint32_t cid = blockIdx.x / CS;
+  const int nbatch = (A.K + 31) >> 5;
 
-  // per-lane constants of each slot block (rounds 0 and 1 of Philox)
   BlockConst bc[NB];
 #pragma unroll
-  for (int m = 0; m < NB; ++m) bc[m] = block_const(A.key, slot_ctr0((uint32_t)m, (uint32_t)lane), A.ctr3);
+  for (int m = 0; m < NB; ++m) bc[m] = block_const(A, slot_ctr0((uint32_t)m, (uint32_t)lane));
+  // the appended target slot S: counter block S >> 7, lane S & 31, word (S >> 5) & 3
+  const BlockConst bs = block_const(A, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u));
+  const uint32_t s_word = ((uint32_t)S >> 5) & 3u;
   const bool vec = (V & 3u) == 0;  // rows start 16-byte aligned
 
   for (int64_t t = cid; t < A.T; t += nclusters) {
@@ -149,42 +152,55 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
             make_float4(expf(z.x - lse_t), expf(z.y - lse_t), expf(z.z - lse_t), expf(z.w - lse_t));
         *reinterpret_cast<float4*>(sg + q) = make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
-        for (uint32_t u = q; u < n_own; ++u) {
+        for (uint32_t u = q; u < n_own && u < q + 4; ++u) {
           sp[u] = expf(zrow[lo + u] - lse_t);
           sg[u] = 0.0f;
         }
       }
     }
+    if (threadIdx.x == 0) s_next = 0;
     int32_t yt = A.y[t];
     if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
     const uint32_t qy = mulmod32((uint32_t)yt, A.a_inv, V);
     const float py = expf(zrow[qy] - lse_t);
-    float* gy = (qy >= lo && qy < hi) ? sg + (qy - lo) : sg_peer + (qy - (lo ^ seg * (CS > 1)));
+    float* gy = (qy >= lo && qy < hi) ? sg + (qy - lo) : sg_peer + (qy - lo_peer);
     if (CS > 1) cluster.sync(); else __syncthreads();
 
     const uint32_t t_abs = A.t_off + (uint32_t)t;
-    // ---- draws: warp w scans draws w*32 + lane, keeps those whose window starts here
-    for (int i0 = warp * 32; i0 < A.K; i0 += kWarps * 32) {
-      const int iq = i0 + lane;
-      uint32_t c = 0;
+    for (;;) {
+      int bidx = 0;
+      if (lane == 0) bidx = atomicAdd(&s_next, 1);
+      bidx = __shfl_sync(0xffffffffu, bidx, 0);
+      if (bidx >= nbatch) break;
+      // ---- per-lane setup of draw bidx*32 + lane
+      const int iq = bidx * 32 + lane;
+      uint32_t c = 0, kyq = 0;
+      float x_extra = 0.0f;
       bool mine = false;
       if (iq < A.K) {
-        const uint32_t b = subset_offset(A.key, t_abs, A.i_off + (uint32_t)iq, A.stream_id, V);
+        const uint32_t i_abs = A.i_off + (uint32_t)iq;
+        const uint32_t b = subset_offset(A.key, t_abs, i_abs, A.stream_id, V);
         c = mulmod32(b, A.a_inv, V);
         mine = (c >= lo) && (c < hi);
+        kyq = (qy >= c) ? qy - c : qy + V - c;
+        if (mine && kyq >= (uint32_t)S) {
+          const U4 w = philox_from2(bs, draw_const(A, t_abs, i_abs), A);
+          const float2 nn = box_muller(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, A.sigma);
+          x_extra = (s_word & 1u) ? nn.y : nn.x;
+        }
       }
       uint32_t mask = __ballot_sync(0xffffffffu, mine);
       while (mask) {
         const int src = __ffs(mask) - 1;
         mask &= mask - 1;
-        const int i = i0 + src;
+        const int i = bidx * 32 + src;
         const uint32_t cw = __shfl_sync(0xffffffffu, c, src);
-        const uint32_t i_abs = A.i_off + (uint32_t)i;
-        const DrawConst dc = draw_const(A.key, t_abs, i_abs);
-        const uint32_t ky = (qy >= cw) ? qy - cw : qy + V - cw;
+        const uint32_t ky = __shfl_sync(0xffffffffu, kyq, src);
+        const float xe = __shfl_sync(0xffffffffu, x_extra, src);
+        const DrawConst dc = draw_const(A, t_abs, A.i_off + (uint32_t)i);
         const bool in_win = ky < (uint32_t)S;
         const bool local = (cw + (uint32_t)S) <= hi;  // whole window in this slice
-        float n[NB][4];
+        float n[NB][4];  // sigma * eps of the draw's slots
         float s = 0.0f;
         if (local) {
           const float* pw = sp + (cw - lo) + lane;
@@ -198,35 +214,35 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
             }
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4(philox_from2(bc[m], dc, A.key));
+            const G4 g = gauss4(philox_from2(bc[m], dc, A), A.sigma);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
-              const float e = (FULL || k < S) ? g.v[j] : 0.0f;
-              n[m][j] = e;
-              s = fmaf(pv[m][j], expm1_small<DEG>(A.sigma * e), s);
+              const float x = (FULL || k < S) ? g.v[j] : 0.0f;
+              n[m][j] = x;
+              s = fmaf(pv[m][j], expm1_small<DEG>(x), s);
             }
           }
         } else {
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4(philox_from2(bc[m], dc, A.key));
+            const G4 g = gauss4(philox_from2(bc[m], dc, A), A.sigma);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
-              float e = 0.0f;
+              float x = 0.0f;
               if (FULL || k < S) {
                 uint32_t q = cw + (uint32_t)k;
                 if (q >= V) q -= V;
-                const float pq = (q >= lo && q < hi) ? sp[q - lo] : sp_peer[q - (lo ^ seg)];
-                e = g.v[j];
-                s = fmaf(pq, expm1_small<DEG>(A.sigma * e), s);
+                const float pq = (q >= lo && q < hi) ? sp[q - lo] : sp_peer[q - lo_peer];
+                x = g.v[j];
+                s = fmaf(pq, expm1_small<DEG>(x), s);
               }
-              n[m][j] = e;
+              n[m][j] = x;
             }
           }
         }
-        float ey;
+        float xy;
         if (in_win) {
           const int my = (int)(ky >> 7), jy = (int)((ky >> 5) & 3u);
           float cand = 0.0f;
@@ -235,20 +251,13 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               if (m == my && j == jy) cand = n[m][j];
-          ey = __shfl_sync(0xffffffffu, cand, (int)(ky & 31u));
+          xy = __shfl_sync(0xffffffffu, cand, (int)(ky & 31u));
         } else {
-          // the appended target takes slot S: counter block S >> 7, lane S & 31,
-          // word (S >> 5) & 3 (computed by every lane; the warp needs one value)
-          const BlockConst bs =
-              block_const(A.key, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u), A.ctr3);
-          const U4 w = philox_from2(bs, dc, A.key);
-          const uint32_t word = ((uint32_t)S >> 5) & 3u;
-          const float2 nn = box_muller(word < 2 ? w.x : w.z, word < 2 ? w.y : w.w);
-          ey = (word & 1u) ? nn.y : nn.x;
-          if (lane == 0) s = fmaf(py, expm1_small<DEG>(A.sigma * ey), s);
+          xy = xe;
+          if (lane == 0) s = fmaf(py, expm1_small<DEG>(xy), s);
         }
         s = warp_sum(s);
-        const float r = A.sigma * ey - log1pf(s);
+        const float r = xy - log1p_small(s);
         if (A.rewards && lane == 0) A.rewards[t * A.K + i] = r;
         if (local) {
           float* gw = sg + (cw - lo) + lane;
@@ -268,17 +277,17 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(Sub2Args A) {
               if (FULL || k < S) {
                 uint32_t q = cw + (uint32_t)k;
                 if (q >= V) q -= V;
-                float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - (lo ^ seg));
+                float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - lo_peer);
                 atomicAdd(dst, r * n[m][j]);
               }
             }
         }
-        if (!in_win && lane == 0) atomicAdd(gy, r * ey);
+        if (!in_win && lane == 0) atomicAdd(gy, r * xy);
       }
     }
     if (CS > 1) cluster.sync(); else __syncthreads();
 
-    // ---- scale and write the owned slice of g
+    // ---- scale and write the owned slice of g (accumulated as sum r * sigma eps)
     for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
       const uint32_t qg = lo + q;
       const float v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
@@ -368,6 +377,10 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   if (!cs) return cudaErrorNotSupported;
   Sub2Args A;
   A.key = key_of(p.seed);
+  for (int r = 0; r < 10; ++r) {
+    A.rk0[r] = A.key.k0 + (uint32_t)r * kPhiloxW0;
+    A.rk1[r] = A.key.k1 + (uint32_t)r * kPhiloxW1;
+  }
   A.t_off = (uint32_t)p.token_offset;
   A.i_off = (uint32_t)p.draw_offset;
   A.ctr3 = ctr3_of(kTagHead, p.stream_id);
@@ -382,7 +395,8 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.seg = cs == 1 ? (uint32_t)((p.V + 3) / 4 * 4) : (uint32_t)(((p.V + 1) / 2 + 3) / 4 * 4);
   A.scale_other = (float)((double)p.V / (double)p.S);
   A.scale_target = (p.flags & DUST_FLAG_LITERAL_TARGET_SCALE) ? A.scale_other : 1.0f;
-  A.fac = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
+  // the accumulator holds sum r (sigma eps): g = -(1/(K sigma)) sum r eps
+  A.fac = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * (double)p.sigma * (double)p.sigma)) : 0.0f;
   A.Z = Z;
   A.lse = lse;
   A.y = y;

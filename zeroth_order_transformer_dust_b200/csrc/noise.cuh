@@ -53,25 +53,21 @@ __device__ __forceinline__ U4 philox10(U4 c, uint32_t k0, uint32_t k1) {
 }
 
 // -ln(u) for u in (0, 1], accurate to a few ulp relative to the result,
-// including u -> 1. u = 2^e m with m in [sqrt(1/2), sqrt(2)); ln m is
-// 2 atanh(s), s = (m-1)/(m+1), |s| <= 0.172, from its Taylor series
-// (2 s (1 + s^2/3 + s^4/5 + s^6/7 + s^8/9), truncation < 1e-9 relative);
-// e ln 2 uses ln 2 split in a high part with 8 trailing zero bits (exact
-// products for |e| <= 2^8) and a low correction (Cody and Waite's argument
-// reduction).
+// including u -> 1. u = 2^e m with m in [sqrt(1/2), sqrt(2)): subtracting the
+// bit pattern of sqrt(1/2) before extracting the exponent lands m in that
+// range without a branch. ln m is 2 atanh(s), s = (m-1)/(m+1), |s| <= 0.1716,
+// from its Taylor series 2 s (1 + s^2/3 + s^4/5 + s^6/7) (truncation below
+// 3e-8 absolute, vanishing as m -> 1); e ln 2 uses ln 2 split in a high part
+// with 8 trailing zero bits (exact products for |e| <= 2^8) and a low
+// correction (Cody and Waite's argument reduction).
 __device__ __forceinline__ float neg_log_unit(float u) {
-  int bits = __float_as_int(u);
-  int e = ((bits >> 23) & 0xff) - 127;
-  float m = __int_as_float((bits & 0x007fffff) | 0x3f800000);
-  if (m > 1.41421356f) {
-    m *= 0.5f;
-    e += 1;
-  }
+  const int bits = __float_as_int(u);
+  const int e = (bits - 0x3f3504f3) >> 23;  // arithmetic shift: floor
+  const float m = __int_as_float(bits - (e << 23));
   const float f = m - 1.0f;  // exact (Sterbenz)
   const float s = __fdividef(f, m + 1.0f);
   const float w = s * s;
-  float poly = fmaf(w, 2.0f / 9.0f, 2.0f / 7.0f);
-  poly = fmaf(w, poly, 2.0f / 5.0f);
+  float poly = fmaf(w, 2.0f / 7.0f, 2.0f / 5.0f);
   poly = fmaf(w, poly, 2.0f / 3.0f);
   poly = fmaf(w, poly, 2.0f);
   const float ln_m = s * poly;
@@ -80,6 +76,17 @@ __device__ __forceinline__ float neg_log_unit(float u) {
   const float kLn2Lo = 1.428606765330187e-06f;    // ln 2 - kLn2Hi
   const float ln_u = fmaf(fe, kLn2Hi, fmaf(fe, kLn2Lo, ln_m));
   return -ln_u;
+}
+
+// sqrt(x) for x >= 0: the hardware reciprocal-square-root estimate y refined
+// by one Newton-Raphson step on r = x y (r' = r + (y/2)(x - r^2)), which
+// leaves about one ulp of error. x is clamped away from 0 (sqrt(0) -> 1e-15).
+__device__ __forceinline__ float sqrt_newton(float x) {
+  const float xs = fmaxf(x, 1e-30f);
+  const float y = rsqrtf(xs);
+  const float r = xs * y;
+  const float e = fmaf(-r, r, xs);
+  return fmaf(0.5f * y, e, r);
 }
 
 // cos and sin of 2 pi m 2^-24 for an integer m in [0, 2^24). The nearest
@@ -109,29 +116,36 @@ __device__ __forceinline__ void sincos_turn24(uint32_t m, float* s_out, float* c
 }
 
 // Box-Muller on 24-bit uniforms: u1 = ((wa>>8)+1) 2^-24, u2 = (wb>>8) 2^-24;
-// returns (R cos 2 pi u2, R sin 2 pi u2), R = sqrt(-2 ln u1).
-__device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb) {
+// returns scale * (R cos 2 pi u2, R sin 2 pi u2), R = sqrt(-2 ln u1).
+__device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb, float scale = 1.0f) {
   const float u1 = (float)((wa >> 8) + 1u) * 5.9604645e-08f;  // exact
-  const float radius = sqrtf(2.0f * neg_log_unit(u1));
+  const float radius = scale * sqrt_newton(2.0f * neg_log_unit(u1));
   float s, c;
   sincos_turn24(wb >> 8, &s, &c);
   return make_float2(radius * c, radius * s);
 }
 
-// Four Gaussians of one counter: element j is output word j.
+// Four Gaussians of one counter (times `scale`): element j is output word j.
 struct G4 {
   float v[4];
 };
 
-__device__ __forceinline__ G4 gauss4(U4 w) {
-  const float2 a = box_muller(w.x, w.y);
-  const float2 b = box_muller(w.z, w.w);
+__device__ __forceinline__ G4 gauss4(U4 w, float scale = 1.0f) {
+  const float2 a = box_muller(w.x, w.y, scale);
+  const float2 b = box_muller(w.z, w.w, scale);
   G4 g;
   g.v[0] = a.x;
   g.v[1] = a.y;
   g.v[2] = b.x;
   g.v[3] = b.y;
   return g;
+}
+
+// log1p(s): short series for |s| < 2^-10 (truncation s^4/4 < 2^-42), the
+// library function otherwise. Callers pass warp-uniform s.
+__device__ __forceinline__ float log1p_small(float s) {
+  if (fabsf(s) < 9.765625e-4f) return s * fmaf(s, fmaf(s, 1.0f / 3.0f, -0.5f), 1.0f);
+  return log1pf(s);
 }
 
 // Counter word 0 for slot block `blk` (128 slots) and lane `lane`.
