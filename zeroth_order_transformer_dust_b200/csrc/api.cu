@@ -548,16 +548,27 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
       e.kind = kEpiSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       DUST_TRY(run_gemm(ctx, g, e));
     }
+    // dz = dh W_head^T with the reward epilogue (dz never reaches memory)
+    int used_parts = nparts;
     {
       GemmDesc g{};
       g.M = rows; g.N = V; g.K = 2 * d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
       g.B = ctx->wh2.p; g.ldb = 2 * d; g.b_kmajor = true; g.dtype = DUST_BF16;
-      DUST_CU(launch_reward_gemm_simt(st, g, Z, targets, t0, p.K, (float*)ctx->part.p,
-                                      (float*)ctx->dzy.p));
+      EpiDesc e{};
+      e.kind = kEpiReward; e.P = Z; e.y = targets; e.t0 = t0; e.draws = p.K;
+      e.part = (float*)ctx->part.p; e.dzy = (float*)ctx->dzy.p;
+      if (ctx->tc_enabled && tc_gemm_supported(g, e)) {
+        DUST_TRY(run_gemm(ctx, g, e));
+        used_parts = (int)((V + kTcTileN - 1) / kTcTileN);
+      } else {
+        DUST_CU(launch_reward_gemm_simt(st, g, Z, targets, t0, p.K, (float*)ctx->part.p,
+                                        (float*)ctx->dzy.p));
+        ctx->launches += 1;
+      }
     }
-    DUST_CU(launch_reward_combine_rows(st, (float*)ctx->part.p, nparts, (float*)ctx->dzy.p, rows,
-                                       t0 * K, p.K, r));
-    ctx->launches += 2;
+    DUST_CU(launch_reward_combine_rows(st, (float*)ctx->part.p, used_parts, (float*)ctx->dzy.p,
+                                       rows, t0 * K, p.K, r));
+    ctx->launches += 1;
   }
   mark(ctx, "perturbed");
   DUST_CU(launch_mlp_g(st, p, r, g_out, ctx->gop.p));

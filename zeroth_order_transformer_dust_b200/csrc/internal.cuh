@@ -41,6 +41,9 @@ enum EpiKind {
                        // hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
   kEpiResidSplit = 3,  // h = resid[m*ldr + n] (bf16) + acc, stored as bf16 hi/lo planes
   kEpiSplit = 4,       // acc stored as bf16 hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
+  kEpiReward = 5,      // MLP perturbed logits dz (never stored): per row m and 256-column
+                       // tile nb, part[m*n_tiles + nb] = sum_n P[t, n] expm1(dz);
+                       // dzy[m] = dz at column y[t]; t = t0 + m / draws
 };
 
 struct EpiDesc {
@@ -53,7 +56,17 @@ struct EpiDesc {
   int64_t c_row_mul = 0;
   const void* resid = nullptr;
   int64_t ldr = 0;
+  // kEpiReward
+  const float* P = nullptr;
+  const int32_t* y = nullptr;
+  int64_t t0 = 0;
+  int32_t draws = 1;
+  float* part = nullptr;
+  float* dzy = nullptr;
 };
+
+// Column tile width of the tensor-core GEMM (reward partials per row = ceil(N / it)).
+constexpr int kTcTileN = 256;
 
 // Exact-erf GELU in fp64. The last product is rounded on its own
 // (__dmul_rn) so that a difference GELU(x) - GELU(x') is not contracted

@@ -17,6 +17,7 @@ namespace dust {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+static_assert(BN == kTcTileN, "reward partials are laid out per BN-column tile");
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -128,6 +129,46 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
         if (n + q < p.N) split_bf16((double)v[q], hi + q, lo + q);
     }
   }
+}
+
+// expm1 of a perturbed logit: degree-5 Taylor polynomial below 1/16
+// (relative truncation < 2e-9), the library function otherwise.
+__device__ __forceinline__ float expm1_guarded(float x) {
+  if (fabsf(x) < 0.0625f) {
+    float q = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
+    q = fmaf(x, q, 1.0f / 6.0f);
+    q = fmaf(x, q, 0.5f);
+    q = fmaf(x, q, 1.0f);
+    return x * q;
+  }
+  return expm1f(x);
+}
+
+// Reward epilogue of 32 columns of row m (token t, target column yt): returns
+// sum_n P[t, n] expm1(dz_n) and records dz at the target column.
+__device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int64_t t, int32_t yt,
+                                          int64_t n, const float* v) {
+  const float* prow = p.e.P + t * p.N + n;
+  float s = 0.0f;
+  if (n + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 pv = __ldg(reinterpret_cast<const float4*>(prow) + q);
+      s = fmaf(pv.x, expm1_guarded(v[4 * q + 0]), s);
+      s = fmaf(pv.y, expm1_guarded(v[4 * q + 1]), s);
+      s = fmaf(pv.z, expm1_guarded(v[4 * q + 2]), s);
+      s = fmaf(pv.w, expm1_guarded(v[4 * q + 3]), s);
+    }
+  } else {
+    for (int q = 0; q < 32; ++q)
+      if (n + q < p.N) s = fmaf(prow[q], expm1_guarded(v[q]), s);
+  }
+  if (yt >= n && yt < n + 32) {
+#pragma unroll
+    for (int q = 0; q < 32; ++q)
+      if (n + q == yt) p.e.dzy[m] = v[q];
+  }
+  return s;
 }
 
 template <int KIND>
@@ -261,13 +302,26 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
         mo = (int64_t)(((unsigned long long)m * (unsigned long long)p.e.c_row_mul) %
                        (unsigned long long)p.M);
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      int64_t t_row = 0;
+      int32_t yt = 0;
+      if (KIND == kEpiReward && m < p.M) {
+        t_row = p.e.t0 + m / p.e.draws;
+        yt = p.e.y[t_row];
+        if (yt < 0 || (int64_t)yt >= p.N) yt = 0;  // reported by the loss kernel
+      }
+      float s_row = 0.0f;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int64_t n = (int64_t)n_blk * BN + c * 32;
         float v[32];
         ptx::tmem_ld32(taddr + (uint32_t)(c * 32), v);
-        if (m < p.M && n < p.N) epilogue32<KIND>(p, m, mo, n, v);
+        if (KIND == kEpiReward) {
+          if (m < p.M && n < p.N) s_row += reward32(p, m, t_row, yt, n, v);
+        } else if (m < p.M && n < p.N) {
+          epilogue32<KIND>(p, m, mo, n, v);
+        }
       }
+      if (KIND == kEpiReward && m < p.M) p.e.part[m * p.n_tiles + n_blk] = s_row;
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sh->tempty[acc]));
@@ -330,9 +384,10 @@ bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
   if (((uintptr_t)g.A & 15) || ((uintptr_t)g.B & 15)) return false;
   if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX) return false;
   if (e.kind == kEpiResidSplit && !e.resid) return false;
+  if (e.kind == kEpiReward && (!e.P || !e.y || !e.part || !e.dzy || e.draws < 1)) return false;
   if (!encode_fn()) return false;
   return e.kind == kEpiF32 || e.kind == kEpiBF16 || e.kind == kEpiGeluSplit ||
-         e.kind == kEpiResidSplit || e.kind == kEpiSplit;
+         e.kind == kEpiResidSplit || e.kind == kEpiSplit || e.kind == kEpiReward;
 }
 
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
@@ -356,6 +411,7 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e,
     case kEpiGeluSplit: return launch_kind<kEpiGeluSplit>(st, ma, mb, p, sm_count);
     case kEpiResidSplit: return launch_kind<kEpiResidSplit>(st, ma, mb, p, sm_count);
     case kEpiSplit: return launch_kind<kEpiSplit>(st, ma, mb, p, sm_count);
+    case kEpiReward: return launch_kind<kEpiReward>(st, ma, mb, p, sm_count);
   }
   return cudaErrorInvalidValue;
 }
