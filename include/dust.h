@@ -169,6 +169,35 @@ int dust_stage_times(dust_ctx* ctx, const char** names, float* ms, int cap);
 /* Number of kernels the context has launched since it was created. */
 int64_t dust_kernel_launches(const dust_ctx* ctx);
 
+/*
+ * The LM-head estimator without any allocation, for callers that cannot call
+ * cudaMalloc: code whose device memory is entirely owned by another allocator
+ * (a framework's caching allocator or a pre-reserved pool, where a fresh
+ * cudaMalloc fails or fragments the pool), and latency-critical code that
+ * cannot afford the device-wide synchronisation cudaMalloc and cudaFree can
+ * cause. The Dust pages have no counterpart to this entry point; it computes
+ * exactly what dust_head_grad computes (same arguments and outputs, all device
+ * pointers owned by the caller, on `cuda_stream` of the current device).
+ *   - No context and no allocation: all scratch (logits, log-sum-exp, partial
+ *     sums, rewards, the g operand, the status word) lives in one fixed 16 MiB
+ *     device array that every GPU loading this library holds until the
+ *     process exits. Problems needing more scratch than that (roughly
+ *     T * V <= 2M fp32 elements) return DUST_ERR_UNSUPPORTED with the needed
+ *     size in `msg`; CUDA-core GEMMs only.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the array, which keeps the previous call's contents
+ *     (each call clears what must start at zero). Calls that overlap on the
+ *     GPU, on any stream or thread, race on it: serialise them.
+ *   - The call synchronises `cuda_stream` to read the device status word.
+ * Errors as dust_head_grad, with the reason in `msg` (may be NULL).
+ */
+dust_status dust_head_grad_noalloc(const dust_params* p, void* cuda_stream,
+                                   const void* H, const void* W, const int32_t* targets,
+                                   float* G_out, float* loss_out, float* rewards_out,
+                                   float* g_out, char* msg, int msg_len);
+
 /* Debug: C (M x N, fp32, row-major) = A B^T for bf16 row-major A (M x K) and
    B (N x K), through the library's GEMMs: path 0 = automatic, 1 = CUDA cores,
    2 = tcgen05 tensor cores (DUST_ERR_UNSUPPORTED when the shape does not fit:
