@@ -382,8 +382,14 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=0,
-                    help="oracle sample size in tokens (default: one or two per host core)")
+                    help="oracle sample size in tokens (default: one per host core, at most 16)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run only the first N tokens of the workload (profiling slices)")
     args = ap.parse_args(argv)
+    if args.tokens:
+        import synth
+        wl = synth.CONFIGS[args.config]
+        synth.CONFIGS[args.config] = wl.with_(T=min(args.tokens, wl.T))
     if args.impl == "reference":
         return run_reference(args)
     return run_dust(args)

@@ -212,6 +212,11 @@ dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4
    under p's seed, offsets and stream_id -> out[(t*ni + i)*nslots + k] fp32. */
 dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag,
                              int64_t nt, int64_t ni, int64_t nslots, float* out);
+/* Debug: the same eps through the table-driven angle step the subset-draw
+   kernel uses (a 1024-entry table of roots of unity plus angle addition);
+   it agrees with dust_debug_gauss to a few 1e-7. */
+dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t tag,
+                                 int64_t nt, int64_t ni, int64_t nslots, float* out);
 
 #ifdef __cplusplus
 }

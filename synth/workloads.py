@@ -1,8 +1,8 @@
 """Workload table and seeded input generators.
 
-Recipe (all host-side, numpy PCG64 via ``default_rng(seed)``, drawn in the
-fixed order H, W, targets for the LM-head workloads and x, W_up, W_down,
-W_head, targets for the MLP workload):
+Recipe (all host-side, numpy PCG64; the workload seed's SeedSequence spawns
+one child stream per tensor, in the order H, W, targets for the LM-head
+workloads and x, W_up, W_down, W_head, targets for the MLP workload):
 
 * H ~ N(0, 1), then each row divided by its RMS sqrt(mean(h^2)).
 * W ~ N(0, 1/d), so logits z = W h are roughly N(0, 1) per entry.
@@ -98,24 +98,31 @@ def _targets(rng, wl: Workload) -> np.ndarray:
     return zipf_targets(rng, wl.T, wl.V)
 
 
+def _streams(seed: int, n: int):
+    """Independent child generators, one per input tensor, so that the size of
+    one tensor never shifts the values of another (a workload cut to its first
+    T tokens keeps the same weights and the same first T rows and targets)."""
+    return [np.random.default_rng(s) for s in np.random.SeedSequence(seed).spawn(n)]
+
+
 def make_head_inputs(wl: Workload) -> dict:
     """H (T x d), W (V x d), targets (T,) for an LM-head workload."""
-    rng = np.random.default_rng(wl.seed)
-    H = rng.standard_normal((wl.T, wl.d))
+    rH, rW, ry = _streams(wl.seed, 3)
+    H = rH.standard_normal((wl.T, wl.d))
     H /= np.sqrt(np.mean(H * H, axis=1, keepdims=True))
-    W = rng.standard_normal((wl.V, wl.d)) * (1.0 / np.sqrt(wl.d))
-    y = _targets(rng, wl)
+    W = rW.standard_normal((wl.V, wl.d)) * (1.0 / np.sqrt(wl.d))
+    y = _targets(ry, wl)
     return {"H": _cast(H, wl.dtype), "W": _cast(W, wl.dtype), "targets": y}
 
 
 def make_mlp_inputs(wl: Workload) -> dict:
     """x (T x d), W_up (d_ff x d), W_down (d x d_ff), W_head (V x d), targets."""
-    rng = np.random.default_rng(wl.seed)
-    X = rng.standard_normal((wl.T, wl.d))
-    W_up = rng.standard_normal((wl.d_ff, wl.d)) * (1.0 / np.sqrt(wl.d))
-    W_down = rng.standard_normal((wl.d, wl.d_ff)) * (1.0 / np.sqrt(wl.d_ff))
-    W_head = rng.standard_normal((wl.V, wl.d)) * (1.0 / np.sqrt(wl.d))
-    y = _targets(rng, wl)
+    rX, rU, rD, rHd, ry = _streams(wl.seed, 5)
+    X = rX.standard_normal((wl.T, wl.d))
+    W_up = rU.standard_normal((wl.d_ff, wl.d)) * (1.0 / np.sqrt(wl.d))
+    W_down = rD.standard_normal((wl.d, wl.d_ff)) * (1.0 / np.sqrt(wl.d_ff))
+    W_head = rHd.standard_normal((wl.V, wl.d)) * (1.0 / np.sqrt(wl.d))
+    y = _targets(ry, wl)
     return {"X": _cast(X, wl.dtype), "W_up": _cast(W_up, wl.dtype),
             "W_down": _cast(W_down, wl.dtype), "W_head": _cast(W_head, wl.dtype),
             "targets": y}

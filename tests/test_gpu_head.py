@@ -88,6 +88,9 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     dict(), dict(S=100), dict(S=1000), dict(S=1), dict(S=129, K=33), dict(T=1), dict(K=1),
     dict(K=1, S=3), dict(V=257, S=256), dict(V=5, S=2, d=3), dict(d=1), dict(sigma=0.2),
     dict(sigma=0.2, S=300), dict(dtype="f32"), dict(dtype="f32", S=77), dict(V=4099, S=640, K=40),
+    # fixed-point accumulation with a reduced scale (16384 < K <= 65536), and the
+    # fp32-atomic fallback (K > 65536)
+    dict(T=3, K=20000, S=32), dict(T=2, K=70000, S=64, V=700),
 ])
 def test_edge_shapes(ctx, kw):
     wl = _small(**kw)

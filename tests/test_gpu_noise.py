@@ -27,22 +27,24 @@ def test_philox_words_bit_exact(ctx):
         assert np.array_equal(got, np.stack(ref, axis=1))
 
 
+@pytest.mark.parametrize("table", [False, True])
 @pytest.mark.parametrize("tag,stream", [(oracle.TAG_HEAD, 0), (oracle.TAG_MLP_UP, 0), (oracle.TAG_HEAD, 77)])
-def test_gaussians_match_oracle(ctx, tag, stream):
+def test_gaussians_match_oracle(ctx, tag, stream, table):
     nt, ni, ns = 64, 96, 50304 // 24 + 5      # ragged slot count
     seed, t0, i0 = 1234567, 1000, 5000
     got = ctx.debug_gauss(nt, ni, ns, tag=tag, seed=seed, token_offset=t0, draw_offset=i0,
-                          stream_id=stream).cpu().numpy().astype(np.float64)
+                          stream_id=stream, table=table).cpu().numpy().astype(np.float64)
     ref = oracle.gaussians(seed, np.arange(nt)[:, None] + t0, np.arange(ni)[None, :] + i0,
                            np.arange(ns), tag, stream)
     err = np.abs(got - ref).max()
     assert err < TOL_GAUSS, err
 
 
-def test_gaussian_extremes_match_oracle(ctx):
+@pytest.mark.parametrize("table", [False, True])
+def test_gaussian_extremes_match_oracle(ctx, table):
     # many draws so that the tails (|eps| > 4.5) are exercised
     nt, ni, ns = 8, 4096, 512
-    got = ctx.debug_gauss(nt, ni, ns, seed=99).cpu().numpy().astype(np.float64)
+    got = ctx.debug_gauss(nt, ni, ns, seed=99, table=table).cpu().numpy().astype(np.float64)
     ref = oracle.gaussians(99, np.arange(nt)[:, None], np.arange(ni)[None, :], np.arange(ns), 0)
     assert np.abs(ref).max() > 4.5
     assert np.abs(got - ref).max() < TOL_GAUSS

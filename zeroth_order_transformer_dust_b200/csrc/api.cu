@@ -638,18 +638,28 @@ dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4
   return DUST_OK;
 }
 
-dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag, int64_t nt,
-                             int64_t ni, int64_t nslots, float* out) {
+static dust_status debug_gauss_impl(dust_ctx* ctx, const dust_params* p, int32_t tag, int64_t nt,
+                                    int64_t ni, int64_t nslots, float* out, int method) {
   if (!ctx) return DUST_ERR_ARG;
   if (!p || nt < 0 || ni < 0 || nslots < 0 || tag < 0 || tag > 255 || !out ||
       p->stream_id >= (1u << 24) || p->token_offset < 0 || p->draw_offset < 0 ||
       p->token_offset + nt > (1LL << 32) || p->draw_offset + ni > (1LL << 32))
     return fail(ctx, DUST_ERR_ARG, "bad gauss arguments");
   DUST_CU(cudaSetDevice(ctx->device));
-  DUST_CU(launch_debug_gauss(ctx->stream, *p, tag, nt, ni, nslots, out));
+  DUST_CU(launch_debug_gauss(ctx->stream, *p, tag, nt, ni, nslots, out, method));
   ctx->launches += 1;
   DUST_CU(cudaStreamSynchronize(ctx->stream));
   return DUST_OK;
+}
+
+dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag, int64_t nt,
+                             int64_t ni, int64_t nslots, float* out) {
+  return debug_gauss_impl(ctx, p, tag, nt, ni, nslots, out, 0);
+}
+
+dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t tag, int64_t nt,
+                                 int64_t ni, int64_t nslots, float* out) {
+  return debug_gauss_impl(ctx, p, tag, nt, ni, nslots, out, 1);
 }
 
 }  // extern "C"

@@ -137,8 +137,9 @@ namespace dust {
 // Kernel launchers (all enqueue on `st`, return cudaGetLastError()).
 cudaError_t launch_debug_philox(cudaStream_t st, uint64_t seed, const uint32_t* ctr, int64_t n,
                                 uint32_t* out);
+// method 0: polynomial angle step; 1: table-driven angle step (subset kernel).
 cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, int64_t nt,
-                               int64_t ni, int64_t nslots, float* out);
+                               int64_t ni, int64_t nslots, float* out, int method);
 
 cudaError_t launch_gemm_simt(cudaStream_t st, const GemmDesc& g, const EpiDesc& e);
 

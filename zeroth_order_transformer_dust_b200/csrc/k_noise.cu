@@ -50,16 +50,51 @@ __global__ void k_debug_gauss(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
   }
 }
 
+// Same with the table-driven angle step of the subset kernel; grid-stride so
+// that each CTA builds its table once.
+__global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off, uint32_t i_off,
+                                                         uint32_t ctr3, int64_t nt, int64_t ni,
+                                                         int64_t nslots, float* __restrict__ out) {
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab);
+  __syncthreads();
+  const int64_t nblk = (nslots + 127) / 128;
+  const int64_t total = nt * ni * nblk * 32;
+  for (int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t lane = (uint32_t)(gid & 31);
+    int64_t rest = gid >> 5;
+    const int64_t blk = rest % nblk;
+    rest /= nblk;
+    const int64_t i = rest % ni;
+    const int64_t t = rest / ni;
+    U4 c{slot_ctr0((uint32_t)blk, lane), t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3};
+    const G4 g = gauss4_tab(philox10(c, key.k0, key.k1), 1.0f, tab);
+    float* row = out + (t * ni + i) * nslots;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t k = blk * 128 + lane + 32 * j;
+      if (k < nslots) row[k] = g.v[j];
+    }
+  }
+}
+
 cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, int64_t nt,
-                               int64_t ni, int64_t nslots, float* out) {
+                               int64_t ni, int64_t nslots, float* out, int method) {
   const int64_t nblk = (nslots + 127) / 128;
   const int64_t total = nt * ni * nblk * 32;
   if (total <= 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
-  k_debug_gauss<<<(unsigned)blocks, threads, 0, st>>>(
-      key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
-      ctr3_of(tag, p.stream_id), nt, ni, nslots, out);
+  if (method == 1) {
+    k_debug_gauss_tab<<<(unsigned)(blocks < 2048 ? blocks : 2048), threads, 0, st>>>(
+        key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
+        ctr3_of(tag, p.stream_id), nt, ni, nslots, out);
+  } else {
+    k_debug_gauss<<<(unsigned)blocks, threads, 0, st>>>(
+        key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
+        ctr3_of(tag, p.stream_id), nt, ni, nslots, out);
+  }
   return cudaGetLastError();
 }
 

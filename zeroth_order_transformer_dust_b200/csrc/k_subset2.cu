@@ -22,6 +22,15 @@
 // sigma, kept in registers from the reward to the accumulation, and the
 // first two Philox rounds are evaluated once per draw and once per slot
 // block (they depend on the draw index or on the slot block only).
+//
+// Accumulation (INT = true): off-target coordinates accumulate r * sigma eps
+// in 2^-16 fixed point (scaled by 1/sigma^2) with native int32 shared-memory
+// atomics; sums wrap modulo 2^32, so only the final per-coordinate sum has to
+// fit, which holds with a wide margin for K <= 65536 (each term is bounded by
+// 66.6 and its mean by max_j p_j; the scale shrinks as 16384/K above 16384
+// draws). The target coordinate, which collects all K draws, keeps an fp32
+// accumulator per warp. INT = false accumulates in fp32 (compare-and-swap
+// atomics) for larger K.
 #include <cooperative_groups.h>
 
 #include "internal.cuh"
@@ -43,7 +52,10 @@ struct Sub2Args {
   int32_t K, S;
   uint32_t a, a_inv;
   uint32_t seg;  // q-slice length owned by one CTA (multiple of 4)
-  float scale_other, scale_target, fac;
+  float scale_other, scale_target;
+  float fac;        // g = fac * sum r * (sigma eps)            (fp32 accumulators)
+  float acc_scale;  // fixed-point units per unit of r * (sigma eps)
+  float fac_int;    // g = fac_int * fixed-point sum
   const float* Z;    // clean logits, permuted columns (T x V)
   const float* lse;  // T
   const int32_t* y;
@@ -106,11 +118,23 @@ __device__ __forceinline__ U4 philox_from2(const BlockConst& bc, const DrawConst
   return c;
 }
 
+template <bool INT>
+__device__ __forceinline__ void accumulate(float* slot, float r, float x, float acc_scale) {
+  if (INT)
+    atomicAdd(reinterpret_cast<int*>(slot), __float2int_rn(r * acc_scale * x));
+  else
+    atomicAdd(slot, r * x);
+}
+
 // NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
-template <int CS, int NB, bool FULL, int DEG>
+template <int CS, int NB, bool FULL, int DEG, bool INT>
 __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__ Sub2Args A) {
   extern __shared__ __align__(16) float smem[];
-  __shared__ int s_next;  // next draw batch of the current token
+  __shared__ int s_next;    // next draw batch of the current token
+  __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
+  __shared__ float2 s_tab[kSinCosTable];
+  fill_sincos_table(s_tab);
+  __syncthreads();
   cg::cluster_group cluster = cg::this_cluster();
   const uint32_t rank = CS > 1 ? cluster.block_rank() : 0;
   const int lane = threadIdx.x & 31;
@@ -121,12 +145,14 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
   const uint32_t n_own = hi - lo;
   const uint32_t lo_peer = lo ^ seg;  // CS = 2: the partner's slice start
   float* sp = smem;        // p of q in [lo, hi)
-  float* sg = smem + seg;  // g accumulator of q in [lo, hi)
+  float* sg = smem + seg;  // g accumulator of q in [lo, hi) (fp32 or int32 fixed point)
   float* sp_peer = sp;
   float* sg_peer = sg;
+  float* tgt_peer = &s_tgt;
   if (CS > 1) {
     sp_peer = cluster.map_shared_rank(sp, rank ^ 1u);
     sg_peer = cluster.map_shared_rank(sg, rank ^ 1u);
+    tgt_peer = cluster.map_shared_rank(&s_tgt, rank ^ 1u);
   }
   const int S = A.S;
   const uint32_t nclusters = gridDim.x / CS;
@@ -158,15 +184,20 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         }
       }
     }
-    if (threadIdx.x == 0) s_next = 0;
+    if (threadIdx.x == 0) {
+      s_next = 0;
+      s_tgt = 0.0f;
+    }
     int32_t yt = A.y[t];
     if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
     const uint32_t qy = mulmod32((uint32_t)yt, A.a_inv, V);
+    const bool own_y = qy >= lo && qy < hi;
     const float py = expf(zrow[qy] - lse_t);
-    float* gy = (qy >= lo && qy < hi) ? sg + (qy - lo) : sg_peer + (qy - lo_peer);
+    float* gy = own_y ? sg + (qy - lo) : sg_peer + (qy - lo_peer);
     if (CS > 1) cluster.sync(); else __syncthreads();
 
     const uint32_t t_abs = A.t_off + (uint32_t)t;
+    float tgt_acc = 0.0f;  // INT: this warp's sum r * (sigma eps_y), lane 0
     for (;;) {
       int bidx = 0;
       if (lane == 0) bidx = atomicAdd(&s_next, 1);
@@ -185,7 +216,8 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         kyq = (qy >= c) ? qy - c : qy + V - c;
         if (mine && kyq >= (uint32_t)S) {
           const U4 w = philox_from2(bs, draw_const(A, t_abs, i_abs), A);
-          const float2 nn = box_muller(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, A.sigma);
+          const float2 nn =
+              box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, A.sigma, s_tab);
           x_extra = (s_word & 1u) ? nn.y : nn.x;
         }
       }
@@ -214,7 +246,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
             }
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4(philox_from2(bc[m], dc, A), A.sigma);
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A), A.sigma, s_tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
@@ -226,7 +258,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         } else {
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4(philox_from2(bc[m], dc, A), A.sigma);
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A), A.sigma, s_tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
@@ -245,12 +277,17 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         float xy;
         if (in_win) {
           const int my = (int)(ky >> 7), jy = (int)((ky >> 5) & 3u);
+          const bool owner = lane == (int)(ky & 31u);
           float cand = 0.0f;
 #pragma unroll
           for (int m = 0; m < NB; ++m)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              if (m == my && j == jy) cand = n[m][j];
+              if (m == my && j == jy) {
+                cand = n[m][j];
+                // INT: the target coordinate is accumulated in fp32 below
+                if (INT && owner) n[m][j] = 0.0f;
+              }
           xy = __shfl_sync(0xffffffffu, cand, (int)(ky & 31u));
         } else {
           xy = xe;
@@ -266,7 +303,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
-              if (FULL || k < S) atomicAdd(gw + m * 128 + 32 * j, r * n[m][j]);
+              if (FULL || k < S) accumulate<INT>(gw + m * 128 + 32 * j, r, n[m][j], A.acc_scale);
             }
         } else {
 #pragma unroll
@@ -278,19 +315,29 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
                 uint32_t q = cw + (uint32_t)k;
                 if (q >= V) q -= V;
                 float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - lo_peer);
-                atomicAdd(dst, r * n[m][j]);
+                accumulate<INT>(dst, r, n[m][j], A.acc_scale);
               }
             }
         }
-        if (!in_win && lane == 0) atomicAdd(gy, r * xy);
+        if (INT) {
+          if (lane == 0) tgt_acc = fmaf(r, xy, tgt_acc);
+        } else if (!in_win && lane == 0) {
+          atomicAdd(gy, r * xy);
+        }
       }
     }
+    if (INT && lane == 0) atomicAdd(own_y ? &s_tgt : tgt_peer, tgt_acc);
     if (CS > 1) cluster.sync(); else __syncthreads();
 
-    // ---- scale and write the owned slice of g (accumulated as sum r * sigma eps)
+    // ---- scale and write the owned slice of g
     for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
       const uint32_t qg = lo + q;
-      const float v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
+      float v;
+      if (INT)
+        v = (qg == qy) ? s_tgt * A.fac * A.scale_target
+                       : (float)reinterpret_cast<const int*>(sg)[q] * A.fac_int * A.scale_other;
+      else
+        v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
       if (A.gop_bf16)
         store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + qg, v);
       else
@@ -309,9 +356,9 @@ int expm1_degree2(float sigma) {
   return 0;
 }
 
-template <int CS, int NB, bool FULL, int DEG>
+template <int CS, int NB, bool FULL, int DEG, bool INT>
 cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_count) {
-  auto fn = k_subset2<CS, NB, FULL, DEG>;
+  auto fn = k_subset2<CS, NB, FULL, DEG, INT>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -338,24 +385,29 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
   return cudaGetLastError();
 }
 
-template <int CS, int NB, bool FULL>
+template <int CS, int NB, bool FULL, bool INT>
 cudaError_t launch_deg(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
-  if (deg == 4) return launch_one<CS, NB, FULL, 4>(st, A, smem, sm);
-  if (deg == 5) return launch_one<CS, NB, FULL, 5>(st, A, smem, sm);
-  return launch_one<CS, NB, FULL, 0>(st, A, smem, sm);
+  if (deg == 4) return launch_one<CS, NB, FULL, 4, INT>(st, A, smem, sm);
+  if (deg == 5) return launch_one<CS, NB, FULL, 5, INT>(st, A, smem, sm);
+  return launch_one<CS, NB, FULL, 0, INT>(st, A, smem, sm);
 }
 
-template <int CS>
-cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
+template <int CS, bool INT>
+cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
   const int nb = (A.S + 127) / 128;
   const bool full = (A.S % 128) == 0;
   switch (nb) {
-    case 1: return full ? launch_deg<CS, 1, true>(st, A, smem, sm, deg) : launch_deg<CS, 1, false>(st, A, smem, sm, deg);
-    case 2: return full ? launch_deg<CS, 2, true>(st, A, smem, sm, deg) : launch_deg<CS, 2, false>(st, A, smem, sm, deg);
-    case 3: return launch_deg<CS, 3, false>(st, A, smem, sm, deg);
-    case 4: return full ? launch_deg<CS, 4, true>(st, A, smem, sm, deg) : launch_deg<CS, 4, false>(st, A, smem, sm, deg);
+    case 1: return full ? launch_deg<CS, 1, true, INT>(st, A, smem, sm, deg) : launch_deg<CS, 1, false, INT>(st, A, smem, sm, deg);
+    case 2: return full ? launch_deg<CS, 2, true, INT>(st, A, smem, sm, deg) : launch_deg<CS, 2, false, INT>(st, A, smem, sm, deg);
+    case 3: return launch_deg<CS, 3, false, INT>(st, A, smem, sm, deg);
+    case 4: return full ? launch_deg<CS, 4, true, INT>(st, A, smem, sm, deg) : launch_deg<CS, 4, false, INT>(st, A, smem, sm, deg);
     default: return cudaErrorNotSupported;
   }
+}
+
+template <int CS>
+cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg, bool use_int) {
+  return use_int ? launch_nb<CS, true>(st, A, smem, sm, deg) : launch_nb<CS, false>(st, A, smem, sm, deg);
 }
 
 }  // namespace
@@ -363,7 +415,7 @@ cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, i
 // Cluster size the shared-memory kernel would use (0: not applicable).
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
   if (S < 1 || S > 512) return 0;
-  const int64_t slack = 1024;
+  const int64_t slack = 1024 + 8 * kSinCosTable;  // static: counters, angle table
   if (2 * V * 4 + slack <= max_smem_optin && V <= 65536) return 1;
   const int64_t seg = ((V + 1) / 2 + 3) / 4 * 4;
   if (2 * seg * 4 + slack <= max_smem_optin && S <= V - seg && S <= seg) return 2;
@@ -395,8 +447,13 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.seg = cs == 1 ? (uint32_t)((p.V + 3) / 4 * 4) : (uint32_t)(((p.V + 1) / 2 + 3) / 4 * 4);
   A.scale_other = (float)((double)p.V / (double)p.S);
   A.scale_target = (p.flags & DUST_FLAG_LITERAL_TARGET_SCALE) ? A.scale_other : 1.0f;
-  // the accumulator holds sum r (sigma eps): g = -(1/(K sigma)) sum r eps
-  A.fac = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * (double)p.sigma * (double)p.sigma)) : 0.0f;
+  // the accumulators hold sum r (sigma eps): g = -(1/(K sigma)) sum r eps
+  const double s2 = (double)p.sigma * (double)p.sigma;
+  A.fac = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * s2)) : 0.0f;
+  // fixed point: 2^16 units per unit of r eps / sigma, fewer above 16384 draws
+  const double units = 65536.0 * (p.K > 16384 ? 16384.0 / (double)p.K : 1.0);
+  A.acc_scale = p.sigma > 0.0f ? (float)(units / s2) : 0.0f;
+  A.fac_int = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * units)) : 0.0f;
   A.Z = Z;
   A.lse = lse;
   A.y = y;
@@ -407,8 +464,9 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.plane = p.T * p.V;
   const size_t smem = (size_t)2 * A.seg * 4;
   const int deg = expm1_degree2(p.sigma);
-  if (cs == 1) return launch_cs<1>(st, A, smem, sm_count, deg);
-  return launch_cs<2>(st, A, smem, sm_count, deg);
+  const bool use_int = p.K <= 65536;
+  if (cs == 1) return launch_cs<1>(st, A, smem, sm_count, deg, use_int);
+  return launch_cs<2>(st, A, smem, sm_count, deg, use_int);
 }
 
 }  // namespace dust

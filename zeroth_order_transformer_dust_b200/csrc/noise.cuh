@@ -125,10 +125,56 @@ __device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb, float sca
   return make_float2(radius * c, radius * s);
 }
 
+// Table-driven variant of the angle step, for kernels that keep a 1024-entry
+// table of roots of unity, tab[k] = (cos 2 pi k/1024, sin 2 pi k/1024), in
+// shared memory: the angle 2 pi m 2^-24 is split into the nearest table angle
+// plus a remainder |x| <= pi/1024, and cos/sin follow from the angle-addition
+// formulas with cos x = 1 - x^2/2 and sin x = x (truncation below 5e-9).
+constexpr int kSinCosTable = 1024;
+
+__device__ __forceinline__ void fill_sincos_table(float2* tab) {
+  for (int k = threadIdx.x; k < kSinCosTable; k += blockDim.x) {
+    float s, c;
+    sincospif((float)k * (2.0f / kSinCosTable), &s, &c);
+    tab[k] = make_float2(c, s);
+  }
+}
+
+__device__ __forceinline__ void sincos_turn24_tab(uint32_t m, const float2* tab, float* s_out,
+                                                  float* c_out) {
+  const uint32_t idx = (m + (1u << 13)) >> 14;             // nearest 1/1024 turn, 0..1024
+  const int r = (int)m - (int)(idx << 14);                  // [-2^13, 2^13)
+  const float x = (float)r * 3.7450702e-07f;                // 2 pi / 2^24
+  const float h = 0.5f * x * x;
+  const float2 t = tab[idx & (kSinCosTable - 1)];
+  *c_out = fmaf(-t.y, x, fmaf(-t.x, h, t.x));
+  *s_out = fmaf(t.x, x, fmaf(-t.y, h, t.y));
+}
+
+__device__ __forceinline__ float2 box_muller_tab(uint32_t wa, uint32_t wb, float scale,
+                                                 const float2* tab) {
+  const float u1 = (float)((wa >> 8) + 1u) * 5.9604645e-08f;  // exact
+  const float radius = scale * sqrt_newton(2.0f * neg_log_unit(u1));
+  float s, c;
+  sincos_turn24_tab(wb >> 8, tab, &s, &c);
+  return make_float2(radius * c, radius * s);
+}
+
 // Four Gaussians of one counter (times `scale`): element j is output word j.
 struct G4 {
   float v[4];
 };
+
+__device__ __forceinline__ G4 gauss4_tab(U4 w, float scale, const float2* tab) {
+  const float2 a = box_muller_tab(w.x, w.y, scale, tab);
+  const float2 b = box_muller_tab(w.z, w.w, scale, tab);
+  G4 g;
+  g.v[0] = a.x;
+  g.v[1] = a.y;
+  g.v[2] = b.x;
+  g.v[3] = b.y;
+  return g;
+}
 
 __device__ __forceinline__ G4 gauss4(U4 w, float scale = 1.0f) {
   const float2 a = box_muller(w.x, w.y, scale);
