@@ -11,9 +11,11 @@ selects another one.
 
 Rank 0 prints one JSON line. Under torchrun (N > 1) each rank runs its own
 token shard (token_offset = rank * T, so the noise is that of one N*T-token
-run) with no collective on the data path: weak scaling, value = all ranks'
-token-draws / the slowest rank's time. ``--impl reference`` times the CPU
-oracle on a bounded sample of the same workload.
+run) and the step ends with the one exchange the path has, a sum all-reduce
+of G_W over NCCL: weak scaling, value = all ranks' token-draws / the slowest
+rank's time. ``--impl reference`` times the CPU oracle on a bounded sample
+of the same workload. ``--tokens N`` cuts the workload to its first N tokens
+(profiling slices).
 """
 from __future__ import annotations
 
@@ -258,9 +260,12 @@ def run_dust(args):
         outs = {"G": torch.empty(wl.V, wl.d, dtype=torch.float32, device=dev),
                 "loss": torch.empty(wl.T, dtype=torch.float32, device=dev)}
 
+        from zeroth_order_transformer_dust_b200.parallel import allreduce_weight_grad
+
         def step():
             ctx.head_grad(Hd, Wd, yd, K=wl.K, sigma=wl.sigma, S=wl.S, seed=wl.seed,
                           token_offset=t_off, out=outs, asynchronous=True)
+            allreduce_weight_grad(outs["G"])   # G_W of all ranks' tokens (no-op at N = 1)
     else:
         inp = synth.make_mlp_inputs(wl)
         X, Wu, Wdn, Wh = (torch.from_numpy(inp[k]).to(torch.bfloat16).to(dev)
@@ -272,6 +277,8 @@ def run_dust(args):
         def step():
             ctx.mlp_grad(X, Wu, Wdn, Wh, yd, K=wl.K, sigma=wl.sigma, seed=wl.seed,
                          token_offset=t_off, out=outs)
+            from zeroth_order_transformer_dust_b200.parallel import allreduce_weight_grad
+            allreduce_weight_grad(outs["G"])
 
     # L2 flush buffer (larger than the 126 MB L2), written between timed steps
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -361,7 +368,8 @@ def run_dust(args):
                 "config": {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V,
                            "K": wl.K, "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype,
                            "d_ff": wl.d_ff, "l2": "flushed between timed steps (256 MiB write)",
-                           "parallelism": f"token-sharded x{world}, no collective"},
+                           "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL "
+                                           "all-reduce" if world > 1 else "dp1")},
                 "stage_ms": stages, "gpu_launches": launches, "e2e": e2e, "roofline": roof,
                 "cpu_baseline": cb, "clocks": clk, **extra}
         print(json.dumps(line), flush=True)

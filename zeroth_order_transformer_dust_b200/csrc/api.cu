@@ -367,8 +367,9 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
       r = (float*)ctx->rew.p;
     }
     DUST_TRY(ensure(ctx, ctx->part, (size_t)p.T * full_vocab_nslab(p.V) * p.K * 4));
-    DUST_CU(launch_full_reward_partial(st, p, Z, (float*)ctx->part.p));
-    DUST_CU(launch_full_reward_combine(st, p, (float*)ctx->part.p, targets, r));
+    DUST_TRY(ensure(ctx, ctx->dzy, full_vocab_xy_bytes(p.T, p.K)));
+    DUST_CU(launch_full_reward_partial(st, p, Z, targets, (float*)ctx->part.p, (float*)ctx->dzy.p));
+    DUST_CU(launch_full_reward_combine(st, p, (float*)ctx->part.p, (float*)ctx->dzy.p, r));
     ctx->launches += 2;
     mark(ctx, "reward");
     DUST_CU(launch_full_g(st, p, r, g_out, ctx->gop.p));

@@ -151,13 +151,15 @@ cudaError_t launch_lse_rows(cudaStream_t st, float* Z, int64_t T, int64_t V, con
                             uint32_t* status);
 
 // Full-vocabulary reward, stage 1: partial sums sum_j p_j expm1(sigma eps_j) per
-// (token, slab, draw) -> part[(t * nslab + slab) * K + i]. Returns nslab.
+// (token, slab, draw) -> part[(t * nslab + slab) * K + i], and sigma eps at the
+// target -> xy[t * K + i] (T x K floats, full_vocab_xy_bytes).
 int full_vocab_nslab(int64_t V);
+size_t full_vocab_xy_bytes(int64_t T, int32_t K);
 cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* P,
-                                       float* part);
-// Stage 2: r[t*K + i] = sigma eps_y - log1p(sum_slab part).
+                                       const int32_t* y, float* part, float* xy);
+// Stage 2: r[t*K + i] = xy - log1p(sum_slab part).
 cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, const float* part,
-                                       const int32_t* y, float* r);
+                                       const float* xy, float* r);
 // Stage 3: g_t = -(1/(K sigma)) sum_i r_i eps_i; writes g (fp32, optional) and the
 // GEMM operand gop (bf16 or fp32 by p.dtype).
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,

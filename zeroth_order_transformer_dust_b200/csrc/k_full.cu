@@ -5,6 +5,13 @@
 // the reward is r = L - L', and g_t = -(1/(K sigma)) sum_i r_i eps_i.
 // The reward needs the whole row before any g entry can be formed, so the
 // noise is generated twice (stage 1 and stage 3); it never reaches memory.
+//
+// Both noise passes are persistent over (token, 4096-entry slab) units: a warp
+// owns four 128-slot blocks of the slab, evaluates Philox rounds 0-1 of its
+// blocks once per unit and those of each draw once per draw, and turns words
+// into sigma-scaled Gaussians with the table-driven Box-Muller step (the
+// table of roots of unity is built once per CTA). Stage 1 also records the
+// target's noise, so stage 2 needs none of its own.
 #include "internal.cuh"
 #include "noise.cuh"
 
@@ -13,8 +20,27 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kBlocksPerWarp = 4;                     // 128-slot blocks per warp
-constexpr int kSlab = kWarps * kBlocksPerWarp * 128;  // vocabulary entries per CTA
+constexpr int kSlab = kWarps * kBlocksPerWarp * 128;  // vocabulary entries per unit
 constexpr int kDrawChunk = 64;
+
+struct FullArgs {
+  RoundKeys keys;
+  uint32_t t_off, i_off, ctr3;
+  float sigma;
+  float fac;  // g = fac * sum_i r_i (sigma eps_i)
+  int64_t T, V;
+  int32_t K;
+  int nslab;
+  const float* P;
+  const int32_t* y;
+  float* part;       // (t * nslab + slab) * K + i
+  float* xy;         // sigma eps at the target, t * K + i
+  const float* r;    // rewards, t * K + i
+  float* g_out;
+  void* gop;
+  int gop_bf16;
+  int64_t plane;
+};
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -23,171 +49,213 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 template <int DEG>
-__global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(
-    Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3, float sigma, int64_t V, int32_t K,
-    int nslab, const float* __restrict__ P, float* __restrict__ part) {
+__global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __grid_constant__ FullArgs A) {
   __shared__ float sh[kWarps][kDrawChunk];
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab);
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t t = blockIdx.x;
-  const int slab = blockIdx.y;
-  const int64_t blk0 = (int64_t)slab * (kSlab / 128) + warp * kBlocksPerWarp;
-  float pv[kBlocksPerWarp][4];
+  const int64_t nunits = A.T * A.nslab;
+  for (int64_t unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
+    const int64_t t = unit / A.nslab;
+    const int slab = (int)(unit % A.nslab);
+    const int64_t blk0 = (int64_t)slab * (kSlab / 128) + warp * kBlocksPerWarp;
+    float pv[kBlocksPerWarp][4];
+    BlockConst bc[kBlocksPerWarp];
 #pragma unroll
-  for (int b = 0; b < kBlocksPerWarp; ++b)
+    for (int b = 0; b < kBlocksPerWarp; ++b) {
+      bc[b] = block_const(A.keys, slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), A.ctr3);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
-      pv[b][j] = pos < V ? P[t * V + pos] : 0.0f;
-    }
-  const uint32_t t_abs = t_off + (uint32_t)t;
-  for (int i0 = 0; i0 < K; i0 += kDrawChunk) {
-    const int n = min(kDrawChunk, K - i0);
-    for (int ii = 0; ii < n; ++ii) {
-      const uint32_t i_abs = i_off + (uint32_t)(i0 + ii);
-      float s = 0.0f;
-#pragma unroll
-      for (int b = 0; b < kBlocksPerWarp; ++b) {
-        if ((blk0 + b) * 128 < V) {
-          U4 c{slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), t_abs, i_abs, ctr3};
-          const G4 g = gauss4(philox10(c, key.k0, key.k1));
-#pragma unroll
-          for (int j = 0; j < 4; ++j) s = fmaf(pv[b][j], expm1_small<DEG>(sigma * g.v[j]), s);
-        }
+      for (int j = 0; j < 4; ++j) {
+        const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
+        pv[b][j] = pos < A.V ? A.P[t * A.V + pos] : 0.0f;
       }
-      s = warp_sum(s);
-      if (lane == 0) sh[warp][ii] = s;
     }
-    __syncthreads();
-    if ((int)threadIdx.x < n) {
-      float s = 0.0f;
+    // the lane holding the target's noise, if this warp's blocks contain it
+    int32_t yt = A.y[t];
+    if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
+    const int64_t yb = (int64_t)yt >> 7;
+    const bool warp_has_y = yb >= blk0 && yb < blk0 + kBlocksPerWarp;  // warp-uniform
+    const bool y_here = warp_has_y && lane == (yt & 31);
+    const int by = (int)(yb - blk0), jy = (yt >> 5) & 3;
+    const uint32_t t_abs = A.t_off + (uint32_t)t;
+    for (int i0 = 0; i0 < A.K; i0 += kDrawChunk) {
+      const int n = min(kDrawChunk, A.K - i0);
+      for (int ii = 0; ii < n; ++ii) {
+        const uint32_t i_abs = A.i_off + (uint32_t)(i0 + ii);
+        const DrawConst dc = draw_const(A.keys, t_abs, i_abs);
+        float s = 0.0f, xyv = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) s += sh[w][threadIdx.x];
-      part[(t * nslab + slab) * (int64_t)K + i0 + threadIdx.x] = s;
+        for (int b = 0; b < kBlocksPerWarp; ++b) {
+          if ((blk0 + b) * 128 < A.V) {
+            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), A.sigma, tab);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s = fmaf(pv[b][j], expm1_small<DEG>(g.v[j]), s);
+            if (warp_has_y) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (b == by && j == jy) xyv = g.v[j];
+            }
+          }
+        }
+        if (y_here) A.xy[t * A.K + i0 + ii] = xyv;
+        s = warp_sum(s);
+        if (lane == 0) sh[warp][ii] = s;
+      }
+      __syncthreads();
+      if ((int)threadIdx.x < n) {
+        float s = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += sh[w][threadIdx.x];
+        A.part[(t * A.nslab + slab) * (int64_t)A.K + i0 + threadIdx.x] = s;
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
 }
 
-__global__ void k_full_reward_combine(Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3,
-                                      float sigma, int64_t T, int64_t V, int32_t K, int nslab,
+__global__ void k_full_reward_combine(int64_t T, int32_t K, int nslab,
                                       const float* __restrict__ part,
-                                      const int32_t* __restrict__ y, float* __restrict__ r) {
+                                      const float* __restrict__ xy, float* __restrict__ r) {
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= T * K) return;
   const int64_t t = id / K;
   const int32_t i = (int32_t)(id % K);
   float s = 0.0f;
   for (int sl = 0; sl < nslab; ++sl) s += part[(t * nslab + sl) * (int64_t)K + i];
-  int32_t yt = y[t];
-  if (yt < 0 || (int64_t)yt >= V) yt = 0;  // reported by the loss kernel
-  const float ey = gauss_slot(key, t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3, (uint32_t)yt);
-  r[id] = sigma * ey - log1pf(s);
+  r[id] = xy[id] - log1pf(s);
 }
 
-template <typename TO>
-__global__ __launch_bounds__(kWarps * 32) void k_full_g(Key key, uint32_t t_off, uint32_t i_off,
-                                                        uint32_t ctr3, float scale, int64_t V,
-                                                        int32_t K, const float* __restrict__ r,
-                                                        float* __restrict__ g_out,
-                                                        TO* __restrict__ gop, int64_t plane) {
+__global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ FullArgs A) {
   __shared__ float rs[1024];
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab);
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t t = blockIdx.x;
-  const int64_t blk0 = (int64_t)blockIdx.y * (kSlab / 128) + warp * kBlocksPerWarp;
-  const uint32_t t_abs = t_off + (uint32_t)t;
-  float acc[kBlocksPerWarp][4];
+  const int64_t nunits = A.T * A.nslab;
+  for (int64_t unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
+    const int64_t t = unit / A.nslab;
+    const int slab = (int)(unit % A.nslab);
+    const int64_t blk0 = (int64_t)slab * (kSlab / 128) + warp * kBlocksPerWarp;
+    const uint32_t t_abs = A.t_off + (uint32_t)t;
+    BlockConst bc[kBlocksPerWarp];
+    float acc[kBlocksPerWarp][4];
 #pragma unroll
-  for (int b = 0; b < kBlocksPerWarp; ++b)
+    for (int b = 0; b < kBlocksPerWarp; ++b) {
+      bc[b] = block_const(A.keys, slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), A.ctr3);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[b][j] = 0.0f;
-  for (int i0 = 0; i0 < K; i0 += 1024) {
-    const int n = min(1024, K - i0);
-    __syncthreads();
-    for (int q = threadIdx.x; q < n; q += blockDim.x) rs[q] = r[t * K + i0 + q];
-    __syncthreads();
-    for (int ii = 0; ii < n; ++ii) {
-      const float ri = rs[ii];
-      const uint32_t i_abs = i_off + (uint32_t)(i0 + ii);
+      for (int j = 0; j < 4; ++j) acc[b][j] = 0.0f;
+    }
+    for (int i0 = 0; i0 < A.K; i0 += 1024) {
+      const int n = min(1024, A.K - i0);
+      __syncthreads();
+      for (int q = threadIdx.x; q < n; q += blockDim.x) rs[q] = A.r[t * A.K + i0 + q];
+      __syncthreads();
+      for (int ii = 0; ii < n; ++ii) {
+        const float ri = rs[ii];
+        const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)(i0 + ii));
 #pragma unroll
-      for (int b = 0; b < kBlocksPerWarp; ++b) {
-        if ((blk0 + b) * 128 < V) {
-          U4 c{slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), t_abs, i_abs, ctr3};
-          const G4 g = gauss4(philox10(c, key.k0, key.k1));
+        for (int b = 0; b < kBlocksPerWarp; ++b) {
+          if ((blk0 + b) * 128 < A.V) {
+            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), A.sigma, tab);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(ri, g.v[j], acc[b][j]);
+            for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(ri, g.v[j], acc[b][j]);
+          }
         }
       }
     }
-  }
 #pragma unroll
-  for (int b = 0; b < kBlocksPerWarp; ++b)
+    for (int b = 0; b < kBlocksPerWarp; ++b)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
-      if (pos < V) {
-        const float v = acc[b][j] * scale;
-        if (g_out) g_out[t * V + pos] = v;
-        store_g_operand(gop, plane, t * V + pos, v);
+      for (int j = 0; j < 4; ++j) {
+        const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
+        if (pos < A.V) {
+          const float v = acc[b][j] * A.fac;
+          if (A.g_out) A.g_out[t * A.V + pos] = v;
+          if (A.gop_bf16)
+            store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + pos, v);
+          else
+            ((float*)A.gop)[t * A.V + pos] = v;
+        }
       }
-    }
+  }
 }
 
-int expm1_degree(float sigma) {
-  const float xmax = sigma * 5.7686f;  // |eps| <= sqrt(48 ln 2)
-  if (xmax <= 0.03f) return 4;
-  if (xmax <= 0.06f) return 5;
-  return 0;
+FullArgs make_args(const dust_params& p) {
+  FullArgs A{};
+  A.keys = round_keys(p.seed);
+  A.t_off = (uint32_t)p.token_offset;
+  A.i_off = (uint32_t)p.draw_offset;
+  A.ctr3 = ctr3_of(kTagHead, p.stream_id);
+  A.sigma = p.sigma;
+  const double s2 = (double)p.sigma * (double)p.sigma;
+  A.fac = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * s2)) : 0.0f;
+  A.T = p.T;
+  A.V = p.V;
+  A.K = p.K;
+  A.nslab = (int)((p.V + kSlab - 1) / kSlab);
+  A.gop_bf16 = p.dtype == DUST_BF16;
+  A.plane = p.T * p.V;
+  return A;
+}
+
+// Persistent grid: every SM filled with as many CTAs as fit, at most one per unit.
+template <typename F>
+int grid_for(F kernel, int64_t units) {
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWarps * 32, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  cudaGetLastError();
+  const int64_t g = (int64_t)sms * per_sm;
+  return (int)(units < g ? units : g);
 }
 
 }  // namespace
 
 int full_vocab_nslab(int64_t V) { return (int)((V + kSlab - 1) / kSlab); }
 
+size_t full_vocab_xy_bytes(int64_t T, int32_t K) { return (size_t)T * K * 4; }
+
 cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* P,
-                                       float* part) {
-  const int nslab = full_vocab_nslab(p.V);
-  dim3 grid((unsigned)p.T, (unsigned)nslab);
-  const Key key = key_of(p.seed);
-  const uint32_t c3 = ctr3_of(kTagHead, p.stream_id);
+                                       const int32_t* y, float* part, float* xy) {
+  FullArgs A = make_args(p);
+  A.P = P;
+  A.y = y;
+  A.part = part;
+  A.xy = xy;
+  const int64_t units = A.T * A.nslab;
   switch (expm1_degree(p.sigma)) {
-    case 4:
-      k_full_reward_partial<4><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-          (uint32_t)p.draw_offset, c3, p.sigma, p.V, p.K, nslab, P, part);
+    case 3:
+      k_full_reward_partial<3><<<grid_for(k_full_reward_partial<3>, units), kWarps * 32, 0, st>>>(A);
       break;
-    case 5:
-      k_full_reward_partial<5><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-          (uint32_t)p.draw_offset, c3, p.sigma, p.V, p.K, nslab, P, part);
+    case 4:
+      k_full_reward_partial<4><<<grid_for(k_full_reward_partial<4>, units), kWarps * 32, 0, st>>>(A);
       break;
     default:
-      k_full_reward_partial<0><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-          (uint32_t)p.draw_offset, c3, p.sigma, p.V, p.K, nslab, P, part);
+      k_full_reward_partial<0><<<grid_for(k_full_reward_partial<0>, units), kWarps * 32, 0, st>>>(A);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, const float* part,
-                                       const int32_t* y, float* r) {
+                                       const float* xy, float* r) {
   const int64_t n = p.T * (int64_t)p.K;
   const int threads = 256;
   k_full_reward_combine<<<(unsigned)((n + threads - 1) / threads), threads, 0, st>>>(
-      key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
-      ctr3_of(kTagHead, p.stream_id), p.sigma, p.T, p.V, p.K, full_vocab_nslab(p.V), part, y, r);
+      p.T, p.K, full_vocab_nslab(p.V), part, xy, r);
   return cudaGetLastError();
 }
 
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
                           void* gop) {
-  dim3 grid((unsigned)p.T, (unsigned)full_vocab_nslab(p.V));
-  const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
-  const Key key = key_of(p.seed);
-  const uint32_t c3 = ctr3_of(kTagHead, p.stream_id);
-  const int64_t plane = p.T * p.V;
-  if (p.dtype == DUST_BF16)
-    k_full_g<__nv_bfloat16><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.V, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
-  else
-    k_full_g<float><<<grid, kWarps * 32, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.V, p.K, r, g_out, (float*)gop, plane);
+  FullArgs A = make_args(p);
+  A.r = r;
+  A.g_out = g_out;
+  A.gop = gop;
+  k_full_g<<<grid_for(k_full_g, A.T * A.nslab), kWarps * 32, 0, st>>>(A);
   return cudaGetLastError();
 }
 

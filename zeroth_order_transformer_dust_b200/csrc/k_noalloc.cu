@@ -132,6 +132,7 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   if (!subset) {
     if (!rewards_out) add(T * K * 4);
     add(T * (size_t)nslab * K * 4);                      // reward partial sums
+    add(full_vocab_xy_bytes(p.T, p.K));                  // noise at the target
   } else {
     add(subset_gacc_bytes(p.T, p.V, max_smem));
   }
@@ -152,10 +153,12 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   float* loss = loss_out ? loss_out : (float*)cv.take(T * 4);
   float* r = nullptr;
   float* part = nullptr;
+  float* xy = nullptr;
   float* gacc = nullptr;
   if (!subset) {
     r = rewards_out ? rewards_out : (float*)cv.take(T * K * 4);
     part = (float*)cv.take(T * (size_t)nslab * K * 4);
+    xy = (float*)cv.take(full_vocab_xy_bytes(p.T, p.K));
   } else {
     const size_t gb = subset_gacc_bytes(p.T, p.V, max_smem);
     if (gb) gacc = (float*)cv.take(gb);
@@ -185,8 +188,8 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   if (e == cudaSuccess)
     e = launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, lse, loss, true, status);
   if (!subset) {
-    if (e == cudaSuccess) e = launch_full_reward_partial(st, p, Z, part);
-    if (e == cudaSuccess) e = launch_full_reward_combine(st, p, part, targets, r);
+    if (e == cudaSuccess) e = launch_full_reward_partial(st, p, Z, targets, part, xy);
+    if (e == cudaSuccess) e = launch_full_reward_combine(st, p, part, xy, r);
     if (e == cudaSuccess) e = launch_full_g(st, p, r, g_out, gop);
   } else if (e == cudaSuccess) {
     e = launch_subset_impl(st, p, a, a_inv, Z, targets, rewards_out, g_out, gop, gacc, max_smem);

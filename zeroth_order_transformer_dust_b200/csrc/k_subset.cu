@@ -174,18 +174,11 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset(SubsetArgs A) {
   }
 }
 
-int expm1_degree(float sigma) {
-  const float xmax = sigma * 5.7686f;
-  if (xmax <= 0.03f) return 4;
-  if (xmax <= 0.06f) return 5;
-  return 0;
-}
-
 template <int NB, bool GSMEM>
 cudaError_t launch_nb(cudaStream_t st, const SubsetArgs& A, int64_t T, size_t smem, int deg) {
   void (*fn)(SubsetArgs);
-  if (deg == 4) fn = k_subset<NB, 4, GSMEM>;
-  else if (deg == 5) fn = k_subset<NB, 5, GSMEM>;
+  if (deg == 3) fn = k_subset<NB, 3, GSMEM>;
+  else if (deg == 4) fn = k_subset<NB, 4, GSMEM>;
   else fn = k_subset<NB, 0, GSMEM>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

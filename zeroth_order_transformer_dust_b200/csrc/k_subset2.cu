@@ -45,7 +45,7 @@ constexpr int kThreads = 512;
 
 struct Sub2Args {
   Key key;
-  uint32_t rk0[10], rk1[10];  // round keys k + r (0x9E3779B9, 0xBB67AE85)
+  RoundKeys keys;
   uint32_t t_off, i_off, ctr3, stream_id;
   float sigma;
   int64_t T, V;
@@ -74,48 +74,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ uint32_t mulmod32(uint32_t x, uint32_t y, uint32_t m) {
   return (uint32_t)(((uint64_t)x * y) % m);
-}
-
-// Philox4x32-10 with rounds 0 and 1 precomputed. Round 0 maps the counter
-// (c0, t, i, c3) to (A, B, C, D) with A, B functions of the draw and C, D of
-// the slot block; round 1 maps it to (E ^ B, F, G ^ D', H) with E, F, D' per
-// slot block and G, H per draw. Rounds 2..9 follow.
-struct DrawConst {
-  uint32_t B, G, H;
-};
-struct BlockConst {
-  uint32_t E, F, Dp;
-};
-
-__device__ __forceinline__ BlockConst block_const(const Sub2Args& A, uint32_t c0) {
-  const uint64_t p0 = (uint64_t)kPhiloxM0 * c0;
-  const uint32_t C = (uint32_t)(p0 >> 32) ^ A.ctr3 ^ A.rk1[0];
-  const uint32_t D = (uint32_t)p0;
-  const uint64_t p1 = (uint64_t)kPhiloxM1 * C;
-  BlockConst b;
-  b.E = (uint32_t)(p1 >> 32) ^ A.rk0[1];
-  b.F = (uint32_t)p1;
-  b.Dp = D ^ A.rk1[1];
-  return b;
-}
-
-__device__ __forceinline__ DrawConst draw_const(const Sub2Args& A, uint32_t t_abs, uint32_t i_abs) {
-  const uint64_t p1 = (uint64_t)kPhiloxM1 * i_abs;
-  const uint32_t Aw = (uint32_t)(p1 >> 32) ^ t_abs ^ A.rk0[0];
-  DrawConst d;
-  d.B = (uint32_t)p1;
-  const uint64_t p0 = (uint64_t)kPhiloxM0 * Aw;
-  d.G = (uint32_t)(p0 >> 32);
-  d.H = (uint32_t)p0;
-  return d;
-}
-
-__device__ __forceinline__ U4 philox_from2(const BlockConst& bc, const DrawConst& dc,
-                                           const Sub2Args& A) {
-  U4 c{bc.E ^ dc.B, bc.F, dc.G ^ bc.Dp, dc.H};
-#pragma unroll
-  for (int r = 2; r < 10; ++r) c = philox_round(c, A.rk0[r], A.rk1[r]);
-  return c;
 }
 
 template <bool INT>
@@ -161,9 +119,9 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
 
   BlockConst bc[NB];
 #pragma unroll
-  for (int m = 0; m < NB; ++m) bc[m] = block_const(A, slot_ctr0((uint32_t)m, (uint32_t)lane));
+  for (int m = 0; m < NB; ++m) bc[m] = block_const(A.keys, slot_ctr0((uint32_t)m, (uint32_t)lane), A.ctr3);
   // the appended target slot S: counter block S >> 7, lane S & 31, word (S >> 5) & 3
-  const BlockConst bs = block_const(A, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u));
+  const BlockConst bs = block_const(A.keys, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u), A.ctr3);
   const uint32_t s_word = ((uint32_t)S >> 5) & 3u;
   const bool vec = (V & 3u) == 0;  // rows start 16-byte aligned
 
@@ -215,7 +173,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         mine = (c >= lo) && (c < hi);
         kyq = (qy >= c) ? qy - c : qy + V - c;
         if (mine && kyq >= (uint32_t)S) {
-          const U4 w = philox_from2(bs, draw_const(A, t_abs, i_abs), A);
+          const U4 w = philox_from2(bs, draw_const(A.keys, t_abs, i_abs), A.keys);
           const float2 nn =
               box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, A.sigma, s_tab);
           x_extra = (s_word & 1u) ? nn.y : nn.x;
@@ -229,7 +187,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         const uint32_t cw = __shfl_sync(0xffffffffu, c, src);
         const uint32_t ky = __shfl_sync(0xffffffffu, kyq, src);
         const float xe = __shfl_sync(0xffffffffu, x_extra, src);
-        const DrawConst dc = draw_const(A, t_abs, A.i_off + (uint32_t)i);
+        const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)i);
         const bool in_win = ky < (uint32_t)S;
         const bool local = (cw + (uint32_t)S) <= hi;  // whole window in this slice
         float n[NB][4];  // sigma * eps of the draw's slots
@@ -246,7 +204,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
             }
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A), A.sigma, s_tab);
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), A.sigma, s_tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
@@ -258,7 +216,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         } else {
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A), A.sigma, s_tab);
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), A.sigma, s_tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
@@ -349,13 +307,6 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
   if (CS > 1) cluster.sync();
 }
 
-int expm1_degree2(float sigma) {
-  const float xmax = sigma * 5.7686f;
-  if (xmax <= 0.03f) return 4;
-  if (xmax <= 0.06f) return 5;
-  return 0;
-}
-
 template <int CS, int NB, bool FULL, int DEG, bool INT>
 cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_count) {
   auto fn = k_subset2<CS, NB, FULL, DEG, INT>;
@@ -387,8 +338,8 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
 
 template <int CS, int NB, bool FULL, bool INT>
 cudaError_t launch_deg(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
+  if (deg == 3) return launch_one<CS, NB, FULL, 3, INT>(st, A, smem, sm);
   if (deg == 4) return launch_one<CS, NB, FULL, 4, INT>(st, A, smem, sm);
-  if (deg == 5) return launch_one<CS, NB, FULL, 5, INT>(st, A, smem, sm);
   return launch_one<CS, NB, FULL, 0, INT>(st, A, smem, sm);
 }
 
@@ -429,10 +380,7 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   if (!cs) return cudaErrorNotSupported;
   Sub2Args A;
   A.key = key_of(p.seed);
-  for (int r = 0; r < 10; ++r) {
-    A.rk0[r] = A.key.k0 + (uint32_t)r * kPhiloxW0;
-    A.rk1[r] = A.key.k1 + (uint32_t)r * kPhiloxW1;
-  }
+  A.keys = round_keys(p.seed);
   A.t_off = (uint32_t)p.token_offset;
   A.i_off = (uint32_t)p.draw_offset;
   A.ctr3 = ctr3_of(kTagHead, p.stream_id);
@@ -463,7 +411,7 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.gop_bf16 = p.dtype == DUST_BF16;
   A.plane = p.T * p.V;
   const size_t smem = (size_t)2 * A.seg * 4;
-  const int deg = expm1_degree2(p.sigma);
+  const int deg = expm1_degree(p.sigma);
   const bool use_int = p.K <= 65536;
   if (cs == 1) return launch_cs<1>(st, A, smem, sm_count, deg, use_int);
   return launch_cs<2>(st, A, smem, sm_count, deg, use_int);

@@ -52,6 +52,12 @@ __device__ __forceinline__ U4 philox10(U4 c, uint32_t k0, uint32_t k1) {
   return c;
 }
 
+// (float)i for |i| < 2^22, exactly, by exponent-bias arithmetic on the ALU
+// pipe: 1.5 * 2^23 + i has i in its low mantissa bits.
+__device__ __forceinline__ float small_int_to_float(int i) {
+  return __int_as_float(0x4B400000 + i) - 12582912.0f;
+}
+
 // -ln(u) for u in (0, 1], accurate to a few ulp relative to the result,
 // including u -> 1. u = 2^e m with m in [sqrt(1/2), sqrt(2)): subtracting the
 // bit pattern of sqrt(1/2) before extracting the exponent lands m in that
@@ -71,7 +77,7 @@ __device__ __forceinline__ float neg_log_unit(float u) {
   poly = fmaf(w, poly, 2.0f / 3.0f);
   poly = fmaf(w, poly, 2.0f);
   const float ln_m = s * poly;
-  const float fe = (float)e;
+  const float fe = small_int_to_float(e);
   const float kLn2Hi = 0.693145751953125f;        // 0x3f317200
   const float kLn2Lo = 1.428606765330187e-06f;    // ln 2 - kLn2Hi
   const float ln_u = fmaf(fe, kLn2Hi, fmaf(fe, kLn2Lo, ln_m));
@@ -144,7 +150,7 @@ __device__ __forceinline__ void sincos_turn24_tab(uint32_t m, const float2* tab,
                                                   float* c_out) {
   const uint32_t idx = (m + (1u << 13)) >> 14;             // nearest 1/1024 turn, 0..1024
   const int r = (int)m - (int)(idx << 14);                  // [-2^13, 2^13)
-  const float x = (float)r * 3.7450702e-07f;                // 2 pi / 2^24
+  const float x = small_int_to_float(r) * 3.7450702e-07f;   // 2 pi / 2^24
   const float h = 0.5f * x * x;
   const float2 t = tab[idx & (kSinCosTable - 1)];
   *c_out = fmaf(-t.y, x, fmaf(-t.x, h, t.x));
@@ -194,6 +200,66 @@ __device__ __forceinline__ float log1p_small(float s) {
   return log1pf(s);
 }
 
+// Round keys of a launch: rk0[r] = k0 + r 0x9E3779B9, rk1[r] = k1 + r 0xBB67AE85.
+// Kernels take them as __grid_constant__ parameters so that the XORs read
+// them from the constant bank.
+struct RoundKeys {
+  uint32_t rk0[10], rk1[10];
+};
+
+__host__ inline RoundKeys round_keys(uint64_t seed) {
+  RoundKeys k;
+  const uint32_t k0 = (uint32_t)(seed & 0xffffffffu), k1 = (uint32_t)(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    k.rk0[r] = k0 + (uint32_t)r * kPhiloxW0;
+    k.rk1[r] = k1 + (uint32_t)r * kPhiloxW1;
+  }
+  return k;
+}
+
+// Philox4x32-10 with rounds 0 and 1 precomputed. Round 0 maps the counter
+// (c0, t, i, c3) to (A, B, C, D), with A and B functions of the draw (t, i)
+// and C, D of the slot block (c0, c3); round 1 maps that to
+// (E ^ B, F, G ^ D', H), with E, F, D' per slot block and G, H per draw.
+// A kernel that loops over draws for fixed slot blocks evaluates these once.
+struct DrawConst {
+  uint32_t B, G, H;
+};
+struct BlockConst {
+  uint32_t E, F, Dp;
+};
+
+__device__ __forceinline__ BlockConst block_const(const RoundKeys& K, uint32_t c0, uint32_t c3) {
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * c0;
+  const uint32_t C = (uint32_t)(p0 >> 32) ^ c3 ^ K.rk1[0];
+  const uint32_t D = (uint32_t)p0;
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * C;
+  BlockConst b;
+  b.E = (uint32_t)(p1 >> 32) ^ K.rk0[1];
+  b.F = (uint32_t)p1;
+  b.Dp = D ^ K.rk1[1];
+  return b;
+}
+
+__device__ __forceinline__ DrawConst draw_const(const RoundKeys& K, uint32_t t_abs, uint32_t i_abs) {
+  const uint64_t p1 = (uint64_t)kPhiloxM1 * i_abs;
+  const uint32_t a = (uint32_t)(p1 >> 32) ^ t_abs ^ K.rk0[0];
+  DrawConst d;
+  d.B = (uint32_t)p1;
+  const uint64_t p0 = (uint64_t)kPhiloxM0 * a;
+  d.G = (uint32_t)(p0 >> 32);
+  d.H = (uint32_t)p0;
+  return d;
+}
+
+__device__ __forceinline__ U4 philox_from2(const BlockConst& bc, const DrawConst& dc,
+                                           const RoundKeys& K) {
+  U4 c{bc.E ^ dc.B, bc.F, dc.G ^ bc.Dp, dc.H};
+#pragma unroll
+  for (int r = 2; r < 10; ++r) c = philox_round(c, K.rk0[r], K.rk1[r]);
+  return c;
+}
+
 // Counter word 0 for slot block `blk` (128 slots) and lane `lane`.
 __host__ __device__ __forceinline__ uint32_t slot_ctr0(uint32_t blk, uint32_t lane) {
   return (blk << 5) | lane;
@@ -227,11 +293,18 @@ __device__ __forceinline__ uint32_t subset_offset(Key key, uint32_t t_abs, uint3
   return (uint32_t)(((uint64_t)w.x * V) >> 32);
 }
 
-// expm1 for |x| <= 0.03 (degree 4) or 0.06 (degree 5) from its Taylor series,
-// relative truncation error below 7e-9 and 2e-9; larger arguments use expm1f.
+// expm1 from its Taylor series of degree DEG (0: the library function). The
+// callers form s = sum_j p_j expm1(x_j) with sum_j p_j <= 1, so a truncation
+// |x|^(DEG+1)/(DEG+1)! bounds the absolute error of s: degree 3 for
+// |x| <= 0.03 leaves < 3.4e-8, degree 4 for |x| <= 0.06 < 6.5e-9
+// (expm1_degree picks DEG from sigma).
 template <int DEG>
 __device__ __forceinline__ float expm1_small(float x) {
-  if constexpr (DEG == 4) {
+  if constexpr (DEG == 3) {
+    float q = fmaf(x, 1.0f / 6.0f, 0.5f);
+    q = fmaf(x, q, 1.0f);
+    return x * q;
+  } else if constexpr (DEG == 4) {
     float q = fmaf(x, 1.0f / 24.0f, 1.0f / 6.0f);
     q = fmaf(x, q, 0.5f);
     q = fmaf(x, q, 1.0f);
@@ -245,6 +318,14 @@ __device__ __forceinline__ float expm1_small(float x) {
   } else {
     return expm1f(x);
   }
+}
+
+// Degree of expm1_small for noise of scale sigma (|eps| <= sqrt(48 ln 2) = 5.7686).
+__host__ __device__ inline int expm1_degree(float sigma) {
+  const float xmax = sigma * 5.7686f;
+  if (xmax <= 0.03f) return 3;
+  if (xmax <= 0.06f) return 4;
+  return 0;
 }
 
 }  // namespace dust

@@ -1,0 +1,50 @@
+"""Token-sharded estimator across GPUs (one process per GPU).
+
+Tokens are independent units of the estimator ("Dust：无需反向传播的
+Transformer零阶预训练", §1: every token is its own population member) and the
+weight gradient is a sum over tokens (G_W = sum_t g_t x_t^T), so a batch splits
+across ranks by tokens: rank r runs the estimator on its contiguous token
+range with token_offset = start, which reproduces exactly the noise a single
+run over the whole batch would draw, and one sum all-reduce of the per-rank
+G_W (NCCL over NVLink/NVSwitch on GPUs) gives the estimate of the full batch.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+import torch.distributed as dist
+
+
+def token_shard(T_total: int, world: int, rank: int) -> Tuple[int, int]:
+    """(first token, token count) of `rank`'s contiguous share of T_total tokens.
+
+    The first T_total % world ranks take one extra token; shares are disjoint
+    and cover [0, T_total) in rank order.
+    """
+    if world < 1 or not 0 <= rank < world or T_total < 0:
+        raise ValueError("bad shard arguments")
+    base, extra = divmod(T_total, world)
+    start = rank * base + min(rank, extra)
+    return start, base + (1 if rank < extra else 0)
+
+
+def allreduce_weight_grad(G: torch.Tensor, group: Optional[dist.ProcessGroup] = None) -> torch.Tensor:
+    """Sum the per-rank weight-gradient estimates in place (G_W over all tokens)."""
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(G, op=dist.ReduceOp.SUM, group=group)
+    return G
+
+
+def sharded_head_grad(ctx, H_local: torch.Tensor, W: torch.Tensor, y_local: torch.Tensor,
+                      token_offset: int, group: Optional[dist.ProcessGroup] = None, **kw) -> dict:
+    """LM-head estimator over this rank's tokens, G_W summed over all ranks.
+
+    H_local / y_local hold this rank's tokens, which start at absolute token
+    `token_offset` of the batch (see token_shard). Returns the rank's outputs
+    with "G" replaced by the all-reduced estimate.
+    """
+    out = ctx.head_grad(H_local, W, y_local, token_offset=token_offset, **kw)
+    if "G" in out:
+        allreduce_weight_grad(out["G"], group)
+    return out
