@@ -356,6 +356,14 @@ def run_dust(args):
             if stages.get(key):
                 extra[key + "_tflops"] = gemm_flops / (stages[key] * 1e-3) / 1e12
 
+    # cos(g, exact gradient) against K, outside the timed region (head workloads at N = 1)
+    align = None
+    if wl.variant == "head" and world == 1 and not args.no_alignment and wl.K >= 64:
+        from zeroth_order_transformer_dust_b200.alignment import cosine_vs_k
+        ks = [k for k in (64, 256, 1024, 4096, 16384) if k <= wl.K]
+        align = cosine_vs_k(ctx, Hd, Wd, yd, ks=ks, sigma=wl.sigma, S=wl.S, seed=wl.seed)
+        torch.cuda.empty_cache()
+
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(args.config, budget_tokens=args.ref_tokens)
@@ -371,7 +379,7 @@ def run_dust(args):
                            "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL "
                                            "all-reduce" if world > 1 else "dp1")},
                 "stage_ms": stages, "gpu_launches": launches, "e2e": e2e, "roofline": roof,
-                "cpu_baseline": cb, "clocks": clk, **extra}
+                "cpu_baseline": cb, "clocks": clk, "alignment": align, **extra}
         print(json.dumps(line), flush=True)
     ctx.close()
     if world > 1:
@@ -389,6 +397,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="dust", choices=["dust", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-alignment", action="store_true",
+                    help="skip the cosine-versus-K report of the head estimator")
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="oracle sample size in tokens (default: one per host core, at most 16)")
     ap.add_argument("--tokens", type=int, default=0,

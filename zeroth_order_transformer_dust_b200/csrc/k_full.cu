@@ -51,7 +51,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <int DEG>
 __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __grid_constant__ FullArgs A) {
   __shared__ float sh[kWarps][kDrawChunk];
-  __shared__ float2 tab[kSinCosTable];
+  __shared__ float2 tab[kSinCosTableAlloc];
   fill_sincos_table(tab);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -128,7 +128,7 @@ __global__ void k_full_reward_combine(int64_t T, int32_t K, int nslab,
 
 __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ FullArgs A) {
   __shared__ float rs[1024];
-  __shared__ float2 tab[kSinCosTable];
+  __shared__ float2 tab[kSinCosTableAlloc];
   fill_sincos_table(tab);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -131,6 +131,22 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
   }
 }
 
+// Tile order: bands of kGroupM M-tiles swept across all N-tiles, M fastest
+// within the band. The CTAs running at the same time then cover a compact
+// kGroupM x (SMs / kGroupM) block of tiles, so the band of A (kGroupM * 128
+// rows) and the current few B tiles stay in L2; A is read from HBM once and B
+// once per band.
+constexpr int kGroupM = 16;
+
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int* m_blk,
+                                            int* n_blk) {
+  const int band = tile / (kGroupM * n_tiles);
+  const int r = tile - band * (kGroupM * n_tiles);
+  const int rows = min(kGroupM, m_tiles - band * kGroupM);
+  *m_blk = band * kGroupM + r % rows;
+  *n_blk = r / rows;
+}
+
 // expm1 of a perturbed logit: degree-5 Taylor polynomial below 1/16
 // (relative truncation < 2e-9), the library function otherwise.
 __device__ __forceinline__ float expm1_guarded(float x) {
@@ -220,7 +236,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       bool armed[STAGES] = {};
       uint32_t armed_parity[STAGES] = {};
       for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
-        const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+        int m_blk, n_blk;
+        tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!wait_bounded(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort, p.status)) break;
           const uint32_t fb = ptx::smem_u32(&sh->full[stage]);
@@ -295,7 +312,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       if (!wait_bounded(ptx::smem_u32(&sh->tfull[acc]), acc_phase, abort, p.status)) break;
       ptx::tc_fence_after();
-      const int m_blk = tile % p.m_tiles, n_blk = tile / p.m_tiles;
+      int m_blk, n_blk;
+        tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
       const int64_t m = (int64_t)m_blk * BM + row;
       int64_t mo = m;
       if (p.e.c_row_mul != 0 && m < p.M)

@@ -55,7 +55,7 @@ __global__ void k_debug_gauss(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
 __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off, uint32_t i_off,
                                                          uint32_t ctr3, int64_t nt, int64_t ni,
                                                          int64_t nslots, float* __restrict__ out) {
-  __shared__ float2 tab[kSinCosTable];
+  __shared__ float2 tab[kSinCosTableAlloc];
   fill_sincos_table(tab);
   __syncthreads();
   const int64_t nblk = (nslots + 127) / 128;

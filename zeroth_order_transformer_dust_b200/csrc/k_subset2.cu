@@ -51,6 +51,7 @@ struct Sub2Args {
   int64_t T, V;
   int32_t K, S;
   uint32_t a, a_inv;
+  uint32_t minv;  // floor((2^32 - 1) / V), V <= 2^16
   uint32_t seg;  // q-slice length owned by one CTA (multiple of 4)
   float scale_other, scale_target;
   float fac;        // g = fac * sum r * (sigma eps)            (fp32 accumulators)
@@ -72,8 +73,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ uint32_t mulmod32(uint32_t x, uint32_t y, uint32_t m) {
-  return (uint32_t)(((uint64_t)x * y) % m);
+// x y mod m for x, y < m <= 2^16 (the product fits 32 bits), with
+// minv = floor((2^32 - 1) / m): the quotient estimate hi32(x y minv) is the
+// true quotient or one less (Barrett), so one conditional subtraction ends it.
+__device__ __forceinline__ uint32_t mulmod32(uint32_t x, uint32_t y, uint32_t m, uint32_t minv) {
+  const uint32_t p = x * y;
+  const uint32_t r = p - __umulhi(p, minv) * m;
+  return r >= m ? r - m : r;
 }
 
 template <bool INT>
@@ -90,7 +96,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_next;    // next draw batch of the current token
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
-  __shared__ float2 s_tab[kSinCosTable];
+  __shared__ float2 s_tab[kSinCosTableAlloc];
   fill_sincos_table(s_tab);
   __syncthreads();
   cg::cluster_group cluster = cg::this_cluster();
@@ -148,7 +154,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
     }
     int32_t yt = A.y[t];
     if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
-    const uint32_t qy = mulmod32((uint32_t)yt, A.a_inv, V);
+    const uint32_t qy = mulmod32((uint32_t)yt, A.a_inv, V, A.minv);
     const bool own_y = qy >= lo && qy < hi;
     const float py = expf(zrow[qy] - lse_t);
     float* gy = own_y ? sg + (qy - lo) : sg_peer + (qy - lo_peer);
@@ -169,7 +175,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
       if (iq < A.K) {
         const uint32_t i_abs = A.i_off + (uint32_t)iq;
         const uint32_t b = subset_offset(A.key, t_abs, i_abs, A.stream_id, V);
-        c = mulmod32(b, A.a_inv, V);
+        c = mulmod32(b, A.a_inv, V, A.minv);
         mine = (c >= lo) && (c < hi);
         kyq = (qy >= c) ? qy - c : qy + V - c;
         if (mine && kyq >= (uint32_t)S) {
@@ -300,7 +306,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + qg, v);
       else
         ((float*)A.gop)[t * A.V + qg] = v;
-      if (A.g_out) A.g_out[t * A.V + mulmod32(qg, A.a, V)] = v;
+      if (A.g_out) A.g_out[t * A.V + mulmod32(qg, A.a, V, A.minv)] = v;
     }
     __syncthreads();
   }
@@ -366,10 +372,10 @@ cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, i
 // Cluster size the shared-memory kernel would use (0: not applicable).
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
   if (S < 1 || S > 512) return 0;
-  const int64_t slack = 1024 + 8 * kSinCosTable;  // static: counters, angle table
+  const int64_t slack = 1024 + 8 * kSinCosTableAlloc;  // static: counters, angle table
   if (2 * V * 4 + slack <= max_smem_optin && V <= 65536) return 1;
   const int64_t seg = ((V + 1) / 2 + 3) / 4 * 4;
-  if (2 * seg * 4 + slack <= max_smem_optin && S <= V - seg && S <= seg) return 2;
+  if (2 * seg * 4 + slack <= max_smem_optin && S <= V - seg && S <= seg && V <= 65536) return 2;
   return 0;
 }
 
@@ -392,6 +398,7 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.S = p.S;
   A.a = (uint32_t)a;
   A.a_inv = (uint32_t)a_inv;
+  A.minv = (uint32_t)(0xffffffffull / (uint64_t)p.V);
   A.seg = cs == 1 ? (uint32_t)((p.V + 3) / 4 * 4) : (uint32_t)(((p.V + 1) / 2 + 3) / 4 * 4);
   A.scale_other = (float)((double)p.V / (double)p.S);
   A.scale_target = (p.flags & DUST_FLAG_LITERAL_TARGET_SCALE) ? A.scale_other : 1.0f;

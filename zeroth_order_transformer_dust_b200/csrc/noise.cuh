@@ -84,6 +84,26 @@ __device__ __forceinline__ float neg_log_unit(float u) {
   return -ln_u;
 }
 
+// -ln(j 2^-24) for an integer j in [1, 2^24], the same computation as
+// neg_log_unit with the 2^-24 scale folded into the exponent (the float of j
+// is exact, and e - 24 comes out of the same exponent-bias subtraction).
+__device__ __forceinline__ float neg_log_u24(uint32_t j) {
+  const int bits = __float_as_int((float)j);
+  const int e = (bits - 0x3f3504f3) >> 23;
+  const float m = __int_as_float(bits - (e << 23));
+  const float f = m - 1.0f;  // exact (Sterbenz)
+  const float s = __fdividef(f, m + 1.0f);
+  const float w = s * s;
+  float poly = fmaf(w, 2.0f / 7.0f, 2.0f / 5.0f);
+  poly = fmaf(w, poly, 2.0f / 3.0f);
+  poly = fmaf(w, poly, 2.0f);
+  const float ln_m = s * poly;
+  const float fe = __int_as_float(0x4B400000 + e) - 12582936.0f;  // e - 24, exact
+  const float kLn2Hi = 0.693145751953125f;
+  const float kLn2Lo = 1.428606765330187e-06f;
+  return -fmaf(fe, kLn2Hi, fmaf(fe, kLn2Lo, ln_m));
+}
+
 // sqrt(x) for x >= 0: the hardware reciprocal-square-root estimate y refined
 // by one Newton-Raphson step on r = x y (r' = r + (y/2)(x - r^2)), which
 // leaves about one ulp of error. x is clamped away from 0 (sqrt(0) -> 1e-15).
@@ -137,11 +157,12 @@ __device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb, float sca
 // plus a remainder |x| <= pi/1024, and cos/sin follow from the angle-addition
 // formulas with cos x = 1 - x^2/2 and sin x = x (truncation below 5e-9).
 constexpr int kSinCosTable = 1024;
+constexpr int kSinCosTableAlloc = kSinCosTable + 1;  // entry 1024 repeats entry 0
 
 __device__ __forceinline__ void fill_sincos_table(float2* tab) {
-  for (int k = threadIdx.x; k < kSinCosTable; k += blockDim.x) {
+  for (int k = threadIdx.x; k < kSinCosTableAlloc; k += blockDim.x) {
     float s, c;
-    sincospif((float)k * (2.0f / kSinCosTable), &s, &c);
+    sincospif((float)(k & (kSinCosTable - 1)) * (2.0f / kSinCosTable), &s, &c);
     tab[k] = make_float2(c, s);
   }
 }
@@ -152,15 +173,14 @@ __device__ __forceinline__ void sincos_turn24_tab(uint32_t m, const float2* tab,
   const int r = (int)m - (int)(idx << 14);                  // [-2^13, 2^13)
   const float x = small_int_to_float(r) * 3.7450702e-07f;   // 2 pi / 2^24
   const float h = 0.5f * x * x;
-  const float2 t = tab[idx & (kSinCosTable - 1)];
+  const float2 t = tab[idx];
   *c_out = fmaf(-t.y, x, fmaf(-t.x, h, t.x));
   *s_out = fmaf(t.x, x, fmaf(-t.y, h, t.y));
 }
 
 __device__ __forceinline__ float2 box_muller_tab(uint32_t wa, uint32_t wb, float scale,
                                                  const float2* tab) {
-  const float u1 = (float)((wa >> 8) + 1u) * 5.9604645e-08f;  // exact
-  const float radius = scale * sqrt_newton(2.0f * neg_log_unit(u1));
+  const float radius = scale * sqrt_newton(2.0f * neg_log_u24((wa >> 8) + 1u));
   float s, c;
   sincos_turn24_tab(wb >> 8, tab, &s, &c);
   return make_float2(radius * c, radius * s);
