@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -37,10 +38,16 @@ METRIC = "token-draws/sec of Dust gradient estimate (LM head d=1024,V=50304); % 
 UNIT = "token-draws/s"
 SM_COUNT = 148
 LANES_PER_SM = 128           # 4 schedulers x 32 lanes issue per clock
-# Algorithmic instruction slots per perturbed element (see DESIGN.md):
+# Algorithmic instruction slots per perturbed element:
 # Philox4x32-10 10, Gaussian transform 4, expm1 2, reward multiply-add and
 # its operand load 2, g accumulation multiply and add 2.
 ALU_OPS_PER_ELEM = 20
+# DRAM bytes (read + write) per token of the subset-draw kernel on the
+# large-subset workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of
+# one launch over its first 2048 tokens (415.44 + 368.23 MB), per token; the
+# kernel's traffic is per token (the logit row in, the g operand planes out).
+SUBSET_DRAM_BYTES_PER_TOKEN = (415.442688e6 + 368.229888e6) / 2048
+PROFILED_SUBSET_WORKLOAD = "large_subset_bf16"
 
 
 def _peaks():
@@ -61,7 +68,8 @@ class ClockSampler:
 
     def __init__(self, out_path=None):
         self.proc = None
-        self.path = out_path or os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = out_path or os.path.join(os.environ.get("DUST_CLOCKS_DIR", tempfile.gettempdir()),
+                                             f"dust_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -349,6 +357,10 @@ def run_dust(args):
         if draw_ms:
             roof = _alu_roofline(wl, draw_ms, peaks)
             roof["peak_kind"] = peak_kind
+            if wl.S > 0 and args.config == PROFILED_SUBSET_WORKLOAD:
+                roof["traffic"] = SUBSET_DRAM_BYTES_PER_TOKEN * wl.T
+                roof["traffic_basis"] = ("ncu DRAM bytes of a 2048-token launch, scaled by "
+                                         "tokens to this launch")
     gemm_flops = 2.0 * wl.T * wl.d * wl.V
     extra = {}
     if wl.variant == "head":

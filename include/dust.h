@@ -198,6 +198,21 @@ dust_status dust_head_grad_noalloc(const dust_params* p, void* cuda_stream,
                                    float* G_out, float* loss_out, float* rewards_out,
                                    float* g_out, char* msg, int msg_len);
 
+/* One step of SGD with momentum on n weights (the Dust pages train with SGD
+   and momentum, "Dust：无需反向传播的Transformer零阶预训练" §2 实证发现, and
+   leave its form open; this is the heavy-ball step without dampening,
+   Nesterov term or weight decay):
+     v <- mu v + G,   W <- W - lr v            (fp32, elementwise)
+   G: the estimator's weight gradient (device, fp32, read only, e.g. G_out of
+   dust_head_grad); v: momentum buffer (device, fp32, in/out; start it at
+   zero); W: fp32 master weights (device, in/out); W_bf16: NULL, or a device
+   bf16 array that receives W rounded to nearest even (the copy the next
+   estimator call reads). G, v and W must not overlap one another; all three
+   16-byte aligned, W_bf16 8-byte aligned (DUST_ERR_ARG otherwise, before any
+   launch). Asynchronous on the context's stream; n = 0 launches nothing. */
+dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, const float* G,
+                              float* v, float* W, void* W_bf16);
+
 /* Debug: C (M x N, fp32, row-major) = A B^T for bf16 row-major A (M x K) and
    B (N x K), through the library's GEMMs: path 0 = automatic, 1 = CUDA cores,
    2 = tcgen05 tensor cores (DUST_ERR_UNSUPPORTED when the shape does not fit:
@@ -217,6 +232,17 @@ dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag,
    it agrees with dust_debug_gauss to a few 1e-7. */
 dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t tag,
                                  int64_t nt, int64_t ni, int64_t nslots, float* out);
+
+/* Debug: the Box-Muller radius for every 24-bit input. out (2^24 fp32,
+   device) receives sigma sqrt(-2 ln u1) for u1 = (j + 1) 2^-24 at index j, as
+   every noise kernel computes it (the pages fix only Gaussian noise; this
+   transform is the library's). Synchronous. */
+dust_status dust_debug_bm_radius(dust_ctx* ctx, float sigma, float* out);
+/* Debug: the Box-Muller angle step for every 24-bit input. out (2 x 2^24
+   fp32, device) receives (cos, sin) of 2 pi m 2^-24 at [2m, 2m+1]; method 0 is
+   the polynomial step (MLP noise), 1 the table step (LM-head noise).
+   Synchronous. */
+dust_status dust_debug_bm_angle(dust_ctx* ctx, int32_t method, float* out);
 
 #ifdef __cplusplus
 }

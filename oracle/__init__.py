@@ -43,3 +43,4 @@ from .head import (  # noqa: F401
     clean_head, head_grad, head_linear_estimate, full_vocab_draws, subset_draws,
 )
 from .mlp import clean_mlp, mlp_grad, mlp_draws, gelu  # noqa: F401
+from .optim import sgd_momentum, train_head, exact_weight_grad  # noqa: F401

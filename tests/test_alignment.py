@@ -21,6 +21,10 @@ def test_fit_recovers_an_exact_law():
         assert abs(f["c_max"] - c_max) < 1e-9 * max(1.0, c_max)
         assert abs(f["c"] - c) < 1e-6 * c
         assert f["rmse"] < 1e-12
+    # c_max = 1 exactly: the constrained fit recovers c too
+    cos = [1.0 / math.sqrt(1 + 4.9e6 / k) for k in ks]
+    f = fit_cos_law(ks, cos)
+    assert abs(f["c_at_cmax1"] - 4.9e6) < 1e-6 * 4.9e6 and f["rmse_at_cmax1"] < 1e-12
 
 
 def test_fit_reports_misfit():

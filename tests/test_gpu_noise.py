@@ -48,3 +48,64 @@ def test_gaussian_extremes_match_oracle(ctx, table):
     ref = oracle.gaussians(99, np.arange(nt)[:, None], np.arange(ni)[None, :], np.arange(ns), 0)
     assert np.abs(ref).max() > 4.5
     assert np.abs(got - ref).max() < TOL_GAUSS
+
+
+# Exhaustive checks of the two one-dimensional pieces of the Box-Muller
+# transform over all 2^24 inputs each. A Gaussian is the rounded product
+# fl(R~ c~) of the radius R~ = R + dR and the cosine (or sine) c~ = c + dc, so
+# |eps error| <= |dR| |c~| + R |dc| + 2^-24 |R~ c~| (round to nearest) <=
+# max|dR| + R_max max|dc| + R_max 2^-24 up to second-order terms, with
+# R_max = sqrt(48 ln 2) the largest radius of 24-bit uniforms; that bound
+# holding is the 2e-6 bar for every pair of words.
+R_MAX = float(np.sqrt(-2.0 * np.log(2.0 ** -24)))
+
+
+def _radius_ref():
+    j = np.arange(1, (1 << 24) + 1, dtype=np.float64)
+    return np.sqrt(-2.0 * np.log(j * 2.0 ** -24))
+
+
+def _angle_ref():
+    theta = np.arange(1 << 24, dtype=np.float64) * (np.pi * 2.0 ** -23)
+    return np.cos(theta), np.sin(theta)
+
+
+@pytest.fixture(scope="module")
+def radius_err(ctx):
+    got = ctx.debug_bm_radius(1.0).cpu().numpy().astype(np.float64)
+    return np.abs(got - _radius_ref())
+
+
+@pytest.fixture(scope="module")
+def angle_err(ctx):
+    c, s = _angle_ref()
+    out = {}
+    for table in (False, True):
+        got = ctx.debug_bm_angle(table).cpu().numpy().astype(np.float64)
+        out[table] = max(np.abs(got[:, 0] - c).max(), np.abs(got[:, 1] - s).max())
+    return out
+
+
+def test_radius_all_inputs(radius_err):
+    # a few 1e-7 everywhere, including u1 -> 1 where the radius -> 0
+    assert radius_err.max() < 8e-7, radius_err.max()
+    assert radius_err[-(1 << 17):].max() < 1e-7      # the series branch, v < 2^-7
+
+
+def test_radius_scales_with_sigma(ctx):
+    base = ctx.debug_bm_radius(1.0)
+    for sigma in (5e-3, 1e-2, 0.37):
+        got = ctx.debug_bm_radius(sigma)
+        assert torch.allclose(got, base * sigma, rtol=2e-7, atol=0)
+    assert not ctx.debug_bm_radius(0.0).any()         # sigma = 0: exact zeros
+
+
+@pytest.mark.parametrize("table", [False, True])
+def test_angle_all_inputs(angle_err, table):
+    assert angle_err[table] < 2e-7, angle_err[table]
+
+
+@pytest.mark.parametrize("table", [False, True])
+def test_gaussian_bound_over_all_words(radius_err, angle_err, table):
+    bound = (radius_err.max() + R_MAX * angle_err[table] + R_MAX * 2.0 ** -24) * (1 + 1e-6)
+    assert bound < TOL_GAUSS, bound

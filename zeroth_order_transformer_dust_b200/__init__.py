@@ -33,7 +33,8 @@ EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
            "dust_head_grad", "dust_head_grad_host", "dust_mlp_grad", "dust_debug_philox",
            "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
            "dust_kernel_launches", "dust_debug_gemm_bf16", "dust_debug_gauss_tab",
-           "dust_head_grad_noalloc")
+           "dust_head_grad_noalloc", "dust_debug_bm_radius", "dust_debug_bm_angle",
+           "dust_sgd_momentum")
 
 
 class DustParams(ctypes.Structure):
@@ -90,6 +91,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "dust_debug_gauss_tab": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_head_grad_noalloc": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_char_p,
                                              ctypes.c_int]),
+            "dust_debug_bm_radius": (I32, [P, ctypes.c_float, P]),
+            "dust_debug_bm_angle": (I32, [P, I32, P]),
+            "dust_sgd_momentum": (I32, [P, I64, ctypes.c_float, ctypes.c_float, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -283,6 +287,21 @@ class Context:
     def kernel_launches(self) -> int:
         return int(self._L.dust_kernel_launches(self._h))
 
+    def sgd_momentum(self, G, v, W, *, lr: float, mu: float, W_bf16=None) -> None:
+        """Heavy-ball step in place: v <- mu v + G, W <- W - lr v (fp32 device
+        tensors of one size); W_bf16, if given, receives W rounded to bf16."""
+        for t, name in ((G, "G"), (v, "v"), (W, "W")):
+            self._dev(t, name)
+            if t.dtype != torch.float32 or t.numel() != G.numel():
+                raise TypeError(f"{name} must be fp32 with G's size")
+        if W_bf16 is not None:
+            self._dev(W_bf16, "W_bf16")
+            if W_bf16.dtype != torch.bfloat16 or W_bf16.numel() != G.numel():
+                raise TypeError("W_bf16 must be bf16 with G's size")
+        self._bind_stream()
+        self._check(self._L.dust_sgd_momentum(self._h, G.numel(), float(lr), float(mu), _ptr(G),
+                                              _ptr(v), _ptr(W), _ptr(W_bf16)))
+
     # -- debug exports -------------------------------------------------------------
     def debug_gemm(self, A: torch.Tensor, B: torch.Tensor, path: int = 0) -> torch.Tensor:
         """C = A B^T (bf16 operands, fp32 out); path 0 auto, 1 CUDA cores, 2 tensor cores."""
@@ -314,6 +333,20 @@ class Context:
         self._bind_stream()
         fn = self._L.dust_debug_gauss_tab if table else self._L.dust_debug_gauss
         self._check(fn(self._h, ctypes.byref(prm), tag, nt, ni, nslots, _ptr(out)))
+        return out
+
+    def debug_bm_radius(self, sigma: float = 1.0) -> torch.Tensor:
+        """Box-Muller radius sigma sqrt(-2 ln u1) for every u1 = (j + 1) 2^-24, j < 2^24."""
+        out = torch.empty(1 << 24, dtype=torch.float32, device=f"cuda:{self.device}")
+        self._bind_stream()
+        self._check(self._L.dust_debug_bm_radius(self._h, float(sigma), _ptr(out)))
+        return out
+
+    def debug_bm_angle(self, table: bool) -> torch.Tensor:
+        """(cos, sin) of 2 pi m 2^-24 for every m < 2^24 (2^24 x 2)."""
+        out = torch.empty(1 << 24, 2, dtype=torch.float32, device=f"cuda:{self.device}")
+        self._bind_stream()
+        self._check(self._L.dust_debug_bm_angle(self._h, 1 if table else 0, _ptr(out)))
         return out
 
 

@@ -38,13 +38,18 @@ def fit_cos_law(ks, cos):
     sxx = sum((x - mx) ** 2 for x in xs)
     slope = sum((x - mx) * (v - my) for x, v in zip(xs, ys)) / sxx if sxx > 0 else 0.0
     icept = my - slope * mx
-    if icept <= 0:
-        return {"c_max": None, "c": None, "rmse": None}
+    # with c_max held at 1: 1/cos^2 - 1 = c/K, least squares in 1/K through 0
+    c1 = sum(x * (v - 1.0) for x, v in zip(xs, ys)) / sum(x * x for x in xs)
+    pred1 = [1.0 / math.sqrt(max(1e-300, 1.0 + c1 / k)) for k in ks]
+    rmse1 = math.sqrt(sum((p - v) ** 2 for p, v in zip(pred1, cos)) / n)
+    out = {"c_max": None, "c": None, "rmse": None, "c_at_cmax1": c1, "rmse_at_cmax1": rmse1}
+    if icept <= 0:   # c >> K over the whole range: only c_max^2 / c is identified
+        return out
     c_max = 1.0 / math.sqrt(icept)
     c = slope / icept
     pred = [c_max / math.sqrt(max(1e-300, 1.0 + c / k)) for k in ks]
-    rmse = math.sqrt(sum((p - v) ** 2 for p, v in zip(pred, cos)) / n)
-    return {"c_max": c_max, "c": c, "rmse": rmse}
+    out.update(c_max=c_max, c=c, rmse=math.sqrt(sum((p - v) ** 2 for p, v in zip(pred, cos)) / n))
+    return out
 
 
 @torch.no_grad()

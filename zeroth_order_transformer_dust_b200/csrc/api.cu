@@ -271,7 +271,7 @@ void dust_destroy(dust_ctx* ctx) {
   Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
                  &ctx->gT, &ctx->hT, &ctx->xdup, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
-                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv};
+                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -349,14 +349,29 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   g.dtype = p.dtype;
   EpiDesc e{};
   e.kind = kEpiF32; e.C = Z; e.ldc = p.V;
-  DUST_TRY(run_gemm(ctx, g, e));
-  mark(ctx, "clean_gemm");
-  // 2. log-sum-exp, clean loss, softmax in place (the shared-memory subset
-  //    kernel forms p itself while it loads a row)
+  // The draw kernels form p = exp(z - LSE) themselves, except the L2-fed
+  // subset kernel, which reads p written in place over z.
   const bool smem_subset =
       subset && ctx->subset2_enabled && subset2_cluster_size(p.V, p.S, ctx->max_smem_optin) > 0;
-  DUST_CU(launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, (float*)ctx->lse.p, loss,
-                          !smem_subset, ctx->d_status));
+  const bool need_prob = subset && !smem_subset;
+  // On tensor cores the GEMM epilogue also leaves per-tile softmax partials
+  // of every row (the per-token max / log-sum-exp cache), so z is not re-read.
+  const bool fused = !need_prob && ctx->tc_enabled && tc_gemm_supported(g, e);
+  const int ntiles = (int)((p.V + kTcTileN - 1) / kTcTileN);
+  if (fused) {
+    DUST_TRY(ensure(ctx, ctx->lsep, (size_t)p.T * ntiles * sizeof(float2)));
+    e.kind = kEpiF32Lse;
+    e.lsep = (float2*)ctx->lsep.p;
+  }
+  DUST_TRY(run_gemm(ctx, g, e));
+  mark(ctx, "clean_gemm");
+  // 2. log-sum-exp and clean loss
+  if (fused)
+    DUST_CU(launch_lse_combine(st, (const float2*)ctx->lsep.p, ntiles, Z, p.T, p.V, targets,
+                               subset ? a_inv : 0, (float*)ctx->lse.p, loss, ctx->d_status));
+  else
+    DUST_CU(launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, (float*)ctx->lse.p,
+                            loss, need_prob, ctx->d_status));
   ctx->launches += 1;
   mark(ctx, "lse");
   // 3. perturbed losses, rewards, g
@@ -368,7 +383,8 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
     }
     DUST_TRY(ensure(ctx, ctx->part, (size_t)p.T * full_vocab_nslab(p.V) * p.K * 4));
     DUST_TRY(ensure(ctx, ctx->dzy, full_vocab_xy_bytes(p.T, p.K)));
-    DUST_CU(launch_full_reward_partial(st, p, Z, targets, (float*)ctx->part.p, (float*)ctx->dzy.p));
+    DUST_CU(launch_full_reward_partial(st, p, Z, (const float*)ctx->lse.p, targets,
+                                       (float*)ctx->part.p, (float*)ctx->dzy.p));
     DUST_CU(launch_full_reward_combine(st, p, (float*)ctx->part.p, (float*)ctx->dzy.p, r));
     ctx->launches += 2;
     mark(ctx, "reward");
@@ -661,6 +677,43 @@ dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag, i
 dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t tag, int64_t nt,
                                  int64_t ni, int64_t nslots, float* out) {
   return debug_gauss_impl(ctx, p, tag, nt, ni, nslots, out, 1);
+}
+
+dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, const float* G,
+                              float* v, float* W, void* W_bf16) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (n < 0 || !std::isfinite(lr) || !std::isfinite(mu))
+    return fail(ctx, DUST_ERR_ARG, "sgd_momentum: n >= 0 and finite lr, mu are required");
+  if (n > 0 && (!G || !v || !W))
+    return fail(ctx, DUST_ERR_ARG, "sgd_momentum: G, v and W are required");
+  if (!aligned(G, 16) || !aligned(v, 16) || !aligned(W, 16) || !aligned(W_bf16, 8))
+    return fail(ctx, DUST_ERR_ARG, "sgd_momentum: G, v, W must be 16-byte and W_bf16 8-byte aligned");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(launch_sgd_momentum(ctx->stream, n, lr, mu, G, v, W, (__nv_bfloat16*)W_bf16,
+                              ctx->sm_count));
+  ctx->launches += n > 0 ? 1 : 0;
+  return DUST_OK;
+}
+
+dust_status dust_debug_bm_radius(dust_ctx* ctx, float sigma, float* out) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (!out || !(sigma >= 0.0f) || !std::isfinite(sigma))
+    return fail(ctx, DUST_ERR_ARG, "bad radius arguments");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(launch_debug_bm(ctx->stream, 0, sigma, out));
+  ctx->launches += 1;
+  DUST_CU(cudaStreamSynchronize(ctx->stream));
+  return DUST_OK;
+}
+
+dust_status dust_debug_bm_angle(dust_ctx* ctx, int32_t method, float* out) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (!out || method < 0 || method > 1) return fail(ctx, DUST_ERR_ARG, "bad angle arguments");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(launch_debug_bm(ctx->stream, 1 + method, 0.0f, out));
+  ctx->launches += 1;
+  DUST_CU(cudaStreamSynchronize(ctx->stream));
+  return DUST_OK;
 }
 
 }  // extern "C"

@@ -44,6 +44,9 @@ enum EpiKind {
   kEpiReward = 5,      // MLP perturbed logits dz (never stored): per row m and 256-column
                        // tile nb, part[m*n_tiles + nb] = sum_n P[t, n] expm1(dz);
                        // dzy[m] = dz at column y[t]; t = t0 + m / draws
+  kEpiF32Lse = 6,      // kEpiF32 without row remap, plus per row m and 256-column tile
+                       // nb the softmax partial lsep[m*n_tiles + nb] =
+                       // (max_n acc, sum_n exp(acc - max)) over the tile's columns < N
 };
 
 struct EpiDesc {
@@ -63,6 +66,8 @@ struct EpiDesc {
   int32_t draws = 1;
   float* part = nullptr;
   float* dzy = nullptr;
+  // kEpiF32Lse
+  float2* lsep = nullptr;
 };
 
 // Column tile width of the tensor-core GEMM (reward partials per row = ceil(N / it)).
@@ -129,7 +134,7 @@ struct dust_ctx {
   bool subset2_enabled = true;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
-      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv;
+      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep;
 };
 
 namespace dust {
@@ -138,6 +143,11 @@ namespace dust {
 cudaError_t launch_debug_philox(cudaStream_t st, uint64_t seed, const uint32_t* ctr, int64_t n,
                                 uint32_t* out);
 // method 0: polynomial angle step; 1: table-driven angle step (subset kernel).
+cudaError_t launch_sgd_momentum(cudaStream_t st, int64_t n, float lr, float mu, const float* G,
+                                float* v, float* W, __nv_bfloat16* Wb, int sm_count);
+// what: 0 = radius for all 2^24 u1 (2^24 floats), 1 = polynomial angle step,
+// 2 = table angle step (2 x 2^24 floats: cos, sin).
+cudaError_t launch_debug_bm(cudaStream_t st, int what, float sigma, float* out);
 cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, int64_t nt,
                                int64_t ni, int64_t nslots, float* out, int method);
 
@@ -146,6 +156,11 @@ cudaError_t launch_gemm_simt(cudaStream_t st, const GemmDesc& g, const EpiDesc& 
 // Row-wise log-sum-exp of Z (T x V). Writes lse[t], loss[t] = lse - Z[t, col(y_t)]
 // with col(y) = y (col_mul == 0) or (y * col_mul) mod V; if to_prob, overwrites Z
 // with exp(Z - lse). Sets kStatusBadTarget for targets outside [0, V).
+// LSE and clean loss of each row from the clean GEMM's per-tile softmax
+// partials (kEpiF32Lse), ntiles = ceil(V / kTcTileN) per row.
+cudaError_t launch_lse_combine(cudaStream_t st, const float2* lsep, int ntiles, const float* Z,
+                               int64_t T, int64_t V, const int32_t* y, int64_t col_mul,
+                               float* lse, float* loss, uint32_t* status);
 cudaError_t launch_lse_rows(cudaStream_t st, float* Z, int64_t T, int64_t V, const int32_t* y,
                             int64_t col_mul, float* lse, float* loss, bool to_prob,
                             uint32_t* status);
@@ -155,7 +170,8 @@ cudaError_t launch_lse_rows(cudaStream_t st, float* Z, int64_t T, int64_t V, con
 // target -> xy[t * K + i] (T x K floats, full_vocab_xy_bytes).
 int full_vocab_nslab(int64_t V);
 size_t full_vocab_xy_bytes(int64_t T, int32_t K);
-cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* P,
+cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* Z,
+                                       const float* lse,
                                        const int32_t* y, float* part, float* xy);
 // Stage 2: r[t*K + i] = xy - log1p(sum_slab part).
 cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, const float* part,

@@ -1,6 +1,6 @@
 // Full-vocabulary LM-head draws ("Dust：无需反向传播的Transformer零阶预训练",
 // §1): every logit of token t gets sigma*eps; the perturbed loss is formed in
-// delta form from the cached softmax p,
+// delta form from the softmax p = exp(z - LSE) of the cached clean logits,
 //   L' - L = log1p(sum_j p_j expm1(sigma eps_j)) - sigma eps_y,
 // the reward is r = L - L', and g_t = -(1/(K sigma)) sum_i r_i eps_i.
 // The reward needs the whole row before any g entry can be formed, so the
@@ -31,7 +31,8 @@ struct FullArgs {
   int64_t T, V;
   int32_t K;
   int nslab;
-  const float* P;
+  const float* Z;    // clean logits (T x V)
+  const float* lse;  // T
   const int32_t* y;
   float* part;       // (t * nslab + slab) * K + i
   float* xy;         // sigma eps at the target, t * K + i
@@ -51,8 +52,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 template <int DEG>
 __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __grid_constant__ FullArgs A) {
   __shared__ float sh[kWarps][kDrawChunk];
-  __shared__ float2 tab[kSinCosTableAlloc];
-  fill_sincos_table(tab);
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab, A.sigma);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nunits = A.T * A.nslab;
@@ -60,15 +61,16 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __gri
     const int64_t t = unit / A.nslab;
     const int slab = (int)(unit % A.nslab);
     const int64_t blk0 = (int64_t)slab * (kSlab / 128) + warp * kBlocksPerWarp;
-    float pv[kBlocksPerWarp][4];
+    float pv[kBlocksPerWarp][4];  // p = exp(z - LSE), formed once per unit
     BlockConst bc[kBlocksPerWarp];
+    const float lse_t = A.lse[t];
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b) {
       bc[b] = block_const(A.keys, slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), A.ctr3);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
-        pv[b][j] = pos < A.V ? A.P[t * A.V + pos] : 0.0f;
+        pv[b][j] = pos < A.V ? expf(A.Z[t * A.V + pos] - lse_t) : 0.0f;
       }
     }
     // the lane holding the target's noise, if this warp's blocks contain it
@@ -88,7 +90,7 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __gri
 #pragma unroll
         for (int b = 0; b < kBlocksPerWarp; ++b) {
           if ((blk0 + b) * 128 < A.V) {
-            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), A.sigma, tab);
+            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) s = fmaf(pv[b][j], expm1_small<DEG>(g.v[j]), s);
             if (warp_has_y) {
@@ -128,8 +130,8 @@ __global__ void k_full_reward_combine(int64_t T, int32_t K, int nslab,
 
 __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ FullArgs A) {
   __shared__ float rs[1024];
-  __shared__ float2 tab[kSinCosTableAlloc];
-  fill_sincos_table(tab);
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab, A.sigma);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nunits = A.T * A.nslab;
@@ -157,7 +159,7 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
 #pragma unroll
         for (int b = 0; b < kBlocksPerWarp; ++b) {
           if ((blk0 + b) * 128 < A.V) {
-            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), A.sigma, tab);
+            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(ri, g.v[j], acc[b][j]);
           }
@@ -219,10 +221,12 @@ int full_vocab_nslab(int64_t V) { return (int)((V + kSlab - 1) / kSlab); }
 
 size_t full_vocab_xy_bytes(int64_t T, int32_t K) { return (size_t)T * K * 4; }
 
-cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* P,
-                                       const int32_t* y, float* part, float* xy) {
+cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* Z,
+                                       const float* lse, const int32_t* y, float* part,
+                                       float* xy) {
   FullArgs A = make_args(p);
-  A.P = P;
+  A.Z = Z;
+  A.lse = lse;
   A.y = y;
   A.part = part;
   A.xy = xy;

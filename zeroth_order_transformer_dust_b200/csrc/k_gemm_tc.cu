@@ -8,6 +8,7 @@
 // the MMAs of tile i+1. Every mbarrier wait is bounded in time: on expiry the
 // CTA raises the timeout bit of the device status word, drains its own
 // copies and MMAs (bounded again), frees its TMEM and returns.
+#include <cfloat>
 #include <cudaTypedefs.h>
 
 #include "internal.cuh"
@@ -24,7 +25,11 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int THREADS = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+// Reward epilogue: each epilogue warp stages the probability rows of the (at
+// most two) tokens its 32 rows belong to, BN columns each, per accumulator.
+constexpr int PSTAGE_FLOATS = 2 * BN;
+constexpr size_t PSTAGE_BYTES = (size_t)4 * 2 * PSTAGE_FLOATS * 4;  // 4 warps x 2 accumulators
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + PSTAGE_BYTES;
 
 struct TcParams {
   int64_t M, N, K;
@@ -38,6 +43,7 @@ struct Shared {
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Shared) <= 256, "barrier block overlaps the staging area");
 
 __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* status) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -61,13 +67,14 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
                                            const float* v) {
   const EpiDesc& e = p.e;
   const bool full = n + 32 <= p.N;
-  if (KIND == kEpiF32 || KIND == kEpiGeluSplit) {
+  if (KIND == kEpiF32 || KIND == kEpiF32Lse || KIND == kEpiGeluSplit) {
     float* dst = e.C + (KIND == kEpiF32 ? mo : m) * e.ldc + n;
     if (full && ((e.ldc & 3) == 0) && (((uintptr_t)e.C & 15) == 0)) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     } else {
+#pragma unroll
       for (int q = 0; q < 32; ++q)
         if (n + q < p.N) dst[q] = v[q];
     }
@@ -89,6 +96,7 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
         reinterpret_cast<uint4*>(dst)[q] = u;
       }
     } else {
+#pragma unroll
       for (int q = 0; q < 32; ++q)
         if (n + q < p.N) dst[q] = __float2bfloat16_rn(v[q]);
     }
@@ -97,7 +105,7 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
     __nv_bfloat16* hi = e.Cb + m * e.ldcb + n;
     __nv_bfloat16* lo = hi + e.split;
     const __nv_bfloat16* r = KIND == kEpiResidSplit ? (const __nv_bfloat16*)e.resid + m * e.ldr + n : nullptr;
-#pragma unroll 4
+#pragma unroll
     for (int q = 0; q < 32; ++q) {
       if (n + q < p.N) {
         const double x = KIND == kEpiGeluSplit ? gelu64((double)v[q])
@@ -125,6 +133,7 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
         reinterpret_cast<uint4*>(lo)[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
     } else {
+#pragma unroll
       for (int q = 0; q < 32; ++q)
         if (n + q < p.N) split_bf16((double)v[q], hi + q, lo + q);
     }
@@ -160,22 +169,25 @@ __device__ __forceinline__ float expm1_guarded(float x) {
   return expm1f(x);
 }
 
-// Reward epilogue of 32 columns of row m (token t, target column yt): returns
-// sum_n P[t, n] expm1(dz_n) and records dz at the target column.
-__device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int64_t t, int32_t yt,
-                                          int64_t n, const float* v) {
-  const float* prow = p.e.P + t * p.N + n;
+// Reward epilogue of 32 columns of row m (target column yt): returns
+// sum_n P[t, n] expm1(dz_n) and records dz at the target column. prow points
+// at P[t, n]: a staged shared-memory copy (zero past column N) when `staged`,
+// else the row in global memory.
+__device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int32_t yt, int64_t n,
+                                          const float* prow, bool staged, const float* v) {
   float s = 0.0f;
-  if (n + 32 <= p.N && (p.N & 3) == 0) {
+  if (staged || (n + 32 <= p.N && (p.N & 3) == 0)) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const float4 pv = __ldg(reinterpret_cast<const float4*>(prow) + q);
+      const float4 pv = staged ? reinterpret_cast<const float4*>(prow)[q]
+                               : __ldg(reinterpret_cast<const float4*>(prow) + q);
       s = fmaf(pv.x, expm1_guarded(v[4 * q + 0]), s);
       s = fmaf(pv.y, expm1_guarded(v[4 * q + 1]), s);
       s = fmaf(pv.z, expm1_guarded(v[4 * q + 2]), s);
       s = fmaf(pv.w, expm1_guarded(v[4 * q + 3]), s);
     }
   } else {
+#pragma unroll
     for (int q = 0; q < 32; ++q)
       if (n + q < p.N) s = fmaf(prow[q], expm1_guarded(v[q]), s);
   }
@@ -198,6 +210,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
   const uint32_t sA = base;                           // STAGES x A tile
   const uint32_t sB = base + STAGES * A_BYTES;        // STAGES x B tile
   Shared* sh = reinterpret_cast<Shared*>(basep + STAGES * STAGE_BYTES);
+  float* pstage = reinterpret_cast<float*>(basep + STAGES * STAGE_BYTES + 256);
   volatile int* abort = &sh->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -233,8 +246,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      bool armed[STAGES] = {};
-      uint32_t armed_parity[STAGES] = {};
+      uint32_t armed = 0, armed_parity = 0;  // bit s: stage s holds a copy / its parity
       for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
         int m_blk, n_blk;
         tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
@@ -244,8 +256,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           ptx::mbar_expect_tx(fb, STAGE_BYTES);
           ptx::tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, m_blk * BM, fb);
           ptx::tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, n_blk * BN, fb);
-          armed[stage] = true;
-          armed_parity[stage] = phase;
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -255,8 +267,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       // every copy this thread issued has landed before the CTA can exit
       int dummy = 0;
       for (int s = 0; s < STAGES; ++s)
-        if (armed[s])
-          wait_bounded(ptx::smem_u32(&sh->full[s]), armed_parity[s], &dummy, p.status);
+        if ((armed >> s) & 1u)
+          wait_bounded(ptx::smem_u32(&sh->full[s]), (armed_parity >> s) & 1u, &dummy, p.status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -310,10 +322,41 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      int m_blk, n_blk;
+      tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
+      // Reward: stage P[t, n-tile] of this warp's tokens while the tile's MMAs
+      // run (each row otherwise waits on its own global loads chunk by chunk).
+      bool staged = false;
+      int64_t t_first = 0;
+      float* stg = pstage + ((warp - 2) * 2 + acc) * PSTAGE_FLOATS;
+      if (KIND == kEpiReward) {
+        const int64_t m_first = (int64_t)m_blk * BM + quad * 32;
+        if (m_first < p.M && (p.N & 3) == 0) {
+          const int64_t m_last = min(m_first + 31, p.M - 1);
+          t_first = p.e.t0 + m_first / p.e.draws;
+          const int64_t t_last = p.e.t0 + m_last / p.e.draws;
+          staged = t_last - t_first <= 1;
+          if (staged) {
+            float4 pv[PSTAGE_FLOATS / 128];
+#pragma unroll
+            for (int j = 0; j < PSTAGE_FLOATS / 128; ++j) {
+              const int q = lane + 32 * j;  // float4 index: token q / (BN/4), column 4 (q % (BN/4))
+              const int64_t t = t_first + q / (BN / 4);
+              const int64_t n = (int64_t)n_blk * BN + 4 * (q % (BN / 4));
+              pv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (t <= t_last && n < p.N)
+                pv[j] = __ldg(reinterpret_cast<const float4*>(p.e.P + t * p.N + n));
+            }
+            __syncwarp();  // the previous tile that used this buffer is done
+#pragma unroll
+            for (int j = 0; j < PSTAGE_FLOATS / 128; ++j)
+              reinterpret_cast<float4*>(stg)[lane + 32 * j] = pv[j];
+            __syncwarp();
+          }
+        }
+      }
       if (!wait_bounded(ptx::smem_u32(&sh->tfull[acc]), acc_phase, abort, p.status)) break;
       ptx::tc_fence_after();
-      int m_blk, n_blk;
-        tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
       const int64_t m = (int64_t)m_blk * BM + row;
       int64_t mo = m;
       if (p.e.c_row_mul != 0 && m < p.M)
@@ -328,17 +371,36 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
         if (yt < 0 || (int64_t)yt >= p.N) yt = 0;  // reported by the loss kernel
       }
       float s_row = 0.0f;
+      float rmax = -FLT_MAX, rsum = 0.0f;  // kEpiF32Lse: online softmax partial of the row
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int64_t n = (int64_t)n_blk * BN + c * 32;
         float v[32];
         ptx::tmem_ld32(taddr + (uint32_t)(c * 32), v);
         if (KIND == kEpiReward) {
-          if (m < p.M && n < p.N) s_row += reward32(p, m, t_row, yt, n, v);
+          if (m < p.M && n < p.N) {
+            const float* prow = staged ? stg + (t_row - t_first) * BN + c * 32
+                                       : p.e.P + t_row * p.N + n;
+            s_row += reward32(p, m, yt, n, prow, staged, v);
+          }
         } else if (m < p.M && n < p.N) {
           epilogue32<KIND>(p, m, mo, n, v);
+          if (KIND == kEpiF32Lse) {
+            float cm = -FLT_MAX;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (n + q < p.N) cm = fmaxf(cm, v[q]);
+            const float nm = fmaxf(rmax, cm);
+            float cs = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (n + q < p.N) cs += __expf(v[q] - nm);
+            rsum = fmaf(rsum, __expf(rmax - nm), cs);
+            rmax = nm;
+          }
         }
       }
+      if (KIND == kEpiF32Lse && m < p.M) p.e.lsep[m * p.n_tiles + n_blk] = make_float2(rmax, rsum);
       if (KIND == kEpiReward && m < p.M) p.e.part[m * p.n_tiles + n_blk] = s_row;
       ptx::tc_fence_before();
       __syncwarp();
@@ -403,9 +465,11 @@ bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
   if (g.M > (int64_t)INT32_MAX || g.N > (int64_t)INT32_MAX || g.K > (int64_t)INT32_MAX) return false;
   if (e.kind == kEpiResidSplit && !e.resid) return false;
   if (e.kind == kEpiReward && (!e.P || !e.y || !e.part || !e.dzy || e.draws < 1)) return false;
+  if (e.kind == kEpiF32Lse && !e.lsep) return false;
   if (!encode_fn()) return false;
   return e.kind == kEpiF32 || e.kind == kEpiBF16 || e.kind == kEpiGeluSplit ||
-         e.kind == kEpiResidSplit || e.kind == kEpiSplit || e.kind == kEpiReward;
+         e.kind == kEpiResidSplit || e.kind == kEpiSplit || e.kind == kEpiReward ||
+         e.kind == kEpiF32Lse;
 }
 
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
@@ -430,6 +494,7 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e,
     case kEpiResidSplit: return launch_kind<kEpiResidSplit>(st, ma, mb, p, sm_count);
     case kEpiSplit: return launch_kind<kEpiSplit>(st, ma, mb, p, sm_count);
     case kEpiReward: return launch_kind<kEpiReward>(st, ma, mb, p, sm_count);
+    case kEpiF32Lse: return launch_kind<kEpiF32Lse>(st, ma, mb, p, sm_count);
   }
   return cudaErrorInvalidValue;
 }

@@ -186,9 +186,9 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   ep.kind = kEpiF32; ep.C = Z; ep.ldc = p.V;
   if (e == cudaSuccess) e = launch_gemm_simt(st, g, ep);
   if (e == cudaSuccess)
-    e = launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, lse, loss, true, status);
+    e = launch_lse_rows(st, Z, p.T, p.V, targets, subset ? a_inv : 0, lse, loss, subset, status);
   if (!subset) {
-    if (e == cudaSuccess) e = launch_full_reward_partial(st, p, Z, targets, part, xy);
+    if (e == cudaSuccess) e = launch_full_reward_partial(st, p, Z, lse, targets, part, xy);
     if (e == cudaSuccess) e = launch_full_reward_combine(st, p, part, xy, r);
     if (e == cudaSuccess) e = launch_full_g(st, p, r, g_out, gop);
   } else if (e == cudaSuccess) {

@@ -55,8 +55,8 @@ __global__ void k_debug_gauss(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
 __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off, uint32_t i_off,
                                                          uint32_t ctr3, int64_t nt, int64_t ni,
                                                          int64_t nslots, float* __restrict__ out) {
-  __shared__ float2 tab[kSinCosTableAlloc];
-  fill_sincos_table(tab);
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab, 1.0f);
   __syncthreads();
   const int64_t nblk = (nslots + 127) / 128;
   const int64_t total = nt * ni * nblk * 32;
@@ -69,7 +69,7 @@ __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off
     const int64_t i = rest % ni;
     const int64_t t = rest / ni;
     U4 c{slot_ctr0((uint32_t)blk, lane), t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3};
-    const G4 g = gauss4_tab(philox10(c, key.k0, key.k1), 1.0f, tab);
+    const G4 g = gauss4_tab(philox10(c, key.k0, key.k1), tab);
     float* row = out + (t * ni + i) * nslots;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -77,6 +77,40 @@ __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off
       if (k < nslots) row[k] = g.v[j];
     }
   }
+}
+
+// Every value of the two Box-Muller inputs: radius(j) for u1 = (j + 1) 2^-24
+// and (cos, sin) of 2 pi m 2^-24, with the device functions the kernels use.
+__global__ void k_debug_bm_radius(float sigma, float* __restrict__ out) {
+  const uint32_t j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < (1u << 24)) out[j] = sigma * bm_radius(j << 8);
+}
+
+__global__ __launch_bounds__(256) void k_debug_bm_angle(int method, float* __restrict__ out) {
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab, 1.0f);
+  __syncthreads();
+  for (uint32_t m = blockIdx.x * blockDim.x + threadIdx.x; m < (1u << 24);
+       m += gridDim.x * blockDim.x) {
+    float s, c;
+    if (method == 1) {
+      const float2 cs = rotate_tab(m << 8, tab);
+      c = cs.x;
+      s = cs.y;
+    } else {
+      sincos_turn24(m, &s, &c);
+    }
+    out[2 * (size_t)m] = c;
+    out[2 * (size_t)m + 1] = s;
+  }
+}
+
+cudaError_t launch_debug_bm(cudaStream_t st, int what, float sigma, float* out) {
+  if (what == 0)
+    k_debug_bm_radius<<<(1u << 24) / 256, 256, 0, st>>>(sigma, out);
+  else
+    k_debug_bm_angle<<<4096, 256, 0, st>>>(what == 2 ? 1 : 0, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, int64_t nt,

@@ -24,13 +24,16 @@
 // block (they depend on the draw index or on the slot block only).
 //
 // Accumulation (INT = true): off-target coordinates accumulate r * sigma eps
-// in 2^-16 fixed point (scaled by 1/sigma^2) with native int32 shared-memory
-// atomics; sums wrap modulo 2^32, so only the final per-coordinate sum has to
-// fit, which holds with a wide margin for K <= 65536 (each term is bounded by
-// 66.6 and its mean by max_j p_j; the scale shrinks as 16384/K above 16384
-// draws). The target coordinate, which collects all K draws, keeps an fp32
-// accumulator per warp. INT = false accumulates in fp32 (compare-and-swap
-// atomics) for larger K.
+// in 2^-15 fixed point (scaled by 1/sigma^2) with native int32 shared-memory
+// atomics. |r| <= 11.54 sigma and |sigma eps| <= 5.77 sigma bound a term by
+// 66.6 units-of-one, 2.2e6 < 2^22 fixed-point units, so the rounding to an
+// integer is the exponent-bias construction fma(x, scale, 1.5 2^23) (the FMA
+// pipe rounds to nearest, no conversion instruction). Sums wrap modulo 2^32,
+// so only the final per-coordinate sum has to fit, which holds with a wide
+// margin for K <= 65536 (a coordinate lies in about K S / V windows, and the
+// scale shrinks as 16384/K above 16384 draws). The target coordinate, which
+// collects all K draws, keeps an fp32 accumulator per warp. INT = false
+// accumulates in fp32 (compare-and-swap atomics) for larger K.
 #include <cooperative_groups.h>
 
 #include "internal.cuh"
@@ -85,7 +88,8 @@ __device__ __forceinline__ uint32_t mulmod32(uint32_t x, uint32_t y, uint32_t m,
 template <bool INT>
 __device__ __forceinline__ void accumulate(float* slot, float r, float x, float acc_scale) {
   if (INT)
-    atomicAdd(reinterpret_cast<int*>(slot), __float2int_rn(r * acc_scale * x));
+    atomicAdd(reinterpret_cast<int*>(slot),
+              __float_as_int(fmaf(r * acc_scale, x, 12582912.0f)) - 0x4B400000);
   else
     atomicAdd(slot, r * x);
 }
@@ -96,8 +100,8 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_next;    // next draw batch of the current token
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
-  __shared__ float2 s_tab[kSinCosTableAlloc];
-  fill_sincos_table(s_tab);
+  __shared__ float2 s_tab[kSinCosTable];
+  fill_sincos_table(s_tab, A.sigma);
   __syncthreads();
   cg::cluster_group cluster = cg::this_cluster();
   const uint32_t rank = CS > 1 ? cluster.block_rank() : 0;
@@ -181,7 +185,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         if (mine && kyq >= (uint32_t)S) {
           const U4 w = philox_from2(bs, draw_const(A.keys, t_abs, i_abs), A.keys);
           const float2 nn =
-              box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, A.sigma, s_tab);
+              box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, s_tab);
           x_extra = (s_word & 1u) ? nn.y : nn.x;
         }
       }
@@ -210,7 +214,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
             }
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), A.sigma, s_tab);
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
@@ -222,7 +226,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset2(const __grid_constant__
         } else {
 #pragma unroll
           for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), A.sigma, s_tab);
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int k = m * 128 + lane + 32 * j;
@@ -372,7 +376,7 @@ cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, i
 // Cluster size the shared-memory kernel would use (0: not applicable).
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
   if (S < 1 || S > 512) return 0;
-  const int64_t slack = 1024 + 8 * kSinCosTableAlloc;  // static: counters, angle table
+  const int64_t slack = 1024 + 8 * kSinCosTable;  // static: counters, angle table
   if (2 * V * 4 + slack <= max_smem_optin && V <= 65536) return 1;
   const int64_t seg = ((V + 1) / 2 + 3) / 4 * 4;
   if (2 * seg * 4 + slack <= max_smem_optin && S <= V - seg && S <= seg && V <= 65536) return 2;
@@ -405,8 +409,8 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   // the accumulators hold sum r (sigma eps): g = -(1/(K sigma)) sum r eps
   const double s2 = (double)p.sigma * (double)p.sigma;
   A.fac = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * s2)) : 0.0f;
-  // fixed point: 2^16 units per unit of r eps / sigma, fewer above 16384 draws
-  const double units = 65536.0 * (p.K > 16384 ? 16384.0 / (double)p.K : 1.0);
+  // fixed point: 2^15 units per unit of r eps / sigma, fewer above 16384 draws
+  const double units = 32768.0 * (p.K > 16384 ? 16384.0 / (double)p.K : 1.0);
   A.acc_scale = p.sigma > 0.0f ? (float)(units / s2) : 0.0f;
   A.fac_int = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * units)) : 0.0f;
   A.Z = Z;

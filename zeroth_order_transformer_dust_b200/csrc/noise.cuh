@@ -52,69 +52,6 @@ __device__ __forceinline__ U4 philox10(U4 c, uint32_t k0, uint32_t k1) {
   return c;
 }
 
-// (float)i for |i| < 2^22, exactly, by exponent-bias arithmetic on the ALU
-// pipe: 1.5 * 2^23 + i has i in its low mantissa bits.
-__device__ __forceinline__ float small_int_to_float(int i) {
-  return __int_as_float(0x4B400000 + i) - 12582912.0f;
-}
-
-// -ln(u) for u in (0, 1], accurate to a few ulp relative to the result,
-// including u -> 1. u = 2^e m with m in [sqrt(1/2), sqrt(2)): subtracting the
-// bit pattern of sqrt(1/2) before extracting the exponent lands m in that
-// range without a branch. ln m is 2 atanh(s), s = (m-1)/(m+1), |s| <= 0.1716,
-// from its Taylor series 2 s (1 + s^2/3 + s^4/5 + s^6/7) (truncation below
-// 3e-8 absolute, vanishing as m -> 1); e ln 2 uses ln 2 split in a high part
-// with 8 trailing zero bits (exact products for |e| <= 2^8) and a low
-// correction (Cody and Waite's argument reduction).
-__device__ __forceinline__ float neg_log_unit(float u) {
-  const int bits = __float_as_int(u);
-  const int e = (bits - 0x3f3504f3) >> 23;  // arithmetic shift: floor
-  const float m = __int_as_float(bits - (e << 23));
-  const float f = m - 1.0f;  // exact (Sterbenz)
-  const float s = __fdividef(f, m + 1.0f);
-  const float w = s * s;
-  float poly = fmaf(w, 2.0f / 7.0f, 2.0f / 5.0f);
-  poly = fmaf(w, poly, 2.0f / 3.0f);
-  poly = fmaf(w, poly, 2.0f);
-  const float ln_m = s * poly;
-  const float fe = small_int_to_float(e);
-  const float kLn2Hi = 0.693145751953125f;        // 0x3f317200
-  const float kLn2Lo = 1.428606765330187e-06f;    // ln 2 - kLn2Hi
-  const float ln_u = fmaf(fe, kLn2Hi, fmaf(fe, kLn2Lo, ln_m));
-  return -ln_u;
-}
-
-// -ln(j 2^-24) for an integer j in [1, 2^24], the same computation as
-// neg_log_unit with the 2^-24 scale folded into the exponent (the float of j
-// is exact, and e - 24 comes out of the same exponent-bias subtraction).
-__device__ __forceinline__ float neg_log_u24(uint32_t j) {
-  const int bits = __float_as_int((float)j);
-  const int e = (bits - 0x3f3504f3) >> 23;
-  const float m = __int_as_float(bits - (e << 23));
-  const float f = m - 1.0f;  // exact (Sterbenz)
-  const float s = __fdividef(f, m + 1.0f);
-  const float w = s * s;
-  float poly = fmaf(w, 2.0f / 7.0f, 2.0f / 5.0f);
-  poly = fmaf(w, poly, 2.0f / 3.0f);
-  poly = fmaf(w, poly, 2.0f);
-  const float ln_m = s * poly;
-  const float fe = __int_as_float(0x4B400000 + e) - 12582936.0f;  // e - 24, exact
-  const float kLn2Hi = 0.693145751953125f;
-  const float kLn2Lo = 1.428606765330187e-06f;
-  return -fmaf(fe, kLn2Hi, fmaf(fe, kLn2Lo, ln_m));
-}
-
-// sqrt(x) for x >= 0: the hardware reciprocal-square-root estimate y refined
-// by one Newton-Raphson step on r = x y (r' = r + (y/2)(x - r^2)), which
-// leaves about one ulp of error. x is clamped away from 0 (sqrt(0) -> 1e-15).
-__device__ __forceinline__ float sqrt_newton(float x) {
-  const float xs = fmaxf(x, 1e-30f);
-  const float y = rsqrtf(xs);
-  const float r = xs * y;
-  const float e = fmaf(-r, r, xs);
-  return fmaf(0.5f * y, e, r);
-}
-
 // cos and sin of 2 pi m 2^-24 for an integer m in [0, 2^24). The nearest
 // quarter turn is removed exactly in integer arithmetic, leaving
 // |x| <= pi/4, where the Taylor series of sin (to x^9) and cos (to x^8) are
@@ -141,49 +78,73 @@ __device__ __forceinline__ void sincos_turn24(uint32_t m, float* s_out, float* c
   *c_out = c;
 }
 
+// Radius of the Box-Muller pair, R = sqrt(-2 ln u1), for
+// u1 = ((wa >> 8) + 1) 2^-24 (exact in fp32). Away from u1 = 1, ln u1 comes
+// from the hardware base-2 logarithm of u1 (MUFU.LG2); as u1 -> 1 the
+// logarithm is small and that estimate loses its relative accuracy, so for
+// v = 1 - u1 < 2^-7 (exact) the series -ln(1 - v) = v (1 + v/2 + v^2/3 +
+// v^3/4 + ...) is used instead, truncated below 2^-28 relative. The square
+// root is the hardware approximation (MUFU.SQRT, sqrt(0) = 0). Checked over
+// all 2^24 values of u1 against fp64: below 8e-7 absolute.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bm_radius(uint32_t wa) {
+  const float u = fmaf((float)(wa >> 8), 5.9604645e-08f, 5.9604645e-08f);  // exact
+  const float far = __log2f(u) * -1.3862944f;                             // -2 ln 2
+  const float v = 1.0f - u;  // exact (u >= 1/2 where it is used)
+  float c = fmaf(v, 0.25f, 1.0f / 3.0f);
+  c = fmaf(v, c, 0.5f);
+  c = fmaf(v, c, 1.0f);
+  const float near = (v + v) * c;
+  return sqrt_approx(v < 0.0078125f ? near : far);
+}
+
 // Box-Muller on 24-bit uniforms: u1 = ((wa>>8)+1) 2^-24, u2 = (wb>>8) 2^-24;
 // returns scale * (R cos 2 pi u2, R sin 2 pi u2), R = sqrt(-2 ln u1).
 __device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb, float scale = 1.0f) {
-  const float u1 = (float)((wa >> 8) + 1u) * 5.9604645e-08f;  // exact
-  const float radius = scale * sqrt_newton(2.0f * neg_log_unit(u1));
+  const float radius = scale * bm_radius(wa);
   float s, c;
   sincos_turn24(wb >> 8, &s, &c);
   return make_float2(radius * c, radius * s);
 }
 
-// Table-driven variant of the angle step, for kernels that keep a 1024-entry
-// table of roots of unity, tab[k] = (cos 2 pi k/1024, sin 2 pi k/1024), in
-// shared memory: the angle 2 pi m 2^-24 is split into the nearest table angle
-// plus a remainder |x| <= pi/1024, and cos/sin follow from the angle-addition
-// formulas with cos x = 1 - x^2/2 and sin x = x (truncation below 5e-9).
+// Table-driven variant of the angle step, for kernels that keep 1024 roots of
+// unity at interval midpoints, theta_k = 2 pi (k + 1/2) / 1024, in shared
+// memory, already scaled by sigma: tab[k] = sigma (cos theta_k, sin theta_k).
+// The 24-bit angle m = wb >> 8 is interval wb >> 22 plus the remainder
+// x = c xr, c = 2 pi 2^-32, xr = (r - 2^13) 2^8 with r bits 8..21 of wb
+// (|x| <= pi/1024; xr's float comes exactly from an exponent-bias
+// construction), and cos/sin follow from the angle-addition formulas with
+// cos x = 1 - x^2/2 and sin x = x (truncation below 5e-9). Checked over all
+// 2^24 angles (sigma = 1): below 2e-7 absolute.
 constexpr int kSinCosTable = 1024;
-constexpr int kSinCosTableAlloc = kSinCosTable + 1;  // entry 1024 repeats entry 0
 
-__device__ __forceinline__ void fill_sincos_table(float2* tab) {
-  for (int k = threadIdx.x; k < kSinCosTableAlloc; k += blockDim.x) {
+__device__ __forceinline__ void fill_sincos_table(float2* tab, float sigma) {
+  for (int k = threadIdx.x; k < kSinCosTable; k += blockDim.x) {
     float s, c;
-    sincospif((float)(k & (kSinCosTable - 1)) * (2.0f / kSinCosTable), &s, &c);
-    tab[k] = make_float2(c, s);
+    sincospif((float)(2 * k + 1) * (1.0f / kSinCosTable), &s, &c);
+    tab[k] = make_float2(sigma * c, sigma * s);
   }
 }
 
-__device__ __forceinline__ void sincos_turn24_tab(uint32_t m, const float2* tab, float* s_out,
-                                                  float* c_out) {
-  const uint32_t idx = (m + (1u << 13)) >> 14;             // nearest 1/1024 turn, 0..1024
-  const int r = (int)m - (int)(idx << 14);                  // [-2^13, 2^13)
-  const float x = small_int_to_float(r) * 3.7450702e-07f;   // 2 pi / 2^24
-  const float h = 0.5f * x * x;
-  const float2 t = tab[idx];
-  *c_out = fmaf(-t.y, x, fmaf(-t.x, h, t.x));
-  *s_out = fmaf(t.x, x, fmaf(-t.y, h, t.y));
+// sigma (cos, sin) of the angle of word wb.
+__device__ __forceinline__ float2 rotate_tab(uint32_t wb, const float2* tab) {
+  // 1.5 2^23 + (r << 8) minus (1.5 2^23 + 2^21): (r - 2^13) 2^8, exact
+  const float xr = __int_as_float((wb & 0x003FFF00u) | 0x4B400000u) - 14680064.0f;
+  const float x = xr * 1.4629181e-09f;  // 2 pi 2^-32
+  const float2 t = tab[wb >> 22];
+  const float q = fmaf(x * x, -0.5f, 1.0f);
+  return make_float2(fmaf(-t.y, x, t.x * q), fmaf(t.x, x, t.y * q));
 }
 
-__device__ __forceinline__ float2 box_muller_tab(uint32_t wa, uint32_t wb, float scale,
-                                                 const float2* tab) {
-  const float radius = scale * sqrt_newton(2.0f * neg_log_u24((wa >> 8) + 1u));
-  float s, c;
-  sincos_turn24_tab(wb >> 8, tab, &s, &c);
-  return make_float2(radius * c, radius * s);
+__device__ __forceinline__ float2 box_muller_tab(uint32_t wa, uint32_t wb, const float2* tab) {
+  const float R = bm_radius(wa);
+  const float2 cs = rotate_tab(wb, tab);
+  return make_float2(R * cs.x, R * cs.y);
 }
 
 // Four Gaussians of one counter (times `scale`): element j is output word j.
@@ -191,9 +152,9 @@ struct G4 {
   float v[4];
 };
 
-__device__ __forceinline__ G4 gauss4_tab(U4 w, float scale, const float2* tab) {
-  const float2 a = box_muller_tab(w.x, w.y, scale, tab);
-  const float2 b = box_muller_tab(w.z, w.w, scale, tab);
+__device__ __forceinline__ G4 gauss4_tab(U4 w, const float2* tab) {
+  const float2 a = box_muller_tab(w.x, w.y, tab);
+  const float2 b = box_muller_tab(w.z, w.w, tab);
   G4 g;
   g.v[0] = a.x;
   g.v[1] = a.y;
