@@ -37,10 +37,11 @@ from .philox import (  # noqa: F401
     TAG_HEAD,
     TAG_SUBSET_OFFSET,
     TAG_MLP_UP,
+    TAG_MLP_DOWN,
 )
 from .params import Params  # noqa: F401
 from .head import (  # noqa: F401
     clean_head, head_grad, head_linear_estimate, full_vocab_draws, subset_draws,
 )
-from .mlp import clean_mlp, mlp_grad, mlp_draws, gelu  # noqa: F401
+from .mlp import clean_mlp, mlp_grad, mlp_draws, gelu, mlp_down_grad, mlp_down_draws  # noqa: F401
 from .optim import sgd_momentum, train_head, exact_weight_grad  # noqa: F401

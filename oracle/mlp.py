@@ -30,7 +30,7 @@ import numpy as np
 from scipy.special import erf
 
 from .params import Params
-from .philox import TAG_MLP_UP, gaussians
+from .philox import TAG_MLP_DOWN, TAG_MLP_UP, gaussians
 
 
 def gelu(x: np.ndarray) -> np.ndarray:
@@ -90,3 +90,48 @@ def mlp_grad(X, W_up, W_down, W_head, targets, prm: Params, draw_chunk: int = 64
     G = np.einsum("tc,td->cd", g, X)
     return {"loss": clean["loss"], "lse": clean["lse"], "rewards": rewards, "g": g, "G": G,
             "u": u, "p": p, "z": clean["z"]}
+
+
+# --------------------------------------------------------------------------
+# Down-projection variant: the perturbed layer is y = W_down a (d outputs per
+# token, a = GELU(u) its cached input). The same pages' reading (one layer
+# type per pass, only what the perturbation changes recomputed): sigma eps
+# adds to the block output h, so the head sees dz = sigma eps W_head^T and
+#   r   = dz_y - log1p(sum_j p_j expm1(dz_j)),
+#   g_t = -(1/(K sigma)) sum_i r_i eps_i      (d entries),
+#   G_down = sum_t g_t a_t^T                  (d x d_ff).
+
+def mlp_down_draws(p_t, y_t, eps, W_head, sig):
+    """Rewards and sum_i r_i eps_i for n draws of noise ``eps`` (n, d) on W_down's output."""
+    dz = (sig * eps) @ W_head.T
+    r = dz[:, y_t] - np.log1p((p_t[None, :] * np.expm1(dz)).sum(axis=1))
+    acc = (r[:, None] * eps).sum(axis=0)
+    return r, acc
+
+
+def mlp_down_grad(X, W_up, W_down, W_head, targets, prm: Params, draw_chunk: int = 256) -> dict:
+    Wh = np.asarray(W_head, dtype=np.float64)
+    y = np.asarray(targets, dtype=np.int64)
+    clean = clean_mlp(X, W_up, W_down, W_head, y)
+    a, p = clean["a"], clean["p"]
+    T = a.shape[0]
+    d = Wh.shape[1]
+    sig = prm.sigma32
+    rewards = np.zeros((T, prm.K))
+    g = np.zeros((T, d))
+    for t in range(T):
+        t_abs = t + prm.token_offset
+        for i0 in range(0, prm.K, draw_chunk):
+            i1 = min(prm.K, i0 + draw_chunk)
+            draws = np.arange(i0, i1, dtype=np.int64) + prm.draw_offset
+            eps = gaussians(prm.seed, t_abs, draws, np.arange(d), TAG_MLP_DOWN, prm.stream_id)
+            r, acc = mlp_down_draws(p[t], y[t], eps, Wh, sig)
+            rewards[t, i0:i1] = r
+            g[t] += acc
+    if sig == 0.0:
+        g[:] = 0.0
+    else:
+        g *= -1.0 / (prm.K * sig)
+    G = np.einsum("tc,tf->cf", g, a)
+    return {"loss": clean["loss"], "lse": clean["lse"], "rewards": rewards, "g": g, "G": G,
+            "a": a, "p": p, "z": clean["z"]}

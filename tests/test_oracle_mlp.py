@@ -111,3 +111,72 @@ def test_estimate_converges_with_population():
         errs.append(np.linalg.norm(G - gW) / np.linalg.norm(gW))
     assert errs[1] < errs[0] / 2.5
     assert errs[1] < 0.25
+
+
+# ---- down-projection variant ----------------------------------------------
+
+def _dL_dh(X, W_up, W_down, W_head, y):
+    """dL/dh for every token from torch autograd (h detached as a leaf)."""
+    t = {k: torch.tensor(v, dtype=torch.float64) for k, v in
+         dict(X=X, W_up=W_up, W_down=W_down, W_head=W_head).items()}
+    a = torch.nn.functional.gelu(t["X"] @ t["W_up"].T, approximate="none")
+    h = (t["X"] + a @ t["W_down"].T).detach().requires_grad_(True)
+    loss = torch.nn.functional.cross_entropy(h @ t["W_head"].T, torch.tensor(y), reduction="sum")
+    loss.backward()
+    return h.grad.numpy()
+
+
+def test_down_estimate_is_unbiased_exact_expectation():
+    """Over +-sqrt(d) e_m noise on W_down's output, g equals dL/dh (to O(sigma^2))."""
+    X, Wu, Wd, Wh, y = _mlp_problem(T=3)
+    gh = _dL_dh(X, Wu, Wd, Wh, y)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y)
+    d = Wh.shape[1]
+    eps = np.concatenate([np.eye(d), -np.eye(d)]) * math.sqrt(d)
+    sig = 1e-6
+    for t in range(3):
+        r, acc = oracle.mlp_down_draws(c["p"][t], y[t], eps, Wh, sig)
+        np.testing.assert_allclose(-acc / (eps.shape[0] * sig), gh[t], rtol=0, atol=1e-8)
+
+
+def test_down_weight_gradient_matches_finite_differences_and_autograd():
+    """sum_t dL/dh_t a_t^T against brute-force differences of the summed loss in W_down."""
+    X, Wu, Wd, Wh, y = _mlp_problem(T=3, d=3, d_ff=4, V=5)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y)
+    closed = _dL_dh(X, Wu, Wd, Wh, y).T @ c["a"]
+    fd = np.zeros_like(Wd)
+    h = 1e-5
+    for i in range(Wd.shape[0]):
+        for j in range(Wd.shape[1]):
+            P, M = Wd.copy(), Wd.copy()
+            P[i, j] += h
+            M[i, j] -= h
+            fd[i, j] = (oracle.clean_mlp(X, Wu, P, Wh, y)["loss"].sum()
+                        - oracle.clean_mlp(X, Wu, M, Wh, y)["loss"].sum()) / (2 * h)
+    np.testing.assert_allclose(fd, closed, rtol=0, atol=1e-8)
+    _, gW = _torch_loss(X, Wu, Wd, Wh, y, wrt="W_down")
+    np.testing.assert_allclose(gW, closed, rtol=0, atol=1e-12)
+
+
+def test_down_sigma_zero_and_noise_stream():
+    X, Wu, Wd, Wh, y = _mlp_problem()
+    prm = oracle.Params(T=4, d=5, V=9, d_ff=7, K=6, sigma=0.0, seed=2)
+    out = oracle.mlp_down_grad(X, Wu, Wd, Wh, y, prm)
+    assert np.all(out["rewards"] == 0.0) and np.all(out["G"] == 0.0)
+    # the down-projection draws its noise from its own counter tag
+    e_up = oracle.gaussians(2, 0, np.arange(3), np.arange(5), oracle.TAG_MLP_UP)
+    e_dn = oracle.gaussians(2, 0, np.arange(3), np.arange(5), oracle.TAG_MLP_DOWN)
+    assert not np.allclose(e_up, e_dn)
+
+
+def test_down_estimate_converges_with_population():
+    X, Wu, Wd, Wh, y = _mlp_problem(T=4, d=4, d_ff=6, V=7, seed=3)
+    _, gW = _torch_loss(X, Wu, Wd, Wh, y, wrt="W_down")
+    errs = []
+    for K in (256, 4096):
+        prm = oracle.Params(T=4, d=4, V=7, d_ff=6, K=K, sigma=1e-4, seed=8)
+        G = oracle.mlp_down_grad(X, Wu, Wd, Wh, y, prm, draw_chunk=4096)["G"]
+        assert G.shape == Wd.shape
+        errs.append(np.linalg.norm(G - gW) / np.linalg.norm(gW))
+    assert errs[1] < errs[0] / 2.5
+    assert errs[1] < 0.25
