@@ -131,8 +131,9 @@ def _oracle_tokens(args):
         for t in toks:
             prm = oracle.Params(T=1, d=wl.d, V=wl.V, d_ff=wl.d_ff, K=wl.K, sigma=wl.sigma,
                                 seed=wl.seed, token_offset=t)
-            oracle.mlp_grad(inp["X"][t:t + 1], inp["W_up"], inp["W_down"], inp["W_head"],
-                            inp["targets"][t:t + 1], prm)
+            fn = oracle.mlp_down_grad if wl.variant == "mlp_down" else oracle.mlp_grad
+            fn(inp["X"][t:t + 1], inp["W_up"], inp["W_down"], inp["W_head"],
+               inp["targets"][t:t + 1], prm)
     return len(toks), time.perf_counter() - t0
 
 
@@ -279,12 +280,15 @@ def run_dust(args):
         X, Wu, Wdn, Wh = (torch.from_numpy(inp[k]).to(torch.bfloat16).to(dev)
                           for k in ("X", "W_up", "W_down", "W_head"))
         yd = torch.from_numpy(inp["targets"]).to(torch.int32).to(dev)
-        outs = {"G": torch.empty(wl.d_ff, wl.d, dtype=torch.float32, device=dev),
+        gshape = (wl.d_ff, wl.d) if wl.variant == "mlp" else (wl.d, wl.d_ff)
+        outs = {"G": torch.empty(*gshape, dtype=torch.float32, device=dev),
                 "loss": torch.empty(wl.T, dtype=torch.float32, device=dev)}
+
+        layer = "down" if wl.variant == "mlp_down" else "up"
 
         def step():
             ctx.mlp_grad(X, Wu, Wdn, Wh, yd, K=wl.K, sigma=wl.sigma, seed=wl.seed,
-                         token_offset=t_off, out=outs)
+                         token_offset=t_off, out=outs, layer=layer)
             from zeroth_order_transformer_dust_b200.parallel import allreduce_weight_grad
             allreduce_weight_grad(outs["G"])
 

@@ -143,8 +143,9 @@ dust_status dust_head_grad_host(dust_ctx* ctx, const dust_params* p,
  * u = x W_up^T (d_ff entries per token); each draw recomputes
  * GELU(u + sigma eps) - GELU(u), the down-projection and the head from the
  * cached x, u and clean logits (exact-erf GELU, residual h = x + a W_down^T,
- * no norm, no bias; bf16 workloads round a, h and the per-draw deltas to bf16
- * as GEMM operands).
+ * no norm, no bias). Inputs are bf16; the activations a, h and the per-draw
+ * deltas enter the tensor-core GEMMs as bf16 hi/lo planes (about 2^-17
+ * relative), against weights duplicated along the contraction.
  *   X        T x d     input, dtype        W_up   d_ff x d   dtype
  *   W_down   d x d_ff  dtype               W_head V x d      dtype
  *   targets  T int32
@@ -159,6 +160,26 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* p,
                           const void* W_head, const int32_t* targets,
                           float* G_up_out, float* loss_out, float* rewards_out,
                           float* g_out);
+
+/*
+ * Hidden-MLP down-projection estimator (same pages and sections as
+ * dust_mlp_grad, the next layer type of the block). Noise goes on
+ * W_down's output (d entries per token), which is the block output h, so each
+ * draw recomputes only the head: dz = sigma eps W_head^T (sigma eps enters the
+ * tensor-core GEMM as bf16 hi/lo planes), r = dz_y - log1p(sum p expm1(dz)),
+ * g_t = -(1/(K sigma)) sum_i r_i eps_i, and the weight gradient is taken
+ * against the layer's cached input a = GELU(u) (fp32, CUDA cores).
+ *   arguments and layouts as dust_mlp_grad, except
+ *   G_down_out d x d_ff fp32 sum_t g_t a_t^T   (or NULL)
+ *   g_out      T x d    fp32                    (or NULL)
+ * Its noise has its own counter tag (3), distinct from the up-projection's.
+ * Same validation and errors as dust_mlp_grad.
+ */
+dust_status dust_mlp_down_grad(dust_ctx* ctx, const dust_params* p,
+                               const void* X, const void* W_up, const void* W_down,
+                               const void* W_head, const int32_t* targets,
+                               float* G_down_out, float* loss_out, float* rewards_out,
+                               float* g_out);
 
 /* Per-stage device timing: when enabled, each call records CUDA events on
    the context's stream between its stages (clean GEMM, log-sum-exp, draws,

@@ -27,7 +27,7 @@ import numpy as np
 @dataclass(frozen=True)
 class Workload:
     name: str
-    variant: str        # "head" or "mlp"
+    variant: str        # "head", "mlp" (up-projection) or "mlp_down"
     T: int
     d: int
     V: int
@@ -60,6 +60,9 @@ CONFIGS = {
     # Hidden MLP up-projection.
     "mlp_bf16": Workload("mlp_bf16", "mlp", T=8192, d=768, V=50304, K=256, S=0,
                          sigma=1e-2, seed=3, dtype="bf16", targets="zipf", d_ff=3072),
+    # Hidden MLP down-projection (noise on W_down's output), same shapes.
+    "mlp_down_bf16": Workload("mlp_down_bf16", "mlp_down", T=8192, d=768, V=50304, K=256, S=0,
+                              sigma=1e-2, seed=3, dtype="bf16", targets="zipf", d_ff=3072),
     # LM head at 243M-model head scale, subset draws (S = 512), 16k draws.
     "large_subset_bf16": Workload("large_subset_bf16", "head", T=16384, d=1024, V=50304,
                                   K=16384, S=512, sigma=5e-3, seed=4, dtype="bf16",

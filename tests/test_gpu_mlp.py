@@ -64,3 +64,53 @@ def test_mlp_workload_slice(ctx):
     inp = synth.make_mlp_inputs(wl)
     got, ref = _run(ctx, inp, wl, t0=5000, T=3)
     _check(got, ref)
+
+
+# ---- down-projection variant ----------------------------------------------
+
+def _run_down(ctx, inp, wl, t0=0, T=None):
+    sl = slice(t0, t0 + (T or wl.T))
+    X = inp["X"][sl]
+    y = inp["targets"][sl]
+    out = ctx.mlp_grad(to_dev(X, "bf16"), to_dev(inp["W_up"], "bf16"), to_dev(inp["W_down"], "bf16"),
+                       to_dev(inp["W_head"], "bf16"), to_dev(y, "i32"), K=wl.K, sigma=wl.sigma,
+                       seed=wl.seed, token_offset=t0, want_rewards=True, want_g=True, layer="down")
+    torch.cuda.synchronize()
+    got = {k: np64(v) for k, v in out.items()}
+    prm = oracle.Params(T=X.shape[0], d=wl.d, V=wl.V, d_ff=wl.d_ff, K=wl.K, sigma=wl.sigma,
+                        seed=wl.seed, token_offset=t0)
+    ref = oracle.mlp_down_grad(X, inp["W_up"], inp["W_down"], inp["W_head"], y, prm)
+    return got, ref
+
+
+def _check_down(got, ref):
+    _check(got, ref)
+    # the weight gradient itself is an fp32 contraction: against g_gpu^T a in fp64
+    assert rel_fro(got["G"], got["g"].T @ ref["a"]) < 1e-5
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(T=1, K=1), dict(d=33, d_ff=200, V=517), dict(K=130),
+                                dict(sigma=0.1)])
+def test_small_mlp_down(ctx, kw):
+    base = dict(T=24, d=64, d_ff=256, V=1000, K=16, sigma=1e-2)
+    base.update(kw)
+    wl = synth.Workload("mlp_small", "mlp", S=0, seed=12, dtype="bf16", targets="zipf", **base)
+    inp = synth.make_mlp_inputs(wl)
+    got, ref = _run_down(ctx, inp, wl)
+    assert got["G"].shape == (wl.d, wl.d_ff) and got["g"].shape == (wl.T, wl.d)
+    _check_down(got, ref)
+
+
+def test_mlp_down_sigma_zero(ctx):
+    wl = synth.Workload("mlp_small", "mlp", T=8, d=32, d_ff=128, V=300, K=4, S=0, sigma=0.0,
+                        seed=2, dtype="bf16", targets="zipf")
+    inp = synth.make_mlp_inputs(wl)
+    got, _ = _run_down(ctx, inp, wl)
+    assert np.all(got["rewards"] == 0) and np.all(got["g"] == 0) and np.all(got["G"] == 0)
+
+
+def test_mlp_down_workload_slice(ctx):
+    wl = synth.CONFIGS["mlp_bf16"]
+    inp = synth.make_mlp_inputs(wl)
+    got, ref = _run_down(ctx, inp, wl, t0=5000, T=3)
+    _check_down(got, ref)

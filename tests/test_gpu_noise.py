@@ -89,7 +89,7 @@ def angle_err(ctx):
 def test_radius_all_inputs(radius_err):
     # a few 1e-7 everywhere, including u1 -> 1 where the radius -> 0
     assert radius_err.max() < 8e-7, radius_err.max()
-    assert radius_err[-(1 << 17):].max() < 1e-7      # the series branch, v < 2^-7
+    assert radius_err[-(1 << 18):].max() < 2e-7      # the series branch, v < 2^-6
 
 
 def test_radius_scales_with_sigma(ctx):

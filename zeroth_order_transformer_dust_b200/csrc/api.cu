@@ -271,7 +271,7 @@ void dust_destroy(dust_ctx* ctx) {
   Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
                  &ctx->gT, &ctx->hT, &ctx->xdup, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
-                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep};
+                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -457,9 +457,13 @@ dust_status dust_head_grad_host(dust_ctx* ctx, const dust_params* pp, const void
   return dust_check(ctx);
 }
 
-dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, const void* W_up,
-                          const void* W_down, const void* W_head, const int32_t* targets,
-                          float* G_up_out, float* loss_out, float* rewards_out, float* g_out) {
+// The two MLP variants share the clean pass and the reward GEMM: `down`
+// perturbs W_down's output (dh = sigma eps directly) instead of W_up's
+// (dh = (GELU(u + sigma eps) - GELU(u)) W_down^T).
+static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, const void* X,
+                            const void* W_up, const void* W_down, const void* W_head,
+                            const int32_t* targets, float* G_out, float* loss_out,
+                            float* rewards_out, float* g_out) {
   if (!ctx) return DUST_ERR_ARG;
   char why[256];
   if (check_params(pp, DUST_VARIANT_MLP, why, sizeof(why)) != DUST_OK)
@@ -468,7 +472,7 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   if (!X || !W_up || !W_down || !W_head || !targets)
     return fail(ctx, DUST_ERR_ARG, "X, W_up, W_down, W_head and targets must be non-NULL");
   if (!aligned(X, 16) || !aligned(W_up, 16) || !aligned(W_down, 16) || !aligned(W_head, 16) ||
-      !aligned(targets, 4) || !aligned(G_up_out, 4) || !aligned(loss_out, 4) ||
+      !aligned(targets, 4) || !aligned(G_out, 4) || !aligned(loss_out, 4) ||
       !aligned(rewards_out, 4) || !aligned(g_out, 4))
     return fail(ctx, DUST_ERR_ARG, "weights and X must be 16-byte aligned, the rest 4-byte");
   DUST_CU(cudaSetDevice(ctx->device));
@@ -479,7 +483,7 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   DUST_TRY(ensure(ctx, ctx->mlp_h, (size_t)T * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->z, (size_t)T * V * 4));
   DUST_TRY(ensure(ctx, ctx->lse, (size_t)T * 4));
-  DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(DUST_BF16, T, dff)));
+  DUST_TRY(ensure(ctx, ctx->gop, down ? (size_t)T * d * 4 : gop_bytes(DUST_BF16, T, dff)));
   float* loss = loss_out;
   if (!loss) {
     DUST_TRY(ensure(ctx, ctx->loss, (size_t)T * 4));
@@ -546,7 +550,7 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   if (tchunk > T) tchunk = T;
   const int64_t rows_cap = tchunk * K;
   const int nparts = (int)((V + 127) / 128);
-  DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * 2 * dff * 2));
+  if (!down) DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * 2 * dff * 2));
   DUST_TRY(ensure(ctx, ctx->mlp_dh, (size_t)rows_cap * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->part, (size_t)rows_cap * nparts * 4));
   DUST_TRY(ensure(ctx, ctx->dzy, (size_t)rows_cap * 4));
@@ -555,9 +559,12 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
   for (int64_t t0 = 0; t0 < T; t0 += tchunk) {
     const int64_t nt = (t0 + tchunk <= T) ? tchunk : T - t0;
     const int64_t rows = nt * K;
-    DUST_CU(launch_mlp_delta_a(st, p, u, t0, nt, da, true, nullptr));
-    ctx->launches += 1;
-    {
+    if (down) {
+      DUST_CU(launch_mlp_noise_split(st, p, t0, nt, dh));
+      ctx->launches += 1;
+    } else {
+      DUST_CU(launch_mlp_delta_a(st, p, u, t0, nt, da, true, nullptr));
+      ctx->launches += 1;
       GemmDesc g{};
       g.M = rows; g.N = d; g.K = 2 * dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
       g.B = ctx->wd2.p; g.ldb = 2 * dff; g.b_kmajor = true; g.dtype = DUST_BF16;
@@ -588,14 +595,40 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* pp, const void* X, c
     ctx->launches += 1;
   }
   mark(ctx, "perturbed");
-  DUST_CU(launch_mlp_g(st, p, r, g_out, ctx->gop.p));
+  DUST_CU(launch_mlp_g(st, p, r, g_out, ctx->gop.p, down));
   ctx->launches += 1;
   mark(ctx, "g");
-  if (G_up_out) {
-    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, dff, X, d, G_up_out, 0));
+  if (G_out && !down) {
+    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, dff, X, d, G_out, 0));
+    mark(ctx, "gw_gemm");
+  } else if (G_out) {
+    // G_down = sum_t g_t a_t^T with a = GELU(u) rounded once to fp32: an fp32
+    // contraction over tokens on CUDA cores (2 T d d_ff flops, small next to
+    // the perturbed pass)
+    DUST_TRY(ensure(ctx, ctx->mlp_a32, (size_t)T * dff * 4));
+    DUST_CU(launch_gelu_f32(st, u, T * dff, (float*)ctx->mlp_a32.p, ctx->sm_count));
+    ctx->launches += 1;
+    dust_params pf = p;
+    pf.dtype = DUST_F32;
+    DUST_TRY(weight_grad(ctx, pf, ctx->gop.p, d, ctx->mlp_a32.p, dff, G_out, 0));
     mark(ctx, "gw_gemm");
   }
   return finish(ctx, p.flags);
+}
+
+dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* p, const void* X, const void* W_up,
+                          const void* W_down, const void* W_head, const int32_t* targets,
+                          float* G_up_out, float* loss_out, float* rewards_out, float* g_out) {
+  return mlp_impl(ctx, p, false, X, W_up, W_down, W_head, targets, G_up_out, loss_out,
+                  rewards_out, g_out);
+}
+
+dust_status dust_mlp_down_grad(dust_ctx* ctx, const dust_params* p, const void* X,
+                               const void* W_up, const void* W_down, const void* W_head,
+                               const int32_t* targets, float* G_down_out, float* loss_out,
+                               float* rewards_out, float* g_out) {
+  return mlp_impl(ctx, p, true, X, W_up, W_down, W_head, targets, G_down_out, loss_out,
+                  rewards_out, g_out);
 }
 
 dust_status dust_set_stage_timing(dust_ctx* ctx, int enable) {

@@ -134,7 +134,7 @@ struct dust_ctx {
   bool subset2_enabled = true;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
-      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep;
+      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32;
 };
 
 namespace dust {
@@ -223,7 +223,14 @@ cudaError_t launch_reward_gemm_simt(cudaStream_t st, const GemmDesc& g, const fl
 cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int nparts,
                                        const float* dzy, int64_t rows, int64_t row0, int32_t K,
                                        float* r);
+// g of the up-projection (width d_ff; gop as bf16 hi/lo planes for bf16 calls)
+// or, with down, of the down-projection (width d; gop fp32).
 cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
-                         void* gop);
+                         void* gop, bool down);
+// Down-projection draws: dh = sigma eps as bf16 hi/lo planes (rows nt K x 2d).
+cudaError_t launch_mlp_noise_split(cudaStream_t st, const dust_params& p, int64_t t0, int64_t nt,
+                                   __nv_bfloat16* dh);
+// a = GELU(u) (fp64, rounded to fp32), n elements.
+cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a, int sm_count);
 
 }  // namespace dust

@@ -61,6 +61,39 @@ __global__ void k_mlp_delta_a(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
   }
 }
 
+// Down-projection draws: sigma eps on W_down's output (the block output h)
+// is itself the head input change, dh = sigma eps, stored as bf16 hi/lo
+// planes dh[row*2d + c], dh[row*2d + d + c]; one thread per (row, 128-channel
+// block, lane) as above.
+__global__ void k_mlp_noise_split(Key key, uint32_t t_off, uint32_t i_off, uint32_t ctr3,
+                                  float sigma, int64_t width, int32_t K, int64_t t0, int64_t rows,
+                                  __nv_bfloat16* __restrict__ dh) {
+  const int64_t nblk = (width + 127) / 128;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= rows * nblk * 32) return;
+  const uint32_t lane = (uint32_t)(gid & 31);
+  const int64_t rest = gid >> 5;
+  const int64_t blk = rest % nblk;
+  const int64_t row = rest / nblk;
+  const int64_t t = t0 + row / K;
+  const int32_t i = (int32_t)(row % K);
+  U4 c{slot_ctr0((uint32_t)blk, lane), t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3};
+  const G4 g = gauss4(philox10(c, key.k0, key.k1), sigma);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t ch = blk * 128 + lane + 32 * j;
+    if (ch < width) split_bf16((double)g.v[j], &dh[row * 2 * width + ch], &dh[row * 2 * width + width + ch]);
+  }
+}
+
+// a = GELU(u) in fp64, rounded once to fp32 (the down-projection's input,
+// the right-hand operand of its weight gradient).
+__global__ void k_gelu_f32(const float* __restrict__ u, int64_t n, float* __restrict__ a) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    a[i] = (float)gelu64((double)u[i]);
+}
+
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -202,6 +235,27 @@ cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const floa
   return cudaGetLastError();
 }
 
+cudaError_t launch_mlp_noise_split(cudaStream_t st, const dust_params& p, int64_t t0, int64_t nt,
+                                   __nv_bfloat16* dh) {
+  const int64_t rows = nt * p.K;
+  const int64_t nblk = (p.d + 127) / 128;
+  const int64_t total = rows * nblk * 32;
+  if (total <= 0) return cudaSuccess;
+  const int threads = 256;
+  k_mlp_noise_split<<<(unsigned)((total + threads - 1) / threads), threads, 0, st>>>(
+      key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
+      ctr3_of(kTagMlpDown, p.stream_id), p.sigma, p.d, p.K, t0, rows, dh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a, int sm_count) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)sm_count * 16) blocks = (int64_t)sm_count * 16;
+  k_gelu_f32<<<(unsigned)blocks, 256, 0, st>>>(u, n, a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_reward_gemm_simt(cudaStream_t st, const GemmDesc& g, const float* P,
                                     const int32_t* y, int64_t t0, int32_t K, float* part,
                                     float* dzy) {
@@ -224,18 +278,19 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
 }
 
 cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
-                         void* gop) {
-  dim3 grid((unsigned)p.T, (unsigned)((p.d_ff + 1023) / 1024));
+                         void* gop, bool down) {
+  const int64_t width = down ? p.d : p.d_ff;
+  dim3 grid((unsigned)p.T, (unsigned)((width + 1023) / 1024));
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
   const Key key = key_of(p.seed);
-  const uint32_t c3 = ctr3_of(kTagMlpUp, p.stream_id);
-  const int64_t plane = p.T * p.d_ff;
-  if (p.dtype == DUST_BF16)
+  const uint32_t c3 = ctr3_of(down ? kTagMlpDown : kTagMlpUp, p.stream_id);
+  const int64_t plane = p.T * width;
+  if (p.dtype == DUST_BF16 && !down)
     k_noise_g<__nv_bfloat16><<<grid, 256, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
+        (uint32_t)p.draw_offset, c3, scale, width, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
   else
     k_noise_g<float><<<grid, 256, 0, st>>>(key, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, p.d_ff, p.K, r, g_out, (float*)gop, plane);
+        (uint32_t)p.draw_offset, c3, scale, width, p.K, r, g_out, (float*)gop, plane);
   return cudaGetLastError();
 }
 

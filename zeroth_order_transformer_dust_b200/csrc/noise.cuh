@@ -20,6 +20,7 @@ constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
 constexpr int kTagHead = 0;
 constexpr int kTagSubsetOffset = 1;
 constexpr int kTagMlpUp = 2;
+constexpr int kTagMlpDown = 3;
 
 struct U4 {
   uint32_t x, y, z, w;
@@ -80,12 +81,13 @@ __device__ __forceinline__ void sincos_turn24(uint32_t m, float* s_out, float* c
 
 // Radius of the Box-Muller pair, R = sqrt(-2 ln u1), for
 // u1 = ((wa >> 8) + 1) 2^-24 (exact in fp32). Away from u1 = 1, ln u1 comes
-// from the hardware base-2 logarithm of u1 (MUFU.LG2); as u1 -> 1 the
-// logarithm is small and that estimate loses its relative accuracy, so for
-// v = 1 - u1 < 2^-7 (exact) the series -ln(1 - v) = v (1 + v/2 + v^2/3 +
-// v^3/4 + ...) is used instead, truncated below 2^-28 relative. The square
-// root is the hardware approximation (MUFU.SQRT, sqrt(0) = 0). Checked over
-// all 2^24 values of u1 against fp64: below 8e-7 absolute.
+// from the hardware base-2 logarithm of u1 (MUFU.LG2). Its error near u1 = 1
+// is absolute (about 2^-23), which the square root turns into a radius error
+// of about 0.7 2^-23 / R, so for v = 1 - u1 < 2^-6 (exact; R < 0.18) the
+// series -2 ln(1 - v) = 2v + v^2 + (2/3) v^3 + ... is used instead (the
+// first omitted term, v^4/2, is below 2^-19 relative there). The square root
+// is the hardware approximation (MUFU.SQRT, sqrt(0) = 0). Checked over all
+// 2^24 values of u1 against fp64: below 8e-7 absolute.
 __device__ __forceinline__ float sqrt_approx(float x) {
   float y;
   asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -96,11 +98,8 @@ __device__ __forceinline__ float bm_radius(uint32_t wa) {
   const float u = fmaf((float)(wa >> 8), 5.9604645e-08f, 5.9604645e-08f);  // exact
   const float far = __log2f(u) * -1.3862944f;                             // -2 ln 2
   const float v = 1.0f - u;  // exact (u >= 1/2 where it is used)
-  float c = fmaf(v, 0.25f, 1.0f / 3.0f);
-  c = fmaf(v, c, 0.5f);
-  c = fmaf(v, c, 1.0f);
-  const float near = (v + v) * c;
-  return sqrt_approx(v < 0.0078125f ? near : far);
+  const float near = v * fmaf(v, fmaf(v, 2.0f / 3.0f, 1.0f), 2.0f);
+  return sqrt_approx(v < 0.015625f ? near : far);
 }
 
 // Box-Muller on 24-bit uniforms: u1 = ((wa>>8)+1) 2^-24, u2 = (wb>>8) 2^-24;
