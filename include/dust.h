@@ -236,8 +236,10 @@ dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, cons
 
 /* Debug: C (M x N, fp32, row-major) = A B^T for bf16 row-major A (M x K) and
    B (N x K), through the library's GEMMs: path 0 = automatic, 1 = CUDA cores,
-   2 = tcgen05 tensor cores (DUST_ERR_UNSUPPORTED when the shape does not fit:
-   K a multiple of 8 and N >= 16 are needed). Synchronous. */
+   2 = tcgen05 tensor cores with one CTA per 128 x 256 tile, 3 = tcgen05 with
+   CTA pairs (cta_group::2) per 256 x 256 tile (2 and 3 return
+   DUST_ERR_UNSUPPORTED when the shape does not fit: K a multiple of 8 and
+   N >= 16 are needed). Synchronous. */
 dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
                                  const void* B, float* C, int path);
 

@@ -1,6 +1,8 @@
 """The library's GEMMs in isolation: C = A B^T with bf16 operands and fp32
-accumulation, tcgen05 tensor-core path and CUDA-core path, against torch's
-fp32 product of the same bf16 values (ragged M, N and K tails included)."""
+accumulation, on the tcgen05 tensor-core path (one CTA per 128 x 256 tile,
+and CTA pairs per 256 x 256 tile) and the CUDA-core path, against torch's
+fp32 product of the same bf16 values (ragged M, N and K tails included; for
+pairs, M tails that leave the second CTA of a pair partly or wholly past M)."""
 import pytest
 import torch
 
@@ -18,8 +20,23 @@ SHAPES = [(128, 256, 64), (256, 512, 128), (300, 500, 72), (1, 16, 8), (129, 257
           (1000, 50304, 64), (2048, 1024, 1024), (4096, 3072, 768), (64, 768, 3072)]
 
 
+def _check(ctx, M, N, K, path):
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K)
+    A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    C = ctx.debug_gemm(A, B, path=path)
+    ref = A.float() @ B.float().T
+    err = ((C - ref).norm() / ref.norm()).item()
+    assert err < 1e-5, err
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 64), (128, 256, 64), (100, 16, 8), (384, 300, 200)])
+def test_pair_gemm_small(ctx, M, N, K):
+    _check(ctx, M, N, K, 3)
+
+
 @pytest.mark.parametrize("M,N,K", SHAPES)
-@pytest.mark.parametrize("path", [2, 1])
+@pytest.mark.parametrize("path", [2, 1, 3])
 def test_gemm_matches_fp32_product(ctx, M, N, K, path):
     g = torch.Generator(device="cuda").manual_seed(M * 7 + N * 3 + K)
     A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
@@ -38,10 +55,19 @@ def test_tensor_core_path_rejects_unaligned_k(ctx):
     assert ei.value.status == 6
 
 
-def test_repeated_launches_are_consistent(ctx):
+@pytest.mark.parametrize("path", [2, 3])
+def test_repeated_launches_are_consistent(ctx, path):
     g = torch.Generator(device="cuda").manual_seed(3)
     A = torch.randn(1024, 512, device="cuda", generator=g).to(torch.bfloat16)
     B = torch.randn(2048, 512, device="cuda", generator=g).to(torch.bfloat16)
-    C0 = ctx.debug_gemm(A, B, path=2)
+    C0 = ctx.debug_gemm(A, B, path=path)
     for _ in range(5):
-        assert torch.equal(ctx.debug_gemm(A, B, path=2), C0)
+        assert torch.equal(ctx.debug_gemm(A, B, path=path), C0)
+
+
+def test_pair_and_single_cta_paths_agree(ctx):
+    g = torch.Generator(device="cuda").manual_seed(5)
+    A = torch.randn(1000, 768, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(3000, 768, device="cuda", generator=g).to(torch.bfloat16)
+    c2, c3 = ctx.debug_gemm(A, B, path=2), ctx.debug_gemm(A, B, path=3)
+    assert ((c2 - c3).norm() / c2.norm()).item() < 1e-6

@@ -310,7 +310,8 @@ class Context:
 
     # -- debug exports -------------------------------------------------------------
     def debug_gemm(self, A: torch.Tensor, B: torch.Tensor, path: int = 0) -> torch.Tensor:
-        """C = A B^T (bf16 operands, fp32 out); path 0 auto, 1 CUDA cores, 2 tensor cores."""
+        """C = A B^T (bf16 operands, fp32 out); path 0 auto, 1 CUDA cores, 2 tensor cores
+        (one CTA per tile), 3 tensor cores with CTA pairs."""
         self._dev(A, "A"), self._dev(B, "B")
         if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
             raise TypeError("A and B must be bfloat16")

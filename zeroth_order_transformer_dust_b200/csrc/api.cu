@@ -1,6 +1,7 @@
 // C ABI of the estimator: validation, scratch management and the order of
 // the kernel stages. Every numerical step runs in the kernels this file
 // launches; nothing here computes on the host beyond index bookkeeping.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -133,12 +134,15 @@ dust_status finish(dust_ctx* ctx, uint32_t flags) {
 }
 
 // path: 0 automatic, 1 CUDA cores, 2 tensor cores.
+// path: 0 automatic, 1 CUDA cores, 2 tensor cores one CTA per tile, 3 tensor
+// cores with CTA pairs.
 dust_status run_gemm(dust_ctx* ctx, const GemmDesc& g, const EpiDesc& e, int path = 0) {
-  const bool tc = path != 1 && (path == 2 || ctx->tc_enabled) && tc_gemm_supported(g, e);
-  if (path == 2 && !tc) return fail(ctx, DUST_ERR_UNSUPPORTED, "shape not taken by the tensor-core GEMM");
+  const bool tc = path != 1 && (path >= 2 || ctx->tc_enabled) && tc_gemm_supported(g, e);
+  if (path >= 2 && !tc) return fail(ctx, DUST_ERR_UNSUPPORTED, "shape not taken by the tensor-core GEMM");
   ctx->launches += 1;
   if (tc) {
-    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count, ctx->d_status));
+    const bool pair = path == 3 || (path == 0 && ctx->tc_pair && g.M >= 256);
+    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count, ctx->d_status, pair));
   } else {
     DUST_CU(launch_gemm_simt(ctx->stream, g, e));
   }
@@ -242,6 +246,8 @@ dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
   ctx->stream = (cudaStream_t)cuda_stream;
   const char* no_tc = getenv("DUST_DISABLE_TC");
   ctx->tc_enabled = !(no_tc && no_tc[0] && no_tc[0] != '0');
+  const char* pair = getenv("DUST_TC_PAIR");
+  ctx->tc_pair = !(pair && pair[0] == '0');
   const char* sk = getenv("DUST_SUBSET_KERNEL");
   ctx->subset2_enabled = !(sk && sk[0] == '1');
   if (cudaSetDevice(device) != cudaSuccess ||
@@ -357,7 +363,7 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   // On tensor cores the GEMM epilogue also leaves per-tile softmax partials
   // of every row (the per-token max / log-sum-exp cache), so z is not re-read.
   const bool fused = !need_prob && ctx->tc_enabled && tc_gemm_supported(g, e);
-  const int ntiles = (int)((p.V + kTcTileN - 1) / kTcTileN);
+  const int ntiles = tc_partials_per_row(p.V);
   if (fused) {
     DUST_TRY(ensure(ctx, ctx->lsep, (size_t)p.T * ntiles * sizeof(float2)));
     e.kind = kEpiF32Lse;
@@ -549,7 +555,9 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
   if (tchunk < 1) tchunk = 1;
   if (tchunk > T) tchunk = T;
   const int64_t rows_cap = tchunk * K;
-  const int nparts = (int)((V + 127) / 128);
+  // reward partials per row: 128-column tiles on CUDA cores, two per 256-column tile on
+  // tensor cores
+  const int nparts = std::max((int)((V + 127) / 128), tc_partials_per_row(V));
   if (!down) DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * 2 * dff * 2));
   DUST_TRY(ensure(ctx, ctx->mlp_dh, (size_t)rows_cap * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->part, (size_t)rows_cap * nparts * 4));
@@ -573,7 +581,7 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
       DUST_TRY(run_gemm(ctx, g, e));
     }
     // dz = dh W_head^T with the reward epilogue (dz never reaches memory)
-    int used_parts = nparts;
+    int used_parts = (int)((V + 127) / 128);  // the CUDA-core reward GEMM's 128-column tiles
     {
       GemmDesc g{};
       g.M = rows; g.N = V; g.K = 2 * d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
@@ -583,7 +591,7 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
       e.part = (float*)ctx->part.p; e.dzy = (float*)ctx->dzy.p;
       if (ctx->tc_enabled && tc_gemm_supported(g, e)) {
         DUST_TRY(run_gemm(ctx, g, e));
-        used_parts = (int)((V + kTcTileN - 1) / kTcTileN);
+        used_parts = tc_partials_per_row(V);
       } else {
         DUST_CU(launch_reward_gemm_simt(st, g, Z, targets, t0, p.K, (float*)ctx->part.p,
                                         (float*)ctx->dzy.p));
@@ -664,7 +672,7 @@ int64_t dust_kernel_launches(const dust_ctx* ctx) { return ctx ? ctx->launches :
 dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
                                  const void* B, float* C, int path) {
   if (!ctx) return DUST_ERR_ARG;
-  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || path < 0 || path > 2)
+  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || path < 0 || path > 3)
     return fail(ctx, DUST_ERR_ARG, "bad gemm arguments");
   DUST_CU(cudaSetDevice(ctx->device));
   DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), ctx->stream));

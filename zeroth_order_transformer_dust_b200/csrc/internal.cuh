@@ -41,12 +41,13 @@ enum EpiKind {
                        // hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
   kEpiResidSplit = 3,  // h = resid[m*ldr + n] (bf16) + acc, stored as bf16 hi/lo planes
   kEpiSplit = 4,       // acc stored as bf16 hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
-  kEpiReward = 5,      // MLP perturbed logits dz (never stored): per row m and 256-column
-                       // tile nb, part[m*n_tiles + nb] = sum_n P[t, n] expm1(dz);
-                       // dzy[m] = dz at column y[t]; t = t0 + m / draws
-  kEpiF32Lse = 6,      // kEpiF32 without row remap, plus per row m and 256-column tile
-                       // nb the softmax partial lsep[m*n_tiles + nb] =
-                       // (max_n acc, sum_n exp(acc - max)) over the tile's columns < N
+  kEpiReward = 5,      // MLP perturbed logits dz (never stored): per row m, 256-column
+                       // tile nb and 128-column half h, part[(m*n_tiles + nb)*2 + h] =
+                       // sum_n P[t, n] expm1(dz); dzy[m] = dz at column y[t];
+                       // t = t0 + m / draws
+  kEpiF32Lse = 6,      // kEpiF32 without row remap, plus per row m, 256-column tile nb
+                       // and half h the softmax partial lsep[(m*n_tiles + nb)*2 + h] =
+                       // (max_n acc, sum_n exp(acc - max)) over its columns < N
 };
 
 struct EpiDesc {
@@ -70,8 +71,10 @@ struct EpiDesc {
   float2* lsep = nullptr;
 };
 
-// Column tile width of the tensor-core GEMM (reward partials per row = ceil(N / it)).
+// Column tile width of the tensor-core GEMM; its epilogues leave two partials
+// per row and tile (tc_partials_per_row).
 constexpr int kTcTileN = 256;
+inline int tc_partials_per_row(int64_t N) { return (int)(2 * ((N + kTcTileN - 1) / kTcTileN)); }
 
 // Exact-erf GELU in fp64. The last product is rounded on its own
 // (__dmul_rn) so that a difference GELU(x) - GELU(x') is not contracted
@@ -130,6 +133,8 @@ struct dust_ctx {
   int64_t launches = 0;
   // tensor-core GEMMs on (DUST_DISABLE_TC=1 at creation routes all GEMMs to CUDA cores)
   bool tc_enabled = true;
+  // CTA-pair tensor-core GEMMs for M >= 256 (DUST_TC_PAIR=0 at creation keeps one CTA per tile)
+  bool tc_pair = true;
   // shared-memory subset kernel on (DUST_SUBSET_KERNEL=1 selects the first, L2-fed one)
   bool subset2_enabled = true;
   // scratch, grown on demand
@@ -199,11 +204,12 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
                            const float* Z, const float* lse, const int32_t* y, float* rewards,
                            float* g_out, void* gop, int max_smem_optin, int sm_count);
 
-// Tensor-core GEMM (tcgen05): shapes it takes, and its launcher. A bounded
-// wait that expires sets kStatusTimeout in *status.
+// Tensor-core GEMM (tcgen05): shapes it takes, and its launcher (pair: a
+// 256 x 256 tile per cluster of two CTAs, cta_group::2; else 128 x 256 per
+// CTA). A bounded wait that expires sets kStatusTimeout in *status.
 bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e);
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
-                           uint32_t* status);
+                           uint32_t* status, bool pair);
 
 // Transpose of a row-major bf16 matrix (rows x cols) into dst (cols x rows,
 // row stride ld_dst >= rows; columns [rows, ld_dst) of dst are zeroed).

@@ -17,29 +17,49 @@
 namespace dust {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+// BM rows of A and BN accumulator columns per CTA; BK-deep stages.
+constexpr int BM = 128, BN = 256, BK = 64;
 static_assert(BN == kTcTileN, "reward partials are laid out per BN-column tile");
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int THREADS = 192;
+// warp 0: TMA producer; warp 1: MMA issuer; warps 2..9: epilogue, two per
+// TMEM lane quarter, each draining one half of the accumulator's columns
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int HALF_N = BN / 2;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 // Reward epilogue: each epilogue warp stages the probability rows of the (at
-// most two) tokens its 32 rows belong to, BN columns each, per accumulator.
-constexpr int PSTAGE_FLOATS = 2 * BN;
-constexpr size_t PSTAGE_BYTES = (size_t)4 * 2 * PSTAGE_FLOATS * 4;  // 4 warps x 2 accumulators
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + PSTAGE_BYTES;
+// most two) tokens its 32 rows belong to, over its HALF_N columns, per
+// accumulator.
+constexpr int PSTAGE_FLOATS = 2 * HALF_N;
+constexpr size_t PSTAGE_BYTES = (size_t)EPI_WARPS * 2 * PSTAGE_FLOATS * 4;
+constexpr int kMaxStages = 6;
+
+// Single CTA: a 128 x 256 tile per SM, A and all 256 rows of B staged by the
+// CTA (48 KB per 64-deep stage, 4 stages). CTA pair (cta_group::2): a
+// 256 x 256 tile per pair of SMs; each CTA stages its 128 rows of A and 128
+// of the 256 rows of B (32 KB per stage, 6 stages) and the leader's MMAs read
+// both CTAs' shared memory, so every SM is fed a third fewer bytes per flop.
+template <bool PAIR>
+struct Cfg {
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + PSTAGE_BYTES;
+  static_assert(STAGES <= kMaxStages, "barrier arrays");
+};
 
 struct TcParams {
   int64_t M, N, K;
-  int m_tiles, n_tiles, num_kb;
+  int m_tiles, n_tiles, num_kb;  // m_tiles counts Cfg::TILE_M-row tiles
   EpiDesc e;
   uint32_t* status;
 };
 
 struct Shared {
-  uint64_t full[STAGES], empty[STAGES], tfull[2], tempty[2], drain;
+  uint64_t full[kMaxStages], empty[kMaxStages], tfull[2], tempty[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -156,17 +176,17 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
   *n_blk = r / rows;
 }
 
-// expm1 of a perturbed logit: degree-5 Taylor polynomial below 1/16
-// (relative truncation < 2e-9), the library function otherwise.
+// expm1 of a perturbed logit without a branch: degree-5 Taylor polynomial
+// below 1/16 (relative truncation < 2e-9); above, e^x - 1 from the hardware
+// exponential, whose few-ulp error on e^x is below 1e-5 relative to
+// expm1(x) >= 0.06 there (the reward needs sum_n p_n expm1 to ~1e-7 absolute).
 __device__ __forceinline__ float expm1_guarded(float x) {
-  if (fabsf(x) < 0.0625f) {
-    float q = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
-    q = fmaf(x, q, 1.0f / 6.0f);
-    q = fmaf(x, q, 0.5f);
-    q = fmaf(x, q, 1.0f);
-    return x * q;
-  }
-  return expm1f(x);
+  float q = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
+  q = fmaf(x, q, 1.0f / 6.0f);
+  q = fmaf(x, q, 0.5f);
+  q = fmaf(x, q, 1.0f);
+  const float big = __expf(x) - 1.0f;
+  return fabsf(x) < 0.0625f ? x * q : big;
 }
 
 // Reward epilogue of 32 columns of row m (target column yt): returns
@@ -175,22 +195,24 @@ __device__ __forceinline__ float expm1_guarded(float x) {
 // else the row in global memory.
 __device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int32_t yt, int64_t n,
                                           const float* prow, bool staged, const float* v) {
-  float s = 0.0f;
+  // four independent sums, so the adds do not form one 32-long chain
+  float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
   if (staged || (n + 32 <= p.N && (p.N & 3) == 0)) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const float4 pv = staged ? reinterpret_cast<const float4*>(prow)[q]
                                : __ldg(reinterpret_cast<const float4*>(prow) + q);
-      s = fmaf(pv.x, expm1_guarded(v[4 * q + 0]), s);
-      s = fmaf(pv.y, expm1_guarded(v[4 * q + 1]), s);
-      s = fmaf(pv.z, expm1_guarded(v[4 * q + 2]), s);
-      s = fmaf(pv.w, expm1_guarded(v[4 * q + 3]), s);
+      s0 = fmaf(pv.x, expm1_guarded(v[4 * q + 0]), s0);
+      s1 = fmaf(pv.y, expm1_guarded(v[4 * q + 1]), s1);
+      s2 = fmaf(pv.z, expm1_guarded(v[4 * q + 2]), s2);
+      s3 = fmaf(pv.w, expm1_guarded(v[4 * q + 3]), s3);
     }
   } else {
 #pragma unroll
     for (int q = 0; q < 32; ++q)
-      if (n + q < p.N) s = fmaf(prow[q], expm1_guarded(v[q]), s);
+      if (n + q < p.N) s0 = fmaf(prow[q], expm1_guarded(v[q]), s0);
   }
+  const float s = (s0 + s1) + (s2 + s3);
   if (yt >= n && yt < n + 32) {
 #pragma unroll
     for (int q = 0; q < 32; ++q)
@@ -199,10 +221,13 @@ __device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int32_t 
   return s;
 }
 
-template <int KIND>
+template <int KIND, bool PAIR>
 __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ CUtensorMap tmA,
                                                         const __grid_constant__ CUtensorMap tmB,
                                                         TcParams p) {
+  using C = Cfg<PAIR>;
+  constexpr int STAGES = C::STAGES, A_BYTES = C::A_BYTES, B_BYTES = C::B_BYTES;
+  constexpr int STAGE_BYTES = C::STAGE_BYTES, TILE_M = C::TILE_M;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -215,6 +240,11 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = p.m_tiles * p.n_tiles;
+  // CTA pairs work on one tile together: unit = pair index, rank 0 leads
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -223,7 +253,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(ptx::smem_u32(&sh->tfull[a]), 1);
-      ptx::mbar_init(ptx::smem_u32(&sh->tempty[a]), 4);
+      // the leader's MMAs wait for the epilogue warps of both CTAs
+      ptx::mbar_init(ptx::smem_u32(&sh->tempty[a]), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
     }
     ptx::mbar_init(ptx::smem_u32(&sh->drain), 1);
     sh->abort = 0;
@@ -233,11 +264,17 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     ptx::prefetch_map(&tmB);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
-    ptx::tmem_relinquish();
+    if (PAIR) {
+      ptx::tmem_alloc_pair(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(ptx::smem_u32(&sh->tmem_base), TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  // both CTAs' barriers and TMEM exist before either signals the other
+  if (PAIR) ptx::cluster_sync(); else __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
 
@@ -247,15 +284,25 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // bit s: stage s holds a copy / its parity
-      for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+      for (int tile = unit0; tile < total && !*abort; tile += units) {
         int m_blk, n_blk;
         tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
+        const int a_row = m_blk * TILE_M + (int)rank * BM;
+        const int b_row = n_blk * BN + (int)rank * C::B_ROWS;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!wait_bounded(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort, p.status)) break;
           const uint32_t fb = ptx::smem_u32(&sh->full[stage]);
-          ptx::mbar_expect_tx(fb, STAGE_BYTES);
-          ptx::tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, m_blk * BM, fb);
-          ptx::tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, n_blk * BN, fb);
+          if (PAIR) {
+            // both CTAs' bytes complete on the leader's barrier
+            if (leader) ptx::mbar_expect_tx(fb, 2 * STAGE_BYTES);
+            const uint32_t lfb = ptx::mapa_shared(fb, 0);
+            ptx::tma_load_2d_pair(sA + stage * A_BYTES, &tmA, kb * BK, a_row, lfb);
+            ptx::tma_load_2d_pair(sB + stage * B_BYTES, &tmB, kb * BK, b_row, lfb);
+          } else {
+            ptx::mbar_expect_tx(fb, STAGE_BYTES);
+            ptx::tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, a_row, fb);
+            ptx::tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, b_row, fb);
+          }
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -264,21 +311,27 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           }
         }
       }
-      // every copy this thread issued has landed before the CTA can exit
+      // every copy this thread issued has landed before the CTA can exit: a
+      // single CTA (or the leader) sees its stages complete; the pair's
+      // second CTA sees them consumed (the MMAs waited for their bytes)
       int dummy = 0;
       for (int s = 0; s < STAGES; ++s)
-        if ((armed >> s) & 1u)
-          wait_bounded(ptx::smem_u32(&sh->full[s]), (armed_parity >> s) & 1u, &dummy, p.status);
+        if ((armed >> s) & 1u) {
+          if (PAIR && !leader)
+            wait_bounded(ptx::smem_u32(&sh->empty[s]), (armed_parity >> s) & 1u, &dummy, p.status);
+          else
+            wait_bounded(ptx::smem_u32(&sh->full[s]), (armed_parity >> s) & 1u, &dummy, p.status);
+        }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
+    if (lane == 0 && leader) {
+      const uint32_t idesc = ptx::idesc_bf16_f32(TILE_M, BN);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool issued = false;
-      for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
+      for (int tile = unit0; tile < total && !*abort; tile += units, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
         if (!wait_bounded(ptx::smem_u32(&sh->tempty[acc]), acc_phase ^ 1u, abort, p.status)) break;
@@ -294,32 +347,54 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           const uint32_t a0 = sA + stage * A_BYTES, b0 = sB + stage * B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            ptx::mma_f16(d_tmem, ptx::sdesc_kmajor_sw128(a0 + k * 32),
-                         ptx::sdesc_kmajor_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+            if (PAIR)
+              ptx::mma_f16_pair(d_tmem, ptx::sdesc_kmajor_sw128(a0 + k * 32),
+                                ptx::sdesc_kmajor_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+            else
+              ptx::mma_f16(d_tmem, ptx::sdesc_kmajor_sw128(a0 + k * 32),
+                           ptx::sdesc_kmajor_sw128(b0 + k * 32), idesc, (kb | k) != 0);
           }
           issued = true;
-          ptx::mma_commit(ptx::smem_u32(&sh->empty[stage]));
+          if (PAIR)
+            ptx::mma_commit_pair(ptx::smem_u32(&sh->empty[stage]), 0x3);
+          else
+            ptx::mma_commit(ptx::smem_u32(&sh->empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        ptx::mma_commit(ptx::smem_u32(&sh->tfull[acc]));
+        if (PAIR)
+          ptx::mma_commit_pair(ptx::smem_u32(&sh->tfull[acc]), 0x3);
+        else
+          ptx::mma_commit(ptx::smem_u32(&sh->tfull[acc]));
       }
       if (issued) {
-        // all MMAs of this CTA complete before TMEM is released
-        ptx::mma_commit(ptx::smem_u32(&sh->drain));
+        // all MMAs complete before TMEM is released (in both CTAs of a pair)
+        if (PAIR)
+          ptx::mma_commit_pair(ptx::smem_u32(&sh->drain), 0x3);
+        else
+          ptx::mma_commit(ptx::smem_u32(&sh->drain));
         int dummy = 0;
         wait_bounded(ptx::smem_u32(&sh->drain), 0, &dummy, p.status);
       }
+    } else if (PAIR && lane == 0 && unit0 < total) {
+      // the second CTA of a pair: the leader's MMAs write this CTA's TMEM too
+      int dummy = 0;
+      wait_bounded(ptx::smem_u32(&sh->drain), 0, &dummy, p.status);
     }
   } else {
-    // ---------------- epilogue warps 2..5 ----------------
+    // ---------------- epilogue warps 2..9 ----------------
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32)
     const int row = quad * 32 + lane;
+    const int half = (warp - 2) >> 2;  // columns [HALF_N half, HALF_N (half + 1)) of the tile
     int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+    const uint32_t tempty0 =
+        PAIR ? ptx::mapa_shared(ptx::smem_u32(&sh->tempty[0]), 0) : ptx::smem_u32(&sh->tempty[0]);
+    const uint32_t tempty1 =
+        PAIR ? ptx::mapa_shared(ptx::smem_u32(&sh->tempty[1]), 0) : ptx::smem_u32(&sh->tempty[1]);
+    for (int tile = unit0; tile < total; tile += units, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       int m_blk, n_blk;
@@ -330,7 +405,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       int64_t t_first = 0;
       float* stg = pstage + ((warp - 2) * 2 + acc) * PSTAGE_FLOATS;
       if (KIND == kEpiReward) {
-        const int64_t m_first = (int64_t)m_blk * BM + quad * 32;
+        const int64_t m_first = (int64_t)m_blk * TILE_M + (int64_t)rank * BM + quad * 32;
         if (m_first < p.M && (p.N & 3) == 0) {
           const int64_t m_last = min(m_first + 31, p.M - 1);
           t_first = p.e.t0 + m_first / p.e.draws;
@@ -340,9 +415,10 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
             float4 pv[PSTAGE_FLOATS / 128];
 #pragma unroll
             for (int j = 0; j < PSTAGE_FLOATS / 128; ++j) {
-              const int q = lane + 32 * j;  // float4 index: token q / (BN/4), column 4 (q % (BN/4))
-              const int64_t t = t_first + q / (BN / 4);
-              const int64_t n = (int64_t)n_blk * BN + 4 * (q % (BN / 4));
+              // float4 index q: token q / (HALF_N/4), column 4 (q % (HALF_N/4)) of the half
+              const int q = lane + 32 * j;
+              const int64_t t = t_first + q / (HALF_N / 4);
+              const int64_t n = (int64_t)n_blk * BN + half * HALF_N + 4 * (q % (HALF_N / 4));
               pv[j] = make_float4(0.f, 0.f, 0.f, 0.f);
               if (t <= t_last && n < p.N)
                 pv[j] = __ldg(reinterpret_cast<const float4*>(p.e.P + t * p.N + n));
@@ -357,7 +433,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       }
       if (!wait_bounded(ptx::smem_u32(&sh->tfull[acc]), acc_phase, abort, p.status)) break;
       ptx::tc_fence_after();
-      const int64_t m = (int64_t)m_blk * BM + row;
+      const int64_t m = (int64_t)m_blk * TILE_M + (int64_t)rank * BM + row;
       int64_t mo = m;
       if (p.e.c_row_mul != 0 && m < p.M)
         mo = (int64_t)(((unsigned long long)m * (unsigned long long)p.e.c_row_mul) %
@@ -373,45 +449,59 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       float s_row = 0.0f;
       float rmax = -FLT_MAX, rsum = 0.0f;  // kEpiF32Lse: online softmax partial of the row
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (HALF_N / 32); c < (half + 1) * (HALF_N / 32); ++c) {
         const int64_t n = (int64_t)n_blk * BN + c * 32;
         float v[32];
         ptx::tmem_ld32(taddr + (uint32_t)(c * 32), v);
         if (KIND == kEpiReward) {
           if (m < p.M && n < p.N) {
-            const float* prow = staged ? stg + (t_row - t_first) * BN + c * 32
+            const float* prow = staged ? stg + (t_row - t_first) * HALF_N + (c * 32 - half * HALF_N)
                                        : p.e.P + t_row * p.N + n;
             s_row += reward32(p, m, yt, n, prow, staged, v);
           }
         } else if (m < p.M && n < p.N) {
           epilogue32<KIND>(p, m, mo, n, v);
           if (KIND == kEpiF32Lse) {
-            float cm = -FLT_MAX;
+            // max and sum of exponentials of the chunk, as 4 independent chains
+            float cm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-              if (n + q < p.N) cm = fmaxf(cm, v[q]);
-            const float nm = fmaxf(rmax, cm);
-            float cs = 0.0f;
+              if (n + q < p.N) cm[q & 3] = fmaxf(cm[q & 3], v[q]);
+            const float nm = fmaxf(rmax, fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])));
+            float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-              if (n + q < p.N) cs += __expf(v[q] - nm);
-            rsum = fmaf(rsum, __expf(rmax - nm), cs);
+              if (n + q < p.N) cs[q & 3] += __expf(v[q] - nm);
+            rsum = fmaf(rsum, __expf(rmax - nm), (cs[0] + cs[1]) + (cs[2] + cs[3]));
             rmax = nm;
           }
         }
       }
-      if (KIND == kEpiF32Lse && m < p.M) p.e.lsep[m * p.n_tiles + n_blk] = make_float2(rmax, rsum);
-      if (KIND == kEpiReward && m < p.M) p.e.part[m * p.n_tiles + n_blk] = s_row;
+      // one partial per row, column tile and half: 2 n_tiles per row
+      const int64_t pidx = ((int64_t)m * p.n_tiles + n_blk) * 2 + half;
+      if (KIND == kEpiF32Lse && m < p.M) p.e.lsep[pidx] = make_float2(rmax, rsum);
+      if (KIND == kEpiReward && m < p.M) p.e.part[pidx] = s_row;
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&sh->tempty[acc]));
+      if (lane == 0) {
+        if (PAIR)
+          ptx::mbar_arrive_cluster(acc ? tempty1 : tempty0);
+        else
+          ptx::mbar_arrive(acc ? tempty1 : tempty0);
+      }
     }
   }
 
   ptx::tc_fence_before();
-  __syncthreads();
+  // neither CTA of a pair leaves while the other may still signal its barriers
+  if (PAIR) ptx::cluster_sync(); else __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 1) ptx::tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == 1) {
+    if (PAIR)
+      ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+    else
+      ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -442,16 +532,34 @@ bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KIND>
+template <int KIND, bool PAIR>
 cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
                         const TcParams& p, int sm_count) {
-  auto fn = k_gemm_tc<KIND>;
-  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+  auto fn = k_gemm_tc<KIND, PAIR>;
+  constexpr size_t smem = Cfg<PAIR>::SMEM;
+  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < sm_count ? tiles : sm_count;
-  fn<<<grid, THREADS, SMEM_BYTES, st>>>(a, b, p);
+  if (!PAIR) {
+    const int grid = tiles < sm_count ? tiles : sm_count;
+    fn<<<grid, THREADS, smem, st>>>(a, b, p);
+    return cudaGetLastError();
+  }
+  const int pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, fn, a, b, p);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
@@ -472,31 +580,43 @@ bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
          e.kind == kEpiF32Lse;
 }
 
-cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
-                           uint32_t* status) {
+namespace {
+
+template <bool PAIR>
+cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
+                        uint32_t* status) {
   CUtensorMap ma, mb;
-  if (!make_map(&ma, g.A, g.M, g.K, g.lda, BM) || !make_map(&mb, g.B, g.N, g.K, g.ldb, BN))
+  if (!make_map(&ma, g.A, g.M, g.K, g.lda, BM) ||
+      !make_map(&mb, g.B, g.N, g.K, g.ldb, Cfg<PAIR>::B_ROWS))
     return cudaErrorInvalidValue;
   TcParams p;
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
-  p.m_tiles = (int)((g.M + BM - 1) / BM);
+  p.m_tiles = (int)((g.M + Cfg<PAIR>::TILE_M - 1) / Cfg<PAIR>::TILE_M);
   p.n_tiles = (int)((g.N + BN - 1) / BN);
   p.num_kb = (int)((g.K + BK - 1) / BK);
   p.e = e;
   p.status = status;
   if (!p.status) return cudaErrorInvalidValue;
   switch (e.kind) {
-    case kEpiF32: return launch_kind<kEpiF32>(st, ma, mb, p, sm_count);
-    case kEpiBF16: return launch_kind<kEpiBF16>(st, ma, mb, p, sm_count);
-    case kEpiGeluSplit: return launch_kind<kEpiGeluSplit>(st, ma, mb, p, sm_count);
-    case kEpiResidSplit: return launch_kind<kEpiResidSplit>(st, ma, mb, p, sm_count);
-    case kEpiSplit: return launch_kind<kEpiSplit>(st, ma, mb, p, sm_count);
-    case kEpiReward: return launch_kind<kEpiReward>(st, ma, mb, p, sm_count);
-    case kEpiF32Lse: return launch_kind<kEpiF32Lse>(st, ma, mb, p, sm_count);
+    case kEpiF32: return launch_kind<kEpiF32, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiBF16: return launch_kind<kEpiBF16, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiGeluSplit: return launch_kind<kEpiGeluSplit, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiResidSplit: return launch_kind<kEpiResidSplit, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiSplit: return launch_kind<kEpiSplit, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiReward: return launch_kind<kEpiReward, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiF32Lse: return launch_kind<kEpiF32Lse, PAIR>(st, ma, mb, p, sm_count);
   }
   return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
+                           uint32_t* status, bool pair) {
+  if (pair && sm_count >= 2) return launch_pair<true>(st, g, e, sm_count, status);
+  return launch_pair<false>(st, g, e, sm_count, status);
 }
 
 }  // namespace dust
