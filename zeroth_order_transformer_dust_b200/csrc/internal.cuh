@@ -83,7 +83,14 @@ __device__ __forceinline__ double gelu64(double x) {
   return __dmul_rn(0.5 * x, 1.0 + erf(x * 0.70710678118654752440));
 }
 
-// v as a bf16 pair with v ~= hi + lo (relative error about 2^-17).
+// v as a bf16 pair with v ~= hi + lo (relative error about 2^-17). For an
+// fp32 v the residual v - hi is exact in fp32 (it has at most 16 significant
+// bits), so the float form gives the same pair as the fp64 one.
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  *hi = h;
+  *lo = __float2bfloat16_rn(v - __bfloat162float(h));
+}
 __device__ __forceinline__ void split_bf16(double v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
   const __nv_bfloat16 h = __float2bfloat16_rn((float)v);
   *hi = h;

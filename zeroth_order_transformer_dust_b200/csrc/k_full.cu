@@ -49,6 +49,48 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Draws [i0, i0 + n) of one unit for one warp; per draw, the warp's sum goes
+// to sh[warp][ii]. ALL: all kBlocksPerWarp blocks of the warp lie below V
+// (every warp but the one that straddles V), so no per-block test runs in the
+// draw loop. The reward sum runs as one chain per block. No barrier inside:
+// the caller's block-wide barriers are the same for every warp.
+template <int DEG, bool ALL>
+__device__ __forceinline__ void reward_chunk(const FullArgs& A, const float2* tab, int64_t t,
+                                             int i0, int n, int nvalid,
+                                             const float (&pv)[kBlocksPerWarp][4],
+                                             const BlockConst (&bc)[kBlocksPerWarp],
+                                             bool warp_has_y, bool y_here, int by, int jy,
+                                             float (*sh)[kDrawChunk]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t t_abs = A.t_off + (uint32_t)t;
+  for (int ii = 0; ii < n; ++ii) {
+    const uint32_t i_abs = A.i_off + (uint32_t)(i0 + ii);
+    const DrawConst dc = draw_const(A.keys, t_abs, i_abs);
+    float sb[kBlocksPerWarp];
+    float xyv = 0.0f;
+#pragma unroll
+    for (int b = 0; b < kBlocksPerWarp; ++b) {
+      sb[b] = 0.0f;
+      if (ALL || b < nvalid) {
+        const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sb[b] = fmaf(pv[b][j], expm1_small<DEG>(g.v[j]), sb[b]);
+        if (warp_has_y) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (b == by && j == jy) xyv = g.v[j];
+        }
+      }
+    }
+    if (y_here) A.xy[t * A.K + i0 + ii] = xyv;
+    float s = 0.0f;
+#pragma unroll
+    for (int b = 0; b < kBlocksPerWarp; ++b) s += sb[b];
+    s = warp_sum(s);
+    if (lane == 0) sh[warp][ii] = s;
+  }
+}
+
 template <int DEG>
 __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __grid_constant__ FullArgs A) {
   __shared__ float sh[kWarps][kDrawChunk];
@@ -61,6 +103,9 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __gri
     const int64_t t = unit / A.nslab;
     const int slab = (int)(unit % A.nslab);
     const int64_t blk0 = (int64_t)slab * (kSlab / 128) + warp * kBlocksPerWarp;
+    // blocks of this warp below V (warp-uniform)
+    const int64_t left = (A.V - blk0 * 128 + 127) / 128;
+    const int nvalid = left <= 0 ? 0 : (left >= kBlocksPerWarp ? kBlocksPerWarp : (int)left);
     float pv[kBlocksPerWarp][4];  // p = exp(z - LSE), formed once per unit
     BlockConst bc[kBlocksPerWarp];
     const float lse_t = A.lse[t];
@@ -80,30 +125,12 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __gri
     const bool warp_has_y = yb >= blk0 && yb < blk0 + kBlocksPerWarp;  // warp-uniform
     const bool y_here = warp_has_y && lane == (yt & 31);
     const int by = (int)(yb - blk0), jy = (yt >> 5) & 3;
-    const uint32_t t_abs = A.t_off + (uint32_t)t;
     for (int i0 = 0; i0 < A.K; i0 += kDrawChunk) {
       const int n = min(kDrawChunk, A.K - i0);
-      for (int ii = 0; ii < n; ++ii) {
-        const uint32_t i_abs = A.i_off + (uint32_t)(i0 + ii);
-        const DrawConst dc = draw_const(A.keys, t_abs, i_abs);
-        float s = 0.0f, xyv = 0.0f;
-#pragma unroll
-        for (int b = 0; b < kBlocksPerWarp; ++b) {
-          if ((blk0 + b) * 128 < A.V) {
-            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) s = fmaf(pv[b][j], expm1_small<DEG>(g.v[j]), s);
-            if (warp_has_y) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                if (b == by && j == jy) xyv = g.v[j];
-            }
-          }
-        }
-        if (y_here) A.xy[t * A.K + i0 + ii] = xyv;
-        s = warp_sum(s);
-        if (lane == 0) sh[warp][ii] = s;
-      }
+      if (nvalid == kBlocksPerWarp)
+        reward_chunk<DEG, true>(A, tab, t, i0, n, nvalid, pv, bc, warp_has_y, y_here, by, jy, sh);
+      else
+        reward_chunk<DEG, false>(A, tab, t, i0, n, nvalid, pv, bc, warp_has_y, y_here, by, jy, sh);
       __syncthreads();
       if ((int)threadIdx.x < n) {
         float s = 0.0f;
@@ -128,6 +155,27 @@ __global__ void k_full_reward_combine(int64_t T, int32_t K, int nslab,
   r[id] = xy[id] - log1pf(s);
 }
 
+// Draws [i0, i0 + n) of sum_i r_i (sigma eps_i) for one warp's blocks, with
+// r staged in rs (ALL: every block lies below V). No barrier inside.
+template <bool ALL>
+__device__ __forceinline__ void g_chunk(const FullArgs& A, const float2* tab, int64_t t, int i0,
+                                        int n, int nvalid, const BlockConst (&bc)[kBlocksPerWarp],
+                                        const float* rs, float (&acc)[kBlocksPerWarp][4]) {
+  const uint32_t t_abs = A.t_off + (uint32_t)t;
+  for (int ii = 0; ii < n; ++ii) {
+    const float ri = rs[ii];
+    const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)(i0 + ii));
+#pragma unroll
+    for (int b = 0; b < kBlocksPerWarp; ++b) {
+      if (ALL || b < nvalid) {
+        const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(ri, g.v[j], acc[b][j]);
+      }
+    }
+  }
+}
+
 __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ FullArgs A) {
   __shared__ float rs[1024];
   __shared__ float2 tab[kSinCosTable];
@@ -139,7 +187,8 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
     const int64_t t = unit / A.nslab;
     const int slab = (int)(unit % A.nslab);
     const int64_t blk0 = (int64_t)slab * (kSlab / 128) + warp * kBlocksPerWarp;
-    const uint32_t t_abs = A.t_off + (uint32_t)t;
+    const int64_t left = (A.V - blk0 * 128 + 127) / 128;
+    const int nvalid = left <= 0 ? 0 : (left >= kBlocksPerWarp ? kBlocksPerWarp : (int)left);
     BlockConst bc[kBlocksPerWarp];
     float acc[kBlocksPerWarp][4];
 #pragma unroll
@@ -153,18 +202,10 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
       __syncthreads();
       for (int q = threadIdx.x; q < n; q += blockDim.x) rs[q] = A.r[t * A.K + i0 + q];
       __syncthreads();
-      for (int ii = 0; ii < n; ++ii) {
-        const float ri = rs[ii];
-        const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)(i0 + ii));
-#pragma unroll
-        for (int b = 0; b < kBlocksPerWarp; ++b) {
-          if ((blk0 + b) * 128 < A.V) {
-            const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(ri, g.v[j], acc[b][j]);
-          }
-        }
-      }
+      if (nvalid == kBlocksPerWarp)
+        g_chunk<true>(A, tab, t, i0, n, nvalid, bc, rs, acc);
+      else
+        g_chunk<false>(A, tab, t, i0, n, nvalid, bc, rs, acc);
     }
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b)

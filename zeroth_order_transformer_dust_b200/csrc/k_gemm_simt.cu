@@ -109,7 +109,7 @@ __global__ __launch_bounds__(256) void k_gemm_simt(GemmDesc g, EpiDesc e) {
           break;
         }
         case kEpiSplit:
-          split_bf16((double)v, &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
+          split_bf16(v, &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
           break;
       }
     }

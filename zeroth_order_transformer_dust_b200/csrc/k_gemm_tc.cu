@@ -155,7 +155,7 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
     } else {
 #pragma unroll
       for (int q = 0; q < 32; ++q)
-        if (n + q < p.N) split_bf16((double)v[q], hi + q, lo + q);
+        if (n + q < p.N) split_bf16(v[q], hi + q, lo + q);
     }
   }
 }
