@@ -38,10 +38,14 @@ from .philox import (  # noqa: F401
     TAG_SUBSET_OFFSET,
     TAG_MLP_UP,
     TAG_MLP_DOWN,
+    TAG_ATTN_OUT,
 )
 from .params import Params  # noqa: F401
 from .head import (  # noqa: F401
     clean_head, head_grad, head_linear_estimate, full_vocab_draws, subset_draws,
 )
-from .mlp import clean_mlp, mlp_grad, mlp_draws, gelu, mlp_down_grad, mlp_down_draws  # noqa: F401
+from .mlp import (  # noqa: F401
+    clean_mlp, mlp_grad, mlp_draws, gelu, mlp_down_grad, mlp_down_draws, attn_out_grad,
+    attn_out_draws,
+)
 from .optim import sgd_momentum, train_head, exact_weight_grad  # noqa: F401

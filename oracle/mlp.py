@@ -30,7 +30,7 @@ import numpy as np
 from scipy.special import erf
 
 from .params import Params
-from .philox import TAG_MLP_DOWN, TAG_MLP_UP, gaussians
+from .philox import TAG_ATTN_OUT, TAG_MLP_DOWN, TAG_MLP_UP, gaussians
 
 
 def gelu(x: np.ndarray) -> np.ndarray:
@@ -135,3 +135,58 @@ def mlp_down_grad(X, W_up, W_down, W_head, targets, prm: Params, draw_chunk: int
     G = np.einsum("tc,tf->cf", g, a)
     return {"loss": clean["loss"], "lse": clean["lse"], "rewards": rewards, "g": g, "G": G,
             "a": a, "p": p, "z": clean["z"]}
+
+
+# --------------------------------------------------------------------------
+# Attention output-projection variant: the perturbed layer is y = W_o o (d
+# outputs per token, o the cached attention output, the layer's input), and y
+# is added to the residual stream that enters the MLP block: x = r + W_o o.
+# Noise sigma eps on y moves x, so each draw recomputes the MLP block and the
+# head from the cached x, u and clean logits (the same per-layer reading):
+#   du = sigma eps W_up^T,  da = GELU(u + du) - GELU(u),
+#   dh = sigma eps + da W_down^T,  dz = dh W_head^T,
+#   r  = dz_y - log1p(sum_j p_j expm1(dz_j)),
+#   g_t = -(1/(K sigma)) sum_i r_i eps_i  (d entries),  G_o = sum_t g_t o_t^T.
+
+def attn_out_draws(u_t, p_t, y_t, eps, W_up, W_down, W_head, sig):
+    """Rewards and sum_i r_i eps_i for n draws of noise ``eps`` (n, d) on x_t."""
+    dx = sig * eps
+    du = dx @ W_up.T
+    da = gelu(u_t[None, :] + du) - gelu(u_t)[None, :]
+    dh = dx + da @ W_down.T
+    dz = dh @ W_head.T
+    r = dz[:, y_t] - np.log1p((p_t[None, :] * np.expm1(dz)).sum(axis=1))
+    acc = (r[:, None] * eps).sum(axis=0)
+    return r, acc
+
+
+def attn_out_grad(X, O, W_up, W_down, W_head, targets, prm: Params, draw_chunk: int = 64) -> dict:
+    """X: residual entering the MLP block (T x d); O: the output projection's
+    input (T x d_o). Returns the estimator's outputs, G of shape d x d_o."""
+    Wu = np.asarray(W_up, dtype=np.float64)
+    Wd = np.asarray(W_down, dtype=np.float64)
+    Wh = np.asarray(W_head, dtype=np.float64)
+    y = np.asarray(targets, dtype=np.int64)
+    clean = clean_mlp(X, W_up, W_down, W_head, y)
+    u, p = clean["u"], clean["p"]
+    T = u.shape[0]
+    d = Wh.shape[1]
+    sig = prm.sigma32
+    rewards = np.zeros((T, prm.K))
+    g = np.zeros((T, d))
+    for t in range(T):
+        t_abs = t + prm.token_offset
+        for i0 in range(0, prm.K, draw_chunk):
+            i1 = min(prm.K, i0 + draw_chunk)
+            draws = np.arange(i0, i1, dtype=np.int64) + prm.draw_offset
+            eps = gaussians(prm.seed, t_abs, draws, np.arange(d), TAG_ATTN_OUT, prm.stream_id)
+            r, acc = attn_out_draws(u[t], p[t], y[t], eps, Wu, Wd, Wh, sig)
+            rewards[t, i0:i1] = r
+            g[t] += acc
+    if sig == 0.0:
+        g[:] = 0.0
+    else:
+        g *= -1.0 / (prm.K * sig)
+    G = np.einsum("tc,tf->cf", g, np.asarray(O, dtype=np.float64))
+    return {"loss": clean["loss"], "lse": clean["lse"], "rewards": rewards, "g": g, "G": G,
+            "u": u, "p": p, "z": clean["z"]}

@@ -40,6 +40,7 @@ TAG_HEAD = 0           # noise on the LM-head logits
 TAG_SUBSET_OFFSET = 1  # the per-draw subset offset b
 TAG_MLP_UP = 2         # noise on the MLP up-projection output
 TAG_MLP_DOWN = 3       # noise on the MLP down-projection output
+TAG_ATTN_OUT = 4       # noise on the attention output projection's output
 
 
 def _u32(x) -> np.ndarray:

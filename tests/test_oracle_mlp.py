@@ -180,3 +180,73 @@ def test_down_estimate_converges_with_population():
         errs.append(np.linalg.norm(G - gW) / np.linalg.norm(gW))
     assert errs[1] < errs[0] / 2.5
     assert errs[1] < 0.25
+
+
+# ---- attention output-projection variant -------------------------------------
+
+def _attn_problem(T=4, d=5, d_o=6, d_ff=7, V=9, seed=0):
+    rng = np.random.default_rng(seed + 100)
+    X, Wu, Wd, Wh, y = _mlp_problem(T=T, d=d, d_ff=d_ff, V=V, seed=seed)
+    R = rng.standard_normal((T, d))                 # residual before the attention write
+    O = rng.standard_normal((T, d_o))               # the output projection's input
+    W_o = rng.standard_normal((d, d_o)) / math.sqrt(d_o)
+    return R, O, W_o, Wu, Wd, Wh, y
+
+
+def _dL_dx(X, W_up, W_down, W_head, y):
+    """dL/dx for the residual entering the MLP block (x a leaf), from autograd."""
+    t = {k: torch.tensor(v, dtype=torch.float64) for k, v in
+         dict(W_up=W_up, W_down=W_down, W_head=W_head).items()}
+    x = torch.tensor(X, dtype=torch.float64, requires_grad=True)
+    a = torch.nn.functional.gelu(x @ t["W_up"].T, approximate="none")
+    z = (x + a @ t["W_down"].T) @ t["W_head"].T
+    torch.nn.functional.cross_entropy(z, torch.tensor(y), reduction="sum").backward()
+    return x.grad.numpy()
+
+
+def test_attn_out_estimate_is_unbiased_exact_expectation():
+    """Over +-sqrt(d) e_m noise on x, g equals dL/dx (to O(sigma^2))."""
+    R, O, W_o, Wu, Wd, Wh, y = _attn_problem(T=3)
+    X = R + O @ W_o.T
+    gx = _dL_dx(X, Wu, Wd, Wh, y)
+    c = oracle.clean_mlp(X, Wu, Wd, Wh, y)
+    d = Wh.shape[1]
+    eps = np.concatenate([np.eye(d), -np.eye(d)]) * math.sqrt(d)
+    sig = 1e-6
+    for t in range(3):
+        r, acc = oracle.attn_out_draws(c["u"][t], c["p"][t], y[t], eps, Wu, Wd, Wh, sig)
+        np.testing.assert_allclose(-acc / (eps.shape[0] * sig), gx[t], rtol=0, atol=1e-7)
+
+
+def test_attn_out_weight_gradient_matches_finite_differences():
+    """sum_t dL/dx_t o_t^T against brute-force differences in W_o, x = r + W_o o."""
+    R, O, W_o, Wu, Wd, Wh, y = _attn_problem(T=3, d=3, d_o=4, d_ff=4, V=5)
+    X = R + O @ W_o.T
+    closed = _dL_dx(X, Wu, Wd, Wh, y).T @ O
+    fd = np.zeros_like(W_o)
+    h = 1e-5
+    for i in range(W_o.shape[0]):
+        for j in range(W_o.shape[1]):
+            P, M = W_o.copy(), W_o.copy()
+            P[i, j] += h
+            M[i, j] -= h
+            fd[i, j] = (oracle.clean_mlp(R + O @ P.T, Wu, Wd, Wh, y)["loss"].sum()
+                        - oracle.clean_mlp(R + O @ M.T, Wu, Wd, Wh, y)["loss"].sum()) / (2 * h)
+    np.testing.assert_allclose(fd, closed, rtol=0, atol=1e-8)
+
+
+def test_attn_out_sigma_zero_and_convergence():
+    R, O, W_o, Wu, Wd, Wh, y = _attn_problem(T=4, d=4, d_o=3, d_ff=6, V=7, seed=3)
+    X = R + O @ W_o.T
+    prm = oracle.Params(T=4, d=4, V=7, d_ff=6, K=6, sigma=0.0, seed=2)
+    out = oracle.attn_out_grad(X, O, Wu, Wd, Wh, y, prm)
+    assert np.all(out["rewards"] == 0.0) and np.all(out["G"] == 0.0)
+    exact = _dL_dx(X, Wu, Wd, Wh, y).T @ O
+    errs = []
+    for K in (256, 4096):
+        prm = oracle.Params(T=4, d=4, V=7, d_ff=6, K=K, sigma=1e-4, seed=8)
+        G = oracle.attn_out_grad(X, O, Wu, Wd, Wh, y, prm, draw_chunk=4096)["G"]
+        assert G.shape == (4, 3)
+        errs.append(np.linalg.norm(G - exact) / np.linalg.norm(exact))
+    # the error falls as 1/sqrt(K) in expectation (4x over these K); one sample each
+    assert errs[1] < errs[0] / 2 and errs[1] < 0.1
