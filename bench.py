@@ -131,9 +131,13 @@ def _oracle_tokens(args):
         for t in toks:
             prm = oracle.Params(T=1, d=wl.d, V=wl.V, d_ff=wl.d_ff, K=wl.K, sigma=wl.sigma,
                                 seed=wl.seed, token_offset=t)
-            fn = oracle.mlp_down_grad if wl.variant == "mlp_down" else oracle.mlp_grad
-            fn(inp["X"][t:t + 1], inp["W_up"], inp["W_down"], inp["W_head"],
-               inp["targets"][t:t + 1], prm)
+            if wl.variant == "attn_out":
+                oracle.attn_out_grad(inp["X"][t:t + 1], inp["O"][t:t + 1], inp["W_up"],
+                                     inp["W_down"], inp["W_head"], inp["targets"][t:t + 1], prm)
+            else:
+                fn = oracle.mlp_down_grad if wl.variant == "mlp_down" else oracle.mlp_grad
+                fn(inp["X"][t:t + 1], inp["W_up"], inp["W_down"], inp["W_head"],
+                   inp["targets"][t:t + 1], prm)
     return len(toks), time.perf_counter() - t0
 
 
@@ -280,15 +284,16 @@ def run_dust(args):
         X, Wu, Wdn, Wh = (torch.from_numpy(inp[k]).to(torch.bfloat16).to(dev)
                           for k in ("X", "W_up", "W_down", "W_head"))
         yd = torch.from_numpy(inp["targets"]).to(torch.int32).to(dev)
-        gshape = (wl.d_ff, wl.d) if wl.variant == "mlp" else (wl.d, wl.d_ff)
+        gshape = {"mlp": (wl.d_ff, wl.d), "mlp_down": (wl.d, wl.d_ff)}.get(wl.variant, (wl.d, wl.d))
         outs = {"G": torch.empty(*gshape, dtype=torch.float32, device=dev),
                 "loss": torch.empty(wl.T, dtype=torch.float32, device=dev)}
 
-        layer = "down" if wl.variant == "mlp_down" else "up"
+        layer = {"mlp_down": "down", "attn_out": "attn_out"}.get(wl.variant, "up")
+        Od = torch.from_numpy(inp["O"]).to(torch.bfloat16).to(dev) if layer == "attn_out" else None
 
         def step():
             ctx.mlp_grad(X, Wu, Wdn, Wh, yd, K=wl.K, sigma=wl.sigma, seed=wl.seed,
-                         token_offset=t_off, out=outs, layer=layer)
+                         token_offset=t_off, out=outs, layer=layer, O=Od)
             from zeroth_order_transformer_dust_b200.parallel import allreduce_weight_grad
             allreduce_weight_grad(outs["G"])
 

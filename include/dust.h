@@ -181,6 +181,30 @@ dust_status dust_mlp_down_grad(dust_ctx* ctx, const dust_params* p,
                                float* G_down_out, float* loss_out, float* rewards_out,
                                float* g_out);
 
+/*
+ * Attention output-projection estimator (same pages and sections: the layer
+ * types of a block perturbed in separate passes on cached intermediates).
+ * The perturbed layer is y = W_o o, whose output is written into the residual
+ * x that enters the MLP block (x = r + W_o o). Noise on y therefore moves x,
+ * and each draw recomputes the MLP block and the head from the cached x, u and
+ * clean logits:
+ *   du = sigma eps W_up^T,  da = GELU(u + du) - GELU(u),
+ *   dh = sigma eps + da W_down^T,  dz = dh W_head^T.
+ * The reward and g_t (d entries) are as for dust_mlp_down_grad.
+ *   X        T x d     the residual entering the block (bf16)
+ *   O        T x d_o   the projection's cached input o_t (bf16), d_o a multiple of 8
+ *   W_up, W_down, W_head, targets as dust_mlp_grad
+ *   G_o_out  d x d_o   fp32 sum_t g_t o_t^T   (or NULL)
+ *   loss_out, rewards_out as dust_mlp_grad;  g_out T x d fp32 (or NULL)
+ * The noise has its own counter tag (4). Same validation and errors as
+ * dust_mlp_grad, plus DUST_ERR_ARG for a NULL or misaligned O or a bad d_o.
+ */
+dust_status dust_attn_out_grad(dust_ctx* ctx, const dust_params* p,
+                               const void* X, const void* O, int64_t d_o,
+                               const void* W_up, const void* W_down, const void* W_head,
+                               const int32_t* targets, float* G_o_out, float* loss_out,
+                               float* rewards_out, float* g_out);
+
 /* Per-stage device timing: when enabled, each call records CUDA events on
    the context's stream between its stages (clean GEMM, log-sum-exp, draws,
    g, G_W GEMM...). dust_stage_times waits for the last call's final event

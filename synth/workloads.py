@@ -2,11 +2,12 @@
 
 Recipe (all host-side, numpy PCG64; the workload seed's SeedSequence spawns
 one child stream per tensor, in the order H, W, targets for the LM-head
-workloads and x, W_up, W_down, W_head, targets for the MLP workload):
+workloads and x, W_up, W_down, W_head, targets, O for the MLP-block workloads):
 
 * H ~ N(0, 1), then each row divided by its RMS sqrt(mean(h^2)).
 * W ~ N(0, 1/d), so logits z = W h are roughly N(0, 1) per entry.
-* MLP: x ~ N(0, 1); W_up ~ N(0, 1/d); W_down ~ N(0, 1/d_ff); W_head ~ N(0, 1/d).
+* MLP: x ~ N(0, 1); W_up ~ N(0, 1/d); W_down ~ N(0, 1/d_ff); W_head ~ N(0, 1/d);
+  the attention output O ~ N(0, 1) for the output-projection variant.
 * targets: uniform on [0, V) for the tiny fp32 workload, otherwise a
   Zipf(1.1) law truncated to ranks 1..V (rank k -> token id k-1), sampled by
   inverse CDF.
@@ -27,7 +28,7 @@ import numpy as np
 @dataclass(frozen=True)
 class Workload:
     name: str
-    variant: str        # "head", "mlp" (up-projection) or "mlp_down"
+    variant: str        # "head", "mlp" (up-projection), "mlp_down" or "attn_out"
     T: int
     d: int
     V: int
@@ -62,6 +63,9 @@ CONFIGS = {
                          sigma=1e-2, seed=3, dtype="bf16", targets="zipf", d_ff=3072),
     # Hidden MLP down-projection (noise on W_down's output), same shapes.
     "mlp_down_bf16": Workload("mlp_down_bf16", "mlp_down", T=8192, d=768, V=50304, K=256, S=0,
+                              sigma=1e-2, seed=3, dtype="bf16", targets="zipf", d_ff=3072),
+    # Attention output projection writing into the MLP block's input, same shapes.
+    "attn_out_bf16": Workload("attn_out_bf16", "attn_out", T=8192, d=768, V=50304, K=256, S=0,
                               sigma=1e-2, seed=3, dtype="bf16", targets="zipf", d_ff=3072),
     # LM head at 243M-model head scale, subset draws (S = 512), 16k draws.
     "large_subset_bf16": Workload("large_subset_bf16", "head", T=16384, d=1024, V=50304,
@@ -119,13 +123,16 @@ def make_head_inputs(wl: Workload) -> dict:
 
 
 def make_mlp_inputs(wl: Workload) -> dict:
-    """x (T x d), W_up (d_ff x d), W_down (d x d_ff), W_head (V x d), targets."""
-    rX, rU, rD, rHd, ry = _streams(wl.seed, 5)
+    """x (T x d), W_up (d_ff x d), W_down (d x d_ff), W_head (V x d), targets, and
+    O (T x d ~ N(0, 1)), the attention output the output-projection variant
+    takes as its layer input (its own sixth stream, so the others are unchanged)."""
+    rX, rU, rD, rHd, ry, rO = _streams(wl.seed, 6)
     X = rX.standard_normal((wl.T, wl.d))
     W_up = rU.standard_normal((wl.d_ff, wl.d)) * (1.0 / np.sqrt(wl.d))
     W_down = rD.standard_normal((wl.d, wl.d_ff)) * (1.0 / np.sqrt(wl.d_ff))
     W_head = rHd.standard_normal((wl.V, wl.d)) * (1.0 / np.sqrt(wl.d))
     y = _targets(ry, wl)
+    O = rO.standard_normal((wl.T, wl.d))
     return {"X": _cast(X, wl.dtype), "W_up": _cast(W_up, wl.dtype),
             "W_down": _cast(W_down, wl.dtype), "W_head": _cast(W_head, wl.dtype),
-            "targets": y}
+            "targets": y, "O": _cast(O, wl.dtype)}

@@ -34,7 +34,7 @@ EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
            "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
            "dust_kernel_launches", "dust_debug_gemm_bf16", "dust_debug_gauss_tab",
            "dust_head_grad_noalloc", "dust_debug_bm_radius", "dust_debug_bm_angle",
-           "dust_sgd_momentum", "dust_mlp_down_grad")
+           "dust_sgd_momentum", "dust_mlp_down_grad", "dust_attn_out_grad")
 
 
 class DustParams(ctypes.Structure):
@@ -82,6 +82,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "dust_head_grad_host": (I32, [P, PP, P, P, P, P, P, P, P]),
             "dust_mlp_grad": (I32, [P, PP, P, P, P, P, P, P, P, P, P]),
             "dust_mlp_down_grad": (I32, [P, PP, P, P, P, P, P, P, P, P, P]),
+            "dust_attn_out_grad": (I32, [P, PP, P, P, I64, P, P, P, P, P, P, P, P]),
             "dust_debug_philox": (I32, [P, U64, P, I64, P]),
             "dust_debug_gauss": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_set_stage_timing": (I32, [P, ctypes.c_int]),
@@ -245,12 +246,18 @@ class Context:
 
     def mlp_grad(self, X, W_up, W_down, W_head, targets, *, K, sigma, seed=0, token_offset=0,
                  draw_offset=0, stream_id=0, want_G=True, want_loss=True, want_rewards=False,
-                 want_g=False, out=None, layer="up") -> dict:
-        """MLP estimator (bf16 inputs) for the up-projection (layer="up": G is
-        d_ff x d, g is T x d_ff) or the down-projection (layer="down": G is
-        d x d_ff, g is T x d). Returns the requested fp32 outputs."""
-        if layer not in ("up", "down"):
-            raise ValueError("layer must be 'up' or 'down'")
+                 want_g=False, out=None, layer="up", O=None) -> dict:
+        """MLP-block estimator (bf16 inputs) for the up-projection (layer="up":
+        G is d_ff x d, g is T x d_ff), the down-projection (layer="down": G is
+        d x d_ff, g is T x d) or the attention output projection whose output
+        enters the block (layer="attn_out", O its T x d_o input: G is d x d_o,
+        g is T x d). Returns the requested fp32 outputs."""
+        if layer not in ("up", "down", "attn_out"):
+            raise ValueError("layer must be 'up', 'down' or 'attn_out'")
+        if (layer == "attn_out") != (O is not None):
+            raise ValueError("O is given exactly for layer='attn_out'")
+        if O is not None:
+            self._dev(O, "O")
         for t, n in ((X, "X"), (W_up, "W_up"), (W_down, "W_down"), (W_head, "W_head"),
                      (targets, "targets")):
             self._dev(t, n)
@@ -262,8 +269,9 @@ class Context:
         out = dict(out or {})
         f32 = dict(dtype=torch.float32, device=X.device)
         width = d_ff if layer == "up" else d
+        gshape = {"up": (d_ff, d), "down": (d, d_ff)}.get(layer) or (d, O.shape[1])
         if want_G and "G" not in out:
-            out["G"] = torch.empty(*((d_ff, d) if layer == "up" else (d, d_ff)), **f32)
+            out["G"] = torch.empty(*gshape, **f32)
         if want_loss and "loss" not in out:
             out["loss"] = torch.empty(T, **f32)
         if want_rewards and "rewards" not in out:
@@ -271,10 +279,16 @@ class Context:
         if want_g and "g" not in out:
             out["g"] = torch.empty(T, width, **f32)
         self._bind_stream()
-        fn = self._L.dust_mlp_grad if layer == "up" else self._L.dust_mlp_down_grad
-        st = fn(self._h, ctypes.byref(prm), _ptr(X), _ptr(W_up), _ptr(W_down), _ptr(W_head),
-                _ptr(targets), _ptr(out.get("G")), _ptr(out.get("loss")),
+        tail = (_ptr(targets), _ptr(out.get("G")), _ptr(out.get("loss")),
                 _ptr(out.get("rewards")), _ptr(out.get("g")))
+        if layer == "attn_out":
+            st = self._L.dust_attn_out_grad(self._h, ctypes.byref(prm), _ptr(X), _ptr(O),
+                                            O.shape[1], _ptr(W_up), _ptr(W_down), _ptr(W_head),
+                                            *tail)
+        else:
+            fn = self._L.dust_mlp_grad if layer == "up" else self._L.dust_mlp_down_grad
+            st = fn(self._h, ctypes.byref(prm), _ptr(X), _ptr(W_up), _ptr(W_down), _ptr(W_head),
+                    *tail)
         self._check(st)
         return out
 

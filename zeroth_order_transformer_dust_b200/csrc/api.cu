@@ -8,6 +8,7 @@
 #include <cstring>
 
 #include "internal.cuh"
+#include "noise.cuh"
 
 using namespace dust;
 
@@ -463,13 +464,19 @@ dust_status dust_head_grad_host(dust_ctx* ctx, const dust_params* pp, const void
   return dust_check(ctx);
 }
 
-// The two MLP variants share the clean pass and the reward GEMM: `down`
-// perturbs W_down's output (dh = sigma eps directly) instead of W_up's
-// (dh = (GELU(u + sigma eps) - GELU(u)) W_down^T).
-static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, const void* X,
-                            const void* W_up, const void* W_down, const void* W_head,
-                            const int32_t* targets, float* G_out, float* loss_out,
-                            float* rewards_out, float* g_out) {
+// The MLP-block layer variants share the clean pass and the reward GEMM; the
+// perturbed layer decides the head-input change dh of each draw:
+//   kLayerUp:      noise on u = W_up x,    dh = (GELU(u + s e) - GELU(u)) W_down^T
+//   kLayerDown:    noise on W_down's output, dh = s e
+//   kLayerAttnOut: noise on W_o o, the residual x entering the block:
+//                  du = s e W_up^T, dh = s e + (GELU(u + du) - GELU(u)) W_down^T
+enum MlpLayer { kLayerUp = 0, kLayerDown = 1, kLayerAttnOut = 2 };
+
+static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, const void* X,
+                            const void* O, int64_t d_o, const void* W_up, const void* W_down,
+                            const void* W_head, const int32_t* targets, float* G_out,
+                            float* loss_out, float* rewards_out, float* g_out) {
+  const bool down = layer == kLayerDown, attn = layer == kLayerAttnOut;
   if (!ctx) return DUST_ERR_ARG;
   char why[256];
   if (check_params(pp, DUST_VARIANT_MLP, why, sizeof(why)) != DUST_OK)
@@ -477,6 +484,8 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
   const dust_params p = *pp;
   if (!X || !W_up || !W_down || !W_head || !targets)
     return fail(ctx, DUST_ERR_ARG, "X, W_up, W_down, W_head and targets must be non-NULL");
+  if (attn && (!O || d_o < 1 || (d_o & 7) || !aligned(O, 16)))
+    return fail(ctx, DUST_ERR_ARG, "O must be non-NULL and 16-byte aligned, d_o >= 1 a multiple of 8");
   if (!aligned(X, 16) || !aligned(W_up, 16) || !aligned(W_down, 16) || !aligned(W_head, 16) ||
       !aligned(targets, 4) || !aligned(G_out, 4) || !aligned(loss_out, 4) ||
       !aligned(rewards_out, 4) || !aligned(g_out, 4))
@@ -489,7 +498,8 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
   DUST_TRY(ensure(ctx, ctx->mlp_h, (size_t)T * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->z, (size_t)T * V * 4));
   DUST_TRY(ensure(ctx, ctx->lse, (size_t)T * 4));
-  DUST_TRY(ensure(ctx, ctx->gop, down ? (size_t)T * d * 4 : gop_bytes(DUST_BF16, T, dff)));
+  DUST_TRY(ensure(ctx, ctx->gop, down ? (size_t)T * d * 4
+                                       : gop_bytes(DUST_BF16, T, attn ? d : dff)));
   float* loss = loss_out;
   if (!loss) {
     DUST_TRY(ensure(ctx, ctx->loss, (size_t)T * 4));
@@ -559,6 +569,15 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
   // tensor cores
   const int nparts = std::max((int)((V + 127) / 128), tc_partials_per_row(V));
   if (!down) DUST_TRY(ensure(ctx, ctx->mlp_da, (size_t)rows_cap * 2 * dff * 2));
+  if (attn) {
+    DUST_TRY(ensure(ctx, ctx->mlp_dn, (size_t)rows_cap * 2 * d * 2));
+    DUST_TRY(ensure(ctx, ctx->mlp_du, (size_t)rows_cap * dff * 4));
+    DUST_TRY(ensure(ctx, ctx->wu2, (size_t)dff * 2 * d * 2));
+    for (int half = 0; half < 2; ++half)
+      DUST_CU(cudaMemcpy2DAsync((char*)ctx->wu2.p + (size_t)half * d * 2, (size_t)2 * d * 2, W_up,
+                                (size_t)d * 2, (size_t)d * 2, (size_t)dff,
+                                cudaMemcpyDeviceToDevice, st));
+  }
   DUST_TRY(ensure(ctx, ctx->mlp_dh, (size_t)rows_cap * 2 * d * 2));
   DUST_TRY(ensure(ctx, ctx->part, (size_t)rows_cap * nparts * 4));
   DUST_TRY(ensure(ctx, ctx->dzy, (size_t)rows_cap * 4));
@@ -568,8 +587,31 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
     const int64_t nt = (t0 + tchunk <= T) ? tchunk : T - t0;
     const int64_t rows = nt * K;
     if (down) {
-      DUST_CU(launch_mlp_noise_split(st, p, t0, nt, dh));
+      DUST_CU(launch_mlp_noise_split(st, p, t0, nt, dh, kTagMlpDown));
       ctx->launches += 1;
+    } else if (attn) {
+      // sigma eps as planes; du = (sigma eps) W_up^T; da; dh = sigma eps + da W_down^T
+      __nv_bfloat16* dn = (__nv_bfloat16*)ctx->mlp_dn.p;
+      float* du = (float*)ctx->mlp_du.p;
+      DUST_CU(launch_mlp_noise_split(st, p, t0, nt, dn, kTagAttnOut));
+      ctx->launches += 1;
+      {
+        GemmDesc g{};
+        g.M = rows; g.N = dff; g.K = 2 * d; g.A = dn; g.lda = 2 * d; g.a_kmajor = true;
+        g.B = ctx->wu2.p; g.ldb = 2 * d; g.b_kmajor = true; g.dtype = DUST_BF16;
+        EpiDesc e{};
+        e.kind = kEpiF32; e.C = du; e.ldc = dff;
+        DUST_TRY(run_gemm(ctx, g, e));
+      }
+      DUST_CU(launch_gelu_delta_rows(st, p, u, du, t0, nt, da));
+      ctx->launches += 1;
+      GemmDesc g{};
+      g.M = rows; g.N = d; g.K = 2 * dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
+      g.B = ctx->wd2.p; g.ldb = 2 * dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      EpiDesc e{};
+      e.kind = kEpiResidSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
+      e.resid = dn; e.ldr = 2 * d; e.rsplit = d;
+      DUST_TRY(run_gemm(ctx, g, e));
     } else {
       DUST_CU(launch_mlp_delta_a(st, p, u, t0, nt, da, true, nullptr));
       ctx->launches += 1;
@@ -603,10 +645,17 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
     ctx->launches += 1;
   }
   mark(ctx, "perturbed");
-  DUST_CU(launch_mlp_g(st, p, r, g_out, ctx->gop.p, down));
+  if (attn)
+    DUST_CU(launch_noise_g_planes(st, p, r, g_out, (__nv_bfloat16*)ctx->gop.p, kTagAttnOut));
+  else
+    DUST_CU(launch_mlp_g(st, p, r, g_out, ctx->gop.p, down));
   ctx->launches += 1;
   mark(ctx, "g");
-  if (G_out && !down) {
+  if (G_out && attn) {
+    // G_o = sum_t g_t o_t^T: g as bf16 hi/lo planes against the bf16 O
+    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, d, O, d_o, G_out, 0));
+    mark(ctx, "gw_gemm");
+  } else if (G_out && !down) {
     DUST_TRY(weight_grad(ctx, p, ctx->gop.p, dff, X, d, G_out, 0));
     mark(ctx, "gw_gemm");
   } else if (G_out) {
@@ -627,16 +676,24 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, bool down, con
 dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* p, const void* X, const void* W_up,
                           const void* W_down, const void* W_head, const int32_t* targets,
                           float* G_up_out, float* loss_out, float* rewards_out, float* g_out) {
-  return mlp_impl(ctx, p, false, X, W_up, W_down, W_head, targets, G_up_out, loss_out,
-                  rewards_out, g_out);
+  return mlp_impl(ctx, p, kLayerUp, X, nullptr, 0, W_up, W_down, W_head, targets, G_up_out,
+                  loss_out, rewards_out, g_out);
 }
 
 dust_status dust_mlp_down_grad(dust_ctx* ctx, const dust_params* p, const void* X,
                                const void* W_up, const void* W_down, const void* W_head,
                                const int32_t* targets, float* G_down_out, float* loss_out,
                                float* rewards_out, float* g_out) {
-  return mlp_impl(ctx, p, true, X, W_up, W_down, W_head, targets, G_down_out, loss_out,
-                  rewards_out, g_out);
+  return mlp_impl(ctx, p, kLayerDown, X, nullptr, 0, W_up, W_down, W_head, targets, G_down_out,
+                  loss_out, rewards_out, g_out);
+}
+
+dust_status dust_attn_out_grad(dust_ctx* ctx, const dust_params* p, const void* X, const void* O,
+                               int64_t d_o, const void* W_up, const void* W_down,
+                               const void* W_head, const int32_t* targets, float* G_o_out,
+                               float* loss_out, float* rewards_out, float* g_out) {
+  return mlp_impl(ctx, p, kLayerAttnOut, X, O, d_o, W_up, W_down, W_head, targets, G_o_out,
+                  loss_out, rewards_out, g_out);
 }
 
 dust_status dust_set_stage_timing(dust_ctx* ctx, int enable) {

@@ -39,7 +39,8 @@ enum EpiKind {
   kEpiBF16 = 1,        // Cb[m*ldcb + n] = bf16(acc)
   kEpiGeluSplit = 2,   // C[m*ldc + n] = acc (u); a = GELU(acc) in fp64, stored as bf16
                        // hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
-  kEpiResidSplit = 3,  // h = resid[m*ldr + n] (bf16) + acc, stored as bf16 hi/lo planes
+  kEpiResidSplit = 3,  // h = resid[m*ldr + n] (bf16; plus resid[m*ldr + rsplit + n] when
+                       // rsplit > 0, a hi/lo pair) + acc, stored as bf16 hi/lo planes
   kEpiSplit = 4,       // acc stored as bf16 hi/lo planes Cb[m*ldcb + n], Cb[m*ldcb + split + n]
   kEpiReward = 5,      // MLP perturbed logits dz (never stored): per row m, 256-column
                        // tile nb and 128-column half h, part[(m*n_tiles + nb)*2 + h] =
@@ -60,6 +61,7 @@ struct EpiDesc {
   int64_t c_row_mul = 0;
   const void* resid = nullptr;
   int64_t ldr = 0;
+  int64_t rsplit = 0;
   // kEpiReward
   const float* P = nullptr;
   const int32_t* y = nullptr;
@@ -146,7 +148,7 @@ struct dust_ctx {
   bool subset2_enabled = true;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
-      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32;
+      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2;
 };
 
 namespace dust {
@@ -240,9 +242,17 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
 // or, with down, of the down-projection (width d; gop fp32).
 cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
                          void* gop, bool down);
-// Down-projection draws: dh = sigma eps as bf16 hi/lo planes (rows nt K x 2d).
+// g over width d with counter tag `tag`, gop as bf16 hi/lo planes (T x d each).
+cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const float* r,
+                                  float* g_out, __nv_bfloat16* gop, int tag);
+// Noise on a width-d output: sigma eps as bf16 hi/lo planes (rows nt K x 2d),
+// counter tag `tag` (down projection: 3; attention output projection: 4).
 cudaError_t launch_mlp_noise_split(cudaStream_t st, const dust_params& p, int64_t t0, int64_t nt,
-                                   __nv_bfloat16* dh);
+                                   __nv_bfloat16* dh, int tag);
+// da = GELU(u + du) - GELU(u) for rows (token, draw) of du (fp32, rows x d_ff),
+// as bf16 hi/lo planes (rows x 2 d_ff).
+cudaError_t launch_gelu_delta_rows(cudaStream_t st, const dust_params& p, const float* u,
+                                   const float* du, int64_t t0, int64_t nt, __nv_bfloat16* da);
 // a = GELU(u) (fp64, rounded to fp32), n elements.
 cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a, int sm_count);
 

@@ -104,7 +104,8 @@ __global__ __launch_bounds__(256) void k_gemm_simt(GemmDesc g, EpiDesc e) {
           split_bf16(gelu64((double)v), &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
           break;
         case kEpiResidSplit: {
-          const double r = (double)to_f(((const TI*)e.resid)[m * e.ldr + n]);
+          double r = (double)to_f(((const TI*)e.resid)[m * e.ldr + n]);
+          if (e.rsplit > 0) r += (double)to_f(((const TI*)e.resid)[m * e.ldr + e.rsplit + n]);
           split_bf16(r + (double)v, &e.Cb[m * e.ldcb + n], &e.Cb[m * e.ldcb + e.split + n]);
           break;
         }

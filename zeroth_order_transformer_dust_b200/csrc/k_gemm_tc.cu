@@ -125,11 +125,14 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
     __nv_bfloat16* hi = e.Cb + m * e.ldcb + n;
     __nv_bfloat16* lo = hi + e.split;
     const __nv_bfloat16* r = KIND == kEpiResidSplit ? (const __nv_bfloat16*)e.resid + m * e.ldr + n : nullptr;
+    const __nv_bfloat16* r2 = (KIND == kEpiResidSplit && e.rsplit > 0) ? r + e.rsplit : nullptr;
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
       if (n + q < p.N) {
-        const double x = KIND == kEpiGeluSplit ? gelu64((double)v[q])
-                                               : (double)__bfloat162float(r[q]) + (double)v[q];
+        const double x = KIND == kEpiGeluSplit
+                             ? gelu64((double)v[q])
+                             : (double)__bfloat162float(r[q]) +
+                                   (r2 ? (double)__bfloat162float(r2[q]) : 0.0) + (double)v[q];
         split_bf16(x, hi + q, lo + q);
       }
     }

@@ -149,6 +149,57 @@ __global__ __launch_bounds__(256) void k_mlp_noise_split(RoundKeys keys, uint32_
   }
 }
 
+// da = GELU(u + du) - GELU(u) for rows (token, draw) with du varying per
+// element (the attention output-projection variant: du = sigma eps W_up^T).
+// One warp per (token, 128-channel block) forms the Taylor coefficients of
+// GELU at its channels' u once (as the up-projection kernel above) and walks
+// the token's draws; the expansion serves |du| <= 1/16 (remainder < 2.3e-8),
+// the quadrature form (gelu_delta) the rare larger du.
+__global__ __launch_bounds__(256) void k_gelu_delta_rows(int64_t d_ff, int32_t K,
+                                                         const float* __restrict__ u,
+                                                         const float* __restrict__ du, int64_t t0,
+                                                         int64_t nt,
+                                                         __nv_bfloat16* __restrict__ da) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nblk = (d_ff + 127) / 128;
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= nt * nblk) return;
+  const int64_t tl = wid / nblk;
+  const int64_t blk = wid % nblk;
+  const int64_t t = t0 + tl;
+  float uu[4], c1[4], c2[4], c3[4], c4[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t ch = blk * 128 + lane + 32 * j;
+    uu[j] = ch < d_ff ? u[t * d_ff + ch] : 0.0f;
+    const double x = (double)uu[j];
+    const double phi = 0.3989422804014327 * exp(-0.5 * x * x);
+    const double Phi = 0.5 * erfc(-x * 0.7071067811865476);
+    const double x2 = x * x;
+    c1[j] = (float)(Phi + x * phi);
+    c2[j] = (float)(phi * (2.0 - x2) * 0.5);
+    c3[j] = (float)(phi * x * (x2 - 4.0) * (1.0 / 6.0));
+    c4[j] = (float)(phi * (7.0 * x2 - x2 * x2 - 4.0) * (1.0 / 24.0));
+  }
+  for (int32_t i = 0; i < K; ++i) {
+    const int64_t row = tl * K + i;
+    __nv_bfloat16* rowp = da + row * 2 * d_ff;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t ch = blk * 128 + lane + 32 * j;
+      if (ch < d_ff) {
+        const float dd = du[row * d_ff + ch];
+        float a;
+        if (fabsf(dd) <= 0.0625f)
+          a = dd * fmaf(dd, fmaf(dd, fmaf(dd, c4[j], c3[j]), c2[j]), c1[j]);
+        else
+          a = gelu_delta(uu[j], dd);
+        split_bf16(a, rowp + ch, rowp + d_ff + ch);
+      }
+    }
+  }
+}
+
 // a = GELU(u) in fp64, rounded once to fp32 (the down-projection's input,
 // the right-hand operand of its weight gradient).
 __global__ void k_gelu_f32(const float* __restrict__ u, int64_t n, float* __restrict__ a) {
@@ -312,12 +363,30 @@ cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const floa
 }
 
 cudaError_t launch_mlp_noise_split(cudaStream_t st, const dust_params& p, int64_t t0, int64_t nt,
-                                   __nv_bfloat16* dh) {
+                                   __nv_bfloat16* dh, int tag) {
   const int64_t warps = nt * ((p.d + 127) / 128);
   if (warps <= 0) return cudaSuccess;
   k_mlp_noise_split<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(
       round_keys(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
-      ctr3_of(kTagMlpDown, p.stream_id), p.sigma, p.d, p.K, t0, nt, dh);
+      ctr3_of(tag, p.stream_id), p.sigma, p.d, p.K, t0, nt, dh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gelu_delta_rows(cudaStream_t st, const dust_params& p, const float* u,
+                                   const float* du, int64_t t0, int64_t nt, __nv_bfloat16* da) {
+  const int64_t warps = nt * ((p.d_ff + 127) / 128);
+  if (warps <= 0) return cudaSuccess;
+  k_gelu_delta_rows<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p.d_ff, p.K, u, du, t0, nt, da);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const float* r,
+                                  float* g_out, __nv_bfloat16* gop, int tag) {
+  dim3 grid((unsigned)p.T, (unsigned)((p.d + 1023) / 1024));
+  const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
+  k_noise_g<__nv_bfloat16><<<grid, 256, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
+      (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.d, p.K, r, g_out, gop,
+      p.T * p.d);
   return cudaGetLastError();
 }
 

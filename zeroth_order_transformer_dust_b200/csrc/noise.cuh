@@ -21,6 +21,7 @@ constexpr int kTagHead = 0;
 constexpr int kTagSubsetOffset = 1;
 constexpr int kTagMlpUp = 2;
 constexpr int kTagMlpDown = 3;
+constexpr int kTagAttnOut = 4;
 
 struct U4 {
   uint32_t x, y, z, w;
