@@ -263,7 +263,10 @@ dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, cons
    2 = tcgen05 tensor cores with one CTA per 128 x 256 tile, 3 = tcgen05 with
    CTA pairs (cta_group::2) per 256 x 256 tile (2 and 3 return
    DUST_ERR_UNSUPPORTED when the shape does not fit: K a multiple of 8 and
-   N >= 16 are needed). Synchronous. */
+   N >= 16 are needed), 4 = path 2 with an injected failure: the pipeline's
+   bounded waits give up at once, the kernel drains its copies and MMAs, frees
+   its TMEM and returns, and the call reports DUST_ERR_TIMEOUT with C
+   undefined (the context stays usable). Synchronous. */
 dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
                                  const void* B, float* C, int path);
 

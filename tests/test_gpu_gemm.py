@@ -71,3 +71,18 @@ def test_pair_and_single_cta_paths_agree(ctx):
     B = torch.randn(3000, 768, device="cuda", generator=g).to(torch.bfloat16)
     c2, c3 = ctx.debug_gemm(A, B, path=2), ctx.debug_gemm(A, B, path=3)
     assert ((c2 - c3).norm() / c2.norm()).item() < 1e-6
+
+
+def test_injected_timeout_is_reported_and_the_context_recovers(ctx):
+    # path 4: the tensor-core GEMM with its pipeline waits limited to zero. The
+    # kernel gives up, drains its own copies and MMAs, frees TMEM and returns;
+    # the call reports DUST_ERR_TIMEOUT and the next call runs normally.
+    g = torch.Generator(device="cuda").manual_seed(9)
+    A = torch.randn(4096, 4096, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(2048, 4096, device="cuda", generator=g).to(torch.bfloat16)
+    with pytest.raises(dust.DustError) as ei:
+        ctx.debug_gemm(A, B, path=4)
+    assert ei.value.status == 5
+    C = ctx.debug_gemm(A, B, path=2)
+    ref = A.float() @ B.float().T
+    assert ((C - ref).norm() / ref.norm()).item() < 1e-5

@@ -325,7 +325,8 @@ class Context:
     # -- debug exports -------------------------------------------------------------
     def debug_gemm(self, A: torch.Tensor, B: torch.Tensor, path: int = 0) -> torch.Tensor:
         """C = A B^T (bf16 operands, fp32 out); path 0 auto, 1 CUDA cores, 2 tensor cores
-        (one CTA per tile), 3 tensor cores with CTA pairs."""
+        (one CTA per tile), 3 tensor cores with CTA pairs, 4 path 2 with an injected
+        timeout of its pipeline waits (raises DustError with DUST_ERR_TIMEOUT)."""
         self._dev(A, "A"), self._dev(B, "B")
         if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
             raise TypeError("A and B must be bfloat16")

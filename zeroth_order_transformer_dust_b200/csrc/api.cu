@@ -136,14 +136,16 @@ dust_status finish(dust_ctx* ctx, uint32_t flags) {
 
 // path: 0 automatic, 1 CUDA cores, 2 tensor cores.
 // path: 0 automatic, 1 CUDA cores, 2 tensor cores one CTA per tile, 3 tensor
-// cores with CTA pairs.
+// cores with CTA pairs, 4 as 2 with the pipeline waits' limit at zero (an
+// injected timeout).
 dust_status run_gemm(dust_ctx* ctx, const GemmDesc& g, const EpiDesc& e, int path = 0) {
   const bool tc = path != 1 && (path >= 2 || ctx->tc_enabled) && tc_gemm_supported(g, e);
   if (path >= 2 && !tc) return fail(ctx, DUST_ERR_UNSUPPORTED, "shape not taken by the tensor-core GEMM");
   ctx->launches += 1;
   if (tc) {
     const bool pair = path == 3 || (path == 0 && ctx->tc_pair && g.M >= 256);
-    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count, ctx->d_status, pair));
+    DUST_CU(launch_gemm_tc(ctx->stream, g, e, ctx->sm_count, ctx->d_status, pair,
+                           path == 4 ? kWaitLimitOff : 0));
   } else {
     DUST_CU(launch_gemm_simt(ctx->stream, g, e));
   }
@@ -729,7 +731,7 @@ int64_t dust_kernel_launches(const dust_ctx* ctx) { return ctx ? ctx->launches :
 dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
                                  const void* B, float* C, int path) {
   if (!ctx) return DUST_ERR_ARG;
-  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || path < 0 || path > 3)
+  if (M < 1 || N < 1 || K < 1 || !A || !B || !C || path < 0 || path > 4)
     return fail(ctx, DUST_ERR_ARG, "bad gemm arguments");
   DUST_CU(cudaSetDevice(ctx->device));
   DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), ctx->stream));

@@ -217,8 +217,11 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
 // 256 x 256 tile per cluster of two CTAs, cta_group::2; else 128 x 256 per
 // CTA). A bounded wait that expires sets kStatusTimeout in *status.
 bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e);
+// wait_ns: limit of the pipeline's bounded waits (0: the default 2 s;
+// kWaitLimitOff: give up at once, the failure-injection path of the debug GEMM).
+constexpr uint64_t kWaitLimitOff = ~0ull;
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
-                           uint32_t* status, bool pair);
+                           uint32_t* status, bool pair, uint64_t wait_ns = 0);
 
 // Transpose of a row-major bf16 matrix (rows x cols) into dst (cols x rows,
 // row stride ld_dst >= rows; columns [rows, ld_dst) of dst are zeroed).

@@ -56,6 +56,7 @@ struct TcParams {
   int m_tiles, n_tiles, num_kb;  // m_tiles counts Cfg::TILE_M-row tiles
   EpiDesc e;
   uint32_t* status;
+  uint64_t wait_ns;  // limit of the pipeline waits (teardown waits keep kWaitLimitNs)
 };
 
 struct Shared {
@@ -65,14 +66,24 @@ struct Shared {
 };
 static_assert(sizeof(Shared) <= 256, "barrier block overlaps the staging area");
 
-__device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+// Wait for phase `parity` of an mbarrier for at most limit_ns (0: a single
+// poll). On expiry the CTA's abort flag and the timeout bit of the status word
+// are set and false returns; a raised abort flag (checked every 64 polls)
+// also ends the wait.
+__device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* status,
+                             uint64_t limit_ns = kWaitLimitNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) {
+    *abort = 1;
+    atomicOr(status, kStatusTimeout);
+    return false;
+  }
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (ptx::globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(status, kStatusTimeout);
         return false;
@@ -121,19 +132,51 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
         if (n + q < p.N) dst[q] = __float2bfloat16_rn(v[q]);
     }
   }
-  if (KIND == kEpiGeluSplit || KIND == kEpiResidSplit) {
+  if (KIND == kEpiGeluSplit) {
     __nv_bfloat16* hi = e.Cb + m * e.ldcb + n;
     __nv_bfloat16* lo = hi + e.split;
-    const __nv_bfloat16* r = KIND == kEpiResidSplit ? (const __nv_bfloat16*)e.resid + m * e.ldr + n : nullptr;
-    const __nv_bfloat16* r2 = (KIND == kEpiResidSplit && e.rsplit > 0) ? r + e.rsplit : nullptr;
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      if (n + q < p.N) {
-        const double x = KIND == kEpiGeluSplit
-                             ? gelu64((double)v[q])
-                             : (double)__bfloat162float(r[q]) +
-                                   (r2 ? (double)__bfloat162float(r2[q]) : 0.0) + (double)v[q];
-        split_bf16(x, hi + q, lo + q);
+    for (int q = 0; q < 32; ++q)
+      if (n + q < p.N) split_bf16(gelu64((double)v[q]), hi + q, lo + q);
+  }
+  if (KIND == kEpiResidSplit) {
+    // h = resid (+ its lo plane) + acc in fp32 (error 2^-24 relative), then
+    // the 2^-17 hi/lo split; 16-byte loads and stores when the row is aligned
+    __nv_bfloat16* hi = e.Cb + m * e.ldcb + n;
+    __nv_bfloat16* lo = hi + e.split;
+    const __nv_bfloat16* r = (const __nv_bfloat16*)e.resid + m * e.ldr + n;
+    const __nv_bfloat16* r2 = e.rsplit > 0 ? r + e.rsplit : nullptr;
+    const bool vec = full && ((e.ldcb | e.split | e.ldr | e.rsplit) & 7) == 0 &&
+                     (((uintptr_t)e.Cb | (uintptr_t)e.resid) & 15) == 0;
+    if (vec) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 ra = reinterpret_cast<const uint4*>(r)[q];
+        const uint4 rb = r2 ? reinterpret_cast<const uint4*>(r2)[q] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const __nv_bfloat162 pa = *reinterpret_cast<const __nv_bfloat162*>(&wa[h]);
+          const __nv_bfloat162 pb = *reinterpret_cast<const __nv_bfloat162*>(&wb[h]);
+          const float x0 = __low2float(pa) + __low2float(pb) + v[8 * q + 2 * h];
+          const float x1 = __high2float(pa) + __high2float(pb) + v[8 * q + 2 * h + 1];
+          const __nv_bfloat162 hh = __floats2bfloat162_rn(x0, x1);
+          const __nv_bfloat162 ll = __floats2bfloat162_rn(x0 - __low2float(hh), x1 - __high2float(hh));
+          hw[h] = *reinterpret_cast<const uint32_t*>(&hh);
+          lw[h] = *reinterpret_cast<const uint32_t*>(&ll);
+        }
+        reinterpret_cast<uint4*>(hi)[q] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        reinterpret_cast<uint4*>(lo)[q] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        if (n + q < p.N) {
+          float x = __bfloat162float(r[q]) + v[q];
+          if (r2) x += __bfloat162float(r2[q]);
+          split_bf16(x, hi + q, lo + q);
+        }
       }
     }
   }
@@ -293,7 +336,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
         const int a_row = m_blk * TILE_M + (int)rank * BM;
         const int b_row = n_blk * BN + (int)rank * C::B_ROWS;
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!wait_bounded(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort, p.status)) break;
+          if (!wait_bounded(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort, p.status, p.wait_ns)) break;
           const uint32_t fb = ptx::smem_u32(&sh->full[stage]);
           if (PAIR) {
             // both CTAs' bytes complete on the leader's barrier
@@ -337,12 +380,12 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
       for (int tile = unit0; tile < total && !*abort; tile += units, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
-        if (!wait_bounded(ptx::smem_u32(&sh->tempty[acc]), acc_phase ^ 1u, abort, p.status)) break;
+        if (!wait_bounded(ptx::smem_u32(&sh->tempty[acc]), acc_phase ^ 1u, abort, p.status, p.wait_ns)) break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!wait_bounded(ptx::smem_u32(&sh->full[stage]), phase, abort, p.status)) {
+          if (!wait_bounded(ptx::smem_u32(&sh->full[stage]), phase, abort, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -434,7 +477,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           }
         }
       }
-      if (!wait_bounded(ptx::smem_u32(&sh->tfull[acc]), acc_phase, abort, p.status)) break;
+      if (!wait_bounded(ptx::smem_u32(&sh->tfull[acc]), acc_phase, abort, p.status, p.wait_ns)) break;
       ptx::tc_fence_after();
       const int64_t m = (int64_t)m_blk * TILE_M + (int64_t)rank * BM + row;
       int64_t mo = m;
@@ -587,7 +630,7 @@ namespace {
 
 template <bool PAIR>
 cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
-                        uint32_t* status) {
+                        uint32_t* status, uint64_t wait_ns) {
   CUtensorMap ma, mb;
   if (!make_map(&ma, g.A, g.M, g.K, g.lda, BM) ||
       !make_map(&mb, g.B, g.N, g.K, g.ldb, Cfg<PAIR>::B_ROWS))
@@ -601,6 +644,7 @@ cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, in
   p.num_kb = (int)((g.K + BK - 1) / BK);
   p.e = e;
   p.status = status;
+  p.wait_ns = wait_ns;
   if (!p.status) return cudaErrorInvalidValue;
   switch (e.kind) {
     case kEpiF32: return launch_kind<kEpiF32, PAIR>(st, ma, mb, p, sm_count);
@@ -617,9 +661,11 @@ cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, in
 }  // namespace
 
 cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
-                           uint32_t* status, bool pair) {
-  if (pair && sm_count >= 2) return launch_pair<true>(st, g, e, sm_count, status);
-  return launch_pair<false>(st, g, e, sm_count, status);
+                           uint32_t* status, bool pair, uint64_t wait_ns) {
+  if (wait_ns == 0) wait_ns = kWaitLimitNs;
+  if (wait_ns == kWaitLimitOff) wait_ns = 0;  // injected failure: one poll per pipeline wait
+  if (pair && sm_count >= 2) return launch_pair<true>(st, g, e, sm_count, status, wait_ns);
+  return launch_pair<false>(st, g, e, sm_count, status, wait_ns);
 }
 
 }  // namespace dust

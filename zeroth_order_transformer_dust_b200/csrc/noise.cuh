@@ -94,10 +94,17 @@ __device__ __forceinline__ float sqrt_approx(float x) {
   asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// base-2 logarithm (MUFU.LG2) for normal arguments: u1 >= 2^-24, so the
+// flush-to-zero form needs no subnormal fix-up
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ float bm_radius(uint32_t wa) {
   const float u = fmaf((float)(wa >> 8), 5.9604645e-08f, 5.9604645e-08f);  // exact
-  const float far = __log2f(u) * -1.3862944f;                             // -2 ln 2
+  const float far = lg2_approx(u) * -1.3862944f;                          // -2 ln 2
   const float v = 1.0f - u;  // exact (u >= 1/2 where it is used)
   const float near = v * fmaf(v, fmaf(v, 2.0f / 3.0f, 1.0f), 2.0f);
   return sqrt_approx(v < 0.015625f ? near : far);
