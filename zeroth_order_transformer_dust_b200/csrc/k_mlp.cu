@@ -181,20 +181,34 @@ __global__ __launch_bounds__(256) void k_gelu_delta_rows(int64_t d_ff, int32_t K
     c3[j] = (float)(phi * x * (x2 - 4.0) * (1.0 / 6.0));
     c4[j] = (float)(phi * (7.0 * x2 - x2 * x2 - 4.0) * (1.0 / 24.0));
   }
-  for (int32_t i = 0; i < K; ++i) {
-    const int64_t row = tl * K + i;
-    __nv_bfloat16* rowp = da + row * 2 * d_ff;
+  // draws in groups of 4: the group's du loads are issued together, so each
+  // warp keeps 16 loads in flight (the kernel streams du from HBM)
+  constexpr int G = 4;
+  for (int32_t i0 = 0; i0 < K; i0 += G) {
+    float dd[G][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t ch = blk * 128 + lane + 32 * j;
-      if (ch < d_ff) {
-        const float dd = du[row * d_ff + ch];
-        float a;
-        if (fabsf(dd) <= 0.0625f)
-          a = dd * fmaf(dd, fmaf(dd, fmaf(dd, c4[j], c3[j]), c2[j]), c1[j]);
-        else
-          a = gelu_delta(uu[j], dd);
-        split_bf16(a, rowp + ch, rowp + d_ff + ch);
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t ch = blk * 128 + lane + 32 * j;
+        dd[g][j] = (i0 + g < K && ch < d_ff) ? du[(tl * K + i0 + g) * d_ff + ch] : 0.0f;
+      }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (i0 + g >= K) break;
+      __nv_bfloat16* rowp = da + (tl * K + i0 + g) * 2 * d_ff;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t ch = blk * 128 + lane + 32 * j;
+        if (ch < d_ff) {
+          const float x = dd[g][j];
+          float a;
+          if (fabsf(x) <= 0.0625f)
+            a = x * fmaf(x, fmaf(x, fmaf(x, c4[j], c3[j]), c2[j]), c1[j]);
+          else
+            a = gelu_delta(uu[j], x);
+          split_bf16(a, rowp + ch, rowp + d_ff + ch);
+        }
       }
     }
   }
