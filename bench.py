@@ -221,6 +221,14 @@ def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
             "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)"}
 
 
+def _config(args, wl, world: int, l2: str) -> dict:
+    """The workload of a JSON line (the same keys on both arms)."""
+    return {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
+            "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype, "d_ff": wl.d_ff, "l2": l2,
+            "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL all-reduce"
+                            if world > 1 else "dp1")}
+
+
 # ----------------------------------------------------------------------------- main arms
 def run_reference(args):
     world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
@@ -241,8 +249,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": wl.token_draws / value * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": args.config, "T": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
-                       "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype},
+            "config": _config(args, wl, 1, "the oracle runs on the host (no L2 flush)"),
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -394,11 +401,7 @@ def run_dust(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic",
-                "config": {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V,
-                           "K": wl.K, "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype,
-                           "d_ff": wl.d_ff, "l2": "flushed between timed steps (256 MiB write)",
-                           "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL "
-                                           "all-reduce" if world > 1 else "dp1")},
+                "config": _config(args, wl, world, "flushed between timed steps (256 MiB write)"),
                 "stage_ms": stages, "gpu_launches": launches, "e2e": e2e, "roofline": roof,
                 "cpu_baseline": cb, "clocks": clk, "alignment": align, **extra}
         print(json.dumps(line), flush=True)
