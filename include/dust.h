@@ -283,14 +283,21 @@ dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag,
 dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t tag,
                                  int64_t nt, int64_t ni, int64_t nslots, float* out);
 
-/* Debug: the Box-Muller radius for every 24-bit input. out (2^24 fp32,
-   device) receives sigma sqrt(-2 ln u1) for u1 = (j + 1) 2^-24 at index j, as
-   every noise kernel computes it (the pages fix only Gaussian noise; this
-   transform is the library's). Synchronous. */
-dust_status dust_debug_bm_radius(dust_ctx* ctx, float sigma, float* out);
+/* Debug: the Box-Muller radius for every 24-bit input (the pages fix only
+   Gaussian noise; this transform is the library's). out (2^24 fp32, device)
+   receives, at index j, for u1 = (j + 1) 2^-24:
+     method 0: sigma sqrt(-2 ln u1) as the polynomial angle step forms it
+               (sigma sqrt(2 ln 2) times rho);
+     method 1: rho = sqrt(-log2 u1), the factor the table angle step
+               multiplies into its table (sigma is not used).
+   sigma must be finite and >= 0. Synchronous. */
+dust_status dust_debug_bm_radius(dust_ctx* ctx, int32_t method, float sigma, float* out);
 /* Debug: the Box-Muller angle step for every 24-bit input. out (2 x 2^24
-   fp32, device) receives (cos, sin) of 2 pi m 2^-24 at [2m, 2m+1]; method 0 is
-   the polynomial step (MLP noise), 1 the table step (LM-head noise).
+   fp32, device) receives at [2m, 2m+1], for the angle 2 pi m 2^-24:
+     method 0: (cos, sin), the polynomial step (MLP noise);
+     method 1: sqrt(2 ln 2) (cos, sin), the table step (LM-head noise) with
+               sigma = 1, whose table carries the radius factor that rho
+               leaves out.
    Synchronous. */
 dust_status dust_debug_bm_angle(dust_ctx* ctx, int32_t method, float* out);
 

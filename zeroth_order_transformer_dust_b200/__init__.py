@@ -93,7 +93,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "dust_debug_gauss_tab": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_head_grad_noalloc": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_char_p,
                                              ctypes.c_int]),
-            "dust_debug_bm_radius": (I32, [P, ctypes.c_float, P]),
+            "dust_debug_bm_radius": (I32, [P, I32, ctypes.c_float, P]),
             "dust_debug_bm_angle": (I32, [P, I32, P]),
             "dust_sgd_momentum": (I32, [P, I64, ctypes.c_float, ctypes.c_float, P, P, P, P]),
         }
@@ -357,15 +357,19 @@ class Context:
         self._check(fn(self._h, ctypes.byref(prm), tag, nt, ni, nslots, _ptr(out)))
         return out
 
-    def debug_bm_radius(self, sigma: float = 1.0) -> torch.Tensor:
-        """Box-Muller radius sigma sqrt(-2 ln u1) for every u1 = (j + 1) 2^-24, j < 2^24."""
+    def debug_bm_radius(self, sigma: float = 1.0, table: bool = False) -> torch.Tensor:
+        """For every u1 = (j + 1) 2^-24, j < 2^24: the radius sigma sqrt(-2 ln u1)
+        of the polynomial angle step, or (table=True) rho = sqrt(-log2 u1), the
+        factor of the table step."""
         out = torch.empty(1 << 24, dtype=torch.float32, device=f"cuda:{self.device}")
         self._bind_stream()
-        self._check(self._L.dust_debug_bm_radius(self._h, float(sigma), _ptr(out)))
+        self._check(self._L.dust_debug_bm_radius(self._h, 1 if table else 0, float(sigma),
+                                                 _ptr(out)))
         return out
 
     def debug_bm_angle(self, table: bool) -> torch.Tensor:
-        """(cos, sin) of 2 pi m 2^-24 for every m < 2^24 (2^24 x 2)."""
+        """(cos, sin) of 2 pi m 2^-24 for every m < 2^24 (2^24 x 2); the table
+        step returns them times sqrt(2 ln 2)."""
         out = torch.empty(1 << 24, 2, dtype=torch.float32, device=f"cuda:{self.device}")
         self._bind_stream()
         self._check(self._L.dust_debug_bm_angle(self._h, 1 if table else 0, _ptr(out)))

@@ -795,12 +795,12 @@ dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, cons
   return DUST_OK;
 }
 
-dust_status dust_debug_bm_radius(dust_ctx* ctx, float sigma, float* out) {
+dust_status dust_debug_bm_radius(dust_ctx* ctx, int32_t method, float sigma, float* out) {
   if (!ctx) return DUST_ERR_ARG;
-  if (!out || !(sigma >= 0.0f) || !std::isfinite(sigma))
+  if (!out || method < 0 || method > 1 || !(sigma >= 0.0f) || !std::isfinite(sigma))
     return fail(ctx, DUST_ERR_ARG, "bad radius arguments");
   DUST_CU(cudaSetDevice(ctx->device));
-  DUST_CU(launch_debug_bm(ctx->stream, 0, sigma, out));
+  DUST_CU(launch_debug_bm(ctx->stream, method == 1 ? 3 : 0, sigma, out));
   ctx->launches += 1;
   DUST_CU(cudaStreamSynchronize(ctx->stream));
   return DUST_OK;

@@ -81,9 +81,11 @@ __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off
 
 // Every value of the two Box-Muller inputs: radius(j) for u1 = (j + 1) 2^-24
 // and (cos, sin) of 2 pi m 2^-24, with the device functions the kernels use.
-__global__ void k_debug_bm_radius(float sigma, float* __restrict__ out) {
+// method 0: the radius sigma R as the polynomial-angle step forms it;
+// method 1: rho = R / sqrt(2 ln 2), the factor the table step uses.
+__global__ void k_debug_bm_radius(int method, float sigma, float* __restrict__ out) {
   const uint32_t j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j < (1u << 24)) out[j] = sigma * bm_radius(j << 8);
+  if (j < (1u << 24)) out[j] = method == 1 ? bm_rho(j << 8) : (sigma * kRhoToR) * bm_rho(j << 8);
 }
 
 __global__ __launch_bounds__(256) void k_debug_bm_angle(int method, float* __restrict__ out) {
@@ -106,8 +108,8 @@ __global__ __launch_bounds__(256) void k_debug_bm_angle(int method, float* __res
 }
 
 cudaError_t launch_debug_bm(cudaStream_t st, int what, float sigma, float* out) {
-  if (what == 0)
-    k_debug_bm_radius<<<(1u << 24) / 256, 256, 0, st>>>(sigma, out);
+  if (what == 0 || what == 3)
+    k_debug_bm_radius<<<(1u << 24) / 256, 256, 0, st>>>(what == 3 ? 1 : 0, sigma, out);
   else
     k_debug_bm_angle<<<4096, 256, 0, st>>>(what == 2 ? 1 : 0, out);
   return cudaGetLastError();

@@ -81,14 +81,17 @@ __device__ __forceinline__ void sincos_turn24(uint32_t m, float* s_out, float* c
 }
 
 // Radius of the Box-Muller pair, R = sqrt(-2 ln u1), for
-// u1 = ((wa >> 8) + 1) 2^-24 (exact in fp32). Away from u1 = 1, ln u1 comes
-// from the hardware base-2 logarithm of u1 (MUFU.LG2). Its error near u1 = 1
-// is absolute (about 2^-23), which the square root turns into a radius error
-// of about 0.7 2^-23 / R, so for v = 1 - u1 < 2^-6 (exact; R < 0.18) the
-// series -2 ln(1 - v) = 2v + v^2 + (2/3) v^3 + ... is used instead (the
-// first omitted term, v^4/2, is below 2^-19 relative there). The square root
-// is the hardware approximation (MUFU.SQRT, sqrt(0) = 0). Checked over all
-// 2^24 values of u1 against fp64: below 8e-7 absolute.
+// u1 = ((wa >> 8) + 1) 2^-24 (exact in fp32), carried as
+// rho = R / sqrt(2 ln 2) = sqrt(-log2 u1): the constant sqrt(2 ln 2) is
+// folded into the angle table (or into the caller's scale) instead of
+// costing a multiply per pair. Away from u1 = 1, log2 u1 is the hardware
+// base-2 logarithm (MUFU.LG2). Its error near u1 = 1 is absolute (about
+// 2^-23), which the square root turns into an error of about 0.5 2^-23 / rho,
+// so for v = 1 - u1 < 2^-6 (exact; R < 0.18) the series
+// -log2(1 - v) = (v + v^2/2 + v^3/3 + ...) / ln 2 is used instead (the first
+// omitted term is below 2^-19 relative there). The square root is the
+// hardware approximation (MUFU.SQRT, sqrt(0) = 0). Checked over all 2^24
+// values of u1 against fp64.
 __device__ __forceinline__ float sqrt_approx(float x) {
   float y;
   asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -102,18 +105,20 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ float bm_radius(uint32_t wa) {
+constexpr float kRhoToR = 1.1774100f;  // sqrt(2 ln 2)
+
+__device__ __forceinline__ float bm_rho(uint32_t wa) {
   const float u = fmaf((float)(wa >> 8), 5.9604645e-08f, 5.9604645e-08f);  // exact
-  const float far = lg2_approx(u) * -1.3862944f;                          // -2 ln 2
   const float v = 1.0f - u;  // exact (u >= 1/2 where it is used)
-  const float near = v * fmaf(v, fmaf(v, 2.0f / 3.0f, 1.0f), 2.0f);
-  return sqrt_approx(v < 0.015625f ? near : far);
+  // log2(1 - v) = -(v + v^2/2 + v^3/3) / ln 2, truncated
+  const float near = v * fmaf(v, fmaf(v, -0.48089835f, -0.7213475f), -1.442695f);
+  return sqrt_approx(-(v < 0.015625f ? near : lg2_approx(u)));
 }
 
 // Box-Muller on 24-bit uniforms: u1 = ((wa>>8)+1) 2^-24, u2 = (wb>>8) 2^-24;
 // returns scale * (R cos 2 pi u2, R sin 2 pi u2), R = sqrt(-2 ln u1).
 __device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb, float scale = 1.0f) {
-  const float radius = scale * bm_radius(wa);
+  const float radius = (scale * kRhoToR) * bm_rho(wa);
   float s, c;
   sincos_turn24(wb >> 8, &s, &c);
   return make_float2(radius * c, radius * s);
@@ -121,37 +126,40 @@ __device__ __forceinline__ float2 box_muller(uint32_t wa, uint32_t wb, float sca
 
 // Table-driven variant of the angle step, for kernels that keep 1024 roots of
 // unity at interval midpoints, theta_k = 2 pi (k + 1/2) / 1024, in shared
-// memory, already scaled by sigma: tab[k] = sigma (cos theta_k, sin theta_k).
+// memory, already scaled by sigma sqrt(2 ln 2) (the radius factor that
+// bm_rho leaves out): tab[k] = sigma sqrt(2 ln 2) (cos theta_k, sin theta_k).
 // The 24-bit angle m = wb >> 8 is interval wb >> 22 plus the remainder
 // x = c xr, c = 2 pi 2^-32, xr = (r - 2^13) 2^8 with r bits 8..21 of wb
-// (|x| <= pi/1024; xr's float comes exactly from an exponent-bias
-// construction), and cos/sin follow from the angle-addition formulas with
-// cos x = 1 - x^2/2 and sin x = x (truncation below 5e-9). Checked over all
-// 2^24 angles (sigma = 1): below 2e-7 absolute.
+// (|x| <= pi/1024). The float F = 1.5 2^23 + r 2^8 comes exactly from an
+// exponent-bias construction and x = fma(F, c, -(1.5 2^23 + 2^21) c) in one
+// rounding (the rounded constant moves x by under 1e-9). cos/sin follow from
+// the angle-addition formulas with cos x = 1 - x^2/2 and sin x = x
+// (truncation below 5e-9). Checked over all 2^24 angles (sigma = 1) against
+// sqrt(2 ln 2) (cos, sin) in fp64.
 constexpr int kSinCosTable = 1024;
 
 __device__ __forceinline__ void fill_sincos_table(float2* tab, float sigma) {
+  const float scale = sigma * kRhoToR;
   for (int k = threadIdx.x; k < kSinCosTable; k += blockDim.x) {
     float s, c;
     sincospif((float)(2 * k + 1) * (1.0f / kSinCosTable), &s, &c);
-    tab[k] = make_float2(sigma * c, sigma * s);
+    tab[k] = make_float2(scale * c, scale * s);
   }
 }
 
-// sigma (cos, sin) of the angle of word wb.
+// sigma sqrt(2 ln 2) (cos, sin) of the angle of word wb.
 __device__ __forceinline__ float2 rotate_tab(uint32_t wb, const float2* tab) {
-  // 1.5 2^23 + (r << 8) minus (1.5 2^23 + 2^21): (r - 2^13) 2^8, exact
-  const float xr = __int_as_float((wb & 0x003FFF00u) | 0x4B400000u) - 14680064.0f;
-  const float x = xr * 1.4629181e-09f;  // 2 pi 2^-32
+  const float F = __int_as_float((wb & 0x003FFF00u) | 0x4B400000u);
+  const float x = fmaf(F, 1.4629181e-09f, -0.021475732f);  // c = 2 pi 2^-32
   const float2 t = tab[wb >> 22];
   const float q = fmaf(x * x, -0.5f, 1.0f);
   return make_float2(fmaf(-t.y, x, t.x * q), fmaf(t.x, x, t.y * q));
 }
 
 __device__ __forceinline__ float2 box_muller_tab(uint32_t wa, uint32_t wb, const float2* tab) {
-  const float R = bm_radius(wa);
+  const float rho = bm_rho(wa);
   const float2 cs = rotate_tab(wb, tab);
-  return make_float2(R * cs.x, R * cs.y);
+  return make_float2(rho * cs.x, rho * cs.y);
 }
 
 // Four Gaussians of one counter (times `scale`): element j is output word j.
