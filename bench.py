@@ -44,9 +44,9 @@ LANES_PER_SM = 128           # 4 schedulers x 32 lanes issue per clock
 ALU_OPS_PER_ELEM = 20
 # DRAM bytes (read + write) per token of the subset-draw kernel on the
 # large-subset workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of
-# one launch over its first 2048 tokens (415.06 + 368.20 MB), per token; the
+# one launch over its first 2048 tokens (415.25 + 367.58 MB), per token; the
 # kernel's traffic is per token (the logit row in, the g operand planes out).
-SUBSET_DRAM_BYTES_PER_TOKEN = (415.059456e6 + 368.201984e6) / 2048
+SUBSET_DRAM_BYTES_PER_TOKEN = (415.249664e6 + 367.584256e6) / 2048
 PROFILED_SUBSET_WORKLOAD = "large_subset_bf16"
 
 
