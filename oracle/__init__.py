@@ -22,6 +22,10 @@ Sources (the Dust pages, cited by title and section):
   (iitog), "Механика такая": noise on each linear layer's output, independent
   per token; reward-weighted noise average is the output-error estimate, its
   outer product with the layer input the weight gradient.
+* The attention-internals variant (``attn.py``) follows §1 of the first page
+  (the attention internals' reward comes from the change of the attention
+  output; only the attention output is recomputed per draw) and the second
+  page's remark that this change is judged together with an error signal.
 
 Parity pins: every function here is checked by ``tests/test_oracle_*.py``
 against closed forms, invariants, brute-force finite differences, library
@@ -39,6 +43,9 @@ from .philox import (  # noqa: F401
     TAG_MLP_UP,
     TAG_MLP_DOWN,
     TAG_ATTN_OUT,
+    TAG_ATTN_Q,
+    TAG_ATTN_K,
+    TAG_ATTN_V,
 )
 from .params import Params  # noqa: F401
 from .head import (  # noqa: F401
@@ -49,3 +56,4 @@ from .mlp import (  # noqa: F401
     attn_out_draws,
 )
 from .optim import sgd_momentum, train_head, exact_weight_grad  # noqa: F401
+from .attn import attention, attention_seq, attn_draws, attn_grad, perturbed_outputs  # noqa: F401

@@ -41,6 +41,9 @@ TAG_SUBSET_OFFSET = 1  # the per-draw subset offset b
 TAG_MLP_UP = 2         # noise on the MLP up-projection output
 TAG_MLP_DOWN = 3       # noise on the MLP down-projection output
 TAG_ATTN_OUT = 4       # noise on the attention output projection's output
+TAG_ATTN_Q = 5         # noise on the query projection's output
+TAG_ATTN_K = 6         # noise on the key projection's output
+TAG_ATTN_V = 7         # noise on the value projection's output
 
 
 def _u32(x) -> np.ndarray:

@@ -10,6 +10,7 @@ from .workloads import (  # noqa: F401
     Workload,
     bf16_round,
     make_head_inputs,
+    make_attn_inputs,
     make_mlp_inputs,
     zipf_targets,
 )

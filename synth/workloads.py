@@ -2,12 +2,18 @@
 
 Recipe (all host-side, numpy PCG64; the workload seed's SeedSequence spawns
 one child stream per tensor, in the order H, W, targets for the LM-head
-workloads and x, W_up, W_down, W_head, targets, O for the MLP-block workloads):
+workloads, x, W_up, W_down, W_head, targets, O for the MLP-block workloads and
+x, Q, K, V, E for the attention-internals workloads):
 
 * H ~ N(0, 1), then each row divided by its RMS sqrt(mean(h^2)).
 * W ~ N(0, 1/d), so logits z = W h are roughly N(0, 1) per entry.
 * MLP: x ~ N(0, 1); W_up ~ N(0, 1/d); W_down ~ N(0, 1/d_ff); W_head ~ N(0, 1/d);
   the attention output O ~ N(0, 1) for the output-projection variant.
+* Attention internals: the projection input x ~ N(0, 1) (rounded like the
+  other float inputs); the cached projections Q, K, V ~ N(0, 1) in fp32, so
+  the scores q.k / sqrt(d_h) are about N(0, 1); the error signal at the
+  attention output E ~ N(0, 1) in fp32. Sequences of L tokens, H heads of
+  width d_h, as in a GPT-2-small block.
 * targets: uniform on [0, V) for the tiny fp32 workload, otherwise a
   Zipf(1.1) law truncated to ranks 1..V (rank k -> token id k-1), sampled by
   inverse CDF.
@@ -28,7 +34,8 @@ import numpy as np
 @dataclass(frozen=True)
 class Workload:
     name: str
-    variant: str        # "head", "mlp" (up-projection), "mlp_down" or "attn_out"
+    variant: str        # "head", "mlp" (up-projection), "mlp_down", "attn_out",
+                        # or "attn_q" / "attn_k" / "attn_v" (attention internals)
     T: int
     d: int
     V: int
@@ -39,6 +46,9 @@ class Workload:
     dtype: str          # "f32" or "bf16"
     targets: str        # "uniform" or "zipf"
     d_ff: int = 0
+    seq_len: int = 0    # attention internals: tokens per sequence
+    n_heads: int = 0
+    head_dim: int = 0
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -67,6 +77,17 @@ CONFIGS = {
     # Attention output projection writing into the MLP block's input, same shapes.
     "attn_out_bf16": Workload("attn_out_bf16", "attn_out", T=8192, d=768, V=50304, K=256, S=0,
                               sigma=1e-2, seed=3, dtype="bf16", targets="zipf", d_ff=3072),
+    # Attention internals: noise on the query, key or value projection's
+    # output of a 12-head, 768-wide causal attention over 8 sequences of 1024.
+    "attn_q_bf16": Workload("attn_q_bf16", "attn_q", T=8192, d=768, V=1, K=256, S=0,
+                            sigma=1e-2, seed=5, dtype="bf16", targets="none", seq_len=1024,
+                            n_heads=12, head_dim=64),
+    "attn_k_bf16": Workload("attn_k_bf16", "attn_k", T=8192, d=768, V=1, K=256, S=0,
+                            sigma=1e-2, seed=5, dtype="bf16", targets="none", seq_len=1024,
+                            n_heads=12, head_dim=64),
+    "attn_v_bf16": Workload("attn_v_bf16", "attn_v", T=8192, d=768, V=1, K=256, S=0,
+                            sigma=1e-2, seed=5, dtype="bf16", targets="none", seq_len=1024,
+                            n_heads=12, head_dim=64),
     # LM head at 243M-model head scale, subset draws (S = 512), 16k draws.
     "large_subset_bf16": Workload("large_subset_bf16", "head", T=16384, d=1024, V=50304,
                                   K=16384, S=512, sigma=5e-3, seed=4, dtype="bf16",
@@ -136,3 +157,15 @@ def make_mlp_inputs(wl: Workload) -> dict:
     return {"X": _cast(X, wl.dtype), "W_up": _cast(W_up, wl.dtype),
             "W_down": _cast(W_down, wl.dtype), "W_head": _cast(W_head, wl.dtype),
             "targets": y, "O": _cast(O, wl.dtype)}
+
+
+def make_attn_inputs(wl: Workload) -> dict:
+    """x (T x d), the cached projections Q, K, V (T x D, fp32) and the error
+    signal E at the attention output (T x D, fp32), D = n_heads head_dim."""
+    rX, rQ, rK, rV, rE = _streams(wl.seed, 5)
+    D = wl.n_heads * wl.head_dim
+    X = rX.standard_normal((wl.T, wl.d))
+    out = {"X": _cast(X, wl.dtype)}
+    for name, r in (("Q", rQ), ("K", rK), ("V", rV), ("E", rE)):
+        out[name] = r.standard_normal((wl.T, D)).astype(np.float32)
+    return out
