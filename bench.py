@@ -42,6 +42,12 @@ LANES_PER_SM = 128           # 4 schedulers x 32 lanes issue per clock
 # Philox4x32-10 10, Gaussian transform 4, expm1 2, reward multiply-add and
 # its operand load 2, g accumulation multiply and add 2.
 ALU_OPS_PER_ELEM = 20
+# attention internals, algorithmic lane operations: per (draw, head, row
+# visited) a d_h-long dot product, an expm1 (8) and two multiply-adds; per
+# noise entry the generator's 14 (Philox 10, Gaussian 4)
+ATTN_OPS_PER_ROW_EXTRA = 10
+ATTN_OPS_PER_NOISE = 14
+ATTN_SAMPLE_DRAWS = 4
 # DRAM bytes (read + write) per token of the subset-draw kernel on the
 # large-subset workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of
 # one launch over its first 2048 tokens (415.25 + 367.58 MB), per token; the
@@ -112,7 +118,7 @@ class ClockSampler:
 def _oracle_tokens(args):
     """Worker: the oracle on a few tokens of a workload (spawned process).
 
-    Returns (tokens done, seconds spent in the oracle); input generation is
+    Returns (token-draws done, seconds spent in the oracle); input generation is
     not timed."""
     import oracle
     import synth
@@ -125,6 +131,23 @@ def _oracle_tokens(args):
             prm = oracle.Params(T=1, d=wl.d, V=wl.V, K=wl.K, S=wl.S, sigma=wl.sigma,
                                 seed=wl.seed, token_offset=t)
             oracle.head_grad(inp["H"][t:t + 1], inp["W"], inp["targets"][t:t + 1], prm)
+    elif wl.variant.startswith("attn_") and wl.variant != "attn_out":
+        # the oracle recomputes the whole perturbed sequence per draw: the
+        # sample is the first ATTN_SAMPLE_DRAWS draws of each token
+        inp = synth.make_attn_inputs(wl)
+        which = wl.variant[-1]
+        L, H, D = wl.seq_len, wl.n_heads, wl.n_heads * wl.head_dim
+        t0 = time.perf_counter()
+        for t in toks:
+            b, pos = divmod(t, L)
+            rows = slice(b * L, (b + 1) * L)
+            Ob, _ = oracle.attention_seq(inp["Q"][rows], inp["K"][rows], inp["V"][rows], H)
+            for i in range(ATTN_SAMPLE_DRAWS):
+                eps = oracle.gaussians(wl.seed, t, np.arange(i, i + 1), np.arange(D),
+                                       oracle.attn.WHICH_TAG[which])
+                oracle.attn_draws(inp["Q"][rows], inp["K"][rows], inp["V"][rows], Ob,
+                                  inp["E"][rows], H, pos, which, eps, float(np.float32(wl.sigma)))
+        return len(toks) * ATTN_SAMPLE_DRAWS, time.perf_counter() - t0
     else:
         inp = synth.make_mlp_inputs(wl)
         t0 = time.perf_counter()
@@ -138,7 +161,7 @@ def _oracle_tokens(args):
                 fn = oracle.mlp_down_grad if wl.variant == "mlp_down" else oracle.mlp_grad
                 fn(inp["X"][t:t + 1], inp["W_up"], inp["W_down"], inp["W_head"],
                    inp["targets"][t:t + 1], prm)
-    return len(toks), time.perf_counter() - t0
+    return len(toks) * wl.K, time.perf_counter() - t0
 
 
 def cpu_baseline(name: str, budget_tokens: int = 0) -> dict:
@@ -150,7 +173,9 @@ def cpu_baseline(name: str, budget_tokens: int = 0) -> dict:
     import multiprocessing as mp
     import synth
     wl = synth.CONFIGS[name]
-    cores = max(1, min(os.cpu_count() or 1, 16))
+    attn = wl.variant.startswith("attn_") and wl.variant != "attn_out"
+    # attention oracle workers hold a few (heads x L x L) fp64 arrays each
+    cores = max(1, min(os.cpu_count() or 1, 8 if attn else 16))
     ntok = min(budget_tokens or cores, wl.T)
     toks = [int(t) for t in np.linspace(0, wl.T - 1, ntok).round()] if ntok > 1 else [0]
     chunks = [(name, toks[i::cores]) for i in range(cores) if toks[i::cores]]
@@ -167,11 +192,13 @@ def cpu_baseline(name: str, budget_tokens: int = 0) -> dict:
                 os.environ.pop(k, None)
             else:
                 os.environ[k] = v
-    done = sum(r[0] for r in res)
+    done = sum(r[0] for r in res)       # token-draws
     dt = max(r[1] for r in res)
-    value = done * wl.K / dt
+    value = done / dt
+    what = (f"{len(toks)} tokens x the first {ATTN_SAMPLE_DRAWS} draws" if attn
+            else f"{len(toks)} tokens x all {wl.K} draws")
     return {"value": value, "unit": UNIT, "cores": len(chunks), "kind": "oracle",
-            "sample": f"{done} tokens x all {wl.K} draws of {name}, fp64 NumPy oracle, "
+            "sample": f"{what} of {name}, fp64 NumPy oracle, "
                       f"{len(chunks)} spawned single-threaded workers, slowest {dt:.1f} s"}
 
 
@@ -221,12 +248,31 @@ def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
             "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)"}
 
 
+def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
+    """ALU-issue roofline of the attention draw kernel."""
+    L, H, dh = wl.seq_len, wl.n_heads, wl.head_dim
+    rows = (wl.T // L) * L * (L + 1) // 2 if wl.variant in ("attn_q", "attn_k") else 0
+    ops = wl.K * H * (rows * (dh + ATTN_OPS_PER_ROW_EXTRA) + wl.T * dh * ATTN_OPS_PER_NOISE)
+    achieved = ops / (draws_ms * 1e-3) / 1e12
+    f = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    peak = SM_COUNT * LANES_PER_SM * f / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s",
+            "frac": achieved / peak, "traffic": None, "kernel": "attn_draws", "ops": ops,
+            "kernel_ms": draws_ms,
+            "ops_basis": (f"K H (rows visited x (d_h + {ATTN_OPS_PER_ROW_EXTRA}) + T d_h x "
+                          f"{ATTN_OPS_PER_NOISE})"),
+            "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)"}
+
+
 def _config(args, wl, world: int, l2: str) -> dict:
     """The workload of a JSON line (the same keys on both arms)."""
-    return {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
-            "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype, "d_ff": wl.d_ff, "l2": l2,
-            "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL all-reduce"
-                            if world > 1 else "dp1")}
+    cfg = {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
+           "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype, "d_ff": wl.d_ff, "l2": l2,
+           "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL all-reduce"
+                           if world > 1 else "dp1")}
+    if wl.seq_len:
+        cfg.update(seq_len=wl.seq_len, n_heads=wl.n_heads, head_dim=wl.head_dim)
+    return cfg
 
 
 # ----------------------------------------------------------------------------- main arms
@@ -286,6 +332,21 @@ def run_dust(args):
             ctx.head_grad(Hd, Wd, yd, K=wl.K, sigma=wl.sigma, S=wl.S, seed=wl.seed,
                           token_offset=t_off, out=outs, asynchronous=True)
             allreduce_weight_grad(outs["G"])   # G_W of all ranks' tokens (no-op at N = 1)
+    elif wl.seq_len:
+        inp = synth.make_attn_inputs(wl)
+        tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        X = torch.from_numpy(inp["X"]).to(tdt).to(dev)
+        Qd, Kd, Vd, Ed = (torch.from_numpy(inp[k]).to(dev) for k in ("Q", "K", "V", "E"))
+        D = wl.n_heads * wl.head_dim
+        outs = {"G": torch.empty(D, wl.d, dtype=torch.float32, device=dev)}
+        which = wl.variant[-1]
+
+        def step():
+            ctx.attn_grad(X, Qd, Kd, Vd, Ed, seq_len=wl.seq_len, n_heads=wl.n_heads,
+                          which=which, K=wl.K, sigma=wl.sigma, seed=wl.seed, token_offset=t_off,
+                          out=outs)
+            from zeroth_order_transformer_dust_b200.parallel import allreduce_weight_grad
+            allreduce_weight_grad(outs["G"])
     else:
         inp = synth.make_mlp_inputs(wl)
         X, Wu, Wdn, Wh = (torch.from_numpy(inp[k]).to(torch.bfloat16).to(dev)
@@ -377,6 +438,9 @@ def run_dust(args):
                 roof["traffic"] = SUBSET_DRAM_BYTES_PER_TOKEN * wl.T
                 roof["traffic_basis"] = ("ncu DRAM bytes of a 2048-token launch, scaled by "
                                          "tokens to this launch")
+    if wl.seq_len and stages.get("draws"):
+        roof = _attn_roofline(wl, stages["draws"], peaks)
+        roof["peak_kind"] = peak_kind
     gemm_flops = 2.0 * wl.T * wl.d * wl.V
     extra = {}
     if wl.variant == "head":

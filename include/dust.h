@@ -65,7 +65,7 @@ enum {
 };
 
 /* Variants accepted by dust_validate. */
-enum { DUST_VARIANT_HEAD = 0, DUST_VARIANT_MLP = 1 };
+enum { DUST_VARIANT_HEAD = 0, DUST_VARIANT_MLP = 1, DUST_VARIANT_ATTN = 2 };
 
 typedef struct dust_params {
   int64_t T;            /* tokens in this call (>= 1) */
@@ -204,6 +204,49 @@ dust_status dust_attn_out_grad(dust_ctx* ctx, const dust_params* p,
                                const void* W_up, const void* W_down, const void* W_head,
                                const int32_t* targets, float* G_o_out, float* loss_out,
                                float* rewards_out, float* g_out);
+
+/*
+ * Attention-internals estimator ("Dust：无需反向传播的Transformer零阶预训练",
+ * §1 无需反向传播的信用分配 and 减少干扰: the attention internals are rewarded
+ * from the change of the attention output, and a draw recomputes only the
+ * attention output; "不用反向传播训练Transformer：Dust零阶优化获突破": that
+ * change is judged together with an error signal).
+ * Noise sigma eps (D = n_heads head_dim entries) goes on one token's output of
+ * the query, key or value projection (shape->which). The attention is causal
+ * multi-head attention over independent sequences of seq_len tokens with
+ * scores q.k / sqrt(head_dim). A draw's reward is the first-order loss
+ * decrease of the attention outputs it moves,
+ *   r = -sum_t <o'_t - o_t, e_t>,
+ * over t = s for query noise on token s and over t >= s of the same sequence
+ * for key or value noise; e is the caller's error signal at the attention
+ * output. Then g_s = -(1/(K sigma)) sum_i r_i eps_i (D entries) and
+ * G = sum_s g_s x_s^T against the projection's input x.
+ *   p        T (a multiple of seq_len), d (the width of x), K, sigma, seed,
+ *            token_offset, draw_offset, stream_id, dtype (of X); V, d_ff,
+ *            subset_a are not used; S must be <= 0
+ *   shape    seq_len in [1, 4096], n_heads >= 1, head_dim 32, 64 or 128
+ *   X        T x d   the projection's input (p->dtype)
+ *   Q, Kc, Vc T x D  fp32 cached projections, head h in columns
+ *                    [h head_dim, (h+1) head_dim)
+ *   E        T x D   fp32 error signal at the attention output
+ *   G_out    D x d   fp32 (or NULL)
+ *   rewards_out T x K fp32 (or NULL);  g_out T x D fp32 (or NULL)
+ * All pointers are device pointers, row-major; inputs 16-byte aligned,
+ * outputs 4-byte. The noise's counter tag is 5, 6 or 7 (query, key, value).
+ * Errors: DUST_ERR_ARG for bad parameters, shape or pointers;
+ * DUST_ERR_UNSUPPORTED when seq_len needs more shared memory than the device
+ * has; DUST_ERR_CUDA / DUST_ERR_OOM as elsewhere.
+ */
+enum { DUST_ATTN_Q = 0, DUST_ATTN_K = 1, DUST_ATTN_V = 2 };
+typedef struct dust_attn_shape {
+  int32_t seq_len;   /* L: tokens per sequence */
+  int32_t n_heads;   /* H */
+  int32_t head_dim;  /* d_h: 32, 64 or 128 */
+  int32_t which;     /* DUST_ATTN_Q, DUST_ATTN_K or DUST_ATTN_V */
+} dust_attn_shape;
+dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* p, const dust_attn_shape* shape,
+                           const void* X, const float* Q, const float* Kc, const float* Vc,
+                           const float* E, float* G_out, float* rewards_out, float* g_out);
 
 /* Per-stage device timing: when enabled, each call records CUDA events on
    the context's stream between its stages (clean GEMM, log-sum-exp, draws,

@@ -79,6 +79,15 @@ def test_mlp_validation(lib):
     assert dust.validate(ok, 7)[0] == 1
 
 
+def test_attention_validation(lib):
+    # the attention-internals variant ignores V and d_ff, perturbs every channel
+    assert dust.validate(_p(V=0, d_ff=0), dust.VARIANT_ATTN)[0] == 0
+    assert dust.validate(_p(dtype=dust.DUST_F32), dust.VARIANT_ATTN)[0] == 0
+    assert dust.validate(_p(S=4), dust.VARIANT_ATTN)[0] == 1
+    assert dust.validate(_p(K=0), dust.VARIANT_ATTN)[0] == 1
+    assert dust.validate(_p(T=0), dust.VARIANT_ATTN)[0] == 1
+
+
 def test_null_params_and_context(lib):
     assert lib.dust_validate(None, 0, None, 0) == 1
     p = _p()

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "DUST_OK", 1: "DUST_ERR_ARG", 2: "DUST_ERR_CUDA", 3: "DUST_ER
 DUST_F32, DUST_BF16 = 0, 1
 FLAG_LITERAL_TARGET_SCALE = 1 << 0
 FLAG_ASYNC = 1 << 1
-VARIANT_HEAD, VARIANT_MLP = 0, 1
+VARIANT_HEAD, VARIANT_MLP, VARIANT_ATTN = 0, 1, 2
 TAG_HEAD, TAG_SUBSET_OFFSET, TAG_MLP_UP = 0, 1, 2
 
 # Every extern "C" symbol include/dust.h declares.
@@ -34,6 +34,7 @@ EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
            "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
            "dust_kernel_launches", "dust_debug_gemm_bf16", "dust_debug_gauss_tab",
            "dust_head_grad_noalloc", "dust_debug_bm_radius", "dust_debug_bm_angle",
+           "dust_attn_grad",
            "dust_sgd_momentum", "dust_mlp_down_grad", "dust_attn_out_grad")
 
 
@@ -44,6 +45,15 @@ class DustParams(ctypes.Structure):
                 ("token_offset", ctypes.c_int64), ("draw_offset", ctypes.c_int64),
                 ("subset_a", ctypes.c_int64), ("stream_id", ctypes.c_uint32),
                 ("flags", ctypes.c_uint32)]
+
+
+class DustAttnShape(ctypes.Structure):
+    """dust_attn_shape: the geometry of the attention-internals variant."""
+    _fields_ = [("seq_len", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("which", ctypes.c_int32)]
+
+
+ATTN_WHICH = {"q": 0, "k": 1, "v": 2}
 
 
 class DustError(RuntimeError):
@@ -83,6 +93,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "dust_mlp_grad": (I32, [P, PP, P, P, P, P, P, P, P, P, P]),
             "dust_mlp_down_grad": (I32, [P, PP, P, P, P, P, P, P, P, P, P]),
             "dust_attn_out_grad": (I32, [P, PP, P, P, I64, P, P, P, P, P, P, P, P]),
+            "dust_attn_grad": (I32, [P, PP, ctypes.POINTER(DustAttnShape), P, P, P, P, P, P, P,
+                                     P]),
             "dust_debug_philox": (I32, [P, U64, P, I64, P]),
             "dust_debug_gauss": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_set_stage_timing": (I32, [P, ctypes.c_int]),
@@ -292,6 +304,44 @@ class Context:
         self._check(st)
         return out
 
+    def attn_grad(self, X, Q, K_cache, V_cache, E, *, seq_len, n_heads, which, K, sigma, seed=0,
+                  token_offset=0, draw_offset=0, stream_id=0, want_G=True, want_rewards=False,
+                  want_g=False, out=None) -> dict:
+        """Attention-internals estimator: noise on the output of the query
+        (which="q"), key ("k") or value ("v") projection. X (T x d, fp32 or
+        bf16) is the projection's input; Q, K_cache, V_cache (T x D fp32) the
+        cached projections; E (T x D fp32) the error signal at the attention
+        output; D = n_heads head_dim. G is D x d, g is T x D, rewards T x K."""
+        if which not in ATTN_WHICH:
+            raise ValueError("which must be 'q', 'k' or 'v'")
+        for t, n in ((X, "X"), (Q, "Q"), (K_cache, "K_cache"), (V_cache, "V_cache"), (E, "E")):
+            self._dev(t, n)
+        for t, n in ((Q, "Q"), (K_cache, "K_cache"), (V_cache, "V_cache"), (E, "E")):
+            if t.dtype != torch.float32 or t.shape != Q.shape:
+                raise TypeError(f"{n} must be fp32 with Q's shape")
+        T, d = X.shape
+        D = Q.shape[1]
+        if D % n_heads:
+            raise ValueError("the width of Q must be a multiple of n_heads")
+        shape = DustAttnShape(seq_len=seq_len, n_heads=n_heads, head_dim=D // n_heads,
+                              which=ATTN_WHICH[which])
+        prm = make_params(T, d, 1, K, sigma, dtype=_dtype_code(X), seed=seed,
+                          token_offset=token_offset, draw_offset=draw_offset, stream_id=stream_id)
+        out = dict(out or {})
+        f32 = dict(dtype=torch.float32, device=X.device)
+        if want_G and "G" not in out:
+            out["G"] = torch.empty(D, d, **f32)
+        if want_rewards and "rewards" not in out:
+            out["rewards"] = torch.empty(T, K, **f32)
+        if want_g and "g" not in out:
+            out["g"] = torch.empty(T, D, **f32)
+        self._bind_stream()
+        self._check(self._L.dust_attn_grad(self._h, ctypes.byref(prm), ctypes.byref(shape),
+                                           _ptr(X), _ptr(Q), _ptr(K_cache), _ptr(V_cache),
+                                           _ptr(E), _ptr(out.get("G")), _ptr(out.get("rewards")),
+                                           _ptr(out.get("g"))))
+        return out
+
     # -- instrumentation -------------------------------------------------------------
     def set_stage_timing(self, enable: bool = True):
         self._check(self._L.dust_set_stage_timing(self._h, 1 if enable else 0))
@@ -395,3 +445,7 @@ def head_grad(H, W, targets, **kw) -> dict:
 
 def mlp_grad(X, W_up, W_down, W_head, targets, **kw) -> dict:
     return context(X.device.index).mlp_grad(X, W_up, W_down, W_head, targets, **kw)
+
+
+def attn_grad(X, Q, K_cache, V_cache, E, **kw) -> dict:
+    return context(X.device.index).attn_grad(X, Q, K_cache, V_cache, E, **kw)

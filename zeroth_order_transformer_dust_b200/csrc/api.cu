@@ -77,11 +77,13 @@ dust_status check_params(const dust_params* p, int variant, char* msg, int msg_l
     return DUST_ERR_ARG;
   };
   if (!p) return bad("params is NULL");
-  if (variant != DUST_VARIANT_HEAD && variant != DUST_VARIANT_MLP) return bad("unknown variant");
+  if (variant != DUST_VARIANT_HEAD && variant != DUST_VARIANT_MLP && variant != DUST_VARIANT_ATTN)
+    return bad("unknown variant");
+  const bool attn = variant == DUST_VARIANT_ATTN;
   if (p->T < 1) return bad("T must be >= 1");
   if (p->d < 1) return bad("d must be >= 1");
-  if (p->V < 1) return bad("V must be >= 1");
-  if (p->V > 0x7fffffffLL) return bad("V must fit int32 targets");
+  if (!attn && p->V < 1) return bad("V must be >= 1");
+  if (!attn && p->V > 0x7fffffffLL) return bad("V must fit int32 targets");
   if (p->K < 1) return bad("K must be >= 1");
   if (!std::isfinite(p->sigma) || p->sigma < 0.0f) return bad("sigma must be finite and >= 0");
   if (p->dtype != DUST_F32 && p->dtype != DUST_BF16) return bad("dtype must be DUST_F32 or DUST_BF16");
@@ -90,7 +92,7 @@ dust_status check_params(const dust_params* p, int variant, char* msg, int msg_l
   if (p->draw_offset < 0 || p->draw_offset + (int64_t)p->K > (1LL << 32))
     return bad("draw_offset + K must lie in [0, 2^32]");
   if (p->stream_id >= (1u << 24)) return bad("stream_id must be < 2^24");
-  if (p->T > (1LL << 40) / p->V) return bad("T * V too large");
+  if (!attn && p->T > (1LL << 40) / p->V) return bad("T * V too large");
   if (p->T > (1LL << 40) / p->K) return bad("T * K too large");
   if (variant == DUST_VARIANT_HEAD) {
     if (p->S > p->V) return bad("S must be <= V");
@@ -98,6 +100,8 @@ dust_status check_params(const dust_params* p, int variant, char* msg, int msg_l
       if (p->subset_a < 1) return bad("subset_a must be >= 1");
       if (gcd64(p->subset_a, p->V) != 1) return bad("subset_a must be coprime to V");
     }
+  } else if (attn) {
+    if (p->S > 0) return bad("the attention variant perturbs every channel: S must be <= 0");
   } else {
     if (p->d_ff < 1) return bad("d_ff must be >= 1");
     if (p->S > 0) return bad("the MLP variant perturbs all d_ff channels: S must be <= 0");
@@ -280,7 +284,9 @@ void dust_destroy(dust_ctx* ctx) {
   Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
                  &ctx->gT, &ctx->hT, &ctx->xdup, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
-                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32};
+                 &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32,
+                 &ctx->mlp_dn, &ctx->mlp_du, &ctx->wu2, &ctx->attn_o, &ctx->attn_lse,
+                 &ctx->attn_gb};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -696,6 +702,78 @@ dust_status dust_attn_out_grad(dust_ctx* ctx, const dust_params* p, const void* 
                                float* loss_out, float* rewards_out, float* g_out) {
   return mlp_impl(ctx, p, kLayerAttnOut, X, O, d_o, W_up, W_down, W_head, targets, G_o_out,
                   loss_out, rewards_out, g_out);
+}
+
+// Attention internals: noise on the query, key or value projection's output;
+// the reward is the first-order loss change -sum_t <o'_t - o_t, e_t> of the
+// attention outputs the perturbation moves (k_attn.cu has the closed forms).
+dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn_shape* as,
+                           const void* X, const float* Q, const float* Kc, const float* Vc,
+                           const float* E, float* G_out, float* rewards_out, float* g_out) {
+  if (!ctx) return DUST_ERR_ARG;
+  char why[256];
+  if (check_params(pp, DUST_VARIANT_ATTN, why, sizeof(why)) != DUST_OK)
+    return fail(ctx, DUST_ERR_ARG, "%s", why);
+  if (!as) return fail(ctx, DUST_ERR_ARG, "shape is NULL");
+  const dust_params p = *pp;
+  const dust_attn_shape a = *as;
+  if (a.which < DUST_ATTN_Q || a.which > DUST_ATTN_V)
+    return fail(ctx, DUST_ERR_ARG, "which must be DUST_ATTN_Q, DUST_ATTN_K or DUST_ATTN_V");
+  if (a.head_dim != 32 && a.head_dim != 64 && a.head_dim != 128)
+    return fail(ctx, DUST_ERR_ARG, "head_dim must be 32, 64 or 128");
+  if (a.n_heads < 1 || a.seq_len < 1 || a.seq_len > 4096)
+    return fail(ctx, DUST_ERR_ARG, "n_heads must be >= 1 and seq_len in [1, 4096]");
+  if (p.T % a.seq_len) return fail(ctx, DUST_ERR_ARG, "T must be a multiple of seq_len");
+  if (p.T * a.n_heads >= (1LL << 31)) return fail(ctx, DUST_ERR_ARG, "T * n_heads too large");
+  const int64_t T = p.T, H = a.n_heads, Dw = H * (int64_t)a.head_dim, K = p.K;
+  if (T > (1LL << 40) / (Dw * K)) return fail(ctx, DUST_ERR_ARG, "T * D * K too large");
+  if (!X || !Q || !Kc || !Vc || !E)
+    return fail(ctx, DUST_ERR_ARG, "X, Q, K, V and E must be non-NULL");
+  if (!aligned(X, 16) || !aligned(Q, 16) || !aligned(Kc, 16) || !aligned(Vc, 16) ||
+      !aligned(E, 16) || !aligned(G_out, 4) || !aligned(rewards_out, 4) || !aligned(g_out, 4))
+    return fail(ctx, DUST_ERR_ARG, "X, Q, K, V, E must be 16-byte aligned, the outputs 4-byte");
+  if ((size_t)ctx->max_smem_optin < attn_fwd_smem(a.seq_len, a.head_dim) ||
+      (size_t)ctx->max_smem_optin < attn_draws_smem(a.seq_len, a.head_dim) + 9216)
+    return fail(ctx, DUST_ERR_UNSUPPORTED, "seq_len too long for shared memory");
+  DUST_CU(cudaSetDevice(ctx->device));
+  const cudaStream_t st = ctx->stream;
+  DUST_TRY(ensure(ctx, ctx->attn_o, (size_t)T * Dw * 4));
+  DUST_TRY(ensure(ctx, ctx->attn_lse, (size_t)T * H * 4));
+  DUST_TRY(ensure(ctx, ctx->attn_gb, (size_t)T * H * 4));
+  DUST_TRY(ensure(ctx, ctx->part, (size_t)T * H * K * 4));
+  DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(p.dtype, T, Dw)));
+  float* r = rewards_out;
+  if (!r) {
+    DUST_TRY(ensure(ctx, ctx->rew, (size_t)T * K * 4));
+    r = (float*)ctx->rew.p;
+  }
+  DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), st));
+  mark(ctx, nullptr);
+  float* O = (float*)ctx->attn_o.p;
+  float* lse = (float*)ctx->attn_lse.p;
+  float* gb = (float*)ctx->attn_gb.p;
+  DUST_CU(launch_attn_fwd(st, T, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse, gb));
+  ctx->launches += 1;
+  mark(ctx, "attn_fwd");
+  DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
+                            gb, (float*)ctx->part.p));
+  DUST_CU(launch_attn_combine(st, (const float*)ctx->part.p, T, (int)H, (int)K, r));
+  ctx->launches += 2;
+  mark(ctx, "draws");
+  dust_params pg = p;
+  pg.d = Dw;  // the noise width
+  const int tag = kTagAttnQ + a.which;
+  if (p.dtype == DUST_BF16)
+    DUST_CU(launch_noise_g_planes(st, pg, r, g_out, (__nv_bfloat16*)ctx->gop.p, tag));
+  else
+    DUST_CU(launch_noise_g_f32(st, pg, r, g_out, (float*)ctx->gop.p, tag));
+  ctx->launches += 1;
+  mark(ctx, "g");
+  if (G_out) {
+    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, Dw, X, p.d, G_out, 0));
+    mark(ctx, "gw_gemm");
+  }
+  return finish(ctx, p.flags);
 }
 
 dust_status dust_set_stage_timing(dust_ctx* ctx, int enable) {

@@ -148,7 +148,8 @@ struct dust_ctx {
   bool subset2_enabled = true;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
-      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2;
+      mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
+      attn_o, attn_lse, attn_gb;
 };
 
 namespace dust {
@@ -248,6 +249,9 @@ cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, 
 // g over width d with counter tag `tag`, gop as bf16 hi/lo planes (T x d each).
 cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const float* r,
                                   float* g_out, __nv_bfloat16* gop, int tag);
+// The same with gop fp32 (T x d).
+cudaError_t launch_noise_g_f32(cudaStream_t st, const dust_params& p, const float* r,
+                              float* g_out, float* gop, int tag);
 // Noise on a width-d output: sigma eps as bf16 hi/lo planes (rows nt K x 2d),
 // counter tag `tag` (down projection: 3; attention output projection: 4).
 cudaError_t launch_mlp_noise_split(cudaStream_t st, const dust_params& p, int64_t t0, int64_t nt,
@@ -258,5 +262,20 @@ cudaError_t launch_gelu_delta_rows(cudaStream_t st, const dust_params& p, const 
                                    const float* du, int64_t t0, int64_t nt, __nv_bfloat16* da);
 // a = GELU(u) (fp64, rounded to fp32), n elements.
 cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a, int sm_count);
+// Attention internals (k_attn.cu): the clean causal attention per (token,
+// head) -> O, LSE, gbar = <o, e>; the per-head rewards of noise on the
+// query (which 0), key (1) or value (2) of every token -> part ((T H) x K);
+// their sum over heads -> r (T x K).
+size_t attn_fwd_smem(int L, int head_dim);
+size_t attn_draws_smem(int L, int head_dim);
+cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
+                            const float* Q, const float* Kc, const float* Vc, const float* E,
+                            float* O, float* lse, float* gbar);
+cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
+                              int head_dim, const float* Q, const float* Kc, const float* Vc,
+                              const float* E, const float* O, const float* lse,
+                              const float* gbar, float* part);
+cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, int H, int K,
+                                float* r);
 
 }  // namespace dust

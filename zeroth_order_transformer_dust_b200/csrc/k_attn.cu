@@ -1,0 +1,401 @@
+// Attention-internals draws ("Dust：无需反向传播的Transformer零阶预训练", §1
+// 无需反向传播的信用分配: the attention internals' reward comes from the change
+// of the attention output rather than the per-token loss; 减少干扰: only the
+// attention output is recomputed per draw, the rest stays cached).
+//
+// Noise sigma eps on the query, key or value of token s (D = H d_h entries,
+// heads side by side) and the reward r = -sum_t <o'_t - o_t, e_t> over the
+// tokens whose attention output moves, e the error signal at the attention
+// output. Heads do not mix, so r is a sum of per-head rewards r_h, and each
+// has a closed form in the clean attention (c = 1/sqrt(d_h), a the clean
+// probabilities, gbar_t = <o_t, e_t> per head):
+//   query s: row s's scores move by d_tau = c (sigma eps) . k_tau, tau <= s:
+//       r_h = -sum_tau a_s,tau expm1(d_tau) (<v_tau, e_s> - gbar_s)
+//             / (1 + sum_tau a_s,tau expm1(d_tau));
+//   key s:   column s of every row t >= s moves by d_t = c (sigma eps) . q_t;
+//       with u_t = a_t,s expm1(d_t) the row's output moves by
+//       u_t / (1 + u_t) (v_s - o_t), so
+//       r_h = -sum_t u_t / (1 + u_t) (<v_s, e_t> - gbar_t);
+//   value s: o_t moves by a_t,s sigma eps, so r_h = -(sigma eps) . w_s with
+//       w_s = sum_{t >= s} a_t,s e_t.
+// These are exact rewrites of the softmax (nothing is linearised).
+//
+// B200 mapping: the clean pass is one warp per (token, head). The draws run
+// one CTA per (token s, head h) and one thread per draw: the thread draws the
+// head's d_h noise entries into registers once, then streams the keys (query
+// noise) or the later queries (key noise) of the sequence through
+// shared-memory tiles, one d_h-long dot product, one expm1 and two FMAs per
+// (draw, row). The per-row coefficients (a, <v, e> - gbar) are formed once per
+// CTA, not per draw. Per-head rewards go to a (token, head, draw) buffer that
+// a second kernel sums over heads in a fixed order.
+#include <cmath>
+
+#include "internal.cuh"
+#include "noise.cuh"
+
+namespace dust {
+namespace {
+
+constexpr int kFwdWarps = 8;
+constexpr int kDrawThreads = 256;
+constexpr int kTile = 64;  // rows per staged tile
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// a . b over DH entries (16-byte aligned rows); four partial sums, eight
+// float4 pairs in flight at most (the rows come from L2 in the callers).
+template <int DH>
+__device__ __forceinline__ float dot_row(const float* __restrict__ a, const float* __restrict__ b) {
+  float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < DH / 4; ++c) {
+    const float4 x = reinterpret_cast<const float4*>(a)[c];
+    const float4 y = reinterpret_cast<const float4*>(b)[c];
+    d0 = fmaf(x.x, y.x, d0);
+    d1 = fmaf(x.y, y.y, d1);
+    d2 = fmaf(x.z, y.z, d2);
+    d3 = fmaf(x.w, y.w, d3);
+  }
+  return (d0 + d1) + (d2 + d3);
+}
+
+// expm1 with full relative accuracy: the Taylor series to x^6 for
+// |x| <= 1/16 (truncation below x^7/5040 < 2^-40 relative), the library
+// function beyond.
+__device__ __forceinline__ float expm1_acc(float x) {
+  if (fabsf(x) <= 0.0625f) {
+    float p = fmaf(x, 1.0f / 720.0f, 1.0f / 120.0f);
+    p = fmaf(x, p, 1.0f / 24.0f);
+    p = fmaf(x, p, 1.0f / 6.0f);
+    p = fmaf(x, p, 0.5f);
+    p = fmaf(x, p, 1.0f);
+    return x * p;
+  }
+  return expm1f(x);
+}
+
+struct FwdArgs {
+  const float* Q;
+  const float* Kc;
+  const float* Vc;
+  const float* E;
+  float* O;
+  float* lse;
+  float* gbar;
+  int64_t T;
+  int32_t L, H;
+  float scale;
+};
+
+// One warp per (token t, head h): the causal scores of row t, their
+// log-sum-exp, o_t = sum a v and gbar_t = <o_t, e_t>. Shared memory per warp:
+// the row's probabilities (L, rounded up to 4) and q_t (d_h).
+template <int DH>
+__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_constant__ FwdArgs A) {
+  extern __shared__ __align__(16) float fsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t idx = (int64_t)blockIdx.x * kFwdWarps + warp;
+  if (idx >= A.T * A.H) return;  // warp-uniform; no block barrier follows
+  const int64_t D = (int64_t)A.H * DH;
+  const int64_t t = idx / A.H;
+  const int h = (int)(idx % A.H);
+  const int64_t s0 = t - t % A.L;
+  const int n = (int)(t - s0) + 1;
+  const int Lp = (A.L + 3) & ~3;
+  float* pr = fsm + (size_t)warp * (Lp + DH);
+  float* qs = pr + Lp;
+  for (int c = lane; c < DH; c += 32) qs[c] = A.Q[t * D + h * DH + c];
+  __syncwarp();
+  float m = -INFINITY;
+  for (int j = lane; j < n; j += 32) {
+    const float v = dot_row<DH>(qs, A.Kc + (s0 + j) * D + h * DH) * A.scale;
+    pr[j] = v;
+    m = fmaxf(m, v);
+  }
+  m = warp_max_f(m);
+  float l = 0.f;
+  for (int j = lane; j < n; j += 32) l += expf(pr[j] - m);
+  l = warp_sum_f(l);
+  const float lse = m + logf(l);
+  for (int j = lane; j < n; j += 32) pr[j] = expf(pr[j] - lse);
+  __syncwarp();
+  float o[DH / 32];
+#pragma unroll
+  for (int u = 0; u < DH / 32; ++u) o[u] = 0.f;
+  for (int j = 0; j < n; ++j) {
+    const float a = pr[j];
+    const float* vp = A.Vc + (s0 + j) * D + h * DH + lane;
+#pragma unroll
+    for (int u = 0; u < DH / 32; ++u) o[u] = fmaf(a, vp[32 * u], o[u]);
+  }
+  float gb = 0.f;
+#pragma unroll
+  for (int u = 0; u < DH / 32; ++u) {
+    const int64_t c = t * D + h * DH + lane + 32 * u;
+    A.O[c] = o[u];
+    gb = fmaf(o[u], A.E[c], gb);
+  }
+  gb = warp_sum_f(gb);
+  if (lane == 0) {
+    A.lse[t * A.H + h] = lse;
+    A.gbar[t * A.H + h] = gb;
+  }
+}
+
+struct DrawArgs {
+  const float* Q;
+  const float* Kc;
+  const float* Vc;
+  const float* E;
+  const float* O;
+  const float* lse;
+  const float* gbar;
+  float* part;  // (T H) x K: r_h of (token, head) for every draw
+  RoundKeys keys;
+  uint32_t t_off, i_off, ctr3;
+  float xscale;  // sigma c (query, key) or sigma (value): the noise's factor
+  int64_t T;
+  int32_t L, H, K;
+  float scale;
+};
+
+// Noise of head h for kDrawThreads draws of token s, times the table's
+// factor, into xs[draw * (d_h + 1) + j] (the odd row stride keeps the
+// per-thread row reads free of bank conflicts). Slot h d_h + j of the layer's
+// D slots uses counter (slot_ctr0(slot >> 7, slot & 31), t, i, ctr3), word
+// (slot >> 5) & 3; words (0, 1) and (2, 3) are the two Box-Muller pairs of a
+// counter. For d_h >= 64 the head's 32-slot groups pair up within one counter
+// (one transform gives both); a 32-wide head uses one word of a pair. Work
+// item (draw, lane, group pair) per thread, so no thread holds a row.
+template <int DH>
+__device__ __forceinline__ void head_noise_smem(float* xs, const RoundKeys& keys, uint32_t t_abs,
+                                                uint32_t i_off, int i0, int K, uint32_t ctr3,
+                                                int h, const float2* tab) {
+  constexpr int kPairs = DH >= 64 ? DH / 64 : 1;
+  const int items = kDrawThreads * 32 * kPairs;
+  for (int it = threadIdx.x; it < items; it += kDrawThreads) {
+    const int l = it & 31;
+    const int rest = it >> 5;
+    const int pr = rest % kPairs;
+    const int d = rest / kPairs;  // draw within the round
+    const int i = i0 + d;
+    if (i >= K) continue;
+    const DrawConst dc = draw_const(keys, t_abs, i_off + (uint32_t)i);
+    const uint32_t sb = (uint32_t)h * DH + 64u * pr;
+    const uint32_t blk = sb >> 7, word = (sb >> 5) & 3u;
+    const U4 w = philox_from2(block_const(keys, slot_ctr0(blk, (uint32_t)l), ctr3), dc, keys);
+    const float2 nn = box_muller_tab(word >= 2 ? w.z : w.x, word >= 2 ? w.w : w.y, tab);
+    float* row = xs + d * (DH + 1);
+    if (DH >= 64) {
+      row[64 * pr + l] = nn.x;
+      row[64 * pr + 32 + l] = nn.y;
+    } else {
+      row[l] = (word & 1u) ? nn.y : nn.x;
+    }
+  }
+}
+
+// One CTA per (token s, head h): blockIdx.x = s H + h. WHICH: 0 query,
+// 1 key, 2 value. Dynamic shared memory: two coefficient rows of L floats
+// (rounded up to 4), a kTile x d_h tile and the noise rows of one round of
+// kDrawThreads draws.
+template <int WHICH, int DH>
+__global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(const __grid_constant__ DrawArgs A) {
+  extern __shared__ __align__(16) float dsm[];
+  __shared__ float2 tab[kSinCosTable];
+  __shared__ __align__(16) float own[2][DH];
+  const int tid = threadIdx.x;
+  const int64_t s = blockIdx.x / A.H;
+  const int h = (int)(blockIdx.x % A.H);
+  const int64_t D = (int64_t)A.H * DH;
+  const int64_t s0 = s - s % A.L;
+  // the other index runs over tau in [s0, s] (query) or t in [s, s0 + L)
+  const int64_t r0 = WHICH == 0 ? s0 : s;
+  const int n = WHICH == 0 ? (int)(s - s0) + 1 : (int)(s0 + A.L - s);
+  const int Lp = (A.L + 3) & ~3;
+  float* ca = dsm;
+  float* cb = dsm + Lp;
+  float* tile = dsm + 2 * Lp;
+  float* xs = tile + kTile * DH;
+  fill_sincos_table(tab, A.xscale);
+  for (int c = tid; c < DH; c += kDrawThreads) {
+    const int64_t o = s * D + h * DH + c;
+    own[0][c] = WHICH == 0 ? A.Q[o] : A.Kc[o];
+    own[1][c] = WHICH == 0 ? A.E[o] : A.Vc[o];
+  }
+  __syncthreads();
+  // per-row coefficients, once per CTA
+  const float lse_s = A.lse[s * A.H + h];
+  const float gb_s = A.gbar[s * A.H + h];
+  for (int j = tid; j < n; j += kDrawThreads) {
+    const int64_t row = (r0 + j) * D + h * DH;
+    if (WHICH == 0) {
+      const float a = expf(dot_row<DH>(own[0], A.Kc + row) * A.scale - lse_s);
+      ca[j] = a;
+      cb[j] = a * (dot_row<DH>(own[1], A.Vc + row) - gb_s);
+    } else {
+      const int64_t t = r0 + j;
+      ca[j] = expf(dot_row<DH>(own[0], A.Q + row) * A.scale - A.lse[t * A.H + h]);
+      if (WHICH == 1) cb[j] = dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h];
+    }
+  }
+  __syncthreads();
+  if (WHICH == 2) {
+    // w_s = sum_{t >= s} a_t,s e_t for this head
+    for (int c = tid; c < DH; c += kDrawThreads) {
+      float w = 0.f;
+      for (int j = 0; j < n; ++j) w = fmaf(ca[j], A.E[(r0 + j) * D + h * DH + c], w);
+      tile[c] = w;
+    }
+  }
+  const uint32_t t_abs = A.t_off + (uint32_t)s;
+  const float* src = WHICH == 0 ? A.Kc : A.Q;  // rows streamed through the tile
+  for (int i0 = 0; i0 < A.K; i0 += kDrawThreads) {
+    const int i = i0 + tid;
+    const bool live = i < A.K;
+    __syncthreads();  // the previous round's rows are consumed
+    head_noise_smem<DH>(xs, A.keys, t_abs, A.i_off, i0, A.K, A.ctr3, h, tab);
+    __syncthreads();
+    float x[DH];
+#pragma unroll
+    for (int c = 0; c < DH; ++c) x[c] = xs[tid * (DH + 1) + c];
+    float r;
+    if (WHICH == 2) {
+      float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < DH; c += 2) {
+        d0 = fmaf(x[c], tile[c], d0);
+        d1 = fmaf(x[c + 1], tile[c + 1], d1);
+      }
+      r = -(d0 + d1);
+    } else {
+      float acc0 = 0.f, acc1 = 0.f;
+      for (int j0 = 0; j0 < n; j0 += kTile) {
+        const int m = min(kTile, n - j0);
+        __syncthreads();
+        for (int e = tid; e < m * (DH / 4); e += kDrawThreads) {
+          const int row = e / (DH / 4), c4 = e % (DH / 4);
+          reinterpret_cast<float4*>(tile)[e] =
+              reinterpret_cast<const float4*>(src + (r0 + j0 + row) * D + h * DH)[c4];
+        }
+        __syncthreads();
+        if (live) {
+#pragma unroll 1
+          for (int jj = 0; jj < m; ++jj) {
+            const float* tr = tile + jj * DH;
+            float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll
+            for (int c = 0; c < DH; c += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(tr + c);
+              d0 = fmaf(x[c], v.x, d0);
+              d1 = fmaf(x[c + 1], v.y, d1);
+              d2 = fmaf(x[c + 2], v.z, d2);
+              d3 = fmaf(x[c + 3], v.w, d3);
+            }
+            const float em = expm1_acc((d0 + d1) + (d2 + d3));
+            if (WHICH == 0) {
+              acc0 = fmaf(ca[j0 + jj], em, acc0);
+              acc1 = fmaf(cb[j0 + jj], em, acc1);
+            } else {
+              const float u = ca[j0 + jj] * em;
+              acc1 = fmaf(__fdividef(u, 1.0f + u), cb[j0 + jj], acc1);
+            }
+          }
+        }
+      }
+      r = WHICH == 0 ? -acc1 / (1.0f + acc0) : -acc1;
+    }
+    if (live) A.part[(int64_t)blockIdx.x * A.K + i] = r;
+  }
+}
+
+// r[s K + i] = sum_h part[(s H + h) K + i], heads in order.
+__global__ void k_attn_combine(const float* __restrict__ part, int64_t T, int32_t H, int32_t K,
+                               float* __restrict__ r) {
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= T * K) return;
+  const int64_t s = gid / K;
+  const int32_t i = (int32_t)(gid % K);
+  float acc = 0.f;
+  for (int h = 0; h < H; ++h) acc += part[(s * H + h) * K + i];
+  r[gid] = acc;
+}
+
+template <int DH>
+cudaError_t fwd_dh(cudaStream_t st, const FwdArgs& A) {
+  const size_t smem = (size_t)kFwdWarps * (((A.L + 3) & ~3) + DH) * 4;
+  cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = A.T * A.H;
+  k_attn_fwd<DH><<<(unsigned)((rows + kFwdWarps - 1) / kFwdWarps), kFwdWarps * 32, smem, st>>>(A);
+  return cudaGetLastError();
+}
+
+template <int WHICH, int DH>
+cudaError_t draws_dh(cudaStream_t st, const DrawArgs& A) {
+  const size_t smem = (size_t)(2 * ((A.L + 3) & ~3) + kTile * DH + kDrawThreads * (DH + 1)) * 4;
+  cudaError_t e = cudaFuncSetAttribute(k_attn_draws<WHICH, DH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_attn_draws<WHICH, DH><<<(unsigned)(A.T * A.H), kDrawThreads, smem, st>>>(A);
+  return cudaGetLastError();
+}
+
+template <int DH>
+cudaError_t draws_which(cudaStream_t st, int which, const DrawArgs& A) {
+  if (which == 0) return draws_dh<0, DH>(st, A);
+  if (which == 1) return draws_dh<1, DH>(st, A);
+  return draws_dh<2, DH>(st, A);
+}
+
+}  // namespace
+
+size_t attn_fwd_smem(int L, int head_dim) {
+  return (size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) * 4;
+}
+size_t attn_draws_smem(int L, int head_dim) {
+  return (size_t)(2 * ((L + 3) & ~3) + kTile * head_dim + kDrawThreads * (head_dim + 1)) * 4;
+}
+
+cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
+                            const float* Q, const float* Kc, const float* Vc, const float* E,
+                            float* O, float* lse, float* gbar) {
+  FwdArgs A{Q, Kc, Vc, E, O, lse, gbar, T, L, H, 1.0f / sqrtf((float)head_dim)};
+  if (head_dim == 32) return fwd_dh<32>(st, A);
+  if (head_dim == 64) return fwd_dh<64>(st, A);
+  return fwd_dh<128>(st, A);
+}
+
+cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
+                              int head_dim, const float* Q, const float* Kc, const float* Vc,
+                              const float* E, const float* O, const float* lse,
+                              const float* gbar, float* part) {
+  if (p.T * H <= 0) return cudaSuccess;
+  const float c = 1.0f / sqrtf((float)head_dim);
+  DrawArgs A{Q, Kc, Vc, E, O, lse, gbar, part, round_keys(p.seed), (uint32_t)p.token_offset,
+             (uint32_t)p.draw_offset, ctr3_of(kTagAttnQ + which, p.stream_id),
+             which == 2 ? p.sigma : p.sigma * c, p.T, L, H, p.K, c};
+  if (head_dim == 32) return draws_which<32>(st, which, A);
+  if (head_dim == 64) return draws_which<64>(st, which, A);
+  return draws_which<128>(st, which, A);
+}
+
+cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, int H, int K,
+                                float* r) {
+  const int64_t n = T * K;
+  if (n <= 0) return cudaSuccess;
+  k_attn_combine<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, T, H, K, r);
+  return cudaGetLastError();
+}
+
+}  // namespace dust

@@ -404,6 +404,15 @@ cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const f
   return cudaGetLastError();
 }
 
+cudaError_t launch_noise_g_f32(cudaStream_t st, const dust_params& p, const float* r,
+                              float* g_out, float* gop, int tag) {
+  dim3 grid((unsigned)p.T, (unsigned)((p.d + 1023) / 1024));
+  const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
+  k_noise_g<float><<<grid, 256, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
+      (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.d, p.K, r, g_out, gop, 0);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a, int sm_count) {
   if (n <= 0) return cudaSuccess;
   int64_t blocks = (n + 255) / 256;

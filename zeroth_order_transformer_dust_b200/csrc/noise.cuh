@@ -22,6 +22,9 @@ constexpr int kTagSubsetOffset = 1;
 constexpr int kTagMlpUp = 2;
 constexpr int kTagMlpDown = 3;
 constexpr int kTagAttnOut = 4;
+constexpr int kTagAttnQ = 5;  // + 1: key, + 2: value
+constexpr int kTagAttnK = 6;
+constexpr int kTagAttnV = 7;
 
 struct U4 {
   uint32_t x, y, z, w;
