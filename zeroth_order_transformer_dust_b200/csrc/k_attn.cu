@@ -34,6 +34,10 @@
 #include "noise.cuh"
 
 namespace dust {
+
+size_t attn_fwd_smem(int L, int head_dim);
+size_t attn_draws_smem(int L, int head_dim);
+
 namespace {
 
 constexpr int kFwdWarps = 8;
@@ -96,30 +100,51 @@ struct FwdArgs {
   float scale;
 };
 
-// One warp per (token t, head h): the causal scores of row t, their
-// log-sum-exp, o_t = sum a v and gbar_t = <o_t, e_t>. Shared memory per warp:
-// the row's probabilities (L, rounded up to 4) and q_t (d_h).
+// One CTA per (sequence, head, block of kFwdWarps rows), one warp per query
+// row t: the causal scores of row t, their log-sum-exp, o_t = sum a v and
+// gbar_t = <o_t, e_t>. The CTA's rows share every key and value row, which
+// are staged through a shared-memory tile (row stride d_h + 4 floats: the
+// lanes' 16-byte reads of different rows fall in distinct banks). Shared
+// memory: per warp the row's probabilities (L rounded up to 4) and q_t
+// (d_h), and the kTile x (d_h + 4) tile.
 template <int DH>
 __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_constant__ FwdArgs A) {
   extern __shared__ __align__(16) float fsm[];
+  constexpr int kStride = DH + 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t idx = (int64_t)blockIdx.x * kFwdWarps + warp;
-  if (idx >= A.T * A.H) return;  // warp-uniform; no block barrier follows
+  const int nrb = (A.L + kFwdWarps - 1) / kFwdWarps;
+  const int rb = blockIdx.x % nrb;
+  const int h = (blockIdx.x / nrb) % A.H;
+  const int64_t seq = blockIdx.x / ((int64_t)nrb * A.H);
   const int64_t D = (int64_t)A.H * DH;
-  const int64_t t = idx / A.H;
-  const int h = (int)(idx % A.H);
-  const int64_t s0 = t - t % A.L;
-  const int n = (int)(t - s0) + 1;
+  const int64_t s0 = seq * A.L;
+  const int pos = rb * kFwdWarps + warp;      // this warp's row within the sequence
+  const bool row_ok = pos < A.L;
+  const int n = row_ok ? pos + 1 : 0;         // keys this row attends to
+  const int nmax = min(A.L, (rb + 1) * kFwdWarps);  // keys any row of the CTA needs
   const int Lp = (A.L + 3) & ~3;
   float* pr = fsm + (size_t)warp * (Lp + DH);
   float* qs = pr + Lp;
-  for (int c = lane; c < DH; c += 32) qs[c] = A.Q[t * D + h * DH + c];
-  __syncwarp();
+  float* tile = fsm + (size_t)kFwdWarps * (Lp + DH);
+  const int64_t t = s0 + pos;
+  if (row_ok)
+    for (int c = lane; c < DH; c += 32) qs[c] = A.Q[t * D + h * DH + c];
+  // pass 1: scores against staged key tiles
   float m = -INFINITY;
-  for (int j = lane; j < n; j += 32) {
-    const float v = dot_row<DH>(qs, A.Kc + (s0 + j) * D + h * DH) * A.scale;
-    pr[j] = v;
-    m = fmaxf(m, v);
+  for (int j0 = 0; j0 < nmax; j0 += kTile) {
+    const int rows = min(kTile, nmax - j0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < rows * (DH / 4); e += kFwdWarps * 32) {
+      const int r = e / (DH / 4), c4 = e % (DH / 4);
+      *reinterpret_cast<float4*>(tile + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(A.Kc + (s0 + j0 + r) * D + h * DH)[c4];
+    }
+    __syncthreads();
+    for (int j = lane; j < rows && j0 + j < n; j += 32) {
+      const float v = dot_row<DH>(qs, tile + j * kStride) * A.scale;
+      pr[j0 + j] = v;
+      m = fmaxf(m, v);
+    }
   }
   m = warp_max_f(m);
   float l = 0.f;
@@ -127,16 +152,27 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_consta
   l = warp_sum_f(l);
   const float lse = m + logf(l);
   for (int j = lane; j < n; j += 32) pr[j] = expf(pr[j] - lse);
-  __syncwarp();
+  // pass 2: o against staged value tiles
   float o[DH / 32];
 #pragma unroll
   for (int u = 0; u < DH / 32; ++u) o[u] = 0.f;
-  for (int j = 0; j < n; ++j) {
-    const float a = pr[j];
-    const float* vp = A.Vc + (s0 + j) * D + h * DH + lane;
+  for (int j0 = 0; j0 < nmax; j0 += kTile) {
+    const int rows = min(kTile, nmax - j0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < rows * (DH / 4); e += kFwdWarps * 32) {
+      const int r = e / (DH / 4), c4 = e % (DH / 4);
+      *reinterpret_cast<float4*>(tile + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(A.Vc + (s0 + j0 + r) * D + h * DH)[c4];
+    }
+    __syncthreads();
+    const int lim = min(rows, n - j0);
+    for (int j = 0; j < lim; ++j) {
+      const float a = pr[j0 + j];
 #pragma unroll
-    for (int u = 0; u < DH / 32; ++u) o[u] = fmaf(a, vp[32 * u], o[u]);
+      for (int u = 0; u < DH / 32; ++u) o[u] = fmaf(a, tile[j * kStride + lane + 32 * u], o[u]);
+    }
   }
+  if (!row_ok) return;  // after the last block barrier
   float gb = 0.f;
 #pragma unroll
   for (int u = 0; u < DH / 32; ++u) {
@@ -188,7 +224,11 @@ __device__ __forceinline__ void head_noise_smem(float* xs, const RoundKeys& keys
     const int pr = rest % kPairs;
     const int d = rest / kPairs;  // draw within the round
     const int i = i0 + d;
-    if (i >= K) continue;
+    if (i >= K) {  // no draw: zero noise, so the pair's shuffles see finite values
+      for (int q = 0; q < (DH >= 64 ? 2 : 1); ++q)
+        xs[d * (DH + 1) + (DH >= 64 ? 64 * pr + 32 * q : 0) + l] = 0.0f;
+      continue;
+    }
     const DrawConst dc = draw_const(keys, t_abs, i_off + (uint32_t)i);
     const uint32_t sb = (uint32_t)h * DH + 64u * pr;
     const uint32_t blk = sb >> 7, word = (sb >> 5) & 3u;
@@ -205,9 +245,9 @@ __device__ __forceinline__ void head_noise_smem(float* xs, const RoundKeys& keys
 }
 
 // One CTA per (token s, head h): blockIdx.x = s H + h. WHICH: 0 query,
-// 1 key, 2 value. Dynamic shared memory: two coefficient rows of L floats
-// (rounded up to 4), a kTile x d_h tile and the noise rows of one round of
-// kDrawThreads draws.
+// 1 key, 2 value. Dynamic shared memory: the per-row coefficient pairs (L
+// float2, L rounded up to 4), a kTile x (d_h + 8) tile and the noise rows of
+// one round of kDrawThreads draws.
 template <int WHICH, int DH>
 __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(const __grid_constant__ DrawArgs A) {
   extern __shared__ __align__(16) float dsm[];
@@ -222,10 +262,12 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
   const int64_t r0 = WHICH == 0 ? s0 : s;
   const int n = WHICH == 0 ? (int)(s - s0) + 1 : (int)(s0 + A.L - s);
   const int Lp = (A.L + 3) & ~3;
-  float* ca = dsm;
-  float* cb = dsm + Lp;
+  // a tile row holds the two halves of d_h with 4 floats between them, so the
+  // pair's two 16-byte reads fall in different banks
+  constexpr int kTileStride = DH + 8;
+  float2* cab = reinterpret_cast<float2*>(dsm);  // per row: (a, b) or (a, beta)
   float* tile = dsm + 2 * Lp;
-  float* xs = tile + kTile * DH;
+  float* xs = tile + kTile * kTileStride;
   fill_sincos_table(tab, A.xscale);
   for (int c = tid; c < DH; c += kDrawThreads) {
     const int64_t o = s * D + h * DH + c;
@@ -240,21 +282,30 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
     const int64_t row = (r0 + j) * D + h * DH;
     if (WHICH == 0) {
       const float a = expf(dot_row<DH>(own[0], A.Kc + row) * A.scale - lse_s);
-      ca[j] = a;
-      cb[j] = a * (dot_row<DH>(own[1], A.Vc + row) - gb_s);
+      cab[j] = make_float2(a, a * (dot_row<DH>(own[1], A.Vc + row) - gb_s));
     } else {
       const int64_t t = r0 + j;
-      ca[j] = expf(dot_row<DH>(own[0], A.Q + row) * A.scale - A.lse[t * A.H + h]);
-      if (WHICH == 1) cb[j] = dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h];
+      const float a = expf(dot_row<DH>(own[0], A.Q + row) * A.scale - A.lse[t * A.H + h]);
+      cab[j] = make_float2(a, WHICH == 1 ? dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h]
+                                         : 0.0f);
     }
   }
   __syncthreads();
   if (WHICH == 2) {
-    // w_s = sum_{t >= s} a_t,s e_t for this head
-    for (int c = tid; c < DH; c += kDrawThreads) {
-      float w = 0.f;
-      for (int j = 0; j < n; ++j) w = fmaf(ca[j], A.E[(r0 + j) * D + h * DH + c], w);
-      tile[c] = w;
+    // w_s = sum_{t >= s} a_t,s e_t for this head: kDrawThreads / d_h threads
+    // per column take interleaved rows, then their partial sums are added in
+    // a fixed order
+    constexpr int P = kDrawThreads / DH;
+    const int c = tid % DH, part = tid / DH;
+    float w = 0.f;
+#pragma unroll 4
+    for (int j = part; j < n; j += P) w = fmaf(cab[j].x, A.E[(r0 + j) * D + h * DH + c], w);
+    xs[part * DH + c] = w;
+    __syncthreads();
+    if (tid < DH) {
+      float acc = 0.f;
+      for (int q = 0; q < P; ++q) acc += xs[q * DH + tid];
+      tile[tid] = acc;
     }
   }
   const uint32_t t_abs = A.t_off + (uint32_t)s;
@@ -265,11 +316,11 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
     __syncthreads();  // the previous round's rows are consumed
     head_noise_smem<DH>(xs, A.keys, t_abs, A.i_off, i0, A.K, A.ctr3, h, tab);
     __syncthreads();
-    float x[DH];
-#pragma unroll
-    for (int c = 0; c < DH; ++c) x[c] = xs[tid * (DH + 1) + c];
     float r;
     if (WHICH == 2) {
+      float x[DH];
+#pragma unroll
+      for (int c = 0; c < DH; ++c) x[c] = xs[tid * (DH + 1) + c];
       float d0 = 0.f, d1 = 0.f;
 #pragma unroll
       for (int c = 0; c < DH; c += 2) {
@@ -278,37 +329,56 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
       }
       r = -(d0 + d1);
     } else {
+      // Thread pairs: both threads of a pair hold the noise of the pair's two
+      // draws, each for one half of the head's dims, so every 16-byte tile
+      // read feeds eight multiply-adds; one shuffle completes the dot product
+      // of the thread's own draw (tid) from the two halves.
+      constexpr int HD = DH / 2;
+      const int half = tid & 1;
+      const float* xa_row = xs + (tid & ~1) * (DH + 1) + half * HD;
+      float xa[HD], xb[HD];
+#pragma unroll
+      for (int c = 0; c < HD; ++c) {
+        xa[c] = xa_row[c];
+        xb[c] = xa_row[DH + 1 + c];
+      }
       float acc0 = 0.f, acc1 = 0.f;
       for (int j0 = 0; j0 < n; j0 += kTile) {
         const int m = min(kTile, n - j0);
         __syncthreads();
         for (int e = tid; e < m * (DH / 4); e += kDrawThreads) {
           const int row = e / (DH / 4), c4 = e % (DH / 4);
-          reinterpret_cast<float4*>(tile)[e] =
+          const int dst = row * kTileStride + 4 * c4 + (4 * c4 >= HD ? 4 : 0);
+          *reinterpret_cast<float4*>(tile + dst) =
               reinterpret_cast<const float4*>(src + (r0 + j0 + row) * D + h * DH)[c4];
         }
         __syncthreads();
-        if (live) {
 #pragma unroll 1
-          for (int jj = 0; jj < m; ++jj) {
-            const float* tr = tile + jj * DH;
-            float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+        for (int jj = 0; jj < m; ++jj) {
+          const float* tr = tile + jj * kTileStride + half * (HD + 4);
+          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < DH; c += 4) {
-              const float4 v = *reinterpret_cast<const float4*>(tr + c);
-              d0 = fmaf(x[c], v.x, d0);
-              d1 = fmaf(x[c + 1], v.y, d1);
-              d2 = fmaf(x[c + 2], v.z, d2);
-              d3 = fmaf(x[c + 3], v.w, d3);
-            }
-            const float em = expm1_acc((d0 + d1) + (d2 + d3));
-            if (WHICH == 0) {
-              acc0 = fmaf(ca[j0 + jj], em, acc0);
-              acc1 = fmaf(cb[j0 + jj], em, acc1);
-            } else {
-              const float u = ca[j0 + jj] * em;
-              acc1 = fmaf(__fdividef(u, 1.0f + u), cb[j0 + jj], acc1);
-            }
+          for (int c = 0; c < HD; c += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(tr + c);
+            a0 = fmaf(xa[c], v.x, a0);
+            b0 = fmaf(xb[c], v.x, b0);
+            a1 = fmaf(xa[c + 1], v.y, a1);
+            b1 = fmaf(xb[c + 1], v.y, b1);
+            a0 = fmaf(xa[c + 2], v.z, a0);
+            b0 = fmaf(xb[c + 2], v.z, b0);
+            a1 = fmaf(xa[c + 3], v.w, a1);
+            b1 = fmaf(xb[c + 3], v.w, b1);
+          }
+          const float pa = a0 + a1, pb = b0 + b1;
+          const float dot = (half ? pb : pa) + __shfl_xor_sync(0xffffffffu, half ? pa : pb, 1);
+          const float em = expm1_acc(dot);
+          const float2 cf = cab[j0 + jj];
+          if (WHICH == 0) {
+            acc0 = fmaf(cf.x, em, acc0);
+            acc1 = fmaf(cf.y, em, acc1);
+          } else {
+            const float u = cf.x * em;
+            acc1 = fmaf(__fdividef(u, 1.0f + u), cf.y, acc1);
           }
         }
       }
@@ -332,18 +402,19 @@ __global__ void k_attn_combine(const float* __restrict__ part, int64_t T, int32_
 
 template <int DH>
 cudaError_t fwd_dh(cudaStream_t st, const FwdArgs& A) {
-  const size_t smem = (size_t)kFwdWarps * (((A.L + 3) & ~3) + DH) * 4;
+  const size_t smem = attn_fwd_smem(A.L, DH);
   cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const int64_t rows = A.T * A.H;
-  k_attn_fwd<DH><<<(unsigned)((rows + kFwdWarps - 1) / kFwdWarps), kFwdWarps * 32, smem, st>>>(A);
+  const int64_t nrb = (A.L + kFwdWarps - 1) / kFwdWarps;
+  const int64_t blocks = (A.T / A.L) * A.H * nrb;
+  k_attn_fwd<DH><<<(unsigned)blocks, kFwdWarps * 32, smem, st>>>(A);
   return cudaGetLastError();
 }
 
 template <int WHICH, int DH>
 cudaError_t draws_dh(cudaStream_t st, const DrawArgs& A) {
-  const size_t smem = (size_t)(2 * ((A.L + 3) & ~3) + kTile * DH + kDrawThreads * (DH + 1)) * 4;
+  const size_t smem = attn_draws_smem(A.L, DH);
   cudaError_t e = cudaFuncSetAttribute(k_attn_draws<WHICH, DH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -361,10 +432,10 @@ cudaError_t draws_which(cudaStream_t st, int which, const DrawArgs& A) {
 }  // namespace
 
 size_t attn_fwd_smem(int L, int head_dim) {
-  return (size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) * 4;
+  return ((size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
 }
 size_t attn_draws_smem(int L, int head_dim) {
-  return (size_t)(2 * ((L + 3) & ~3) + kTile * head_dim + kDrawThreads * (head_dim + 1)) * 4;
+  return (size_t)(2 * ((L + 3) & ~3) + kTile * (head_dim + 8) + kDrawThreads * (head_dim + 1)) * 4;
 }
 
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
