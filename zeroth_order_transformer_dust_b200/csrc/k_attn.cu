@@ -72,13 +72,12 @@ __device__ __forceinline__ float dot_row(const float* __restrict__ a, const floa
   return (d0 + d1) + (d2 + d3);
 }
 
-// expm1 with full relative accuracy: the Taylor series to x^6 for
-// |x| <= 1/16 (truncation below x^7/5040 < 2^-40 relative), the library
+// expm1 with full relative accuracy: the Taylor series to x^5 for
+// |x| <= 1/16 (truncation below x^5/720 < 2^-29 relative), the library
 // function beyond.
 __device__ __forceinline__ float expm1_acc(float x) {
   if (fabsf(x) <= 0.0625f) {
-    float p = fmaf(x, 1.0f / 720.0f, 1.0f / 120.0f);
-    p = fmaf(x, p, 1.0f / 24.0f);
+    float p = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
     p = fmaf(x, p, 1.0f / 6.0f);
     p = fmaf(x, p, 0.5f);
     p = fmaf(x, p, 1.0f);
@@ -353,7 +352,7 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
               reinterpret_cast<const float4*>(src + (r0 + j0 + row) * D + h * DH)[c4];
         }
         __syncthreads();
-#pragma unroll 1
+#pragma unroll 2
         for (int jj = 0; jj < m; ++jj) {
           const float* tr = tile + jj * kTileStride + half * (HD + 4);
           float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
