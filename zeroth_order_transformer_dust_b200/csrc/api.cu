@@ -286,7 +286,7 @@ void dust_destroy(dust_ctx* ctx) {
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32,
                  &ctx->mlp_dn, &ctx->mlp_du, &ctx->wu2, &ctx->attn_o, &ctx->attn_lse,
-                 &ctx->attn_gb};
+                 &ctx->attn_gb, &ctx->attn_w};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -733,14 +733,19 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
       !aligned(E, 16) || !aligned(G_out, 4) || !aligned(rewards_out, 4) || !aligned(g_out, 4))
     return fail(ctx, DUST_ERR_ARG, "X, Q, K, V, E must be 16-byte aligned, the outputs 4-byte");
   if ((size_t)ctx->max_smem_optin < attn_fwd_smem(a.seq_len, a.head_dim) ||
-      (size_t)ctx->max_smem_optin < attn_draws_smem(a.seq_len, a.head_dim) + 9216)
+      (size_t)ctx->max_smem_optin < attn_draws_smem(a.seq_len, a.head_dim) + 9216 ||
+      (size_t)ctx->max_smem_optin < attn_colsum_smem(a.head_dim) ||
+      (size_t)ctx->max_smem_optin < (size_t)(Dw + 127) / 128 * 512 + 8192)
     return fail(ctx, DUST_ERR_UNSUPPORTED, "seq_len too long for shared memory");
   DUST_CU(cudaSetDevice(ctx->device));
   const cudaStream_t st = ctx->stream;
   DUST_TRY(ensure(ctx, ctx->attn_o, (size_t)T * Dw * 4));
   DUST_TRY(ensure(ctx, ctx->attn_lse, (size_t)T * H * 4));
   DUST_TRY(ensure(ctx, ctx->attn_gb, (size_t)T * H * 4));
-  DUST_TRY(ensure(ctx, ctx->part, (size_t)T * H * K * 4));
+  if (a.which == DUST_ATTN_V)
+    DUST_TRY(ensure(ctx, ctx->attn_w, (size_t)T * Dw * 4));
+  else
+    DUST_TRY(ensure(ctx, ctx->part, (size_t)T * H * K * 4));
   DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(p.dtype, T, Dw)));
   float* r = rewards_out;
   if (!r) {
@@ -756,8 +761,7 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
   ctx->launches += 1;
   mark(ctx, "attn_fwd");
   DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
-                            gb, (float*)ctx->part.p));
-  DUST_CU(launch_attn_combine(st, (const float*)ctx->part.p, T, (int)H, (int)K, r));
+                            gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r));
   ctx->launches += 2;
   mark(ctx, "draws");
   dust_params pg = p;

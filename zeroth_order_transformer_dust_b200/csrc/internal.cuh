@@ -149,7 +149,7 @@ struct dust_ctx {
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
-      attn_o, attn_lse, attn_gb;
+      attn_o, attn_lse, attn_gb, attn_w;
 };
 
 namespace dust {
@@ -263,10 +263,12 @@ cudaError_t launch_gelu_delta_rows(cudaStream_t st, const dust_params& p, const 
 // a = GELU(u) (fp64, rounded to fp32), n elements.
 cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a, int sm_count);
 // Attention internals (k_attn.cu): the clean causal attention per (token,
-// head) -> O, LSE, gbar = <o, e>; the per-head rewards of noise on the
-// query (which 0), key (1) or value (2) of every token -> part ((T H) x K);
-// their sum over heads -> r (T x K).
+// head) -> O, LSE, gbar = <o, e>; the rewards of noise on the query (which 0)
+// or key (1) of every token per head -> part ((T H) x K), summed over heads
+// into r (T x K); for the value (2), w = A^T E per head -> W (T x D), then
+// the rewards straight into r.
 size_t attn_fwd_smem(int L, int head_dim);
+size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
                             const float* Q, const float* Kc, const float* Vc, const float* E,
@@ -274,7 +276,7 @@ cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_d
 cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
-                              const float* gbar, float* part);
+                              const float* gbar, float* part, float* W, float* r);
 cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, int H, int K,
                                 float* r);
 

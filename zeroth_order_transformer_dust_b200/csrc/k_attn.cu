@@ -27,7 +27,10 @@
 // shared-memory tiles, one d_h-long dot product, one expm1 and two FMAs per
 // (draw, row). The per-row coefficients (a, <v, e> - gbar) are formed once per
 // CTA, not per draw. Per-head rewards go to a (token, head, draw) buffer that
-// a second kernel sums over heads in a fixed order.
+// a second kernel sums over heads in a fixed order. Value noise needs no per-row
+// work per draw: w_s = sum_{t >= s} a_t,s e_t comes from one tiled pass (the
+// transpose of the clean pass), and each draw is one D-long dot product over
+// all heads at once.
 #include <cmath>
 
 #include "internal.cuh"
@@ -36,6 +39,7 @@
 namespace dust {
 
 size_t attn_fwd_smem(int L, int head_dim);
+size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
 
 namespace {
@@ -244,7 +248,7 @@ __device__ __forceinline__ void head_noise_smem(float* xs, const RoundKeys& keys
 }
 
 // One CTA per (token s, head h): blockIdx.x = s H + h. WHICH: 0 query,
-// 1 key, 2 value. Dynamic shared memory: the per-row coefficient pairs (L
+// 1 key. Dynamic shared memory: the per-row coefficient pairs (L
 // float2, L rounded up to 4), a kTile x (d_h + 8) tile and the noise rows of
 // one round of kDrawThreads draws.
 template <int WHICH, int DH>
@@ -257,7 +261,7 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
   const int h = (int)(blockIdx.x % A.H);
   const int64_t D = (int64_t)A.H * DH;
   const int64_t s0 = s - s % A.L;
-  // the other index runs over tau in [s0, s] (query) or t in [s, s0 + L)
+  // the other index runs over tau in [s0, s] (query) or t in [s, s0 + L) (key)
   const int64_t r0 = WHICH == 0 ? s0 : s;
   const int n = WHICH == 0 ? (int)(s - s0) + 1 : (int)(s0 + A.L - s);
   const int Lp = (A.L + 3) & ~3;
@@ -285,28 +289,10 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
     } else {
       const int64_t t = r0 + j;
       const float a = expf(dot_row<DH>(own[0], A.Q + row) * A.scale - A.lse[t * A.H + h]);
-      cab[j] = make_float2(a, WHICH == 1 ? dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h]
-                                         : 0.0f);
+      cab[j] = make_float2(a, dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h]);
     }
   }
   __syncthreads();
-  if (WHICH == 2) {
-    // w_s = sum_{t >= s} a_t,s e_t for this head: kDrawThreads / d_h threads
-    // per column take interleaved rows, then their partial sums are added in
-    // a fixed order
-    constexpr int P = kDrawThreads / DH;
-    const int c = tid % DH, part = tid / DH;
-    float w = 0.f;
-#pragma unroll 4
-    for (int j = part; j < n; j += P) w = fmaf(cab[j].x, A.E[(r0 + j) * D + h * DH + c], w);
-    xs[part * DH + c] = w;
-    __syncthreads();
-    if (tid < DH) {
-      float acc = 0.f;
-      for (int q = 0; q < P; ++q) acc += xs[q * DH + tid];
-      tile[tid] = acc;
-    }
-  }
   const uint32_t t_abs = A.t_off + (uint32_t)s;
   const float* src = WHICH == 0 ? A.Kc : A.Q;  // rows streamed through the tile
   for (int i0 = 0; i0 < A.K; i0 += kDrawThreads) {
@@ -316,18 +302,7 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
     head_noise_smem<DH>(xs, A.keys, t_abs, A.i_off, i0, A.K, A.ctr3, h, tab);
     __syncthreads();
     float r;
-    if (WHICH == 2) {
-      float x[DH];
-#pragma unroll
-      for (int c = 0; c < DH; ++c) x[c] = xs[tid * (DH + 1) + c];
-      float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < DH; c += 2) {
-        d0 = fmaf(x[c], tile[c], d0);
-        d1 = fmaf(x[c + 1], tile[c + 1], d1);
-      }
-      r = -(d0 + d1);
-    } else {
+    {
       // Thread pairs: both threads of a pair hold the noise of the pair's two
       // draws, each for one half of the head's dims, so every 16-byte tile
       // read feeds eight multiply-adds; one shuffle completes the dot product
@@ -387,6 +362,103 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
   }
 }
 
+// Value noise, step 1: w_s = sum_{t >= s} a_t,s e_t per head, the transpose
+// of the clean pass. One CTA per (sequence, head, block of kFwdWarps key
+// positions), one warp per key position s; the CTA's later query and error
+// rows are staged through shared-memory tiles (row stride d_h + 4), and each
+// warp forms a_t,s = exp(q_t . k_s c - LSE_t) for its tile rows, then adds
+// a e_t into the lanes' d_h / 32 columns. Shared memory: kTile x (d_h + 4)
+// for Q and for E, kTile LSE values, and per warp k_s (d_h) and the tile's
+// a (kTile).
+template <int DH>
+__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_colsum(const __grid_constant__ FwdArgs A,
+                                                               float* __restrict__ W) {
+  extern __shared__ __align__(16) float csm[];
+  constexpr int kStride = DH + 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nrb = (A.L + kFwdWarps - 1) / kFwdWarps;
+  const int rb = blockIdx.x % nrb;
+  const int h = (blockIdx.x / nrb) % A.H;
+  const int64_t seq = blockIdx.x / ((int64_t)nrb * A.H);
+  const int64_t D = (int64_t)A.H * DH;
+  const int64_t s0 = seq * A.L;
+  const int pos = rb * kFwdWarps + warp;  // this warp's key position
+  const bool ok = pos < A.L;
+  const int first = rb * kFwdWarps;       // earliest query row any warp needs
+  float* qt = csm;
+  float* et = qt + kTile * kStride;
+  float* lt = et + kTile * kStride;
+  float* ks = lt + kTile + (size_t)warp * (DH + kTile);
+  float* ab = ks + DH;
+  if (ok)
+    for (int c = lane; c < DH; c += 32) ks[c] = A.Kc[(s0 + pos) * D + h * DH + c];
+  float w[DH / 32];
+#pragma unroll
+  for (int u = 0; u < DH / 32; ++u) w[u] = 0.f;
+  for (int j0 = first; j0 < A.L; j0 += kTile) {
+    const int rows = min(kTile, A.L - j0);
+    __syncthreads();
+    for (int e = threadIdx.x; e < rows * (DH / 4); e += kFwdWarps * 32) {
+      const int r = e / (DH / 4), c4 = e % (DH / 4);
+      const int64_t src = (s0 + j0 + r) * D + h * DH;
+      *reinterpret_cast<float4*>(qt + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(A.Q + src)[c4];
+      *reinterpret_cast<float4*>(et + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(A.E + src)[c4];
+    }
+    for (int r = threadIdx.x; r < rows; r += kFwdWarps * 32) lt[r] = A.lse[(s0 + j0 + r) * A.H + h];
+    __syncthreads();
+    if (ok) {
+      for (int j = lane; j < rows; j += 32)
+        ab[j] = (j0 + j >= pos) ? expf(dot_row<DH>(ks, qt + j * kStride) * A.scale - lt[j]) : 0.0f;
+      __syncwarp();
+      for (int j = 0; j < rows; ++j) {
+        const float a = ab[j];
+#pragma unroll
+        for (int u = 0; u < DH / 32; ++u) w[u] = fmaf(a, et[j * kStride + lane + 32 * u], w[u]);
+      }
+    }
+  }
+  if (!ok) return;  // after the last block barrier
+#pragma unroll
+  for (int u = 0; u < DH / 32; ++u) W[(s0 + pos) * D + h * DH + lane + 32 * u] = w[u];
+}
+
+// Value noise, step 2: r_s,i = -(sigma eps_s,i) . w_s over all D channels.
+// One CTA per token, one thread per draw; the table carries sigma, so the
+// Gaussians come out as sigma eps. Each counter (slot block, lane) gives the
+// four channels blk 128 + lane + 32 j.
+__global__ __launch_bounds__(kDrawThreads) void k_attn_vdraws(
+    const float* __restrict__ W, int64_t D, RoundKeys keys, uint32_t t_off, uint32_t i_off,
+    uint32_t ctr3, float sigma, int32_t K, float* __restrict__ r) {
+  extern __shared__ __align__(16) float ws[];  // D, padded to 128
+  __shared__ float2 tab[kSinCosTable];
+  fill_sincos_table(tab, sigma);
+  const int64_t s = blockIdx.x;
+  const int nblk = (int)((D + 127) / 128);
+  for (int c = threadIdx.x; c < nblk * 128; c += kDrawThreads) ws[c] = c < D ? W[s * D + c] : 0.f;
+  __syncthreads();
+  const uint32_t t_abs = t_off + (uint32_t)s;
+  for (int i = threadIdx.x; i < K; i += kDrawThreads) {
+    const DrawConst dc = draw_const(keys, t_abs, i_off + (uint32_t)i);
+    float a0 = 0.f, a1 = 0.f;
+    for (int blk = 0; blk < nblk; ++blk) {
+      const float* wb = ws + blk * 128;
+#pragma unroll 4
+      for (int l = 0; l < 32; ++l) {
+        const G4 g = gauss4_tab(
+            philox_from2(block_const(keys, slot_ctr0((uint32_t)blk, (uint32_t)l), ctr3), dc, keys),
+            tab);
+        a0 = fmaf(g.v[0], wb[l], a0);
+        a1 = fmaf(g.v[1], wb[l + 32], a1);
+        a0 = fmaf(g.v[2], wb[l + 64], a0);
+        a1 = fmaf(g.v[3], wb[l + 96], a1);
+      }
+    }
+    r[s * K + i] = -(a0 + a1);
+  }
+}
+
 // r[s K + i] = sum_h part[(s H + h) K + i], heads in order.
 __global__ void k_attn_combine(const float* __restrict__ part, int64_t T, int32_t H, int32_t K,
                                float* __restrict__ r) {
@@ -424,14 +496,27 @@ cudaError_t draws_dh(cudaStream_t st, const DrawArgs& A) {
 template <int DH>
 cudaError_t draws_which(cudaStream_t st, int which, const DrawArgs& A) {
   if (which == 0) return draws_dh<0, DH>(st, A);
-  if (which == 1) return draws_dh<1, DH>(st, A);
-  return draws_dh<2, DH>(st, A);
+  return draws_dh<1, DH>(st, A);
+}
+
+template <int DH>
+cudaError_t colsum_dh(cudaStream_t st, const FwdArgs& A, float* W) {
+  const size_t smem = attn_colsum_smem(DH);
+  cudaError_t e = cudaFuncSetAttribute(k_attn_colsum<DH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t nrb = (A.L + kFwdWarps - 1) / kFwdWarps;
+  k_attn_colsum<DH><<<(unsigned)((A.T / A.L) * A.H * nrb), kFwdWarps * 32, smem, st>>>(A, W);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t attn_fwd_smem(int L, int head_dim) {
   return ((size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
+}
+size_t attn_colsum_smem(int head_dim) {
+  return ((size_t)2 * kTile * (head_dim + 4) + kTile + (size_t)kFwdWarps * (head_dim + kTile)) * 4;
 }
 size_t attn_draws_smem(int L, int head_dim) {
   return (size_t)(2 * ((L + 3) & ~3) + kTile * (head_dim + 8) + kDrawThreads * (head_dim + 1)) * 4;
@@ -449,15 +534,31 @@ cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_d
 cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
-                              const float* gbar, float* part) {
+                              const float* gbar, float* part, float* W, float* r) {
   if (p.T * H <= 0) return cudaSuccess;
   const float c = 1.0f / sqrtf((float)head_dim);
+  const uint32_t ctr3 = ctr3_of(kTagAttnQ + which, p.stream_id);
+  if (which == 2) {
+    // value noise: w_s once, then one D-long dot per draw (rewards go to r)
+    FwdArgs F{Q, Kc, Vc, E, nullptr, const_cast<float*>(lse), nullptr, p.T, L, H, c};
+    cudaError_t e = head_dim == 32 ? colsum_dh<32>(st, F, W)
+                    : head_dim == 64 ? colsum_dh<64>(st, F, W) : colsum_dh<128>(st, F, W);
+    if (e != cudaSuccess) return e;
+    const int64_t D = (int64_t)H * head_dim;
+    const size_t smem = (size_t)((D + 127) / 128) * 128 * 4;
+    e = cudaFuncSetAttribute(k_attn_vdraws, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_attn_vdraws<<<(unsigned)p.T, kDrawThreads, smem, st>>>(
+        W, D, round_keys(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset, ctr3,
+        p.sigma, p.K, r);
+    return cudaGetLastError();
+  }
   DrawArgs A{Q, Kc, Vc, E, O, lse, gbar, part, round_keys(p.seed), (uint32_t)p.token_offset,
-             (uint32_t)p.draw_offset, ctr3_of(kTagAttnQ + which, p.stream_id),
-             which == 2 ? p.sigma : p.sigma * c, p.T, L, H, p.K, c};
-  if (head_dim == 32) return draws_which<32>(st, which, A);
-  if (head_dim == 64) return draws_which<64>(st, which, A);
-  return draws_which<128>(st, which, A);
+             (uint32_t)p.draw_offset, ctr3, p.sigma * c, p.T, L, H, p.K, c};
+  cudaError_t e = head_dim == 32 ? draws_which<32>(st, which, A)
+                  : head_dim == 64 ? draws_which<64>(st, which, A) : draws_which<128>(st, which, A);
+  if (e != cudaSuccess) return e;
+  return launch_attn_combine(st, part, p.T, H, p.K, r);
 }
 
 cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, int H, int K,
