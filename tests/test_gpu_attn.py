@@ -76,6 +76,32 @@ def test_long_sequence_tiles(ctx):
         _check(got, _oracle(wl, x, which), "bf16")
 
 
+@pytest.mark.parametrize("which", ["q", "k"])
+def test_cuda_core_path(ctx, which, monkeypatch):
+    # the CUDA-core form of the query and key draws (the tensor-core form is
+    # the default for head widths 64 and 128)
+    monkeypatch.setenv("DUST_ATTN_TC", "0")
+    x, got = _run(ctx, BASE, which)
+    _check(got, _oracle(BASE, x, which), "bf16")
+
+
+def test_tensor_core_range_is_reported(ctx, monkeypatch):
+    # fp16 operands hold |x| < 32768: a larger key is reported, not wrapped
+    wl = BASE.with_(T=20, seq_len=10, n_heads=2, K=8, d=8)
+    x = synth.make_attn_inputs(wl)
+    dev = {k: to_dev(v, "f32") for k, v in x.items() if k != "X"}
+    X = to_dev(x["X"], "bf16")
+    dev["K"][3, 5] = 1e6
+    with pytest.raises(dust.DustError, match="fp16 range"):
+        ctx.attn_grad(X, dev["Q"], dev["K"], dev["V"], dev["E"], seq_len=10, n_heads=2,
+                      which="q", K=8, sigma=1e-2)
+    # the context stays usable, and the CUDA-core path takes the same input
+    monkeypatch.setenv("DUST_ATTN_TC", "0")
+    ctx.attn_grad(X, dev["Q"], dev["K"], dev["V"], dev["E"], seq_len=10, n_heads=2, which="q",
+                  K=8, sigma=1e-2)
+    torch.cuda.synchronize()
+
+
 def test_offsets_and_stream(ctx):
     wl = BASE.with_(T=24, seq_len=12, n_heads=2, K=40, d=16)
     x, got = _run(ctx, wl, "k", token_offset=1000, draw_offset=77, stream_id=5)

@@ -286,7 +286,7 @@ void dust_destroy(dust_ctx* ctx) {
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32,
                  &ctx->mlp_dn, &ctx->mlp_du, &ctx->wu2, &ctx->attn_o, &ctx->attn_lse,
-                 &ctx->attn_gb, &ctx->attn_w};
+                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -310,6 +310,10 @@ dust_status dust_check(dust_ctx* ctx) {
   if (st) DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), ctx->stream));
   if (st & kStatusBadTarget) return fail(ctx, DUST_ERR_BOUNDS, "a target lies outside [0, V)");
   if (st & kStatusTimeout) return fail(ctx, DUST_ERR_TIMEOUT, "a bounded device wait expired");
+  if (st & kStatusRange)
+    return fail(ctx, DUST_ERR_UNSUPPORTED,
+                "a query or key value lies outside the fp16 range of the tensor-core attention "
+                "path (|x| < 32768); DUST_ATTN_TC=0 selects the CUDA-core path");
   return DUST_OK;
 }
 
@@ -760,8 +764,16 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
   DUST_CU(launch_attn_fwd(st, T, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse, gb));
   ctx->launches += 1;
   mark(ctx, "attn_fwd");
+  // query and key draws on tensor cores (d_h 64 or 128) unless DUST_ATTN_TC=0
+  const char* tc_env = getenv("DUST_ATTN_TC");
+  const bool use_tc = a.which != DUST_ATTN_V && a.head_dim >= 64 &&
+                      !(tc_env && tc_env[0] == '0') &&
+                      (size_t)ctx->max_smem_optin >= attn_tc_smem(a.seq_len, a.head_dim) + 9216;
+  if (use_tc)
+    DUST_TRY(ensure(ctx, ctx->attn_tcr, attn_tc_rows_bytes(T, a.seq_len, (int)H, a.head_dim)));
   DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
-                            gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r));
+                            gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r, use_tc,
+                            (uint8_t*)ctx->attn_tcr.p, ctx->d_status));
   ctx->launches += 2;
   mark(ctx, "draws");
   dust_params pg = p;

@@ -14,6 +14,7 @@ namespace dust {
 enum : uint32_t {
   kStatusBadTarget = 1u << 0,
   kStatusTimeout = 1u << 1,
+  kStatusRange = 1u << 2,  // an operand outside the range a kernel's format holds
 };
 
 struct Buf {
@@ -149,7 +150,7 @@ struct dust_ctx {
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
-      attn_o, attn_lse, attn_gb, attn_w;
+      attn_o, attn_lse, attn_gb, attn_w, attn_tcr;
 };
 
 namespace dust {
@@ -270,13 +271,17 @@ cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a
 size_t attn_fwd_smem(int L, int head_dim);
 size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
+size_t attn_tc_smem(int L, int head_dim);  // the tensor-core query/key draws (d_h 64, 128)
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
                             const float* Q, const float* Kc, const float* Vc, const float* E,
                             float* O, float* lse, float* gbar);
 cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
-                              const float* gbar, float* part, float* W, float* r);
+                              const float* gbar, float* part, float* W, float* r, bool use_tc,
+                              uint8_t* tc_rows, uint32_t* status);
+// bytes of the converted row tiles the tensor-core draws read
+size_t attn_tc_rows_bytes(int64_t T, int L, int H, int head_dim);
 cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, int H, int K,
                                 float* r);
 

@@ -33,14 +33,18 @@
 // all heads at once.
 #include <cmath>
 
+#include <cuda_fp16.h>
+
 #include "internal.cuh"
 #include "noise.cuh"
+#include "tc_ptx.cuh"
 
 namespace dust {
 
 size_t attn_fwd_smem(int L, int head_dim);
 size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
+size_t attn_tc_smem(int L, int head_dim);
 
 namespace {
 
@@ -362,6 +366,327 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core form of the query/key draws (d_h = 64 or 128). Per (token s,
+// head h) and round of 256 draws, the (draw x row) dot products are the
+// product X R^T of the draws' noise X (256 x d_h) and the streamed rows R
+// (64 x d_h per tile). Both are split into fp16 hi + lo parts and the product
+// is taken as X_hi R_hi + X_hi R_lo + X_lo R_hi, with fp32 accumulation in
+// TMEM: the dropped X_lo R_lo term is 2^-22 of |x| |r|. The noise carries a
+// power-of-two factor S (in the Box-Muller table) that keeps its lo parts
+// normal in fp16; the epilogue divides it out. One thread issues the MMAs
+// (M = 128 per half of the draws, N = 64, K = 16 per instruction, operands
+// K-major in 128-byte-swizzled shared memory tiles written by the threads);
+// every thread then reads its own draw's 64 dot products from TMEM and runs
+// the expm1 epilogue of the CUDA-core kernel. TMEM holds two tiles (double
+// buffered), so the MMAs of tile j + 1 run under the epilogue of tile j.
+constexpr int kTcRows = 64;         // rows per tile: the MMA's N
+constexpr int kTcTmemCols = 256;    // 2 buffers x 2 halves of the draws x 64 columns
+constexpr uint64_t kTcWaitNs = 2000000000ull;
+
+struct TcDrawArgs {
+  const float* Q;
+  const float* Kc;
+  const float* Vc;
+  const float* E;
+  const float* lse;
+  const float* gbar;
+  float* part;
+  const uint8_t* rows;  // the streamed rows, converted (k_attn_tc_rows)
+  RoundKeys keys;
+  uint32_t t_off, i_off, ctr3;
+  float xscale;  // sigma c S: the noise's factor
+  float inv_s;   // 1 / S
+  int64_t T;
+  int32_t L, H, K;
+  float scale;
+  uint32_t* status;
+};
+
+// Byte offset of fp16 element (row, col) of a K-major tile of 64 columns with
+// 128-byte swizzling: 16-byte chunk c of row r sits at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t sw128_off(int row, int col) {
+  return (uint32_t)row * 128u + ((((uint32_t)col >> 3) ^ ((uint32_t)row & 7u)) << 4) +
+         ((uint32_t)col & 7u) * 2u;
+}
+
+template <int DH>
+struct TcLayout {
+  static constexpr int KB = DH / 64;                      // 64-column K blocks
+  static constexpr uint32_t A_TILE = 128 * 128;           // 128 rows x 64 fp16
+  static constexpr uint32_t B_TILE = kTcRows * 128;       // 64 rows x 64 fp16
+  static constexpr uint32_t A_BYTES = 2 * 2 * KB * A_TILE;  // [half][hi, lo][kb]
+  static constexpr uint32_t B_BYTES = 2 * 2 * KB * B_TILE;  // [buffer][hi, lo][kb]
+  __host__ __device__ static constexpr uint32_t a_off(int mh, int part, int kb) {
+    return ((uint32_t)(mh * 2 + part) * KB + kb) * A_TILE;
+  }
+  __host__ __device__ static constexpr uint32_t b_off(int buf, int part, int kb) {
+    return A_BYTES + ((uint32_t)(buf * 2 + part) * KB + kb) * B_TILE;
+  }
+};
+
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && ptx::globaltimer_ns() - t0 > kTcWaitNs) return false;
+  }
+}
+
+// The round's noise (draws i0 .. i0 + 255, head h), times S, as fp16 hi and
+// lo parts in the A tiles. Work item (draw, lane, 64-slot group): one counter
+// and one Box-Muller pair give channels 64 g + lane and 64 g + 32 + lane.
+template <int DH>
+__device__ __forceinline__ void tc_noise(uint8_t* sm, const TcDrawArgs& A, uint32_t t_abs, int i0,
+                                         int h) {
+  using Ly = TcLayout<DH>;
+  for (int it = threadIdx.x; it < kDrawThreads * 32 * Ly::KB; it += kDrawThreads) {
+    const int l = it & 31;
+    const int rest = it >> 5;
+    const int g = rest % Ly::KB;
+    const int d = rest / Ly::KB;
+    float v0 = 0.f, v1 = 0.f;
+    if (i0 + d < A.K) {
+      const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)(i0 + d));
+      const uint32_t sb = (uint32_t)h * DH + 64u * g;
+      const bool hi_pair = ((sb >> 5) & 3u) != 0u;
+      const U4 w = philox_from2(block_const(A.keys, slot_ctr0(sb >> 7, (uint32_t)l), A.ctr3), dc,
+                                A.keys);
+      const float2 nn = box_muller(hi_pair ? w.z : w.x, hi_pair ? w.w : w.y, A.xscale);
+      v0 = nn.x;
+      v1 = nn.y;
+    }
+    const int r = d & 127, mh = d >> 7;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float v = q ? v1 : v0;
+      const __half hi = __float2half_rn(v);
+      const __half lo = __float2half_rn(v - __half2float(hi));
+      const uint32_t o = sw128_off(r, 32 * q + l);
+      *reinterpret_cast<__half*>(sm + Ly::a_off(mh, 0, g) + o) = hi;
+      *reinterpret_cast<__half*>(sm + Ly::a_off(mh, 1, g) + o) = lo;
+    }
+  }
+}
+
+// The streamed rows (keys for query noise, queries for key noise) as fp16
+// hi and lo parts, converted once per call into the B-tile layout: for each
+// (sequence, head, 64-row tile of the sequence) the tiles [hi | lo] x K
+// blocks, 16 KB per 64 head dims, rows past the sequence end zero. Values
+// beyond +-32768 set kStatusRange. One CTA per tile.
+template <int DH>
+__global__ __launch_bounds__(kDrawThreads) void k_attn_tc_rows(const float* __restrict__ src,
+                                                               int64_t T, int32_t L, int32_t H,
+                                                               uint8_t* __restrict__ out,
+                                                               uint32_t* status) {
+  using Ly = TcLayout<DH>;
+  const int ntile = (L + kTcRows - 1) / kTcRows;
+  const int64_t unit = blockIdx.x;  // ((seq H) + h) ntile + k
+  const int k = (int)(unit % ntile);
+  const int h = (int)((unit / ntile) % H);
+  const int64_t seq = unit / ((int64_t)ntile * H);
+  const int64_t D = (int64_t)H * DH;
+  uint8_t* dst = out + (size_t)unit * 2 * Ly::KB * Ly::B_TILE;
+  bool bad = false;
+  for (int e = threadIdx.x; e < kTcRows * (DH / 4); e += kDrawThreads) {
+    const int r = e / (DH / 4), c = 4 * (e % (DH / 4));
+    const int pos = k * kTcRows + r;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (pos < L) v = *reinterpret_cast<const float4*>(src + (seq * L + pos) * D + h * DH + c);
+    const float f[4] = {v.x, v.y, v.z, v.w};
+    __half hi[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      bad |= !(fabsf(f[q]) < 32768.0f);
+      hi[q] = __float2half_rn(f[q]);
+      lo[q] = __float2half_rn(f[q] - __half2float(hi[q]));
+    }
+    const int kb = c >> 6, col = c & 63;
+    const uint32_t o = sw128_off(r, col);
+    *reinterpret_cast<uint2*>(dst + (size_t)kb * Ly::B_TILE + o) =
+        make_uint2(((uint32_t)__half_as_ushort(hi[1]) << 16) | __half_as_ushort(hi[0]),
+                   ((uint32_t)__half_as_ushort(hi[3]) << 16) | __half_as_ushort(hi[2]));
+    *reinterpret_cast<uint2*>(dst + (size_t)(Ly::KB + kb) * Ly::B_TILE + o) =
+        make_uint2(((uint32_t)__half_as_ushort(lo[1]) << 16) | __half_as_ushort(lo[0]),
+                   ((uint32_t)__half_as_ushort(lo[3]) << 16) | __half_as_ushort(lo[2]));
+  }
+  if (bad) atomicOr(status, kStatusRange);
+}
+
+// Copy one converted tile (hi, lo: 2 KB-blocks x 8 KB each) into B buffer buf.
+template <int DH>
+__device__ __forceinline__ void tc_stage_tile(uint8_t* sm, const uint8_t* tile, int buf) {
+  using Ly = TcLayout<DH>;
+  constexpr int kVec = 2 * Ly::KB * Ly::B_TILE / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(tile);
+  uint4* dst = reinterpret_cast<uint4*>(sm + Ly::b_off(buf, 0, 0));
+#pragma unroll
+  for (int e = threadIdx.x; e < kVec; e += kDrawThreads) dst[e] = __ldg(src + e);
+}
+
+// The MMAs of one tile into TMEM buffer `buf`: for each half of the draws,
+// X_hi R_hi + X_hi R_lo + X_lo R_hi over the K blocks, 16 columns per MMA.
+template <int DH>
+__device__ __forceinline__ void tc_issue(uint32_t base, uint32_t tmem, int buf, uint32_t bar) {
+  using Ly = TcLayout<DH>;
+  constexpr uint32_t idesc = ptx::idesc_f16_f32(128, kTcRows);
+#pragma unroll
+  for (int mh = 0; mh < 2; ++mh) {
+    const uint32_t d = tmem + (uint32_t)(buf * 128 + mh * 64);
+    uint32_t accum = 0;
+#pragma unroll
+    for (int kb = 0; kb < Ly::KB; ++kb)
+#pragma unroll
+      for (int term = 0; term < 3; ++term) {
+        const uint32_t a = base + Ly::a_off(mh, term == 2 ? 1 : 0, kb);
+        const uint32_t b = base + Ly::b_off(buf, term == 1 ? 1 : 0, kb);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          ptx::mma_f16(d, ptx::sdesc_kmajor_sw128(a + 32u * k), ptx::sdesc_kmajor_sw128(b + 32u * k),
+                       idesc, accum);
+          accum = 1;
+        }
+      }
+  }
+  ptx::mma_commit(bar);
+}
+
+// One CTA per (token s, head h), as k_attn_draws; thread tid is draw i0 + tid
+// of each round, and TMEM lane (tid & 127) of the draws' half tid >> 7.
+template <int WHICH, int DH>
+__global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_tc(const __grid_constant__ TcDrawArgs A) {
+  using Ly = TcLayout<DH>;
+  extern __shared__ uint8_t tsm_raw[];
+  __shared__ __align__(16) float own[2][DH];
+  __shared__ __align__(8) uint64_t mbar[2];
+  __shared__ uint32_t tmem_slot;
+  const uint32_t raw = ptx::smem_u32(tsm_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sm = tsm_raw + (base - raw);
+  float2* cab = reinterpret_cast<float2*>(sm + Ly::A_BYTES + Ly::B_BYTES);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t s = blockIdx.x / A.H;
+  const int h = (int)(blockIdx.x % A.H);
+  const int64_t D = (int64_t)A.H * DH;
+  const int64_t s0 = s - s % A.L;
+  // rows streamed: tau in [s0, s] (query noise) or t in [s, s0 + L) (key
+  // noise), in the converted 64-row tiles of the sequence: from tile k0 on,
+  // with zero coefficients for the rows of tile k0 before s (key noise)
+  const int k0 = WHICH == 0 ? 0 : (int)((s - s0) / kTcRows);
+  const int64_t r0 = s0 + (int64_t)k0 * kTcRows;
+  const int n = WHICH == 0 ? (int)(s - s0) + 1 : (int)(s0 + A.L - r0);
+  const int ntile_seq = (A.L + kTcRows - 1) / kTcRows;
+  const uint8_t* tiles = A.rows + ((size_t)(s / A.L) * A.H + h) * ntile_seq * (2 * Ly::KB * Ly::B_TILE) +
+                         (size_t)k0 * (2 * Ly::KB * Ly::B_TILE);
+  for (int c = tid; c < DH; c += kDrawThreads) {
+    const int64_t o = s * D + h * DH + c;
+    own[0][c] = WHICH == 0 ? A.Q[o] : A.Kc[o];
+    own[1][c] = WHICH == 0 ? A.E[o] : A.Vc[o];
+  }
+  if (tid == 0) {
+    ptx::mbar_init(ptx::smem_u32(&mbar[0]), 1);
+    ptx::mbar_init(ptx::smem_u32(&mbar[1]), 1);
+    ptx::fence_barrier_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), kTcTmemCols);
+    ptx::tmem_relinquish();
+  }
+  __syncthreads();
+  const float lse_s = A.lse[s * A.H + h];
+  const float gb_s = A.gbar[s * A.H + h];
+  for (int j = tid; j < n; j += kDrawThreads) {
+    const int64_t row = (r0 + j) * D + h * DH;
+    if (WHICH == 0) {
+      const float a = expf(dot_row<DH>(own[0], A.Kc + row) * A.scale - lse_s);
+      cab[j] = make_float2(a, a * (dot_row<DH>(own[1], A.Vc + row) - gb_s));
+    } else {
+      const int64_t t = r0 + j;
+      if (t < s) {
+        cab[j] = make_float2(0.f, 0.f);
+      } else {
+        const float a = expf(dot_row<DH>(own[0], A.Q + row) * A.scale - A.lse[t * A.H + h]);
+        cab[j] = make_float2(a, dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h]);
+      }
+    }
+  }
+  for (int j = n + tid; j < ((n + kTcRows - 1) / kTcRows) * kTcRows; j += kDrawThreads)
+    cab[j] = make_float2(0.f, 0.f);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const uint32_t bar0 = ptx::smem_u32(&mbar[0]), bar1 = ptx::smem_u32(&mbar[1]);
+  const int ntiles = (n + kTcRows - 1) / kTcRows;
+  constexpr size_t kTileBytes = 2 * Ly::KB * Ly::B_TILE;
+  const int mh = warp >> 2, quad = warp & 3;
+  const uint32_t tlane = (uint32_t)(quad * 32) << 16;
+  const uint32_t t_abs = A.t_off + (uint32_t)s;
+  uint32_t parity = 0;  // bit b: parity of the next completion of mbar[b]
+  bool ok = true;
+  for (int i0 = 0; i0 < A.K && ok; i0 += kDrawThreads) {
+    tc_noise<DH>(sm, A, t_abs, i0, h);
+    tc_stage_tile<DH>(sm, tiles, 0);
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (tid == 0) tc_issue<DH>(base, tmem, 0, bar0);
+    float acc0 = 0.f, acc1 = 0.f;
+    for (int j = 0; j < ntiles; ++j) {
+      const int buf = j & 1;
+      if (j + 1 < ntiles)
+        tc_stage_tile<DH>(sm, tiles + (size_t)(j + 1) * kTileBytes, buf ^ 1);
+      ptx::fence_proxy_async();
+      ptx::tc_fence_before();
+      __syncthreads();  // tile j+1 staged; TMEM buffer buf^1 read out (tile j-1)
+      ptx::tc_fence_after();
+      if (tid == 0 && j + 1 < ntiles) tc_issue<DH>(base, tmem, buf ^ 1, buf ? bar0 : bar1);
+      const bool got = tc_wait(buf ? bar1 : bar0, (parity >> buf) & 1u);
+      parity ^= 1u << buf;
+      if (!__syncthreads_and(got)) {  // a completion that never came: stop uniformly
+        if (tid == 0) atomicOr(A.status, kStatusTimeout);
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      // rows beyond n of a partial tile are zero rows of B with zero
+      // coefficients (cab is zero-filled up to the tile boundary), so every
+      // tile runs all 64 columns, 32 at a time
+      const uint32_t ta = tmem + tlane + (uint32_t)(buf * 128 + mh * 64);
+#pragma unroll 1
+      for (int hc = 0; hc < 2; ++hc) {
+        float v[32];
+        ptx::tmem_ld32(ta + 32u * hc, v);
+        const float2* cf = cab + j * kTcRows + 32 * hc;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const float em = expm1_acc(v[q] * A.inv_s);
+          const float2 c = cf[q];
+          if (WHICH == 0) {
+            acc0 = fmaf(c.x, em, acc0);
+            acc1 = fmaf(c.y, em, acc1);
+          } else {
+            const float u = c.x * em;
+            acc1 = fmaf(__fdividef(u, 1.0f + u), c.y, acc1);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+    }
+    if (ok && i0 + tid < A.K)
+      A.part[(int64_t)blockIdx.x * A.K + i0 + tid] = WHICH == 0 ? -acc1 / (1.0f + acc0) : -acc1;
+    ptx::tc_fence_before();
+    __syncthreads();  // the round's epilogues are done before the next round's MMAs
+    ptx::tc_fence_after();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(tmem, kTcTmemCols);
+}
+
 // Value noise, step 1: w_s = sum_{t >= s} a_t,s e_t per head, the transpose
 // of the clean pass. One CTA per (sequence, head, block of kFwdWarps key
 // positions), one warp per key position s; the CTA's later query and error
@@ -499,6 +824,16 @@ cudaError_t draws_which(cudaStream_t st, int which, const DrawArgs& A) {
   return draws_dh<1, DH>(st, A);
 }
 
+template <int WHICH, int DH>
+cudaError_t draws_tc(cudaStream_t st, const TcDrawArgs& A) {
+  const size_t smem = attn_tc_smem(A.L, DH);
+  cudaError_t e = cudaFuncSetAttribute(k_attn_draws_tc<WHICH, DH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_attn_draws_tc<WHICH, DH><<<(unsigned)(A.T * A.H), kDrawThreads, smem, st>>>(A);
+  return cudaGetLastError();
+}
+
 template <int DH>
 cudaError_t colsum_dh(cudaStream_t st, const FwdArgs& A, float* W) {
   const size_t smem = attn_colsum_smem(DH);
@@ -514,6 +849,11 @@ cudaError_t colsum_dh(cudaStream_t st, const FwdArgs& A, float* W) {
 
 size_t attn_fwd_smem(int L, int head_dim) {
   return ((size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
+}
+size_t attn_tc_smem(int L, int head_dim) {
+  const size_t kb = (size_t)head_dim / 64;
+  return 1024 + 2 * 2 * kb * 128 * 128 + 2 * 2 * kb * kTcRows * 128 +
+         (size_t)((L + kTcRows - 1) / kTcRows) * kTcRows * 8;
 }
 size_t attn_colsum_smem(int head_dim) {
   return ((size_t)2 * kTile * (head_dim + 4) + kTile + (size_t)kFwdWarps * (head_dim + kTile)) * 4;
@@ -534,7 +874,8 @@ cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_d
 cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
-                              const float* gbar, float* part, float* W, float* r) {
+                              const float* gbar, float* part, float* W, float* r, bool use_tc,
+                              uint8_t* tc_rows, uint32_t* status) {
   if (p.T * H <= 0) return cudaSuccess;
   const float c = 1.0f / sqrtf((float)head_dim);
   const uint32_t ctr3 = ctr3_of(kTagAttnQ + which, p.stream_id);
@@ -553,6 +894,27 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
         p.sigma, p.K, r);
     return cudaGetLastError();
   }
+  if (use_tc && head_dim >= 64) {
+    // the noise's power-of-two factor S puts max |S sigma c eps| near 8
+    float S = 1.0f;
+    const float xmax = p.sigma * c * 5.7687f;
+    if (xmax > 0.0f) S = exp2f(floorf(log2f(8.0f / xmax)));
+    S = fminf(fmaxf(S, 0x1p-40f), 0x1p40f);
+    const int ntile = (L + kTcRows - 1) / kTcRows;
+    const unsigned units = (unsigned)((p.T / L) * H * ntile);
+    const float* rsrc = which == 0 ? Kc : Q;
+    if (head_dim == 64)
+      k_attn_tc_rows<64><<<units, kDrawThreads, 0, st>>>(rsrc, p.T, L, H, tc_rows, status);
+    else
+      k_attn_tc_rows<128><<<units, kDrawThreads, 0, st>>>(rsrc, p.T, L, H, tc_rows, status);
+    TcDrawArgs T{Q, Kc, Vc, E, lse, gbar, part, tc_rows, round_keys(p.seed),
+                 (uint32_t)p.token_offset, (uint32_t)p.draw_offset, ctr3, p.sigma * c * S,
+                 1.0f / S, p.T, L, H, p.K, c, status};
+    cudaError_t e = head_dim == 64 ? (which == 0 ? draws_tc<0, 64>(st, T) : draws_tc<1, 64>(st, T))
+                                   : (which == 0 ? draws_tc<0, 128>(st, T) : draws_tc<1, 128>(st, T));
+    if (e != cudaSuccess) return e;
+    return launch_attn_combine(st, part, p.T, H, p.K, r);
+  }
   DrawArgs A{Q, Kc, Vc, E, O, lse, gbar, part, round_keys(p.seed), (uint32_t)p.token_offset,
              (uint32_t)p.draw_offset, ctr3, p.sigma * c, p.T, L, H, p.K, c};
   cudaError_t e = head_dim == 32 ? draws_which<32>(st, which, A)
@@ -569,4 +931,11 @@ cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, i
   return cudaGetLastError();
 }
 
+}  // namespace dust
+
+namespace dust {
+size_t attn_tc_rows_bytes(int64_t T, int L, int H, int head_dim) {
+  const int64_t ntile = (L + kTcRows - 1) / kTcRows;
+  return (size_t)(T / L) * H * ntile * 2 * (head_dim / 64) * kTcRows * 128;
+}
 }  // namespace dust
