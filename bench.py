@@ -42,11 +42,13 @@ LANES_PER_SM = 128           # 4 schedulers x 32 lanes issue per clock
 # Philox4x32-10 10, Gaussian transform 4, expm1 2, reward multiply-add and
 # its operand load 2, g accumulation multiply and add 2.
 ALU_OPS_PER_ELEM = 20
-# attention internals, algorithmic lane operations: per (draw, head, row
-# visited) a d_h-long dot product, an expm1 (8) and two multiply-adds; per
-# noise entry the generator's 14 (Philox 10, Gaussian 4)
-ATTN_OPS_PER_ROW_EXTRA = 10
+# attention internals: per (draw, head, row visited) a d_h-long dot product
+# on the tensor cores, taken as three fp16 products (6 d_h flops), and on the
+# CUDA cores an expm1 (8 lane operations) and two multiply-adds; per noise
+# entry the generator's 14 lane operations (Philox 10, Gaussian 4)
+ATTN_OPS_PER_ROW = 10
 ATTN_OPS_PER_NOISE = 14
+ATTN_TC_FLOPS_PER_ROW_DH = 6
 ATTN_SAMPLE_DRAWS = 4
 # DRAM bytes (read + write) per token of the subset-draw kernel on the
 # large-subset workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of
@@ -249,19 +251,29 @@ def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
 
 
 def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
-    """ALU-issue roofline of the attention draw kernel."""
+    """Roofline of the attention draw stage. Query and key noise: tensor-core
+    products plus a CUDA-core epilogue, bound by the larger of the two times
+    (the CUDA-core side here); value noise: CUDA cores only."""
     L, H, dh = wl.seq_len, wl.n_heads, wl.head_dim
     rows = (wl.T // L) * L * (L + 1) // 2 if wl.variant in ("attn_q", "attn_k") else 0
-    ops = wl.K * H * (rows * (dh + ATTN_OPS_PER_ROW_EXTRA) + wl.T * dh * ATTN_OPS_PER_NOISE)
-    achieved = ops / (draws_ms * 1e-3) / 1e12
+    ops = wl.K * H * (rows * ATTN_OPS_PER_ROW + wl.T * dh * ATTN_OPS_PER_NOISE)
+    flops = ATTN_TC_FLOPS_PER_ROW_DH * dh * wl.K * H * rows
+    t = draws_ms * 1e-3
     f = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
     peak = SM_COUNT * LANES_PER_SM * f / 1e12
-    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s",
-            "frac": achieved / peak, "traffic": None, "kernel": "attn_draws", "ops": ops,
+    tc_peak = float(peaks.get("bf16_tflops", 1640.9))   # fp16 runs at the bf16 rate
+    roof = {"bound": "alu", "achieved": ops / t / 1e12, "peak": peak, "unit": "Tops/s",
+            "frac": ops / t / 1e12 / peak, "traffic": None, "kernel": "attn_draws", "ops": ops,
             "kernel_ms": draws_ms,
-            "ops_basis": (f"K H (rows visited x (d_h + {ATTN_OPS_PER_ROW_EXTRA}) + T d_h x "
-                          f"{ATTN_OPS_PER_NOISE})"),
+            "ops_basis": (f"K H (rows visited x {ATTN_OPS_PER_ROW} + T d_h x "
+                          f"{ATTN_OPS_PER_NOISE}) on CUDA cores"),
             "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)"}
+    if flops:
+        roof["tensor"] = {"flops": flops, "achieved_tflops": flops / t / 1e12,
+                          "peak_tflops": tc_peak, "frac": flops / t / 1e12 / tc_peak,
+                          "basis": f"{ATTN_TC_FLOPS_PER_ROW_DH} d_h flops per (draw, head, row): "
+                                   "fp16 hi/lo split, three products; peak = measured bf16 burst"}
+    return roof
 
 
 def _config(args, wl, world: int, l2: str) -> dict:
