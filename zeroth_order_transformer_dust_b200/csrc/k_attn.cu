@@ -378,8 +378,12 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
 // (M = 128 per half of the draws, N = 64, K = 16 per instruction, operands
 // K-major in 128-byte-swizzled shared memory tiles written by the threads);
 // every thread then reads its own draw's 64 dot products from TMEM and runs
-// the expm1 epilogue of the CUDA-core kernel. TMEM holds two tiles (double
-// buffered), so the MMAs of tile j + 1 run under the epilogue of tile j.
+// the expm1 epilogue of the CUDA-core kernel. TMEM and the row tiles are
+// double buffered and handed over through mbarriers, without block barriers
+// inside a round: thread 0 bulk-copies row tile j + 2 while the epilogue of
+// tile j runs, and issues the MMAs of tile j + 1 once its rows have landed
+// (full) and the epilogue of tile j - 1 has read its TMEM buffer (empty, one
+// arrival per warp); the epilogue waits for its tile's MMAs (done).
 constexpr int kTcRows = 64;         // rows per tile: the MMA's N
 constexpr int kTcTmemCols = 256;    // 2 buffers x 2 halves of the draws x 64 columns
 constexpr uint64_t kTcWaitNs = 2000000000ull;
@@ -425,12 +429,23 @@ struct TcLayout {
   }
 };
 
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity) {
+// Bounded mbarrier wait: gives up after kTcWaitNs, or at once when another
+// thread of the CTA has given up (abort), setting the abort flag and the
+// timeout bit of the status word.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                        uint32_t* status) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && ptx::globaltimer_ns() - t0 > kTcWaitNs) return false;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (ptx::globaltimer_ns() - t0 > kTcWaitNs) {
+        *abort = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
   }
 }
 
@@ -514,17 +529,6 @@ __global__ __launch_bounds__(kDrawThreads) void k_attn_tc_rows(const float* __re
   if (bad) atomicOr(status, kStatusRange);
 }
 
-// Copy one converted tile (hi, lo: 2 KB-blocks x 8 KB each) into B buffer buf.
-template <int DH>
-__device__ __forceinline__ void tc_stage_tile(uint8_t* sm, const uint8_t* tile, int buf) {
-  using Ly = TcLayout<DH>;
-  constexpr int kVec = 2 * Ly::KB * Ly::B_TILE / 16;
-  const uint4* src = reinterpret_cast<const uint4*>(tile);
-  uint4* dst = reinterpret_cast<uint4*>(sm + Ly::b_off(buf, 0, 0));
-#pragma unroll
-  for (int e = threadIdx.x; e < kVec; e += kDrawThreads) dst[e] = __ldg(src + e);
-}
-
 // The MMAs of one tile into TMEM buffer `buf`: for each half of the draws,
 // X_hi R_hi + X_hi R_lo + X_lo R_hi over the K blocks, 16 columns per MMA.
 template <int DH>
@@ -559,8 +563,9 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
   using Ly = TcLayout<DH>;
   extern __shared__ uint8_t tsm_raw[];
   __shared__ __align__(16) float own[2][DH];
-  __shared__ __align__(8) uint64_t mbar[2];
+  __shared__ __align__(8) uint64_t full[2], done[2], empty[2];
   __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
   const uint32_t raw = ptx::smem_u32(tsm_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sm = tsm_raw + (base - raw);
@@ -585,8 +590,12 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
     own[1][c] = WHICH == 0 ? A.E[o] : A.Vc[o];
   }
   if (tid == 0) {
-    ptx::mbar_init(ptx::smem_u32(&mbar[0]), 1);
-    ptx::mbar_init(ptx::smem_u32(&mbar[1]), 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_u32(&full[b]), 1);
+      ptx::mbar_init(ptx::smem_u32(&done[b]), 1);
+      ptx::mbar_init(ptx::smem_u32(&empty[b]), kDrawThreads / 32);
+    }
+    abort_flag = 0;
     ptx::fence_barrier_init();
   }
   if (warp == 0) {
@@ -617,44 +626,58 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  const uint32_t bar0 = ptx::smem_u32(&mbar[0]), bar1 = ptx::smem_u32(&mbar[1]);
   const int ntiles = (n + kTcRows - 1) / kTcRows;
-  constexpr size_t kTileBytes = 2 * Ly::KB * Ly::B_TILE;
+  constexpr uint32_t kTileBytes = 2 * Ly::KB * Ly::B_TILE;
   const int mh = warp >> 2, quad = warp & 3;
   const uint32_t tlane = (uint32_t)(quad * 32) << 16;
   const uint32_t t_abs = A.t_off + (uint32_t)s;
-  uint32_t parity = 0;  // bit b: parity of the next completion of mbar[b]
-  bool ok = true;
-  for (int i0 = 0; i0 < A.K && ok; i0 += kDrawThreads) {
+  volatile int* abort = &abort_flag;
+  // parities of the next completion of full/done/empty[b] (bit b); uses of
+  // each TMEM buffer so far (its first use needs no empty wait)
+  uint32_t pf = 0, pd = 0, pe = 0, used = 0;
+  auto copy_tile = [&](int j) {  // thread 0: row tile j into B buffer j & 1
+    const uint32_t fb = ptx::smem_u32(&full[j & 1]);
+    ptx::mbar_expect_tx(fb, kTileBytes);
+    ptx::bulk_load(base + Ly::b_off(j & 1, 0, 0), tiles + (size_t)j * kTileBytes, kTileBytes, fb);
+  };
+  auto issue = [&](int j) -> bool {  // thread 0: the MMAs of tile j
+    const int b = j & 1;
+    if (!tc_wait(ptx::smem_u32(&full[b]), (pf >> b) & 1u, abort, A.status)) return false;
+    pf ^= 1u << b;
+    if (used & (1u << b)) {
+      if (!tc_wait(ptx::smem_u32(&empty[b]), (pe >> b) & 1u, abort, A.status)) return false;
+      pe ^= 1u << b;
+    }
+    used |= 1u << b;
+    ptx::tc_fence_after();
+    tc_issue<DH>(base, tmem, b, ptx::smem_u32(&done[b]));
+    return true;
+  };
+  for (int i0 = 0; i0 < A.K && !*abort; i0 += kDrawThreads) {
+    if (tid == 0) {
+      copy_tile(0);
+      if (ntiles > 1) copy_tile(1);
+    }
     tc_noise<DH>(sm, A, t_abs, i0, h);
-    tc_stage_tile<DH>(sm, tiles, 0);
     ptx::fence_proxy_async();
     ptx::tc_fence_before();
-    __syncthreads();
+    __syncthreads();  // the round's noise is in place; the last round's epilogues are done
     ptx::tc_fence_after();
-    if (tid == 0) tc_issue<DH>(base, tmem, 0, bar0);
+    // a failed wait sets the abort flag; every thread still reaches the next
+    // done-wait, and the warps leave the tile loop warp-uniformly
+    if (tid == 0) issue(0);
     float acc0 = 0.f, acc1 = 0.f;
     for (int j = 0; j < ntiles; ++j) {
-      const int buf = j & 1;
-      if (j + 1 < ntiles)
-        tc_stage_tile<DH>(sm, tiles + (size_t)(j + 1) * kTileBytes, buf ^ 1);
-      ptx::fence_proxy_async();
-      ptx::tc_fence_before();
-      __syncthreads();  // tile j+1 staged; TMEM buffer buf^1 read out (tile j-1)
-      ptx::tc_fence_after();
-      if (tid == 0 && j + 1 < ntiles) tc_issue<DH>(base, tmem, buf ^ 1, buf ? bar0 : bar1);
-      const bool got = tc_wait(buf ? bar1 : bar0, (parity >> buf) & 1u);
-      parity ^= 1u << buf;
-      if (!__syncthreads_and(got)) {  // a completion that never came: stop uniformly
-        if (tid == 0) atomicOr(A.status, kStatusTimeout);
-        ok = false;
-        break;
-      }
+      const int b = j & 1;
+      if (tid == 0 && j + 1 < ntiles) issue(j + 1);
+      const bool got = tc_wait(ptx::smem_u32(&done[b]), (pd >> b) & 1u, abort, A.status);
+      if (!__all_sync(0xffffffffu, got)) break;  // the warp converges here (tcgen05.ld is .aligned)
+      pd ^= 1u << b;
       ptx::tc_fence_after();
       // rows beyond n of a partial tile are zero rows of B with zero
       // coefficients (cab is zero-filled up to the tile boundary), so every
       // tile runs all 64 columns, 32 at a time
-      const uint32_t ta = tmem + tlane + (uint32_t)(buf * 128 + mh * 64);
+      const uint32_t ta = tmem + tlane + (uint32_t)(b * 128 + mh * 64);
 #pragma unroll 1
       for (int hc = 0; hc < 2; ++hc) {
         float v[32];
@@ -674,11 +697,15 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
         }
       }
       ptx::tc_fence_before();
+      __syncwarp();
+      if ((tid & 31) == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[b]));
+      // B buffer b is free again (the MMAs of tile j are done): tile j + 2
+      if (tid == 0 && j + 2 < ntiles) copy_tile(j + 2);
     }
-    if (ok && i0 + tid < A.K)
+    if (!*abort && i0 + tid < A.K)
       A.part[(int64_t)blockIdx.x * A.K + i0 + tid] = WHICH == 0 ? -acc1 / (1.0f + acc0) : -acc1;
     ptx::tc_fence_before();
-    __syncthreads();  // the round's epilogues are done before the next round's MMAs
+    __syncthreads();  // every epilogue of the round is done before the next round's noise
     ptx::tc_fence_after();
   }
   ptx::tc_fence_before();
