@@ -138,7 +138,6 @@ dust_status finish(dust_ctx* ctx, uint32_t flags) {
   return dust_check(ctx);
 }
 
-// path: 0 automatic, 1 CUDA cores, 2 tensor cores.
 // path: 0 automatic, 1 CUDA cores, 2 tensor cores one CTA per tile, 3 tensor
 // cores with CTA pairs, 4 as 2 with the pipeline waits' limit at zero (an
 // injected timeout).

@@ -20,14 +20,17 @@
 //       w_s = sum_{t >= s} a_t,s e_t.
 // These are exact rewrites of the softmax (nothing is linearised).
 //
-// B200 mapping: the clean pass is one warp per (token, head). The draws run
-// one CTA per (token s, head h) and one thread per draw: the thread draws the
-// head's d_h noise entries into registers once, then streams the keys (query
-// noise) or the later queries (key noise) of the sequence through
-// shared-memory tiles, one d_h-long dot product, one expm1 and two FMAs per
-// (draw, row). The per-row coefficients (a, <v, e> - gbar) are formed once per
-// CTA, not per draw. Per-head rewards go to a (token, head, draw) buffer that
-// a second kernel sums over heads in a fixed order. Value noise needs no per-row
+// B200 mapping: the clean pass is one CTA per (sequence, head, 8 query rows)
+// with the rows' keys and values staged through shared memory. The query and
+// key draws run one CTA per (token s, head h) and one thread per draw: the
+// per-row coefficients (a, <v, e> - gbar) are formed once per CTA, the noise
+// of a round of 256 draws once per round, and the keys (query noise) or the
+// later queries (key noise) of the sequence stream through 64-row tiles: one
+// d_h-long dot product per (draw, row), on tcgen05 in the default form
+// (fp16 hi/lo products into TMEM, k_attn_draws_tc) or on the CUDA cores
+// (k_attn_draws), then one expm1 and two FMAs on the CUDA cores. Per-head
+// rewards go to a (token, head, draw) buffer that a second kernel sums over
+// heads in a fixed order. Value noise needs no per-row
 // work per draw: w_s = sum_{t >= s} a_t,s e_t comes from one tiled pass (the
 // transpose of the clean pass), and each draw is one D-long dot product over
 // all heads at once.
