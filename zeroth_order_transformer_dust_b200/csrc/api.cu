@@ -285,7 +285,7 @@ void dust_destroy(dust_ctx* ctx) {
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32,
                  &ctx->mlp_dn, &ctx->mlp_du, &ctx->wu2, &ctx->attn_o, &ctx->attn_lse,
-                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr};
+                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr, &ctx->attn_coef};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -768,11 +768,13 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
   const bool use_tc = a.which != DUST_ATTN_V && a.head_dim >= 64 &&
                       !(tc_env && tc_env[0] == '0') &&
                       (size_t)ctx->max_smem_optin >= attn_tc_smem(a.seq_len, a.head_dim) + 9216;
-  if (use_tc)
+  if (use_tc) {
     DUST_TRY(ensure(ctx, ctx->attn_tcr, attn_tc_rows_bytes(T, a.seq_len, (int)H, a.head_dim)));
+    DUST_TRY(ensure(ctx, ctx->attn_coef, attn_coef_bytes(T, a.seq_len, (int)H)));
+  }
   DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
                             gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r, use_tc,
-                            (uint8_t*)ctx->attn_tcr.p, ctx->d_status));
+                            (uint8_t*)ctx->attn_tcr.p, (float2*)ctx->attn_coef.p, ctx->d_status));
   ctx->launches += 2;
   mark(ctx, "draws");
   dust_params pg = p;

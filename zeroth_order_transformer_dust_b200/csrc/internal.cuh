@@ -150,7 +150,7 @@ struct dust_ctx {
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
-      attn_o, attn_lse, attn_gb, attn_w, attn_tcr;
+      attn_o, attn_lse, attn_gb, attn_w, attn_tcr, attn_coef;
 };
 
 namespace dust {
@@ -279,9 +279,11 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
                               const float* gbar, float* part, float* W, float* r, bool use_tc,
-                              uint8_t* tc_rows, uint32_t* status);
-// bytes of the converted row tiles the tensor-core draws read
+                              uint8_t* tc_rows, float2* coef, uint32_t* status);
+// bytes of the converted row tiles and of the coefficient rows the
+// tensor-core draws read
 size_t attn_tc_rows_bytes(int64_t T, int L, int H, int head_dim);
+size_t attn_coef_bytes(int64_t T, int L, int H);
 cudaError_t launch_attn_combine(cudaStream_t st, const float* part, int64_t T, int H, int K,
                                 float* r);
 

@@ -48,12 +48,14 @@ size_t attn_fwd_smem(int L, int head_dim);
 size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
 size_t attn_tc_smem(int L, int head_dim);
+size_t attn_coef_smem(int head_dim);
 
 namespace {
 
 constexpr int kFwdWarps = 8;
 constexpr int kDrawThreads = 256;
 constexpr int kTile = 64;  // rows per staged tile
+constexpr int kTcRows = 64;  // rows per tile of the tensor-core draws: the MMA's N
 
 __device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
@@ -369,6 +371,86 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
   }
 }
 
+// Per-row coefficients of the query and key draws, for every (token s, head
+// h) at once: row (s, h) of C holds, at column c of s's sequence (c < the
+// sequence length rounded up to 64; zero where the row does not reach),
+//   query noise: (a_s,c, a_s,c (<v_c, e_s> - gbar_s))   for c <= pos(s),
+//   key noise:   (a_c,s, <v_s, e_c> - gbar_c)           for c >= pos(s).
+// One CTA per (sequence, head, block of kFwdWarps rows s), one warp per s;
+// the streamed rows (keys and values, or queries and errors) are staged in
+// shared-memory tiles (row stride d_h + 4) shared by the CTA's warps, each
+// lane takes tile rows lane and lane + 32, and the row's writes are
+// coalesced float2 stores.
+template <int WHICH, int DH>
+__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_coef(const __grid_constant__ FwdArgs A,
+                                                             float2* __restrict__ C) {
+  extern __shared__ __align__(16) float qsm[];
+  constexpr int kStride = DH + 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nrb = (A.L + kFwdWarps - 1) / kFwdWarps;
+  const int rb = blockIdx.x % nrb;
+  const int h = (blockIdx.x / nrb) % A.H;
+  const int64_t seq = blockIdx.x / ((int64_t)nrb * A.H);
+  const int64_t D = (int64_t)A.H * DH;
+  const int64_t s0 = seq * A.L;
+  const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
+  const int pos = rb * kFwdWarps + warp;
+  const bool ok = pos < A.L;
+  float* t1 = qsm;                          // keys (query) / queries (key)
+  float* t2 = t1 + kTile * kStride;         // values (query) / errors (key)
+  float* lt = t2 + kTile * kStride;         // per tile row: LSE and gbar (key)
+  float* gt = lt + kTile;
+  float* own = gt + kTile + (size_t)warp * 2 * DH;  // q_s, e_s (query) / k_s, v_s (key)
+  const int64_t so = (s0 + pos) * D + h * DH;
+  if (ok)
+    for (int c = lane; c < DH; c += 32) {
+      own[c] = WHICH == 0 ? A.Q[so + c] : A.Kc[so + c];
+      own[DH + c] = WHICH == 0 ? A.E[so + c] : A.Vc[so + c];
+    }
+  const float lse_s = ok ? A.lse[(s0 + pos) * A.H + h] : 0.f;
+  const float gb_s = ok ? A.gbar[(s0 + pos) * A.H + h] : 0.f;
+  // columns: query noise needs [0, pos] of each row, key noise [pos, L), both
+  // padded to whole 64-column tiles
+  const int c_lo = WHICH == 0 ? 0 : rb * kFwdWarps / kTcRows * kTcRows;
+  const int c_hi = WHICH == 0 ? min(Lt, ((rb + 1) * kFwdWarps + kTcRows - 1) / kTcRows * kTcRows)
+                              : Lt;
+  float2* crow = C + ((s0 + pos) * A.H + h) * (int64_t)Lt;
+  for (int j0 = c_lo; j0 < c_hi; j0 += kTile) {
+    const int rows = min(kTile, A.L - j0);  // rows past the sequence end stay unread
+    __syncthreads();
+    for (int e = threadIdx.x; e < max(rows, 0) * (DH / 4); e += kFwdWarps * 32) {
+      const int r = e / (DH / 4), c4 = e % (DH / 4);
+      const int64_t src = (s0 + j0 + r) * D + h * DH;
+      *reinterpret_cast<float4*>(t1 + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(WHICH == 0 ? A.Kc + src : A.Q + src)[c4];
+      *reinterpret_cast<float4*>(t2 + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(WHICH == 0 ? A.Vc + src : A.E + src)[c4];
+    }
+    if (WHICH == 1)
+      for (int r = threadIdx.x; r < rows; r += kFwdWarps * 32) {
+        lt[r] = A.lse[(s0 + j0 + r) * A.H + h];
+        gt[r] = A.gbar[(s0 + j0 + r) * A.H + h];
+      }
+    __syncthreads();
+    if (ok) {
+      for (int j = lane; j < kTile; j += 32) {
+        const int c = j0 + j;
+        float2 v = make_float2(0.f, 0.f);
+        if (c < A.L && (WHICH == 0 ? c <= pos : c >= pos)) {
+          if (WHICH == 0) {
+            const float a = expf(dot_row<DH>(own, t1 + j * kStride) * A.scale - lse_s);
+            v = make_float2(a, a * (dot_row<DH>(own + DH, t2 + j * kStride) - gb_s));
+          } else {
+            const float a = expf(dot_row<DH>(own, t1 + j * kStride) * A.scale - lt[j]);
+            v = make_float2(a, dot_row<DH>(own + DH, t2 + j * kStride) - gt[j]);
+          }
+        }
+        crow[c] = v;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Tensor-core form of the query/key draws (d_h = 64 or 128). Per (token s,
 // head h) and round of 256 draws, the (draw x row) dot products are the
@@ -387,7 +469,6 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
 // tile j runs, and issues the MMAs of tile j + 1 once its rows have landed
 // (full) and the epilogue of tile j - 1 has read its TMEM buffer (empty, one
 // arrival per warp); the epilogue waits for its tile's MMAs (done).
-constexpr int kTcRows = 64;         // rows per tile: the MMA's N
 constexpr int kTcTmemCols = 256;    // 2 buffers x 2 halves of the draws x 64 columns
 constexpr uint64_t kTcWaitNs = 2000000000ull;
 
@@ -400,6 +481,7 @@ struct TcDrawArgs {
   const float* gbar;
   float* part;
   const uint8_t* rows;  // the streamed rows, converted (k_attn_tc_rows)
+  const float2* coef;   // the per-row coefficients (k_attn_coef), rows of Lt
   RoundKeys keys;
   uint32_t t_off, i_off, ctr3;
   float xscale;  // sigma c S: the noise's factor
@@ -565,7 +647,6 @@ template <int WHICH, int DH>
 __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_tc(const __grid_constant__ TcDrawArgs A) {
   using Ly = TcLayout<DH>;
   extern __shared__ uint8_t tsm_raw[];
-  __shared__ __align__(16) float own[2][DH];
   __shared__ __align__(8) uint64_t full[2], done[2], empty[2];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -576,7 +657,6 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t s = blockIdx.x / A.H;
   const int h = (int)(blockIdx.x % A.H);
-  const int64_t D = (int64_t)A.H * DH;
   const int64_t s0 = s - s % A.L;
   // rows streamed: tau in [s0, s] (query noise) or t in [s, s0 + L) (key
   // noise), in the converted 64-row tiles of the sequence: from tile k0 on,
@@ -587,11 +667,6 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
   const int ntile_seq = (A.L + kTcRows - 1) / kTcRows;
   const uint8_t* tiles = A.rows + ((size_t)(s / A.L) * A.H + h) * ntile_seq * (2 * Ly::KB * Ly::B_TILE) +
                          (size_t)k0 * (2 * Ly::KB * Ly::B_TILE);
-  for (int c = tid; c < DH; c += kDrawThreads) {
-    const int64_t o = s * D + h * DH + c;
-    own[0][c] = WHICH == 0 ? A.Q[o] : A.Kc[o];
-    own[1][c] = WHICH == 0 ? A.E[o] : A.Vc[o];
-  }
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(ptx::smem_u32(&full[b]), 1);
@@ -605,26 +680,13 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
     ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), kTcTmemCols);
     ptx::tmem_relinquish();
   }
-  __syncthreads();
-  const float lse_s = A.lse[s * A.H + h];
-  const float gb_s = A.gbar[s * A.H + h];
-  for (int j = tid; j < n; j += kDrawThreads) {
-    const int64_t row = (r0 + j) * D + h * DH;
-    if (WHICH == 0) {
-      const float a = expf(dot_row<DH>(own[0], A.Kc + row) * A.scale - lse_s);
-      cab[j] = make_float2(a, a * (dot_row<DH>(own[1], A.Vc + row) - gb_s));
-    } else {
-      const int64_t t = r0 + j;
-      if (t < s) {
-        cab[j] = make_float2(0.f, 0.f);
-      } else {
-        const float a = expf(dot_row<DH>(own[0], A.Q + row) * A.scale - A.lse[t * A.H + h]);
-        cab[j] = make_float2(a, dot_row<DH>(own[1], A.E + row) - A.gbar[t * A.H + h]);
-      }
-    }
+  // the coefficient row of (s, h) from column r0 - s0 on, whole tiles
+  {
+    const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
+    const float2* crow = A.coef + (s * A.H + h) * (int64_t)Lt + (r0 - s0);
+    const int m = (n + kTcRows - 1) / kTcRows * kTcRows;
+    for (int j = tid; j < m; j += kDrawThreads) cab[j] = __ldg(crow + j);
   }
-  for (int j = n + tid; j < ((n + kTcRows - 1) / kTcRows) * kTcRows; j += kDrawThreads)
-    cab[j] = make_float2(0.f, 0.f);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -855,6 +917,15 @@ cudaError_t draws_which(cudaStream_t st, int which, const DrawArgs& A) {
 }
 
 template <int WHICH, int DH>
+cudaError_t coef_dh(cudaStream_t st, const FwdArgs& F, float2* C, size_t smem, unsigned blocks) {
+  cudaError_t e = cudaFuncSetAttribute(k_attn_coef<WHICH, DH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_attn_coef<WHICH, DH><<<blocks, kFwdWarps * 32, smem, st>>>(F, C);
+  return cudaGetLastError();
+}
+
+template <int WHICH, int DH>
 cudaError_t draws_tc(cudaStream_t st, const TcDrawArgs& A) {
   const size_t smem = attn_tc_smem(A.L, DH);
   cudaError_t e = cudaFuncSetAttribute(k_attn_draws_tc<WHICH, DH>,
@@ -879,6 +950,9 @@ cudaError_t colsum_dh(cudaStream_t st, const FwdArgs& A, float* W) {
 
 size_t attn_fwd_smem(int L, int head_dim) {
   return ((size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
+}
+size_t attn_coef_smem(int head_dim) {
+  return ((size_t)2 * kTile * (head_dim + 4) + 2 * kTile + (size_t)kFwdWarps * 2 * head_dim) * 4;
 }
 size_t attn_tc_smem(int L, int head_dim) {
   const size_t kb = (size_t)head_dim / 64;
@@ -905,7 +979,7 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
                               const float* gbar, float* part, float* W, float* r, bool use_tc,
-                              uint8_t* tc_rows, uint32_t* status) {
+                              uint8_t* tc_rows, float2* coef, uint32_t* status) {
   if (p.T * H <= 0) return cudaSuccess;
   const float c = 1.0f / sqrtf((float)head_dim);
   const uint32_t ctr3 = ctr3_of(kTagAttnQ + which, p.stream_id);
@@ -937,7 +1011,20 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
       k_attn_tc_rows<64><<<units, kDrawThreads, 0, st>>>(rsrc, p.T, L, H, tc_rows, status);
     else
       k_attn_tc_rows<128><<<units, kDrawThreads, 0, st>>>(rsrc, p.T, L, H, tc_rows, status);
-    TcDrawArgs T{Q, Kc, Vc, E, lse, gbar, part, tc_rows, round_keys(p.seed),
+    {
+      FwdArgs F{Q, Kc, Vc, E, nullptr, const_cast<float*>(lse), const_cast<float*>(gbar), p.T, L,
+                H, c};
+      const size_t csm = attn_coef_smem(head_dim);
+      const unsigned cblocks = (unsigned)((p.T / L) * H * ((L + kFwdWarps - 1) / kFwdWarps));
+      cudaError_t ce;
+      if (head_dim == 64)
+        ce = which == 0 ? coef_dh<0, 64>(st, F, coef, csm, cblocks) : coef_dh<1, 64>(st, F, coef, csm, cblocks);
+      else
+        ce = which == 0 ? coef_dh<0, 128>(st, F, coef, csm, cblocks)
+                        : coef_dh<1, 128>(st, F, coef, csm, cblocks);
+      if (ce != cudaSuccess) return ce;
+    }
+    TcDrawArgs T{Q, Kc, Vc, E, lse, gbar, part, tc_rows, coef, round_keys(p.seed),
                  (uint32_t)p.token_offset, (uint32_t)p.draw_offset, ctr3, p.sigma * c * S,
                  1.0f / S, p.T, L, H, p.K, c, status};
     cudaError_t e = head_dim == 64 ? (which == 0 ? draws_tc<0, 64>(st, T) : draws_tc<1, 64>(st, T))
@@ -967,5 +1054,8 @@ namespace dust {
 size_t attn_tc_rows_bytes(int64_t T, int L, int H, int head_dim) {
   const int64_t ntile = (L + kTcRows - 1) / kTcRows;
   return (size_t)(T / L) * H * ntile * 2 * (head_dim / 64) * kTcRows * 128;
+}
+size_t attn_coef_bytes(int64_t T, int L, int H) {
+  return (size_t)T * H * ((L + kTcRows - 1) / kTcRows * kTcRows) * 8;
 }
 }  // namespace dust
