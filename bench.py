@@ -276,6 +276,27 @@ def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
     return roof
 
 
+def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
+    """Tensor-core roofline of the MLP-block perturbed pass: the flops its
+    GEMMs execute per (token, draw) row, the activations contracted as bf16
+    hi/lo planes (K doubled), against the sustained bf16 peak (a pass of
+    hundreds of milliseconds runs under the power cap)."""
+    d, dff, V = wl.d, wl.d_ff, wl.V
+    per_row = 2.0 * (2 * d) * V                   # dz = dh W_head^T with the reward epilogue
+    if wl.variant in ("mlp", "attn_out"):
+        per_row += 2.0 * (2 * dff) * d            # dh = da W_down^T
+    if wl.variant == "attn_out":
+        per_row += 2.0 * (2 * d) * dff            # du = (sigma eps) W_up^T
+    flops = per_row * wl.T * wl.K
+    t = perturbed_ms * 1e-3
+    peak = float(peaks.get("bf16_tflops_sustained", 1416.7))
+    return {"bound": "tensor", "achieved": flops / t / 1e12, "peak": peak, "unit": "TFLOP/s",
+            "frac": flops / t / 1e12 / peak, "traffic": None, "kernel": "perturbed GEMMs",
+            "flops": flops, "kernel_ms": perturbed_ms,
+            "flops_basis": "executed flops of the perturbed GEMMs (hi/lo planes: K doubled)",
+            "peak_basis": "measured bf16 sustained (power-capped) peak"}
+
+
 def _config(args, wl, world: int, l2: str) -> dict:
     """The workload of a JSON line (the same keys on both arms)."""
     cfg = {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
@@ -452,6 +473,9 @@ def run_dust(args):
                                          "tokens to this launch")
     if wl.seq_len and stages.get("draws"):
         roof = _attn_roofline(wl, stages["draws"], peaks)
+        roof["peak_kind"] = peak_kind
+    if wl.variant in ("mlp", "mlp_down", "attn_out") and stages.get("perturbed"):
+        roof = _mlp_roofline(wl, stages["perturbed"], peaks)
         roof["peak_kind"] = peak_kind
     gemm_flops = 2.0 * wl.T * wl.d * wl.V
     extra = {}
