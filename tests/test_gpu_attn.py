@@ -68,6 +68,14 @@ def test_parity_other_head_widths(ctx, head_dim, which):
     _check(got, _oracle(wl, x, which), "f32")
 
 
+def test_wide_heads_two_rounds(ctx):
+    # 128-wide heads on the tensor cores (two K blocks per operand) with two
+    # rounds of draws
+    wl = BASE.with_(T=70, seq_len=35, n_heads=2, head_dim=128, K=300, d=24)
+    x, got = _run(ctx, wl, "q")
+    _check(got, _oracle(wl, x, "q"), "bf16")
+
+
 def test_long_sequence_tiles(ctx):
     # 150 keys per row at the end: three 64-row tiles, the last ragged
     wl = BASE.with_(T=150, seq_len=150, n_heads=1, K=20, d=24)
