@@ -775,7 +775,9 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
   DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
                             gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r, use_tc,
                             (uint8_t*)ctx->attn_tcr.p, (float2*)ctx->attn_coef.p, ctx->d_status));
-  ctx->launches += 2;
+  // value: column sums + draws; tensor cores: coefficients, row conversion,
+  // draws, head sum; CUDA cores: draws, head sum
+  ctx->launches += use_tc ? 4 : 2;
   mark(ctx, "draws");
   dust_params pg = p;
   pg.d = Dw;  // the noise width
