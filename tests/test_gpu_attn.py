@@ -76,6 +76,15 @@ def test_wide_heads_two_rounds(ctx):
     _check(got, _oracle(wl, x, "q"), "bf16")
 
 
+@pytest.mark.parametrize("which", ["q", "k"])
+def test_large_sigma(ctx, which):
+    # sigma = 0.5: the score changes reach far beyond 1/16, so the exact expm1
+    # path of the epilogues runs as well as the series
+    wl = BASE.with_(T=40, seq_len=20, n_heads=2, K=64, d=16, sigma=0.5)
+    x, got = _run(ctx, wl, which)
+    _check(got, _oracle(wl, x, which), "bf16")
+
+
 def test_long_sequence_tiles(ctx):
     # 150 keys per row at the end: three 64-row tiles, the last ragged
     wl = BASE.with_(T=150, seq_len=150, n_heads=1, K=20, d=24)

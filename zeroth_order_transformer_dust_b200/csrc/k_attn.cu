@@ -641,6 +641,29 @@ __device__ __forceinline__ void tc_issue(uint32_t base, uint32_t tmem, int buf, 
   ptx::mma_commit(bar);
 }
 
+// The epilogue of 32 columns with the exact expm1 (a product beyond
+// |x| = 1/16 among them): reads the columns from TMEM again, out of line so
+// that the common path keeps its registers. Called by whole warps.
+template <int WHICH>
+__device__ __noinline__ float2 tc_exact_chunk(uint32_t taddr, const float2* cf, float inv_s) {
+  float v[32];
+  ptx::tmem_ld32(taddr, v);
+  float c0 = 0.f, c1 = 0.f;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const float em = expm1_acc(v[q] * inv_s);
+    const float2 c = cf[q];
+    if (WHICH == 0) {
+      c0 = fmaf(c.x, em, c0);
+      c1 = fmaf(c.y, em, c1);
+    } else {
+      const float u = c.x * em;
+      c1 = fmaf(__fdividef(u, 1.0f + u), c.y, c1);
+    }
+  }
+  return make_float2(c0, c1);
+}
+
 // One CTA per (token s, head h), as k_attn_draws; thread tid is draw i0 + tid
 // of each round, and TMEM lane (tid & 127) of the draws' half tid >> 7.
 template <int WHICH, int DH>
@@ -748,18 +771,36 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
         float v[32];
         ptx::tmem_ld32(ta + 32u * hc, v);
         const float2* cf = cab + j * kTcRows + 32 * hc;
+        // the degree-5 series of expm1 without a branch per element; a
+        // product beyond |x| = 1/16 (rare at the usual sigma) sends the
+        // warp's 32 columns through the exact form instead
+        float c0 = 0.f, c1 = 0.f;
+        bool wide = false;
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-          const float em = expm1_acc(v[q] * A.inv_s);
+          const float x = v[q] * A.inv_s;
+          wide |= fabsf(x) > 0.0625f;
+          float pp = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
+          pp = fmaf(x, pp, 1.0f / 6.0f);
+          pp = fmaf(x, pp, 0.5f);
+          pp = fmaf(x, pp, 1.0f);
+          const float em = x * pp;
           const float2 c = cf[q];
           if (WHICH == 0) {
-            acc0 = fmaf(c.x, em, acc0);
-            acc1 = fmaf(c.y, em, acc1);
+            c0 = fmaf(c.x, em, c0);
+            c1 = fmaf(c.y, em, c1);
           } else {
             const float u = c.x * em;
-            acc1 = fmaf(__fdividef(u, 1.0f + u), c.y, acc1);
+            c1 = fmaf(__fdividef(u, 1.0f + u), c.y, c1);
           }
         }
+        if (__any_sync(0xffffffffu, wide)) {  // warp-uniform
+          const float2 cc = tc_exact_chunk<WHICH>(ta + 32u * hc, cf, A.inv_s);
+          c0 = cc.x;
+          c1 = cc.y;
+        }
+        acc0 += c0;
+        acc1 += c1;
       }
       ptx::tc_fence_before();
       __syncwarp();
