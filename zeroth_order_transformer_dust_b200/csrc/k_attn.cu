@@ -670,7 +670,7 @@ template <int WHICH, int DH>
 __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_tc(const __grid_constant__ TcDrawArgs A) {
   using Ly = TcLayout<DH>;
   extern __shared__ uint8_t tsm_raw[];
-  __shared__ __align__(8) uint64_t full[2], done[2], empty[2];
+  __shared__ __align__(8) uint64_t full[2], done[2], empty[2], cfull;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   const uint32_t raw = ptx::smem_u32(tsm_raw);
@@ -696,6 +696,7 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
       ptx::mbar_init(ptx::smem_u32(&done[b]), 1);
       ptx::mbar_init(ptx::smem_u32(&empty[b]), kDrawThreads / 32);
     }
+    ptx::mbar_init(ptx::smem_u32(&cfull), 1);
     abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -703,15 +704,18 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
     ptx::tmem_alloc(ptx::smem_u32(&tmem_slot), kTcTmemCols);
     ptx::tmem_relinquish();
   }
-  // the coefficient row of (s, h) from column r0 - s0 on, whole tiles
-  {
-    const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
-    const float2* crow = A.coef + (s * A.H + h) * (int64_t)Lt + (r0 - s0);
-    const int m = (n + kTcRows - 1) / kTcRows * kTcRows;
-    for (int j = tid; j < m; j += kDrawThreads) cab[j] = __ldg(crow + j);
-  }
   ptx::tc_fence_before();
   __syncthreads();
+  // the coefficient row of (s, h) from column r0 - s0 on, whole tiles, by
+  // bulk copy: it lands while the round's noise is drawn
+  if (tid == 0) {
+    const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
+    const float2* crow = A.coef + (s * A.H + h) * (int64_t)Lt + (r0 - s0);
+    const uint32_t bytes = (uint32_t)((n + kTcRows - 1) / kTcRows * kTcRows) * 8u;
+    const uint32_t cb = ptx::smem_u32(&cfull);
+    ptx::mbar_expect_tx(cb, bytes);
+    ptx::bulk_load(ptx::smem_u32(cab), crow, bytes, cb);
+  }
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_slot;
   const int ntiles = (n + kTcRows - 1) / kTcRows;
@@ -754,6 +758,9 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
     // a failed wait sets the abort flag; every thread still reaches the next
     // done-wait, and the warps leave the tile loop warp-uniformly
     if (tid == 0) issue(0);
+    // the coefficient row (phase 0 of cfull: at once in later rounds); a
+    // failure sets the abort flag, which ends the tile loop below
+    (void)__all_sync(0xffffffffu, tc_wait(ptx::smem_u32(&cfull), 0u, abort, A.status));
     float acc0 = 0.f, acc1 = 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
