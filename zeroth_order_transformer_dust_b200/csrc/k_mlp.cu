@@ -322,7 +322,7 @@ __global__ __launch_bounds__(256) void k_noise_g(RoundKeys keys, uint32_t t_off,
   fill_sincos_table(tab, 1.0f);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = blockIdx.x;
-  const int64_t blk = (int64_t)blockIdx.y * 8 + warp;
+  const int64_t blk = (int64_t)blockIdx.y * (blockDim.x >> 5) + warp;
   const uint32_t t_abs = t_off + (uint32_t)t;
   const BlockConst bc = block_const(keys, slot_ctr0((uint32_t)blk, (uint32_t)lane), ctr3);
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -353,6 +353,18 @@ __global__ __launch_bounds__(256) void k_noise_g(RoundKeys keys, uint32_t t_off,
 }
 
 }  // namespace
+
+// k_noise_g geometry: one warp per 128-channel block, at most 8 warps per CTA
+// and no idle warps when the width has fewer than 8 blocks.
+struct NoiseGGeom {
+  dim3 grid;
+  unsigned threads;
+};
+static NoiseGGeom noise_g_geom(int64_t T, int64_t width) {
+  const int64_t nblk = (width + 127) / 128;
+  const int64_t warps = nblk < 8 ? nblk : 8;
+  return {dim3((unsigned)T, (unsigned)((nblk + warps - 1) / warps)), (unsigned)(32 * warps)};
+}
 
 cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const float* u, int64_t t0,
                                int64_t nt, __nv_bfloat16* da, bool round_bf16, float* da_f32) {
@@ -396,9 +408,9 @@ cudaError_t launch_gelu_delta_rows(cudaStream_t st, const dust_params& p, const 
 
 cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const float* r,
                                   float* g_out, __nv_bfloat16* gop, int tag) {
-  dim3 grid((unsigned)p.T, (unsigned)((p.d + 1023) / 1024));
+  const NoiseGGeom gg = noise_g_geom(p.T, p.d);
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
-  k_noise_g<__nv_bfloat16><<<grid, 256, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
+  k_noise_g<__nv_bfloat16><<<gg.grid, gg.threads, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
       (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.d, p.K, r, g_out, gop,
       p.T * p.d);
   return cudaGetLastError();
@@ -406,9 +418,9 @@ cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const f
 
 cudaError_t launch_noise_g_f32(cudaStream_t st, const dust_params& p, const float* r,
                               float* g_out, float* gop, int tag) {
-  dim3 grid((unsigned)p.T, (unsigned)((p.d + 1023) / 1024));
+  const NoiseGGeom gg = noise_g_geom(p.T, p.d);
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
-  k_noise_g<float><<<grid, 256, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
+  k_noise_g<float><<<gg.grid, gg.threads, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
       (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.d, p.K, r, g_out, gop, 0);
   return cudaGetLastError();
 }
@@ -445,16 +457,16 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
 cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
                          void* gop, bool down) {
   const int64_t width = down ? p.d : p.d_ff;
-  dim3 grid((unsigned)p.T, (unsigned)((width + 1023) / 1024));
+  const NoiseGGeom gg = noise_g_geom(p.T, width);
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
   const RoundKeys keys = round_keys(p.seed);
   const uint32_t c3 = ctr3_of(down ? kTagMlpDown : kTagMlpUp, p.stream_id);
   const int64_t plane = p.T * width;
   if (p.dtype == DUST_BF16 && !down)
-    k_noise_g<__nv_bfloat16><<<grid, 256, 0, st>>>(keys, (uint32_t)p.token_offset,
+    k_noise_g<__nv_bfloat16><<<gg.grid, gg.threads, 0, st>>>(keys, (uint32_t)p.token_offset,
         (uint32_t)p.draw_offset, c3, scale, width, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
   else
-    k_noise_g<float><<<grid, 256, 0, st>>>(keys, (uint32_t)p.token_offset,
+    k_noise_g<float><<<gg.grid, gg.threads, 0, st>>>(keys, (uint32_t)p.token_offset,
         (uint32_t)p.draw_offset, c3, scale, width, p.K, r, g_out, (float*)gop, plane);
   return cudaGetLastError();
 }
