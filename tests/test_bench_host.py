@@ -1,0 +1,67 @@
+"""Host-side pieces of bench.py (no GPU): the roofline arithmetic, the
+workload block of the JSON line and the oracle CPU baseline."""
+import math
+
+import bench
+import synth
+
+PEAKS = {"sm_max_mhz": 1965.0, "bf16_tflops": 1640.9, "bf16_tflops_sustained": 1416.7}
+
+
+def test_subset_roofline_counts_elements_and_lanes():
+    wl = synth.CONFIGS["large_subset_bf16"]
+    r = bench._alu_roofline(wl, 176.7, PEAKS)
+    elems = wl.T * wl.K * (wl.S + 1)
+    assert r["elements"] == elems
+    assert math.isclose(r["achieved"], elems * 20 / 0.1767 / 1e12, rel_tol=1e-12)
+    assert math.isclose(r["peak"], 148 * 128 * 1965e6 / 1e12, rel_tol=1e-12)
+    assert math.isclose(r["frac"], r["achieved"] / r["peak"], rel_tol=1e-12)
+    assert r["bound"] == "alu" and 0.3 < r["frac"] < 0.6
+
+
+def test_attention_roofline_splits_tensor_and_cuda_core_work():
+    for name, rows_expected in (("attn_q_bf16", True), ("attn_k_bf16", True),
+                                ("attn_v_bf16", False)):
+        wl = synth.CONFIGS[name]
+        r = bench._attn_roofline(wl, 10.0, PEAKS)
+        L, H, dh = wl.seq_len, wl.n_heads, wl.head_dim
+        rows = (wl.T // L) * L * (L + 1) // 2 if rows_expected else 0
+        ops = wl.K * H * (rows * bench.ATTN_OPS_PER_ROW + wl.T * dh * bench.ATTN_OPS_PER_NOISE)
+        assert r["ops"] == ops
+        assert math.isclose(r["achieved"], ops / 0.01 / 1e12, rel_tol=1e-12)
+        if rows_expected:
+            assert r["tensor"]["flops"] == 6 * dh * wl.K * H * rows
+        else:
+            assert "tensor" not in r
+
+
+def test_mlp_roofline_flops():
+    for name in ("mlp_bf16", "mlp_down_bf16", "attn_out_bf16"):
+        wl = synth.CONFIGS[name]
+        r = bench._mlp_roofline(wl, 300.0, PEAKS)
+        d, dff, V = wl.d, wl.d_ff, wl.V
+        per_row = 2 * (2 * d) * V
+        if name != "mlp_down_bf16":
+            per_row += 2 * (2 * dff) * d
+        if name == "attn_out_bf16":
+            per_row += 2 * (2 * d) * dff
+        assert math.isclose(r["flops"], per_row * wl.T * wl.K, rel_tol=1e-12)
+        assert r["bound"] == "tensor" and r["peak"] == PEAKS["bf16_tflops_sustained"]
+
+
+def test_config_block():
+    class Args:
+        config = "attn_q_bf16"
+    cfg = bench._config(Args, synth.CONFIGS["attn_q_bf16"], 1, "flushed")
+    assert cfg["workload"] == "attn_q_bf16" and cfg["parallelism"] == "dp1"
+    assert (cfg["seq_len"], cfg["n_heads"], cfg["head_dim"]) == (1024, 12, 64)
+    Args.config = "large_subset_bf16"
+    cfg = bench._config(Args, synth.CONFIGS["large_subset_bf16"], 2, "flushed")
+    assert "seq_len" not in cfg and cfg["parallelism"].startswith("dp2")
+    assert (cfg["T_per_gpu"], cfg["K"], cfg["S"]) == (16384, 16384, 512)
+
+
+def test_cpu_baseline_on_a_small_sample():
+    cb = bench.cpu_baseline("tiny_fp32", budget_tokens=2)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert "2 tokens x all 16 draws of tiny_fp32" in cb["sample"]
