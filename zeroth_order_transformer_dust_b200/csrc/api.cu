@@ -760,9 +760,6 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
   float* O = (float*)ctx->attn_o.p;
   float* lse = (float*)ctx->attn_lse.p;
   float* gb = (float*)ctx->attn_gb.p;
-  DUST_CU(launch_attn_fwd(st, T, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse, gb));
-  ctx->launches += 1;
-  mark(ctx, "attn_fwd");
   // query and key draws on tensor cores (d_h 64 or 128) unless DUST_ATTN_TC=0
   const char* tc_env = getenv("DUST_ATTN_TC");
   const bool use_tc = a.which != DUST_ATTN_V && a.head_dim >= 64 &&
@@ -772,12 +769,17 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
     DUST_TRY(ensure(ctx, ctx->attn_tcr, attn_tc_rows_bytes(T, a.seq_len, (int)H, a.head_dim)));
     DUST_TRY(ensure(ctx, ctx->attn_coef, attn_coef_bytes(T, a.seq_len, (int)H)));
   }
+  // the clean pass also writes the query-noise coefficient rows
+  float2* qcoef = use_tc && a.which == DUST_ATTN_Q ? (float2*)ctx->attn_coef.p : nullptr;
+  DUST_CU(launch_attn_fwd(st, T, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse, gb, qcoef));
+  ctx->launches += 1;
+  mark(ctx, "attn_fwd");
   DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
                             gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r, use_tc,
                             (uint8_t*)ctx->attn_tcr.p, (float2*)ctx->attn_coef.p, ctx->d_status));
-  // value: column sums + draws; tensor cores: coefficients, row conversion,
-  // draws, head sum; CUDA cores: draws, head sum
-  ctx->launches += use_tc ? 4 : 2;
+  // value: column sums + draws; tensor cores: (key) coefficients, row
+  // conversion, draws, head sum; CUDA cores: draws, head sum
+  ctx->launches += use_tc ? (a.which == DUST_ATTN_K ? 4 : 3) : 2;
   mark(ctx, "draws");
   dust_params pg = p;
   pg.d = Dw;  // the noise width

@@ -274,7 +274,7 @@ size_t attn_draws_smem(int L, int head_dim);
 size_t attn_tc_smem(int L, int head_dim);  // the tensor-core query/key draws (d_h 64, 128)
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
                             const float* Q, const float* Kc, const float* Vc, const float* E,
-                            float* O, float* lse, float* gbar);
+                            float* O, float* lse, float* gbar, float2* qcoef);
 cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,

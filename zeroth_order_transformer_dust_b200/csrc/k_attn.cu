@@ -110,6 +110,7 @@ struct FwdArgs {
   int64_t T;
   int32_t L, H;
   float scale;
+  float2* qcoef;  // optional: (a_s,tau, a_s,tau <v_tau, e_s>) rows for query noise
 };
 
 // One CTA per (sequence, head, block of kFwdWarps rows), one warp per query
@@ -135,12 +136,16 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_consta
   const int n = row_ok ? pos + 1 : 0;         // keys this row attends to
   const int nmax = min(A.L, (rb + 1) * kFwdWarps);  // keys any row of the CTA needs
   const int Lp = (A.L + 3) & ~3;
-  float* pr = fsm + (size_t)warp * (Lp + DH);
+  float* pr = fsm + (size_t)warp * (Lp + 2 * DH);
   float* qs = pr + Lp;
-  float* tile = fsm + (size_t)kFwdWarps * (Lp + DH);
+  float* es = qs + DH;
+  float* tile = fsm + (size_t)kFwdWarps * (Lp + 2 * DH);
   const int64_t t = s0 + pos;
   if (row_ok)
-    for (int c = lane; c < DH; c += 32) qs[c] = A.Q[t * D + h * DH + c];
+    for (int c = lane; c < DH; c += 32) {
+      qs[c] = A.Q[t * D + h * DH + c];
+      es[c] = A.E[t * D + h * DH + c];
+    }
   // pass 1: scores against staged key tiles
   float m = -INFINITY;
   for (int j0 = 0; j0 < nmax; j0 += kTile) {
@@ -182,6 +187,20 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_consta
       const float a = pr[j0 + j];
 #pragma unroll
       for (int u = 0; u < DH / 32; ++u) o[u] = fmaf(a, tile[j * kStride + lane + 32 * u], o[u]);
+    }
+    if (A.qcoef && row_ok) {
+      // the query-noise coefficient row: (a, a <v, e_s>) up to the tile
+      // boundary, zero past the causal limit (<o_s, e_s> is taken off later)
+      const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
+      float2* crow = A.qcoef + (t * A.H + h) * (int64_t)Lt + j0;
+      for (int j = lane; j < kTile; j += 32) {
+        float2 v = make_float2(0.f, 0.f);
+        if (j < lim) {
+          const float a = pr[j0 + j];
+          v = make_float2(a, a * dot_row<DH>(es, tile + j * kStride));
+        }
+        crow[j] = v;
+      }
     }
   }
   if (!row_ok) return;  // after the last block barrier
@@ -374,8 +393,9 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
 // Per-row coefficients of the query and key draws, for every (token s, head
 // h) at once: row (s, h) of C holds, at column c of s's sequence (c < the
 // sequence length rounded up to 64; zero where the row does not reach),
-//   query noise: (a_s,c, a_s,c (<v_c, e_s> - gbar_s))   for c <= pos(s),
-//   key noise:   (a_c,s, <v_s, e_c> - gbar_c)           for c >= pos(s).
+//   query noise: (a_s,c, a_s,c <v_c, e_s>)   for c <= pos(s) (the draws take
+//                <o_s, e_s> off; the clean pass writes these rows itself),
+//   key noise:   (a_c,s, <v_s, e_c> - gbar_c)  for c >= pos(s).
 // One CTA per (sequence, head, block of kFwdWarps rows s), one warp per s;
 // the streamed rows (keys and values, or queries and errors) are staged in
 // shared-memory tiles (row stride d_h + 4) shared by the CTA's warps, each
@@ -408,7 +428,6 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_coef(const __grid_const
       own[DH + c] = WHICH == 0 ? A.E[so + c] : A.Vc[so + c];
     }
   const float lse_s = ok ? A.lse[(s0 + pos) * A.H + h] : 0.f;
-  const float gb_s = ok ? A.gbar[(s0 + pos) * A.H + h] : 0.f;
   // columns: query noise needs [0, pos] of each row, key noise [pos, L), both
   // padded to whole 64-column tiles
   const int c_lo = WHICH == 0 ? 0 : rb * kFwdWarps / kTcRows * kTcRows;
@@ -439,7 +458,7 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_coef(const __grid_const
         if (c < A.L && (WHICH == 0 ? c <= pos : c >= pos)) {
           if (WHICH == 0) {
             const float a = expf(dot_row<DH>(own, t1 + j * kStride) * A.scale - lse_s);
-            v = make_float2(a, a * (dot_row<DH>(own + DH, t2 + j * kStride) - gb_s));
+            v = make_float2(a, a * dot_row<DH>(own + DH, t2 + j * kStride));
           } else {
             const float a = expf(dot_row<DH>(own, t1 + j * kStride) * A.scale - lt[j]);
             v = make_float2(a, dot_row<DH>(own + DH, t2 + j * kStride) - gt[j]);
@@ -723,6 +742,7 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
   const int mh = warp >> 2, quad = warp & 3;
   const uint32_t tlane = (uint32_t)(quad * 32) << 16;
   const uint32_t t_abs = A.t_off + (uint32_t)s;
+  const float gb_s = WHICH == 0 ? A.gbar[s * A.H + h] : 0.f;  // <o_s, e_s>
   volatile int* abort = &abort_flag;
   // parities of the next completion of full/done/empty[b] (bit b); uses of
   // each TMEM buffer so far (its first use needs no empty wait)
@@ -816,7 +836,8 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
       if (tid == 0 && j + 2 < ntiles) copy_tile(j + 2);
     }
     if (!*abort && i0 + tid < A.K)
-      A.part[(int64_t)blockIdx.x * A.K + i0 + tid] = WHICH == 0 ? -acc1 / (1.0f + acc0) : -acc1;
+      A.part[(int64_t)blockIdx.x * A.K + i0 + tid] =
+          WHICH == 0 ? -fmaf(-gb_s, acc0, acc1) / (1.0f + acc0) : -acc1;
     ptx::tc_fence_before();
     __syncthreads();  // every epilogue of the round is done before the next round's noise
     ptx::tc_fence_after();
@@ -997,7 +1018,7 @@ cudaError_t colsum_dh(cudaStream_t st, const FwdArgs& A, float* W) {
 }  // namespace
 
 size_t attn_fwd_smem(int L, int head_dim) {
-  return ((size_t)kFwdWarps * (((L + 3) & ~3) + head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
+  return ((size_t)kFwdWarps * (((L + 3) & ~3) + 2 * head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
 }
 size_t attn_coef_smem(int head_dim) {
   return ((size_t)2 * kTile * (head_dim + 4) + 2 * kTile + (size_t)kFwdWarps * 2 * head_dim) * 4;
@@ -1016,8 +1037,8 @@ size_t attn_draws_smem(int L, int head_dim) {
 
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
                             const float* Q, const float* Kc, const float* Vc, const float* E,
-                            float* O, float* lse, float* gbar) {
-  FwdArgs A{Q, Kc, Vc, E, O, lse, gbar, T, L, H, 1.0f / sqrtf((float)head_dim)};
+                            float* O, float* lse, float* gbar, float2* qcoef) {
+  FwdArgs A{Q, Kc, Vc, E, O, lse, gbar, T, L, H, 1.0f / sqrtf((float)head_dim), qcoef};
   if (head_dim == 32) return fwd_dh<32>(st, A);
   if (head_dim == 64) return fwd_dh<64>(st, A);
   return fwd_dh<128>(st, A);
@@ -1033,7 +1054,7 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
   const uint32_t ctr3 = ctr3_of(kTagAttnQ + which, p.stream_id);
   if (which == 2) {
     // value noise: w_s once, then one D-long dot per draw (rewards go to r)
-    FwdArgs F{Q, Kc, Vc, E, nullptr, const_cast<float*>(lse), nullptr, p.T, L, H, c};
+    FwdArgs F{Q, Kc, Vc, E, nullptr, const_cast<float*>(lse), nullptr, p.T, L, H, c, nullptr};
     cudaError_t e = head_dim == 32 ? colsum_dh<32>(st, F, W)
                     : head_dim == 64 ? colsum_dh<64>(st, F, W) : colsum_dh<128>(st, F, W);
     if (e != cudaSuccess) return e;
@@ -1061,15 +1082,14 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
       k_attn_tc_rows<128><<<units, kDrawThreads, 0, st>>>(rsrc, p.T, L, H, tc_rows, status);
     {
       FwdArgs F{Q, Kc, Vc, E, nullptr, const_cast<float*>(lse), const_cast<float*>(gbar), p.T, L,
-                H, c};
+                H, c, nullptr};
       const size_t csm = attn_coef_smem(head_dim);
       const unsigned cblocks = (unsigned)((p.T / L) * H * ((L + kFwdWarps - 1) / kFwdWarps));
-      cudaError_t ce;
-      if (head_dim == 64)
-        ce = which == 0 ? coef_dh<0, 64>(st, F, coef, csm, cblocks) : coef_dh<1, 64>(st, F, coef, csm, cblocks);
-      else
-        ce = which == 0 ? coef_dh<0, 128>(st, F, coef, csm, cblocks)
-                        : coef_dh<1, 128>(st, F, coef, csm, cblocks);
+      // query noise: the clean pass wrote the rows (launch_attn_fwd's qcoef)
+      cudaError_t ce = cudaSuccess;
+      if (which == 1)
+        ce = head_dim == 64 ? coef_dh<1, 64>(st, F, coef, csm, cblocks)
+                            : coef_dh<1, 128>(st, F, coef, csm, cblocks);
       if (ce != cudaSuccess) return ce;
     }
     TcDrawArgs T{Q, Kc, Vc, E, lse, gbar, part, tc_rows, coef, round_keys(p.seed),
