@@ -390,20 +390,17 @@ __global__ __launch_bounds__(kDrawThreads, DH <= 64 ? 2 : 1) void k_attn_draws(c
   }
 }
 
-// Per-row coefficients of the query and key draws, for every (token s, head
-// h) at once: row (s, h) of C holds, at column c of s's sequence (c < the
-// sequence length rounded up to 64; zero where the row does not reach),
-//   query noise: (a_s,c, a_s,c <v_c, e_s>)   for c <= pos(s) (the draws take
-//                <o_s, e_s> off; the clean pass writes these rows itself),
-//   key noise:   (a_c,s, <v_s, e_c> - gbar_c)  for c >= pos(s).
-// One CTA per (sequence, head, block of kFwdWarps rows s), one warp per s;
-// the streamed rows (keys and values, or queries and errors) are staged in
-// shared-memory tiles (row stride d_h + 4) shared by the CTA's warps, each
-// lane takes tile rows lane and lane + 32, and the row's writes are
-// coalesced float2 stores.
-template <int WHICH, int DH>
-__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_coef(const __grid_constant__ FwdArgs A,
-                                                             float2* __restrict__ C) {
+// Per-row coefficients of the key draws, for every (token s, head h) at
+// once: row (s, h) of C holds, at column c of s's sequence (c < the sequence
+// length rounded up to 64), (a_c,s, <v_s, e_c> - gbar_c) for c >= pos(s) and
+// zero before (the query draws' rows come from the clean pass). One CTA per
+// (sequence, head, block of kFwdWarps key positions s), one warp per s; the
+// later queries and their error rows are staged in shared-memory tiles (row
+// stride d_h + 4) shared by the CTA's warps, each lane takes tile rows lane
+// and lane + 32, and the row's writes are coalesced float2 stores.
+template <int DH>
+__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_kcoef(const __grid_constant__ FwdArgs A,
+                                                              float2* __restrict__ C) {
   extern __shared__ __align__(16) float qsm[];
   constexpr int kStride = DH + 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -416,53 +413,43 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_coef(const __grid_const
   const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
   const int pos = rb * kFwdWarps + warp;
   const bool ok = pos < A.L;
-  float* t1 = qsm;                          // keys (query) / queries (key)
-  float* t2 = t1 + kTile * kStride;         // values (query) / errors (key)
-  float* lt = t2 + kTile * kStride;         // per tile row: LSE and gbar (key)
-  float* gt = lt + kTile;
-  float* own = gt + kTile + (size_t)warp * 2 * DH;  // q_s, e_s (query) / k_s, v_s (key)
+  float* tq = qsm;                          // queries of the tile rows
+  float* te = tq + kTile * kStride;         // their error signals
+  float* lt = te + kTile * kStride;         // their LSE
+  float* gt = lt + kTile;                   // and <o, e>
+  float* own = gt + kTile + (size_t)warp * 2 * DH;  // k_s, v_s
   const int64_t so = (s0 + pos) * D + h * DH;
   if (ok)
     for (int c = lane; c < DH; c += 32) {
-      own[c] = WHICH == 0 ? A.Q[so + c] : A.Kc[so + c];
-      own[DH + c] = WHICH == 0 ? A.E[so + c] : A.Vc[so + c];
+      own[c] = A.Kc[so + c];
+      own[DH + c] = A.Vc[so + c];
     }
-  const float lse_s = ok ? A.lse[(s0 + pos) * A.H + h] : 0.f;
-  // columns: query noise needs [0, pos] of each row, key noise [pos, L), both
-  // padded to whole 64-column tiles
-  const int c_lo = WHICH == 0 ? 0 : rb * kFwdWarps / kTcRows * kTcRows;
-  const int c_hi = WHICH == 0 ? min(Lt, ((rb + 1) * kFwdWarps + kTcRows - 1) / kTcRows * kTcRows)
-                              : Lt;
+  // columns [pos, L) of each row, from the block's first whole tile
+  const int c_lo = rb * kFwdWarps / kTcRows * kTcRows;
   float2* crow = C + ((s0 + pos) * A.H + h) * (int64_t)Lt;
-  for (int j0 = c_lo; j0 < c_hi; j0 += kTile) {
+  for (int j0 = c_lo; j0 < Lt; j0 += kTile) {
     const int rows = min(kTile, A.L - j0);  // rows past the sequence end stay unread
     __syncthreads();
-    for (int e = threadIdx.x; e < max(rows, 0) * (DH / 4); e += kFwdWarps * 32) {
+    for (int e = threadIdx.x; e < rows * (DH / 4); e += kFwdWarps * 32) {
       const int r = e / (DH / 4), c4 = e % (DH / 4);
       const int64_t src = (s0 + j0 + r) * D + h * DH;
-      *reinterpret_cast<float4*>(t1 + r * kStride + 4 * c4) =
-          reinterpret_cast<const float4*>(WHICH == 0 ? A.Kc + src : A.Q + src)[c4];
-      *reinterpret_cast<float4*>(t2 + r * kStride + 4 * c4) =
-          reinterpret_cast<const float4*>(WHICH == 0 ? A.Vc + src : A.E + src)[c4];
+      *reinterpret_cast<float4*>(tq + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(A.Q + src)[c4];
+      *reinterpret_cast<float4*>(te + r * kStride + 4 * c4) =
+          reinterpret_cast<const float4*>(A.E + src)[c4];
     }
-    if (WHICH == 1)
-      for (int r = threadIdx.x; r < rows; r += kFwdWarps * 32) {
-        lt[r] = A.lse[(s0 + j0 + r) * A.H + h];
-        gt[r] = A.gbar[(s0 + j0 + r) * A.H + h];
-      }
+    for (int r = threadIdx.x; r < rows; r += kFwdWarps * 32) {
+      lt[r] = A.lse[(s0 + j0 + r) * A.H + h];
+      gt[r] = A.gbar[(s0 + j0 + r) * A.H + h];
+    }
     __syncthreads();
     if (ok) {
       for (int j = lane; j < kTile; j += 32) {
         const int c = j0 + j;
         float2 v = make_float2(0.f, 0.f);
-        if (c < A.L && (WHICH == 0 ? c <= pos : c >= pos)) {
-          if (WHICH == 0) {
-            const float a = expf(dot_row<DH>(own, t1 + j * kStride) * A.scale - lse_s);
-            v = make_float2(a, a * dot_row<DH>(own + DH, t2 + j * kStride));
-          } else {
-            const float a = expf(dot_row<DH>(own, t1 + j * kStride) * A.scale - lt[j]);
-            v = make_float2(a, dot_row<DH>(own + DH, t2 + j * kStride) - gt[j]);
-          }
+        if (c < A.L && c >= pos) {
+          const float a = expf(dot_row<DH>(own, tq + j * kStride) * A.scale - lt[j]);
+          v = make_float2(a, dot_row<DH>(own + DH, te + j * kStride) - gt[j]);
         }
         crow[c] = v;
       }
@@ -492,22 +479,16 @@ constexpr int kTcTmemCols = 256;    // 2 buffers x 2 halves of the draws x 64 co
 constexpr uint64_t kTcWaitNs = 2000000000ull;
 
 struct TcDrawArgs {
-  const float* Q;
-  const float* Kc;
-  const float* Vc;
-  const float* E;
-  const float* lse;
-  const float* gbar;
+  const float* gbar;    // <o, e> per (token, head)
   float* part;
   const uint8_t* rows;  // the streamed rows, converted (k_attn_tc_rows)
-  const float2* coef;   // the per-row coefficients (k_attn_coef), rows of Lt
+  const float2* coef;   // the per-row coefficients, rows of Lt
   RoundKeys keys;
   uint32_t t_off, i_off, ctr3;
   float xscale;  // sigma c S: the noise's factor
   float inv_s;   // 1 / S
   int64_t T;
   int32_t L, H, K;
-  float scale;
   uint32_t* status;
 };
 
@@ -985,12 +966,12 @@ cudaError_t draws_which(cudaStream_t st, int which, const DrawArgs& A) {
   return draws_dh<1, DH>(st, A);
 }
 
-template <int WHICH, int DH>
-cudaError_t coef_dh(cudaStream_t st, const FwdArgs& F, float2* C, size_t smem, unsigned blocks) {
-  cudaError_t e = cudaFuncSetAttribute(k_attn_coef<WHICH, DH>,
+template <int DH>
+cudaError_t kcoef_dh(cudaStream_t st, const FwdArgs& F, float2* C, size_t smem, unsigned blocks) {
+  cudaError_t e = cudaFuncSetAttribute(k_attn_kcoef<DH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_attn_coef<WHICH, DH><<<blocks, kFwdWarps * 32, smem, st>>>(F, C);
+  k_attn_kcoef<DH><<<blocks, kFwdWarps * 32, smem, st>>>(F, C);
   return cudaGetLastError();
 }
 
@@ -1088,13 +1069,13 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
       // query noise: the clean pass wrote the rows (launch_attn_fwd's qcoef)
       cudaError_t ce = cudaSuccess;
       if (which == 1)
-        ce = head_dim == 64 ? coef_dh<1, 64>(st, F, coef, csm, cblocks)
-                            : coef_dh<1, 128>(st, F, coef, csm, cblocks);
+        ce = head_dim == 64 ? kcoef_dh<64>(st, F, coef, csm, cblocks)
+                            : kcoef_dh<128>(st, F, coef, csm, cblocks);
       if (ce != cudaSuccess) return ce;
     }
-    TcDrawArgs T{Q, Kc, Vc, E, lse, gbar, part, tc_rows, coef, round_keys(p.seed),
-                 (uint32_t)p.token_offset, (uint32_t)p.draw_offset, ctr3, p.sigma * c * S,
-                 1.0f / S, p.T, L, H, p.K, c, status};
+    TcDrawArgs T{gbar, part, tc_rows, coef, round_keys(p.seed), (uint32_t)p.token_offset,
+                 (uint32_t)p.draw_offset, ctr3, p.sigma * c * S, 1.0f / S, p.T, L, H, p.K,
+                 status};
     cudaError_t e = head_dim == 64 ? (which == 0 ? draws_tc<0, 64>(st, T) : draws_tc<1, 64>(st, T))
                                    : (which == 0 ? draws_tc<0, 128>(st, T) : draws_tc<1, 128>(st, T));
     if (e != cudaSuccess) return e;
