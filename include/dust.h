@@ -233,9 +233,14 @@ dust_status dust_attn_out_grad(dust_ctx* ctx, const dust_params* p,
  *   rewards_out T x K fp32 (or NULL);  g_out T x D fp32 (or NULL)
  * All pointers are device pointers, row-major; inputs 16-byte aligned,
  * outputs 4-byte. The noise's counter tag is 5, 6 or 7 (query, key, value).
+ * Query and key noise with head_dim 64 or 128 runs its dot products on the
+ * tensor cores in fp16 hi/lo parts (about fp32 accuracy); the environment
+ * variable DUST_ATTN_TC=0 selects the CUDA-core form instead.
  * Errors: DUST_ERR_ARG for bad parameters, shape or pointers;
  * DUST_ERR_UNSUPPORTED when seq_len needs more shared memory than the device
- * has; DUST_ERR_CUDA / DUST_ERR_OOM as elsewhere.
+ * has, or (reported at the end of the call) when a query or key value lies
+ * beyond +-32768 on the tensor-core form; DUST_ERR_CUDA / DUST_ERR_OOM as
+ * elsewhere.
  */
 enum { DUST_ATTN_Q = 0, DUST_ATTN_K = 1, DUST_ATTN_V = 2 };
 typedef struct dust_attn_shape {
