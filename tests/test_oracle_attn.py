@@ -13,7 +13,9 @@ The oracle is checked against things other than itself:
   <eps, e_t> with the clean probabilities, at any sigma;
 * one-token sequences: q and k noise cannot move a softmax over one key;
 * convergence of g to the autograd gradient as K grows;
-* G = sum_s g_s x_s^T as an explicit loop.
+* G = sum_s g_s x_s^T as an explicit loop;
+* the per-head closed forms the draw kernels evaluate (query, key, value)
+  agree with the recompute to rounding at small and large sigma.
 """
 
 import numpy as np
@@ -171,3 +173,45 @@ def test_sequences_are_independent_and_offsets_compose():
     second = oracle.attn_grad(x["X"][6:], x["Q"][6:], x["K"][6:], x["V"][6:], x["E"][6:], 6, 2,
                               "q", prm2)
     assert np.array_equal(both["rewards"][6:], second["rewards"])
+
+
+def test_closed_forms_of_the_kernels_equal_the_recompute():
+    # The draw kernels never recompute a perturbed softmax: per head they use
+    #   query: r_h = -sum_tau a expm1(d_tau) (<v_tau, e_s> - gbar_s)
+    #                 / (1 + sum_tau a expm1(d_tau)),  d_tau = sigma eps.k_tau / sqrt(d_h)
+    #   key:   r_h = -sum_{t>=s} u_t / (1 + u_t) (<v_s, e_t> - gbar_t),
+    #          u_t = a_t,s expm1(sigma eps.q_t / sqrt(d_h))
+    #   value: r_h = -sigma eps . sum_{t>=s} a_t,s e_t
+    # with a the clean probabilities and gbar_t = <o_t, e_t> per head. These
+    # are exact rewrites, so they match the oracle's recompute to rounding at
+    # any sigma.
+    L, H, dh = 7, 2, 4
+    x = _inputs(T=L, L=L, H=H, dh=dh)
+    Q, K, V, E = (x[k].astype(np.float64) for k in ("Q", "K", "V", "E"))
+    O, A = oracle.attention(Q, K, V, L, H)
+    c = 1.0 / np.sqrt(dh)
+    eps = np.random.default_rng(3).standard_normal((5, H * dh))
+    for sig in (0.01, 0.7):
+        for s in (0, 3, 6):
+            for which in ("q", "k", "v"):
+                r_ref, _ = oracle.attn_draws(Q, K, V, O, E, H, s, which, eps, sig)
+                r = np.zeros(len(eps))
+                for h in range(H):
+                    cols = slice(h * dh, (h + 1) * dh)
+                    a = A[0, h]
+                    gbar = (O[:, cols] * E[:, cols]).sum(axis=1)
+                    x_h = sig * eps[:, cols]
+                    if which == "q":
+                        em = np.expm1(c * x_h @ K[: s + 1, cols].T)          # (n, s+1)
+                        gam = V[: s + 1, cols] @ E[s, cols]
+                        D = em @ a[s, : s + 1]
+                        N = em @ (a[s, : s + 1] * (gam - gbar[s]))
+                        r += -N / (1 + D)
+                    elif which == "k":
+                        u = a[s:, s][None, :] * np.expm1(c * x_h @ Q[s:, cols].T)
+                        beta = E[s:, cols] @ V[s, cols] - gbar[s:]
+                        r += -(u / (1 + u)) @ beta
+                    else:
+                        w = a[s:, s] @ E[s:, cols]
+                        r += -(x_h @ w)
+                assert np.allclose(r, r_ref, rtol=1e-10, atol=1e-13), (which, s, sig)
