@@ -29,6 +29,18 @@ def token_shard(T_total: int, world: int, rank: int) -> Tuple[int, int]:
     return start, base + (1 if rank < extra else 0)
 
 
+def sequence_shard(T_total: int, seq_len: int, world: int, rank: int) -> Tuple[int, int]:
+    """(first token, token count) of `rank`'s share when the batch must split
+    at sequence boundaries: the attention-internals estimator couples the
+    tokens of one sequence (noise on a key or value row moves the outputs of
+    every later token of its sequence), so ranks take whole sequences of
+    seq_len tokens, distributed as token_shard distributes tokens."""
+    if seq_len < 1 or T_total % seq_len:
+        raise ValueError("T_total must be a positive multiple of seq_len")
+    first, count = token_shard(T_total // seq_len, world, rank)
+    return first * seq_len, count * seq_len
+
+
 def allreduce_weight_grad(G: torch.Tensor, group: Optional[dist.ProcessGroup] = None) -> torch.Tensor:
     """Sum the per-rank weight-gradient estimates in place (G_W over all tokens)."""
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
@@ -45,6 +57,30 @@ def sharded_head_grad(ctx, H_local: torch.Tensor, W: torch.Tensor, y_local: torc
     with "G" replaced by the all-reduced estimate.
     """
     out = ctx.head_grad(H_local, W, y_local, token_offset=token_offset, **kw)
+    if "G" in out:
+        allreduce_weight_grad(out["G"], group)
+    return out
+
+
+def sharded_mlp_grad(ctx, X_local: torch.Tensor, W_up: torch.Tensor, W_down: torch.Tensor,
+                     W_head: torch.Tensor, y_local: torch.Tensor, token_offset: int,
+                     group: Optional[dist.ProcessGroup] = None, **kw) -> dict:
+    """Hidden-MLP estimator over this rank's tokens (split as token_shard
+    splits them), G_W summed over all ranks."""
+    out = ctx.mlp_grad(X_local, W_up, W_down, W_head, y_local, token_offset=token_offset, **kw)
+    if "G" in out:
+        allreduce_weight_grad(out["G"], group)
+    return out
+
+
+def sharded_attn_grad(ctx, X_local: torch.Tensor, Q_local: torch.Tensor, K_local: torch.Tensor,
+                      V_local: torch.Tensor, E_local: torch.Tensor, token_offset: int,
+                      group: Optional[dist.ProcessGroup] = None, **kw) -> dict:
+    """Attention-internals estimator over this rank's whole sequences (see
+    sequence_shard; token_offset is the rank's first token), G_W summed over
+    all ranks."""
+    out = ctx.attn_grad(X_local, Q_local, K_local, V_local, E_local, token_offset=token_offset,
+                        **kw)
     if "G" in out:
         allreduce_weight_grad(out["G"], group)
     return out
