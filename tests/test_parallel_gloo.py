@@ -190,3 +190,30 @@ def test_sharded_layer_estimators_equal_single_run(kind):
         np.testing.assert_allclose(G, ref["G"], rtol=0, atol=1e-12)
         np.testing.assert_array_equal(rewards, ref["rewards"][t0:t0 + n])
         np.testing.assert_allclose(g, ref["g"][t0:t0 + n], rtol=0, atol=1e-13)
+
+
+def _max_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        q.put((rank, bench._max_over_ranks(10.0 + 5.0 * (rank == 1) - rank * 0.25, world,
+                                           device="cpu")))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_times_the_slowest_rank():
+    # bench.py reports the max over ranks of the per-step time
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_max_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == {0: 14.75, 1: 14.75}
