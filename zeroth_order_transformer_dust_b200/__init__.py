@@ -149,6 +149,82 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}: use float32 or bfloat16")
 
 
+# The C-ABI takes plain pointers and reads every size from its parameters, so
+# the binding checks that each tensor's shape agrees with those sizes: a
+# mismatch would otherwise read or write beyond the tensor.
+def _matrix(t: torch.Tensor, name: str):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return tuple(t.shape)
+
+
+def _shape(t: torch.Tensor, shape, name: str):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_outputs(out: dict, shapes: dict, device: Optional[int]):
+    """Caller-supplied outputs: fp32, contiguous, the expected shape, and on
+    cuda:device (device None: host memory)."""
+    for key, shape in shapes.items():
+        t = out.get(key)
+        if t is None:
+            continue
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"output {key} must be a contiguous fp32 tensor")
+        on_dev = t.is_cuda and t.device.index == device
+        if (device is None and t.is_cuda) or (device is not None and not on_dev):
+            raise ValueError(f"output {key} is on the wrong device")
+        _shape(t, shape, f"output {key}")
+
+
+def _head_shapes(H, W, targets):
+    """(T, d, V) of the LM-head call; raises on inconsistent shapes."""
+    T, d = _matrix(H, "H")
+    V, dw = _matrix(W, "W")
+    if dw != d:
+        raise ValueError(f"W must be V x {d} (H is T x {d}), got {tuple(W.shape)}")
+    _shape(targets, (T,), "targets")
+    return T, d, V
+
+
+def _mlp_shapes(X, W_up, W_down, W_head, targets, O=None):
+    """(T, d, d_ff, V) of the MLP-block call; raises on inconsistent shapes
+    or dtypes (every operand bf16)."""
+    T, d = _matrix(X, "X")
+    d_ff = _matrix(W_up, "W_up")[0]
+    _shape(W_up, (d_ff, d), "W_up")
+    _shape(W_down, (d, d_ff), "W_down")
+    V = _matrix(W_head, "W_head")[0]
+    _shape(W_head, (V, d), "W_head")
+    _shape(targets, (T,), "targets")
+    ops = [(X, "X"), (W_up, "W_up"), (W_down, "W_down"), (W_head, "W_head")]
+    if O is not None:
+        if _matrix(O, "O")[0] != T:
+            raise ValueError(f"O must have {T} rows, got {tuple(O.shape)}")
+        ops.append((O, "O"))
+    for t, n in ops:
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{n} must be bfloat16")
+    if targets.dtype != torch.int32:
+        raise TypeError("targets must be int32")
+    return T, d, d_ff, V
+
+
+def _attn_shapes(X, Q, K_cache, V_cache, E, n_heads):
+    """(T, d, D) of the attention-internals call; raises on inconsistent
+    shapes or dtypes."""
+    T, d = _matrix(X, "X")
+    D = _matrix(Q, "Q")[1]
+    for t, n in ((Q, "Q"), (K_cache, "K_cache"), (V_cache, "V_cache"), (E, "E")):
+        if t.dtype != torch.float32:
+            raise TypeError(f"{n} must be fp32")
+        _shape(t, (T, D), n)
+    if n_heads < 1 or D % n_heads:
+        raise ValueError("the width of Q must be a positive multiple of n_heads")
+    return T, d, D
+
+
 class Context:
     """A library context bound to one CUDA device and (by default) torch's current stream."""
 
@@ -207,14 +283,15 @@ class Context:
             raise TypeError("H and W must share a dtype")
         if targets.dtype != torch.int32:
             raise TypeError("targets must be int32")
-        T, d = H.shape
-        V = W.shape[0]
+        T, d, V = _head_shapes(H, W, targets)
         flags = (FLAG_LITERAL_TARGET_SCALE if literal_target_scale else 0) | (
             FLAG_ASYNC if asynchronous else 0)
         prm = make_params(T, d, V, K, sigma, S=S, dtype=_dtype_code(H), seed=seed,
                           token_offset=token_offset, draw_offset=draw_offset, subset_a=subset_a,
                           stream_id=stream_id, flags=flags)
         out = dict(out or {})
+        _check_outputs(out, {"G": (V, d), "loss": (T,), "rewards": (T, K), "g": (T, V)},
+                       self.device)
         dev = H.device
         f32 = dict(dtype=torch.float32, device=dev)
         if want_G and "G" not in out:
@@ -239,12 +316,16 @@ class Context:
         for t, n in ((H, "H"), (W, "W"), (targets, "targets")):
             if t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{n} must be a contiguous host tensor")
-        T, d = H.shape
-        V = W.shape[0]
+        if H.dtype != W.dtype:
+            raise TypeError("H and W must share a dtype")
+        if targets.dtype != torch.int32:
+            raise TypeError("targets must be int32")
+        T, d, V = _head_shapes(H, W, targets)
         prm = make_params(T, d, V, K, sigma, S=S, dtype=_dtype_code(H), seed=seed,
                           token_offset=token_offset, draw_offset=draw_offset, subset_a=subset_a,
                           stream_id=stream_id)
         out = dict(out or {})
+        _check_outputs(out, {"G": (V, d), "loss": (T,)}, None)
         if want_G and "G" not in out:
             out["G"] = torch.empty(V, d, dtype=torch.float32, pin_memory=True)
         if want_loss and "loss" not in out:
@@ -273,15 +354,15 @@ class Context:
         for t, n in ((X, "X"), (W_up, "W_up"), (W_down, "W_down"), (W_head, "W_head"),
                      (targets, "targets")):
             self._dev(t, n)
-        T, d = X.shape
-        d_ff = W_up.shape[0]
-        V = W_head.shape[0]
+        T, d, d_ff, V = _mlp_shapes(X, W_up, W_down, W_head, targets, O)
         prm = make_params(T, d, V, K, sigma, d_ff=d_ff, dtype=_dtype_code(X), seed=seed,
                           token_offset=token_offset, draw_offset=draw_offset, stream_id=stream_id)
         out = dict(out or {})
         f32 = dict(dtype=torch.float32, device=X.device)
         width = d_ff if layer == "up" else d
         gshape = {"up": (d_ff, d), "down": (d, d_ff)}.get(layer) or (d, O.shape[1])
+        _check_outputs(out, {"G": gshape, "loss": (T,), "rewards": (T, K), "g": (T, width)},
+                       self.device)
         if want_G and "G" not in out:
             out["G"] = torch.empty(*gshape, **f32)
         if want_loss and "loss" not in out:
@@ -316,18 +397,13 @@ class Context:
             raise ValueError("which must be 'q', 'k' or 'v'")
         for t, n in ((X, "X"), (Q, "Q"), (K_cache, "K_cache"), (V_cache, "V_cache"), (E, "E")):
             self._dev(t, n)
-        for t, n in ((Q, "Q"), (K_cache, "K_cache"), (V_cache, "V_cache"), (E, "E")):
-            if t.dtype != torch.float32 or t.shape != Q.shape:
-                raise TypeError(f"{n} must be fp32 with Q's shape")
-        T, d = X.shape
-        D = Q.shape[1]
-        if D % n_heads:
-            raise ValueError("the width of Q must be a multiple of n_heads")
+        T, d, D = _attn_shapes(X, Q, K_cache, V_cache, E, n_heads)
         shape = DustAttnShape(seq_len=seq_len, n_heads=n_heads, head_dim=D // n_heads,
                               which=ATTN_WHICH[which])
         prm = make_params(T, d, 1, K, sigma, dtype=_dtype_code(X), seed=seed,
                           token_offset=token_offset, draw_offset=draw_offset, stream_id=stream_id)
         out = dict(out or {})
+        _check_outputs(out, {"G": (D, d), "rewards": (T, K), "g": (T, D)}, self.device)
         f32 = dict(dtype=torch.float32, device=X.device)
         if want_G and "G" not in out:
             out["G"] = torch.empty(D, d, **f32)
