@@ -163,3 +163,17 @@ def test_attention_call_marshals_sizes(which):
         c.attn_grad(_t(T - 1, d, dtype=bf16), *qkve, seq_len=4, n_heads=H, which=which, K=6,
                     sigma=0.1)
     assert len(_estimator_calls(c)) == 1
+
+
+def test_debug_exports_check_layouts():
+    c = _fake_context()
+    C = c.debug_gemm(_t(3, 16, dtype=bf16), _t(5, 16, dtype=bf16))
+    assert tuple(C.shape) == (3, 5)
+    with pytest.raises(ValueError, match="B must have shape"):
+        c.debug_gemm(_t(3, 16, dtype=bf16), _t(5, 8, dtype=bf16))
+    assert tuple(c.debug_philox(1, _t(7, 4, dtype=torch.int32)).shape) == (7, 4)
+    for bad in (_t(7, 3, dtype=torch.int32), _t(28, dtype=torch.int32), _t(7, 4)):
+        with pytest.raises(ValueError, match="n x 4 int32"):
+            c.debug_philox(1, bad)
+    assert [n for n, _ in c._L.calls if n.startswith("dust_debug")] == [
+        "dust_debug_gemm_bf16", "dust_debug_philox"]

@@ -456,8 +456,9 @@ class Context:
         self._dev(A, "A"), self._dev(B, "B")
         if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
             raise TypeError("A and B must be bfloat16")
-        M, K = A.shape
-        N = B.shape[0]
+        M, K = _matrix(A, "A")
+        N = _matrix(B, "B")[0]
+        _shape(B, (N, K), "B")
         C = torch.empty(M, N, dtype=torch.float32, device=A.device)
         self._bind_stream()
         self._check(self._L.dust_debug_gemm_bf16(self._h, M, N, K, _ptr(A), _ptr(B), _ptr(C), path))
@@ -466,6 +467,8 @@ class Context:
     def debug_philox(self, seed: int, ctr: torch.Tensor) -> torch.Tensor:
         """Raw Philox4x32-10 words for counters ctr (n x 4, int32 storage of uint32)."""
         self._dev(ctr, "ctr")
+        if ctr.dtype != torch.int32 or ctr.dim() != 2 or ctr.shape[1] != 4:
+            raise ValueError("ctr must be an n x 4 int32 tensor")
         out = torch.empty_like(ctr)
         self._bind_stream()
         self._check(self._L.dust_debug_philox(self._h, seed & 0xFFFFFFFFFFFFFFFF, _ptr(ctr),
