@@ -177,3 +177,24 @@ def test_debug_exports_check_layouts():
             c.debug_philox(1, bad)
     assert [n for n, _ in c._L.calls if n.startswith("dust_debug")] == [
         "dust_debug_gemm_bf16", "dust_debug_philox"]
+
+
+def test_training_loop_draw_offsets_and_reduction():
+    # step s of a run resumed at first_step draws at [(first_step + s) K, ...),
+    # the all-reduce hook sees every step's G before its update, and the
+    # update receives the bf16 copy to refresh
+    from zeroth_order_transformer_dust_b200.train import train_head
+    c = _fake_context()
+    c.device = None                     # outputs live in host memory here
+    reduced = []
+    W_lp = _t(30, 8, dtype=bf16)
+    train_head(c, _t(5, 8, dtype=bf16), _t(30, 8), _t(5, dtype=torch.int32), steps=3, lr=0.1,
+               mu=0.9, K=16, sigma=0.01, S=4, seed=2, token_offset=40, W_lp=W_lp, first_step=5,
+               allreduce=lambda G: reduced.append(G.data_ptr()))
+    heads = [a[1]._obj for n, a in c._L.calls if n == "dust_head_grad"]
+    assert [p.draw_offset for p in heads] == [80, 96, 112]
+    assert all((p.token_offset, p.K, p.S, p.seed) == (40, 16, 4, 2) for p in heads)
+    updates = [a for n, a in c._L.calls if n == "dust_sgd_momentum"]
+    assert len(updates) == 3 and len(reduced) == 3
+    assert all(u[7].value == W_lp.data_ptr() for u in updates)
+    assert [n for n, _ in c._L.calls].count("dust_check") == 1
