@@ -26,12 +26,17 @@
  *    invalid call returns DUST_ERR_ARG and launches nothing.
  *  - The context owns its scratch memory (grown on demand, freed by
  *    dust_destroy). A context is not thread-safe; use one per thread.
+ *  - A context belongs to the device given to dust_create. Every call that
+ *    touches the GPU first makes that device current (cudaSetDevice) and
+ *    leaves it current on return; the stream must belong to that device.
  *  - Noise is Philox4x32-10 keyed by (seed, token, draw, slot) and is never
  *    stored: slot k of (token t, draw i) is output word ((k>>5)&3) of counter
  *    (((k>>7)<<5)|(k&31), t+token_offset, i+draw_offset, tag|(stream_id<<8)),
  *    key (seed lo, seed hi), turned into N(0,1) by Box-Muller on 24-bit
  *    uniforms (words 0,1 -> cos, sin; words 2,3 -> cos, sin). Tags: 0 = head
- *    logits, 1 = subset offset, 2 = MLP up-projection.
+ *    logits, 1 = subset offset, 2 = MLP up-projection, 3 = MLP
+ *    down-projection, 4 = attention output projection, 5 / 6 / 7 = query /
+ *    key / value projection.
  */
 #ifndef DUST_H
 #define DUST_H

@@ -302,6 +302,7 @@ const char* dust_last_error(const dust_ctx* ctx) {
 
 dust_status dust_check(dust_ctx* ctx) {
   if (!ctx) return DUST_ERR_ARG;
+  DUST_CU(cudaSetDevice(ctx->device));
   DUST_CU(cudaMemcpyAsync(ctx->h_status, ctx->d_status, sizeof(uint32_t), cudaMemcpyDeviceToHost,
                           ctx->stream));
   DUST_CU(cudaStreamSynchronize(ctx->stream));
