@@ -65,3 +65,40 @@ def test_cpu_baseline_on_a_small_sample():
     cb = bench.cpu_baseline("tiny_fp32", budget_tokens=2)
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
     assert "2 tokens x all 16 draws of tiny_fp32" in cb["sample"]
+
+
+def _run_bench(*args, env=None):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    e = dict(os.environ, **(env or {}))
+    res = subprocess.run([sys.executable, "bench.py", *args], cwd=root, env=e,
+                         capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(s) for s in res.stdout.splitlines() if s.startswith("{")]
+    return lines
+
+
+def test_reference_arm_prints_one_contract_line():
+    # the reference arm times the oracle on the host: one JSON line with the
+    # metric, unit and workload of the product arm, marked impl=reference
+    lines = _run_bench("--impl", "reference", "--steps", "1", "--warmup", "0",
+                       "--config", "tiny_fp32")
+    assert len(lines) == 1
+    ln = lines[0]
+    assert ln["impl"] == "reference" and ln["metric"] == bench.METRIC and ln["unit"] == bench.UNIT
+    assert ln["n_gpus"] == 1 and ln["steps"] == 1 and ln["higher_is_better"] is True
+    assert ln["config"]["workload"] == "tiny_fp32" and ln["value"] > 0
+    cb = ln["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == ln["value"]
+    assert ln["e2e"] == {"value": ln["value"], "unit": ln["unit"], "h2d_bytes_per_step": 0,
+                         "d2h_bytes_per_step": 0}
+    assert ln["ms_per_step"] > 0 and ln["dtype"] == "f64"
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    lines = _run_bench("--impl", "reference", "--steps", "1", "--warmup", "0",
+                       "--config", "tiny_fp32", env={"RANK": "1", "WORLD_SIZE": "2"})
+    assert lines == []
