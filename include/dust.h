@@ -284,12 +284,18 @@ int64_t dust_kernel_launches(const dust_ctx* ctx);
  *     size in `msg`; CUDA-core GEMMs only.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture. The address is kept with the CUDA context
+ *     current at that call: after the device's primary context is destroyed
+ *     and created anew (cudaDeviceReset), the next call looks it up again,
+ *     so make that call outside a capture too.
  *   - Every call shares the array, which keeps the previous call's contents
  *     (each call clears what must start at zero). Calls that overlap on the
  *     GPU, on any stream or thread, race on it: serialise them.
- *   - The call synchronises `cuda_stream` to read the device status word.
- * Errors as dust_head_grad, with the reason in `msg` (may be NULL).
+ *   - The call synchronises `cuda_stream` to read the device status word
+ *     (DUST_FLAG_ASYNC in p->flags is ignored).
+ * Errors as dust_head_grad, with the reason in `msg` (may be NULL): invalid
+ * parameters, NULL inputs, H or W not 16-byte aligned or another pointer not
+ * 4-byte aligned return DUST_ERR_ARG before any CUDA call.
  */
 dust_status dust_head_grad_noalloc(const dust_params* p, void* cuda_stream,
                                    const void* H, const void* W, const int32_t* targets,

@@ -112,3 +112,37 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
             dust.load_library(str(tmp_path / "nope.so"))
         finally:
             dust._lib = dust._lib_saved
+
+
+def _noalloc(lib):
+    fn = lib.dust_head_grad_noalloc
+    fn.restype = ctypes.c_int32
+    fn.argtypes = ([ctypes.POINTER(dust.DustParams), ctypes.c_void_p] + [ctypes.c_void_p] * 7
+                   + [ctypes.c_char_p, ctypes.c_int])
+    return fn
+
+
+@pytest.mark.parametrize("bad", ["H", "W", "targets", "G", "loss", "rewards", "g"])
+def test_noalloc_rejects_misaligned_pointers_before_any_cuda_call(lib, bad):
+    """The allocation-free entry point checks alignment on the host: the call
+    returns DUST_ERR_ARG without touching a device (none exists here), so the
+    fake addresses below are never dereferenced."""
+    prm = _p(S=10)
+    ptrs = {"H": 0x10000, "W": 0x20000, "targets": 0x30000, "G": 0x40000, "loss": 0x50000,
+            "rewards": 0x60000, "g": 0x70000}
+    ptrs[bad] += 2 if bad in ("H", "W", "targets") else 1
+    if bad in ("H", "W"):
+        ptrs[bad] = ptrs[bad] - 2 + 8          # 8-byte but not 16-byte aligned
+    msg = ctypes.create_string_buffer(256)
+    st = _noalloc(lib)(ctypes.byref(prm), None, *[ctypes.c_void_p(ptrs[k]) for k in
+                       ("H", "W", "targets", "G", "loss", "rewards", "g")], msg, 256)
+    assert st == 1 and b"aligned" in msg.value
+
+
+def test_noalloc_rejects_bad_parameters_on_the_host(lib):
+    msg = ctypes.create_string_buffer(256)
+    p = ctypes.c_void_p(0x10000)
+    st = _noalloc(lib)(ctypes.byref(_p(K=0)), None, p, p, p, p, p, p, p, msg, 256)
+    assert st == 1 and b"K must" in msg.value
+    st = _noalloc(lib)(ctypes.byref(_p()), None, None, p, p, p, p, p, p, msg, 256)
+    assert st == 1 and b"non-NULL" in msg.value

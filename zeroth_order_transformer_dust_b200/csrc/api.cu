@@ -12,6 +12,15 @@
 
 using namespace dust;
 
+namespace dust {
+int64_t default_stride(int64_t V) {
+  int64_t a = (int64_t)std::ceil((double)V * ((std::sqrt(5.0) - 1.0) / 2.0));
+  if (a < 1) a = 1;
+  while (gcd64(a, V) != 1) ++a;
+  return a;
+}
+}  // namespace dust
+
 namespace {
 
 dust_status fail(dust_ctx* ctx, dust_status s, const char* fmt, ...) {
@@ -38,38 +47,6 @@ dust_status fail(dust_ctx* ctx, dust_status s, const char* fmt, ...) {
     dust_status s_ = (expr);      \
     if (s_ != DUST_OK) return s_; \
   } while (0)
-
-int64_t gcd64(int64_t a, int64_t b) {
-  while (b) {
-    const int64_t t = a % b;
-    a = b;
-    b = t;
-  }
-  return a < 0 ? -a : a;
-}
-
-// Inverse of a modulo m (gcd(a, m) = 1), extended Euclid.
-int64_t modinv(int64_t a, int64_t m) {
-  if (m == 1) return 0;
-  int64_t t = 0, nt = 1, r = m, nr = a % m;
-  while (nr != 0) {
-    const int64_t q = r / nr;
-    int64_t tmp = t - q * nt;
-    t = nt;
-    nt = tmp;
-    tmp = r - q * nr;
-    r = nr;
-    nr = tmp;
-  }
-  return t < 0 ? t + m : t;
-}
-
-int64_t default_stride(int64_t V) {
-  int64_t a = (int64_t)std::ceil((double)V * ((std::sqrt(5.0) - 1.0) / 2.0));
-  if (a < 1) a = 1;
-  while (gcd64(a, V) != 1) ++a;
-  return a;
-}
 
 dust_status check_params(const dust_params* p, int variant, char* msg, int msg_len) {
   auto bad = [&](const char* why) {
@@ -236,7 +213,7 @@ dust_status dust_validate(const dust_params* p, int variant, char* msg, int msg_
 
 int64_t dust_subset_stride(const dust_params* p) {
   if (check_params(p, DUST_VARIANT_HEAD, nullptr, 0) != DUST_OK || p->S <= 0) return 0;
-  return p->subset_a ? p->subset_a % p->V : default_stride(p->V);
+  return subset_stride_of(*p);
 }
 
 dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
@@ -331,7 +308,7 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
     return fail(ctx, DUST_ERR_ARG, "H and W must be 16-byte aligned, the other pointers 4-byte");
   DUST_CU(cudaSetDevice(ctx->device));
   const bool subset = p.S > 0;
-  const int64_t a = subset ? (p.subset_a ? p.subset_a % p.V : default_stride(p.V)) : 0;
+  const int64_t a = subset ? subset_stride_of(p) : 0;
   const int64_t a_inv = subset ? modinv(a, p.V) : 0;
   const size_t TV = (size_t)p.T * (size_t)p.V;
   DUST_TRY(ensure(ctx, ctx->z, TV * 4));

@@ -22,6 +22,40 @@ struct Buf {
   size_t bytes = 0;
 };
 
+// Host helpers of the subset rule j_k = (a k + b) mod V, shared by every entry
+// point that draws vocabulary subsets, so all of them pick the same stride.
+inline int64_t gcd64(int64_t a, int64_t b) {
+  while (b) {
+    const int64_t t = a % b;
+    a = b;
+    b = t;
+  }
+  return a < 0 ? -a : a;
+}
+
+// Inverse of a modulo m (gcd(a, m) = 1), extended Euclid.
+inline int64_t modinv(int64_t a, int64_t m) {
+  if (m == 1) return 0;
+  int64_t t = 0, nt = 1, r = m, nr = a % m;
+  while (nr != 0) {
+    const int64_t q = r / nr;
+    int64_t tmp = t - q * nt;
+    t = nt;
+    nt = tmp;
+    tmp = r - q * nr;
+    r = nr;
+    nr = tmp;
+  }
+  return t < 0 ? t + m : t;
+}
+
+// Default stride: the smallest integer >= V (sqrt 5 - 1) / 2 coprime to V.
+int64_t default_stride(int64_t V);
+// The stride a call uses: subset_a mod V when given, else default_stride(V).
+inline int64_t subset_stride_of(const dust_params& p) {
+  return p.subset_a ? p.subset_a % p.V : default_stride(p.V);
+}
+
 // Launch geometry of the GEMMs: A(m, k) and B(n, k) addressing.
 struct GemmDesc {
   int64_t M, N, K;

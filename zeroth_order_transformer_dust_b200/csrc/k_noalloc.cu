@@ -17,6 +17,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "internal.cuh"
 
 namespace dust {
@@ -35,6 +37,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_base[kMaxDevices] = {};
+CUcontext g_ctx[kMaxDevices] = {};
 
 dust_status say(char* msg, int len, dust_status s, const char* fmt, ...) {
   if (msg && len > 0) {
@@ -46,23 +49,50 @@ dust_status say(char* msg, int len, dust_status s, const char* fmt, ...) {
   return s;
 }
 
+// The CUDA context current on this thread (NULL if none), through the
+// runtime's driver entry-point query, so the library needs no link to the
+// driver library itself.
+CUcontext current_context() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;  // guarded by g_mu
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuCtxGetCurrent_v4000)ptr;
+    else
+      cudaGetLastError();
+  }
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
 // Device address of the array on the current device (host code only ever sees
-// a host-side stand-in under its name). Looked up once per device.
+// a host-side stand-in under its name). Looked up once per device and kept
+// with the context that was current then; a call under another context (the
+// device's primary context destroyed by cudaDeviceReset and created anew)
+// looks it up again.
 dust_status scratch_base(int dev, void** out, char* msg, int len) {
   if (dev < 0 || dev >= kMaxDevices) return say(msg, len, DUST_ERR_UNSUPPORTED, "device %d out of range", dev);
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_base[dev]) {
+  CUcontext cur = current_context();
+  if (!g_base[dev] || !cur || cur != g_ctx[dev]) {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || !ptr) {
       cudaGetLastError();
       return say(msg, len, DUST_ERR_CUDA, "cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
     }
+    cur = current_context();
     g_base[dev] = ptr;
+    g_ctx[dev] = cur;
   }
   *out = g_base[dev];
   return DUST_OK;
 }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 struct Carve {
   char* base;
@@ -73,30 +103,6 @@ struct Carve {
     return p;
   }
 };
-
-int64_t gcd64(int64_t a, int64_t b) {
-  while (b) {
-    const int64_t t = a % b;
-    a = b;
-    b = t;
-  }
-  return a < 0 ? -a : a;
-}
-
-int64_t modinv(int64_t a, int64_t m) {
-  if (m == 1) return 0;
-  int64_t t = 0, nt = 1, r = m, nr = a % m;
-  while (nr != 0) {
-    const int64_t q = r / nr;
-    int64_t tmp = t - q * nt;
-    t = nt;
-    nt = tmp;
-    tmp = r - q * nr;
-    r = nr;
-    nr = tmp;
-  }
-  return t < 0 ? t + m : t;
-}
 
 }  // namespace
 
@@ -110,6 +116,9 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   if (v != DUST_OK) return v;
   const dust_params p = *pp;
   if (!H || !W || !targets) return say(msg, msg_len, DUST_ERR_ARG, "H, W and targets must be non-NULL");
+  if (!aligned(H, 16) || !aligned(W, 16) || !aligned(targets, 4) || !aligned(G_out, 4) ||
+      !aligned(loss_out, 4) || !aligned(rewards_out, 4) || !aligned(g_out, 4))
+    return say(msg, msg_len, DUST_ERR_ARG, "H and W must be 16-byte aligned, the other pointers 4-byte");
   const cudaStream_t st = (cudaStream_t)cuda_stream;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -166,17 +175,8 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   void* gop = cv.take(bf16 ? 2 * T * V * 2 : T * V * 4);
   void* xdup = (bf16 && G_out) ? cv.take(2 * T * (size_t)p.d * 2) : nullptr;
 
-  int64_t a = 0, a_inv = 0;
-  if (subset) {
-    if (p.subset_a) {
-      a = p.subset_a % p.V;
-    } else {
-      a = (int64_t)std::ceil((double)p.V * ((std::sqrt(5.0) - 1.0) / 2.0));
-      if (a < 1) a = 1;
-      while (gcd64(a, p.V) != 1) ++a;
-    }
-    a_inv = modinv(a, p.V);
-  }
+  const int64_t a = subset ? subset_stride_of(p) : 0;
+  const int64_t a_inv = subset ? modinv(a, p.V) : 0;
 
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(uint32_t), st);
   GemmDesc g{};
