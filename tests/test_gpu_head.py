@@ -100,6 +100,41 @@ def test_edge_shapes(ctx, kw):
     _compare(got, ref, TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
 
 
+def _host(x, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    t = t.to(torch.int32) if dtype == "i32" else t.to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+    return t.pin_memory()
+
+
+@pytest.mark.parametrize("wl", [synth.CONFIGS["tiny_fp32"], _small(S=100, K=40),
+                                _small(dtype="f32", S=77), _small(T=3, K=20000, S=32)],
+                         ids=["tiny_fp32", "subset_bf16", "subset_f32", "subset_bf16_k20000"])
+def test_host_entry_matches_the_oracle(ctx, wl):
+    """dust_head_grad_host (inputs and outputs in pinned host memory, the copies
+    inside the call): all four outputs against the oracle."""
+    H, W, y = _inputs(wl)
+    out = ctx.head_grad_host(_host(H, wl.dtype), _host(W, wl.dtype), _host(y, "i32"), K=wl.K,
+                             sigma=wl.sigma, S=wl.S, seed=wl.seed, want_rewards=True, want_g=True)
+    assert all(not v.is_cuda for v in out.values())
+    got = {k: v.double().numpy() for k, v in out.items()}
+    _compare(got, _oracle(H, W, y, wl), TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
+    # and the same bits as the device-buffer entry point on the same inputs
+    dev = _gpu(ctx, H, W, y, wl)
+    np.testing.assert_array_equal(got["rewards"], dev["rewards"])
+    np.testing.assert_array_equal(got["loss"], dev["loss"])
+
+
+def test_host_entry_reports_a_bad_target(ctx):
+    wl = _small(S=50)
+    H, W, y = _inputs(wl)
+    y = y.copy()
+    y[5] = -1
+    with pytest.raises(dust.DustError) as ei:
+        ctx.head_grad_host(_host(H, wl.dtype), _host(W, wl.dtype), _host(y, "i32"), K=wl.K,
+                           sigma=wl.sigma, S=wl.S, seed=wl.seed)
+    assert ei.value.status == 4
+
+
 def test_single_entry_vocabulary(ctx):
     # V = 1: the loss is exactly 0 and every reward vanishes (up to rounding)
     for S in (0, 1):

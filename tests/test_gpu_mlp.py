@@ -1,6 +1,9 @@
-"""MLP up-projection estimator on the GPU vs the fp64 oracle (bf16 rounding
-points mirrored), on small shapes and on token slices of the d=768,
-d_ff=3072, V=50304 workload."""
+"""MLP-block estimators on the GPU (up-projection, down-projection and the
+attention output projection) vs the exact fp64 oracle on the same bf16
+inputs: small shapes, calls long enough (T K > 131072 rows) that the
+perturbed pass runs in several token chunks with a ragged last one, token
+slices of the d=768, d_ff=3072, V=50304 workload, and the full workload in
+the benchmark's launch configuration on sampled token rows."""
 import numpy as np
 import pytest
 import torch
@@ -168,3 +171,86 @@ def test_attn_out_rejects_bad_O(ctx):
     O = torch.zeros(8, 12, dtype=torch.bfloat16, device="cuda")     # d_o not a multiple of 8
     with pytest.raises(dust.DustError):
         ctx.mlp_grad(*args, to_dev(inp["targets"], "i32"), K=4, sigma=1e-2, layer="attn_out", O=O)
+
+
+# ---- several token chunks in one call ----------------------------------------
+# The perturbed pass takes floor(131072 / K) tokens (all K draws each) per
+# chunk. These calls run three chunks, the last one ragged, so the chunk
+# offsets into u, the logits, the targets and the reward rows are all used.
+
+_RUNNERS = {"up": (_run, _check), "down": (_run_down, _check_down), "attn_out": (_run_attn, _check)}
+
+
+def _chunk_workload(layer, T, K):
+    variant = "attn_out" if layer == "attn_out" else "mlp"
+    return synth.Workload("mlp_chunks", variant, T=T, d=32, d_ff=64, V=300, K=K, S=0,
+                          sigma=1e-2, seed=21, dtype="bf16", targets="zipf")
+
+
+@pytest.mark.parametrize("layer", ["up", "down", "attn_out"])
+@pytest.mark.parametrize("T,K", [(5, 50000), (7, 40000)])
+def test_mlp_block_multi_chunk(ctx, layer, T, K):
+    per_chunk = 131072 // K
+    assert T > 2 * per_chunk and T % per_chunk != 0     # three chunks, the last one ragged
+    wl = _chunk_workload(layer, T, K)
+    run, check = _RUNNERS[layer]
+    got, ref = run(ctx, synth.make_mlp_inputs(wl), wl)
+    check(got, ref)
+
+
+@pytest.mark.parametrize("layer", ["up", "down", "attn_out"])
+def test_mlp_block_multi_chunk_token_offset(ctx, layer):
+    """A token shard (token_offset 11) whose call also spans three chunks."""
+    wl = _chunk_workload(layer, 32, 50000)
+    run, check = _RUNNERS[layer]
+    got, ref = run(ctx, synth.make_mlp_inputs(wl), wl, t0=11, T=5)
+    check(got, ref)
+
+
+# ---- the full workloads, sampled rows ----------------------------------------
+
+def _full_size(ctx, layer):
+    wl = synth.CONFIGS["attn_out_bf16" if layer == "attn_out" else
+                       ("mlp_down_bf16" if layer == "down" else "mlp_bf16")]
+    inp = synth.make_mlp_inputs(wl)
+    dev = {k: to_dev(inp[k], "bf16") for k in ("X", "W_up", "W_down", "W_head")}
+    kw = dict(O=to_dev(inp["O"], "bf16")) if layer == "attn_out" else {}
+    out = ctx.mlp_grad(dev["X"], dev["W_up"], dev["W_down"], dev["W_head"],
+                       to_dev(inp["targets"], "i32"), K=wl.K, sigma=wl.sigma, seed=wl.seed,
+                       want_rewards=True, want_g=True, layer=layer, **kw)
+    torch.cuda.synchronize()
+    return wl, inp, dev, out
+
+
+@pytest.mark.parametrize("layer", ["up", "down", "attn_out"])
+def test_mlp_block_full_size_sampled_rows(ctx, layer):
+    """The whole T=8192, K=256 call (16 chunks of 512 tokens, as the benchmark
+    runs it); token rows from chunks 0, 7 and 15 against the oracle, and G
+    against sum_t g_t x_t^T rebuilt in fp64 from the returned g."""
+    wl, inp, dev, out = _full_size(ctx, layer)
+    assert (131072 // wl.K) == 512 and wl.T == 16 * 512
+    for t in (1, 7 * 512 + 100, 16 * 512 - 1):
+        prm = oracle.Params(T=1, d=wl.d, V=wl.V, d_ff=wl.d_ff, K=wl.K, sigma=wl.sigma,
+                            seed=wl.seed, token_offset=t)
+        args = (inp["X"][t:t + 1],)
+        if layer == "attn_out":
+            args += (inp["O"][t:t + 1],)
+        fn = {"up": oracle.mlp_grad, "down": oracle.mlp_down_grad,
+              "attn_out": oracle.attn_out_grad}[layer]
+        ref = fn(*args, inp["W_up"], inp["W_down"], inp["W_head"], inp["targets"][t:t + 1], prm)
+        assert abs(out["loss"][t].item() - ref["loss"][0]) < TOL_LOSS
+        assert np.abs(np64(out["rewards"][t]) - ref["rewards"][0]).max() < TOL_LOSS
+        assert rel_fro(np64(out["g"][t]), ref["g"][0]) < TOL_G
+    # G = sum_t g_t z_t^T over all tokens, z the layer input: x (up), GELU(u) (down), o (attn_out)
+    g = out["g"].double()
+    if layer == "up":
+        Z = dev["X"].double()
+    elif layer == "attn_out":
+        Z = to_dev(inp["O"], "bf16").double()
+    else:
+        u = dev["X"].double() @ dev["W_up"].double().T
+        Z = 0.5 * u * (1.0 + torch.erf(u / np.sqrt(2.0)))
+    rows = torch.randint(0, g.shape[1], (48,), generator=torch.Generator().manual_seed(1)).cuda()
+    ref_rows = (g[:, rows].T @ Z).cpu().numpy()
+    tol = 1e-5 if layer == "down" else TOL_GW_BF16
+    assert rel_fro(np64(out["G"][rows]), ref_rows) < tol

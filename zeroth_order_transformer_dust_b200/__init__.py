@@ -311,8 +311,9 @@ class Context:
 
     def head_grad_host(self, H, W, targets, *, K, sigma, S=0, seed=0, token_offset=0,
                        draw_offset=0, subset_a=0, stream_id=0, out=None, want_G=True,
-                       want_loss=True) -> dict:
-        """Same estimator with every tensor in host memory (pin it for fast copies)."""
+                       want_loss=True, want_rewards=False, want_g=False) -> dict:
+        """Same estimator with every tensor in host memory (pin it for fast copies);
+        the call copies the inputs to the device and the outputs back."""
         for t, n in ((H, "H"), (W, "W"), (targets, "targets")):
             if t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{n} must be a contiguous host tensor")
@@ -325,15 +326,15 @@ class Context:
                           token_offset=token_offset, draw_offset=draw_offset, subset_a=subset_a,
                           stream_id=stream_id)
         out = dict(out or {})
-        _check_outputs(out, {"G": (V, d), "loss": (T,)}, None)
-        if want_G and "G" not in out:
-            out["G"] = torch.empty(V, d, dtype=torch.float32, pin_memory=True)
-        if want_loss and "loss" not in out:
-            out["loss"] = torch.empty(T, dtype=torch.float32, pin_memory=True)
+        _check_outputs(out, {"G": (V, d), "loss": (T,), "rewards": (T, K), "g": (T, V)}, None)
+        for name, want, shape in (("G", want_G, (V, d)), ("loss", want_loss, (T,)),
+                                  ("rewards", want_rewards, (T, K)), ("g", want_g, (T, V))):
+            if want and name not in out:
+                out[name] = torch.empty(*shape, dtype=torch.float32, pin_memory=True)
         self._bind_stream()
         st = self._L.dust_head_grad_host(self._h, ctypes.byref(prm), _ptr(H), _ptr(W),
                                          _ptr(targets), _ptr(out.get("G")), _ptr(out.get("loss")),
-                                         None, None)
+                                         _ptr(out.get("rewards")), _ptr(out.get("g")))
         self._check(st)
         return out
 
