@@ -9,7 +9,9 @@ selects another one.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl dust|reference]
 
-Rank 0 prints one JSON line. Under torchrun (N > 1) each rank runs its own
+``--gpus N`` with N > 1 starts N ranks itself (torch.distributed.run, one
+process per GPU) unless a launcher already did; under a launcher it must
+equal WORLD_SIZE. Rank 0 prints one JSON line. With N > 1 each rank runs its own
 token shard (token_offset = rank * T, so the noise is that of one N*T-token
 run) and the step ends with the one exchange the path has, a sum all-reduce
 of G_W over NCCL: weak scaling, value = all ranks' token-draws / the slowest
@@ -38,10 +40,17 @@ METRIC = "token-draws/sec of Dust gradient estimate (LM head d=1024,V=50304); % 
 UNIT = "token-draws/s"
 SM_COUNT = 148
 LANES_PER_SM = 128           # 4 schedulers x 32 lanes issue per clock
-# Algorithmic instruction slots per perturbed element:
-# Philox4x32-10 10, Gaussian transform 4, expm1 2, reward multiply-add and
-# its operand load 2, g accumulation multiply and add 2.
-ALU_OPS_PER_ELEM = 20
+SFU_PER_SM = 16              # transcendental (MUFU) lanes per SM per clock
+# Algorithmic minimum of issue slots per perturbed element (the roofline's
+# `frac`): Philox4x32-10 10 (2.5 rounds per word, each two wide multiplies and
+# two three-input XORs), the Gaussian 2 (half of a log, a square root and a
+# sine/cosine pair, one slot each), the expm1 1 and one multiply-add 1.
+ALU_OPS_PER_ELEM = 14
+# A second count, reported beside it: the same generator with the sine and
+# cosine as two slots and the expm1 as two (a degree-3 series), the p operand
+# load that feeds the reward's multiply-add, and the g accumulation's
+# multiply and shared-memory add, which the fused kernel must also issue.
+ALU_OPS_PER_ELEM_WITH_ACCUMULATE = 20
 # attention internals: per (draw, head, row visited) a d_h-long dot product
 # on the tensor cores, taken as three fp16 products (6 d_h flops), and on the
 # CUDA cores an expm1 (8 lane operations) and two multiply-adds; per noise
@@ -200,8 +209,21 @@ def cpu_baseline(name: str, budget_tokens: int = 0) -> dict:
     what = (f"{len(toks)} tokens x the first {ATTN_SAMPLE_DRAWS} draws" if attn
             else f"{len(toks)} tokens x all {wl.K} draws")
     return {"value": value, "unit": UNIT, "cores": len(chunks), "kind": "oracle",
+            "host_cores": os.cpu_count(), "cpu_model": _cpu_model(), "seconds": dt,
             "sample": f"{what} of {name}, fp64 NumPy oracle, "
-                      f"{len(chunks)} spawned single-threaded workers, slowest {dt:.1f} s"}
+                      f"{len(chunks)} spawned single-threaded workers on a host of "
+                      f"{os.cpu_count()} cores, slowest {dt:.1f} s"}
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -238,18 +260,31 @@ def _barrier(world):
 
 
 def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
-    """ALU-issue roofline of the draw kernel (algorithmic elements x ops / time)."""
+    """ALU-issue roofline of the draw kernel: algorithmic elements x the minimum
+    issue slots per element / time, against every lane issuing each clock; the
+    SFU (exp) ceiling and the second instruction count are reported beside it.
+    Full-vocabulary draws generate the noise twice (reward, then g); the
+    algorithmic count is one generation."""
     if wl.S > 0:
         elems = wl.T * wl.K * (wl.S + 1)
     else:
         elems = wl.T * wl.K * wl.V
-    achieved = elems * ALU_OPS_PER_ELEM / (draw_ms * 1e-3) / 1e12      # Tops/s
+    t = draw_ms * 1e-3
     f = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
     peak = SM_COUNT * LANES_PER_SM * f / 1e12
+    achieved = elems * ALU_OPS_PER_ELEM / t / 1e12                   # T lane-ops/s
+    alt = elems * ALU_OPS_PER_ELEM_WITH_ACCUMULATE / t / 1e12
+    sfu_peak = SM_COUNT * SFU_PER_SM * f / 1e12                        # T exp/s
     return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s",
-            "frac": achieved / peak, "traffic": None, "kernel": "subset_draws" if wl.S > 0 else "reward+g",
+            "frac": achieved / peak, "traffic": None,
+            "kernel": "subset_draws" if wl.S > 0 else "reward+g",
             "elements": elems, "ops_per_element": ALU_OPS_PER_ELEM, "kernel_ms": draw_ms,
-            "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)"}
+            "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)",
+            "with_accumulate": {"ops_per_element": ALU_OPS_PER_ELEM_WITH_ACCUMULATE,
+                                "achieved": alt, "frac": alt / peak},
+            "sfu": {"exp_per_element": 1, "achieved": elems / t / 1e12, "peak": sfu_peak,
+                    "unit": "Texp/s", "frac": elems / t / 1e12 / sfu_peak,
+                    "peak_basis": f"{SM_COUNT} SMs x {SFU_PER_SM} SFU lanes x {f / 1e6:.0f} MHz"}}
 
 
 def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
@@ -278,31 +313,56 @@ def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
     return roof
 
 
-def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
-    """Tensor-core roofline of the MLP-block perturbed pass: the flops its
-    GEMMs execute per (token, draw) row, the activations contracted as bf16
-    hi/lo planes (K doubled), against the sustained bf16 peak (a pass of
-    hundreds of milliseconds runs under the power cap)."""
+def _mlp_flops_per_row(wl) -> tuple:
+    """(algorithmic, executed) flops of the perturbed pass per (token, draw):
+    the method's GEMMs dh = da W_down^T (up), du = (sigma eps) W_up^T and dh
+    (attention output projection) and dz = dh W_head^T; the kernels carry
+    each activation operand as two bf16 planes (hi and lo), so they execute
+    twice the depth of every contraction."""
     d, dff, V = wl.d, wl.d_ff, wl.V
-    per_row = 2.0 * (2 * d) * V                   # dz = dh W_head^T with the reward epilogue
+    alg = 2.0 * d * V
     if wl.variant in ("mlp", "attn_out"):
-        per_row += 2.0 * (2 * dff) * d            # dh = da W_down^T
+        alg += 2.0 * dff * d
     if wl.variant == "attn_out":
-        per_row += 2.0 * (2 * d) * dff            # du = (sigma eps) W_up^T
-    flops = per_row * wl.T * wl.K
+        alg += 2.0 * d * dff
+    return alg, 2.0 * alg
+
+
+def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
+    """Tensor-core roofline of the MLP-block perturbed pass: the method's flops
+    per (token, draw) over the stage time, against the sustained bf16 peak (a
+    pass of hundreds of milliseconds runs under the power cap); the flops the
+    hi/lo-plane GEMMs execute are reported beside it."""
+    alg, exe = _mlp_flops_per_row(wl)
+    rows = wl.T * wl.K
     t = perturbed_ms * 1e-3
     peak = float(peaks.get("bf16_tflops_sustained", 1416.7))
-    return {"bound": "tensor", "achieved": flops / t / 1e12, "peak": peak, "unit": "TFLOP/s",
-            "frac": flops / t / 1e12 / peak, "traffic": None, "kernel": "perturbed GEMMs",
-            "flops": flops, "kernel_ms": perturbed_ms,
-            "flops_basis": "executed flops of the perturbed GEMMs (hi/lo planes: K doubled)",
-            "peak_basis": "measured bf16 sustained (power-capped) peak"}
+    return {"bound": "tensor", "achieved": alg * rows / t / 1e12, "peak": peak, "unit": "TFLOP/s",
+            "frac": alg * rows / t / 1e12 / peak, "traffic": None, "kernel": "perturbed GEMMs",
+            "flops": alg * rows, "kernel_ms": perturbed_ms,
+            "flops_basis": "algorithmic flops of the perturbed pass's GEMMs per (token, draw)",
+            "peak_basis": "measured bf16 sustained (power-capped) peak",
+            "executed": {"flops": exe * rows, "achieved": exe * rows / t / 1e12,
+                         "frac": exe * rows / t / 1e12 / peak,
+                         "basis": "hi/lo bf16 planes: each contraction executed at twice its depth"}}
 
 
-def _config(args, wl, world: int, l2: str) -> dict:
-    """The workload of a JSON line (the same keys on both arms)."""
+def _gemm_report(flops: float, ms: float, peaks) -> dict:
+    """Algorithmic TFLOP/s of one GEMM stage and its share of the measured bf16 peaks."""
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"ms": ms, "tflops": tf,
+            "frac_burst": tf / float(peaks.get("bf16_tflops", 1640.9)),
+            "frac_sustained": tf / float(peaks.get("bf16_tflops_sustained", 1416.7))}
+
+
+L2_NOTE = ("GPU arm: a 256 MiB write flushes L2 between timed steps; "
+           "the oracle arm runs on the host cores")
+
+
+def _config(args, wl, world: int) -> dict:
+    """The workload of a JSON line (the same dict on both arms)."""
     cfg = {"workload": args.config, "T_per_gpu": wl.T, "d": wl.d, "V": wl.V, "K": wl.K,
-           "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype, "d_ff": wl.d_ff, "l2": l2,
+           "S": wl.S, "sigma": wl.sigma, "dtype_inputs": wl.dtype, "d_ff": wl.d_ff, "l2": L2_NOTE,
            "parallelism": (f"dp{world}: token-sharded, G_W summed by NCCL all-reduce"
                            if world > 1 else "dp1")}
     if wl.seq_len:
@@ -312,25 +372,29 @@ def _config(args, wl, world: int, l2: str) -> dict:
 
 # ----------------------------------------------------------------------------- main arms
 def run_reference(args):
-    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    """The oracle on the host, each step a bounded token sample of the workload
+    (all K draws of each sampled token): value = the sample's token-draws / its
+    time, ms_per_step = the sample's measured time. Rank 0 alone runs."""
+    world, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import synth
     wl = synth.CONFIGS[args.config]
-    per_step = []
+    per_step, secs = [], []
     cb = None
     for _ in range(args.warmup):
         cpu_baseline(args.config, budget_tokens=args.ref_tokens)
     for _ in range(args.steps):
         cb = cpu_baseline(args.config, budget_tokens=args.ref_tokens)
         per_step.append(cb["value"])
+        secs.append(cb["seconds"])
     value = statistics.median(per_step)
     cb["value"] = value
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": wl.token_draws / value * 1e3,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": _config(args, wl, 1, "the oracle runs on the host (no L2 flush)"),
+            "config": _config(args, wl, world),
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -479,12 +543,15 @@ def run_dust(args):
     if wl.variant in ("mlp", "mlp_down", "attn_out") and stages.get("perturbed"):
         roof = _mlp_roofline(wl, stages["perturbed"], peaks)
         roof["peak_kind"] = peak_kind
+    # the two dense contractions of the head, 2 T d V flops each (G_W: the
+    # stage includes the transposes that make both operands K-major)
     gemm_flops = 2.0 * wl.T * wl.d * wl.V
     extra = {}
     if wl.variant == "head":
-        for key in ("clean_gemm", "gw_gemm"):
-            if stages.get(key):
-                extra[key + "_tflops"] = gemm_flops / (stages[key] * 1e-3) / 1e12
+        gemms = {key: _gemm_report(gemm_flops, stages[key], peaks)
+                 for key in ("clean_gemm", "gw_gemm") if stages.get(key)}
+        if gemms:
+            extra["gemms"] = gemms
 
     # cos(g, exact gradient) against K, outside the timed region (head workloads at N = 1)
     align = None
@@ -503,7 +570,7 @@ def run_dust(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic",
-                "config": _config(args, wl, world, "flushed between timed steps (256 MiB write)"),
+                "config": _config(args, wl, world),
                 "stage_ms": stages, "gpu_launches": launches, "e2e": e2e, "roofline": roof,
                 "cpu_baseline": cb, "clocks": clk, "alignment": align, **extra}
         print(json.dumps(line), flush=True)
@@ -512,6 +579,18 @@ def run_dust(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def _launch_ranks(argv, n: int) -> int:
+    """Start n ranks of this script on this node (one process per GPU) with
+    torch.distributed.run and return its exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def main(argv=None):
@@ -530,6 +609,13 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=0,
                     help="run only the first N tokens of the workload (profiling slices)")
     args = ap.parse_args(argv)
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        return _launch_ranks(sys.argv[1:] if argv is None else list(argv), args.gpus)
+    if world_env is not None and int(world_env) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but the launcher started WORLD_SIZE={world_env} ranks",
+              file=sys.stderr)
+        return 2
     if args.tokens:
         import synth
         wl = synth.CONFIGS[args.config]
