@@ -91,7 +91,12 @@ typedef struct dust_params {
 } dust_params;
 
 /* Create a context on CUDA device `device`, enqueuing on `cuda_stream`
-   (a cudaStream_t; NULL = the legacy default stream). */
+   (a cudaStream_t; NULL = the legacy default stream). Environment variables
+   read here select alternative kernels of the context (all give the same
+   results within the parity tolerances): DUST_DISABLE_TC=1 runs every GEMM
+   on CUDA cores; DUST_TC_PAIR=0 gives each tensor-core GEMM tile one CTA
+   instead of a CTA pair; DUST_SUBSET_KERNEL=1 uses the L2-fed subset-draw
+   kernel instead of the shared-memory one. */
 dust_status dust_create(dust_ctx** out, int device, void* cuda_stream);
 dust_status dust_set_stream(dust_ctx* ctx, void* cuda_stream);
 /* Frees the context's scratch memory; waits for its stream first. */
@@ -336,11 +341,18 @@ dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4
    under p's seed, offsets and stream_id -> out[(t*ni + i)*nslots + k] fp32. */
 dust_status dust_debug_gauss(dust_ctx* ctx, const dust_params* p, int32_t tag,
                              int64_t nt, int64_t ni, int64_t nslots, float* out);
-/* Debug: the same eps through the table-driven angle step the subset-draw
-   kernel uses (a 1024-entry table of roots of unity plus angle addition);
-   it agrees with dust_debug_gauss to a few 1e-7. */
+/* Debug: the same eps through the table-driven angle step the LM-head draw
+   kernels use (a 1024-entry table of roots of unity plus angle addition), in
+   the packed fp32x2 form those kernels run (the two Box-Muller pairs of a
+   Philox counter side by side); it agrees with dust_debug_gauss to a few
+   1e-7. */
 dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t tag,
                                  int64_t nt, int64_t ni, int64_t nslots, float* out);
+/* Debug: the table-driven step in scalar form, one Box-Muller pair at a
+   time; equal to dust_debug_gauss_tab bit for bit (same operations, same
+   rounding). */
+dust_status dust_debug_gauss_tab_scalar(dust_ctx* ctx, const dust_params* p, int32_t tag,
+                                        int64_t nt, int64_t ni, int64_t nslots, float* out);
 
 /* Debug: the Box-Muller radius for every 24-bit input (the pages fix only
    Gaussian noise; this transform is the library's). out (2^24 fp32, device)

@@ -88,6 +88,16 @@ CONFIGS = {
     "attn_v_bf16": Workload("attn_v_bf16", "attn_v", T=8192, d=768, V=1, K=256, S=0,
                             sigma=1e-2, seed=5, dtype="bf16", targets="none", seq_len=1024,
                             n_heads=12, head_dim=64),
+    # The subset estimator at a 128256-entry vocabulary (a Llama-3-size head):
+    # the shared-memory kernel with a cluster of 8 CTAs per token.
+    "subset_v128k_bf16": Workload("subset_v128k_bf16", "head", T=8192, d=1024, V=128256,
+                                  K=1024, S=512, sigma=1e-2, seed=6, dtype="bf16",
+                                  targets="zipf"),
+    # Subset draws of S = 1024 entries, beyond the shared-memory kernel's 512:
+    # the L2-fed kernel that keeps only the g row in shared memory.
+    "subset_s1024_bf16": Workload("subset_s1024_bf16", "head", T=8192, d=1024, V=50304,
+                                  K=1024, S=1024, sigma=1e-2, seed=7, dtype="bf16",
+                                  targets="zipf"),
     # LM head at 243M-model head scale, subset draws (S = 512), 16k draws.
     "large_subset_bf16": Workload("large_subset_bf16", "head", T=16384, d=1024, V=50304,
                                   K=16384, S=512, sigma=5e-3, seed=4, dtype="bf16",

@@ -91,6 +91,16 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     # fixed-point accumulation with a reduced scale (16384 < K <= 65536), and the
     # fp32-atomic fallback (K > 65536)
     dict(T=3, K=20000, S=32), dict(T=2, K=70000, S=64, V=700),
+    # vocabularies beyond one or two CTAs' shared memory: clusters of 4 and 8
+    # CTAs (windows crossing into the next CTA's slice and wrapping past V)
+    dict(V=70001, S=300, K=256, T=4), dict(V=128256, S=512, K=256, T=4, d=24),
+    dict(V=200003, S=512, K=256, T=4, d=16), dict(V=200003, S=77, K=300, T=3, d=16, dtype="f32"),
+    # fp32 accumulators (K > 65536) with the target in another CTA's slice
+    dict(V=70001, S=64, K=70000, T=1, d=16),
+    # full vocabulary: ragged slabs at several V, more tokens than CTAs
+    dict(V=4099, K=20), dict(V=20000, K=33, T=5, d=16), dict(V=100000, K=9, T=3, d=16),
+    dict(T=200, K=5, V=1000), dict(T=300, K=2, V=3000, dtype="f32"),
+    dict(V=120000, K=8, T=3, d=16),
 ])
 def test_edge_shapes(ctx, kw):
     wl = _small(**kw)

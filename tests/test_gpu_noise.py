@@ -40,6 +40,18 @@ def test_gaussians_match_oracle(ctx, tag, stream, table):
     assert err < TOL_GAUSS, err
 
 
+def test_packed_table_step_equals_the_scalar_one_bit_for_bit(ctx):
+    """The draw kernels run the table-driven Box-Muller step in packed fp32x2
+    form (two pairs per instruction); the scalar form that the exhaustive
+    radius and angle checks below cover must give the same bits."""
+    for seed, tag, t0 in ((3, oracle.TAG_HEAD, 0), (0xFFFFFFFFFFFF, oracle.TAG_HEAD, 123456),
+                          (77, oracle.TAG_MLP_UP, 9)):
+        a = ctx.debug_gauss(128, 256, 1024, tag=tag, seed=seed, token_offset=t0, table=True)
+        b = ctx.debug_gauss(128, 256, 1024, tag=tag, seed=seed, token_offset=t0, table=True,
+                            scalar=True)
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
 @pytest.mark.parametrize("table", [False, True])
 def test_gaussian_extremes_match_oracle(ctx, table):
     # many draws so that the tails (|eps| > 4.5) are exercised

@@ -33,6 +33,7 @@ EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
            "dust_head_grad", "dust_head_grad_host", "dust_mlp_grad", "dust_debug_philox",
            "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
            "dust_kernel_launches", "dust_debug_gemm_bf16", "dust_debug_gauss_tab",
+           "dust_debug_gauss_tab_scalar",
            "dust_head_grad_noalloc", "dust_debug_bm_radius", "dust_debug_bm_angle",
            "dust_attn_grad",
            "dust_sgd_momentum", "dust_mlp_down_grad", "dust_attn_out_grad")
@@ -103,6 +104,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "dust_kernel_launches": (I64, [P]),
             "dust_debug_gemm_bf16": (I32, [P, I64, I64, I64, P, P, P, ctypes.c_int]),
             "dust_debug_gauss_tab": (I32, [P, PP, I32, I64, I64, I64, P]),
+            "dust_debug_gauss_tab_scalar": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_head_grad_noalloc": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_char_p,
                                              ctypes.c_int]),
             "dust_debug_bm_radius": (I32, [P, I32, ctypes.c_float, P]),
@@ -477,13 +479,15 @@ class Context:
         return out
 
     def debug_gauss(self, nt, ni, nslots, *, tag=TAG_HEAD, seed=0, token_offset=0, draw_offset=0,
-                    stream_id=0, table=False) -> torch.Tensor:
-        """eps[t, i, k]; table=True uses the subset kernel's table-driven angle step."""
+                    stream_id=0, table=False, scalar=False) -> torch.Tensor:
+        """eps[t, i, k]; table=True uses the LM-head kernels' table-driven angle
+        step in their packed form, with scalar=True in scalar form."""
         prm = make_params(1, 1, 1, 1, 0.0, seed=seed, token_offset=token_offset,
                           draw_offset=draw_offset, stream_id=stream_id)
         out = torch.empty(nt, ni, nslots, dtype=torch.float32, device=f"cuda:{self.device}")
         self._bind_stream()
-        fn = self._L.dust_debug_gauss_tab if table else self._L.dust_debug_gauss
+        fn = ((self._L.dust_debug_gauss_tab_scalar if scalar else self._L.dust_debug_gauss_tab)
+              if table else self._L.dust_debug_gauss)
         self._check(fn(self._h, ctypes.byref(prm), tag, nt, ni, nslots, _ptr(out)))
         return out
 

@@ -856,6 +856,11 @@ dust_status dust_debug_gauss_tab(dust_ctx* ctx, const dust_params* p, int32_t ta
   return debug_gauss_impl(ctx, p, tag, nt, ni, nslots, out, 1);
 }
 
+dust_status dust_debug_gauss_tab_scalar(dust_ctx* ctx, const dust_params* p, int32_t tag,
+                                        int64_t nt, int64_t ni, int64_t nslots, float* out) {
+  return debug_gauss_impl(ctx, p, tag, nt, ni, nslots, out, 2);
+}
+
 dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, const float* G,
                               float* v, float* W, void* W_bf16) {
   if (!ctx) return DUST_ERR_ARG;

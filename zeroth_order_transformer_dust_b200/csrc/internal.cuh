@@ -192,7 +192,8 @@ namespace dust {
 // Kernel launchers (all enqueue on `st`, return cudaGetLastError()).
 cudaError_t launch_debug_philox(cudaStream_t st, uint64_t seed, const uint32_t* ctr, int64_t n,
                                 uint32_t* out);
-// method 0: polynomial angle step; 1: table-driven angle step (subset kernel).
+// method 0: polynomial angle step; 1: table-driven angle step in the packed
+// fp32x2 form of the draw kernels; 2: the same step in scalar form.
 cudaError_t launch_sgd_momentum(cudaStream_t st, int64_t n, float lr, float mu, const float* G,
                                 float* v, float* W, __nv_bfloat16* Wb, int sm_count);
 // what: 0 = radius for all 2^24 u1 (2^24 floats), 1 = polynomial angle step,

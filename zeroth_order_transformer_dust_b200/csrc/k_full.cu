@@ -52,12 +52,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Draws [i0, i0 + n) of one unit for one warp; per draw, the warp's sum goes
 // to sh[warp][ii]. ALL: all kBlocksPerWarp blocks of the warp lie below V
 // (every warp but the one that straddles V), so no per-block test runs in the
-// draw loop. The reward sum runs as one chain per block. No barrier inside:
+// draw loop. The noise, expm1 and the reward sums run in packed fp32x2
+// arithmetic on the pairs of slots (lane, lane + 64) and (lane + 32, lane + 96)
+// of each block (p02, p13), one pair of chains per block. No barrier inside:
 // the caller's block-wide barriers are the same for every warp.
 template <int DEG, bool ALL>
 __device__ __forceinline__ void reward_chunk(const FullArgs& A, const float2* tab, int64_t t,
                                              int i0, int n, int nvalid,
-                                             const float (&pv)[kBlocksPerWarp][4],
+                                             const float2 (&p02)[kBlocksPerWarp],
+                                             const float2 (&p13)[kBlocksPerWarp],
                                              const BlockConst (&bc)[kBlocksPerWarp],
                                              bool warp_has_y, bool y_here, int by, int jy,
                                              float (*sh)[kDrawChunk]) {
@@ -72,13 +75,15 @@ __device__ __forceinline__ void reward_chunk(const FullArgs& A, const float2* ta
     for (int b = 0; b < kBlocksPerWarp; ++b) {
       sb[b] = 0.0f;
       if (ALL || b < nvalid) {
-        const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) sb[b] = fmaf(pv[b][j], expm1_small<DEG>(g.v[j]), sb[b]);
-        if (warp_has_y) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (b == by && j == jy) xyv = g.v[j];
+        float2 e02, e13;
+        gauss4_tab_x2(philox_from2(bc[b], dc, A.keys), tab, e02, e13);
+        float2 s2 = __fmul2_rn(p02[b], expm1_small_x2<DEG>(e02));
+        s2 = __ffma2_rn(p13[b], expm1_small_x2<DEG>(e13), s2);
+        sb[b] = s2.x + s2.y;
+        if (warp_has_y && b == by) {
+          // word jy of the counter: 0, 2 in e02 and 1, 3 in e13
+          const float2 e = (jy & 1) ? e13 : e02;
+          xyv = (jy & 2) ? e.y : e.x;
         }
       }
     }
@@ -106,17 +111,22 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __gri
     // blocks of this warp below V (warp-uniform)
     const int64_t left = (A.V - blk0 * 128 + 127) / 128;
     const int nvalid = left <= 0 ? 0 : (left >= kBlocksPerWarp ? kBlocksPerWarp : (int)left);
-    float pv[kBlocksPerWarp][4];  // p = exp(z - LSE), formed once per unit
+    // p = exp(z - LSE), formed once per unit, as the packed pairs of slots
+    // (lane, lane + 64) and (lane + 32, lane + 96) of each block
+    float2 p02[kBlocksPerWarp], p13[kBlocksPerWarp];
     BlockConst bc[kBlocksPerWarp];
     const float lse_t = A.lse[t];
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b) {
       bc[b] = block_const(A.keys, slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), A.ctr3);
+      float pv[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
-        pv[b][j] = pos < A.V ? expf(A.Z[t * A.V + pos] - lse_t) : 0.0f;
+        pv[j] = pos < A.V ? expf(A.Z[t * A.V + pos] - lse_t) : 0.0f;
       }
+      p02[b] = make_float2(pv[0], pv[2]);
+      p13[b] = make_float2(pv[1], pv[3]);
     }
     // the lane holding the target's noise, if this warp's blocks contain it
     int32_t yt = A.y[t];
@@ -128,9 +138,9 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_reward_partial(const __gri
     for (int i0 = 0; i0 < A.K; i0 += kDrawChunk) {
       const int n = min(kDrawChunk, A.K - i0);
       if (nvalid == kBlocksPerWarp)
-        reward_chunk<DEG, true>(A, tab, t, i0, n, nvalid, pv, bc, warp_has_y, y_here, by, jy, sh);
+        reward_chunk<DEG, true>(A, tab, t, i0, n, nvalid, p02, p13, bc, warp_has_y, y_here, by, jy, sh);
       else
-        reward_chunk<DEG, false>(A, tab, t, i0, n, nvalid, pv, bc, warp_has_y, y_here, by, jy, sh);
+        reward_chunk<DEG, false>(A, tab, t, i0, n, nvalid, p02, p13, bc, warp_has_y, y_here, by, jy, sh);
       __syncthreads();
       if ((int)threadIdx.x < n) {
         float s = 0.0f;
@@ -156,21 +166,26 @@ __global__ void k_full_reward_combine(int64_t T, int32_t K, int nslab,
 }
 
 // Draws [i0, i0 + n) of sum_i r_i (sigma eps_i) for one warp's blocks, with
-// r staged in rs (ALL: every block lies below V). No barrier inside.
+// r staged in rs (ALL: every block lies below V), accumulated in packed pairs
+// (slots lane, lane + 64 in acc02; lane + 32, lane + 96 in acc13). No barrier
+// inside.
 template <bool ALL>
 __device__ __forceinline__ void g_chunk(const FullArgs& A, const float2* tab, int64_t t, int i0,
                                         int n, int nvalid, const BlockConst (&bc)[kBlocksPerWarp],
-                                        const float* rs, float (&acc)[kBlocksPerWarp][4]) {
+                                        const float* rs, float2 (&acc02)[kBlocksPerWarp],
+                                        float2 (&acc13)[kBlocksPerWarp]) {
   const uint32_t t_abs = A.t_off + (uint32_t)t;
   for (int ii = 0; ii < n; ++ii) {
     const float ri = rs[ii];
+    const float2 r2 = make_float2(ri, ri);
     const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)(i0 + ii));
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b) {
       if (ALL || b < nvalid) {
-        const G4 g = gauss4_tab(philox_from2(bc[b], dc, A.keys), tab);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[b][j] = fmaf(ri, g.v[j], acc[b][j]);
+        float2 e02, e13;
+        gauss4_tab_x2(philox_from2(bc[b], dc, A.keys), tab, e02, e13);
+        acc02[b] = __ffma2_rn(r2, e02, acc02[b]);
+        acc13[b] = __ffma2_rn(r2, e13, acc13[b]);
       }
     }
   }
@@ -190,12 +205,12 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
     const int64_t left = (A.V - blk0 * 128 + 127) / 128;
     const int nvalid = left <= 0 ? 0 : (left >= kBlocksPerWarp ? kBlocksPerWarp : (int)left);
     BlockConst bc[kBlocksPerWarp];
-    float acc[kBlocksPerWarp][4];
+    float2 acc02[kBlocksPerWarp], acc13[kBlocksPerWarp];
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b) {
       bc[b] = block_const(A.keys, slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), A.ctr3);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[b][j] = 0.0f;
+      acc02[b] = make_float2(0.0f, 0.0f);
+      acc13[b] = make_float2(0.0f, 0.0f);
     }
     for (int i0 = 0; i0 < A.K; i0 += 1024) {
       const int n = min(1024, A.K - i0);
@@ -203,9 +218,9 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
       for (int q = threadIdx.x; q < n; q += blockDim.x) rs[q] = A.r[t * A.K + i0 + q];
       __syncthreads();
       if (nvalid == kBlocksPerWarp)
-        g_chunk<true>(A, tab, t, i0, n, nvalid, bc, rs, acc);
+        g_chunk<true>(A, tab, t, i0, n, nvalid, bc, rs, acc02, acc13);
       else
-        g_chunk<false>(A, tab, t, i0, n, nvalid, bc, rs, acc);
+        g_chunk<false>(A, tab, t, i0, n, nvalid, bc, rs, acc02, acc13);
     }
 #pragma unroll
     for (int b = 0; b < kBlocksPerWarp; ++b)
@@ -213,7 +228,8 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
       for (int j = 0; j < 4; ++j) {
         const int64_t pos = (blk0 + b) * 128 + lane + 32 * j;
         if (pos < A.V) {
-          const float v = acc[b][j] * A.fac;
+          const float2 a = (j & 1) ? acc13[b] : acc02[b];
+          const float v = ((j & 2) ? a.y : a.x) * A.fac;
           if (A.g_out) A.g_out[t * A.V + pos] = v;
           if (A.gop_bf16)
             store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + pos, v);

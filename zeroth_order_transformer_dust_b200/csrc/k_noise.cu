@@ -50,11 +50,13 @@ __global__ void k_debug_gauss(Key key, uint32_t t_off, uint32_t i_off, uint32_t 
   }
 }
 
-// Same with the table-driven angle step of the subset kernel; grid-stride so
-// that each CTA builds its table once.
+// Same with the table-driven angle step of the draw kernels (packed: the
+// fp32x2 form they use; else the scalar form); grid-stride so that each CTA
+// builds its table once.
 __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off, uint32_t i_off,
                                                          uint32_t ctr3, int64_t nt, int64_t ni,
-                                                         int64_t nslots, float* __restrict__ out) {
+                                                         int64_t nslots, float* __restrict__ out,
+                                                         int packed) {
   __shared__ float2 tab[kSinCosTable];
   fill_sincos_table(tab, 1.0f);
   __syncthreads();
@@ -69,7 +71,18 @@ __global__ __launch_bounds__(256) void k_debug_gauss_tab(Key key, uint32_t t_off
     const int64_t i = rest % ni;
     const int64_t t = rest / ni;
     U4 c{slot_ctr0((uint32_t)blk, lane), t_off + (uint32_t)t, i_off + (uint32_t)i, ctr3};
-    const G4 g = gauss4_tab(philox10(c, key.k0, key.k1), tab);
+    const U4 w = philox10(c, key.k0, key.k1);
+    G4 g;
+    if (packed) {
+      float2 e02, e13;
+      gauss4_tab_x2(w, tab, e02, e13);
+      g.v[0] = e02.x;
+      g.v[1] = e13.x;
+      g.v[2] = e02.y;
+      g.v[3] = e13.y;
+    } else {
+      g = gauss4_tab(w, tab);
+    }
     float* row = out + (t * ni + i) * nslots;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -122,10 +135,10 @@ cudaError_t launch_debug_gauss(cudaStream_t st, const dust_params& p, int tag, i
   if (total <= 0) return cudaSuccess;
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
-  if (method == 1) {
+  if (method == 1 || method == 2) {
     k_debug_gauss_tab<<<(unsigned)(blocks < 2048 ? blocks : 2048), threads, 0, st>>>(
         key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,
-        ctr3_of(tag, p.stream_id), nt, ni, nslots, out);
+        ctr3_of(tag, p.stream_id), nt, ni, nslots, out, method == 1);
   } else {
     k_debug_gauss<<<(unsigned)blocks, threads, 0, st>>>(
         key_of(p.seed), (uint32_t)p.token_offset, (uint32_t)p.draw_offset,

@@ -9,19 +9,23 @@
 // log1p(sum_drawn p_j expm1(sigma eps_j)), r = sigma eps_y - log1p(.), and
 // r eps (scaled by the inverse inclusion probability) accumulates into g_t.
 //
-// B200 mapping: one cluster of CS CTAs (one per SM) per token at a time,
+// B200 mapping: one cluster of CS CTAs (one per SM; CS = 1, 2, 4 or 8, the
+// smallest whose slices fit in shared memory) per token at a time,
 // persistent over tokens. CTA r of the cluster holds the probability row and
-// the g accumulator for its slice of q in shared memory (CS = 2 at V = 50304:
-// 2 x 100.6 KB per CTA), so the hot loop touches no global memory. Warps take
-// batches of 32 draws from a shared counter; in a batch each lane works out
-// one draw's window start, whether its window holds the target and the noise
-// of the appended target slot, and the warp then processes, one after the
-// other, the draws whose window starts in its CTA's slice. Windows that run
-// into the next slice (or wrap past V) reach the partner's shared memory
-// through DSMEM. The noise of a draw is generated once, already multiplied by
-// sigma, kept in registers from the reward to the accumulation, and the
-// first two Philox rounds are evaluated once per draw and once per slot
-// block (they depend on the draw index or on the slot block only).
+// the g accumulator for its slice [r seg, (r+1) seg) of q in shared memory
+// (CS = 2 at V = 50304: 2 x 100.6 KB per CTA; CS = 8 reaches V ~ 223k), so
+// the hot loop touches no global memory. Warps take batches of 32 draws from
+// a shared counter; in a batch each lane works out one draw's window start,
+// whether its window holds the target and the noise of the appended target
+// slot, and the warp then processes, one after the other, the draws whose
+// window starts in its CTA's slice. A window is no longer than a slice, so
+// the part that runs past the slice (or wraps past V, which only a window
+// starting in the last slice can do) lies in the next CTA's slice,
+// (r + 1) mod CS, reached through DSMEM. The noise of a draw is generated
+// once, already multiplied by sigma, kept in registers from the reward to the
+// accumulation, and the first two Philox rounds are evaluated once per draw
+// and once per slot block (they depend on the draw index or on the slot block
+// only).
 //
 // Accumulation (INT = true): off-target coordinates accumulate r * sigma eps
 // in 2^-15 fixed point (scaled by 1/sigma^2) with native int32 shared-memory
@@ -44,12 +48,22 @@ namespace cg = cooperative_groups;
 namespace dust {
 namespace {
 
-// Threads per CTA. The fixed-point cluster kernel fits 64 registers, so it
-// runs 32 warps per SM (8 per scheduler), which hides the dependent-issue
-// latency of the generator better than 16 warps at 116 registers (4.5% less
-// time at 32 than at 16 warps on the large-subset workload); the other
-// variants keep 16 warps, where they need no spills.
-__host__ __device__ constexpr int sub2_threads(int cs, bool use_int) { return cs == 2 && use_int ? 1024 : 512; }
+// Threads per CTA. The fixed-point kernel with a series expm1 fits 64
+// registers, so it runs 32 warps per SM (8 per scheduler), which hides the
+// dependent-issue latency of the generator better than 16 warps at 116
+// registers (4.5% less time at 32 than at 16 warps on the large-subset
+// workload); the fp32-accumulator variant and the library expm1 (large sigma)
+// keep 16 warps, where they need no spills.
+__host__ __device__ constexpr int sub2_threads(bool use_int, int deg) {
+  return use_int && deg != 0 ? 1024 : 512;
+}
+
+// Draws of one token the shared list holds (16 bytes each). With K <= kListCap
+// every draw of a token is set up once per CTA up front and the warps take the
+// CTA's draws one at a time, so a token's work splits evenly however the
+// window starts fall; with more draws the warps take batches of 32 as they go.
+constexpr int kListCap = 1024;
+constexpr int64_t kStaticSmem = 1024 + 8 * kSinCosTable;  // counters, angle table
 
 struct Sub2Args {
   Key key;
@@ -59,8 +73,9 @@ struct Sub2Args {
   int64_t T, V;
   int32_t K, S;
   uint32_t a, a_inv;
-  uint32_t minv;  // floor((2^32 - 1) / V), V <= 2^16
-  uint32_t seg;  // q-slice length owned by one CTA (multiple of 4)
+  uint64_t minv;  // floor((2^64 - 1) / V)
+  uint32_t cs;    // CTAs per cluster
+  uint32_t seg;   // q-slice length owned by one CTA (multiple of 4)
   float scale_other, scale_target;
   float fac;        // g = fac * sum r * (sigma eps)            (fp32 accumulators)
   float acc_scale;  // fixed-point units per unit of r * (sigma eps)
@@ -81,13 +96,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// x y mod m for x, y < m <= 2^16 (the product fits 32 bits), with
-// minv = floor((2^32 - 1) / m): the quotient estimate hi32(x y minv) is the
-// true quotient or one less (Barrett), so one conditional subtraction ends it.
-__device__ __forceinline__ uint32_t mulmod32(uint32_t x, uint32_t y, uint32_t m, uint32_t minv) {
-  const uint32_t p = x * y;
-  const uint32_t r = p - __umulhi(p, minv) * m;
-  return r >= m ? r - m : r;
+// x y mod m for x, y < m < 2^31, with minv = floor((2^64 - 1) / m): the
+// quotient estimate hi64(x y minv) is the true quotient or one less
+// (Barrett), so one conditional subtraction ends it.
+__device__ __forceinline__ uint32_t mulmod(uint32_t x, uint32_t y, uint32_t m, uint64_t minv) {
+  const uint64_t p = (uint64_t)x * y;
+  const uint64_t r = p - __umul64hi(p, minv) * m;
+  return (uint32_t)(r >= m ? r - m : r);
 }
 
 template <bool INT>
@@ -99,38 +114,37 @@ __device__ __forceinline__ void accumulate(float* slot, float r, float x, float 
     atomicAdd(slot, r * x);
 }
 
-// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
-template <int CS, int NB, bool FULL, int DEG, bool INT>
-__global__ __launch_bounds__(sub2_threads(CS, INT), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
-  constexpr int kThreads = sub2_threads(CS, INT);
+// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB; LIST: the
+// draws of a token are set up together and taken from a shared list one at a
+// time (K <= kListCap), else taken in batches of 32.
+template <int NB, bool FULL, int DEG, bool INT, bool LIST>
+__global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
+  constexpr int kThreads = sub2_threads(INT, DEG);
   extern __shared__ __align__(16) float smem[];
-  __shared__ int s_next;    // next draw batch of the current token
+  __shared__ int s_next;    // next draw batch (or list entry) of the current token
+  __shared__ int s_cnt;     // LIST: entries of the current token's list
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
   __shared__ float2 s_tab[kSinCosTable];
   fill_sincos_table(s_tab, A.sigma);
   __syncthreads();
   cg::cluster_group cluster = cg::this_cluster();
-  const uint32_t rank = CS > 1 ? cluster.block_rank() : 0;
+  const uint32_t cs = A.cs;
+  const uint32_t rank = cluster.block_rank();
   const int lane = threadIdx.x & 31;
   const uint32_t V = (uint32_t)A.V;
   const uint32_t seg = A.seg;
   const uint32_t lo = rank * seg;
   const uint32_t hi = min(V, lo + seg);
   const uint32_t n_own = hi - lo;
-  const uint32_t lo_peer = lo ^ seg;  // CS = 2: the partner's slice start
+  const uint32_t peer = rank + 1 == cs ? 0u : rank + 1;  // holds the slice after this one
+  const uint32_t lo_peer = peer * seg;
   float* sp = smem;        // p of q in [lo, hi)
   float* sg = smem + seg;  // g accumulator of q in [lo, hi) (fp32 or int32 fixed point)
-  float* sp_peer = sp;
-  float* sg_peer = sg;
-  float* tgt_peer = &s_tgt;
-  if (CS > 1) {
-    sp_peer = cluster.map_shared_rank(sp, rank ^ 1u);
-    sg_peer = cluster.map_shared_rank(sg, rank ^ 1u);
-    tgt_peer = cluster.map_shared_rank(&s_tgt, rank ^ 1u);
-  }
+  float* const sp_peer = cluster.map_shared_rank(sp, peer);
+  float* const sg_peer = cluster.map_shared_rank(sg, peer);
   const int S = A.S;
-  const uint32_t nclusters = gridDim.x / CS;
-  const uint32_t cid = blockIdx.x / CS;
+  const uint32_t nclusters = gridDim.x / cs;
+  const uint32_t cid = blockIdx.x / cs;
   const int nbatch = (A.K + 31) >> 5;
 
   BlockConst bc[NB];
@@ -160,148 +174,221 @@ __global__ __launch_bounds__(sub2_threads(CS, INT), 1) void k_subset2(const __gr
     }
     if (threadIdx.x == 0) {
       s_next = 0;
+      s_cnt = 0;
       s_tgt = 0.0f;
     }
     int32_t yt = A.y[t];
     if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
-    const uint32_t qy = mulmod32((uint32_t)yt, A.a_inv, V, A.minv);
-    const bool own_y = qy >= lo && qy < hi;
+    const uint32_t qy = mulmod((uint32_t)yt, A.a_inv, V, A.minv);
+    const uint32_t owner_y = qy / seg;  // the CTA whose slice holds the target
     const float py = expf(zrow[qy] - lse_t);
-    float* gy = own_y ? sg + (qy - lo) : sg_peer + (qy - lo_peer);
-    if (CS > 1) cluster.sync(); else __syncthreads();
+    float* gy = cluster.map_shared_rank(sg, owner_y) + (qy - owner_y * seg);
+    cluster.sync();
 
     const uint32_t t_abs = A.t_off + (uint32_t)t;
     float tgt_acc = 0.0f;  // INT: this warp's sum r * (sigma eps_y), lane 0
-    for (;;) {
-      int bidx = 0;
-      if (lane == 0) bidx = atomicAdd(&s_next, 1);
-      bidx = __shfl_sync(0xffffffffu, bidx, 0);
-      if (bidx >= nbatch) break;
-      // ---- per-lane setup of draw bidx*32 + lane
-      const int iq = bidx * 32 + lane;
-      uint32_t c = 0, kyq = 0;
-      float x_extra = 0.0f;
-      bool mine = false;
-      if (iq < A.K) {
-        const uint32_t i_abs = A.i_off + (uint32_t)iq;
-        const uint32_t b = subset_offset(A.key, t_abs, i_abs, A.stream_id, V);
-        c = mulmod32(b, A.a_inv, V, A.minv);
-        mine = (c >= lo) && (c < hi);
-        kyq = (qy >= c) ? qy - c : qy + V - c;
-        if (mine && kyq >= (uint32_t)S) {
-          const U4 w = philox_from2(bs, draw_const(A.keys, t_abs, i_abs), A.keys);
-          const float2 nn =
-              box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, s_tab);
-          x_extra = (s_word & 1u) ? nn.y : nn.x;
+    // Setup of draw iq (one lane): its window start in permuted order, the
+    // target's slot in the window, and whether the window starts in this
+    // CTA's slice; for those, the noise of the appended target slot.
+    auto setup = [&](int iq, uint32_t& c, uint32_t& kyq, float& x_extra) -> bool {
+      const uint32_t i_abs = A.i_off + (uint32_t)iq;
+      const uint32_t b = subset_offset(A.key, t_abs, i_abs, A.stream_id, V);
+      c = mulmod(b, A.a_inv, V, A.minv);
+      const bool mine = (c >= lo) && (c < hi);
+      kyq = (qy >= c) ? qy - c : qy + V - c;
+      x_extra = 0.0f;
+      if (mine && kyq >= (uint32_t)S) {
+        const U4 w = philox_from2(bs, draw_const(A.keys, t_abs, i_abs), A.keys);
+        const float2 nn = box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, s_tab);
+        x_extra = (s_word & 1u) ? nn.y : nn.x;
+      }
+      return mine;
+    };
+    // Draw i with window start cw, target slot ky and appended-slot noise xe,
+    // by the whole warp: reward, then accumulation into g.
+    auto draw = [&](int i, uint32_t cw, uint32_t ky, float xe) {
+      const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)i);
+      const bool in_win = ky < (uint32_t)S;
+      const bool local = (cw + (uint32_t)S) <= hi;  // whole window in this slice
+      float n[NB][4];  // sigma * eps of the draw's slots
+      float s = 0.0f;
+      // packed fp32x2 generation and accumulation (at NB = 2 they need more
+      // than the 64 registers of a 1024-thread CTA, so those variants keep
+      // the scalar form)
+      constexpr bool kPacked = NB != 2;
+      if (local && kPacked) {
+        // packed pairs: slots (lane, lane + 64) and (lane + 32, lane + 96)
+        // of each block, words (0, 2) and (1, 3) of its counter
+        const float* pw = sp + (cw - lo) + lane;
+        float2 s2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int m = 0; m < NB; ++m) {
+          const int k0 = m * 128 + lane;
+          const bool u0 = FULL || k0 < S, u1 = FULL || k0 + 32 < S;
+          const bool u2 = FULL || k0 + 64 < S, u3 = FULL || k0 + 96 < S;
+          const float2 p02 = make_float2(u0 ? pw[m * 128] : 0.0f, u2 ? pw[m * 128 + 64] : 0.0f);
+          const float2 p13 = make_float2(u1 ? pw[m * 128 + 32] : 0.0f, u3 ? pw[m * 128 + 96] : 0.0f);
+          float2 e02, e13;
+          gauss4_tab_x2(philox_from2(bc[m], dc, A.keys), s_tab, e02, e13);
+          if (!FULL) {
+            e02 = make_float2(u0 ? e02.x : 0.0f, u2 ? e02.y : 0.0f);
+            e13 = make_float2(u1 ? e13.x : 0.0f, u3 ? e13.y : 0.0f);
+          }
+          n[m][0] = e02.x;
+          n[m][1] = e13.x;
+          n[m][2] = e02.y;
+          n[m][3] = e13.y;
+          s2 = __ffma2_rn(p02, expm1_small_x2<DEG>(e02), s2);
+          s2 = __ffma2_rn(p13, expm1_small_x2<DEG>(e13), s2);
+        }
+        s = s2.x + s2.y;
+      } else if (local) {
+        const float* pw = sp + (cw - lo) + lane;
+        float pv[NB][4];
+#pragma unroll
+        for (int m = 0; m < NB; ++m)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int k = m * 128 + lane + 32 * j;
+            pv[m][j] = (FULL || k < S) ? pw[m * 128 + 32 * j] : 0.0f;
+          }
+#pragma unroll
+        for (int m = 0; m < NB; ++m) {
+          const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int k = m * 128 + lane + 32 * j;
+            const float x = (FULL || k < S) ? g.v[j] : 0.0f;
+            n[m][j] = x;
+            s = fmaf(pv[m][j], expm1_small<DEG>(x), s);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < NB; ++m) {
+          const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int k = m * 128 + lane + 32 * j;
+            float x = 0.0f;
+            if (FULL || k < S) {
+              uint32_t q = cw + (uint32_t)k;
+              if (q >= V) q -= V;
+              const float pq = (q >= lo && q < hi) ? sp[q - lo] : sp_peer[q - lo_peer];
+              x = g.v[j];
+              s = fmaf(pq, expm1_small<DEG>(x), s);
+            }
+            n[m][j] = x;
+          }
         }
       }
-      uint32_t mask = __ballot_sync(0xffffffffu, mine);
-      while (mask) {
-        const int src = __ffs(mask) - 1;
-        mask &= mask - 1;
-        const int i = bidx * 32 + src;
-        const uint32_t cw = __shfl_sync(0xffffffffu, c, src);
-        const uint32_t ky = __shfl_sync(0xffffffffu, kyq, src);
-        const float xe = __shfl_sync(0xffffffffu, x_extra, src);
-        const DrawConst dc = draw_const(A.keys, t_abs, A.i_off + (uint32_t)i);
-        const bool in_win = ky < (uint32_t)S;
-        const bool local = (cw + (uint32_t)S) <= hi;  // whole window in this slice
-        float n[NB][4];  // sigma * eps of the draw's slots
-        float s = 0.0f;
-        if (local) {
-          const float* pw = sp + (cw - lo) + lane;
-          float pv[NB][4];
+      float xy;
+      if (in_win) {
+        const int my = (int)(ky >> 7), jy = (int)((ky >> 5) & 3u);
+        const bool owner = lane == (int)(ky & 31u);
+        float cand = 0.0f;
 #pragma unroll
-          for (int m = 0; m < NB; ++m)
+        for (int m = 0; m < NB; ++m)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int k = m * 128 + lane + 32 * j;
-              pv[m][j] = (FULL || k < S) ? pw[m * 128 + 32 * j] : 0.0f;
+          for (int j = 0; j < 4; ++j)
+            if (m == my && j == jy) {
+              cand = n[m][j];
+              // INT: the target coordinate is accumulated in fp32 below
+              if (INT && owner) n[m][j] = 0.0f;
             }
+        xy = __shfl_sync(0xffffffffu, cand, (int)(ky & 31u));
+      } else {
+        xy = xe;
+        if (lane == 0) s = fmaf(py, expm1_small<DEG>(xy), s);
+      }
+      // a series expm1 bounds |s| by e^0.06 - 1: the fixed-point warp sum applies
+      s = DEG != 0 ? warp_sum_fixed34(s) : warp_sum(s);
+      const float r = xy - log1p_small(s);
+      if (A.rewards && lane == 0) A.rewards[t * A.K + i] = r;
+      if (local && INT && kPacked) {
+        // fixed point as in accumulate<true>, two slots per packed FMA
+        float* gw = sg + (cw - lo) + lane;
+        const float ra = r * A.acc_scale;
+        const float2 ra2 = make_float2(ra, ra), bias = make_float2(12582912.0f, 12582912.0f);
 #pragma unroll
-          for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
+        for (int m = 0; m < NB; ++m) {
+          const int k0 = m * 128 + lane;
+          const float2 a02 = __ffma2_rn(ra2, make_float2(n[m][0], n[m][2]), bias);
+          const float2 a13 = __ffma2_rn(ra2, make_float2(n[m][1], n[m][3]), bias);
+          int* g = reinterpret_cast<int*>(gw + m * 128);
+          if (FULL || k0 < S) atomicAdd(g, __float_as_int(a02.x) - 0x4B400000);
+          if (FULL || k0 + 32 < S) atomicAdd(g + 32, __float_as_int(a13.x) - 0x4B400000);
+          if (FULL || k0 + 64 < S) atomicAdd(g + 64, __float_as_int(a02.y) - 0x4B400000);
+          if (FULL || k0 + 96 < S) atomicAdd(g + 96, __float_as_int(a13.y) - 0x4B400000);
+        }
+      } else if (local) {
+        float* gw = sg + (cw - lo) + lane;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int k = m * 128 + lane + 32 * j;
-              const float x = (FULL || k < S) ? g.v[j] : 0.0f;
-              n[m][j] = x;
-              s = fmaf(pv[m][j], expm1_small<DEG>(x), s);
+        for (int m = 0; m < NB; ++m)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int k = m * 128 + lane + 32 * j;
+            if (FULL || k < S) accumulate<INT>(gw + m * 128 + 32 * j, r, n[m][j], A.acc_scale);
+          }
+      } else {
+#pragma unroll
+        for (int m = 0; m < NB; ++m)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int k = m * 128 + lane + 32 * j;
+            if (FULL || k < S) {
+              uint32_t q = cw + (uint32_t)k;
+              if (q >= V) q -= V;
+              float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - lo_peer);
+              accumulate<INT>(dst, r, n[m][j], A.acc_scale);
             }
           }
-        } else {
-#pragma unroll
-          for (int m = 0; m < NB; ++m) {
-            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int k = m * 128 + lane + 32 * j;
-              float x = 0.0f;
-              if (FULL || k < S) {
-                uint32_t q = cw + (uint32_t)k;
-                if (q >= V) q -= V;
-                const float pq = (q >= lo && q < hi) ? sp[q - lo] : sp_peer[q - lo_peer];
-                x = g.v[j];
-                s = fmaf(pq, expm1_small<DEG>(x), s);
-              }
-              n[m][j] = x;
-            }
-          }
-        }
-        float xy;
-        if (in_win) {
-          const int my = (int)(ky >> 7), jy = (int)((ky >> 5) & 3u);
-          const bool owner = lane == (int)(ky & 31u);
-          float cand = 0.0f;
-#pragma unroll
-          for (int m = 0; m < NB; ++m)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (m == my && j == jy) {
-                cand = n[m][j];
-                // INT: the target coordinate is accumulated in fp32 below
-                if (INT && owner) n[m][j] = 0.0f;
-              }
-          xy = __shfl_sync(0xffffffffu, cand, (int)(ky & 31u));
-        } else {
-          xy = xe;
-          if (lane == 0) s = fmaf(py, expm1_small<DEG>(xy), s);
-        }
-        s = warp_sum(s);
-        const float r = xy - log1p_small(s);
-        if (A.rewards && lane == 0) A.rewards[t * A.K + i] = r;
-        if (local) {
-          float* gw = sg + (cw - lo) + lane;
-#pragma unroll
-          for (int m = 0; m < NB; ++m)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int k = m * 128 + lane + 32 * j;
-              if (FULL || k < S) accumulate<INT>(gw + m * 128 + 32 * j, r, n[m][j], A.acc_scale);
-            }
-        } else {
-#pragma unroll
-          for (int m = 0; m < NB; ++m)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int k = m * 128 + lane + 32 * j;
-              if (FULL || k < S) {
-                uint32_t q = cw + (uint32_t)k;
-                if (q >= V) q -= V;
-                float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - lo_peer);
-                accumulate<INT>(dst, r, n[m][j], A.acc_scale);
-              }
-            }
-        }
-        if (INT) {
-          if (lane == 0) tgt_acc = fmaf(r, xy, tgt_acc);
-        } else if (!in_win && lane == 0) {
-          atomicAdd(gy, r * xy);
+      }
+      if (INT) {
+        if (lane == 0) tgt_acc = fmaf(r, xy, tgt_acc);
+      } else if (!in_win && lane == 0) {
+        atomicAdd(gy, r * xy);
+      }
+    };
+    if constexpr (LIST) {
+      __shared__ uint4 s_list[kListCap];
+      for (int iq = threadIdx.x; iq < A.K; iq += kThreads) {
+        uint32_t c, kyq;
+        float x_extra;
+        if (setup(iq, c, kyq, x_extra))
+          s_list[atomicAdd(&s_cnt, 1)] = make_uint4((uint32_t)iq, c, kyq, __float_as_uint(x_extra));
+      }
+      __syncthreads();
+      const int cnt = s_cnt;
+      for (;;) {
+        int idx = 0;
+        if (lane == 0) idx = atomicAdd(&s_next, 1);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx >= cnt) break;
+        const uint4 e = s_list[idx];
+        draw((int)e.x, e.y, e.z, __uint_as_float(e.w));
+      }
+    } else {
+      for (;;) {
+        int bidx = 0;
+        if (lane == 0) bidx = atomicAdd(&s_next, 1);
+        bidx = __shfl_sync(0xffffffffu, bidx, 0);
+        if (bidx >= nbatch) break;
+        const int iq = bidx * 32 + lane;
+        uint32_t c = 0, kyq = 0;
+        float x_extra = 0.0f;
+        const bool mine = iq < A.K && setup(iq, c, kyq, x_extra);
+        uint32_t mask = __ballot_sync(0xffffffffu, mine);
+        while (mask) {
+          const int src = __ffs(mask) - 1;
+          mask &= mask - 1;
+          draw(bidx * 32 + src, __shfl_sync(0xffffffffu, c, src), __shfl_sync(0xffffffffu, kyq, src),
+               __shfl_sync(0xffffffffu, x_extra, src));
         }
       }
     }
-    if (INT && lane == 0) atomicAdd(own_y ? &s_tgt : tgt_peer, tgt_acc);
-    if (CS > 1) cluster.sync(); else __syncthreads();
+    if (INT && lane == 0) atomicAdd(cluster.map_shared_rank(&s_tgt, owner_y), tgt_acc);
+    cluster.sync();
 
     // ---- scale and write the owned slice of g
     for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
@@ -316,76 +403,82 @@ __global__ __launch_bounds__(sub2_threads(CS, INT), 1) void k_subset2(const __gr
         store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + qg, v);
       else
         ((float*)A.gop)[t * A.V + qg] = v;
-      if (A.g_out) A.g_out[t * A.V + mulmod32(qg, A.a, V, A.minv)] = v;
+      if (A.g_out) A.g_out[t * A.V + mulmod(qg, A.a, V, A.minv)] = v;
     }
     __syncthreads();
   }
-  if (CS > 1) cluster.sync();
+  cluster.sync();
 }
 
-template <int CS, int NB, bool FULL, int DEG, bool INT>
+template <int NB, bool FULL, int DEG, bool INT, bool LIST>
 cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_count) {
-  auto fn = k_subset2<CS, NB, FULL, DEG, INT>;
+  auto fn = k_subset2<NB, FULL, DEG, INT, LIST>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  const int cs = (int)A.cs;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(sub2_threads(CS, INT));
+  cfg.blockDim = dim3(sub2_threads(INT, DEG));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int max_clusters = sm_count / CS;
-  cfg.gridDim = dim3((unsigned)(max_clusters * CS));
+  int max_clusters = sm_count / cs;
+  cfg.gridDim = dim3((unsigned)(max_clusters * cs));
   int active = 0;
   if (cudaOccupancyMaxActiveClusters(&active, (void*)fn, &cfg) == cudaSuccess && active > 0)
     max_clusters = active;
   cudaGetLastError();
   int64_t nc = A.T < max_clusters ? A.T : max_clusters;
-  cfg.gridDim = dim3((unsigned)(nc * CS));
+  cfg.gridDim = dim3((unsigned)(nc * cs));
   e = cudaLaunchKernelEx(&cfg, fn, A);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-template <int CS, int NB, bool FULL, bool INT>
+template <int NB, bool FULL, bool INT, bool LIST>
 cudaError_t launch_deg(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
-  if (deg == 3) return launch_one<CS, NB, FULL, 3, INT>(st, A, smem, sm);
-  if (deg == 4) return launch_one<CS, NB, FULL, 4, INT>(st, A, smem, sm);
-  return launch_one<CS, NB, FULL, 0, INT>(st, A, smem, sm);
+  if (deg == 3) return launch_one<NB, FULL, 3, INT, LIST>(st, A, smem, sm);
+  if (deg == 4) return launch_one<NB, FULL, 4, INT, LIST>(st, A, smem, sm);
+  return launch_one<NB, FULL, 0, INT, LIST>(st, A, smem, sm);
 }
 
-template <int CS, bool INT>
+template <bool INT, bool LIST>
 cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
   const int nb = (A.S + 127) / 128;
   const bool full = (A.S % 128) == 0;
   switch (nb) {
-    case 1: return full ? launch_deg<CS, 1, true, INT>(st, A, smem, sm, deg) : launch_deg<CS, 1, false, INT>(st, A, smem, sm, deg);
-    case 2: return full ? launch_deg<CS, 2, true, INT>(st, A, smem, sm, deg) : launch_deg<CS, 2, false, INT>(st, A, smem, sm, deg);
-    case 3: return launch_deg<CS, 3, false, INT>(st, A, smem, sm, deg);
-    case 4: return full ? launch_deg<CS, 4, true, INT>(st, A, smem, sm, deg) : launch_deg<CS, 4, false, INT>(st, A, smem, sm, deg);
+    case 1: return full ? launch_deg<1, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<1, false, INT, LIST>(st, A, smem, sm, deg);
+    case 2: return full ? launch_deg<2, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<2, false, INT, LIST>(st, A, smem, sm, deg);
+    case 3: return launch_deg<3, false, INT, LIST>(st, A, smem, sm, deg);
+    case 4: return full ? launch_deg<4, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<4, false, INT, LIST>(st, A, smem, sm, deg);
     default: return cudaErrorNotSupported;
   }
 }
 
-template <int CS>
-cudaError_t launch_cs(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg, bool use_int) {
-  return use_int ? launch_nb<CS, true>(st, A, smem, sm, deg) : launch_nb<CS, false>(st, A, smem, sm, deg);
-}
+// q-slice length of one CTA of a cs-CTA cluster (a multiple of 4, so rows
+// start 16-byte aligned in shared memory).
+int64_t slice_len(int64_t V, int cs) { return ((V + cs - 1) / cs + 3) / 4 * 4; }
 
 }  // namespace
 
-// Cluster size the shared-memory kernel would use (0: not applicable).
+// Cluster size the shared-memory kernel would use (0: not applicable): the
+// smallest of 1, 2, 4, 8 whose slices (p and g, 4 bytes each) fit in shared
+// memory, with every slice at least S long, so that a window reaches at most
+// the next slice.
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
-  if (S < 1 || S > 512) return 0;
-  const int64_t slack = 1024 + 8 * kSinCosTable;  // static: counters, angle table
-  if (2 * V * 4 + slack <= max_smem_optin && V <= 65536) return 1;
-  const int64_t seg = ((V + 1) / 2 + 3) / 4 * 4;
-  if (2 * seg * 4 + slack <= max_smem_optin && S <= V - seg && S <= seg && V <= 65536) return 2;
+  if (S < 1 || S > 512 || V >= (1LL << 31)) return 0;
+  for (int cs = 1; cs <= 8; cs *= 2) {
+    const int64_t seg = slice_len(V, cs);
+    const int64_t last = V - (cs - 1) * seg;  // the last (shortest) slice
+    if (2 * seg * 4 + kStaticSmem > max_smem_optin) continue;
+    if (cs > 1 && (S > seg || S > last)) continue;
+    return cs;
+  }
   return 0;
 }
 
@@ -408,8 +501,9 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.S = p.S;
   A.a = (uint32_t)a;
   A.a_inv = (uint32_t)a_inv;
-  A.minv = (uint32_t)(0xffffffffull / (uint64_t)p.V);
-  A.seg = cs == 1 ? (uint32_t)((p.V + 3) / 4 * 4) : (uint32_t)(((p.V + 1) / 2 + 3) / 4 * 4);
+  A.minv = ~0ull / (uint64_t)p.V;
+  A.cs = (uint32_t)cs;
+  A.seg = (uint32_t)slice_len(p.V, cs);
   A.scale_other = (float)((double)p.V / (double)p.S);
   A.scale_target = (p.flags & DUST_FLAG_LITERAL_TARGET_SCALE) ? A.scale_other : 1.0f;
   // the accumulators hold sum r (sigma eps): g = -(1/(K sigma)) sum r eps
@@ -430,8 +524,12 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   const size_t smem = (size_t)2 * A.seg * 4;
   const int deg = expm1_degree(p.sigma);
   const bool use_int = p.K <= 65536;
-  if (cs == 1) return launch_cs<1>(st, A, smem, sm_count, deg, use_int);
-  return launch_cs<2>(st, A, smem, sm_count, deg, use_int);
+  if (!use_int) return launch_nb<false, false>(st, A, smem, sm_count, deg);
+  // the list of a token's draws, when it fits beside the slices
+  const bool list = p.K <= kListCap &&
+                    (int64_t)smem + kStaticSmem + kListCap * 16 <= (int64_t)max_smem_optin;
+  return list ? launch_nb<true, true>(st, A, smem, sm_count, deg)
+              : launch_nb<true, false>(st, A, smem, sm_count, deg);
 }
 
 }  // namespace dust

@@ -181,6 +181,35 @@ __device__ __forceinline__ G4 gauss4_tab(U4 w, const float2* tab) {
   return g;
 }
 
+// gauss4_tab with the two Box-Muller pairs of the counter, (w.x, w.y) and
+// (w.z, w.w), computed side by side in packed fp32x2 arithmetic (one
+// instruction per pair of operations; each lane of a packed operation rounds
+// as the scalar one does): the same operations on the same values in the same
+// order, so the results equal gauss4_tab's bit for bit. e02 holds words 0 and
+// 2 (the cosine outputs of the two pairs), e13 words 1 and 3 (the sines).
+__device__ __forceinline__ void gauss4_tab_x2(U4 w, const float2* tab, float2& e02, float2& e13) {
+  const float2 k24 = make_float2(5.9604645e-08f, 5.9604645e-08f);
+  const float2 u = __ffma2_rn(make_float2((float)(w.x >> 8), (float)(w.z >> 8)), k24, k24);
+  const float2 v = __ffma2_rn(u, make_float2(-1.0f, -1.0f), make_float2(1.0f, 1.0f));  // 1 - u
+  float2 near = __ffma2_rn(v, make_float2(-0.48089835f, -0.48089835f),
+                           make_float2(-0.7213475f, -0.7213475f));
+  near = __ffma2_rn(v, near, make_float2(-1.442695f, -1.442695f));
+  near = __fmul2_rn(v, near);
+  const float2 rho = make_float2(sqrt_approx(-(v.x < 0.015625f ? near.x : lg2_approx(u.x))),
+                                 sqrt_approx(-(v.y < 0.015625f ? near.y : lg2_approx(u.y))));
+  const float2 F = make_float2(__int_as_float((w.y & 0x003FFF00u) | 0x4B400000u),
+                               __int_as_float((w.w & 0x003FFF00u) | 0x4B400000u));
+  const float2 x = __ffma2_rn(F, make_float2(1.4629181e-09f, 1.4629181e-09f),
+                              make_float2(-0.021475732f, -0.021475732f));
+  const float2 nx = __ffma2_rn(F, make_float2(-1.4629181e-09f, -1.4629181e-09f),
+                               make_float2(0.021475732f, 0.021475732f));  // -x, exactly
+  const float2 q = __ffma2_rn(__fmul2_rn(x, x), make_float2(-0.5f, -0.5f), make_float2(1.0f, 1.0f));
+  const float2 ta = tab[w.y >> 22], tb = tab[w.w >> 22];
+  const float2 c = make_float2(ta.x, tb.x), s = make_float2(ta.y, tb.y);
+  e02 = __fmul2_rn(rho, __ffma2_rn(s, nx, __fmul2_rn(c, q)));
+  e13 = __fmul2_rn(rho, __ffma2_rn(c, x, __fmul2_rn(s, q)));
+}
+
 __device__ __forceinline__ G4 gauss4(U4 w, float scale = 1.0f) {
   const float2 a = box_muller(w.x, w.y, scale);
   const float2 b = box_muller(w.z, w.w, scale);
@@ -317,6 +346,41 @@ __device__ __forceinline__ float expm1_small(float x) {
   } else {
     return expm1f(x);
   }
+}
+
+// expm1_small of a pair, in packed fp32x2 arithmetic (the same operations per
+// lane as the scalar form).
+template <int DEG>
+__device__ __forceinline__ float2 expm1_small_x2(float2 x) {
+  if constexpr (DEG == 3) {
+    float2 q = __ffma2_rn(x, make_float2(1.0f / 6.0f, 1.0f / 6.0f), make_float2(0.5f, 0.5f));
+    q = __ffma2_rn(x, q, make_float2(1.0f, 1.0f));
+    return __fmul2_rn(x, q);
+  } else if constexpr (DEG == 4) {
+    float2 q = __ffma2_rn(x, make_float2(1.0f / 24.0f, 1.0f / 24.0f),
+                          make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+    q = __ffma2_rn(x, q, make_float2(0.5f, 0.5f));
+    q = __ffma2_rn(x, q, make_float2(1.0f, 1.0f));
+    return __fmul2_rn(x, q);
+  } else if constexpr (DEG == 5) {
+    float2 q = __ffma2_rn(x, make_float2(1.0f / 120.0f, 1.0f / 120.0f),
+                          make_float2(1.0f / 24.0f, 1.0f / 24.0f));
+    q = __ffma2_rn(x, q, make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+    q = __ffma2_rn(x, q, make_float2(0.5f, 0.5f));
+    q = __ffma2_rn(x, q, make_float2(1.0f, 1.0f));
+    return __fmul2_rn(x, q);
+  } else {
+    return make_float2(expm1f(x.x), expm1f(x.y));
+  }
+}
+
+// Sum over the warp (all lanes get it) of values whose magnitudes add up to
+// less than 2^-3: each rounded to 2^-34 fixed point, the integers added
+// exactly by the warp-reduction unit (no overflow below 2^31), the sum scaled
+// back. The rounding moves each lane's share by at most 2^-35.
+__device__ __forceinline__ float warp_sum_fixed34(float v) {
+  const int q = __float2int_rn(v * 17179869184.0f);  // 2^34
+  return (float)__reduce_add_sync(0xffffffffu, q) * 5.8207661e-11f;  // 2^-34
 }
 
 // Degree of expm1_small for noise of scale sigma (|eps| <= sqrt(48 ln 2) = 5.7686).
