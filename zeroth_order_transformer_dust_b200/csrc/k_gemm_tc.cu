@@ -239,11 +239,42 @@ __device__ __forceinline__ float expm1_guarded(float x) {
 // sum_n P[t, n] expm1(dz_n) and records dz at the target column. prow points
 // at P[t, n]: a staged shared-memory copy (zero past column N) when `staged`,
 // else the row in global memory.
+// The degree-5 series of expm1_guarded for a pair, in packed fp32x2
+// arithmetic (each lane rounds as the scalar form does).
+__device__ __forceinline__ float2 expm1_series5_x2(float2 x) {
+  float2 q = __ffma2_rn(x, make_float2(1.0f / 120.0f, 1.0f / 120.0f),
+                        make_float2(1.0f / 24.0f, 1.0f / 24.0f));
+  q = __ffma2_rn(x, q, make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+  q = __ffma2_rn(x, q, make_float2(0.5f, 0.5f));
+  q = __ffma2_rn(x, q, make_float2(1.0f, 1.0f));
+  return __fmul2_rn(x, q);
+}
+
 __device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int32_t yt, int64_t n,
                                           const float* prow, bool staged, const float* v) {
   // four independent sums, so the adds do not form one 32-long chain
   float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-  if (staged || (n + 32 <= p.N && (p.N & 3) == 0)) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) amax = fmaxf(amax, fabsf(v[q]));
+  if (amax < 0.0625f && (staged || (n + 32 <= p.N && (p.N & 3) == 0))) {
+    // every |dz| of the lane's 32 columns in the series' range (the usual
+    // case): the series alone, two columns per packed operation
+    float2 sa = make_float2(0.0f, 0.0f), sb = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 pv = staged ? reinterpret_cast<const float4*>(prow)[q]
+                               : __ldg(reinterpret_cast<const float4*>(prow) + q);
+      sa = __ffma2_rn(make_float2(pv.x, pv.y),
+                      expm1_series5_x2(make_float2(v[4 * q + 0], v[4 * q + 1])), sa);
+      sb = __ffma2_rn(make_float2(pv.z, pv.w),
+                      expm1_series5_x2(make_float2(v[4 * q + 2], v[4 * q + 3])), sb);
+    }
+    s0 = sa.x;
+    s1 = sa.y;
+    s2 = sb.x;
+    s3 = sb.y;
+  } else if (staged || (n + 32 <= p.N && (p.N & 3) == 0)) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const float4 pv = staged ? reinterpret_cast<const float4*>(prow)[q]

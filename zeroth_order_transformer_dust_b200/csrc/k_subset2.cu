@@ -58,11 +58,15 @@ __host__ __device__ constexpr int sub2_threads(bool use_int, int deg) {
   return use_int && deg != 0 ? 1024 : 512;
 }
 
-// Draws of one token the shared list holds (16 bytes each). With K <= kListCap
-// every draw of a token is set up once per CTA up front and the warps take the
-// CTA's draws one at a time, so a token's work splits evenly however the
-// window starts fall; with more draws the warps take batches of 32 as they go.
-constexpr int kListCap = 1024;
+// The Box-Muller step of NB-block draws in packed fp32x2 form, else scalar
+// and paired up afterwards for the packed expm1 and accumulation. The packed
+// operations run on the FMA-heavy pipe, which the Philox multiplies already
+// load, so the scalar step (whose operations also use the FMA-lite pipe) is
+// the faster one (0.3-0.7% on B200); at NB = 3 it needs more than the 64
+// registers of a 1024-thread CTA, and those variants take the packed form.
+template <int NB>
+constexpr bool packed_generator() { return NB == 3; }
+
 constexpr int64_t kStaticSmem = 1024 + 8 * kSinCosTable;  // counters, angle table
 
 struct Sub2Args {
@@ -114,15 +118,12 @@ __device__ __forceinline__ void accumulate(float* slot, float r, float x, float 
     atomicAdd(slot, r * x);
 }
 
-// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB; LIST: the
-// draws of a token are set up together and taken from a shared list one at a
-// time (K <= kListCap), else taken in batches of 32.
-template <int NB, bool FULL, int DEG, bool INT, bool LIST>
+// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
+template <int NB, bool FULL, int DEG, bool INT>
 __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
   constexpr int kThreads = sub2_threads(INT, DEG);
   extern __shared__ __align__(16) float smem[];
-  __shared__ int s_next;    // next draw batch (or list entry) of the current token
-  __shared__ int s_cnt;     // LIST: entries of the current token's list
+  __shared__ int s_next;    // next draw batch of the current token
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
   __shared__ float2 s_tab[kSinCosTable];
   fill_sincos_table(s_tab, A.sigma);
@@ -174,7 +175,6 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
     }
     if (threadIdx.x == 0) {
       s_next = 0;
-      s_cnt = 0;
       s_tgt = 0.0f;
     }
     int32_t yt = A.y[t];
@@ -229,7 +229,13 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
           const float2 p02 = make_float2(u0 ? pw[m * 128] : 0.0f, u2 ? pw[m * 128 + 64] : 0.0f);
           const float2 p13 = make_float2(u1 ? pw[m * 128 + 32] : 0.0f, u3 ? pw[m * 128 + 96] : 0.0f);
           float2 e02, e13;
-          gauss4_tab_x2(philox_from2(bc[m], dc, A.keys), s_tab, e02, e13);
+          if (packed_generator<NB>()) {
+            gauss4_tab_x2(philox_from2(bc[m], dc, A.keys), s_tab, e02, e13);
+          } else {
+            const G4 g = gauss4_tab(philox_from2(bc[m], dc, A.keys), s_tab);
+            e02 = make_float2(g.v[0], g.v[2]);
+            e13 = make_float2(g.v[1], g.v[3]);
+          }
           if (!FULL) {
             e02 = make_float2(u0 ? e02.x : 0.0f, u2 ? e02.y : 0.0f);
             e13 = make_float2(u1 ? e13.x : 0.0f, u3 ? e13.y : 0.0f);
@@ -350,41 +356,21 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
         atomicAdd(gy, r * xy);
       }
     };
-    if constexpr (LIST) {
-      __shared__ uint4 s_list[kListCap];
-      for (int iq = threadIdx.x; iq < A.K; iq += kThreads) {
-        uint32_t c, kyq;
-        float x_extra;
-        if (setup(iq, c, kyq, x_extra))
-          s_list[atomicAdd(&s_cnt, 1)] = make_uint4((uint32_t)iq, c, kyq, __float_as_uint(x_extra));
-      }
-      __syncthreads();
-      const int cnt = s_cnt;
-      for (;;) {
-        int idx = 0;
-        if (lane == 0) idx = atomicAdd(&s_next, 1);
-        idx = __shfl_sync(0xffffffffu, idx, 0);
-        if (idx >= cnt) break;
-        const uint4 e = s_list[idx];
-        draw((int)e.x, e.y, e.z, __uint_as_float(e.w));
-      }
-    } else {
-      for (;;) {
-        int bidx = 0;
-        if (lane == 0) bidx = atomicAdd(&s_next, 1);
-        bidx = __shfl_sync(0xffffffffu, bidx, 0);
-        if (bidx >= nbatch) break;
-        const int iq = bidx * 32 + lane;
-        uint32_t c = 0, kyq = 0;
-        float x_extra = 0.0f;
-        const bool mine = iq < A.K && setup(iq, c, kyq, x_extra);
-        uint32_t mask = __ballot_sync(0xffffffffu, mine);
-        while (mask) {
-          const int src = __ffs(mask) - 1;
-          mask &= mask - 1;
-          draw(bidx * 32 + src, __shfl_sync(0xffffffffu, c, src), __shfl_sync(0xffffffffu, kyq, src),
-               __shfl_sync(0xffffffffu, x_extra, src));
-        }
+    for (;;) {
+      int bidx = 0;
+      if (lane == 0) bidx = atomicAdd(&s_next, 1);
+      bidx = __shfl_sync(0xffffffffu, bidx, 0);
+      if (bidx >= nbatch) break;
+      const int iq = bidx * 32 + lane;
+      uint32_t c = 0, kyq = 0;
+      float x_extra = 0.0f;
+      const bool mine = iq < A.K && setup(iq, c, kyq, x_extra);
+      uint32_t mask = __ballot_sync(0xffffffffu, mine);
+      while (mask) {
+        const int src = __ffs(mask) - 1;
+        mask &= mask - 1;
+        draw(bidx * 32 + src, __shfl_sync(0xffffffffu, c, src), __shfl_sync(0xffffffffu, kyq, src),
+             __shfl_sync(0xffffffffu, x_extra, src));
       }
     }
     if (INT && lane == 0) atomicAdd(cluster.map_shared_rank(&s_tgt, owner_y), tgt_acc);
@@ -410,9 +396,9 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
   cluster.sync();
 }
 
-template <int NB, bool FULL, int DEG, bool INT, bool LIST>
+template <int NB, bool FULL, int DEG, bool INT>
 cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_count) {
-  auto fn = k_subset2<NB, FULL, DEG, INT, LIST>;
+  auto fn = k_subset2<NB, FULL, DEG, INT>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int cs = (int)A.cs;
@@ -440,22 +426,22 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
   return cudaGetLastError();
 }
 
-template <int NB, bool FULL, bool INT, bool LIST>
+template <int NB, bool FULL, bool INT>
 cudaError_t launch_deg(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
-  if (deg == 3) return launch_one<NB, FULL, 3, INT, LIST>(st, A, smem, sm);
-  if (deg == 4) return launch_one<NB, FULL, 4, INT, LIST>(st, A, smem, sm);
-  return launch_one<NB, FULL, 0, INT, LIST>(st, A, smem, sm);
+  if (deg == 3) return launch_one<NB, FULL, 3, INT>(st, A, smem, sm);
+  if (deg == 4) return launch_one<NB, FULL, 4, INT>(st, A, smem, sm);
+  return launch_one<NB, FULL, 0, INT>(st, A, smem, sm);
 }
 
-template <bool INT, bool LIST>
+template <bool INT>
 cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
   const int nb = (A.S + 127) / 128;
   const bool full = (A.S % 128) == 0;
   switch (nb) {
-    case 1: return full ? launch_deg<1, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<1, false, INT, LIST>(st, A, smem, sm, deg);
-    case 2: return full ? launch_deg<2, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<2, false, INT, LIST>(st, A, smem, sm, deg);
-    case 3: return launch_deg<3, false, INT, LIST>(st, A, smem, sm, deg);
-    case 4: return full ? launch_deg<4, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<4, false, INT, LIST>(st, A, smem, sm, deg);
+    case 1: return full ? launch_deg<1, true, INT>(st, A, smem, sm, deg) : launch_deg<1, false, INT>(st, A, smem, sm, deg);
+    case 2: return full ? launch_deg<2, true, INT>(st, A, smem, sm, deg) : launch_deg<2, false, INT>(st, A, smem, sm, deg);
+    case 3: return launch_deg<3, false, INT>(st, A, smem, sm, deg);
+    case 4: return full ? launch_deg<4, true, INT>(st, A, smem, sm, deg) : launch_deg<4, false, INT>(st, A, smem, sm, deg);
     default: return cudaErrorNotSupported;
   }
 }
@@ -524,12 +510,8 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   const size_t smem = (size_t)2 * A.seg * 4;
   const int deg = expm1_degree(p.sigma);
   const bool use_int = p.K <= 65536;
-  if (!use_int) return launch_nb<false, false>(st, A, smem, sm_count, deg);
-  // the list of a token's draws, when it fits beside the slices
-  const bool list = p.K <= kListCap &&
-                    (int64_t)smem + kStaticSmem + kListCap * 16 <= (int64_t)max_smem_optin;
-  return list ? launch_nb<true, true>(st, A, smem, sm_count, deg)
-              : launch_nb<true, false>(st, A, smem, sm_count, deg);
+  return use_int ? launch_nb<true>(st, A, smem, sm_count, deg)
+                 : launch_nb<false>(st, A, smem, sm_count, deg);
 }
 
 }  // namespace dust
