@@ -22,12 +22,14 @@ constexpr int kWarps = 8;
 constexpr int kBlocksPerWarp = 4;                     // 128-slot blocks per warp
 constexpr int kSlab = kWarps * kBlocksPerWarp * 128;  // vocabulary entries per unit
 constexpr int kDrawChunk = 64;
-// The Box-Muller step in packed fp32x2 form (else scalar, paired up for the
-// packed expm1 and accumulation).
-constexpr bool kPackedGenerator = true;
-
+// The Box-Muller step in packed fp32x2 form (PACKED) or scalar and paired up
+// afterwards. Packed operations run on the FMA-heavy pipe, which the Philox
+// multiplies also need: measured on B200, the reward pass (with its packed
+// expm1 and sums) is faster with the packed step (15.5 against 15.9 ms on
+// full_bf16), the g pass with the scalar one (12.3 against 12.5 ms).
+template <bool PACKED>
 __device__ __forceinline__ void noise4(U4 w, const float2* tab, float2& e02, float2& e13) {
-  if (kPackedGenerator) {
+  if (PACKED) {
     gauss4_tab_x2(w, tab, e02, e13);
   } else {
     const G4 g = gauss4_tab(w, tab);
@@ -89,7 +91,7 @@ __device__ __forceinline__ void reward_chunk(const FullArgs& A, const float2* ta
       sb[b] = 0.0f;
       if (ALL || b < nvalid) {
         float2 e02, e13;
-        noise4(philox_from2(bc[b], dc, A.keys), tab, e02, e13);
+        noise4<true>(philox_from2(bc[b], dc, A.keys), tab, e02, e13);
         float2 s2 = __fmul2_rn(p02[b], expm1_small_x2<DEG>(e02));
         s2 = __ffma2_rn(p13[b], expm1_small_x2<DEG>(e13), s2);
         sb[b] = s2.x + s2.y;
@@ -196,7 +198,7 @@ __device__ __forceinline__ void g_chunk(const FullArgs& A, const float2* tab, in
     for (int b = 0; b < kBlocksPerWarp; ++b) {
       if (ALL || b < nvalid) {
         float2 e02, e13;
-        noise4(philox_from2(bc[b], dc, A.keys), tab, e02, e13);
+        noise4<false>(philox_from2(bc[b], dc, A.keys), tab, e02, e13);
         acc02[b] = __ffma2_rn(r2, e02, acc02[b]);
         acc13[b] = __ffma2_rn(r2, e13, acc13[b]);
       }
