@@ -333,6 +333,14 @@ dust_status dust_sgd_momentum(dust_ctx* ctx, int64_t n, float lr, float mu, cons
    undefined (the context stays usable). Synchronous. */
 dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* A,
                                  const void* B, float* C, int path);
+/* Debug: the same product with both operands stored MN-major: At (K x M,
+   bf16, row-major) and Bt (K x N), C (M x N, fp32) = At^T Bt. The tensor-core
+   paths read the K x M and K x N rows as stored (M and N multiples of 8 are
+   needed for 16-byte rows; else paths 2 and 3 return DUST_ERR_UNSUPPORTED
+   and path 0 runs on CUDA cores). Paths and errors as dust_debug_gemm_bf16.
+   This is the layout of the weight-gradient contraction sum_t g_t x_t^T. */
+dust_status dust_debug_gemm_bf16_mn(dust_ctx* ctx, int64_t M, int64_t N, int64_t K,
+                                    const void* At, const void* Bt, float* C, int path);
 
 /* Debug: raw Philox4x32-10 words. ctr4 (n x 4 uint32, device) -> out (n x 4). */
 dust_status dust_debug_philox(dust_ctx* ctx, uint64_t seed, const uint32_t* ctr4,

@@ -110,6 +110,19 @@ def test_edge_shapes(ctx, kw):
     _compare(got, ref, TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
 
 
+@pytest.mark.parametrize("kw", [dict(), dict(S=129, K=33), dict(V=4099, S=640, K=40),
+                                dict(T=200, K=5, V=1000), dict(T=300, K=3, V=3001, S=50)])
+def test_single_cta_tensor_core_path(cuda_ok, monkeypatch, kw):
+    """The GEMMs in single-CTA mode (one 128 x 256 tile per SM, fewer operand
+    stages) give the same estimator as the CTA-pair default, on ragged rows
+    and columns."""
+    monkeypatch.setenv("DUST_TC_PAIR", "0")
+    c = dust.Context(0)
+    wl = _small(**kw)
+    H, W, y = _inputs(wl)
+    _compare(_gpu(c, H, W, y, wl), _oracle(H, W, y, wl), TOL_GW_BF16)
+
+
 def _host(x, dtype):
     t = torch.from_numpy(np.ascontiguousarray(x))
     t = t.to(torch.int32) if dtype == "i32" else t.to(torch.bfloat16 if dtype == "bf16" else torch.float32)

@@ -32,7 +32,8 @@ EXPORTS = ("dust_create", "dust_set_stream", "dust_destroy", "dust_last_error",
            "dust_status_string", "dust_validate", "dust_subset_stride", "dust_check",
            "dust_head_grad", "dust_head_grad_host", "dust_mlp_grad", "dust_debug_philox",
            "dust_debug_gauss", "dust_set_stage_timing", "dust_stage_times",
-           "dust_kernel_launches", "dust_debug_gemm_bf16", "dust_debug_gauss_tab",
+           "dust_kernel_launches", "dust_debug_gemm_bf16", "dust_debug_gemm_bf16_mn",
+           "dust_debug_gauss_tab",
            "dust_debug_gauss_tab_scalar",
            "dust_head_grad_noalloc", "dust_debug_bm_radius", "dust_debug_bm_angle",
            "dust_attn_grad",
@@ -103,6 +104,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                 ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
             "dust_kernel_launches": (I64, [P]),
             "dust_debug_gemm_bf16": (I32, [P, I64, I64, I64, P, P, P, ctypes.c_int]),
+            "dust_debug_gemm_bf16_mn": (I32, [P, I64, I64, I64, P, P, P, ctypes.c_int]),
             "dust_debug_gauss_tab": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_debug_gauss_tab_scalar": (I32, [P, PP, I32, I64, I64, I64, P]),
             "dust_head_grad_noalloc": (I32, [PP, P, P, P, P, P, P, P, P, ctypes.c_char_p,
@@ -465,6 +467,21 @@ class Context:
         C = torch.empty(M, N, dtype=torch.float32, device=A.device)
         self._bind_stream()
         self._check(self._L.dust_debug_gemm_bf16(self._h, M, N, K, _ptr(A), _ptr(B), _ptr(C), path))
+        return C
+
+    def debug_gemm_mn(self, At: torch.Tensor, Bt: torch.Tensor, path: int = 0) -> torch.Tensor:
+        """C = At^T Bt for MN-major operands At (K x M) and Bt (K x N), bf16, fp32 out;
+        paths as debug_gemm."""
+        self._dev(At, "At"), self._dev(Bt, "Bt")
+        if At.dtype != torch.bfloat16 or Bt.dtype != torch.bfloat16:
+            raise TypeError("At and Bt must be bfloat16")
+        K, M = _matrix(At, "At")
+        N = _matrix(Bt, "Bt")[1]
+        _shape(Bt, (K, N), "Bt")
+        C = torch.empty(M, N, dtype=torch.float32, device=At.device)
+        self._bind_stream()
+        self._check(self._L.dust_debug_gemm_bf16_mn(self._h, M, N, K, _ptr(At), _ptr(Bt), _ptr(C),
+                                                    path))
         return C
 
     def debug_philox(self, seed: int, ctr: torch.Tensor) -> torch.Tensor:

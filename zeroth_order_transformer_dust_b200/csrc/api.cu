@@ -142,7 +142,9 @@ size_t gop_bytes(int dtype, int64_t T, int64_t width) {
 // out (width x N, fp32) = sum_t g_t x_t^T, row w written at (w * row_mul) mod width
 // when row_mul != 0. gop holds g (T x width) as fp32 or as bf16 hi/lo planes;
 // X is T x N in p.dtype. The bf16 path contracts over 2T (both planes against
-// a duplicated X), on tensor cores after transposing both operands to K-major.
+// a duplicated X) on tensor cores, reading both operands MN-major as they are
+// stored; when their rows are not 16-byte multiples (width or N not a
+// multiple of 8) it transposes them to K-major first.
 dust_status weight_grad(dust_ctx* ctx, const dust_params& p, const void* gop, int64_t width,
                         const void* X, int64_t N, float* out, int64_t row_mul) {
   const int64_t T = p.T;
@@ -159,6 +161,10 @@ dust_status weight_grad(dust_ctx* ctx, const dust_params& p, const void* gop, in
   DUST_TRY(ensure(ctx, ctx->xdup, 2 * xb));
   DUST_CU(cudaMemcpyAsync(ctx->xdup.p, X, xb, cudaMemcpyDeviceToDevice, ctx->stream));
   DUST_CU(cudaMemcpyAsync((char*)ctx->xdup.p + xb, X, xb, cudaMemcpyDeviceToDevice, ctx->stream));
+  GemmDesc s{};
+  s.M = width; s.N = N; s.K = K2; s.A = gop; s.lda = width; s.a_kmajor = false;
+  s.B = ctx->xdup.p; s.ldb = N; s.b_kmajor = false; s.dtype = DUST_BF16;
+  if (!ctx->tc_enabled || tc_gemm_supported(s, e)) return run_gemm(ctx, s, e);
   const int64_t ld = (K2 + 7) / 8 * 8;
   DUST_TRY(ensure(ctx, ctx->gT, (size_t)width * ld * 2));
   DUST_TRY(ensure(ctx, ctx->hT, (size_t)N * ld * 2));
@@ -173,9 +179,6 @@ dust_status weight_grad(dust_ctx* ctx, const dust_params& p, const void* gop, in
     ctx->launches += 2;
     return run_gemm(ctx, g, e);
   }
-  GemmDesc s{};
-  s.M = width; s.N = N; s.K = K2; s.A = gop; s.lda = width; s.a_kmajor = false;
-  s.B = ctx->xdup.p; s.ldb = N; s.b_kmajor = false; s.dtype = DUST_BF16;
   return run_gemm(ctx, s, e);
 }
 
@@ -815,6 +818,22 @@ dust_status dust_debug_gemm_bf16(dust_ctx* ctx, int64_t M, int64_t N, int64_t K,
   GemmDesc g{};
   g.M = M; g.N = N; g.K = K; g.A = A; g.lda = K; g.a_kmajor = true;
   g.B = B; g.ldb = K; g.b_kmajor = true; g.dtype = DUST_BF16;
+  EpiDesc e{};
+  e.kind = kEpiF32; e.C = C; e.ldc = N;
+  DUST_TRY(run_gemm(ctx, g, e, path));
+  return dust_check(ctx);
+}
+
+dust_status dust_debug_gemm_bf16_mn(dust_ctx* ctx, int64_t M, int64_t N, int64_t K, const void* At,
+                                    const void* Bt, float* C, int path) {
+  if (!ctx) return DUST_ERR_ARG;
+  if (M < 1 || N < 1 || K < 1 || !At || !Bt || !C || path < 0 || path > 4)
+    return fail(ctx, DUST_ERR_ARG, "bad gemm arguments");
+  DUST_CU(cudaSetDevice(ctx->device));
+  DUST_CU(cudaMemsetAsync(ctx->d_status, 0, sizeof(uint32_t), ctx->stream));
+  GemmDesc g{};
+  g.M = M; g.N = N; g.K = K; g.A = At; g.lda = M; g.a_kmajor = false;
+  g.B = Bt; g.ldb = N; g.b_kmajor = false; g.dtype = DUST_BF16;
   EpiDesc e{};
   e.kind = kEpiF32; e.C = C; e.ldc = N;
   DUST_TRY(run_gemm(ctx, g, e, path));

@@ -1,5 +1,6 @@
 // Tensor-core GEMM for sm_100a: C = A B^T with bf16 operands and fp32
-// accumulation, A (M x K) and B (N x K) both K-major.
+// accumulation. Each operand is K-major (A as M x K rows, B as N x K) or
+// MN-major (A stored as K x M rows, B as K x N), read as stored by TMA.
 //
 // Persistent, warp-specialised CTA (one per SM): warp 0 issues TMA tile loads
 // into a 4-stage shared-memory ring, warp 1 issues tcgen05.mma (128 x 256 x 16)
@@ -9,6 +10,7 @@
 // CTA raises the timeout bit of the device status word, drains its own
 // copies and MMAs (bounded again), frees its TMEM and returns.
 #include <cfloat>
+#include <cstring>
 #include <cudaTypedefs.h>
 
 #include "internal.cuh"
@@ -33,27 +35,48 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int PSTAGE_FLOATS = 2 * HALF_N;
 constexpr size_t PSTAGE_BYTES = (size_t)EPI_WARPS * 2 * PSTAGE_FLOATS * 4;
 constexpr int kMaxStages = 6;
+// An MN-major operand tile: boxes of 64 MN elements x BK rows of K.
+constexpr uint32_t MN_BOX = 64 * BK * 2;
+
+// The fp32 store of kEpiF32Lse goes through shared memory: each epilogue
+// warp writes its 32 rows x 32 columns into one of STORE_BUFS 4 KB boxes
+// (128-byte swizzled, so the row-per-thread writes hit distinct banks) and
+// one lane stores the box by TMA, instead of every thread writing 16 bytes
+// into each of 32 rows per instruction.
+constexpr int STORE_BOX = 32;
+constexpr int STORE_BOX_BYTES = STORE_BOX * STORE_BOX * 4;
+constexpr int STORE_BUFS = 1;
+constexpr size_t STORE_BYTES = (size_t)EPI_WARPS * STORE_BUFS * STORE_BOX_BYTES;
 
 // Single CTA: a 128 x 256 tile per SM, A and all 256 rows of B staged by the
 // CTA (48 KB per 64-deep stage, 4 stages). CTA pair (cta_group::2): a
 // 256 x 256 tile per pair of SMs; each CTA stages its 128 rows of A and 128
 // of the 256 rows of B (32 KB per stage, 6 stages) and the leader's MMAs read
 // both CTAs' shared memory, so every SM is fed a third fewer bytes per flop.
-template <bool PAIR>
+// kEpiF32Lse gives up one operand stage per 32 KB of store boxes.
+template <bool PAIR, int KIND>
 struct Cfg {
+  static constexpr bool STORE = KIND == kEpiF32Lse;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;
-  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int STAGES = PAIR ? (STORE ? 6 - STORE_BUFS : 6) : (STORE ? 5 - STORE_BUFS : 4);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + PSTAGE_BYTES;
+  // after the stages (1024-byte aligned): the store boxes or the reward's
+  // probability staging, then the barrier block
+  static constexpr size_t EXTRA = STORE ? STORE_BYTES : PSTAGE_BYTES;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EXTRA + 256;
   static_assert(STAGES <= kMaxStages, "barrier arrays");
+  static_assert(EXTRA % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 struct TcParams {
   int64_t M, N, K;
   int m_tiles, n_tiles, num_kb;  // m_tiles counts Cfg::TILE_M-row tiles
+  int tma_store;                 // kEpiF32Lse: C is stored through tmC
+  int a_mn, b_mn;                // operand stored MN-major (K x M, K x N rows)
   EpiDesc e;
   uint32_t* status;
   uint64_t wait_ns;  // limit of the pipeline waits (teardown waits keep kWaitLimitNs)
@@ -206,6 +229,23 @@ __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t
   }
 }
 
+// Online softmax partial of a row over 32 more columns [n, n+32): the running
+// maximum and the sum of exponentials relative to it, as 4 independent chains.
+__device__ __forceinline__ void lse_chunk(const TcParams& p, int64_t n, const float* v, float& rmax,
+                                          float& rsum) {
+  float cm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+#pragma unroll
+  for (int q = 0; q < 32; ++q)
+    if (n + q < p.N) cm[q & 3] = fmaxf(cm[q & 3], v[q]);
+  const float nm = fmaxf(rmax, fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])));
+  float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int q = 0; q < 32; ++q)
+    if (n + q < p.N) cs[q & 3] += __expf(v[q] - nm);
+  rsum = fmaf(rsum, __expf(rmax - nm), (cs[0] + cs[1]) + (cs[2] + cs[3]));
+  rmax = nm;
+}
+
 // Tile order: bands of kGroupM M-tiles swept across all N-tiles, M fastest
 // within the band. The CTAs running at the same time then cover a compact
 // kGroupM x (SMs / kGroupM) block of tiles, so the band of A (kGroupM * 128
@@ -301,8 +341,9 @@ __device__ __forceinline__ float reward32(const TcParams& p, int64_t m, int32_t 
 template <int KIND, bool PAIR>
 __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ CUtensorMap tmA,
                                                         const __grid_constant__ CUtensorMap tmB,
+                                                        const __grid_constant__ CUtensorMap tmC,
                                                         TcParams p) {
-  using C = Cfg<PAIR>;
+  using C = Cfg<PAIR, KIND>;
   constexpr int STAGES = C::STAGES, A_BYTES = C::A_BYTES, B_BYTES = C::B_BYTES;
   constexpr int STAGE_BYTES = C::STAGE_BYTES, TILE_M = C::TILE_M;
   extern __shared__ uint8_t smem_raw[];
@@ -311,8 +352,9 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
   uint8_t* basep = smem_raw + (base - raw);
   const uint32_t sA = base;                           // STAGES x A tile
   const uint32_t sB = base + STAGES * A_BYTES;        // STAGES x B tile
-  Shared* sh = reinterpret_cast<Shared*>(basep + STAGES * STAGE_BYTES);
-  float* pstage = reinterpret_cast<float*>(basep + STAGES * STAGE_BYTES + 256);
+  float* pstage = reinterpret_cast<float*>(basep + STAGES * STAGE_BYTES);
+  const uint32_t sStore = base + STAGES * STAGE_BYTES;  // kEpiF32Lse store boxes
+  Shared* sh = reinterpret_cast<Shared*>(basep + STAGES * STAGE_BYTES + C::EXTRA);
   volatile int* abort = &sh->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -339,6 +381,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     ptx::fence_proxy_async();
     ptx::prefetch_map(&tmA);
     ptx::prefetch_map(&tmB);
+    if (C::STORE && p.tma_store) ptx::prefetch_map(&tmC);
   }
   if (warp == 1) {
     if (PAIR) {
@@ -366,20 +409,33 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
         tile_coords(tile, p.m_tiles, p.n_tiles, &m_blk, &n_blk);
         const int a_row = m_blk * TILE_M + (int)rank * BM;
         const int b_row = n_blk * BN + (int)rank * C::B_ROWS;
+        // a K-major operand tile is one box of rows x 64 K; an MN-major one
+        // is rows / 64 boxes of 64 MN x 64 K rows, MN_BOX bytes apart
+        auto load = [&](uint32_t dst, const CUtensorMap* map, bool mn, int rows, int r0, int k0,
+                        uint32_t bar) {
+          if (!mn) {
+            if (PAIR) ptx::tma_load_2d_pair(dst, map, k0, r0, bar);
+            else ptx::tma_load_2d(dst, map, k0, r0, bar);
+            return;
+          }
+          for (int j = 0; j < rows / 64; ++j) {
+            if (PAIR) ptx::tma_load_2d_pair(dst + j * MN_BOX, map, r0 + 64 * j, k0, bar);
+            else ptx::tma_load_2d(dst + j * MN_BOX, map, r0 + 64 * j, k0, bar);
+          }
+        };
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!wait_bounded(ptx::smem_u32(&sh->empty[stage]), phase ^ 1u, abort, p.status, p.wait_ns)) break;
           const uint32_t fb = ptx::smem_u32(&sh->full[stage]);
+          uint32_t bar = fb;
           if (PAIR) {
             // both CTAs' bytes complete on the leader's barrier
             if (leader) ptx::mbar_expect_tx(fb, 2 * STAGE_BYTES);
-            const uint32_t lfb = ptx::mapa_shared(fb, 0);
-            ptx::tma_load_2d_pair(sA + stage * A_BYTES, &tmA, kb * BK, a_row, lfb);
-            ptx::tma_load_2d_pair(sB + stage * B_BYTES, &tmB, kb * BK, b_row, lfb);
+            bar = ptx::mapa_shared(fb, 0);
           } else {
             ptx::mbar_expect_tx(fb, STAGE_BYTES);
-            ptx::tma_load_2d(sA + stage * A_BYTES, &tmA, kb * BK, a_row, fb);
-            ptx::tma_load_2d(sB + stage * B_BYTES, &tmB, kb * BK, b_row, fb);
           }
+          load(sA + stage * A_BYTES, &tmA, p.a_mn != 0, BM, a_row, kb * BK, bar);
+          load(sB + stage * B_BYTES, &tmB, p.b_mn != 0, C::B_ROWS, b_row, kb * BK, bar);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -403,7 +459,11 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && leader) {
-      const uint32_t idesc = ptx::idesc_bf16_f32(TILE_M, BN);
+      const uint32_t idesc = ptx::idesc_bf16_f32(TILE_M, BN) | (p.a_mn ? ptx::kIdescAMn : 0u) |
+                             (p.b_mn ? ptx::kIdescBMn : 0u);
+      // per 16-deep MMA step: 32 bytes along a K-major row, two 8-row
+      // swizzle atoms (2048 bytes) down an MN-major tile
+      const uint32_t a_step = p.a_mn ? 2048u : 32u, b_step = p.b_mn ? 2048u : 32u;
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -424,12 +484,13 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           const uint32_t a0 = sA + stage * A_BYTES, b0 = sB + stage * B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t ak = a0 + k * a_step, bk = b0 + k * b_step;
+            const uint64_t ad = p.a_mn ? ptx::sdesc_mnmajor_sw128(ak, MN_BOX) : ptx::sdesc_kmajor_sw128(ak);
+            const uint64_t bd = p.b_mn ? ptx::sdesc_mnmajor_sw128(bk, MN_BOX) : ptx::sdesc_kmajor_sw128(bk);
             if (PAIR)
-              ptx::mma_f16_pair(d_tmem, ptx::sdesc_kmajor_sw128(a0 + k * 32),
-                                ptx::sdesc_kmajor_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+              ptx::mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
             else
-              ptx::mma_f16(d_tmem, ptx::sdesc_kmajor_sw128(a0 + k * 32),
-                           ptx::sdesc_kmajor_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+              ptx::mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
           }
           issued = true;
           if (PAIR)
@@ -467,6 +528,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     const int row = quad * 32 + lane;
     const int half = (warp - 2) >> 2;  // columns [HALF_N half, HALF_N (half + 1)) of the tile
     int it = 0;
+    int nbox = 0;  // kEpiF32Lse: store boxes this warp has issued
+    const uint32_t box0 = sStore + (uint32_t)((warp - 2) * STORE_BUFS * STORE_BOX_BYTES);
     const uint32_t tempty0 =
         PAIR ? ptx::mapa_shared(ptx::smem_u32(&sh->tempty[0]), 0) : ptx::smem_u32(&sh->tempty[0]);
     const uint32_t tempty1 =
@@ -536,22 +599,31 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
                                        : p.e.P + t_row * p.N + n;
             s_row += reward32(p, m, yt, n, prow, staged, v);
           }
+        } else if (C::STORE && p.tma_store && n < p.N) {
+          // this warp's 32 x 32 box: row `lane` at byte 128 lane, its 16-byte
+          // chunk q at position q ^ (lane & 7) (the 128-byte swizzle of tmC);
+          // the box's previous store from this buffer has read it by now
+          const uint32_t box = box0 + (uint32_t)((nbox % STORE_BUFS) * STORE_BOX_BYTES);
+          if (lane == 0) ptx::bulk_wait_read<STORE_BUFS - 1>();
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t a = box + (uint32_t)(lane * 128 + ((q ^ (lane & 7)) << 4));
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v[4 * q]),
+                         "f"(v[4 * q + 1]), "f"(v[4 * q + 2]), "f"(v[4 * q + 3])
+                         : "memory");
+          }
+          ptx::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmC, (int)n, (int)(m - lane), box);
+            ptx::bulk_commit();
+          }
+          ++nbox;
+          if (m < p.M) lse_chunk(p, n, v, rmax, rsum);
         } else if (m < p.M && n < p.N) {
           epilogue32<KIND>(p, m, mo, n, v);
-          if (KIND == kEpiF32Lse) {
-            // max and sum of exponentials of the chunk, as 4 independent chains
-            float cm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (n + q < p.N) cm[q & 3] = fmaxf(cm[q & 3], v[q]);
-            const float nm = fmaxf(rmax, fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])));
-            float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (n + q < p.N) cs[q & 3] += __expf(v[q] - nm);
-            rsum = fmaf(rsum, __expf(rmax - nm), (cs[0] + cs[1]) + (cs[2] + cs[3]));
-            rmax = nm;
-          }
+          if (KIND == kEpiF32Lse) lse_chunk(p, n, v, rmax, rsum);
         }
       }
       // one partial per row, column tile and half: 2 n_tiles per row
@@ -567,6 +639,9 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           ptx::mbar_arrive(acc ? tempty1 : tempty0);
       }
     }
+    // the boxes' stores have left shared memory and completed before the CTA
+    // (and its shared memory) goes away
+    if (C::STORE && lane == 0) ptx::bulk_wait<0>();
   }
 
   ptx::tc_fence_before();
@@ -609,17 +684,31 @@ bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-major fp32 matrix (rows x cols, row stride ld elements) as a TMA store
+// map: 32 x 32 boxes, 128-byte swizzling.
+bool make_map_f32(CUtensorMap* map, const float* ptr, int64_t rows, int64_t cols, int64_t ld) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  cuuint32_t box[2] = {(cuuint32_t)STORE_BOX, (cuuint32_t)STORE_BOX};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int KIND, bool PAIR>
 cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
-                        const TcParams& p, int sm_count) {
+                        const CUtensorMap& c, const TcParams& p, int sm_count) {
   auto fn = k_gemm_tc<KIND, PAIR>;
-  constexpr size_t smem = Cfg<PAIR>::SMEM;
+  constexpr size_t smem = Cfg<PAIR, KIND>::SMEM;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int tiles = p.m_tiles * p.n_tiles;
   if (!PAIR) {
     const int grid = tiles < sm_count ? tiles : sm_count;
-    fn<<<grid, THREADS, smem, st>>>(a, b, p);
+    fn<<<grid, THREADS, smem, st>>>(a, b, c, p);
     return cudaGetLastError();
   }
   const int pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
@@ -635,7 +724,7 @@ cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, fn, a, b, p);
+  err = cudaLaunchKernelEx(&cfg, fn, a, b, c, p);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -643,7 +732,7 @@ cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap
 }  // namespace
 
 bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
-  if (g.dtype != DUST_BF16 || !g.a_kmajor || !g.b_kmajor || g.b_row_mul != 0) return false;
+  if (g.dtype != DUST_BF16 || g.b_row_mul != 0) return false;
   if (g.M < 1 || g.N < 16 || g.K < 8) return false;
   if ((g.lda & 7) || (g.ldb & 7)) return false;
   if (((uintptr_t)g.A & 15) || ((uintptr_t)g.B & 15)) return false;
@@ -662,15 +751,25 @@ namespace {
 template <bool PAIR>
 cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
                         uint32_t* status, uint64_t wait_ns) {
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, g.A, g.M, g.K, g.lda, BM) ||
-      !make_map(&mb, g.B, g.N, g.K, g.ldb, Cfg<PAIR>::B_ROWS))
-    return cudaErrorInvalidValue;
+  CUtensorMap ma, mb, mc;
+  const bool ok_a = g.a_kmajor ? make_map(&ma, g.A, g.M, g.K, g.lda, BM)
+                               : make_map(&ma, g.A, g.K, g.M, g.lda, BK);
+  const bool ok_b = g.b_kmajor ? make_map(&mb, g.B, g.N, g.K, g.ldb, Cfg<PAIR, kEpiF32>::B_ROWS)
+                               : make_map(&mb, g.B, g.K, g.N, g.ldb, BK);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+  memset(&mc, 0, sizeof(mc));
+  // kEpiF32Lse stores C through a TMA map when its rows are 16-byte aligned
+  // (else the direct per-row stores run)
+  const bool tma_store = e.kind == kEpiF32Lse && ((uintptr_t)e.C & 15) == 0 &&
+                         (e.ldc & 3) == 0 && make_map_f32(&mc, e.C, g.M, g.N, e.ldc);
   TcParams p;
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
-  p.m_tiles = (int)((g.M + Cfg<PAIR>::TILE_M - 1) / Cfg<PAIR>::TILE_M);
+  p.m_tiles = (int)((g.M + Cfg<PAIR, kEpiF32>::TILE_M - 1) / Cfg<PAIR, kEpiF32>::TILE_M);
+  p.tma_store = tma_store ? 1 : 0;
+  p.a_mn = g.a_kmajor ? 0 : 1;
+  p.b_mn = g.b_kmajor ? 0 : 1;
   p.n_tiles = (int)((g.N + BN - 1) / BN);
   p.num_kb = (int)((g.K + BK - 1) / BK);
   p.e = e;
@@ -678,13 +777,13 @@ cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, in
   p.wait_ns = wait_ns;
   if (!p.status) return cudaErrorInvalidValue;
   switch (e.kind) {
-    case kEpiF32: return launch_kind<kEpiF32, PAIR>(st, ma, mb, p, sm_count);
-    case kEpiBF16: return launch_kind<kEpiBF16, PAIR>(st, ma, mb, p, sm_count);
-    case kEpiGeluSplit: return launch_kind<kEpiGeluSplit, PAIR>(st, ma, mb, p, sm_count);
-    case kEpiResidSplit: return launch_kind<kEpiResidSplit, PAIR>(st, ma, mb, p, sm_count);
-    case kEpiSplit: return launch_kind<kEpiSplit, PAIR>(st, ma, mb, p, sm_count);
-    case kEpiReward: return launch_kind<kEpiReward, PAIR>(st, ma, mb, p, sm_count);
-    case kEpiF32Lse: return launch_kind<kEpiF32Lse, PAIR>(st, ma, mb, p, sm_count);
+    case kEpiF32: return launch_kind<kEpiF32, PAIR>(st, ma, mb, mc, p, sm_count);
+    case kEpiBF16: return launch_kind<kEpiBF16, PAIR>(st, ma, mb, mc, p, sm_count);
+    case kEpiGeluSplit: return launch_kind<kEpiGeluSplit, PAIR>(st, ma, mb, mc, p, sm_count);
+    case kEpiResidSplit: return launch_kind<kEpiResidSplit, PAIR>(st, ma, mb, mc, p, sm_count);
+    case kEpiSplit: return launch_kind<kEpiSplit, PAIR>(st, ma, mb, mc, p, sm_count);
+    case kEpiReward: return launch_kind<kEpiReward, PAIR>(st, ma, mb, mc, p, sm_count);
+    case kEpiF32Lse: return launch_kind<kEpiF32Lse, PAIR>(st, ma, mb, mc, p, sm_count);
   }
   return cudaErrorInvalidValue;
 }

@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a tensor-core path: mbarriers, TMA
-// tile loads, TMEM allocation, tcgen05.mma / commit / ld, and the shared
+// tile loads and stores, TMEM allocation, tcgen05.mma / commit / ld, and the shared
 // memory and instruction descriptors of kind::f16 MMAs.
 #pragma once
 #include <cuda.h>
@@ -69,6 +69,32 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"((uint64_t)map), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// 2-D tiled TMA store of a box from this CTA's shared memory to global
+// memory, in the issuing thread's current bulk async-group. Elements of the
+// box outside the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::
+                   "l"((uint64_t)map), "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+
+// Close the issuing thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until at most N of this thread's bulk groups are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
@@ -222,6 +248,21 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor: MN-major operand tile written by TMA with
+// 128-byte swizzling as boxes of 64 MN elements x K rows (each K row of a
+// box 128 bytes; 8-row / 1024-byte swizzle atoms down K). Leading byte
+// offset = `mn_stride`, the bytes between consecutive 64-element boxes along
+// MN; stride byte offset = 1024, the bytes between 8-row groups along K.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 D, both
 // operands K-major: D format (bits 4-5) = 1, A format (7-9) = 1, B format
 // (10-12) = 1, N >> 3 (17-22), M >> 4 (24-28).
@@ -229,6 +270,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
 }
+
+// Operand major-ness bits of the instruction descriptor: A MN-major (bit 15),
+// B MN-major (bit 16); clear means K-major.
+constexpr uint32_t kIdescAMn = 1u << 15, kIdescBMn = 1u << 16;
 
 // The same with fp16 A and B (A and B format 0).
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
