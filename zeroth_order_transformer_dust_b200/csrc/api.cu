@@ -392,7 +392,8 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
     mark(ctx, "g");
   } else if (smem_subset) {
     DUST_CU(launch_subset2(st, p, a, a_inv, Z, (const float*)ctx->lse.p, targets, rewards_out,
-                           g_out, ctx->gop.p, ctx->max_smem_optin, ctx->sm_count));
+                           g_out, ctx->gop.p, ctx->max_smem_optin, ctx->sm_count,
+                           ctx->d_status));
     ctx->launches += 1;
     mark(ctx, "subset_draws");
   } else {

@@ -242,13 +242,15 @@ cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a,
                                void* gop, float* gacc, int max_smem_optin);
 
 // Subset draws with the probability row and the g accumulator resident in
-// shared memory, one cluster of 1 or 2 CTAs per token (0: not applicable to
+// shared memory, one cluster of 1, 2, 4 or 8 CTAs per token (0: not applicable to
 // this V, S). Z holds clean logits in permuted column order, lse the row
-// log-sum-exp; p = exp(z - lse) is formed while the row is loaded.
+// log-sum-exp; p = exp(z - lse) is formed while the row is loaded. A row
+// copy that does not arrive in time sets kStatusTimeout in *status.
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin);
 cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                            const float* Z, const float* lse, const int32_t* y, float* rewards,
-                           float* g_out, void* gop, int max_smem_optin, int sm_count);
+                           float* g_out, void* gop, int max_smem_optin, int sm_count,
+                           uint32_t* status);
 
 // Tensor-core GEMM (tcgen05): shapes it takes, and its launcher (pair: a
 // 256 x 256 tile per cluster of two CTAs, cta_group::2; else 128 x 256 per

@@ -38,10 +38,20 @@
 // scale shrinks as 16384/K above 16384 draws). The target coordinate, which
 // collects all K draws, keeps an fp32 accumulator per warp. INT = false
 // accumulates in fp32 (compare-and-swap atomics) for larger K.
+//
+// Token pipeline (rows of 16-byte multiples, V % 4 == 0): a CTA's slice of
+// the next token's Z row is prefetched into L2 while the current token's
+// draws run, and copied into shared memory by one bulk copy as soon as the
+// draws are done, so that it lands while the g slice is written out (the
+// write pass also clears the accumulator). Without it every token began with
+// a chain of dependent global loads per thread, about a third of the launch
+// at K = 1024. The wait for the copy is bounded: on expiry the kernel raises
+// the timeout bit of the status word and runs on without waiting again.
 #include <cooperative_groups.h>
 
 #include "internal.cuh"
 #include "noise.cuh"
+#include "tc_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -84,6 +94,7 @@ struct Sub2Args {
   float fac;        // g = fac * sum r * (sigma eps)            (fp32 accumulators)
   float acc_scale;  // fixed-point units per unit of r * (sigma eps)
   float fac_int;    // g = fac_int * fixed-point sum
+  uint32_t* status;  // kStatusTimeout when a row copy does not arrive
   const float* Z;    // clean logits, permuted columns (T x V)
   const float* lse;  // T
   const int32_t* y;
@@ -126,7 +137,17 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
   __shared__ int s_next;    // next draw batch of the current token
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
   __shared__ float2 s_tab[kSinCosTable];
+  __shared__ __align__(8) uint64_t s_row;  // completion of the row copy
+  __shared__ float s_lse_n;                // LSE and target of the next token
+  __shared__ int32_t s_y_n;
+  __shared__ const float* s_row_n;         // its Z slice to copy (null: none)
+  __shared__ uint32_t s_phase;             // phase of s_row the next row completes
   fill_sincos_table(s_tab, A.sigma);
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(ptx::smem_u32(&s_row), 1);
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async();
+  }
   __syncthreads();
   cg::cluster_group cluster = cg::this_cluster();
   const uint32_t cs = A.cs;
@@ -141,8 +162,27 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
   const uint32_t lo_peer = peer * seg;
   float* sp = smem;        // p of q in [lo, hi)
   float* sg = smem + seg;  // g accumulator of q in [lo, hi) (fp32 or int32 fixed point)
-  float* const sp_peer = cluster.map_shared_rank(sp, peer);
-  float* const sg_peer = cluster.map_shared_rank(sg, peer);
+  // the next CTA's p and g slices (DSMEM). NB = 2 and 3 read their
+  // addresses from shared memory where a window crosses into them: held in
+  // registers they push those variants past the 64 registers of a
+  // 1024-thread CTA. NB = 1 and 4 keep them in registers (1.4 % faster on the
+  // large-subset workload than reading them from shared memory).
+  constexpr bool kPeerRegs = NB == 1 || NB == 4;
+  __shared__ float* s_peer[2];
+  float* sp_peer = nullptr;
+  float* sg_peer = nullptr;
+  if constexpr (kPeerRegs) {
+    sp_peer = cluster.map_shared_rank(sp, peer);
+    sg_peer = cluster.map_shared_rank(sg, peer);
+  } else {
+    if (threadIdx.x == 0) {
+      s_peer[0] = cluster.map_shared_rank(sp, peer);
+      s_peer[1] = cluster.map_shared_rank(sg, peer);
+    }
+    __syncthreads();
+  }
+  auto peer_p = [&]() { return kPeerRegs ? sp_peer : *(float* volatile*)&s_peer[0]; };
+  auto peer_g = [&]() { return kPeerRegs ? sg_peer : *(float* volatile*)&s_peer[1]; };
   const int S = A.S;
   const uint32_t nclusters = gridDim.x / cs;
   const uint32_t cid = blockIdx.x / cs;
@@ -155,12 +195,65 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
   const BlockConst bs = block_const(A.keys, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u), A.ctr3);
   const uint32_t s_word = ((uint32_t)S >> 5) & 3u;
   const bool vec = (V & 3u) == 0;  // rows start 16-byte aligned
+  // the pipelined row copy (one bulk copy of n_own floats; 16-byte aligned
+  // source and size when V % 4 == 0, the slices being multiples of 4)
+  const bool bulk = vec;
+  // thread 0: copy a slice of n_own floats at src into sp (every generic
+  // access to sp of the previous token is ordered before the barrier that
+  // precedes this)
+  auto issue_row = [&](const float* src) {
+    const uint32_t bar = ptx::smem_u32(&s_row);
+    ptx::fence_proxy_async();
+    ptx::mbar_expect_tx(bar, n_own * 4u);
+    ptx::bulk_load(ptx::smem_u32(sp), src, n_own * 4u, bar);
+  };
+
+  if (bulk) {
+    if (threadIdx.x == 0 && (int64_t)cid < A.T) issue_row(A.Z + (int64_t)cid * A.V + lo);
+    for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4)
+      *reinterpret_cast<float4*>(sg + q) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // the LSE and target of a token are loaded a token ahead (thread 0, into
+  // shared memory, read after the barrier that ends the previous token)
+  if (threadIdx.x == 0 && (int64_t)cid < A.T) {
+    s_lse_n = A.lse[cid];
+    s_y_n = A.y[cid];
+    s_phase = 0;
+  }
+  __syncthreads();
 
   for (int64_t t = cid; t < A.T; t += nclusters) {
-    // ---- load p = exp(z - LSE) for the owned slice, clear g
+    const float lse_t = s_lse_n;
+    int32_t yt = s_y_n;
+    // ---- p = exp(z - LSE) for the owned slice (and clear g without bulk)
     const float* zrow = A.Z + t * A.V;
-    const float lse_t = A.lse[t];
-    for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
+    if (bulk) {
+      // thread 0 waits for the row (the k-th token of this cluster for
+      // phase k & 1), the block barrier passes its arrival on; once a wait
+      // has expired (the status word says so) none waits again
+      if (threadIdx.x == 0) {
+        const uint32_t row_bar = ptx::smem_u32(&s_row);
+        const uint32_t row_phase = s_phase;
+        s_phase = row_phase ^ 1u;
+        if (!(*(volatile uint32_t*)A.status & kStatusTimeout)) {
+          bool ok = ptx::mbar_try_wait(row_bar, row_phase);
+          if (!ok) {
+            const uint64_t t0 = ptx::globaltimer_ns();
+            for (uint32_t it = 1; !ok; ++it) {
+              ok = ptx::mbar_try_wait(row_bar, row_phase);
+              if (!ok && (it & 63u) == 0 && ptx::globaltimer_ns() - t0 > 2000000000ull) break;
+            }
+          }
+          if (!ok) atomicOr(A.status, kStatusTimeout);
+        }
+      }
+      __syncthreads();
+      for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
+        const float4 z = *reinterpret_cast<const float4*>(sp + q);
+        *reinterpret_cast<float4*>(sp + q) =
+            make_float4(expf(z.x - lse_t), expf(z.y - lse_t), expf(z.z - lse_t), expf(z.w - lse_t));
+      }
+    } else for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
       if (vec && q + 3 < n_own) {
         const float4 z = *reinterpret_cast<const float4*>(zrow + lo + q);
         *reinterpret_cast<float4*>(sp + q) =
@@ -177,13 +270,24 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
       s_next = 0;
       s_tgt = 0.0f;
     }
-    int32_t yt = A.y[t];
     if (yt < 0 || (int64_t)yt >= A.V) yt = 0;  // reported by the loss kernel
     const uint32_t qy = mulmod((uint32_t)yt, A.a_inv, V, A.minv);
     const uint32_t owner_y = qy / seg;  // the CTA whose slice holds the target
-    const float py = expf(zrow[qy] - lse_t);
     float* gy = cluster.map_shared_rank(sg, owner_y) + (qy - owner_y * seg);
     cluster.sync();
+    // p of the target, from the owner's shared memory
+    const float py = cluster.map_shared_rank(sp, owner_y)[qy - owner_y * seg];
+    if (threadIdx.x == 0) {
+      const int64_t tn = t + nclusters;
+      const float* zn = nullptr;
+      if (tn < A.T) {
+        zn = A.Z + tn * A.V + lo;
+        if (bulk) ptx::bulk_prefetch_l2(zn, n_own * 4u);
+        s_lse_n = A.lse[tn];
+        s_y_n = A.y[tn];
+      }
+      s_row_n = bulk ? zn : nullptr;
+    }
 
     const uint32_t t_abs = A.t_off + (uint32_t)t;
     float tgt_acc = 0.0f;  // INT: this warp's sum r * (sigma eps_y), lane 0
@@ -280,7 +384,7 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
             if (FULL || k < S) {
               uint32_t q = cw + (uint32_t)k;
               if (q >= V) q -= V;
-              const float pq = (q >= lo && q < hi) ? sp[q - lo] : sp_peer[q - lo_peer];
+              const float pq = (q >= lo && q < hi) ? sp[q - lo] : peer_p()[q - lo_peer];
               x = g.v[j];
               s = fmaf(pq, expm1_small<DEG>(x), s);
             }
@@ -345,7 +449,7 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
             if (FULL || k < S) {
               uint32_t q = cw + (uint32_t)k;
               if (q >= V) q -= V;
-              float* dst = (q >= lo && q < hi) ? sg + (q - lo) : sg_peer + (q - lo_peer);
+              float* dst = (q >= lo && q < hi) ? sg + (q - lo) : peer_g() + (q - lo_peer);
               accumulate<INT>(dst, r, n[m][j], A.acc_scale);
             }
           }
@@ -375,8 +479,11 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
     }
     if (INT && lane == 0) atomicAdd(cluster.map_shared_rank(&s_tgt, owner_y), tgt_acc);
     cluster.sync();
+    // no CTA of the cluster reads sp any more: the next row can come in
+    if (threadIdx.x == 0 && s_row_n) issue_row(s_row_n);
 
-    // ---- scale and write the owned slice of g
+    // ---- scale and write the owned slice of g, and clear it for the next
+    // token
     for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
       const uint32_t qg = lo + q;
       float v;
@@ -385,6 +492,7 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
                        : (float)reinterpret_cast<const int*>(sg)[q] * A.fac_int * A.scale_other;
       else
         v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
+      sg[q] = 0.0f;
       if (A.gop_bf16)
         store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + qg, v);
       else
@@ -470,8 +578,10 @@ int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
 
 cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                            const float* Z, const float* lse, const int32_t* y, float* rewards,
-                           float* g_out, void* gop, int max_smem_optin, int sm_count) {
+                           float* g_out, void* gop, int max_smem_optin, int sm_count,
+                           uint32_t* status) {
   const int cs = subset2_cluster_size(p.V, p.S, max_smem_optin);
+  if (!status) return cudaErrorInvalidValue;
   if (!cs) return cudaErrorNotSupported;
   Sub2Args A;
   A.key = key_of(p.seed);
@@ -499,6 +609,7 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   const double units = 32768.0 * (p.K > 16384 ? 16384.0 / (double)p.K : 1.0);
   A.acc_scale = p.sigma > 0.0f ? (float)(units / s2) : 0.0f;
   A.fac_int = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * units)) : 0.0f;
+  A.status = status;
   A.Z = Z;
   A.lse = lse;
   A.y = y;
