@@ -123,6 +123,32 @@ def test_single_cta_tensor_core_path(cuda_ok, monkeypatch, kw):
     _compare(_gpu(c, H, W, y, wl), _oracle(H, W, y, wl), TOL_GW_BF16)
 
 
+@pytest.mark.parametrize("c", [2.0 ** 20, 2.0 ** -26])
+@pytest.mark.parametrize("S", [0, 100])
+def test_gw_with_h_outside_the_fp16_range(ctx, c, S):
+    """The G_W GEMM reads H as fp16 with a power-of-two scale taken from its
+    largest magnitude: H scaled by 2^20 (beyond the fp16 maximum) or 2^-26
+    (below its normal range), with W scaled by the inverse so the logits stay
+    the same, gives the oracle's G_W."""
+    wl = _small(T=37, d=40, V=1000, K=9, S=S)
+    H, W, y = _inputs(wl)
+    H, W = H * c, W / c
+    got = _gpu(ctx, H, W, y, wl)
+    ref = _oracle(H, W, y, wl)
+    _compare(got, ref, TOL_GW_BF16)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(S=129, K=33), dict(V=4099, K=20), dict(T=200, K=5, V=1000)])
+def test_cuda_core_gemms(cuda_ok, monkeypatch, kw):
+    """With the tensor cores off every GEMM runs on CUDA cores, G_W on the
+    fp16 g operand and the fp16 copy of H included."""
+    monkeypatch.setenv("DUST_DISABLE_TC", "1")
+    c = dust.Context(0)
+    wl = _small(**kw)
+    H, W, y = _inputs(wl)
+    _compare(_gpu(c, H, W, y, wl), _oracle(H, W, y, wl), TOL_GW_BF16)
+
+
 def _host(x, dtype):
     t = torch.from_numpy(np.ascontiguousarray(x))
     t = t.to(torch.int32) if dtype == "i32" else t.to(torch.bfloat16 if dtype == "bf16" else torch.float32)

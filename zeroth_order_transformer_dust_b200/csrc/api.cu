@@ -19,6 +19,23 @@ int64_t default_stride(int64_t V) {
   while (gcd64(a, V) != 1) ++a;
   return a;
 }
+
+GopFormat head_gop_format(const dust_params& p) {
+  if (p.dtype != DUST_BF16) return GopFormat{kGopF32, 1.0f};
+  // Every g entry is bounded by the noise: |r| <= 11.54 sigma and
+  // |sigma eps| <= 5.77 sigma (the largest Box-Muller radius of a 24-bit
+  // uniform) give |g| <= 66.6 times the entry's inverse-inclusion scale
+  // (V/S off the target for subset draws, at most that on it; 1 for the
+  // full vocabulary). With 70 for 66.6, g 2^e stays below the fp16 maximum.
+  const double scale = p.S > 0 ? (double)p.V / (double)p.S : 1.0;
+  const int e = (int)std::floor(std::log2(65504.0 / (70.0 * scale)));
+  return GopFormat{kGopF16, std::ldexp(1.0f, e)};
+}
+
+size_t gop_format_bytes(GopFormat f, int64_t T, int64_t width) {
+  const size_t n = (size_t)T * (size_t)width;
+  return f.kind == kGopF32 ? n * 4 : (f.kind == kGopBf16Planes ? n * 4 : n * 2);
+}
 }  // namespace dust
 
 namespace {
@@ -182,6 +199,49 @@ dust_status weight_grad(dust_ctx* ctx, const dust_params& p, const void* gop, in
   return run_gemm(ctx, s, e);
 }
 
+// out (width x N, fp32) = sum_t g_t x_t^T from the fp16 g operand (g * gscale,
+// T x width) and bf16 X (T x N): X is converted to fp16 with a power-of-two
+// scale from its largest magnitude (on the device), and the GEMM (K = T, both
+// operands MN-major as stored) multiplies its sums by the two scales'
+// inverse. Rows that are not 16-byte multiples are transposed to K-major
+// first; without tensor cores the CUDA-core GEMM reads the fp16 operands.
+dust_status weight_grad_f16(dust_ctx* ctx, const dust_params& p, const void* gop, float gscale,
+                            int64_t width, const void* X, int64_t N, float* out,
+                            int64_t row_mul) {
+  const int64_t T = p.T;
+  DUST_TRY(ensure(ctx, ctx->xdup, (size_t)T * N * 2));
+  DUST_TRY(ensure(ctx, ctx->hsc, 16));
+  uint32_t* absmax = (uint32_t*)ctx->hsc.p;
+  float* escale = (float*)ctx->hsc.p + 1;
+  DUST_CU(cudaMemsetAsync(absmax, 0, sizeof(uint32_t), ctx->stream));
+  DUST_CU(launch_absmax_bf16(ctx->stream, (const __nv_bfloat16*)X, T * N, absmax));
+  DUST_CU(launch_to_f16_scaled(ctx->stream, (const __nv_bfloat16*)X, T * N, absmax, gscale,
+                               (__half*)ctx->xdup.p, escale));
+  ctx->launches += 2;
+  EpiDesc e{};
+  e.kind = kEpiF32; e.C = out; e.ldc = N; e.c_row_mul = row_mul; e.scale = escale;
+  GemmDesc s{};
+  s.M = width; s.N = N; s.K = T; s.A = gop; s.lda = width; s.a_kmajor = false;
+  s.B = ctx->xdup.p; s.ldb = N; s.b_kmajor = false; s.dtype = DUST_BF16; s.f16 = true;
+  if (!ctx->tc_enabled || tc_gemm_supported(s, e)) return run_gemm(ctx, s, e);
+  const int64_t ld = (T + 7) / 8 * 8;
+  DUST_TRY(ensure(ctx, ctx->gT, (size_t)width * ld * 2));
+  DUST_TRY(ensure(ctx, ctx->hT, (size_t)N * ld * 2));
+  GemmDesc g{};
+  g.M = width; g.N = N; g.K = T; g.A = ctx->gT.p; g.lda = ld; g.a_kmajor = true;
+  g.B = ctx->hT.p; g.ldb = ld; g.b_kmajor = true; g.dtype = DUST_BF16; g.f16 = true;
+  if (tc_gemm_supported(g, e)) {
+    // the transposes move 2-byte words, whatever their type
+    DUST_CU(launch_transpose_bf16(ctx->stream, (const __nv_bfloat16*)gop, T, width,
+                                  (__nv_bfloat16*)ctx->gT.p, ld));
+    DUST_CU(launch_transpose_bf16(ctx->stream, (const __nv_bfloat16*)ctx->xdup.p, T, N,
+                                  (__nv_bfloat16*)ctx->hT.p, ld));
+    ctx->launches += 2;
+    return run_gemm(ctx, g, e);
+  }
+  return run_gemm(ctx, s, e);
+}
+
 // Stage marks: mark(ctx, nullptr) opens a call, mark(ctx, "name") closes the
 // stage that ran since the previous mark.
 void mark(dust_ctx* ctx, const char* name) {
@@ -265,7 +325,7 @@ void dust_destroy(dust_ctx* ctx) {
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32,
                  &ctx->mlp_dn, &ctx->mlp_du, &ctx->wu2, &ctx->attn_o, &ctx->attn_lse,
-                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr, &ctx->attn_coef};
+                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr, &ctx->attn_coef, &ctx->hsc};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -316,7 +376,8 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   const size_t TV = (size_t)p.T * (size_t)p.V;
   DUST_TRY(ensure(ctx, ctx->z, TV * 4));
   DUST_TRY(ensure(ctx, ctx->lse, (size_t)p.T * 4));
-  DUST_TRY(ensure(ctx, ctx->gop, gop_bytes(p.dtype, p.T, p.V)));
+  const GopFormat gf = head_gop_format(p);
+  DUST_TRY(ensure(ctx, ctx->gop, gop_format_bytes(gf, p.T, p.V)));
   float* loss = loss_out;
   if (!loss) {
     DUST_TRY(ensure(ctx, ctx->loss, (size_t)p.T * 4));
@@ -387,12 +448,12 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
     DUST_CU(launch_full_reward_combine(st, p, (float*)ctx->part.p, (float*)ctx->dzy.p, r));
     ctx->launches += 2;
     mark(ctx, "reward");
-    DUST_CU(launch_full_g(st, p, r, g_out, ctx->gop.p));
+    DUST_CU(launch_full_g(st, p, r, g_out, ctx->gop.p, gf));
     ctx->launches += 1;
     mark(ctx, "g");
   } else if (smem_subset) {
     DUST_CU(launch_subset2(st, p, a, a_inv, Z, (const float*)ctx->lse.p, targets, rewards_out,
-                           g_out, ctx->gop.p, ctx->max_smem_optin, ctx->sm_count,
+                           g_out, ctx->gop.p, gf, ctx->max_smem_optin, ctx->sm_count,
                            ctx->d_status));
     ctx->launches += 1;
     mark(ctx, "subset_draws");
@@ -403,14 +464,17 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
       DUST_TRY(ensure(ctx, ctx->part, gb));
       gacc = (float*)ctx->part.p;
     }
-    DUST_CU(launch_subset_impl(st, p, a, a_inv, Z, targets, rewards_out, g_out, ctx->gop.p, gacc,
+    DUST_CU(launch_subset_impl(st, p, a, a_inv, Z, targets, rewards_out, g_out, ctx->gop.p, gf, gacc,
                                ctx->max_smem_optin));
     ctx->launches += 1;
     mark(ctx, "subset_draws");
   }
   // 4. G_W = sum_t g_t h_t^T (rows un-permuted on the store)
   if (G_out) {
-    DUST_TRY(weight_grad(ctx, p, ctx->gop.p, p.V, H, p.d, G_out, subset ? a : 0));
+    if (gf.kind == kGopF16)
+      DUST_TRY(weight_grad_f16(ctx, p, ctx->gop.p, gf.scale, p.V, H, p.d, G_out, subset ? a : 0));
+    else
+      DUST_TRY(weight_grad(ctx, p, ctx->gop.p, p.V, H, p.d, G_out, subset ? a : 0));
     mark(ctx, "gw_gemm");
   }
   return finish(ctx, p.flags);

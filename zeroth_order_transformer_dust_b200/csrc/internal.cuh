@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cstdint>
 #include <string>
@@ -67,6 +68,7 @@ struct GemmDesc {
   bool b_kmajor;
   int64_t b_row_mul;  // nonzero: B row n is source row (n * b_row_mul) mod N
   int dtype;          // DUST_F32 or DUST_BF16 for both operands
+  bool f16 = false;   // with DUST_BF16: the 2-byte operands are fp16 instead
 };
 
 enum EpiKind {
@@ -106,6 +108,9 @@ struct EpiDesc {
   float* dzy = nullptr;
   // kEpiF32Lse
   float2* lsep = nullptr;
+  // kEpiF32: when set, every stored value is acc * (*scale) (a power of two
+  // written on the device by the kernel that scaled the operands)
+  const float* scale = nullptr;
 };
 
 // Column tile width of the tensor-core GEMM; its epilogues leave two partials
@@ -158,6 +163,30 @@ __device__ __forceinline__ void store_g_operand(float* gop, int64_t, int64_t o, 
   gop[o] = v;
 }
 
+// Formats of the g operand the LM-head draw kernels leave for the G_W GEMM.
+// kGopF16: one fp16 plane holding g * scale, scale = 2^e chosen on the host
+// from the bound the noise puts on g (head_gop_format), so every value is in
+// range; its rounding (2^-11 relative) sits well inside the bf16 G_W
+// tolerance and the GEMM contracts over T instead of the planes' 2T.
+enum GopKind : int { kGopF32 = 0, kGopBf16Planes = 1, kGopF16 = 2 };
+struct GopFormat {
+  int kind;
+  float scale;  // kGopF16 only
+};
+__device__ __forceinline__ void store_gop(void* gop, GopFormat f, int64_t plane, int64_t o,
+                                          float v) {
+  if (f.kind == kGopF16)
+    ((__half*)gop)[o] = __float2half_rn(v * f.scale);
+  else if (f.kind == kGopBf16Planes)
+    store_g_operand((__nv_bfloat16*)gop, plane, o, v);
+  else
+    ((float*)gop)[o] = v;
+}
+// The format of the estimator call: fp32 for fp32 inputs, else kGopF16.
+GopFormat head_gop_format(const dust_params& p);
+// Bytes of a g operand of T x width in format f.
+size_t gop_format_bytes(GopFormat f, int64_t T, int64_t width);
+
 }  // namespace dust
 
 struct dust_ctx {
@@ -184,7 +213,8 @@ struct dust_ctx {
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
-      attn_o, attn_lse, attn_gb, attn_w, attn_tcr, attn_coef;
+      attn_o, attn_lse, attn_gb, attn_w, attn_tcr, attn_coef,
+      hsc;  // the fp16 G_W path's largest |h| and epilogue scale
 };
 
 namespace dust {
@@ -228,9 +258,9 @@ cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, co
 cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, const float* part,
                                        const float* xy, float* r);
 // Stage 3: g_t = -(1/(K sigma)) sum_i r_i eps_i; writes g (fp32, optional) and the
-// GEMM operand gop (bf16 or fp32 by p.dtype).
+// GEMM operand gop in format gf.
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
-                          void* gop);
+                          void* gop, GopFormat gf);
 
 // Subset draws, fused reward + accumulation. P is the probability matrix in
 // permuted column order (column q holds vocabulary index (a q) mod V).
@@ -239,7 +269,7 @@ cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r,
 size_t subset_gacc_bytes(int64_t T, int64_t V, int max_smem_optin);
 cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                                const float* P, const int32_t* y, float* rewards, float* g_out,
-                               void* gop, float* gacc, int max_smem_optin);
+                               void* gop, GopFormat gf, float* gacc, int max_smem_optin);
 
 // Subset draws with the probability row and the g accumulator resident in
 // shared memory, one cluster of 1, 2, 4 or 8 CTAs per token (0: not applicable to
@@ -249,8 +279,8 @@ cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a,
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin);
 cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                            const float* Z, const float* lse, const int32_t* y, float* rewards,
-                           float* g_out, void* gop, int max_smem_optin, int sm_count,
-                           uint32_t* status);
+                           float* g_out, void* gop, GopFormat gf, int max_smem_optin,
+                           int sm_count, uint32_t* status);
 
 // Tensor-core GEMM (tcgen05): shapes it takes, and its launcher (pair: a
 // 256 x 256 tile per cluster of two CTAs, cta_group::2; else 128 x 256 per
@@ -266,6 +296,15 @@ cudaError_t launch_gemm_tc(cudaStream_t st, const GemmDesc& g, const EpiDesc& e,
 // row stride ld_dst >= rows; columns [rows, ld_dst) of dst are zeroed).
 cudaError_t launch_transpose_bf16(cudaStream_t st, const __nv_bfloat16* src, int64_t rows,
                                   int64_t cols, __nv_bfloat16* dst, int64_t ld_dst);
+// H (n bf16 values) as fp16 for the G_W GEMM with the fp16 g operand, in
+// two launches: the largest magnitude into *absmax (as float bits; zero it
+// first), then dst = fp16(x * 2^-s) with s putting that magnitude in
+// [2^14, 2^15), and *epi_scale = 2^s / g_scale for the GEMM epilogue.
+cudaError_t launch_absmax_bf16(cudaStream_t st, const __nv_bfloat16* x, int64_t n,
+                               uint32_t* absmax);
+cudaError_t launch_to_f16_scaled(cudaStream_t st, const __nv_bfloat16* x, int64_t n,
+                                 const uint32_t* absmax, float g_scale, __half* dst,
+                                 float* epi_scale);
 // dst row q = src row (q * mul) mod rows (rows x cols bf16).
 cudaError_t launch_permute_rows_bf16(cudaStream_t st, const __nv_bfloat16* src, int64_t rows,
                                      int64_t cols, int64_t mul, __nv_bfloat16* dst);

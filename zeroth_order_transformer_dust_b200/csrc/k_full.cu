@@ -54,7 +54,7 @@ struct FullArgs {
   const float* r;    // rewards, t * K + i
   float* g_out;
   void* gop;
-  int gop_bf16;
+  GopFormat gf;
   int64_t plane;
 };
 
@@ -246,10 +246,7 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
           const float2 a = (j & 1) ? acc13[b] : acc02[b];
           const float v = ((j & 2) ? a.y : a.x) * A.fac;
           if (A.g_out) A.g_out[t * A.V + pos] = v;
-          if (A.gop_bf16)
-            store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + pos, v);
-          else
-            ((float*)A.gop)[t * A.V + pos] = v;
+          store_gop(A.gop, A.gf, A.plane, t * A.V + pos, v);
         }
       }
   }
@@ -268,7 +265,6 @@ FullArgs make_args(const dust_params& p) {
   A.V = p.V;
   A.K = p.K;
   A.nslab = (int)((p.V + kSlab - 1) / kSlab);
-  A.gop_bf16 = p.dtype == DUST_BF16;
   A.plane = p.T * p.V;
   return A;
 }
@@ -326,11 +322,12 @@ cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, co
 }
 
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
-                          void* gop) {
+                          void* gop, GopFormat gf) {
   FullArgs A = make_args(p);
   A.r = r;
   A.g_out = g_out;
   A.gop = gop;
+  A.gf = gf;
   k_full_g<<<grid_for(k_full_g, A.T * A.nslab), kWarps * 32, 0, st>>>(A);
   return cudaGetLastError();
 }

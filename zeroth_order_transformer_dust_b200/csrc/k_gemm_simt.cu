@@ -10,6 +10,7 @@ constexpr int BM = 128, BN = 128, BKT = 16, PAD = 4;
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 
 // Loads the A (or B) tile of rows [r0, r0+128) and k in [k0, k0+16) into
 // S[k][row] as fp32, zero-filling outside the matrix.
@@ -80,6 +81,7 @@ __global__ __launch_bounds__(256) void k_gemm_simt(GemmDesc g, EpiDesc e) {
     __syncthreads();
   }
 
+  const float escale = (e.kind == kEpiF32 && e.scale) ? *e.scale : 1.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
@@ -94,7 +96,7 @@ __global__ __launch_bounds__(256) void k_gemm_simt(GemmDesc g, EpiDesc e) {
       const float v = acc[i][j];
       switch (e.kind) {
         case kEpiF32:
-          e.C[mo * e.ldc + n] = v;
+          e.C[mo * e.ldc + n] = v * escale;
           break;
         case kEpiBF16:
           e.Cb[m * e.ldcb + n] = __float2bfloat16_rn(v);
@@ -131,6 +133,7 @@ cudaError_t dispatch(cudaStream_t st, const GemmDesc& g, const EpiDesc& e) {
 
 cudaError_t launch_gemm_simt(cudaStream_t st, const GemmDesc& g, const EpiDesc& e) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
+  if (g.dtype == DUST_BF16 && g.f16) return dispatch<__half>(st, g, e);
   if (g.dtype == DUST_BF16) return dispatch<__nv_bfloat16>(st, g, e);
   return dispatch<float>(st, g, e);
 }

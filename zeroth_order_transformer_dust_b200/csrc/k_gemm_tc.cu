@@ -1,5 +1,5 @@
-// Tensor-core GEMM for sm_100a: C = A B^T with bf16 operands and fp32
-// accumulation. Each operand is K-major (A as M x K rows, B as N x K) or
+// Tensor-core GEMM for sm_100a: C = A B^T with bf16 (or fp16) operands and
+// fp32 accumulation. Each operand is K-major (A as M x K rows, B as N x K) or
 // MN-major (A stored as K x M rows, B as K x N), read as stored by TMA.
 //
 // Persistent, warp-specialised CTA (one per SM): warp 0 issues TMA tile loads
@@ -77,6 +77,7 @@ struct TcParams {
   int m_tiles, n_tiles, num_kb;  // m_tiles counts Cfg::TILE_M-row tiles
   int tma_store;                 // kEpiF32Lse: C is stored through tmC
   int a_mn, b_mn;                // operand stored MN-major (K x M, K x N rows)
+  int f16;                       // fp16 operands (kind::f16 takes both types)
   EpiDesc e;
   uint32_t* status;
   uint64_t wait_ns;  // limit of the pipeline waits (teardown waits keep kWaitLimitNs)
@@ -118,9 +119,13 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
 // Epilogue of 32 consecutive columns [n, n+32) of row m (output row mo).
 template <int KIND>
 __device__ __forceinline__ void epilogue32(const TcParams& p, int64_t m, int64_t mo, int64_t n,
-                                           const float* v) {
+                                           float* v, float escale) {
   const EpiDesc& e = p.e;
   const bool full = n + 32 <= p.N;
+  if (KIND == kEpiF32) {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) v[q] *= escale;
+  }
   if (KIND == kEpiF32 || KIND == kEpiF32Lse || KIND == kEpiGeluSplit) {
     float* dst = e.C + (KIND == kEpiF32 ? mo : m) * e.ldc + n;
     if (full && ((e.ldc & 3) == 0) && (((uintptr_t)e.C & 15) == 0)) {
@@ -459,8 +464,9 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && leader) {
-      const uint32_t idesc = ptx::idesc_bf16_f32(TILE_M, BN) | (p.a_mn ? ptx::kIdescAMn : 0u) |
-                             (p.b_mn ? ptx::kIdescBMn : 0u);
+      const uint32_t idesc =
+          (p.f16 ? ptx::idesc_f16_f32(TILE_M, BN) : ptx::idesc_bf16_f32(TILE_M, BN)) |
+          (p.a_mn ? ptx::kIdescAMn : 0u) | (p.b_mn ? ptx::kIdescBMn : 0u);
       // per 16-deep MMA step: 32 bytes along a K-major row, two 8-row
       // swizzle atoms (2048 bytes) down an MN-major tile
       const uint32_t a_step = p.a_mn ? 2048u : 32u, b_step = p.b_mn ? 2048u : 32u;
@@ -528,6 +534,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     const int row = quad * 32 + lane;
     const int half = (warp - 2) >> 2;  // columns [HALF_N half, HALF_N (half + 1)) of the tile
     int it = 0;
+    // kEpiF32: the output scale (a power of two the operands' producer wrote)
+    const float escale = (KIND == kEpiF32 && p.e.scale) ? *p.e.scale : 1.0f;
     int nbox = 0;  // kEpiF32Lse: store boxes this warp has issued
     const uint32_t box0 = sStore + (uint32_t)((warp - 2) * STORE_BUFS * STORE_BOX_BYTES);
     const uint32_t tempty0 =
@@ -622,7 +630,7 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           ++nbox;
           if (m < p.M) lse_chunk(p, n, v, rmax, rsum);
         } else if (m < p.M && n < p.N) {
-          epilogue32<KIND>(p, m, mo, n, v);
+          epilogue32<KIND>(p, m, mo, n, v, escale);
           if (KIND == kEpiF32Lse) lse_chunk(p, n, v, rmax, rsum);
         }
       }
@@ -669,17 +677,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix (rows x cols, row stride ld elements) as a TMA map with
-// a box of 64 columns x box_rows rows and 128-byte swizzling.
+// Row-major bf16 (or fp16) matrix (rows x cols, row stride ld elements) as a
+// TMA map with a box of 64 columns x box_rows rows and 128-byte swizzling.
 bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
-              int box_rows) {
+              int box_rows, bool f16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
   cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+  return fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -752,10 +761,10 @@ template <bool PAIR>
 cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, int sm_count,
                         uint32_t* status, uint64_t wait_ns) {
   CUtensorMap ma, mb, mc;
-  const bool ok_a = g.a_kmajor ? make_map(&ma, g.A, g.M, g.K, g.lda, BM)
-                               : make_map(&ma, g.A, g.K, g.M, g.lda, BK);
-  const bool ok_b = g.b_kmajor ? make_map(&mb, g.B, g.N, g.K, g.ldb, Cfg<PAIR, kEpiF32>::B_ROWS)
-                               : make_map(&mb, g.B, g.K, g.N, g.ldb, BK);
+  const bool ok_a = g.a_kmajor ? make_map(&ma, g.A, g.M, g.K, g.lda, BM, g.f16)
+                               : make_map(&ma, g.A, g.K, g.M, g.lda, BK, g.f16);
+  const bool ok_b = g.b_kmajor ? make_map(&mb, g.B, g.N, g.K, g.ldb, Cfg<PAIR, kEpiF32>::B_ROWS, g.f16)
+                               : make_map(&mb, g.B, g.K, g.N, g.ldb, BK, g.f16);
   if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   memset(&mc, 0, sizeof(mc));
   // kEpiF32Lse stores C through a TMA map when its rows are 16-byte aligned
@@ -768,6 +777,7 @@ cudaError_t launch_pair(cudaStream_t st, const GemmDesc& g, const EpiDesc& e, in
   p.K = g.K;
   p.m_tiles = (int)((g.M + Cfg<PAIR, kEpiF32>::TILE_M - 1) / Cfg<PAIR, kEpiF32>::TILE_M);
   p.tma_store = tma_store ? 1 : 0;
+  p.f16 = g.f16 ? 1 : 0;
   p.a_mn = g.a_kmajor ? 0 : 1;
   p.b_mn = g.b_kmajor ? 0 : 1;
   p.n_tiles = (int)((g.N + BN - 1) / BN);

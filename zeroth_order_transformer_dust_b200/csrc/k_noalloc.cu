@@ -172,6 +172,8 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
     const size_t gb = subset_gacc_bytes(p.T, p.V, max_smem);
     if (gb) gacc = (float*)cv.take(gb);
   }
+  // g operand: bf16 hi/lo planes (2T rows) for bf16 inputs, fp32 otherwise
+  const GopFormat gf{bf16 ? kGopBf16Planes : kGopF32, 1.0f};
   void* gop = cv.take(bf16 ? 2 * T * V * 2 : T * V * 4);
   void* xdup = (bf16 && G_out) ? cv.take(2 * T * (size_t)p.d * 2) : nullptr;
 
@@ -190,9 +192,9 @@ extern "C" dust_status dust_head_grad_noalloc(const dust_params* pp, void* cuda_
   if (!subset) {
     if (e == cudaSuccess) e = launch_full_reward_partial(st, p, Z, lse, targets, part, xy);
     if (e == cudaSuccess) e = launch_full_reward_combine(st, p, part, xy, r);
-    if (e == cudaSuccess) e = launch_full_g(st, p, r, g_out, gop);
+    if (e == cudaSuccess) e = launch_full_g(st, p, r, g_out, gop, gf);
   } else if (e == cudaSuccess) {
-    e = launch_subset_impl(st, p, a, a_inv, Z, targets, rewards_out, g_out, gop, gacc, max_smem);
+    e = launch_subset_impl(st, p, a, a_inv, Z, targets, rewards_out, g_out, gop, gf, gacc, max_smem);
   }
   if (G_out && e == cudaSuccess) {
     GemmDesc w{};

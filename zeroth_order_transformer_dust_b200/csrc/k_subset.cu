@@ -35,7 +35,7 @@ struct SubsetArgs {
   float* g_out;
   void* gop;
   float* gacc;  // global accumulator rows (only when the row does not fit in smem)
-  int gop_bf16;
+  GopFormat gf;
   int64_t plane;  // distance between the hi and lo planes of the bf16 operand
 };
 
@@ -166,10 +166,7 @@ __global__ __launch_bounds__(kThreads, 1) void k_subset(SubsetArgs A) {
 
   for (int64_t q = threadIdx.x; q < V; q += kThreads) {
     const float v = G[q] * ((uint32_t)q == qy ? A.scale_target : A.scale_other) * A.fac;
-    if (A.gop_bf16)
-      store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * V + q, v);
-    else
-      ((float*)A.gop)[t * V + q] = v;
+    store_gop(A.gop, A.gf, A.plane, t * V + q, v);
     if (A.g_out) A.g_out[t * V + mulmod((uint32_t)q, (uint64_t)A.a, V)] = v;
   }
 }
@@ -206,7 +203,7 @@ size_t subset_gacc_bytes(int64_t T, int64_t V, int max_smem_optin) {
 
 cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                                const float* P, const int32_t* y, float* rewards, float* g_out,
-                               void* gop, float* gacc, int max_smem_optin) {
+                               void* gop, GopFormat gf, float* gacc, int max_smem_optin) {
   SubsetArgs A;
   A.key = key_of(p.seed);
   A.t_off = (uint32_t)p.token_offset;
@@ -228,7 +225,7 @@ cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a,
   A.g_out = g_out;
   A.gop = gop;
   A.gacc = gacc;
-  A.gop_bf16 = p.dtype == DUST_BF16;
+  A.gf = gf;
   A.plane = p.T * p.V;
   const int deg = expm1_degree(p.sigma);
   const size_t smem = (size_t)p.V * 4;

@@ -101,7 +101,7 @@ struct Sub2Args {
   float* rewards;
   float* g_out;
   void* gop;
-  int gop_bf16;
+  GopFormat gf;
   int64_t plane;
 };
 
@@ -493,10 +493,7 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
       else
         v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
       sg[q] = 0.0f;
-      if (A.gop_bf16)
-        store_g_operand((__nv_bfloat16*)A.gop, A.plane, t * A.V + qg, v);
-      else
-        ((float*)A.gop)[t * A.V + qg] = v;
+      store_gop(A.gop, A.gf, A.plane, t * A.V + qg, v);
       if (A.g_out) A.g_out[t * A.V + mulmod(qg, A.a, V, A.minv)] = v;
     }
     __syncthreads();
@@ -578,8 +575,8 @@ int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
 
 cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
                            const float* Z, const float* lse, const int32_t* y, float* rewards,
-                           float* g_out, void* gop, int max_smem_optin, int sm_count,
-                           uint32_t* status) {
+                           float* g_out, void* gop, GopFormat gf, int max_smem_optin,
+                           int sm_count, uint32_t* status) {
   const int cs = subset2_cluster_size(p.V, p.S, max_smem_optin);
   if (!status) return cudaErrorInvalidValue;
   if (!cs) return cudaErrorNotSupported;
@@ -616,7 +613,7 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.rewards = rewards;
   A.g_out = g_out;
   A.gop = gop;
-  A.gop_bf16 = p.dtype == DUST_BF16;
+  A.gf = gf;
   A.plane = p.T * p.V;
   const size_t smem = (size_t)2 * A.seg * 4;
   const int deg = expm1_degree(p.sigma);
