@@ -130,8 +130,16 @@ dust_status dust_check(dust_ctx* ctx);
  * first word of counter (0, t, i, 1|(stream_id<<8)); the target is always
  * included (as slot S when not drawn); g is scaled per coordinate by its
  * inverse inclusion probability (V/S; 1 for the target).
+ * With bf16 inputs G_out is contracted on tensor cores from g as one fp16
+ * plane scaled by a power of two (the noise bounds |g| by 66.6 times its
+ * inclusion scale, so every value is in range) and from H as fp16 with a
+ * power-of-two scale taken from its largest magnitude (exact for bf16 values
+ * in fp16's normal range): about 3e-4 relative error (Frobenius) from the
+ * rounding of g. fp32 inputs keep fp32 throughout.
  * Errors: DUST_ERR_ARG (validation), DUST_ERR_BOUNDS (a target outside
- * [0, V): outputs are then unspecified), DUST_ERR_OOM, DUST_ERR_CUDA.
+ * [0, V): outputs are then unspecified), DUST_ERR_OOM, DUST_ERR_CUDA,
+ * DUST_ERR_TIMEOUT (a bounded device wait expired: a GEMM pipeline stage or a
+ * subset-draw row copy; outputs unspecified, the context stays usable).
  */
 dust_status dust_head_grad(dust_ctx* ctx, const dust_params* p,
                            const void* H, const void* W, const int32_t* targets,

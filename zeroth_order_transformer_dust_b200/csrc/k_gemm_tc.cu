@@ -364,6 +364,11 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = p.m_tiles * p.n_tiles;
+  // MN-major and fp16 operands are taken by the plain fp32 epilogue (the
+  // weight gradient) only; the other kinds keep the K-major bf16 code
+  const bool a_mn = KIND == kEpiF32 && p.a_mn != 0;
+  const bool b_mn = KIND == kEpiF32 && p.b_mn != 0;
+  const bool f16 = KIND == kEpiF32 && p.f16 != 0;
   // CTA pairs work on one tile together: unit = pair index, rank 0 leads
   const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
   const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
@@ -439,8 +444,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
           } else {
             ptx::mbar_expect_tx(fb, STAGE_BYTES);
           }
-          load(sA + stage * A_BYTES, &tmA, p.a_mn != 0, BM, a_row, kb * BK, bar);
-          load(sB + stage * B_BYTES, &tmB, p.b_mn != 0, C::B_ROWS, b_row, kb * BK, bar);
+          load(sA + stage * A_BYTES, &tmA, a_mn, BM, a_row, kb * BK, bar);
+          load(sB + stage * B_BYTES, &tmB, b_mn, C::B_ROWS, b_row, kb * BK, bar);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -465,11 +470,11 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
     // ---------------- MMA issuer ----------------
     if (lane == 0 && leader) {
       const uint32_t idesc =
-          (p.f16 ? ptx::idesc_f16_f32(TILE_M, BN) : ptx::idesc_bf16_f32(TILE_M, BN)) |
-          (p.a_mn ? ptx::kIdescAMn : 0u) | (p.b_mn ? ptx::kIdescBMn : 0u);
+          (f16 ? ptx::idesc_f16_f32(TILE_M, BN) : ptx::idesc_bf16_f32(TILE_M, BN)) |
+          (a_mn ? ptx::kIdescAMn : 0u) | (b_mn ? ptx::kIdescBMn : 0u);
       // per 16-deep MMA step: 32 bytes along a K-major row, two 8-row
       // swizzle atoms (2048 bytes) down an MN-major tile
-      const uint32_t a_step = p.a_mn ? 2048u : 32u, b_step = p.b_mn ? 2048u : 32u;
+      const uint32_t a_step = a_mn ? 2048u : 32u, b_step = b_mn ? 2048u : 32u;
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -491,8 +496,8 @@ __global__ __launch_bounds__(THREADS, 1) void k_gemm_tc(const __grid_constant__ 
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint32_t ak = a0 + k * a_step, bk = b0 + k * b_step;
-            const uint64_t ad = p.a_mn ? ptx::sdesc_mnmajor_sw128(ak, MN_BOX) : ptx::sdesc_kmajor_sw128(ak);
-            const uint64_t bd = p.b_mn ? ptx::sdesc_mnmajor_sw128(bk, MN_BOX) : ptx::sdesc_kmajor_sw128(bk);
+            const uint64_t ad = a_mn ? ptx::sdesc_mnmajor_sw128(ak, MN_BOX) : ptx::sdesc_kmajor_sw128(ak);
+            const uint64_t bd = b_mn ? ptx::sdesc_mnmajor_sw128(bk, MN_BOX) : ptx::sdesc_kmajor_sw128(bk);
             if (PAIR)
               ptx::mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
             else
@@ -742,6 +747,8 @@ cudaError_t launch_kind(cudaStream_t st, const CUtensorMap& a, const CUtensorMap
 
 bool tc_gemm_supported(const GemmDesc& g, const EpiDesc& e) {
   if (g.dtype != DUST_BF16 || g.b_row_mul != 0) return false;
+  // MN-major or fp16 operands: the plain fp32 epilogue only
+  if ((!g.a_kmajor || !g.b_kmajor || g.f16) && e.kind != kEpiF32) return false;
   if (g.M < 1 || g.N < 16 || g.K < 8) return false;
   if ((g.lda & 7) || (g.ldb & 7)) return false;
   if (((uintptr_t)g.A & 15) || ((uintptr_t)g.B & 15)) return false;
