@@ -54,6 +54,11 @@ def _compile(src: str, extra) -> str:
     proc = subprocess.run(cmd, capture_output=True, text=True)
     if proc.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{proc.stdout}\n{proc.stderr}")
+    # warnings (register spills among them: -warn-spills) are shown even when
+    # the compile succeeds
+    warn = [ln for ln in (proc.stdout + proc.stderr).splitlines() if "warning" in ln.lower()]
+    if warn:
+        print(f"{os.path.basename(src)}:\n  " + "\n  ".join(warn), file=sys.stderr)
     return obj
 
 

@@ -64,8 +64,10 @@ namespace {
 // registers (4.5% less time at 32 than at 16 warps on the large-subset
 // workload); the fp32-accumulator variant and the library expm1 (large sigma)
 // keep 16 warps, where they need no spills.
-__host__ __device__ constexpr int sub2_threads(bool use_int, int deg) {
-  return use_int && deg != 0 ? 1024 : 512;
+// NB = 3 (the packed Box-Muller step, the tightest variant) also keeps 16
+// warps: at 64 registers it spills whatever else the kernel holds.
+__host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb) {
+  return use_int && deg != 0 && nb != 3 ? 1024 : 512;
 }
 
 // The Box-Muller step of NB-block draws in packed fp32x2 form, else scalar
@@ -103,6 +105,9 @@ struct Sub2Args {
   void* gop;
   GopFormat gf;
   int64_t plane;
+  // g = accumulator * w_other off the target; on it s_tgt * w_target (fixed
+  // point) or its accumulator * w_target (fp32)
+  float w_other, w_target;
 };
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -131,8 +136,8 @@ __device__ __forceinline__ void accumulate(float* slot, float r, float x, float 
 
 // NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
 template <int NB, bool FULL, int DEG, bool INT>
-__global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
-  constexpr int kThreads = sub2_threads(INT, DEG);
+__global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
+  constexpr int kThreads = sub2_threads(INT, DEG, NB);
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_next;    // next draw batch of the current token
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
@@ -191,9 +196,6 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
   BlockConst bc[NB];
 #pragma unroll
   for (int m = 0; m < NB; ++m) bc[m] = block_const(A.keys, slot_ctr0((uint32_t)m, (uint32_t)lane), A.ctr3);
-  // the appended target slot S: counter block S >> 7, lane S & 31, word (S >> 5) & 3
-  const BlockConst bs = block_const(A.keys, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u), A.ctr3);
-  const uint32_t s_word = ((uint32_t)S >> 5) & 3u;
   const bool vec = (V & 3u) == 0;  // rows start 16-byte aligned
   // the pipelined row copy (one bulk copy of n_own floats; 16-byte aligned
   // source and size when V % 4 == 0, the slices being multiples of 4)
@@ -302,6 +304,11 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
       kyq = (qy >= c) ? qy - c : qy + V - c;
       x_extra = 0.0f;
       if (mine && kyq >= (uint32_t)S) {
+        // the appended target slot S: counter block S >> 7, lane S & 31,
+        // word (S >> 5) & 3 (its block constants formed here, once per
+        // batch and lane, rather than held in registers)
+        const BlockConst bs = block_const(A.keys, slot_ctr0((uint32_t)S >> 7, (uint32_t)S & 31u), A.ctr3);
+        const uint32_t s_word = ((uint32_t)S >> 5) & 3u;
         const U4 w = philox_from2(bs, draw_const(A.keys, t_abs, i_abs), A.keys);
         const float2 nn = box_muller_tab(s_word < 2 ? w.x : w.z, s_word < 2 ? w.y : w.w, s_tab);
         x_extra = (s_word & 1u) ? nn.y : nn.x;
@@ -483,8 +490,51 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
     if (threadIdx.x == 0 && s_row_n) issue_row(s_row_n);
 
     // ---- scale and write the owned slice of g, and clear it for the next
-    // token
-    for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
+    // token: four entries per step for the fp16 operand of 16-byte rows
+    // (one shared-memory read and clear, one 8-byte store), else one
+    // (NB <= 2 only: NB = 3 and 4 have no registers to spare around their
+    // draw loop, and at their sizes the pass is a smaller share of a token)
+    bool vec_out = false;
+    if constexpr (NB <= 2) vec_out = (V & 3u) == 0 && A.gf.kind == kGopF16;
+    if constexpr (NB <= 2) if (vec_out) {
+      // g = acc so, the target's from its own sum; the optional fp32 g in
+      // vocabulary order first, while the accumulator is intact
+      if (A.g_out) {
+        for (uint32_t q = threadIdx.x; q < n_own; q += kThreads) {
+          const uint32_t qg = lo + q;
+          const float x = INT ? (float)reinterpret_cast<const int*>(sg)[q] : sg[q];
+          A.g_out[t * A.V + mulmod(qg, A.a, V, A.minv)] =
+              qg == qy ? (INT ? s_tgt : x) * A.w_target : x * A.w_other;
+        }
+        __syncthreads();  // every entry read before the loop below clears it
+      }
+      __half* orow = (__half*)A.gop + t * A.V + lo;
+      for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
+        float4 a4 = *reinterpret_cast<const float4*>(sg + q);
+        *reinterpret_cast<float4*>(sg + q) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (INT)
+          a4 = make_float4((float)__float_as_int(a4.x), (float)__float_as_int(a4.y),
+                           (float)__float_as_int(a4.z), (float)__float_as_int(a4.w));
+        float v0 = a4.x * A.w_other, v1 = a4.y * A.w_other, v2 = a4.z * A.w_other,
+              v3 = a4.w * A.w_other;
+        if (qy - lo - q < 4u) {  // the target among these four
+          const uint32_t j = qy - lo - q;
+          const float vt =
+              (INT ? s_tgt : (j == 0 ? a4.x : j == 1 ? a4.y : j == 2 ? a4.z : a4.w)) * A.w_target;
+          v0 = j == 0 ? vt : v0;
+          v1 = j == 1 ? vt : v1;
+          v2 = j == 2 ? vt : v2;
+          v3 = j == 3 ? vt : v3;
+        }
+        const __half2 h01 = __floats2half2_rn(v0 * A.gf.scale, v1 * A.gf.scale);
+        const __half2 h23 = __floats2half2_rn(v2 * A.gf.scale, v3 * A.gf.scale);
+        *reinterpret_cast<uint2*>(orow + q) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+      }
+    }
+    // one entry per step otherwise; the operand is fp16 (bf16 inputs) or
+    // fp32, the launch takes no other, and each has a loop of its own
+    auto entry = [&](uint32_t q) {
       const uint32_t qg = lo + q;
       float v;
       if (INT)
@@ -493,8 +543,15 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG), 1) void k_subset2(const __g
       else
         v = sg[q] * (qg == qy ? A.scale_target : A.scale_other) * A.fac;
       sg[q] = 0.0f;
-      store_gop(A.gop, A.gf, A.plane, t * A.V + qg, v);
       if (A.g_out) A.g_out[t * A.V + mulmod(qg, A.a, V, A.minv)] = v;
+      return v;
+    };
+    if (!vec_out && A.gf.kind == kGopF16) {
+      for (uint32_t q = threadIdx.x; q < n_own; q += kThreads)
+        ((__half*)A.gop)[t * A.V + lo + q] = __float2half_rn(entry(q) * A.gf.scale);
+    } else if (!vec_out) {
+      for (uint32_t q = threadIdx.x; q < n_own; q += kThreads)
+        ((float*)A.gop)[t * A.V + lo + q] = entry(q);
     }
     __syncthreads();
   }
@@ -513,7 +570,7 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(sub2_threads(INT, DEG));
+  cfg.blockDim = dim3(sub2_threads(INT, DEG, NB));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -578,7 +635,7 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
                            float* g_out, void* gop, GopFormat gf, int max_smem_optin,
                            int sm_count, uint32_t* status) {
   const int cs = subset2_cluster_size(p.V, p.S, max_smem_optin);
-  if (!status) return cudaErrorInvalidValue;
+  if (!status || gf.kind == kGopBf16Planes) return cudaErrorInvalidValue;
   if (!cs) return cudaErrorNotSupported;
   Sub2Args A;
   A.key = key_of(p.seed);
@@ -606,6 +663,9 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   const double units = 32768.0 * (p.K > 16384 ? 16384.0 / (double)p.K : 1.0);
   A.acc_scale = p.sigma > 0.0f ? (float)(units / s2) : 0.0f;
   A.fac_int = p.sigma > 0.0f ? (float)(-1.0 / ((double)p.K * units)) : 0.0f;
+  const bool use_int = p.K <= 65536;
+  A.w_other = use_int ? A.fac_int * A.scale_other : A.fac * A.scale_other;
+  A.w_target = A.fac * A.scale_target;
   A.status = status;
   A.Z = Z;
   A.lse = lse;
@@ -617,7 +677,6 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.plane = p.T * p.V;
   const size_t smem = (size_t)2 * A.seg * 4;
   const int deg = expm1_degree(p.sigma);
-  const bool use_int = p.K <= 65536;
   return use_int ? launch_nb<true>(st, A, smem, sm_count, deg)
                  : launch_nb<false>(st, A, smem, sm_count, deg);
 }
