@@ -227,7 +227,9 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
   for (int64_t t = cid; t < A.T; t += nclusters) {
     const float lse_t = s_lse_n;
     int32_t yt = s_y_n;
-    // ---- p = exp(z - LSE) for the owned slice (and clear g without bulk)
+    // ---- p = exp(z - LSE) for the owned slice (and clear g without bulk),
+    // by the hardware exponential: its relative error, about 1e-6 at
+    // z - LSE = -20 and less nearer 0, moves the reward sum by under 1e-7
     const float* zrow = A.Z + t * A.V;
     if (bulk) {
       // thread 0 waits for the row (the k-th token of this cluster for
@@ -253,17 +255,17 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
       for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
         const float4 z = *reinterpret_cast<const float4*>(sp + q);
         *reinterpret_cast<float4*>(sp + q) =
-            make_float4(expf(z.x - lse_t), expf(z.y - lse_t), expf(z.z - lse_t), expf(z.w - lse_t));
+            make_float4(__expf(z.x - lse_t), __expf(z.y - lse_t), __expf(z.z - lse_t), __expf(z.w - lse_t));
       }
     } else for (uint32_t q = threadIdx.x * 4; q < n_own; q += kThreads * 4) {
       if (vec && q + 3 < n_own) {
         const float4 z = *reinterpret_cast<const float4*>(zrow + lo + q);
         *reinterpret_cast<float4*>(sp + q) =
-            make_float4(expf(z.x - lse_t), expf(z.y - lse_t), expf(z.z - lse_t), expf(z.w - lse_t));
+            make_float4(__expf(z.x - lse_t), __expf(z.y - lse_t), __expf(z.z - lse_t), __expf(z.w - lse_t));
         *reinterpret_cast<float4*>(sg + q) = make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
         for (uint32_t u = q; u < n_own && u < q + 4; ++u) {
-          sp[u] = expf(zrow[lo + u] - lse_t);
+          sp[u] = __expf(zrow[lo + u] - lse_t);
           sg[u] = 0.0f;
         }
       }
