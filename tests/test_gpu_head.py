@@ -101,6 +101,9 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     dict(V=4099, K=20), dict(V=20000, K=33, T=5, d=16), dict(V=100000, K=9, T=3, d=16),
     dict(T=200, K=5, V=1000), dict(T=300, K=2, V=3000, dtype="f32"),
     dict(V=120000, K=8, T=3, d=16),
+    # the per-token draw list (K <= 512, S <= 256) with clusters of two CTAs
+    # and several tokens per cluster
+    dict(V=50304, S=256, K=512, T=160, d=16),
 ])
 def test_edge_shapes(ctx, kw):
     wl = _small(**kw)

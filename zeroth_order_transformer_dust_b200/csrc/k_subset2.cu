@@ -18,7 +18,9 @@
 // a shared counter; in a batch each lane works out one draw's window start,
 // whether its window holds the target and the noise of the appended target
 // slot, and the warp then processes, one after the other, the draws whose
-// window starts in its CTA's slice. A window is no longer than a slice, so
+// window starts in its CTA's slice. With few draws (K <= 512, S <= 256) the
+// draws of a token are set up together instead, the CTA's own collected in a
+// shared list that is dealt out to the warps in turn (LIST). A window is no longer than a slice, so
 // the part that runs past the slice (or wraps past V, which only a window
 // starting in the last slice can do) lies in the next CTA's slice,
 // (r + 1) mod CS, reached through DSMEM. The noise of a draw is generated
@@ -134,12 +136,14 @@ __device__ __forceinline__ void accumulate(float* slot, float r, float x, float 
     atomicAdd(slot, r * x);
 }
 
-// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB.
-template <int NB, bool FULL, int DEG, bool INT>
+// NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB; LIST: the
+// per-token draw list (its 16-byte entries follow the slices in shared memory).
+template <int NB, bool FULL, int DEG, bool INT, bool LIST>
 __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
   constexpr int kThreads = sub2_threads(INT, DEG, NB);
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_next;    // next draw batch of the current token
+  __shared__ int s_cnt;     // LIST: entries of the current token's draw list
   __shared__ float s_tgt;   // INT: sum r * (sigma eps_y) of the target coordinate
   __shared__ float2 s_tab[kSinCosTable];
   __shared__ __align__(8) uint64_t s_row;  // completion of the row copy
@@ -217,6 +221,7 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
   }
   // the LSE and target of a token are loaded a token ahead (thread 0, into
   // shared memory, read after the barrier that ends the previous token)
+  if (threadIdx.x == 0) s_cnt = 0;
   if (threadIdx.x == 0 && (int64_t)cid < A.T) {
     s_lse_n = A.lse[cid];
     s_y_n = A.y[cid];
@@ -278,23 +283,7 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
     const uint32_t qy = mulmod((uint32_t)yt, A.a_inv, V, A.minv);
     const uint32_t owner_y = qy / seg;  // the CTA whose slice holds the target
     float* gy = cluster.map_shared_rank(sg, owner_y) + (qy - owner_y * seg);
-    cluster.sync();
-    // p of the target, from the owner's shared memory
-    const float py = cluster.map_shared_rank(sp, owner_y)[qy - owner_y * seg];
-    if (threadIdx.x == 0) {
-      const int64_t tn = t + nclusters;
-      const float* zn = nullptr;
-      if (tn < A.T) {
-        zn = A.Z + tn * A.V + lo;
-        if (bulk) ptx::bulk_prefetch_l2(zn, n_own * 4u);
-        s_lse_n = A.lse[tn];
-        s_y_n = A.y[tn];
-      }
-      s_row_n = bulk ? zn : nullptr;
-    }
-
     const uint32_t t_abs = A.t_off + (uint32_t)t;
-    float tgt_acc = 0.0f;  // INT: this warp's sum r * (sigma eps_y), lane 0
     // Setup of draw iq (one lane): its window start in permuted order, the
     // target's slot in the window, and whether the window starts in this
     // CTA's slice; for those, the noise of the appended target slot.
@@ -317,6 +306,40 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
       }
       return mine;
     };
+    if constexpr (LIST) {
+      // every draw set up at once, the ones whose window starts in this
+      // CTA's slice appended to the list (one atomic per warp)
+      uint4* s_list = reinterpret_cast<uint4*>(smem + 2 * seg);
+      for (int iq0 = (int)(threadIdx.x & ~31u); iq0 < A.K; iq0 += kThreads) {
+        const int iq = iq0 + lane;
+        uint32_t c = 0, kyq = 0;
+        float xe = 0.0f;
+        const bool mine = iq < A.K && setup(iq, c, kyq, xe);
+        const uint32_t m = __ballot_sync(0xffffffffu, mine);
+        int base = 0;
+        if (lane == 0 && m) base = atomicAdd(&s_cnt, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (mine)
+          s_list[base + __popc(m & ((1u << lane) - 1u))] =
+              make_uint4((uint32_t)iq, c, kyq, __float_as_uint(xe));
+      }
+    }
+    cluster.sync();
+    // p of the target, from the owner's shared memory
+    const float py = cluster.map_shared_rank(sp, owner_y)[qy - owner_y * seg];
+    if (threadIdx.x == 0) {
+      const int64_t tn = t + nclusters;
+      const float* zn = nullptr;
+      if (tn < A.T) {
+        zn = A.Z + tn * A.V + lo;
+        if (bulk) ptx::bulk_prefetch_l2(zn, n_own * 4u);
+        s_lse_n = A.lse[tn];
+        s_y_n = A.y[tn];
+      }
+      s_row_n = bulk ? zn : nullptr;
+    }
+
+    float tgt_acc = 0.0f;  // INT: this warp's sum r * (sigma eps_y), lane 0
     // Draw i with window start cw, target slot ky and appended-slot noise xe,
     // by the whole warp: reward, then accumulation into g.
     auto draw = [&](int i, uint32_t cw, uint32_t ky, float xe) {
@@ -469,25 +492,37 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
         atomicAdd(gy, r * xy);
       }
     };
-    for (;;) {
-      int bidx = 0;
-      if (lane == 0) bidx = atomicAdd(&s_next, 1);
-      bidx = __shfl_sync(0xffffffffu, bidx, 0);
-      if (bidx >= nbatch) break;
-      const int iq = bidx * 32 + lane;
-      uint32_t c = 0, kyq = 0;
-      float x_extra = 0.0f;
-      const bool mine = iq < A.K && setup(iq, c, kyq, x_extra);
-      uint32_t mask = __ballot_sync(0xffffffffu, mine);
-      while (mask) {
-        const int src = __ffs(mask) - 1;
-        mask &= mask - 1;
-        draw(bidx * 32 + src, __shfl_sync(0xffffffffu, c, src), __shfl_sync(0xffffffffu, kyq, src),
-             __shfl_sync(0xffffffffu, x_extra, src));
+    if constexpr (LIST) {
+      // the list dealt out in turn: entry j to warp j mod (warps per CTA),
+      // so no warp runs more than one draw beyond another
+      const uint4* s_list = reinterpret_cast<const uint4*>(smem + 2 * seg);
+      const int cnt = s_cnt;
+      for (int j = (int)(threadIdx.x >> 5); j < cnt; j += kThreads / 32) {
+        const uint4 e = s_list[j];
+        draw((int)e.x, e.y, e.z, __uint_as_float(e.w));
+      }
+    } else {
+      for (;;) {
+        int bidx = 0;
+        if (lane == 0) bidx = atomicAdd(&s_next, 1);
+        bidx = __shfl_sync(0xffffffffu, bidx, 0);
+        if (bidx >= nbatch) break;
+        const int iq = bidx * 32 + lane;
+        uint32_t c = 0, kyq = 0;
+        float x_extra = 0.0f;
+        const bool mine = iq < A.K && setup(iq, c, kyq, x_extra);
+        uint32_t mask = __ballot_sync(0xffffffffu, mine);
+        while (mask) {
+          const int src = __ffs(mask) - 1;
+          mask &= mask - 1;
+          draw(bidx * 32 + src, __shfl_sync(0xffffffffu, c, src), __shfl_sync(0xffffffffu, kyq, src),
+               __shfl_sync(0xffffffffu, x_extra, src));
+        }
       }
     }
     if (INT && lane == 0) atomicAdd(cluster.map_shared_rank(&s_tgt, owner_y), tgt_acc);
     cluster.sync();
+    if (LIST && threadIdx.x == 0) s_cnt = 0;  // every warp has read this token's count
     // no CTA of the cluster reads sp any more: the next row can come in
     if (threadIdx.x == 0 && s_row_n) issue_row(s_row_n);
 
@@ -560,9 +595,9 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
   cluster.sync();
 }
 
-template <int NB, bool FULL, int DEG, bool INT>
+template <int NB, bool FULL, int DEG, bool INT, bool LIST>
 cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_count) {
-  auto fn = k_subset2<NB, FULL, DEG, INT>;
+  auto fn = k_subset2<NB, FULL, DEG, INT, LIST>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int cs = (int)A.cs;
@@ -590,22 +625,24 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
   return cudaGetLastError();
 }
 
-template <int NB, bool FULL, bool INT>
+template <int NB, bool FULL, bool INT, bool LIST>
 cudaError_t launch_deg(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
-  if (deg == 3) return launch_one<NB, FULL, 3, INT>(st, A, smem, sm);
-  if (deg == 4) return launch_one<NB, FULL, 4, INT>(st, A, smem, sm);
-  return launch_one<NB, FULL, 0, INT>(st, A, smem, sm);
+  if (deg == 3) return launch_one<NB, FULL, 3, INT, LIST>(st, A, smem, sm);
+  if (deg == 4) return launch_one<NB, FULL, 4, INT, LIST>(st, A, smem, sm);
+  return launch_one<NB, FULL, 0, INT, LIST>(st, A, smem, sm);
 }
 
-template <bool INT>
+template <bool INT, bool LIST>
 cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, int deg) {
   const int nb = (A.S + 127) / 128;
   const bool full = (A.S % 128) == 0;
   switch (nb) {
-    case 1: return full ? launch_deg<1, true, INT>(st, A, smem, sm, deg) : launch_deg<1, false, INT>(st, A, smem, sm, deg);
-    case 2: return full ? launch_deg<2, true, INT>(st, A, smem, sm, deg) : launch_deg<2, false, INT>(st, A, smem, sm, deg);
-    case 3: return launch_deg<3, false, INT>(st, A, smem, sm, deg);
-    case 4: return full ? launch_deg<4, true, INT>(st, A, smem, sm, deg) : launch_deg<4, false, INT>(st, A, smem, sm, deg);
+    case 1: return full ? launch_deg<1, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<1, false, INT, LIST>(st, A, smem, sm, deg);
+    case 2: return full ? launch_deg<2, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<2, false, INT, LIST>(st, A, smem, sm, deg);
+    case 3: if constexpr (!LIST) return launch_deg<3, false, INT, LIST>(st, A, smem, sm, deg);
+            return cudaErrorNotSupported;
+    case 4: if constexpr (!LIST) return full ? launch_deg<4, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<4, false, INT, LIST>(st, A, smem, sm, deg);
+            return cudaErrorNotSupported;
     default: return cudaErrorNotSupported;
   }
 }
@@ -677,10 +714,22 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   A.gop = gop;
   A.gf = gf;
   A.plane = p.T * p.V;
-  const size_t smem = (size_t)2 * A.seg * 4;
+  // the per-token draw list (16 bytes a draw) for up to 512 draws and
+  // S <= 256, when it fits beside the slices. At that K a warp has at most
+  // about 8 draws of a token, and a batch of 32 leaves the slowest warp
+  // several draws behind (on B200 at S = 256: K = 32 1.56 -> 1.09 ms,
+  // K = 128 1.86 -> 1.58, K = 512 2.84 -> 2.73 for 8192 tokens). At K = 1024
+  // the list's longer draw loop (6 % more instructions) costs more than the
+  // balance gains (4.11 -> 4.30 ms), and larger S keeps batches: those
+  // variants have no registers to spare.
+  const size_t slices = (size_t)2 * A.seg * 4, list_bytes = (size_t)p.K * 16;
+  const bool list = use_int && p.K <= 512 && p.S <= 256 &&
+                    slices + list_bytes + (size_t)kStaticSmem <= (size_t)max_smem_optin;
+  const size_t smem = slices + (list ? list_bytes : 0);
   const int deg = expm1_degree(p.sigma);
-  return use_int ? launch_nb<true>(st, A, smem, sm_count, deg)
-                 : launch_nb<false>(st, A, smem, sm_count, deg);
+  if (!use_int) return launch_nb<false, false>(st, A, smem, sm_count, deg);
+  return list ? launch_nb<true, true>(st, A, smem, sm_count, deg)
+              : launch_nb<true, false>(st, A, smem, sm_count, deg);
 }
 
 }  // namespace dust
