@@ -544,7 +544,7 @@ def run_dust(args):
         roof = _mlp_roofline(wl, stages["perturbed"], peaks)
         roof["peak_kind"] = peak_kind
     # the two dense contractions of the head, 2 T d V flops each (G_W: the
-    # stage includes the transposes that make both operands K-major)
+    # stage includes H's conversion to fp16, two small kernels)
     gemm_flops = 2.0 * wl.T * wl.d * wl.V
     extra = {}
     if wl.variant == "head":
