@@ -815,17 +815,23 @@ dust_status dust_attn_grad(dust_ctx* ctx, const dust_params* pp, const dust_attn
     DUST_TRY(ensure(ctx, ctx->attn_tcr, attn_tc_rows_bytes(T, a.seq_len, (int)H, a.head_dim)));
     DUST_TRY(ensure(ctx, ctx->attn_coef, attn_coef_bytes(T, a.seq_len, (int)H)));
   }
-  // the clean pass also writes the query-noise coefficient rows
+  // the clean pass also writes the query-noise coefficient rows, and the
+  // key-noise rows when they fit its shared memory (else a pass of their own)
   float2* qcoef = use_tc && a.which == DUST_ATTN_Q ? (float2*)ctx->attn_coef.p : nullptr;
-  DUST_CU(launch_attn_fwd(st, T, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse, gb, qcoef));
+  const bool kfused = use_tc && a.which == DUST_ATTN_K &&
+                      (size_t)ctx->max_smem_optin >= attn_fwd_smem(a.seq_len, a.head_dim, true);
+  float2* kcoef = kfused ? (float2*)ctx->attn_coef.p : nullptr;
+  DUST_CU(launch_attn_fwd(st, T, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse, gb, qcoef,
+                          kcoef));
   ctx->launches += 1;
   mark(ctx, "attn_fwd");
   DUST_CU(launch_attn_draws(st, p, a.which, a.seq_len, (int)H, a.head_dim, Q, Kc, Vc, E, O, lse,
                             gb, (float*)ctx->part.p, (float*)ctx->attn_w.p, r, use_tc,
-                            (uint8_t*)ctx->attn_tcr.p, (float2*)ctx->attn_coef.p, ctx->d_status));
-  // value: column sums + draws; tensor cores: (key) coefficients, row
-  // conversion, draws, head sum; CUDA cores: draws, head sum
-  ctx->launches += use_tc ? (a.which == DUST_ATTN_K ? 4 : 3) : 2;
+                            (uint8_t*)ctx->attn_tcr.p, (float2*)ctx->attn_coef.p, kfused,
+                            ctx->d_status));
+  // value: column sums + draws; tensor cores: (key, unfused) coefficients,
+  // row conversion, draws, head sum; CUDA cores: draws, head sum
+  ctx->launches += use_tc ? (a.which == DUST_ATTN_K && !kfused ? 4 : 3) : 2;
   mark(ctx, "draws");
   dust_params pg = p;
   pg.d = Dw;  // the noise width

@@ -344,18 +344,19 @@ cudaError_t launch_gelu_f32(cudaStream_t st, const float* u, int64_t n, float* a
 // or key (1) of every token per head -> part ((T H) x K), summed over heads
 // into r (T x K); for the value (2), w = A^T E per head -> W (T x D), then
 // the rewards straight into r.
-size_t attn_fwd_smem(int L, int head_dim);
+// kcoef: the clean pass also writes the key-noise coefficient rows
+size_t attn_fwd_smem(int L, int head_dim, bool kcoef = false);
 size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
 size_t attn_tc_smem(int L, int head_dim);  // the tensor-core query/key draws (d_h 64, 128)
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
                             const float* Q, const float* Kc, const float* Vc, const float* E,
-                            float* O, float* lse, float* gbar, float2* qcoef);
+                            float* O, float* lse, float* gbar, float2* qcoef, float2* kcoef);
 cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, int L, int H,
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
                               const float* gbar, float* part, float* W, float* r, bool use_tc,
-                              uint8_t* tc_rows, float2* coef, uint32_t* status);
+                              uint8_t* tc_rows, float2* coef, bool coef_done, uint32_t* status);
 // bytes of the converted row tiles and of the coefficient rows the
 // tensor-core draws read
 size_t attn_tc_rows_bytes(int64_t T, int L, int H, int head_dim);

@@ -44,7 +44,7 @@
 
 namespace dust {
 
-size_t attn_fwd_smem(int L, int head_dim);
+size_t attn_fwd_smem(int L, int head_dim, bool kcoef);
 size_t attn_colsum_smem(int head_dim);
 size_t attn_draws_smem(int L, int head_dim);
 size_t attn_tc_smem(int L, int head_dim);
@@ -111,6 +111,10 @@ struct FwdArgs {
   int32_t L, H;
   float scale;
   float2* qcoef;  // optional: (a_s,tau, a_s,tau <v_tau, e_s>) rows for query noise
+  // optional: the key-noise rows, row (s, h) holding at column t of the
+  // sequence (a_t,s, <v_s, e_t> - gbar_t) for t >= s (zero for the CTA's rows
+  // t < s; entries no CTA writes are cleared by the key draws)
+  float2* kcoef = nullptr;
 };
 
 // One CTA per (sequence, head, block of kFwdWarps rows), one warp per query
@@ -119,9 +123,12 @@ struct FwdArgs {
 // are staged through a shared-memory tile (row stride d_h + 4 floats: the
 // lanes' 16-byte reads of different rows fall in distinct banks). Shared
 // memory: per warp the row's probabilities (L rounded up to 4) and q_t
-// (d_h), and the kTile x (d_h + 4) tile.
-template <int DH>
-__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_constant__ FwdArgs A) {
+// (d_h), and the kTile x (d_h + 4) tile; with key-noise rows also per warp
+// <v_s, e_t> for the row's keys (L rounded up to 4) and gbar_t. The key rows
+// are written at the end, when gbar_t is known: for each key s of the block
+// the CTA's kFwdWarps rows are consecutive columns of row (s, h), 64 bytes.
+template <int DH, bool KC>
+__device__ __forceinline__ void attn_fwd_body(const FwdArgs& A) {
   extern __shared__ __align__(16) float fsm[];
   constexpr int kStride = DH + 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,6 +147,8 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_consta
   float* qs = pr + Lp;
   float* es = qs + DH;
   float* tile = fsm + (size_t)kFwdWarps * (Lp + 2 * DH);
+  // key rows: <v_s, e_t> per warp (L rounded up to 4), then gbar_t per warp
+  float* ev = tile + kTile * kStride + warp * Lp;
   const int64_t t = s0 + pos;
   if (row_ok)
     for (int c = lane; c < DH; c += 32) {
@@ -188,6 +197,8 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_consta
 #pragma unroll
       for (int u = 0; u < DH / 32; ++u) o[u] = fmaf(a, tile[j * kStride + lane + 32 * u], o[u]);
     }
+    if (KC)
+      for (int j = lane; j < lim; j += 32) ev[j0 + j] = dot_row<DH>(es, tile + j * kStride);
     if (A.qcoef && row_ok) {
       // the query-noise coefficient row: (a, a <v, e_s>) up to the tile
       // boundary, zero past the causal limit (<o_s, e_s> is taken off later)
@@ -203,19 +214,50 @@ __global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_consta
       }
     }
   }
-  if (!row_ok) return;  // after the last block barrier
   float gb = 0.f;
+  if (row_ok) {
 #pragma unroll
-  for (int u = 0; u < DH / 32; ++u) {
-    const int64_t c = t * D + h * DH + lane + 32 * u;
-    A.O[c] = o[u];
-    gb = fmaf(o[u], A.E[c], gb);
+    for (int u = 0; u < DH / 32; ++u) {
+      const int64_t c = t * D + h * DH + lane + 32 * u;
+      A.O[c] = o[u];
+      gb = fmaf(o[u], A.E[c], gb);
+    }
+    gb = warp_sum_f(gb);
+    if (lane == 0) {
+      A.lse[t * A.H + h] = lse;
+      A.gbar[t * A.H + h] = gb;
+    }
   }
-  gb = warp_sum_f(gb);
-  if (lane == 0) {
-    A.lse[t * A.H + h] = lse;
-    A.gbar[t * A.H + h] = gb;
+  if (!KC) return;
+  const float* evs = tile + kTile * kStride;
+  float* gbs = const_cast<float*>(evs) + kFwdWarps * Lp;
+  if (lane == 0) gbs[warp] = gb;
+  __syncthreads();
+  // key rows: entry e = (key s, warp w), w fastest, so every 8 threads write
+  // columns rb kFwdWarps .. + 7 of row (s, h)
+  const int Lt = (A.L + kTcRows - 1) / kTcRows * kTcRows;
+  float2* kbase = A.kcoef + (s0 * A.H + h) * (int64_t)Lt + rb * kFwdWarps;
+  for (int e = threadIdx.x; e < nmax * kFwdWarps; e += kFwdWarps * 32) {
+    const int w = e % kFwdWarps, sk = e / kFwdWarps;
+    const int c = rb * kFwdWarps + w;  // the row (query position) of warp w
+    float2 v = make_float2(0.f, 0.f);
+    if (c < A.L && sk <= c)
+      v = make_float2(fsm[w * (Lp + 2 * DH) + sk], evs[w * Lp + sk] - gbs[w]);
+    if (c < Lt) kbase[(int64_t)sk * A.H * Lt + w] = v;
   }
+}
+
+template <int DH>
+__global__ __launch_bounds__(kFwdWarps * 32) void k_attn_fwd(const __grid_constant__ FwdArgs A) {
+  attn_fwd_body<DH, false>(A);
+}
+
+// The clean pass that also writes the key-noise rows. Its shared memory
+// (the extra <v_s, e_t> rows) allows two CTAs per SM, and so do its
+// registers: with that bound ptxas keeps every value in registers.
+template <int DH>
+__global__ __launch_bounds__(kFwdWarps * 32, 2) void k_attn_fwd_kc(const __grid_constant__ FwdArgs A) {
+  attn_fwd_body<DH, true>(A);
 }
 
 struct DrawArgs {
@@ -762,6 +804,15 @@ __global__ __launch_bounds__(kDrawThreads, DH == 64 ? 2 : 1) void k_attn_draws_t
     // the coefficient row (phase 0 of cfull: at once in later rounds); a
     // failure sets the abort flag, which ends the tile loop below
     (void)__all_sync(0xffffffffu, tc_wait(ptx::smem_u32(&cfull), 0u, abort, A.status));
+    if (WHICH == 1 && i0 == 0) {
+      // key rows: the entries of tile k0 before s and those past the
+      // sequence end carry no coefficient (the clean pass that writes the
+      // rows leaves some of them unwritten); clear them once
+      const int before = (int)(s - r0);
+      for (int q = tid; q < ntiles * kTcRows; q += kDrawThreads)
+        if (q < before || q >= n) cab[q] = make_float2(0.f, 0.f);
+      __syncthreads();
+    }
     float acc0 = 0.f, acc1 = 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
@@ -940,13 +991,14 @@ __global__ void k_attn_combine(const float* __restrict__ part, int64_t T, int32_
 
 template <int DH>
 cudaError_t fwd_dh(cudaStream_t st, const FwdArgs& A) {
-  const size_t smem = attn_fwd_smem(A.L, DH);
-  cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const bool kc = A.kcoef != nullptr;
+  const size_t smem = attn_fwd_smem(A.L, DH, kc);
+  auto fn = kc ? k_attn_fwd_kc<DH> : k_attn_fwd<DH>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t nrb = (A.L + kFwdWarps - 1) / kFwdWarps;
   const int64_t blocks = (A.T / A.L) * A.H * nrb;
-  k_attn_fwd<DH><<<(unsigned)blocks, kFwdWarps * 32, smem, st>>>(A);
+  fn<<<(unsigned)blocks, kFwdWarps * 32, smem, st>>>(A);
   return cudaGetLastError();
 }
 
@@ -998,8 +1050,10 @@ cudaError_t colsum_dh(cudaStream_t st, const FwdArgs& A, float* W) {
 
 }  // namespace
 
-size_t attn_fwd_smem(int L, int head_dim) {
-  return ((size_t)kFwdWarps * (((L + 3) & ~3) + 2 * head_dim) + (size_t)kTile * (head_dim + 4)) * 4;
+size_t attn_fwd_smem(int L, int head_dim, bool kcoef) {
+  const size_t Lp = (size_t)((L + 3) & ~3);
+  return ((size_t)kFwdWarps * (Lp + 2 * head_dim) + (size_t)kTile * (head_dim + 4) +
+          (kcoef ? (size_t)kFwdWarps * (Lp + 1) : 0)) * 4;
 }
 size_t attn_coef_smem(int head_dim) {
   return ((size_t)2 * kTile * (head_dim + 4) + 2 * kTile + (size_t)kFwdWarps * 2 * head_dim) * 4;
@@ -1018,8 +1072,8 @@ size_t attn_draws_smem(int L, int head_dim) {
 
 cudaError_t launch_attn_fwd(cudaStream_t st, int64_t T, int L, int H, int head_dim,
                             const float* Q, const float* Kc, const float* Vc, const float* E,
-                            float* O, float* lse, float* gbar, float2* qcoef) {
-  FwdArgs A{Q, Kc, Vc, E, O, lse, gbar, T, L, H, 1.0f / sqrtf((float)head_dim), qcoef};
+                            float* O, float* lse, float* gbar, float2* qcoef, float2* kcoef) {
+  FwdArgs A{Q, Kc, Vc, E, O, lse, gbar, T, L, H, 1.0f / sqrtf((float)head_dim), qcoef, kcoef};
   if (head_dim == 32) return fwd_dh<32>(st, A);
   if (head_dim == 64) return fwd_dh<64>(st, A);
   return fwd_dh<128>(st, A);
@@ -1029,7 +1083,7 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
                               int head_dim, const float* Q, const float* Kc, const float* Vc,
                               const float* E, const float* O, const float* lse,
                               const float* gbar, float* part, float* W, float* r, bool use_tc,
-                              uint8_t* tc_rows, float2* coef, uint32_t* status) {
+                              uint8_t* tc_rows, float2* coef, bool coef_done, uint32_t* status) {
   if (p.T * H <= 0) return cudaSuccess;
   const float c = 1.0f / sqrtf((float)head_dim);
   const uint32_t ctr3 = ctr3_of(kTagAttnQ + which, p.stream_id);
@@ -1066,9 +1120,10 @@ cudaError_t launch_attn_draws(cudaStream_t st, const dust_params& p, int which, 
                 H, c, nullptr};
       const size_t csm = attn_coef_smem(head_dim);
       const unsigned cblocks = (unsigned)((p.T / L) * H * ((L + kFwdWarps - 1) / kFwdWarps));
-      // query noise: the clean pass wrote the rows (launch_attn_fwd's qcoef)
+      // query noise, and key noise where the rows fit its shared memory: the
+      // clean pass wrote the rows (launch_attn_fwd's qcoef, kcoef)
       cudaError_t ce = cudaSuccess;
-      if (which == 1)
+      if (which == 1 && !coef_done)
         ce = head_dim == 64 ? kcoef_dh<64>(st, F, coef, csm, cblocks)
                             : kcoef_dh<128>(st, F, coef, csm, cblocks);
       if (ce != cudaSuccess) return ce;
