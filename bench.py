@@ -228,13 +228,19 @@ def _cpu_model() -> str:
 
 # ----------------------------------------------------------------------------- helpers
 def _dist_init():
+    """One rank per GPU: the rank's device is made current before the NCCL
+    group is created, and the group is bound to it (its communicator is set
+    up at once, so a failure shows here rather than in the first step)."""
+    import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
     return world, rank, local
 
 
