@@ -92,3 +92,30 @@ def test_attention_shards_by_whole_sequences(ctx, which):
 
     spans = [(0, 80), (80, 40)]
     _compare(run(0, wl.T), [run(t0, n) for t0, n in spans], spans, ("rewards", "g"))
+
+
+@pytest.mark.parametrize("S,dtype", [(50, "bf16"), (0, "bf16"), (50, "f32")])
+def test_head_draw_shards(ctx, S, dtype):
+    """Draw sharding: two calls over every token with disjoint draw ranges
+    (draw_offset = the range's first draw) give the whole run's rewards as
+    their columns, and its g and G_W once each is weighted by its share of
+    the draws (parallel.combine_draw_shards, here without a process group)."""
+    from zeroth_order_transformer_dust_b200.parallel import combine_draw_shards, draw_shard
+    wl = synth.Workload("shard_draws", "head", T=24, d=64, V=1000, K=45, S=S, sigma=1e-2,
+                        seed=19, dtype=dtype, targets="zipf")
+    inp = synth.make_head_inputs(wl)
+    H, W, y = to_dev(inp["H"], dtype), to_dev(inp["W"], dtype), to_dev(inp["targets"], "i32")
+    kw = dict(sigma=wl.sigma, S=S, seed=wl.seed, want_rewards=True, want_g=True)
+    whole = ctx.head_grad(H, W, y, K=wl.K, **kw)
+    G = torch.zeros_like(whole["G"])
+    g = torch.zeros_like(whole["g"])
+    for rank in range(2):
+        i0, k = draw_shard(wl.K, 2, rank)
+        part = ctx.head_grad(H, W, y, K=k, draw_offset=i0, **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(part["rewards"], whole["rewards"][:, i0:i0 + k])
+        G += combine_draw_shards(part["G"], k, wl.K)
+        g += combine_draw_shards(part["g"], k, wl.K)
+    torch.cuda.synchronize()
+    assert rel_fro(np64(g), np64(whole["g"])) < 1e-5
+    assert rel_fro(np64(G), np64(whole["G"])) < (2e-3 if dtype == "bf16" else 1e-5)

@@ -17,7 +17,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from zeroth_order_transformer_dust_b200.parallel import allreduce_weight_grad, token_shard
+from zeroth_order_transformer_dust_b200.parallel import (allreduce_weight_grad, combine_draw_shards,
+                                                         draw_shard, token_shard)
 
 
 def _free_port():
@@ -217,3 +218,64 @@ def test_bench_times_the_slowest_rank():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert res == {0: 14.75, 1: 14.75}
+
+
+def _draw_worker(rank, world, port, S, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import synth
+        wl = synth.Workload("gloo", "head", T=6, d=5, V=30, K=7, S=S, sigma=0.05, seed=4,
+                            dtype="f32", targets="zipf")
+        inp = synth.make_head_inputs(wl)
+        i0, k = draw_shard(wl.K, world, rank)
+        prm = oracle.Params(T=wl.T, d=wl.d, V=wl.V, K=k, S=wl.S, sigma=wl.sigma, seed=wl.seed,
+                            draw_offset=i0)
+        out = oracle.head_grad(inp["H"], inp["W"], inp["targets"], prm)
+        G = torch.from_numpy(out["G"])
+        g = torch.from_numpy(out["g"])
+        combine_draw_shards(G, k, wl.K)
+        combine_draw_shards(g, k, wl.K)
+        q.put((rank, i0, k, G.numpy(), g.numpy(), out["rewards"]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("S", [0, 4])
+def test_draw_sharded_estimate_equals_single_run(S):
+    """Ranks with disjoint draw ranges (7 draws as 4 + 3), each over every
+    token, combine to the single run's G_W and g; their rewards are the
+    single run's columns."""
+    import oracle
+    import synth
+    world = 2
+    assert [draw_shard(7, world, r) for r in range(world)] == [(0, 4), (4, 3)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_draw_worker, args=(r, world, port, S, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=300) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    wl = synth.Workload("gloo", "head", T=6, d=5, V=30, K=7, S=S, sigma=0.05, seed=4,
+                        dtype="f32", targets="zipf")
+    inp = synth.make_head_inputs(wl)
+    prm = oracle.Params(T=wl.T, d=wl.d, V=wl.V, K=wl.K, S=wl.S, sigma=wl.sigma, seed=wl.seed)
+    ref = oracle.head_grad(inp["H"], inp["W"], inp["targets"], prm)
+    for rank, i0, k, G, g, rewards in res:
+        np.testing.assert_allclose(G, ref["G"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(g, ref["g"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_array_equal(rewards, ref["rewards"][:, i0:i0 + k])
+
+
+def test_combine_draw_shards_checks_counts():
+    with pytest.raises(ValueError):
+        combine_draw_shards(torch.zeros(2), 5, 4)
+    with pytest.raises(ValueError):
+        combine_draw_shards(torch.zeros(2), 1, 0)
+    x = torch.ones(3)
+    assert torch.equal(combine_draw_shards(x, 2, 4), torch.full((3,), 0.5))  # one process: no reduce

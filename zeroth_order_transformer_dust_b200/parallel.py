@@ -7,6 +7,12 @@ across ranks by tokens: rank r runs the estimator on its contiguous token
 range with token_offset = start, which reproduces exactly the noise a single
 run over the whole batch would draw, and one sum all-reduce of the per-rank
 G_W (NCCL over NVLink/NVSwitch on GPUs) gives the estimate of the full batch.
+
+The draws split the same way: rank r can run every token with its own
+contiguous range of the K draws (draw_offset = its first draw), again the
+noise of a single run. Its estimate carries 1/K_r for its K_r draws, so it is
+weighted by K_r / K before the same sum all-reduce (draw_shard,
+combine_draw_shards).
 """
 from __future__ import annotations
 
@@ -39,6 +45,24 @@ def sequence_shard(T_total: int, seq_len: int, world: int, rank: int) -> Tuple[i
         raise ValueError("T_total must be a positive multiple of seq_len")
     first, count = token_shard(T_total // seq_len, world, rank)
     return first * seq_len, count * seq_len
+
+
+def draw_shard(K_total: int, world: int, rank: int) -> Tuple[int, int]:
+    """(first draw, draw count) of `rank`'s contiguous share of K_total draws,
+    distributed as token_shard distributes tokens."""
+    return token_shard(K_total, world, rank)
+
+
+def combine_draw_shards(x: torch.Tensor, K_local: int, K_total: int,
+                        group: Optional[dist.ProcessGroup] = None) -> torch.Tensor:
+    """In place: the estimate over all K_total draws from this rank's estimate
+    over its K_local draws, x <- sum over ranks of (K_local / K_total) x. The
+    estimator scales its sum over draws by 1/K, so the weighted sum equals a
+    single run over all draws (G_W, or g_t of the same tokens)."""
+    if K_total < 1 or not 0 <= K_local <= K_total:
+        raise ValueError("bad draw counts")
+    x.mul_(K_local / K_total)
+    return allreduce_weight_grad(x, group)
 
 
 def allreduce_weight_grad(G: torch.Tensor, group: Optional[dist.ProcessGroup] = None) -> torch.Tensor:
