@@ -309,61 +309,88 @@ __global__ void k_reward_combine_rows(const float* __restrict__ part, int nparts
   r[row0 + m] = dzy[m] - log1pf(s);
 }
 
-// g_t[c] = scale * sum_i r[t*K + i] eps(t, i, c): one warp per 128 channels,
-// the first two Philox rounds hoisted, the table angle step (unit noise).
+// g_t[c] = scale * sum_i r[t*K + i] eps(t, i, c). A warp takes up to
+// kNoiseGBlocks 128-channel blocks of one token (a unit), so the first two
+// Philox rounds of a draw are formed once for all of them (those of a block
+// once per unit); the table angle step (unit noise); the sums over draws in
+// packed fp32x2 arithmetic (each lane rounds as fma(r, eps, acc) in draw
+// order). A CTA holds 8 units, each warp staging its token's rewards.
+constexpr int kNoiseGBlocks = 4;
+constexpr int kNoiseGChunk = 256;  // rewards staged per warp at a time
+
 template <typename TO>
 __global__ __launch_bounds__(256) void k_noise_g(RoundKeys keys, uint32_t t_off, uint32_t i_off,
-                                                 uint32_t ctr3, float scale, int64_t width,
-                                                 int32_t K, const float* __restrict__ r,
+                                                 uint32_t ctr3, float scale, int64_t T,
+                                                 int64_t width, int32_t K,
+                                                 const float* __restrict__ r,
                                                  float* __restrict__ g_out, TO* __restrict__ gop,
                                                  int64_t plane) {
-  __shared__ float rs[1024];
+  __shared__ float rs[8][kNoiseGChunk];
   __shared__ float2 tab[kSinCosTable];
   fill_sincos_table(tab, 1.0f);
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t t = blockIdx.x;
-  const int64_t blk = (int64_t)blockIdx.y * (blockDim.x >> 5) + warp;
+  const int64_t nblk = (width + 127) / 128;
+  const int64_t ngroups = (nblk + kNoiseGBlocks - 1) / kNoiseGBlocks;
+  const int64_t unit = (int64_t)blockIdx.x * 8 + warp;
+  if (unit >= T * ngroups) return;  // no block-wide barrier follows
+  const int64_t t = unit / ngroups;
+  const int64_t blk0 = (unit % ngroups) * kNoiseGBlocks;
+  const int nvalid = (int)min((int64_t)kNoiseGBlocks, nblk - blk0);
   const uint32_t t_abs = t_off + (uint32_t)t;
-  const BlockConst bc = block_const(keys, slot_ctr0((uint32_t)blk, (uint32_t)lane), ctr3);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int i0 = 0; i0 < K; i0 += 1024) {
-    const int n = min(1024, K - i0);
-    __syncthreads();
-    for (int q = threadIdx.x; q < n; q += blockDim.x) rs[q] = r[t * K + i0 + q];
-    __syncthreads();
-    if (blk * 128 < width) {
-      for (int ii = 0; ii < n; ++ii) {
-        const G4 g = gauss4_tab(
-            philox_from2(bc, draw_const(keys, t_abs, i_off + (uint32_t)(i0 + ii)), keys), tab);
-        const float ri = rs[ii];
+  BlockConst bc[kNoiseGBlocks];
+  float2 a02[kNoiseGBlocks], a13[kNoiseGBlocks];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] = fmaf(ri, g.v[j], acc[j]);
+  for (int b = 0; b < kNoiseGBlocks; ++b) {
+    bc[b] = block_const(keys, slot_ctr0((uint32_t)(blk0 + b), (uint32_t)lane), ctr3);
+    a02[b] = make_float2(0.f, 0.f);
+    a13[b] = make_float2(0.f, 0.f);
+  }
+  for (int i0 = 0; i0 < K; i0 += kNoiseGChunk) {
+    const int n = min(kNoiseGChunk, K - i0);
+    __syncwarp();
+    for (int q = lane; q < n; q += 32) rs[warp][q] = r[t * K + i0 + q];
+    __syncwarp();
+    for (int ii = 0; ii < n; ++ii) {
+      const DrawConst dc = draw_const(keys, t_abs, i_off + (uint32_t)(i0 + ii));
+      const float ri = rs[warp][ii];
+      const float2 r2 = make_float2(ri, ri);
+#pragma unroll
+      for (int b = 0; b < kNoiseGBlocks; ++b) {
+        if (b < nvalid) {
+          const G4 g = gauss4_tab(philox_from2(bc[b], dc, keys), tab);
+          a02[b] = __ffma2_rn(r2, make_float2(g.v[0], g.v[2]), a02[b]);
+          a13[b] = __ffma2_rn(r2, make_float2(g.v[1], g.v[3]), a13[b]);
+        }
       }
     }
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int64_t ch = blk * 128 + lane + 32 * j;
-    if (ch < width) {
-      const float v = acc[j] * scale;
-      if (g_out) g_out[t * width + ch] = v;
-      store_g_operand(gop, plane, t * width + ch, v);
+  for (int b = 0; b < kNoiseGBlocks; ++b)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t ch = (blk0 + b) * 128 + lane + 32 * j;
+      if (b < nvalid && ch < width) {
+        const float2 a = (j & 1) ? a13[b] : a02[b];
+        const float v = ((j & 2) ? a.y : a.x) * scale;
+        if (g_out) g_out[t * width + ch] = v;
+        store_g_operand(gop, plane, t * width + ch, v);
+      }
     }
-  }
 }
 
 }  // namespace
 
-// k_noise_g geometry: one warp per 128-channel block, at most 8 warps per CTA
-// and no idle warps when the width has fewer than 8 blocks.
+// k_noise_g geometry: T x (groups of kNoiseGBlocks 128-channel blocks) units,
+// 8 per CTA of 256 threads.
 struct NoiseGGeom {
   dim3 grid;
   unsigned threads;
 };
 static NoiseGGeom noise_g_geom(int64_t T, int64_t width) {
   const int64_t nblk = (width + 127) / 128;
-  const int64_t warps = nblk < 8 ? nblk : 8;
-  return {dim3((unsigned)T, (unsigned)((nblk + warps - 1) / warps)), (unsigned)(32 * warps)};
+  const int64_t units = T * ((nblk + kNoiseGBlocks - 1) / kNoiseGBlocks);
+  return {dim3((unsigned)((units + 7) / 8)), 256u};
 }
 
 cudaError_t launch_mlp_delta_a(cudaStream_t st, const dust_params& p, const float* u, int64_t t0,
@@ -411,7 +438,7 @@ cudaError_t launch_noise_g_planes(cudaStream_t st, const dust_params& p, const f
   const NoiseGGeom gg = noise_g_geom(p.T, p.d);
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
   k_noise_g<__nv_bfloat16><<<gg.grid, gg.threads, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
-      (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.d, p.K, r, g_out, gop,
+      (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.T, p.d, p.K, r, g_out, gop,
       p.T * p.d);
   return cudaGetLastError();
 }
@@ -421,7 +448,7 @@ cudaError_t launch_noise_g_f32(cudaStream_t st, const dust_params& p, const floa
   const NoiseGGeom gg = noise_g_geom(p.T, p.d);
   const float scale = p.sigma > 0.0f ? -1.0f / ((float)p.K * p.sigma) : 0.0f;
   k_noise_g<float><<<gg.grid, gg.threads, 0, st>>>(round_keys(p.seed), (uint32_t)p.token_offset,
-      (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.d, p.K, r, g_out, gop, 0);
+      (uint32_t)p.draw_offset, ctr3_of(tag, p.stream_id), scale, p.T, p.d, p.K, r, g_out, gop, 0);
   return cudaGetLastError();
 }
 
@@ -464,10 +491,10 @@ cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, 
   const int64_t plane = p.T * width;
   if (p.dtype == DUST_BF16 && !down)
     k_noise_g<__nv_bfloat16><<<gg.grid, gg.threads, 0, st>>>(keys, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, width, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
+        (uint32_t)p.draw_offset, c3, scale, p.T, width, p.K, r, g_out, (__nv_bfloat16*)gop, plane);
   else
     k_noise_g<float><<<gg.grid, gg.threads, 0, st>>>(keys, (uint32_t)p.token_offset,
-        (uint32_t)p.draw_offset, c3, scale, width, p.K, r, g_out, (float*)gop, plane);
+        (uint32_t)p.draw_offset, c3, scale, p.T, width, p.K, r, g_out, (float*)gop, plane);
   return cudaGetLastError();
 }
 
