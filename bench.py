@@ -81,7 +81,8 @@ def _peaks():
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "pci.bus_id")
 
     def __init__(self, out_path=None):
         self.proc = None
@@ -111,18 +112,57 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
+                if len(parts) >= 10:
                     rows.append(parts)
         if not rows:
             return None
-        idx = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0]
-        mine = [r for r in rows if r[0] == idx] or [r for r in rows if r[0] == rows[0][0]]
+        mine = [r for r in rows if _same_bus(r[9])] or [r for r in rows if r[0] == rows[0][0]]
         sm = [float(r[1]) for r in mine if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in mine for k in range(4) if r[5 + k].lower() == "active"})
+        reasons = sorted({CLOCK_REASONS[k] for r in mine for k in range(4)
+                          if r[5 + k].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(mine)}
+
+
+def _same_bus(bus_id: str) -> bool:
+    """Whether nvidia-smi's PCI bus id ("00000000:18:00.0") is this rank's GPU."""
+    try:
+        import torch
+        pr = torch.cuda.get_device_properties(torch.cuda.current_device())
+        dom, bus, rest = bus_id.split(":")
+        dev = rest.split(".")[0]
+        return (int(dom, 16), int(bus, 16), int(dev, 16)) == (
+            pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+    except (ValueError, AttributeError, RuntimeError):
+        return False
+
+
+CLOCK_REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+def _merge_clocks(clk, world: int, device: str = "cuda"):
+    """The clock record of the whole job: the lowest median SM clock and the
+    union of the throttle reasons over all ranks (every rank calls this; the
+    tensors live on the process group's device)."""
+    if world == 1:
+        return clk
+    import torch
+    import torch.distributed as dist
+    sm = clk["sm_mhz"] if clk and clk["sm_mhz"] is not None else float("inf")
+    bits = sum(1 << k for k, n in enumerate(CLOCK_REASONS) if clk and n in clk["reasons"])
+    hi = torch.tensor([clk["sm_max_mhz"] or 0.0 if clk else 0.0, float(bits),
+                       float(clk["samples"] if clk else 0)], dtype=torch.float64, device=device)
+    lo = torch.tensor([sm], dtype=torch.float64, device=device)
+    dist.all_reduce(hi, op=dist.ReduceOp.MAX)
+    dist.all_reduce(lo, op=dist.ReduceOp.MIN)
+    if float(hi[2]) == 0.0:
+        return None
+    b = int(hi[1].item())
+    return {"sm_mhz": None if lo.item() == float("inf") else float(lo.item()),
+            "sm_max_mhz": float(hi[0]) or None,
+            "reasons": [n for k, n in enumerate(CLOCK_REASONS) if b >> k & 1],
+            "samples": int(hi[2]), "ranks": world}
 
 
 # ----------------------------------------------------------------------------- oracle baseline
@@ -494,7 +534,7 @@ def run_dust(args):
         ev[k][1].record(stream)
         stage_ms.append(ctx.stage_times())
     _barrier(world)
-    clk = clocks.stop()
+    clk = _merge_clocks(clocks.stop(), world)
     launches = ctx.kernel_launches - launches0
     ctx.check()
     step_ms = [a.elapsed_time(b) for a, b in ev]

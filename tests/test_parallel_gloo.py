@@ -279,3 +279,35 @@ def test_combine_draw_shards_checks_counts():
         combine_draw_shards(torch.zeros(2), 1, 0)
     x = torch.ones(3)
     assert torch.equal(combine_draw_shards(x, 2, 4), torch.full((3,), 0.5))  # one process: no reduce
+
+
+def _clock_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        mine = [{"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 5},
+                {"sm_mhz": 1402.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 4}][rank]
+        q.put((rank, bench._merge_clocks(mine, world, device="cpu")))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_clock_record_covers_every_rank():
+    """The JSON line's clock record at N > 1: the lowest median SM clock and
+    the union of the throttle reasons over the ranks, the same on every rank."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_clock_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank in range(world):
+        assert res[rank] == {"sm_mhz": 1402.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                             "samples": 5, "ranks": 2}
