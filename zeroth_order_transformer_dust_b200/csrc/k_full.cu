@@ -6,8 +6,8 @@
 // The reward needs the whole row before any g entry can be formed, so the
 // noise is generated twice (stage 1 and stage 3); it never reaches memory.
 //
-// Both noise passes are persistent over (token, 4096-entry slab) units: a warp
-// owns four 128-slot blocks of the slab, evaluates Philox rounds 0-1 of its
+// Both noise passes are persistent over (token, 3072-entry slab) units: a warp
+// owns three 128-slot blocks of the slab, evaluates Philox rounds 0-1 of its
 // blocks once per unit and those of each draw once per draw, and turns words
 // into sigma-scaled Gaussians with the table-driven Box-Muller step (the
 // table of roots of unity is built once per CTA). Stage 1 also records the
@@ -19,7 +19,10 @@ namespace dust {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kBlocksPerWarp = 4;                     // 128-slot blocks per warp
+// 128-slot blocks per warp: three keeps both passes within 64 registers, so
+// they run 32 warps per SM (four blocks, 72 registers in the reward pass:
+// 24 warps; 2 % slower on full_bf16)
+constexpr int kBlocksPerWarp = 3;
 constexpr int kSlab = kWarps * kBlocksPerWarp * 128;  // vocabulary entries per unit
 constexpr int kDrawChunk = 64;
 // The Box-Muller step in packed fp32x2 form (PACKED) or scalar and paired up
