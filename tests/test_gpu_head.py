@@ -113,6 +113,22 @@ def test_edge_shapes(ctx, kw):
     _compare(got, ref, TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
 
 
+# More full-vocabulary shapes: K = 2, 3, 4 and odd K, single tokens with many
+# draws, exact and ragged 128-slot blocks, the largest vocabularies here, sigma
+# that needs the exact expm1, fp32 inputs, and more tokens than CTAs.
+@pytest.mark.parametrize("kw", [
+    dict(K=2), dict(K=3), dict(K=4, T=3), dict(K=33, V=3000), dict(T=1, K=64, V=50304, d=16),
+    dict(V=128, K=7), dict(V=129, K=7), dict(V=2, K=5), dict(V=122000, K=6, T=3, d=16),
+    dict(V=124000, K=6, T=2, d=16), dict(sigma=0.2, K=35), dict(dtype="f32", K=10, V=2049),
+    dict(T=97, K=3, V=50304, d=16),
+])
+def test_full_vocab_more_shapes(ctx, kw):
+    wl = _small(**kw)
+    H, W, y = _inputs(wl)
+    _compare(_gpu(ctx, H, W, y, wl), _oracle(H, W, y, wl),
+             TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
+
+
 @pytest.mark.parametrize("kw", [dict(), dict(S=129, K=33), dict(V=4099, S=640, K=40),
                                 dict(T=200, K=5, V=1000), dict(T=300, K=3, V=3001, S=50)])
 def test_single_cta_tensor_core_path(cuda_ok, monkeypatch, kw):
