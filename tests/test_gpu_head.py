@@ -115,12 +115,17 @@ def test_edge_shapes(ctx, kw):
 
 # More full-vocabulary shapes: K = 2, 3, 4 and odd K, single tokens with many
 # draws, exact and ragged 128-slot blocks, the largest vocabularies here, sigma
-# that needs the exact expm1, fp32 inputs, and more tokens than CTAs.
+# that needs the exact expm1 and sigma that does not, fp32 inputs, and more
+# tokens than CTAs.
 @pytest.mark.parametrize("kw", [
     dict(K=2), dict(K=3), dict(K=4, T=3), dict(K=33, V=3000), dict(T=1, K=64, V=50304, d=16),
     dict(V=128, K=7), dict(V=129, K=7), dict(V=2, K=5), dict(V=122000, K=6, T=3, d=16),
     dict(V=124000, K=6, T=2, d=16), dict(sigma=0.2, K=35), dict(dtype="f32", K=10, V=2049),
     dict(T=97, K=3, V=50304, d=16),
+    # sigma small enough for the series degrees (the reward pass's hardware
+    # exponential): degree 4 at 1e-2, degree 3 at 5e-3
+    dict(sigma=0.01, K=20, V=3000), dict(sigma=0.005, K=20, V=4099, T=9),
+    dict(sigma=0.01, dtype="f32", K=16, V=1024), dict(sigma=0.0104, K=64, V=50304, T=2, d=16),
 ])
 def test_full_vocab_more_shapes(ctx, kw):
     wl = _small(**kw)
