@@ -93,8 +93,8 @@ CONFIGS = {
     "subset_v128k_bf16": Workload("subset_v128k_bf16", "head", T=8192, d=1024, V=128256,
                                   K=1024, S=512, sigma=1e-2, seed=6, dtype="bf16",
                                   targets="zipf"),
-    # Subset draws of S = 1024 entries, beyond the shared-memory kernel's 512:
-    # the L2-fed kernel that keeps only the g row in shared memory.
+    # Subset draws of S = 1024 entries: eight 128-slot blocks a draw in the
+    # shared-memory kernel (16 warps per SM).
     "subset_s1024_bf16": Workload("subset_s1024_bf16", "head", T=8192, d=1024, V=50304,
                                   K=1024, S=1024, sigma=1e-2, seed=7, dtype="bf16",
                                   targets="zipf"),

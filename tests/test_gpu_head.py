@@ -104,6 +104,14 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     # the per-token draw list (K <= 512, S <= 256) with clusters of two CTAs
     # and several tokens per cluster
     dict(V=50304, S=256, K=512, T=160, d=16),
+    # five to eight 128-slot blocks a draw (S up to 1024): exact and ragged S,
+    # windows crossing slices of a two-CTA cluster, the library expm1 (large
+    # sigma) and fp32 accumulators (K > 65536) at ragged S
+    dict(V=50304, S=1024, K=64, T=5, d=16), dict(V=50304, S=777, K=100, T=4, d=16),
+    dict(V=3000, S=640, K=50), dict(V=3000, S=1000, K=33, sigma=0.2), dict(V=9000, S=900, K=40, T=6),
+    dict(T=2, K=70000, S=700, V=2000, d=8), dict(V=100003, S=1023, K=40, T=3, d=16),
+    # beyond 1024 entries a draw: the L2-fed kernel
+    dict(V=5000, S=1500, K=30), dict(V=50304, S=2048, K=20, T=3, d=16),
 ])
 def test_edge_shapes(ctx, kw):
     wl = _small(**kw)
@@ -132,6 +140,20 @@ def test_full_vocab_more_shapes(ctx, kw):
     H, W, y = _inputs(wl)
     _compare(_gpu(ctx, H, W, y, wl), _oracle(H, W, y, wl),
              TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
+
+
+@pytest.mark.parametrize("kw", [dict(S=100), dict(S=1000), dict(V=4099, S=640, K=40),
+                                dict(V=50304, S=512, K=64, T=3, d=16), dict(T=2, K=70000, S=64, V=700),
+                                dict(V=20000, S=300, K=33, sigma=0.2, T=4, d=16)])
+def test_l2_fed_subset_kernel(cuda_ok, monkeypatch, kw):
+    """The L2-fed subset kernel (DUST_SUBSET_KERNEL=1), which runs beyond the
+    shared-memory kernel's reach (S > 1024 or larger V), on shapes the
+    shared-memory kernel would otherwise take."""
+    monkeypatch.setenv("DUST_SUBSET_KERNEL", "1")
+    c = dust.Context(0)
+    wl = _small(**kw)
+    H, W, y = _inputs(wl)
+    _compare(_gpu(c, H, W, y, wl), _oracle(H, W, y, wl), TOL_GW_BF16)
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(S=129, K=33), dict(V=4099, S=640, K=40),

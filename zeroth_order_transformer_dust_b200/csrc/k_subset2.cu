@@ -14,7 +14,8 @@
 // persistent over tokens. CTA r of the cluster holds the probability row and
 // the g accumulator for its slice [r seg, (r+1) seg) of q in shared memory
 // (CS = 2 at V = 50304: 2 x 100.6 KB per CTA; CS = 8 reaches V ~ 223k), so
-// the hot loop touches no global memory. Warps take batches of 32 draws from
+// the hot loop touches no global memory. A draw's S slots are NB blocks of
+// 128 per warp (S <= 1024, NB <= 8). Warps take batches of 32 draws from
 // a shared counter; in a batch each lane works out one draw's window start,
 // whether its window holds the target and the noise of the appended target
 // slot, and the warp then processes, one after the other, the draws whose
@@ -67,9 +68,13 @@ namespace {
 // workload); the fp32-accumulator variant and the library expm1 (large sigma)
 // keep 16 warps, where they need no spills.
 // NB = 3 (the packed Box-Muller step, the tightest variant) also keeps 16
-// warps: at 64 registers it spills whatever else the kernel holds.
-__host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb) {
-  return use_int && deg != 0 && nb != 3 ? 1024 : 512;
+// warps: at 64 registers it spills whatever else the kernel holds. So do
+// NB = 5 to 8 (S up to 1024), whose draws hold 20 to 32 noise values a lane;
+// their ragged-S forms with the library expm1 or fp32 accumulators need more
+// than 128 registers and run 12 warps (8 at NB = 7, 8 with the library expm1).
+__host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb, bool full) {
+  return nb >= 5 ? (!full && (deg == 0 || !use_int) ? (nb >= 7 && deg == 0 ? 256 : 384) : 512)
+                 : (use_int && deg != 0 && nb != 3 ? 1024 : 512);
 }
 
 // The Box-Muller step of NB-block draws in packed fp32x2 form, else scalar
@@ -77,9 +82,10 @@ __host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb) {
 // operations run on the FMA-heavy pipe, which the Philox multiplies already
 // load, so the scalar step (whose operations also use the FMA-lite pipe) is
 // the faster one (0.3-0.7% on B200); at NB = 3 it needs more than the 64
-// registers of a 1024-thread CTA, and those variants take the packed form.
+// registers of a 1024-thread CTA, and those variants take the packed form, as
+// do the 512-thread variants of NB = 5 to 8.
 template <int NB>
-constexpr bool packed_generator() { return NB == 3; }
+constexpr bool packed_generator() { return NB == 3 || NB >= 5; }
 
 constexpr int64_t kStaticSmem = 1024 + 8 * kSinCosTable;  // counters, angle table
 
@@ -139,8 +145,8 @@ __device__ __forceinline__ void accumulate(float* slot, float r, float x, float 
 // NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB; LIST: the
 // per-token draw list (its 16-byte entries follow the slices in shared memory).
 template <int NB, bool FULL, int DEG, bool INT, bool LIST>
-__global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
-  constexpr int kThreads = sub2_threads(INT, DEG, NB);
+__global__ __launch_bounds__(sub2_threads(INT, DEG, NB, FULL), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
+  constexpr int kThreads = sub2_threads(INT, DEG, NB, FULL);
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_next;    // next draw batch of the current token
   __shared__ int s_cnt;     // LIST: entries of the current token's draw list
@@ -175,8 +181,9 @@ __global__ __launch_bounds__(sub2_threads(INT, DEG, NB), 1) void k_subset2(const
   // addresses from shared memory where a window crosses into them: held in
   // registers they push those variants past the 64 registers of a
   // 1024-thread CTA. NB = 1 and 4 keep them in registers (1.4 % faster on the
-  // large-subset workload than reading them from shared memory).
-  constexpr bool kPeerRegs = NB == 1 || NB == 4;
+  // large-subset workload than reading them from shared memory), and so do the
+  // 512-thread NB = 5 to 8.
+  constexpr bool kPeerRegs = NB == 1 || NB >= 4;
   __shared__ float* s_peer[2];
   float* sp_peer = nullptr;
   float* sg_peer = nullptr;
@@ -607,7 +614,7 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(sub2_threads(INT, DEG, NB));
+  cfg.blockDim = dim3(sub2_threads(INT, DEG, NB, FULL));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -643,6 +650,14 @@ cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, i
             return cudaErrorNotSupported;
     case 4: if constexpr (!LIST) return full ? launch_deg<4, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<4, false, INT, LIST>(st, A, smem, sm, deg);
             return cudaErrorNotSupported;
+    case 5: if constexpr (!LIST) return full ? launch_deg<5, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<5, false, INT, LIST>(st, A, smem, sm, deg);
+            return cudaErrorNotSupported;
+    case 6: if constexpr (!LIST) return full ? launch_deg<6, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<6, false, INT, LIST>(st, A, smem, sm, deg);
+            return cudaErrorNotSupported;
+    case 7: if constexpr (!LIST) return full ? launch_deg<7, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<7, false, INT, LIST>(st, A, smem, sm, deg);
+            return cudaErrorNotSupported;
+    case 8: if constexpr (!LIST) return full ? launch_deg<8, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<8, false, INT, LIST>(st, A, smem, sm, deg);
+            return cudaErrorNotSupported;
     default: return cudaErrorNotSupported;
   }
 }
@@ -658,7 +673,7 @@ int64_t slice_len(int64_t V, int cs) { return ((V + cs - 1) / cs + 3) / 4 * 4; }
 // memory, with every slice at least S long, so that a window reaches at most
 // the next slice.
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
-  if (S < 1 || S > 512 || V >= (1LL << 31)) return 0;
+  if (S < 1 || S > 1024 || V >= (1LL << 31)) return 0;
   for (int cs = 1; cs <= 8; cs *= 2) {
     const int64_t seg = slice_len(V, cs);
     const int64_t last = V - (cs - 1) * seg;  // the last (shortest) slice
