@@ -112,6 +112,10 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     dict(T=2, K=70000, S=700, V=2000, d=8), dict(V=100003, S=1023, K=40, T=3, d=16),
     # beyond 1024 entries a draw: the L2-fed kernel
     dict(V=5000, S=1500, K=30), dict(V=50304, S=2048, K=20, T=3, d=16),
+    # the draw list at three and four blocks a draw in clusters of 4 and 8
+    # CTAs (up to 256 draws a CTA), with several tokens per cluster
+    dict(V=128256, S=512, K=1024, T=3, d=16), dict(V=70001, S=400, K=1024, T=3, d=16),
+    dict(V=100003, S=257, K=300, T=40, d=16), dict(V=128256, S=511, K=2048, T=2, d=16),
 ])
 def test_edge_shapes(ctx, kw):
     wl = _small(**kw)

@@ -72,9 +72,12 @@ namespace {
 // NB = 5 to 8 (S up to 1024), whose draws hold 20 to 32 noise values a lane;
 // their ragged-S forms with the library expm1 or fp32 accumulators need more
 // than 128 registers and run 12 warps (8 at NB = 7, 8 with the library expm1).
-__host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb, bool full) {
+// The draw-list variants of NB = 3 and 4 (clusters of 4 and 8 CTAs) run 16
+// warps too: the list's setup leaves them no register to spare at 64.
+__host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb, bool full,
+                                               bool list) {
   return nb >= 5 ? (!full && (deg == 0 || !use_int) ? (nb >= 7 && deg == 0 ? 256 : 384) : 512)
-                 : (use_int && deg != 0 && nb != 3 ? 1024 : 512);
+                 : (use_int && deg != 0 && nb != 3 && !(list && nb >= 3) ? 1024 : 512);
 }
 
 // The Box-Muller step of NB-block draws in packed fp32x2 form, else scalar
@@ -145,8 +148,8 @@ __device__ __forceinline__ void accumulate(float* slot, float r, float x, float 
 // NB: 128-slot blocks per draw (S <= 128 NB); FULL: S == 128 NB; LIST: the
 // per-token draw list (its 16-byte entries follow the slices in shared memory).
 template <int NB, bool FULL, int DEG, bool INT, bool LIST>
-__global__ __launch_bounds__(sub2_threads(INT, DEG, NB, FULL), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
-  constexpr int kThreads = sub2_threads(INT, DEG, NB, FULL);
+__global__ __launch_bounds__(sub2_threads(INT, DEG, NB, FULL, LIST), 1) void k_subset2(const __grid_constant__ Sub2Args A) {
+  constexpr int kThreads = sub2_threads(INT, DEG, NB, FULL, LIST);
   extern __shared__ __align__(16) float smem[];
   __shared__ int s_next;    // next draw batch of the current token
   __shared__ int s_cnt;     // LIST: entries of the current token's draw list
@@ -614,7 +617,7 @@ cudaError_t launch_one(cudaStream_t st, const Sub2Args& A, size_t smem, int sm_c
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(sub2_threads(INT, DEG, NB, FULL));
+  cfg.blockDim = dim3(sub2_threads(INT, DEG, NB, FULL, LIST));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -646,10 +649,8 @@ cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, i
   switch (nb) {
     case 1: return full ? launch_deg<1, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<1, false, INT, LIST>(st, A, smem, sm, deg);
     case 2: return full ? launch_deg<2, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<2, false, INT, LIST>(st, A, smem, sm, deg);
-    case 3: if constexpr (!LIST) return launch_deg<3, false, INT, LIST>(st, A, smem, sm, deg);
-            return cudaErrorNotSupported;
-    case 4: if constexpr (!LIST) return full ? launch_deg<4, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<4, false, INT, LIST>(st, A, smem, sm, deg);
-            return cudaErrorNotSupported;
+    case 3: return launch_deg<3, false, INT, LIST>(st, A, smem, sm, deg);
+    case 4: return full ? launch_deg<4, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<4, false, INT, LIST>(st, A, smem, sm, deg);
     case 5: if constexpr (!LIST) return full ? launch_deg<5, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<5, false, INT, LIST>(st, A, smem, sm, deg);
             return cudaErrorNotSupported;
     case 6: if constexpr (!LIST) return full ? launch_deg<6, true, INT, LIST>(st, A, smem, sm, deg) : launch_deg<6, false, INT, LIST>(st, A, smem, sm, deg);
@@ -737,8 +738,11 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   // the list's longer draw loop (6 % more instructions) costs more than the
   // balance gains (4.11 -> 4.30 ms), and larger S keeps batches: those
   // variants have no registers to spare.
+  // Clusters of 4 and 8 CTAs (the larger vocabularies) split a token's draws
+  // finer still: there the list serves S <= 512 up to 256 draws a CTA.
   const size_t slices = (size_t)2 * A.seg * 4, list_bytes = (size_t)p.K * 16;
-  const bool list = use_int && p.K <= 512 && p.S <= 256 &&
+  const bool list = use_int &&
+                    ((p.K <= 512 && p.S <= 256) || (cs >= 4 && p.S <= 512 && p.K <= 256 * cs)) &&
                     slices + list_bytes + (size_t)kStaticSmem <= (size_t)max_smem_optin;
   const size_t smem = slices + (list ? list_bytes : 0);
   const int deg = expm1_degree(p.sigma);
