@@ -61,9 +61,9 @@ ATTN_TC_FLOPS_PER_ROW_DH = 6
 ATTN_SAMPLE_DRAWS = 4
 # DRAM bytes (read + write) per token of the subset-draw kernel on the
 # large-subset workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of
-# one launch over its first 2048 tokens (413.35 + 176.61 MB), per token; the
+# one launch over its first 2048 tokens (415.33 + 179.30 MB), per token; the
 # kernel's traffic is per token (the logit row in, the fp16 g operand out).
-SUBSET_DRAM_BYTES_PER_TOKEN = (413.354752e6 + 176.610304e6) / 2048
+SUBSET_DRAM_BYTES_PER_TOKEN = (415.334144e6 + 179.300096e6) / 2048
 PROFILED_SUBSET_WORKLOAD = "large_subset_bf16"
 
 
