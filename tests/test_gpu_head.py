@@ -110,6 +110,9 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     dict(V=50304, S=1024, K=64, T=5, d=16), dict(V=50304, S=777, K=100, T=4, d=16),
     dict(V=3000, S=640, K=50), dict(V=3000, S=1000, K=33, sigma=0.2), dict(V=9000, S=900, K=40, T=6),
     dict(T=2, K=70000, S=700, V=2000, d=8), dict(V=100003, S=1023, K=40, T=3, d=16),
+    # windows that cover the whole vocabulary (S = V; the target always in
+    # the window), and eight blocks with fp32 accumulators
+    dict(V=1000, S=1000, K=20), dict(V=1024, S=1024, K=16, T=9), dict(T=1, K=66000, S=1024, V=2048, d=8),
     # beyond 1024 entries a draw: the L2-fed kernel
     dict(V=5000, S=1500, K=30), dict(V=50304, S=2048, K=20, T=3, d=16),
     # the draw list at three and four blocks a draw in clusters of 4 and 8
