@@ -362,23 +362,25 @@ def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
 def _mlp_flops_per_row(wl) -> tuple:
     """(algorithmic, executed) flops of the perturbed pass per (token, draw):
     the method's GEMMs dh = da W_down^T (up), du = (sigma eps) W_up^T and dh
-    (attention output projection) and dz = dh W_head^T; the kernels carry
-    each activation operand as two bf16 planes (hi and lo), so they execute
-    twice the depth of every contraction."""
+    (attention output projection) and dz = dh W_head^T. The kernels carry
+    the activation operands of the first two as two bf16 planes (hi and lo),
+    executing twice their depth; dz contracts the hi plane of dh only (the lo
+    plane's first-order effect is added per row, 2d flops)."""
     d, dff, V = wl.d, wl.d_ff, wl.V
-    alg = 2.0 * d * V
+    head = 2.0 * d * V
+    rest = 0.0
     if wl.variant in ("mlp", "attn_out"):
-        alg += 2.0 * dff * d
+        rest += 2.0 * dff * d
     if wl.variant == "attn_out":
-        alg += 2.0 * d * dff
-    return alg, 2.0 * alg
+        rest += 2.0 * d * dff
+    return head + rest, head + 2.0 * rest + 2.0 * d
 
 
 def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
     """Tensor-core roofline of the MLP-block perturbed pass: the method's flops
     per (token, draw) over the stage time, against the sustained bf16 peak (a
     pass of hundreds of milliseconds runs under the power cap); the flops the
-    hi/lo-plane GEMMs execute are reported beside it."""
+    GEMMs execute are reported beside it."""
     alg, exe = _mlp_flops_per_row(wl)
     rows = wl.T * wl.K
     t = perturbed_ms * 1e-3
@@ -390,7 +392,9 @@ def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
             "peak_basis": "measured bf16 sustained (power-capped) peak",
             "executed": {"flops": exe * rows, "achieved": exe * rows / t / 1e12,
                          "frac": exe * rows / t / 1e12 / peak,
-                         "basis": "hi/lo bf16 planes: each contraction executed at twice its depth"}}
+                         "basis": ("dz on the hi plane of dh plus a d-long correction per row; "
+                                   "the smaller contractions on hi/lo bf16 planes at twice "
+                                   "their depth")}}
 
 
 def _gemm_report(flops: float, ms: float, peaks) -> dict:

@@ -58,7 +58,10 @@ def test_mlp_roofline_flops():
         if name == "attn_out_bf16":
             per_row += 2 * d * dff                   # du = (sigma eps) W_up^T
         assert math.isclose(r["flops"], per_row * wl.T * wl.K, rel_tol=1e-12)
-        assert math.isclose(r["executed"]["flops"], 2 * r["flops"], rel_tol=1e-12)
+        # dz on the hi plane only (plus a d-long correction per row), the rest
+        # on hi/lo planes at twice their depth
+        executed = 2 * d * V + 2 * (per_row - 2 * d * V) + 2 * d
+        assert math.isclose(r["executed"]["flops"], executed * wl.T * wl.K, rel_tol=1e-12)
         assert r["bound"] == "tensor" and r["peak"] == PEAKS["bf16_tflops_sustained"]
     # the up-projection's 82.0 MFLOP per token-draw
     alg, _ = bench._mlp_flops_per_row(synth.CONFIGS["mlp_bf16"])

@@ -615,6 +615,26 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
   DUST_CU(launch_lse_rows(st, Z, T, V, targets, 0, (float*)ctx->lse.p, loss, true, ctx->d_status));
   ctx->launches += 1;
   mark(ctx, "lse");
+  // U = P W_head (T x d, fp32) from the softmax P (now in Z) rounded to bf16:
+  // the perturbed rewards take the head GEMM on the hi plane of dh only and add
+  // the lo plane's first-order effect, lo . (W_head[y_t] - U_t), per row.
+  // (The dropped terms are of second order in the lo plane and in P's
+  // rounding: about 6e-8 on the rewards and 3e-6 relative on g in the oracle's
+  // arithmetic on the mlp_bf16 shapes, against 2e-5 and 1e-4.)
+  DUST_TRY(ensure(ctx, ctx->mlp_pb, (size_t)T * V * 2));
+  DUST_TRY(ensure(ctx, ctx->mlp_uw, (size_t)T * d * 4));
+  float* Uw = (float*)ctx->mlp_uw.p;
+  DUST_CU(launch_f32_to_bf16(st, Z, T * V, (__nv_bfloat16*)ctx->mlp_pb.p, ctx->sm_count));
+  ctx->launches += 1;
+  {
+    GemmDesc g{};
+    g.M = T; g.N = d; g.K = V; g.A = ctx->mlp_pb.p; g.lda = V; g.a_kmajor = true;
+    g.B = W_head; g.ldb = d; g.b_kmajor = false; g.dtype = DUST_BF16;
+    EpiDesc e{};
+    e.kind = kEpiF32; e.C = Uw; e.ldc = d;
+    DUST_TRY(run_gemm(ctx, g, e));
+  }
+  mark(ctx, "head_mean");
 
   // perturbed passes, a chunk of tokens (all K draws each) at a time
   const int64_t max_rows = 131072;
@@ -679,12 +699,12 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
       e.kind = kEpiSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       DUST_TRY(run_gemm(ctx, g, e));
     }
-    // dz = dh W_head^T with the reward epilogue (dz never reaches memory)
+    // dz = dh_hi W_head^T with the reward epilogue (dz never reaches memory)
     int used_parts = (int)((V + 127) / 128);  // the CUDA-core reward GEMM's 128-column tiles
     {
       GemmDesc g{};
-      g.M = rows; g.N = V; g.K = 2 * d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
-      g.B = ctx->wh2.p; g.ldb = 2 * d; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = V; g.K = d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
+      g.B = W_head; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
       e.kind = kEpiReward; e.P = Z; e.y = targets; e.t0 = t0; e.draws = p.K;
       e.part = (float*)ctx->part.p; e.dzy = (float*)ctx->dzy.p;
@@ -699,7 +719,9 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
     }
     DUST_CU(launch_reward_combine_rows(st, (float*)ctx->part.p, used_parts, (float*)ctx->dzy.p,
                                        rows, t0 * K, p.K, r));
-    ctx->launches += 1;
+    DUST_CU(launch_mlp_reward_corr(st, dh, d, (const __nv_bfloat16*)W_head, V, targets, Uw, t0,
+                                   p.K, rows, r));
+    ctx->launches += 2;
   }
   mark(ctx, "perturbed");
   if (attn)

@@ -214,7 +214,8 @@ struct dust_ctx {
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
       attn_o, attn_lse, attn_gb, attn_w, attn_tcr, attn_coef,
-      hsc;  // the fp16 G_W path's largest |h| and epilogue scale
+      hsc,            // the fp16 G_W path's largest |h| and epilogue scale
+      mlp_pb, mlp_uw;  // the MLP rewards' correction: P in bf16, U = P W_head
 };
 
 namespace dust {
@@ -319,6 +320,16 @@ cudaError_t launch_reward_gemm_simt(cudaStream_t st, const GemmDesc& g, const fl
 cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int nparts,
                                        const float* dzy, int64_t rows, int64_t row0, int32_t K,
                                        float* r);
+// The perturbed head GEMM contracts only the hi plane of dh = [hi | lo]
+// (rows x 2d bf16); this adds the first-order effect of the lo plane to each
+// reward: r[t0 K + row] += lo_row . (W_head[y_t] - U_t), t = t0 + row / K,
+// U (T x d fp32) = P W_head with P the clean softmax.
+cudaError_t launch_mlp_reward_corr(cudaStream_t st, const __nv_bfloat16* dh, int64_t d,
+                                   const __nv_bfloat16* W_head, int64_t V, const int32_t* y,
+                                   const float* U, int64_t t0, int32_t K, int64_t rows, float* r);
+// out[i] = bf16(x[i]) (round to nearest even), n elements.
+cudaError_t launch_f32_to_bf16(cudaStream_t st, const float* x, int64_t n, __nv_bfloat16* out,
+                               int sm_count);
 // g of the up-projection (width d_ff; gop as bf16 hi/lo planes for bf16 calls)
 // or, with down, of the down-projection (width d; gop fp32).
 cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,

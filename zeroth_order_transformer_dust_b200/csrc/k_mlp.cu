@@ -481,6 +481,85 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
   return cudaGetLastError();
 }
 
+// First-order correction of the rewards for the lo plane of dh (the head GEMM
+// contracts the hi plane only): a warp per (token, draw) row, 16-byte loads
+// of lo, of W_head's target row and of U_t where d is a multiple of 8.
+__global__ __launch_bounds__(256) void k_mlp_reward_corr(const __nv_bfloat16* __restrict__ dh,
+                                                         int64_t d,
+                                                         const __nv_bfloat16* __restrict__ Wh,
+                                                         int64_t V, const int32_t* __restrict__ y,
+                                                         const float* __restrict__ U, int64_t t0,
+                                                         int32_t K, int64_t rows,
+                                                         float* __restrict__ r) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int64_t t = t0 + row / K;
+  int32_t yt = y[t];
+  if (yt < 0 || (int64_t)yt >= V) yt = 0;  // reported by the loss kernel
+  const __nv_bfloat16* lo = dh + row * 2 * d + d;
+  const __nv_bfloat16* wy = Wh + (int64_t)yt * d;
+  const float* ut = U + t * d;
+  float s = 0.0f;
+  if ((d & 7) == 0) {
+    for (int64_t i = (int64_t)lane * 8; i < d; i += 256) {
+      const uint4 lv = *reinterpret_cast<const uint4*>(lo + i);
+      const uint4 wv = *reinterpret_cast<const uint4*>(wy + i);
+      const float4 u0 = *reinterpret_cast<const float4*>(ut + i);
+      const float4 u1 = *reinterpret_cast<const float4*>(ut + i + 4);
+      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lv);
+      const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
+      const float uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 lf = __bfloat1622float2(l2[q]), wf = __bfloat1622float2(w2[q]);
+        s = fmaf(lf.x, wf.x - uu[2 * q], s);
+        s = fmaf(lf.y, wf.y - uu[2 * q + 1], s);
+      }
+    }
+  } else {
+    for (int64_t i = lane; i < d; i += 32)
+      s = fmaf(__bfloat162float(lo[i]), __bfloat162float(wy[i]) - ut[i], s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) r[t0 * K + row] += s;
+}
+
+__global__ void k_f32_to_bf16(const float* __restrict__ x, int64_t n,
+                              __nv_bfloat16* __restrict__ out) {
+  const int64_t n4 = n / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(x)[i];
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out + 4 * i);
+    o[0] = __floats2bfloat162_rn(v.x, v.y);
+    o[1] = __floats2bfloat162_rn(v.z, v.w);
+  }
+  for (int64_t i = 4 * n4 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(x[i]);
+}
+
+cudaError_t launch_mlp_reward_corr(cudaStream_t st, const __nv_bfloat16* dh, int64_t d,
+                                   const __nv_bfloat16* W_head, int64_t V, const int32_t* y,
+                                   const float* U, int64_t t0, int32_t K, int64_t rows, float* r) {
+  if (rows <= 0) return cudaSuccess;
+  k_mlp_reward_corr<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(dh, d, W_head, V, y, U, t0, K,
+                                                                 rows, r);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(cudaStream_t st, const float* x, int64_t n, __nv_bfloat16* out,
+                               int sm_count) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n / 4 + 255) / 256;
+  if (blocks > (int64_t)sm_count * 16) blocks = (int64_t)sm_count * 16;
+  if (blocks < 1) blocks = 1;
+  k_f32_to_bf16<<<(unsigned)blocks, 256, 0, st>>>(x, n, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mlp_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
                          void* gop, bool down) {
   const int64_t width = down ? p.d : p.d_ff;
