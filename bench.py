@@ -362,18 +362,19 @@ def _attn_roofline(wl, draws_ms: float, peaks) -> dict:
 def _mlp_flops_per_row(wl) -> tuple:
     """(algorithmic, executed) flops of the perturbed pass per (token, draw):
     the method's GEMMs dh = da W_down^T (up), du = (sigma eps) W_up^T and dh
-    (attention output projection) and dz = dh W_head^T. The kernels carry
-    the activation operands of the first two as two bf16 planes (hi and lo),
-    executing twice their depth; dz contracts the hi plane of dh only (the lo
-    plane's first-order effect is added per row, 2d flops)."""
+    (attention output projection) and dz = dh W_head^T. dz and dh contract
+    the hi planes of their bf16 operands only (the lo planes' first-order
+    effects are added per row: 2d flops, and 2 d_ff where dh comes from da);
+    du contracts both planes of sigma eps, twice its depth."""
     d, dff, V = wl.d, wl.d_ff, wl.V
-    head = 2.0 * d * V
-    rest = 0.0
+    alg = exe = 2.0 * d * V + 2.0 * d
     if wl.variant in ("mlp", "attn_out"):
-        rest += 2.0 * dff * d
+        alg += 2.0 * dff * d
+        exe += 2.0 * dff * d + 2.0 * dff
     if wl.variant == "attn_out":
-        rest += 2.0 * d * dff
-    return head + rest, head + 2.0 * rest + 2.0 * d
+        alg += 2.0 * d * dff
+        exe += 2.0 * 2.0 * d * dff
+    return alg - 2.0 * d, exe
 
 
 def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
@@ -392,9 +393,8 @@ def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:
             "peak_basis": "measured bf16 sustained (power-capped) peak",
             "executed": {"flops": exe * rows, "achieved": exe * rows / t / 1e12,
                          "frac": exe * rows / t / 1e12 / peak,
-                         "basis": ("dz on the hi plane of dh plus a d-long correction per row; "
-                                   "the smaller contractions on hi/lo bf16 planes at twice "
-                                   "their depth")}}
+                         "basis": ("dz and dh on the hi planes of their operands plus a "
+                                   "correction per row; du on both planes of sigma eps")}}
 
 
 def _gemm_report(flops: float, ms: float, peaks) -> dict:

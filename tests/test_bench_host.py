@@ -58,9 +58,13 @@ def test_mlp_roofline_flops():
         if name == "attn_out_bf16":
             per_row += 2 * d * dff                   # du = (sigma eps) W_up^T
         assert math.isclose(r["flops"], per_row * wl.T * wl.K, rel_tol=1e-12)
-        # dz on the hi plane only (plus a d-long correction per row), the rest
-        # on hi/lo planes at twice their depth
-        executed = 2 * d * V + 2 * (per_row - 2 * d * V) + 2 * d
+        # dz and dh on the hi planes only, plus a correction per row (2d, and
+        # 2 d_ff where dh comes from da); du on both planes of sigma eps
+        executed = per_row + 2 * d
+        if name != "mlp_down_bf16":
+            executed += 2 * dff
+        if name == "attn_out_bf16":
+            executed += 2 * d * dff
         assert math.isclose(r["executed"]["flops"], executed * wl.T * wl.K, rel_tol=1e-12)
         assert r["bound"] == "tensor" and r["peak"] == PEAKS["bf16_tflops_sustained"]
     # the up-projection's 82.0 MFLOP per token-draw

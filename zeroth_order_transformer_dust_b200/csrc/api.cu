@@ -325,7 +325,8 @@ void dust_destroy(dust_ctx* ctx) {
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
                  &ctx->out_loss, &ctx->out_r, &ctx->out_gv, &ctx->lsep, &ctx->mlp_a32,
                  &ctx->mlp_dn, &ctx->mlp_du, &ctx->wu2, &ctx->attn_o, &ctx->attn_lse,
-                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr, &ctx->attn_coef, &ctx->hsc};
+                 &ctx->attn_gb, &ctx->attn_w, &ctx->attn_tcr, &ctx->attn_coef, &ctx->hsc,
+                 &ctx->mlp_pb, &ctx->mlp_uw, &ctx->mlp_ub, &ctx->mlp_wv, &ctx->mlp_wt};
   for (Buf* b : bufs)
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
@@ -621,17 +622,46 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
   // (The dropped terms are of second order in the lo plane and in P's
   // rounding: about 6e-8 on the rewards and 3e-6 relative on g in the oracle's
   // arithmetic on the mlp_bf16 shapes, against 2e-5 and 1e-4.)
+  // (both GEMMs K-major: W_head and W_down transposed once per call)
+  const int64_t ldv = (V + 7) / 8 * 8, ldd = (d + 7) / 8 * 8;
   DUST_TRY(ensure(ctx, ctx->mlp_pb, (size_t)T * V * 2));
   DUST_TRY(ensure(ctx, ctx->mlp_uw, (size_t)T * d * 4));
+  DUST_TRY(ensure(ctx, ctx->mlp_wt, (size_t)std::max(d * ldv, dff * ldd) * 2));
   float* Uw = (float*)ctx->mlp_uw.p;
   DUST_CU(launch_f32_to_bf16(st, Z, T * V, (__nv_bfloat16*)ctx->mlp_pb.p, ctx->sm_count));
-  ctx->launches += 1;
+  DUST_CU(launch_transpose_bf16(st, (const __nv_bfloat16*)W_head, V, d,
+                                (__nv_bfloat16*)ctx->mlp_wt.p, ldv));
+  ctx->launches += 2;
   {
     GemmDesc g{};
     g.M = T; g.N = d; g.K = V; g.A = ctx->mlp_pb.p; g.lda = V; g.a_kmajor = true;
-    g.B = W_head; g.ldb = d; g.b_kmajor = false; g.dtype = DUST_BF16;
+    g.B = ctx->mlp_wt.p; g.ldb = ldv; g.b_kmajor = true; g.dtype = DUST_BF16;
     EpiDesc e{};
     e.kind = kEpiF32; e.C = Uw; e.ldc = d;
+    DUST_TRY(run_gemm(ctx, g, e));
+  }
+  // u_t = W_head[y_t] - U_t in place of U (and in bf16 where Wv needs it).
+  // Where dh = da W_down^T (up-projection, attention output projection), that
+  // GEMM too contracts only the hi plane of da; the lo plane moves a reward by
+  // da_lo . Wv_t to first order, Wv = u W_down (T x d_ff, from u in bf16).
+  // With both corrections the oracle's rewards move by 1.1e-7 and g by 4.9e-6
+  // relative on the mlp_bf16 shapes.
+  if (!down) DUST_TRY(ensure(ctx, ctx->mlp_ub, (size_t)T * d * 2));
+  DUST_CU(launch_head_ut(st, (const __nv_bfloat16*)W_head, V, targets, Uw, T, d,
+                         down ? nullptr : (__nv_bfloat16*)ctx->mlp_ub.p, ctx->sm_count));
+  ctx->launches += 1;
+  float* Wv = nullptr;
+  if (!down) {
+    DUST_TRY(ensure(ctx, ctx->mlp_wv, (size_t)T * dff * 4));
+    Wv = (float*)ctx->mlp_wv.p;
+    DUST_CU(launch_transpose_bf16(st, (const __nv_bfloat16*)W_down, d, dff,
+                                  (__nv_bfloat16*)ctx->mlp_wt.p, ldd));
+    ctx->launches += 1;
+    GemmDesc g{};
+    g.M = T; g.N = dff; g.K = d; g.A = ctx->mlp_ub.p; g.lda = d; g.a_kmajor = true;
+    g.B = ctx->mlp_wt.p; g.ldb = ldd; g.b_kmajor = true; g.dtype = DUST_BF16;
+    EpiDesc e{};
+    e.kind = kEpiF32; e.C = Wv; e.ldc = dff;
     DUST_TRY(run_gemm(ctx, g, e));
   }
   mark(ctx, "head_mean");
@@ -683,8 +713,8 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
       DUST_CU(launch_gelu_delta_rows(st, p, u, du, t0, nt, da));
       ctx->launches += 1;
       GemmDesc g{};
-      g.M = rows; g.N = d; g.K = 2 * dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
-      g.B = ctx->wd2.p; g.ldb = 2 * dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
+      g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
       e.kind = kEpiResidSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       e.resid = dn; e.ldr = 2 * d; e.rsplit = d;
@@ -693,8 +723,8 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
       DUST_CU(launch_mlp_delta_a(st, p, u, t0, nt, da, true, nullptr));
       ctx->launches += 1;
       GemmDesc g{};
-      g.M = rows; g.N = d; g.K = 2 * dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
-      g.B = ctx->wd2.p; g.ldb = 2 * dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
+      g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
       e.kind = kEpiSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       DUST_TRY(run_gemm(ctx, g, e));
@@ -719,8 +749,8 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
     }
     DUST_CU(launch_reward_combine_rows(st, (float*)ctx->part.p, used_parts, (float*)ctx->dzy.p,
                                        rows, t0 * K, p.K, r));
-    DUST_CU(launch_mlp_reward_corr(st, dh, d, (const __nv_bfloat16*)W_head, V, targets, Uw, t0,
-                                   p.K, rows, r));
+    DUST_CU(launch_mlp_reward_corr(st, dh, d, Uw, down ? nullptr : da, dff, Wv, t0, p.K, rows,
+                                   r));
     ctx->launches += 2;
   }
   mark(ctx, "perturbed");

@@ -215,7 +215,9 @@ struct dust_ctx {
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
       attn_o, attn_lse, attn_gb, attn_w, attn_tcr, attn_coef,
       hsc,            // the fp16 G_W path's largest |h| and epilogue scale
-      mlp_pb, mlp_uw;  // the MLP rewards' correction: P in bf16, U = P W_head
+      mlp_pb, mlp_uw,  // the MLP rewards' correction: P in bf16, U = P W_head,
+      mlp_ub, mlp_wv,  // U in bf16, Wv = U W_down
+      mlp_wt;          // W_head or W_down transposed for those GEMMs
 };
 
 namespace dust {
@@ -322,11 +324,18 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
                                        float* r);
 // The perturbed head GEMM contracts only the hi plane of dh = [hi | lo]
 // (rows x 2d bf16); this adds the first-order effect of the lo plane to each
-// reward: r[t0 K + row] += lo_row . (W_head[y_t] - U_t), t = t0 + row / K,
-// U (T x d fp32) = P W_head with P the clean softmax.
+// reward: r[t0 K + row] += lo_row . u_t, t = t0 + row / K, with
+// u_t = W_head[y_t] - (P W_head)_t (Ut, T x d fp32; P the clean softmax).
+// Where dh itself came from the hi plane of da = [hi | lo] (rows x 2 d_ff
+// bf16, non-null), it also adds da_lo_row . Wv_t, Wv = u W_down (T x d_ff fp32).
 cudaError_t launch_mlp_reward_corr(cudaStream_t st, const __nv_bfloat16* dh, int64_t d,
-                                   const __nv_bfloat16* W_head, int64_t V, const int32_t* y,
-                                   const float* U, int64_t t0, int32_t K, int64_t rows, float* r);
+                                   const float* Ut, const __nv_bfloat16* da, int64_t dff,
+                                   const float* Wv, int64_t t0, int32_t K, int64_t rows, float* r);
+// U := W_head[y_t] - U row by row (T x d fp32, in place), and bf16(U) into Ub
+// (may be null). Targets outside [0, V) take row 0.
+cudaError_t launch_head_ut(cudaStream_t st, const __nv_bfloat16* W_head, int64_t V,
+                           const int32_t* y, float* U, int64_t T, int64_t d, __nv_bfloat16* Ub,
+                           int sm_count);
 // out[i] = bf16(x[i]) (round to nearest even), n elements.
 cudaError_t launch_f32_to_bf16(cudaStream_t st, const float* x, int64_t n, __nv_bfloat16* out,
                                int sm_count);

@@ -481,49 +481,67 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
   return cudaGetLastError();
 }
 
+// a . b over n entries of a bf16 row and an fp32 row (one warp; 16-byte loads
+// where n is a multiple of 8 and the rows 16-byte aligned)
+__device__ __forceinline__ float warp_dot_bf16_f32(const __nv_bfloat16* __restrict__ a,
+                                                   const float* __restrict__ b, int64_t n,
+                                                   int lane) {
+  float s = 0.0f;
+  if ((n & 7) == 0) {
+    for (int64_t i = (int64_t)lane * 8; i < n; i += 256) {
+      const uint4 av = *reinterpret_cast<const uint4*>(a + i);
+      const float4 b0 = *reinterpret_cast<const float4*>(b + i);
+      const float4 b1 = *reinterpret_cast<const float4*>(b + i + 4);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&av);
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 af = __bfloat1622float2(a2[q]);
+        s = fmaf(af.x, bb[2 * q], s);
+        s = fmaf(af.y, bb[2 * q + 1], s);
+      }
+    }
+  } else {
+    for (int64_t i = lane; i < n; i += 32) s = fmaf(__bfloat162float(a[i]), b[i], s);
+  }
+  return s;
+}
+
 // First-order correction of the rewards for the lo plane of dh (the head GEMM
-// contracts the hi plane only): a warp per (token, draw) row, 16-byte loads
-// of lo, of W_head's target row and of U_t where d is a multiple of 8.
+// contracts the hi plane only), and for the lo plane of da where dh came from
+// its hi plane: a warp per (token, draw) row, 16-byte loads where the row
+// lengths are multiples of 8.
 __global__ __launch_bounds__(256) void k_mlp_reward_corr(const __nv_bfloat16* __restrict__ dh,
-                                                         int64_t d,
-                                                         const __nv_bfloat16* __restrict__ Wh,
-                                                         int64_t V, const int32_t* __restrict__ y,
-                                                         const float* __restrict__ U, int64_t t0,
+                                                         int64_t d, const float* __restrict__ Ut,
+                                                         const __nv_bfloat16* __restrict__ da,
+                                                         int64_t dff,
+                                                         const float* __restrict__ Wv, int64_t t0,
                                                          int32_t K, int64_t rows,
                                                          float* __restrict__ r) {
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   const int64_t t = t0 + row / K;
-  int32_t yt = y[t];
-  if (yt < 0 || (int64_t)yt >= V) yt = 0;  // reported by the loss kernel
-  const __nv_bfloat16* lo = dh + row * 2 * d + d;
-  const __nv_bfloat16* wy = Wh + (int64_t)yt * d;
-  const float* ut = U + t * d;
-  float s = 0.0f;
-  if ((d & 7) == 0) {
-    for (int64_t i = (int64_t)lane * 8; i < d; i += 256) {
-      const uint4 lv = *reinterpret_cast<const uint4*>(lo + i);
-      const uint4 wv = *reinterpret_cast<const uint4*>(wy + i);
-      const float4 u0 = *reinterpret_cast<const float4*>(ut + i);
-      const float4 u1 = *reinterpret_cast<const float4*>(ut + i + 4);
-      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lv);
-      const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&wv);
-      const float uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 lf = __bfloat1622float2(l2[q]), wf = __bfloat1622float2(w2[q]);
-        s = fmaf(lf.x, wf.x - uu[2 * q], s);
-        s = fmaf(lf.y, wf.y - uu[2 * q + 1], s);
-      }
-    }
-  } else {
-    for (int64_t i = lane; i < d; i += 32)
-      s = fmaf(__bfloat162float(lo[i]), __bfloat162float(wy[i]) - ut[i], s);
-  }
+  float s = warp_dot_bf16_f32(dh + row * 2 * d + d, Ut + t * d, d, lane);
+  if (da) s += warp_dot_bf16_f32(da + row * 2 * dff + dff, Wv + t * dff, dff, lane);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) r[t0 * K + row] += s;
+}
+
+// U_t := W_head[y_t] - U_t in place (T x d), and its bf16 copy.
+__global__ void k_head_ut(const __nv_bfloat16* __restrict__ Wh, int64_t V,
+                          const int32_t* __restrict__ y, float* __restrict__ U, int64_t T,
+                          int64_t d, __nv_bfloat16* __restrict__ Ub) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T * d;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / d;
+    int32_t yt = y[t];
+    if (yt < 0 || (int64_t)yt >= V) yt = 0;  // reported by the loss kernel
+    const float v = __bfloat162float(Wh[(int64_t)yt * d + (i - t * d)]) - U[i];
+    U[i] = v;
+    if (Ub) Ub[i] = __float2bfloat16_rn(v);
+  }
 }
 
 __global__ void k_f32_to_bf16(const float* __restrict__ x, int64_t n,
@@ -542,11 +560,21 @@ __global__ void k_f32_to_bf16(const float* __restrict__ x, int64_t n,
 }
 
 cudaError_t launch_mlp_reward_corr(cudaStream_t st, const __nv_bfloat16* dh, int64_t d,
-                                   const __nv_bfloat16* W_head, int64_t V, const int32_t* y,
-                                   const float* U, int64_t t0, int32_t K, int64_t rows, float* r) {
+                                   const float* Ut, const __nv_bfloat16* da, int64_t dff,
+                                   const float* Wv, int64_t t0, int32_t K, int64_t rows, float* r) {
   if (rows <= 0) return cudaSuccess;
-  k_mlp_reward_corr<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(dh, d, W_head, V, y, U, t0, K,
+  k_mlp_reward_corr<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(dh, d, Ut, da, dff, Wv, t0, K,
                                                                  rows, r);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_head_ut(cudaStream_t st, const __nv_bfloat16* W_head, int64_t V,
+                           const int32_t* y, float* U, int64_t T, int64_t d, __nv_bfloat16* Ub,
+                           int sm_count) {
+  if (T * d <= 0) return cudaSuccess;
+  int64_t blocks = (T * d + 255) / 256;
+  if (blocks > (int64_t)sm_count * 16) blocks = (int64_t)sm_count * 16;
+  k_head_ut<<<(unsigned)blocks, 256, 0, st>>>(W_head, V, y, U, T, d, Ub);
   return cudaGetLastError();
 }
 
