@@ -365,7 +365,8 @@ def _mlp_flops_per_row(wl) -> tuple:
     (attention output projection) and dz = dh W_head^T. dz and dh contract
     the hi planes of their bf16 operands only (the lo planes' first-order
     effects are added per row: 2d flops, and 2 d_ff where dh comes from da);
-    du contracts both planes of sigma eps, twice its depth."""
+    du contracts both planes of sigma eps, twice its depth. Above sigma = 0.05
+    every contraction takes both planes."""
     d, dff, V = wl.d, wl.d_ff, wl.V
     alg = exe = 2.0 * d * V + 2.0 * d
     if wl.variant in ("mlp", "attn_out"):
@@ -374,7 +375,10 @@ def _mlp_flops_per_row(wl) -> tuple:
     if wl.variant == "attn_out":
         alg += 2.0 * d * dff
         exe += 2.0 * 2.0 * d * dff
-    return alg - 2.0 * d, exe
+    alg -= 2.0 * d
+    if wl.sigma > 0.05:  # both planes everywhere, no corrections
+        exe = 2.0 * alg
+    return alg, exe
 
 
 def _mlp_roofline(wl, perturbed_ms: float, peaks) -> dict:

@@ -43,8 +43,10 @@ def _check(got, ref):
     assert rel_fro(got["G"], ref["G"]) < TOL_GW_BF16
 
 
+# sigma 0.05 is the largest the one-plane GEMMs with their first-order
+# corrections take; above it both planes are contracted
 @pytest.mark.parametrize("kw", [dict(), dict(T=1, K=1), dict(d=33, d_ff=200, V=517), dict(K=130),
-                                dict(sigma=0.1)])
+                                dict(sigma=0.1), dict(sigma=0.05, K=64), dict(sigma=0.06, K=64)])
 def test_small_mlp(ctx, kw):
     base = dict(T=24, d=64, d_ff=256, V=1000, K=16, sigma=1e-2)
     base.update(kw)
@@ -93,7 +95,7 @@ def _check_down(got, ref):
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(T=1, K=1), dict(d=33, d_ff=200, V=517), dict(K=130),
-                                dict(sigma=0.1)])
+                                dict(sigma=0.1), dict(sigma=0.05, K=64)])
 def test_small_mlp_down(ctx, kw):
     base = dict(T=24, d=64, d_ff=256, V=1000, K=16, sigma=1e-2)
     base.update(kw)
@@ -137,7 +139,7 @@ def _run_attn(ctx, inp, wl, t0=0, T=None):
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(T=1, K=1), dict(d=40, d_ff=200, V=517), dict(K=130),
-                                dict(sigma=0.1)])
+                                dict(sigma=0.1), dict(sigma=0.05, K=64)])
 def test_small_attn_out(ctx, kw):
     base = dict(T=24, d=64, d_ff=256, V=1000, K=16, sigma=1e-2)
     base.update(kw)

@@ -619,52 +619,60 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
   // U = P W_head (T x d, fp32) from the softmax P (now in Z) rounded to bf16:
   // the perturbed rewards take the head GEMM on the hi plane of dh only and add
   // the lo plane's first-order effect, lo . (W_head[y_t] - U_t), per row.
-  // (The dropped terms are of second order in the lo plane and in P's
-  // rounding: about 6e-8 on the rewards and 3e-6 relative on g in the oracle's
-  // arithmetic on the mlp_bf16 shapes, against 2e-5 and 1e-4.)
-  // (both GEMMs K-major: W_head and W_down transposed once per call)
-  const int64_t ldv = (V + 7) / 8 * 8, ldd = (d + 7) / 8 * 8;
-  DUST_TRY(ensure(ctx, ctx->mlp_pb, (size_t)T * V * 2));
-  DUST_TRY(ensure(ctx, ctx->mlp_uw, (size_t)T * d * 4));
-  DUST_TRY(ensure(ctx, ctx->mlp_wt, (size_t)std::max(d * ldv, dff * ldd) * 2));
-  float* Uw = (float*)ctx->mlp_uw.p;
-  DUST_CU(launch_f32_to_bf16(st, Z, T * V, (__nv_bfloat16*)ctx->mlp_pb.p, ctx->sm_count));
-  DUST_CU(launch_transpose_bf16(st, (const __nv_bfloat16*)W_head, V, d,
-                                (__nv_bfloat16*)ctx->mlp_wt.p, ldv));
-  ctx->launches += 2;
-  {
-    GemmDesc g{};
-    g.M = T; g.N = d; g.K = V; g.A = ctx->mlp_pb.p; g.lda = V; g.a_kmajor = true;
-    g.B = ctx->mlp_wt.p; g.ldb = ldv; g.b_kmajor = true; g.dtype = DUST_BF16;
-    EpiDesc e{};
-    e.kind = kEpiF32; e.C = Uw; e.ldc = d;
-    DUST_TRY(run_gemm(ctx, g, e));
-  }
-  // u_t = W_head[y_t] - U_t in place of U (and in bf16 where Wv needs it).
-  // Where dh = da W_down^T (up-projection, attention output projection), that
-  // GEMM too contracts only the hi plane of da; the lo plane moves a reward by
-  // da_lo . Wv_t to first order, Wv = u W_down (T x d_ff, from u in bf16).
-  // With both corrections the oracle's rewards move by 1.1e-7 and g by 4.9e-6
-  // relative on the mlp_bf16 shapes.
-  if (!down) DUST_TRY(ensure(ctx, ctx->mlp_ub, (size_t)T * d * 2));
-  DUST_CU(launch_head_ut(st, (const __nv_bfloat16*)W_head, V, targets, Uw, T, d,
-                         down ? nullptr : (__nv_bfloat16*)ctx->mlp_ub.p, ctx->sm_count));
-  ctx->launches += 1;
+  // (The dropped terms are of second order in the lo plane, in Delta z and in
+  // P's rounding: about 6e-8 on the rewards and 3e-6 relative on g in the
+  // oracle's arithmetic on the mlp_bf16 shapes, against 2e-5 and 1e-4.)
+  // The dropped terms grow as sigma^2 (the oracle's rewards: 2.8e-6 at sigma =
+  // 0.05, 9e-6 at 0.1, 4e-5 at 0.2 on small shapes), so above sigma = 0.05 the
+  // GEMMs contract both planes (K = 2d and 2 d_ff, against the weights
+  // duplicated along K) and no correction is made.
+  const bool one_plane = p.sigma <= 0.05f;
+  float* Uw = nullptr;
   float* Wv = nullptr;
-  if (!down) {
-    DUST_TRY(ensure(ctx, ctx->mlp_wv, (size_t)T * dff * 4));
-    Wv = (float*)ctx->mlp_wv.p;
-    DUST_CU(launch_transpose_bf16(st, (const __nv_bfloat16*)W_down, d, dff,
-                                  (__nv_bfloat16*)ctx->mlp_wt.p, ldd));
+  if (one_plane) {
+    // (both GEMMs K-major: W_head and W_down transposed once per call)
+    const int64_t ldv = (V + 7) / 8 * 8, ldd = (d + 7) / 8 * 8;
+    DUST_TRY(ensure(ctx, ctx->mlp_pb, (size_t)T * V * 2));
+    DUST_TRY(ensure(ctx, ctx->mlp_uw, (size_t)T * d * 4));
+    DUST_TRY(ensure(ctx, ctx->mlp_wt, (size_t)std::max(d * ldv, dff * ldd) * 2));
+    Uw = (float*)ctx->mlp_uw.p;
+    DUST_CU(launch_f32_to_bf16(st, Z, T * V, (__nv_bfloat16*)ctx->mlp_pb.p, ctx->sm_count));
+    DUST_CU(launch_transpose_bf16(st, (const __nv_bfloat16*)W_head, V, d,
+                                  (__nv_bfloat16*)ctx->mlp_wt.p, ldv));
+    ctx->launches += 2;
+    {
+      GemmDesc g{};
+      g.M = T; g.N = d; g.K = V; g.A = ctx->mlp_pb.p; g.lda = V; g.a_kmajor = true;
+      g.B = ctx->mlp_wt.p; g.ldb = ldv; g.b_kmajor = true; g.dtype = DUST_BF16;
+      EpiDesc e{};
+      e.kind = kEpiF32; e.C = Uw; e.ldc = d;
+      DUST_TRY(run_gemm(ctx, g, e));
+    }
+    // u_t = W_head[y_t] - U_t in place of U (and in bf16 where Wv needs it).
+    // Where dh = da W_down^T (up-projection, attention output projection), that
+    // GEMM too contracts only the hi plane of da; the lo plane moves a reward by
+    // da_lo . Wv_t to first order, Wv = u W_down (T x d_ff, from u in bf16).
+    // With both corrections the oracle's rewards move by 1.1e-7 and g by 4.9e-6
+    // relative on the mlp_bf16 shapes.
+    if (!down) DUST_TRY(ensure(ctx, ctx->mlp_ub, (size_t)T * d * 2));
+    DUST_CU(launch_head_ut(st, (const __nv_bfloat16*)W_head, V, targets, Uw, T, d,
+                           down ? nullptr : (__nv_bfloat16*)ctx->mlp_ub.p, ctx->sm_count));
     ctx->launches += 1;
-    GemmDesc g{};
-    g.M = T; g.N = dff; g.K = d; g.A = ctx->mlp_ub.p; g.lda = d; g.a_kmajor = true;
-    g.B = ctx->mlp_wt.p; g.ldb = ldd; g.b_kmajor = true; g.dtype = DUST_BF16;
-    EpiDesc e{};
-    e.kind = kEpiF32; e.C = Wv; e.ldc = dff;
-    DUST_TRY(run_gemm(ctx, g, e));
+    if (!down) {
+      DUST_TRY(ensure(ctx, ctx->mlp_wv, (size_t)T * dff * 4));
+      Wv = (float*)ctx->mlp_wv.p;
+      DUST_CU(launch_transpose_bf16(st, (const __nv_bfloat16*)W_down, d, dff,
+                                    (__nv_bfloat16*)ctx->mlp_wt.p, ldd));
+      ctx->launches += 1;
+      GemmDesc g{};
+      g.M = T; g.N = dff; g.K = d; g.A = ctx->mlp_ub.p; g.lda = d; g.a_kmajor = true;
+      g.B = ctx->mlp_wt.p; g.ldb = ldd; g.b_kmajor = true; g.dtype = DUST_BF16;
+      EpiDesc e{};
+      e.kind = kEpiF32; e.C = Wv; e.ldc = dff;
+      DUST_TRY(run_gemm(ctx, g, e));
+    }
+    mark(ctx, "head_mean");
   }
-  mark(ctx, "head_mean");
 
   // perturbed passes, a chunk of tokens (all K draws each) at a time
   const int64_t max_rows = 131072;
@@ -713,8 +721,10 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
       DUST_CU(launch_gelu_delta_rows(st, p, u, du, t0, nt, da));
       ctx->launches += 1;
       GemmDesc g{};
-      g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
-      g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = d; g.K = one_plane ? dff : 2 * dff; g.A = da; g.lda = 2 * dff;
+      g.a_kmajor = true;
+      g.B = one_plane ? W_down : ctx->wd2.p; g.ldb = one_plane ? dff : 2 * dff;
+      g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
       e.kind = kEpiResidSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       e.resid = dn; e.ldr = 2 * d; e.rsplit = d;
@@ -723,8 +733,10 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
       DUST_CU(launch_mlp_delta_a(st, p, u, t0, nt, da, true, nullptr));
       ctx->launches += 1;
       GemmDesc g{};
-      g.M = rows; g.N = d; g.K = dff; g.A = da; g.lda = 2 * dff; g.a_kmajor = true;
-      g.B = W_down; g.ldb = dff; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = d; g.K = one_plane ? dff : 2 * dff; g.A = da; g.lda = 2 * dff;
+      g.a_kmajor = true;
+      g.B = one_plane ? W_down : ctx->wd2.p; g.ldb = one_plane ? dff : 2 * dff;
+      g.b_kmajor = true; g.dtype = DUST_BF16;
       EpiDesc e{};
       e.kind = kEpiSplit; e.Cb = dh; e.ldcb = 2 * d; e.split = d;
       DUST_TRY(run_gemm(ctx, g, e));
@@ -733,8 +745,9 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
     int used_parts = (int)((V + 127) / 128);  // the CUDA-core reward GEMM's 128-column tiles
     {
       GemmDesc g{};
-      g.M = rows; g.N = V; g.K = d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
-      g.B = W_head; g.ldb = d; g.b_kmajor = true; g.dtype = DUST_BF16;
+      g.M = rows; g.N = V; g.K = one_plane ? d : 2 * d; g.A = dh; g.lda = 2 * d; g.a_kmajor = true;
+      g.B = one_plane ? W_head : ctx->wh2.p; g.ldb = one_plane ? d : 2 * d; g.b_kmajor = true;
+      g.dtype = DUST_BF16;
       EpiDesc e{};
       e.kind = kEpiReward; e.P = Z; e.y = targets; e.t0 = t0; e.draws = p.K;
       e.part = (float*)ctx->part.p; e.dzy = (float*)ctx->dzy.p;
@@ -749,9 +762,12 @@ static dust_status mlp_impl(dust_ctx* ctx, const dust_params* pp, int layer, con
     }
     DUST_CU(launch_reward_combine_rows(st, (float*)ctx->part.p, used_parts, (float*)ctx->dzy.p,
                                        rows, t0 * K, p.K, r));
-    DUST_CU(launch_mlp_reward_corr(st, dh, d, Uw, down ? nullptr : da, dff, Wv, t0, p.K, rows,
-                                   r));
-    ctx->launches += 2;
+    ctx->launches += 1;
+    if (one_plane) {
+      DUST_CU(launch_mlp_reward_corr(st, dh, d, Uw, down ? nullptr : da, dff, Wv, t0, p.K, rows,
+                                     r));
+      ctx->launches += 1;
+    }
   }
   mark(ctx, "perturbed");
   if (attn)
