@@ -161,9 +161,15 @@ dust_status dust_head_grad_host(dust_ctx* ctx, const dust_params* p,
  * u = x W_up^T (d_ff entries per token); each draw recomputes
  * GELU(u + sigma eps) - GELU(u), the down-projection and the head from the
  * cached x, u and clean logits (exact-erf GELU, residual h = x + a W_down^T,
- * no norm, no bias). Inputs are bf16; the activations a, h and the per-draw
- * deltas enter the tensor-core GEMMs as bf16 hi/lo planes (about 2^-17
- * relative), against weights duplicated along the contraction.
+ * no norm, no bias). Inputs are bf16; the clean activations a, h enter the
+ * tensor-core GEMMs as bf16 hi/lo planes (about 2^-17 relative), against
+ * weights duplicated along the contraction. The per-draw deltas are split the
+ * same way; for sigma <= 0.05 the delta GEMMs contract their hi planes only,
+ * and each reward gets the lo planes' first-order effect,
+ * lo(dh) . u_t + lo(da) . (W_down^T u_t) with u_t = W_head[y_t] - W_head^T p_t
+ * (p_t the clean softmax): two per-token vectors formed once per call by two
+ * GEMMs. What that drops is of second order (rewards within about 3e-6 at
+ * sigma = 0.05); above 0.05 both planes are contracted.
  *   X        T x d     input, dtype        W_up   d_ff x d   dtype
  *   W_down   d x d_ff  dtype               W_head V x d      dtype
  *   targets  T int32
@@ -183,8 +189,10 @@ dust_status dust_mlp_grad(dust_ctx* ctx, const dust_params* p,
  * Hidden-MLP down-projection estimator (same pages and sections as
  * dust_mlp_grad, the next layer type of the block). Noise goes on
  * W_down's output (d entries per token), which is the block output h, so each
- * draw recomputes only the head: dz = sigma eps W_head^T (sigma eps enters the
- * tensor-core GEMM as bf16 hi/lo planes), r = dz_y - log1p(sum p expm1(dz)),
+ * draw recomputes only the head: dz = sigma eps W_head^T (sigma eps as bf16
+ * hi/lo planes, the GEMM on the hi plane with the lo plane's first-order
+ * effect added as in dust_mlp_grad for sigma <= 0.05),
+ * r = dz_y - log1p(sum p expm1(dz)),
  * g_t = -(1/(K sigma)) sum_i r_i eps_i, and the weight gradient is taken
  * against the layer's cached input a = GELU(u) (fp32, CUDA cores).
  *   arguments and layouts as dust_mlp_grad, except
