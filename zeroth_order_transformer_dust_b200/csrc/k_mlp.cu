@@ -481,8 +481,10 @@ cudaError_t launch_reward_combine_rows(cudaStream_t st, const float* part, int n
   return cudaGetLastError();
 }
 
-// a . b over n entries of a bf16 row and an fp32 row (one warp; 16-byte loads
-// where n is a multiple of 8 and the rows 16-byte aligned)
+// a . b over n entries of a bf16 row and an fp32 row, this lane's share of it
+// (the caller sums the warp). 16-byte loads where n is a multiple of 8: the
+// callers' rows then start 16-byte aligned (allocation-aligned bases, row
+// strides that are multiples of n).
 __device__ __forceinline__ float warp_dot_bf16_f32(const __nv_bfloat16* __restrict__ a,
                                                    const float* __restrict__ b, int64_t n,
                                                    int lane) {
