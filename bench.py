@@ -309,8 +309,9 @@ def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
     """ALU-issue roofline of the draw kernel: algorithmic elements x the minimum
     issue slots per element / time, against every lane issuing each clock; the
     SFU (exp) ceiling and the second instruction count are reported beside it.
-    Full-vocabulary draws generate the noise twice (reward, then g); the
-    algorithmic count is one generation."""
+    Full-vocabulary draws generate the noise once (one pass) or twice (a
+    reward pass, then a g pass, where no one-pass plan fits); the algorithmic
+    count is one generation."""
     if wl.S > 0:
         elems = wl.T * wl.K * (wl.S + 1)
     else:
@@ -323,7 +324,7 @@ def _alu_roofline(wl, draw_ms: float, peaks) -> dict:
     sfu_peak = SM_COUNT * SFU_PER_SM * f / 1e12                        # T exp/s
     return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tops/s",
             "frac": achieved / peak, "traffic": None,
-            "kernel": "subset_draws" if wl.S > 0 else "reward+g",
+            "kernel": "subset_draws" if wl.S > 0 else "full_draws",
             "elements": elems, "ops_per_element": ALU_OPS_PER_ELEM, "kernel_ms": draw_ms,
             "peak_basis": f"{SM_COUNT} SMs x {LANES_PER_SM} lanes x {f / 1e6:.0f} MHz (sm_max_mhz)",
             "with_accumulate": {"ops_per_element": ALU_OPS_PER_ELEM_WITH_ACCUMULATE,
@@ -583,7 +584,10 @@ def run_dust(args):
     roof = None
     draw_key = "subset_draws" if wl.S > 0 else None
     if wl.variant == "head":
-        draw_ms = stages.get("subset_draws") if wl.S > 0 else stages.get("reward", 0) + stages.get("g", 0)
+        if wl.S > 0:
+            draw_ms = stages.get("subset_draws")
+        else:  # one pass, or the reward and g passes where no one-pass plan fits
+            draw_ms = stages.get("full_draws") or stages.get("reward", 0) + stages.get("g", 0)
         if draw_ms:
             roof = _alu_roofline(wl, draw_ms, peaks)
             roof["peak_kind"] = peak_kind

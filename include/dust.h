@@ -96,7 +96,9 @@ typedef struct dust_params {
    results within the parity tolerances): DUST_DISABLE_TC=1 runs every GEMM
    on CUDA cores; DUST_TC_PAIR=0 gives each tensor-core GEMM tile one CTA
    instead of a CTA pair; DUST_SUBSET_KERNEL=1 uses the L2-fed subset-draw
-   kernel instead of the shared-memory one. */
+   kernel instead of the shared-memory one; DUST_FULL_KERNEL=2 runs
+   full-vocabulary draws as a reward pass and a g pass (the noise generated
+   twice) instead of one pass. */
 dust_status dust_create(dust_ctx** out, int device, void* cuda_stream);
 dust_status dust_set_stream(dust_ctx* ctx, void* cuda_stream);
 /* Frees the context's scratch memory; waits for its stream first. */

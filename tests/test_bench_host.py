@@ -28,7 +28,7 @@ def test_subset_roofline_counts_elements_and_lanes():
 def test_full_vocab_roofline_counts_one_generation():
     wl = synth.CONFIGS["full_bf16"]
     r = bench._alu_roofline(wl, 29.8, PEAKS)
-    assert r["elements"] == wl.T * wl.K * wl.V and r["kernel"] == "reward+g"
+    assert r["elements"] == wl.T * wl.K * wl.V and r["kernel"] == "full_draws"
 
 
 def test_attention_roofline_splits_tensor_and_cuda_core_work():

@@ -149,6 +149,39 @@ def test_full_vocab_more_shapes(ctx, kw):
              TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
 
 
+@pytest.mark.parametrize("kw", [dict(), dict(K=1), dict(V=4099, K=20), dict(T=200, K=5, V=1000),
+                                dict(T=2, K=64, V=50304, d=16, sigma=0.01), dict(sigma=0.2),
+                                dict(T=40, K=7, V=20000, d=16, sigma=0.005)])
+def test_full_vocab_two_passes(cuda_ok, monkeypatch, kw):
+    """The reward pass and the g pass (DUST_FULL_KERNEL=2), which run where no
+    one-pass plan fits, against the oracle."""
+    monkeypatch.setenv("DUST_FULL_KERNEL", "2")
+    c = dust.Context(0)
+    wl = _small(**kw)
+    H, W, y = _inputs(wl)
+    _compare(_gpu(c, H, W, y, wl), _oracle(H, W, y, wl), TOL_GW_BF16)
+
+
+def test_full_vocab_runs_in_one_pass(ctx):
+    """The full_bf16 shapes take the one-pass kernel (its stage name), with
+    more tokens than clusters; sampled rows against the oracle."""
+    wl = synth.CONFIGS["full_bf16"]
+    t0, n = 3000, 40
+    H, W, y = _inputs(wl, n, t0)
+    ctx.set_stage_timing(True)
+    try:
+        got = _gpu(ctx, H, W, y, wl, token_offset=t0)
+        stages = ctx.stage_times()
+    finally:
+        ctx.set_stage_timing(False)
+    assert "full_draws" in stages and "reward" not in stages
+    for t in (0, 17, 39):
+        ref = _oracle(H[t:t + 1], W, y[t:t + 1], wl, token_offset=t0 + t)
+        assert abs(got["loss"][t] - ref["loss"][0]) < TOL_LOSS
+        assert np.abs(got["rewards"][t] - ref["rewards"][0]).max() < TOL_LOSS
+        assert rel_fro(got["g"][t], ref["g"][0]) < TOL_G
+
+
 @pytest.mark.parametrize("kw", [dict(S=100), dict(S=1000), dict(V=4099, S=640, K=40),
                                 dict(V=50304, S=512, K=64, T=3, d=16), dict(T=2, K=70000, S=64, V=700),
                                 dict(V=20000, S=300, K=33, sigma=0.2, T=4, d=16)])

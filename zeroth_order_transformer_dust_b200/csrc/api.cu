@@ -296,6 +296,8 @@ dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
   ctx->tc_pair = !(pair && pair[0] == '0');
   const char* sk = getenv("DUST_SUBSET_KERNEL");
   ctx->subset2_enabled = !(sk && sk[0] == '1');
+  const char* fk = getenv("DUST_FULL_KERNEL");
+  ctx->full_one_enabled = !(fk && fk[0] == '2');
   if (cudaSetDevice(device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess ||
@@ -436,7 +438,14 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   ctx->launches += 1;
   mark(ctx, "lse");
   // 3. perturbed losses, rewards, g
-  if (!subset) {
+  FullOnePlan one;
+  if (!subset && ctx->full_one_enabled &&
+      full_one_plan(p, ctx->sm_count, ctx->max_smem_optin, &one)) {
+    DUST_CU(launch_full_one(st, p, one, Z, (const float*)ctx->lse.p, targets, rewards_out, g_out,
+                            ctx->gop.p, gf, ctx->d_status));
+    ctx->launches += 1;
+    mark(ctx, "full_draws");
+  } else if (!subset) {
     float* r = rewards_out;
     if (!r) {
       DUST_TRY(ensure(ctx, ctx->rew, (size_t)p.T * p.K * 4));

@@ -210,6 +210,8 @@ struct dust_ctx {
   bool tc_pair = true;
   // shared-memory subset kernel on (DUST_SUBSET_KERNEL=1 selects the first, L2-fed one)
   bool subset2_enabled = true;
+  // full-vocabulary draws in one pass where a plan fits (DUST_FULL_KERNEL=2 at creation: two)
+  bool full_one_enabled = true;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
@@ -264,6 +266,21 @@ cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, co
 // GEMM operand gop in format gf.
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
                           void* gop, GopFormat gf);
+
+// Full-vocabulary draws in one pass (the noise generated once): clusters of nb
+// CTAs (at most 4), one token row per cluster at a time, W generator warps and
+// one reducer warp per CTA. full_one_plan returns false where no configuration
+// fits (the three stages above run then).
+struct FullOnePlan {
+  int nb = 0, W = 0, ncl = 0;
+  size_t smem = 0;
+};
+bool full_one_plan(const dust_params& p, int sm_count, int max_smem_optin, FullOnePlan* out);
+// Rewards to r (T x K, may be null), g and the GEMM operand as launch_full_g; a
+// wait that expires sets kStatusTimeout in *status.
+cudaError_t launch_full_one(cudaStream_t st, const dust_params& p, const FullOnePlan& plan,
+                            const float* Z, const float* lse, const int32_t* y, float* r,
+                            float* g_out, void* gop, GopFormat gf, uint32_t* status);
 
 // Subset draws, fused reward + accumulation. P is the probability matrix in
 // permuted column order (column q holds vocabulary index (a q) mod V).
