@@ -270,7 +270,7 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
 // blocks [c * bpc, (c + 1) * bpc), with p = exp(z - LSE), the g accumulators and
 // two buffers of noise in shared memory (the four slots of a lane side by side,
 // in the order 0, 2, 1, 3 of the packed pairs). Warps 0..W-1 generate: warp w
-// takes the blocks w, w + W, w + 2W, w + 3W of its CTA. For draw i it writes the
+// takes the blocks w, w + W, w + 2W, ... (at most kOneR) of its CTA. For draw i it writes the
 // blocks' sigma*eps to buffer i & 1, adds up p * expm1(sigma eps), and posts the
 // warp's sum to its CTA's reducer (shared memory, then an arrive on the draw's
 // local barrier); it then takes the reward of draw i - 1 from the reducer and
@@ -289,7 +289,9 @@ __global__ __launch_bounds__(kWarps * 32) void k_full_g(const __grid_constant__ 
 // then the status word's timeout bit and no further waits).
 constexpr int kOneSlots = 4;
 constexpr int kOneMaxW = 31;  // generator warps (one more reduces)
-constexpr int kOneR = 4;      // blocks per generator warp
+// blocks per generator warp: 5 measured best on full_bf16 (23.1 ms against 24.7
+// at 4, 26.5 at 6, 25.8 at 7; clusters of 4, so 20, 25, 17 and 15 warps)
+constexpr int kOneR = 5;
 constexpr int kOneOffL = kSinCosTable * 8;             // warp shares [4][32]
 constexpr int kOneOffC = kOneOffL + kOneSlots * 32 * 4;  // CTA totals [4][8]
 constexpr int kOneOffR = kOneOffC + kOneSlots * 8 * 4;   // rewards [4]
@@ -449,8 +451,11 @@ __global__ __launch_bounds__((kOneMaxW + 1) * 32, 1) void k_full_one(const __gri
           for (int j = 0; j < kOneR; ++j) {
             if (j < nmine) {
               const int o = (warp + W * j) * 32 + lane;
+              // the scalar Box-Muller step: its operations spread over both FMA
+              // pipes, where the packed form loads the FMA-heavy one the Philox
+              // multiplies already keep busy (0.7 % faster here)
               float2 e02, e13;
-              noise4<true>(philox_from2(bc[j], dc, A.keys), tab, e02, e13);
+              noise4<false>(philox_from2(bc[j], dc, A.keys), tab, e02, e13);
               const float4 pv = p4[o];
               eb[o] = make_float4(e02.x, e02.y, e13.x, e13.y);
               acc = __ffma2_rn(make_float2(pv.x, pv.y), expm1_small_x2<DEG>(e02), acc);
@@ -621,8 +626,8 @@ int g_one_n = 0;
 }  // namespace
 
 // Clusters of up to 4 CTAs (larger ones fit fewer SMs; measured slower): the one
-// with the least work per SM, counting per draw W generator warps of four block
-// rounds each, and ceil(T / clusters) tokens per cluster, clusters beyond one
+// with the least work per SM, counting per draw W generator warps of kOneR
+// block rounds each, and ceil(T / clusters) tokens per cluster, clusters beyond one
 // per SM sharing their SMs.
 bool full_one_plan(const dust_params& p, int sm_count, int max_smem_optin, FullOnePlan* out) {
   int dev = 0;
