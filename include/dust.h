@@ -98,10 +98,16 @@ typedef struct dust_params {
    instead of a CTA pair; DUST_SUBSET_KERNEL=1 uses the L2-fed subset-draw
    kernel instead of the shared-memory one; DUST_FULL_KERNEL=2 runs
    full-vocabulary draws as a reward pass and a g pass (the noise generated
-   twice) instead of one pass. */
+   twice) instead of one pass; DUST_FULL_SPLIT=0 keeps a one-pass call on
+   the context's stream, where by default the last ~8 % of its tokens go to
+   the two passes on the SMs that the one-pass clusters leave empty, from
+   two streams of the context's own (high and low priority) that fork from
+   and join `cuda_stream` inside the call. A CUDA graph captured from such a
+   call keeps the order but not the priorities unless it is instantiated
+   with node priorities. */
 dust_status dust_create(dust_ctx** out, int device, void* cuda_stream);
 dust_status dust_set_stream(dust_ctx* ctx, void* cuda_stream);
-/* Frees the context's scratch memory; waits for its stream first. */
+/* Frees the context's scratch memory and streams; waits for its streams first. */
 void dust_destroy(dust_ctx* ctx);
 /* Last error message of the context (never NULL). */
 const char* dust_last_error(const dust_ctx* ctx);

@@ -182,6 +182,34 @@ def test_full_vocab_runs_in_one_pass(ctx):
         assert rel_fro(got["g"][t], ref["g"][0]) < TOL_G
 
 
+def test_full_vocab_split_over_two_streams(cuda_ok, monkeypatch):
+    """On full_bf16 shapes the two passes take the last tokens on the SMs the
+    one-pass clusters leave empty (three more launches than the one-pass
+    kernel alone, DUST_FULL_SPLIT=0); every row, g and G_W agree with the
+    unsplit call, and rows on both sides of the split with the oracle."""
+    wl = synth.CONFIGS["full_bf16"]
+    t0, n = 1234, 600
+    H, W, y = _inputs(wl, n, t0)
+    split = dust.Context(0)
+    monkeypatch.setenv("DUST_FULL_SPLIT", "0")
+    whole = dust.Context(0)
+    l0 = split.kernel_launches
+    a = _gpu(split, H, W, y, wl, token_offset=t0)
+    la = split.kernel_launches - l0
+    l0 = whole.kernel_launches
+    b = _gpu(whole, H, W, y, wl, token_offset=t0)
+    lb = whole.kernel_launches - l0
+    assert la == lb + 3
+    np.testing.assert_array_equal(a["loss"], b["loss"])
+    assert np.abs(a["rewards"] - b["rewards"]).max() < TOL_LOSS
+    assert rel_fro(a["g"], b["g"]) < TOL_G
+    assert rel_fro(a["G"], b["G"]) < TOL_GW_BF16
+    for t in (0, 300, 540, 570, 599):
+        ref = _oracle(H[t:t + 1], W, y[t:t + 1], wl, token_offset=t0 + t)
+        assert np.abs(a["rewards"][t] - ref["rewards"][0]).max() < TOL_LOSS
+        assert rel_fro(a["g"][t], ref["g"][0]) < TOL_G
+
+
 @pytest.mark.parametrize("kw", [dict(S=100), dict(S=1000), dict(V=4099, S=640, K=40),
                                 dict(V=50304, S=512, K=64, T=3, d=16), dict(T=2, K=70000, S=64, V=700),
                                 dict(V=20000, S=300, K=33, sigma=0.2, T=4, d=16)])

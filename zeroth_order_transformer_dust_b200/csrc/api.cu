@@ -242,6 +242,62 @@ dust_status weight_grad_f16(dust_ctx* ctx, const dust_params& p, const void* gop
   return run_gemm(ctx, s, e);
 }
 
+// The full-vocabulary draws split over two streams (full_split_plan): the one-pass
+// kernel over tokens [0, T - T2) at the higher priority, so that its clusters are
+// placed first, and the two passes over the last T2 tokens at the lower, their
+// CTAs kept off the one-pass SMs. Both streams fork from the call's stream after
+// the log-sum-exp and join it before the G_W GEMM; the join is recorded even
+// when a launch fails.
+dust_status full_split_draws(dust_ctx* ctx, const dust_params& p, const FullOnePlan& one,
+                             const FullSide& side, int64_t T2, const float* Z,
+                             const int32_t* targets, float* rewards_out, float* g_out,
+                             GopFormat gf) {
+  if (!ctx->side_hi) {
+    int least = 0, greatest = 0;
+    DUST_CU(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    DUST_CU(cudaStreamCreateWithPriority(&ctx->side_hi, cudaStreamNonBlocking, greatest));
+    DUST_CU(cudaStreamCreateWithPriority(&ctx->side_lo, cudaStreamNonBlocking, least));
+    DUST_CU(cudaEventCreateWithFlags(&ctx->fork_ev, cudaEventDisableTiming));
+    DUST_CU(cudaEventCreateWithFlags(&ctx->join_hi, cudaEventDisableTiming));
+    DUST_CU(cudaEventCreateWithFlags(&ctx->join_lo, cudaEventDisableTiming));
+  }
+  const int64_t T1 = p.T - T2;
+  dust_params p1 = p, p2 = p;
+  p1.T = T1;
+  p2.T = T2;
+  p2.token_offset = p.token_offset + T1;
+  float* r2 = rewards_out ? rewards_out + T1 * p.K : nullptr;
+  if (!r2) {
+    DUST_TRY(ensure(ctx, ctx->rew, (size_t)T2 * p.K * 4));
+    r2 = (float*)ctx->rew.p;
+  }
+  DUST_TRY(ensure(ctx, ctx->part, (size_t)T2 * full_vocab_nslab(p.V) * p.K * 4));
+  DUST_TRY(ensure(ctx, ctx->dzy, full_vocab_xy_bytes(T2, p.K)));
+  const float* lse = (const float*)ctx->lse.p;
+  const size_t esz = gf.kind == kGopF32 ? 4 : 2;
+  void* gop2 = (char*)ctx->gop.p + (size_t)T1 * p.V * esz;
+  const cudaStream_t st = ctx->stream;
+  DUST_CU(cudaEventRecord(ctx->fork_ev, st));
+  DUST_CU(cudaStreamWaitEvent(ctx->side_hi, ctx->fork_ev, 0));
+  DUST_CU(cudaStreamWaitEvent(ctx->side_lo, ctx->fork_ev, 0));
+  cudaError_t e = launch_full_one(ctx->side_hi, p1, one, Z, lse, targets, rewards_out, g_out,
+                                  ctx->gop.p, gf, ctx->d_status);
+  if (e == cudaSuccess)
+    e = launch_full_reward_partial(ctx->side_lo, p2, Z + T1 * p.V, lse + T1, targets + T1,
+                                   (float*)ctx->part.p, (float*)ctx->dzy.p, &side);
+  if (e == cudaSuccess)
+    e = launch_full_reward_combine(ctx->side_lo, p2, (float*)ctx->part.p, (float*)ctx->dzy.p, r2);
+  if (e == cudaSuccess)
+    e = launch_full_g(ctx->side_lo, p2, r2, g_out ? g_out + T1 * p.V : nullptr, gop2, gf, &side);
+  DUST_CU(cudaEventRecord(ctx->join_hi, ctx->side_hi));
+  DUST_CU(cudaEventRecord(ctx->join_lo, ctx->side_lo));
+  DUST_CU(cudaStreamWaitEvent(st, ctx->join_hi, 0));
+  DUST_CU(cudaStreamWaitEvent(st, ctx->join_lo, 0));
+  DUST_CU(e);
+  ctx->launches += 4;
+  return DUST_OK;
+}
+
 // Stage marks: mark(ctx, nullptr) opens a call, mark(ctx, "name") closes the
 // stage that ran since the previous mark.
 void mark(dust_ctx* ctx, const char* name) {
@@ -298,6 +354,8 @@ dust_status dust_create(dust_ctx** out, int device, void* cuda_stream) {
   ctx->subset2_enabled = !(sk && sk[0] == '1');
   const char* fk = getenv("DUST_FULL_KERNEL");
   ctx->full_one_enabled = !(fk && fk[0] == '2');
+  const char* fs = getenv("DUST_FULL_SPLIT");
+  ctx->full_split = !(fs && fs[0] == '0');
   if (cudaSetDevice(device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess ||
@@ -322,6 +380,8 @@ void dust_destroy(dust_ctx* ctx) {
   if (!ctx) return;
   cudaSetDevice(ctx->device);
   if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+  for (cudaStream_t s : {ctx->side_hi, ctx->side_lo})
+    if (s) cudaStreamSynchronize(s);
   Buf* bufs[] = {&ctx->z, &ctx->lse, &ctx->loss, &ctx->gop, &ctx->rew, &ctx->part, &ctx->wperm,
                  &ctx->gT, &ctx->hT, &ctx->xdup, &ctx->dzy, &ctx->mlp_u, &ctx->mlp_a, &ctx->mlp_h,
                  &ctx->mlp_da, &ctx->mlp_dh, &ctx->wd2, &ctx->wh2, &ctx->in_h, &ctx->in_w, &ctx->in_y, &ctx->out_g,
@@ -333,6 +393,10 @@ void dust_destroy(dust_ctx* ctx) {
     if (b->p) cudaFree(b->p);
   for (int i = 0; i < dust_ctx::kMaxMarks; ++i)
     if (ctx->ev[i]) cudaEventDestroy(ctx->ev[i]);
+  for (cudaStream_t s : {ctx->side_hi, ctx->side_lo})
+    if (s) cudaStreamDestroy(s);
+  for (cudaEvent_t e : {ctx->fork_ev, ctx->join_hi, ctx->join_lo})
+    if (e) cudaEventDestroy(e);
   if (ctx->d_status) cudaFree(ctx->d_status);
   if (ctx->h_status) cudaFreeHost(ctx->h_status);
   cudaGetLastError();
@@ -441,9 +505,17 @@ dust_status dust_head_grad(dust_ctx* ctx, const dust_params* pp, const void* H, 
   FullOnePlan one;
   if (!subset && ctx->full_one_enabled &&
       full_one_plan(p, ctx->sm_count, ctx->max_smem_optin, &one)) {
-    DUST_CU(launch_full_one(st, p, one, Z, (const float*)ctx->lse.p, targets, rewards_out, g_out,
-                            ctx->gop.p, gf, ctx->d_status));
-    ctx->launches += 1;
+    FullSide side;
+    const int64_t T2 = ctx->full_split && gf.kind != kGopBf16Planes
+                           ? full_split_plan(p, one, ctx->sm_count, &side)
+                           : 0;
+    if (T2 > 0) {
+      DUST_TRY(full_split_draws(ctx, p, one, side, T2, Z, targets, rewards_out, g_out, gf));
+    } else {
+      DUST_CU(launch_full_one(st, p, one, Z, (const float*)ctx->lse.p, targets, rewards_out,
+                              g_out, ctx->gop.p, gf, ctx->d_status));
+      ctx->launches += 1;
+    }
     mark(ctx, "full_draws");
   } else if (!subset) {
     float* r = rewards_out;

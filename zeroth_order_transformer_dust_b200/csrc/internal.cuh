@@ -212,6 +212,12 @@ struct dust_ctx {
   bool subset2_enabled = true;
   // full-vocabulary draws in one pass where a plan fits (DUST_FULL_KERNEL=2 at creation: two)
   bool full_one_enabled = true;
+  // the two passes beside the one-pass kernel on the SMs its clusters leave empty
+  // (DUST_FULL_SPLIT=0 at creation: off); their streams (high and low priority)
+  // and the fork/join events are made at first use
+  bool full_split = true;
+  cudaStream_t side_hi = nullptr, side_lo = nullptr;
+  cudaEvent_t fork_ev = nullptr, join_hi = nullptr, join_lo = nullptr;
   // scratch, grown on demand
   dust::Buf z, lse, loss, gop, rew, part, wperm, gT, hT, xdup, dzy, mlp_u, mlp_a, mlp_h, mlp_da,
       mlp_dh, wd2, wh2, in_h, in_w, in_y, out_g, out_loss, out_r, out_gv, lsep, mlp_a32, mlp_dn, mlp_du, wu2,
@@ -256,16 +262,24 @@ cudaError_t launch_lse_rows(cudaStream_t st, float* Z, int64_t T, int64_t V, con
 // target -> xy[t * K + i] (T x K floats, full_vocab_xy_bytes).
 int full_vocab_nslab(int64_t V);
 size_t full_vocab_xy_bytes(int64_t T, int32_t K);
+// Where the two passes share the GPU with a one-pass launch (full_split_plan):
+// their grids fill only `sms` SMs, each CTA with `pad` bytes of dynamic shared
+// memory it does not use, so that none fits on an SM beside a one-pass CTA.
+struct FullSide {
+  int sms = 0;
+  size_t pad = 0;
+};
 cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* Z,
                                        const float* lse,
-                                       const int32_t* y, float* part, float* xy);
+                                       const int32_t* y, float* part, float* xy,
+                                       const FullSide* side = nullptr);
 // Stage 2: r[t*K + i] = xy - log1p(sum_slab part).
 cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, const float* part,
                                        const float* xy, float* r);
 // Stage 3: g_t = -(1/(K sigma)) sum_i r_i eps_i; writes g (fp32, optional) and the
 // GEMM operand gop in format gf.
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
-                          void* gop, GopFormat gf);
+                          void* gop, GopFormat gf, const FullSide* side = nullptr);
 
 // Full-vocabulary draws in one pass (the noise generated once): clusters of nb
 // CTAs (at most 4), one token row per cluster at a time, W generator warps and
@@ -281,6 +295,12 @@ bool full_one_plan(const dust_params& p, int sm_count, int max_smem_optin, FullO
 cudaError_t launch_full_one(cudaStream_t st, const dust_params& p, const FullOnePlan& plan,
                             const float* Z, const float* lse, const int32_t* y, float* r,
                             float* g_out, void* gop, GopFormat gf, uint32_t* status);
+// Tokens of a call that the two passes take from the end of the batch, on the
+// SMs that `one`'s clusters leave empty and concurrently with the one-pass
+// launch over the rest (which then fills `one.ncl` clusters a whole number of
+// times); 0 where that does not pay. Fills *side.
+int64_t full_split_plan(const dust_params& p, const FullOnePlan& one, int sm_count,
+                        FullSide* side);
 
 // Subset draws, fused reward + accumulation. P is the probability matrix in
 // permuted column order (column q holds vocabulary index (a q) mod V).

@@ -19,6 +19,8 @@
 #include "noise.cuh"
 #include "tc_ptx.cuh"
 
+#include <cmath>
+#include <cstdint>
 #include <mutex>
 
 namespace dust {
@@ -523,13 +525,16 @@ FullArgs make_args(const dust_params& p) {
   return A;
 }
 
-// Persistent grid: every SM filled with as many CTAs as fit, at most one per unit.
+// Persistent grid: every SM filled with as many CTAs as fit, at most one per unit;
+// with `side`, side->sms SMs and CTAs of side->pad bytes of dynamic shared memory.
 template <typename F>
-int grid_for(F kernel, int64_t units) {
+int grid_for(F kernel, int64_t units, const FullSide* side = nullptr) {
   int dev = 0, sms = 148, per_sm = 1;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWarps * 32, 0) != cudaSuccess ||
+  if (side) sms = side->sms;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kWarps * 32,
+                                                    side ? side->pad : 0) != cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
   cudaGetLastError();
@@ -545,7 +550,7 @@ size_t full_vocab_xy_bytes(int64_t T, int32_t K) { return (size_t)T * K * 4; }
 
 cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, const float* Z,
                                        const float* lse, const int32_t* y, float* part,
-                                       float* xy) {
+                                       float* xy, const FullSide* side) {
   FullArgs A = make_args(p);
   A.Z = Z;
   A.lse = lse;
@@ -553,15 +558,16 @@ cudaError_t launch_full_reward_partial(cudaStream_t st, const dust_params& p, co
   A.part = part;
   A.xy = xy;
   const int64_t units = A.T * A.nslab;
+  const size_t pad = side ? side->pad : 0;
   switch (expm1_degree(p.sigma)) {
     case 3:
-      k_full_reward_partial<3><<<grid_for(k_full_reward_partial<3>, units), kWarps * 32, 0, st>>>(A);
+      k_full_reward_partial<3><<<grid_for(k_full_reward_partial<3>, units, side), kWarps * 32, pad, st>>>(A);
       break;
     case 4:
-      k_full_reward_partial<4><<<grid_for(k_full_reward_partial<4>, units), kWarps * 32, 0, st>>>(A);
+      k_full_reward_partial<4><<<grid_for(k_full_reward_partial<4>, units, side), kWarps * 32, pad, st>>>(A);
       break;
     default:
-      k_full_reward_partial<0><<<grid_for(k_full_reward_partial<0>, units), kWarps * 32, 0, st>>>(A);
+      k_full_reward_partial<0><<<grid_for(k_full_reward_partial<0>, units, side), kWarps * 32, pad, st>>>(A);
   }
   return cudaGetLastError();
 }
@@ -576,13 +582,13 @@ cudaError_t launch_full_reward_combine(cudaStream_t st, const dust_params& p, co
 }
 
 cudaError_t launch_full_g(cudaStream_t st, const dust_params& p, const float* r, float* g_out,
-                          void* gop, GopFormat gf) {
+                          void* gop, GopFormat gf, const FullSide* side) {
   FullArgs A = make_args(p);
   A.r = r;
   A.g_out = g_out;
   A.gop = gop;
   A.gf = gf;
-  k_full_g<<<grid_for(k_full_g, A.T * A.nslab), kWarps * 32, 0, st>>>(A);
+  k_full_g<<<grid_for(k_full_g, A.T * A.nslab, side), kWarps * 32, side ? side->pad : 0, st>>>(A);
   return cudaGetLastError();
 }
 
@@ -713,6 +719,49 @@ cudaError_t launch_full_one(cudaStream_t st, const dust_params& p, const FullOne
   e = cudaLaunchKernelEx(&cfg, fn, A);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// Per SM, the one-pass kernel finishes this many times the tokens of the two passes
+// (4096 tokens of V = 50304, K = 64: 23.2 ms on 132 SMs against 14.9 + 12.4 ms on 148).
+constexpr double kOneVsTwo = 1.3;
+
+int64_t full_split_plan(const dust_params& p, const FullOnePlan& one, int sm_count,
+                        FullSide* side) {
+  const int used = one.nb * one.ncl;
+  const int free_sms = sm_count - used;
+  if (one.ncl < 1 || free_sms < 8) return 0;
+  int dev = 0, cap = 0, res = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&cap, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&res, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  // the two passes' CTAs, padded, must not fit into what a one-pass CTA leaves of an SM
+  const void* fns[2] = {(const void*)k_full_g, (const void*)k_full_reward_partial<0>};
+  const int deg = expm1_degree(p.sigma);
+  if (deg == 3) fns[1] = (const void*)k_full_reward_partial<3>;
+  if (deg == 4) fns[1] = (const void*)k_full_reward_partial<4>;
+  size_t stat = SIZE_MAX;
+  for (const void* f : fns) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, f) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    if (fa.sharedSizeBytes < stat) stat = fa.sharedSizeBytes;
+  }
+  const int64_t left = (int64_t)cap - (int64_t)one.smem - 2 * (int64_t)res - (int64_t)stat;
+  const size_t pad = left < 0 ? 0 : (size_t)((left + 128) / 128 * 128);
+  if (pad > 48 * 1024) return 0;
+  // the one-pass clusters take a whole number of rounds of tokens
+  const double share1 = used * kOneVsTwo / (used * kOneVsTwo + free_sms);
+  const int64_t rounds = (int64_t)std::llround((double)p.T * share1 / one.ncl);
+  const int64_t T1 = rounds * one.ncl;
+  if (rounds < 4 || T1 >= p.T) return 0;
+  side->sms = free_sms;
+  side->pad = pad;
+  return p.T - T1;
 }
 
 }  // namespace dust
