@@ -210,6 +210,30 @@ def test_full_vocab_split_over_two_streams(cuda_ok, monkeypatch):
         assert rel_fro(a["g"][t], ref["g"][0]) < TOL_G
 
 
+@pytest.mark.parametrize("kw", [dict(T=300, d=64, K=4, dtype="f32"), dict(T=300, d=32, K=3, sigma=0.2)])
+def test_full_vocab_split_shapes(cuda_ok, monkeypatch, kw):
+    """The split on other V = 50304 shapes: fp32 inputs (an fp32 g operand) and
+    a sigma beyond the expm1 series' range, every row against the oracle; then
+    G_W again without rewards or g requested (the two passes' rewards go to
+    scratch), equal to the first."""
+    wl = _small(V=50304, **kw)
+    H, W, y = _inputs(wl)
+    c = dust.Context(0)
+    monkeypatch.setenv("DUST_FULL_SPLIT", "0")
+    whole = dust.Context(0)
+    l0 = c.kernel_launches
+    got = _gpu(c, H, W, y, wl)
+    launches = c.kernel_launches - l0
+    _gpu(whole, H, W, y, wl)
+    assert launches == whole.kernel_launches + 3
+    _compare(got, _oracle(H, W, y, wl), TOL_GW_F32 if wl.dtype == "f32" else TOL_GW_BF16)
+    out = c.head_grad(to_dev(H, wl.dtype), to_dev(W, wl.dtype), to_dev(y, "i32"), K=wl.K,
+                      sigma=wl.sigma, seed=wl.seed)
+    torch.cuda.synchronize()
+    assert c.kernel_launches - l0 == 2 * launches
+    assert rel_fro(np64(out["G"]), got["G"]) < 1e-6
+
+
 @pytest.mark.parametrize("kw", [dict(S=100), dict(S=1000), dict(V=4099, S=640, K=40),
                                 dict(V=50304, S=512, K=64, T=3, d=16), dict(T=2, K=70000, S=64, V=700),
                                 dict(V=20000, S=300, K=33, sigma=0.2, T=4, d=16)])
