@@ -9,8 +9,9 @@
 // log1p(sum_drawn p_j expm1(sigma eps_j)), r = sigma eps_y - log1p(.), and
 // r eps (scaled by the inverse inclusion probability) accumulates into g_t.
 //
-// B200 mapping: one cluster of CS CTAs (one per SM; CS = 1, 2, 4 or 8, the
-// smallest whose slices fit in shared memory) per token at a time,
+// B200 mapping: one cluster of CS CTAs (one per SM; CS = 1 or 2 where the
+// slices fit in shared memory, else the size of 3 to 8 whose clusters cover
+// the most SMs) per token at a time,
 // persistent over tokens. CTA r of the cluster holds the probability row and
 // the g accumulator for its slice [r seg, (r+1) seg) of q in shared memory
 // (CS = 2 at V = 50304: 2 x 100.6 KB per CTA; CS = 8 reaches V ~ 223k), so
@@ -51,6 +52,7 @@
 // at K = 1024. The wait for the copy is bounded: on expiry the kernel raises
 // the timeout bit of the status word and runs on without waiting again.
 #include <cooperative_groups.h>
+#include <mutex>
 
 #include "internal.cuh"
 #include "noise.cuh"
@@ -667,22 +669,73 @@ cudaError_t launch_nb(cudaStream_t st, const Sub2Args& A, size_t smem, int sm, i
 // start 16-byte aligned in shared memory).
 int64_t slice_len(int64_t V, int cs) { return ((V + cs - 1) / cs + 3) / 4 * 4; }
 
+// Never launched: the occupancy query below asks it how many clusters of a
+// size fit at once with one CTA per SM, which the GPCs' SM counts decide.
+__global__ void k_cluster_probe() {}
+
+// SMs that clusters of cs CTAs of one CTA per SM cover at once (0 if unknown),
+// cached per device.
+int cluster_sms(int cs, int max_smem_optin) {
+  static std::mutex mu;
+  static int cache[16][9] = {};
+  int dev = 0, sms = 0;
+  if (cs < 1 || cs > 8 || cudaGetDevice(&dev) != cudaSuccess || dev >= 16 ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev][cs]) return cache[dev][cs] > 0 ? cache[dev][cs] : 0;
+  int n = 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)((sms / cs > 0 ? sms / cs : 1) * cs));
+  cfg.blockDim = dim3(32);
+  cfg.dynamicSmemBytes = (size_t)max_smem_optin;  // one CTA per SM
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaFuncSetAttribute(k_cluster_probe, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           max_smem_optin) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, (void*)k_cluster_probe, &cfg) != cudaSuccess)
+    n = 0;
+  cudaGetLastError();
+  cache[dev][cs] = n > 0 ? n * cs : -1;
+  return n > 0 ? n * cs : 0;
+}
+
 }  // namespace
 
-// Cluster size the shared-memory kernel would use (0: not applicable): the
-// smallest of 1, 2, 4, 8 whose slices (p and g, 4 bytes each) fit in shared
-// memory, with every slice at least S long, so that a window reaches at most
-// the next slice.
+// Cluster size the shared-memory kernel would use (0: not applicable). The
+// slices (p and g, 4 bytes each) must fit in shared memory, and every slice
+// be at least S long, so that a window reaches at most the next slice. One
+// CTA, or two, where they fit; else, of 3 to 8 CTAs, the size whose clusters
+// cover the most SMs at once (clusters of 8 fit 15 times on a 148-SM B200,
+// 120 SMs, while smaller ones fill more of each GPC), the smaller on a tie.
 int subset2_cluster_size(int64_t V, int32_t S, int max_smem_optin) {
   if (S < 1 || S > 1024 || V >= (1LL << 31)) return 0;
-  for (int cs = 1; cs <= 8; cs *= 2) {
+  auto fits = [&](int cs) {
     const int64_t seg = slice_len(V, cs);
     const int64_t last = V - (cs - 1) * seg;  // the last (shortest) slice
-    if (2 * seg * 4 + kStaticSmem > max_smem_optin) continue;
-    if (cs > 1 && (S > seg || S > last)) continue;
-    return cs;
+    if (2 * seg * 4 + kStaticSmem > max_smem_optin) return false;
+    return cs == 1 || (S <= seg && S <= last);
+  };
+  if (fits(1)) return 1;
+  if (fits(2)) return 2;
+  int best = 0, best_sms = 0, fallback = 0;
+  for (int cs = 3; cs <= 8; ++cs) {
+    if (!fits(cs)) continue;
+    if (!fallback && (cs == 4 || cs == 8)) fallback = cs;
+    const int n = cluster_sms(cs, max_smem_optin);
+    if (n > best_sms) {
+      best = cs;
+      best_sms = n;
+    }
   }
-  return 0;
+  return best ? best : fallback;
 }
 
 cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int64_t a_inv,
@@ -738,11 +791,11 @@ cudaError_t launch_subset2(cudaStream_t st, const dust_params& p, int64_t a, int
   // the list's longer draw loop (6 % more instructions) costs more than the
   // balance gains (4.11 -> 4.30 ms), and larger S keeps batches: those
   // variants have no registers to spare.
-  // Clusters of 4 and 8 CTAs (the larger vocabularies) split a token's draws
+  // Clusters of 3 to 8 CTAs (the larger vocabularies) split a token's draws
   // finer still: there the list serves S <= 512 up to 256 draws a CTA.
   const size_t slices = (size_t)2 * A.seg * 4, list_bytes = (size_t)p.K * 16;
   const bool list = use_int &&
-                    ((p.K <= 512 && p.S <= 256) || (cs >= 4 && p.S <= 512 && p.K <= 256 * cs)) &&
+                    ((p.K <= 512 && p.S <= 256) || (cs >= 3 && p.S <= 512 && p.K <= 256 * cs)) &&
                     slices + list_bytes + (size_t)kStaticSmem <= (size_t)max_smem_optin;
   const size_t smem = slices + (list ? list_bytes : 0);
   const int deg = expm1_degree(p.sigma);
