@@ -119,6 +119,11 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     # CTAs (up to 256 draws a CTA), with several tokens per cluster
     dict(V=128256, S=512, K=1024, T=3, d=16), dict(V=70001, S=400, K=1024, T=3, d=16),
     dict(V=100003, S=257, K=300, T=40, d=16), dict(V=128256, S=511, K=2048, T=2, d=16),
+    # cluster sizes other than powers of two (3 to 8 CTAs, whichever covers the
+    # most SMs): clusters of 3 with the draw list, and vocabularies whose
+    # smallest fitting cluster has 4, 5 or 6 CTAs
+    dict(V=60000, S=512, K=700, T=5, d=16), dict(V=90001, S=129, K=100, T=7, d=16),
+    dict(V=120001, S=384, K=600, T=3, d=16), dict(V=150001, S=300, K=500, T=4, d=16),
 ])
 def test_edge_shapes(ctx, kw):
     wl = _small(**kw)
