@@ -91,7 +91,7 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     # fixed-point accumulation with a reduced scale (16384 < K <= 65536), and the
     # fp32-atomic fallback (K > 65536)
     dict(T=3, K=20000, S=32), dict(T=2, K=70000, S=64, V=700),
-    # vocabularies beyond one or two CTAs' shared memory: clusters of 4 and 8
+    # vocabularies beyond one or two CTAs' shared memory: clusters of 4 to 8
     # CTAs (windows crossing into the next CTA's slice and wrapping past V)
     dict(V=70001, S=300, K=256, T=4), dict(V=128256, S=512, K=256, T=4, d=24),
     dict(V=200003, S=512, K=256, T=4, d=16), dict(V=200003, S=77, K=300, T=3, d=16, dtype="f32"),
@@ -115,7 +115,7 @@ def _small(T=37, d=40, V=1000, K=9, S=0, sigma=0.02, seed=5, dtype="bf16"):
     dict(V=1000, S=1000, K=20), dict(V=1024, S=1024, K=16, T=9), dict(T=1, K=66000, S=1024, V=2048, d=8),
     # beyond 1024 entries a draw: the L2-fed kernel
     dict(V=5000, S=1500, K=30), dict(V=50304, S=2048, K=20, T=3, d=16),
-    # the draw list at three and four blocks a draw in clusters of 4 and 8
+    # the draw list at three and four blocks a draw in clusters of 3 to 8
     # CTAs (up to 256 draws a CTA), with several tokens per cluster
     dict(V=128256, S=512, K=1024, T=3, d=16), dict(V=70001, S=400, K=1024, T=3, d=16),
     dict(V=100003, S=257, K=300, T=40, d=16), dict(V=128256, S=511, K=2048, T=2, d=16),

@@ -312,7 +312,7 @@ cudaError_t launch_subset_impl(cudaStream_t st, const dust_params& p, int64_t a,
                                void* gop, GopFormat gf, float* gacc, int max_smem_optin);
 
 // Subset draws with the probability row and the g accumulator resident in
-// shared memory, one cluster of 1, 2, 4 or 8 CTAs per token (0: not applicable to
+// shared memory, one cluster of 1 to 8 CTAs per token (0: not applicable to
 // this V, S). Z holds clean logits in permuted column order, lse the row
 // log-sum-exp; p = exp(z - lse) is formed while the row is loaded. A row
 // copy that does not arrive in time sets kStatusTimeout in *status.

@@ -74,7 +74,7 @@ namespace {
 // NB = 5 to 8 (S up to 1024), whose draws hold 20 to 32 noise values a lane;
 // their ragged-S forms with the library expm1 or fp32 accumulators need more
 // than 128 registers and run 12 warps (8 at NB = 7, 8 with the library expm1).
-// The draw-list variants of NB = 3 and 4 (clusters of 4 and 8 CTAs) run 16
+// The draw-list variants of NB = 3 and 4 (clusters of 3 to 8 CTAs) run 16
 // warps too: the list's setup leaves them no register to spare at 64.
 __host__ __device__ constexpr int sub2_threads(bool use_int, int deg, int nb, bool full,
                                                bool list) {
