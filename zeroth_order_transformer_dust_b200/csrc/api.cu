@@ -252,14 +252,16 @@ dust_status full_split_draws(dust_ctx* ctx, const dust_params& p, const FullOneP
                              const FullSide& side, int64_t T2, const float* Z,
                              const int32_t* targets, float* rewards_out, float* g_out,
                              GopFormat gf) {
-  if (!ctx->side_hi) {
+  // made at first use; what a failed attempt left unmade is made by the next
+  if (!ctx->side_hi || !ctx->side_lo || !ctx->fork_ev || !ctx->join_hi || !ctx->join_lo) {
     int least = 0, greatest = 0;
     DUST_CU(cudaDeviceGetStreamPriorityRange(&least, &greatest));
-    DUST_CU(cudaStreamCreateWithPriority(&ctx->side_hi, cudaStreamNonBlocking, greatest));
-    DUST_CU(cudaStreamCreateWithPriority(&ctx->side_lo, cudaStreamNonBlocking, least));
-    DUST_CU(cudaEventCreateWithFlags(&ctx->fork_ev, cudaEventDisableTiming));
-    DUST_CU(cudaEventCreateWithFlags(&ctx->join_hi, cudaEventDisableTiming));
-    DUST_CU(cudaEventCreateWithFlags(&ctx->join_lo, cudaEventDisableTiming));
+    if (!ctx->side_hi)
+      DUST_CU(cudaStreamCreateWithPriority(&ctx->side_hi, cudaStreamNonBlocking, greatest));
+    if (!ctx->side_lo)
+      DUST_CU(cudaStreamCreateWithPriority(&ctx->side_lo, cudaStreamNonBlocking, least));
+    for (cudaEvent_t* ev : {&ctx->fork_ev, &ctx->join_hi, &ctx->join_lo})
+      if (!*ev) DUST_CU(cudaEventCreateWithFlags(ev, cudaEventDisableTiming));
   }
   const int64_t T1 = p.T - T2;
   dust_params p1 = p, p2 = p;
